@@ -1,0 +1,189 @@
+"""CPU oracle for the MoE routing hot path (router, dispatch, gather, combine).
+
+TEST INFRASTRUCTURE ONLY: the test-suite, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` are the only callers.  The product package
+(``token_dispatch_fp32_b200``) never imports this module, and this module
+never imports the product package; the two share only the seeded input
+generators in ``workloads.py``.
+
+The arithmetic lives in ``moe_oracle.c`` (plain C, binary64, sort-based top-k,
+one token at a time); this file only builds it with gcc and marshals numpy
+arrays.  Each function's docstring names the page passage it follows.
+
+Parity status: every function here is pinned by ``tests/test_oracle_pins.py``
+(brute force, closed forms, library routines, invariants, hand-derived golden
+cases); none is "parity unpinned".
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "moe_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+NEAR_TIE_EPS = 1e-5
+
+
+def build(force: bool = False) -> str:
+    """Compile moe_oracle.c into liboracle.so (gcc, -O2, OpenMP, portable ISA)."""
+    if force or not os.path.exists(_LIB_PATH) or (
+            os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC)):
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared",
+                               "-std=c11", "-Wall", "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        # MO_ORACLE_LIB: test hook used by the mutation test to load a
+        # deliberately broken copy of the oracle; never set otherwise.
+        path = os.environ.get("MO_ORACLE_LIB") or build()
+        lib = C.CDLL(path)
+        p = C.c_void_p
+        lib.mo_router.argtypes = [p, p, p, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int,
+                                  C.c_int, C.c_double, C.c_int, p, p, p, p, C.c_int]
+        lib.mo_dispatch.argtypes = [p, C.c_int, C.c_int, C.c_int, p, p, p, p]
+        lib.mo_gather.argtypes = [p, C.c_long, C.c_int, C.c_int, p, p, C.c_long, p]
+        lib.mo_round_bf16.argtypes = [C.c_double]
+        lib.mo_round_bf16.restype = C.c_double
+        lib.mo_round_bf16_array.argtypes = [p, C.c_long, p]
+        lib.mo_combine.argtypes = [p, C.c_int, p, p, p, C.c_int, C.c_int, C.c_int, p,
+                                   C.c_long, p, p, C.c_int]
+        _lib = lib
+    return _lib
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(C.c_void_p)
+
+
+def num_threads() -> int:
+    return int(_load().mo_num_threads())
+
+
+def router(x, W, b, n_group, topk_group, k, route_scale, mask_mode,
+           want_logits=False, threads=0) -> dict:
+    """Gate forward for every row of x (Kimi K2 "Normalize weights" page,
+    MoEGate.forward; DeepSeek-V3.2-Exp "Normalize weights" page,
+    Gate.forward; DeepSeek-V3 "MoE Router" note, "How it works").
+
+    x [T,d] fp32 values, W [N_r,d] fp32, b [N_r] fp32 or None.
+    Returns idx [T,k] int32 in canonical order (masked biased score
+    descending, index ascending), w [T,k] float64, margins [T,3] float64
+    (selection, group, slot-order margins) and optionally logits [T,N_r].
+    """
+    lib = _load()
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    W = np.ascontiguousarray(W, dtype=np.float32)
+    b = None if b is None else np.ascontiguousarray(b, dtype=np.float32)
+    T, d = x.shape
+    N_r = W.shape[0]
+    assert W.shape[1] == d
+    idx = np.empty((T, k), np.int32)
+    w = np.empty((T, k), np.float64)
+    margins = np.empty((T, 3), np.float64)
+    logits = np.empty((T, N_r), np.float64) if want_logits else None
+    rc = lib.mo_router(_ptr(x), _ptr(W), _ptr(b), T, d, N_r, n_group, topk_group, k,
+                       float(route_scale), mask_mode, _ptr(idx), _ptr(w), _ptr(logits),
+                       _ptr(margins), threads)
+    if rc != 0:
+        raise ValueError(f"oracle router rejected the arguments (rc={rc})")
+    return {"idx": idx, "w": w, "margins": margins, "logits": logits}
+
+
+def near_tie(margins, eps=NEAR_TIE_EPS):
+    """Tokens whose selection (k-th vs k+1-th) or group margin is <= eps."""
+    return np.minimum(margins[:, 0], margins[:, 1]) <= eps
+
+
+def order_tie(margins, eps=NEAR_TIE_EPS):
+    """Tokens whose slot order within the top-k is decided by a gap <= eps."""
+    return near_tie(margins, eps) | (margins[:, 2] <= eps)
+
+
+def dispatch(idx, N_r):
+    """moe_infer dispatch (Kimi K2 "Add shared output" page, moe_infer:
+    tokens_per_expert, idxs = argsort(topk_ids.view(-1)) as a stable sort,
+    and the inverse of idxs used by new_x[idxs] = outs).
+
+    Returns counts [N_r], offsets [N_r+1], perm [T*k], inv [T*k] (int32).
+    """
+    lib = _load()
+    idx = np.ascontiguousarray(idx, dtype=np.int32)
+    T, k = idx.shape
+    counts = np.empty(N_r, np.int32)
+    offsets = np.empty(N_r + 1, np.int32)
+    perm = np.empty(T * k, np.int32)
+    inv = np.empty(T * k, np.int32)
+    rc = lib.mo_dispatch(_ptr(idx), T, k, N_r, _ptr(counts), _ptr(offsets), _ptr(perm),
+                         _ptr(inv))
+    if rc != 0:
+        raise ValueError(f"oracle dispatch rejected the input (rc={rc})")
+    return counts, offsets, perm, inv
+
+
+def gather(x, k, perm, rows=None):
+    """sorted_tokens = x[idxs // k] (Kimi K2 "Add shared output" page,
+    moe_infer).  x is [T,d] of any element type, copied byte for byte;
+    rows selects a subset of output rows (all rows when None)."""
+    lib = _load()
+    x = np.ascontiguousarray(x)
+    perm = np.ascontiguousarray(perm, dtype=np.int32)
+    T = x.shape[0]
+    rows_a = None if rows is None else np.ascontiguousarray(rows, dtype=np.int32)
+    n = perm.shape[0] if rows is None else rows_a.shape[0]
+    out = np.empty((n,) + x.shape[1:], x.dtype)
+    rc = lib.mo_gather(_ptr(x), x.strides[0], T, k, _ptr(perm), _ptr(rows_a), n, _ptr(out))
+    if rc != 0:
+        raise ValueError(f"oracle gather: index out of range (rc={rc})")
+    return out
+
+
+def round_bf16(a):
+    """binary64 -> nearest-even bf16 value (returned as binary64)."""
+    a = np.ascontiguousarray(a, dtype=np.float64)
+    out = np.empty_like(a)
+    _load().mo_round_bf16_array(_ptr(a), a.size, _ptr(out))
+    return out
+
+
+def combine(E, w, inv, shared, k, tokens=None, threads=0):
+    """Weighted combine and shared add (Kimi K2 "Add shared output" page:
+    moe_infer scatter-back and weighted sum, DeepseekV3MoE.forward shared
+    add, formula Delta_ffn = y_routed + y_shared).
+
+    E [T*k,d] expert outputs in expert-sorted order, fp32 or bf16 bits
+    (uint16); w [T,k] fp32; inv [T*k] int32; shared [T,d] same dtype as E,
+    or None.  Returns (y, routed) as float64 [n_tok,d], already rounded to
+    the row dtype for bf16.
+    """
+    lib = _load()
+    E = np.ascontiguousarray(E)
+    dtype = 1 if E.dtype == np.uint16 else 0
+    assert E.dtype in (np.uint16, np.float32)
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    inv = np.ascontiguousarray(inv, dtype=np.int32)
+    T, kk = w.shape
+    assert kk == k
+    d = E.shape[1]
+    if shared is not None:
+        shared = np.ascontiguousarray(shared)
+        assert shared.dtype == E.dtype and shared.shape == (T, d)
+    tok = None if tokens is None else np.ascontiguousarray(tokens, dtype=np.int32)
+    n = T if tokens is None else tok.shape[0]
+    y = np.empty((n, d), np.float64)
+    routed = np.empty((n, d), np.float64)
+    rc = lib.mo_combine(_ptr(E), dtype, _ptr(w), _ptr(inv), _ptr(shared), T, d, k,
+                        _ptr(tok), n, _ptr(y), _ptr(routed), threads)
+    if rc != 0:
+        raise ValueError(f"oracle combine rejected the input (rc={rc})")
+    return y, routed

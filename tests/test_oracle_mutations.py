@@ -1,0 +1,50 @@
+"""The oracle's pins must catch plausible mistakes.  Each case plants one
+mistake in a temporary copy of the oracle's C source (on the CPU), builds it,
+and runs the pin suite against it; the suite has to fail."""
+import os
+import shutil
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "oracle", "moe_oracle.c")
+
+MUTATIONS = {
+    "weights_from_biased_scores": ("den += s[ord[j].i];", "den += m[ord[j].i];"),
+    "bias_dropped_from_selection": ("m[i] = s[i] + (bias ? (double)bias[i] : 0.0);",
+                                    "m[i] = s[i];"),
+    "group_score_is_max": ("gs[g] = tmp[0] + tmp[1];", "gs[g] = tmp[0];"),
+    "mask_value_swapped": ("m[i] = (mask_mode == 0) ? -INFINITY : 0.0;",
+                           "m[i] = (mask_mode == 1) ? -INFINITY : 0.0;"),
+    "ties_to_highest_index": ("return (a->i > b->i) - (a->i < b->i);",
+                              "return (a->i < b->i) - (a->i > b->i);"),
+    "no_renormalisation": ("w[j] = route_scale * (s[ord[j].i] / den);",
+                           "w[j] = route_scale * s[ord[j].i];"),
+    "unstable_dispatch": ("return (a->slot > b->slot) - (a->slot < b->slot);",
+                          "return (a->slot < b->slot) - (a->slot > b->slot);"),
+    "perm_inverse_swapped": ("inv[perm[i]] = (int32_t)i;", "inv[i] = perm[i];"),
+    "routed_not_rounded": ("double routed = dtype == 1 ? mo_round_bf16(acc) : acc;",
+                           "double routed = acc;"),
+    "bf16_round_half_up": ("double r = nearbyint(ldexp(fabs(v), -q));",
+                           "double r = floor(ldexp(fabs(v), -q) + 0.5);"),
+    "logit_sign_flip": ("s[i] = 1.0 / (1.0 + exp(-acc));", "s[i] = 1.0 / (1.0 + exp(acc));"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_pins_catch_mutation(name, tmp_path):
+    old, new = MUTATIONS[name]
+    src = open(SRC).read()
+    assert src.count(old) == 1, f"mutation anchor not found once: {old}"
+    mut = tmp_path / "moe_oracle_mut.c"
+    mut.write_text(src.replace(old, new))
+    lib = tmp_path / "liboracle_mut.so"
+    subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11",
+                           "-o", str(lib), str(mut), "-lm"])
+    env = dict(os.environ, MO_ORACLE_LIB=str(lib))
+    r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
+                        os.path.join(ROOT, "tests", "test_oracle_pins.py")],
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode != 0, f"pins did not catch '{name}':\n{r.stdout[-2000:]}"

@@ -1,0 +1,391 @@
+"""Pins for the CPU oracle: each test checks the oracle against something other
+than itself -- a hand-derived case, a brute-force search, a closed form, a
+library routine (BLAS, numpy sorting, torch's bf16 cast) or an invariant the
+pages state.  Each is chosen so that a plausible slip in the oracle (dropped
+bias, bias in the weights, wrong group score, wrong mask value, transposed
+perm/inverse, wrong tie order, missing rounding) fails at least one of them.
+"""
+import itertools
+import json
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+from scipy.special import expit
+
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "hand_cases.json")
+
+
+def _frac(v):
+    return Fraction(v) if isinstance(v, str) else Fraction(v)
+
+
+def _one_hot_logits(s_list):
+    """Token x = e_0 with W[:,0] = logit(s): logits are exactly W[:,0]."""
+    L = np.array([math.log(float(s) / (1 - float(s))) for s in s_list], np.float64)
+    N = len(L)
+    x = np.zeros((1, 4), np.float32)
+    x[0, 0] = 1.0
+    W = np.zeros((N, 4), np.float32)
+    W[:, 0] = L.astype(np.float32)
+    return x, W
+
+
+def _rand_problem(rng, T, d, N_r, bias_scale=0.1):
+    x = rng.standard_normal((T, d)).astype(np.float32)
+    W = (rng.standard_normal((N_r, d)) / math.sqrt(d)).astype(np.float32)
+    b = rng.uniform(-bias_scale, bias_scale, N_r).astype(np.float32)
+    return x, W, b
+
+
+# --------------------------------------------------------------------------
+# Hand-derived cases (tests/golden/hand_cases.json)
+
+with open(GOLDEN) as f:
+    _G = json.load(f)
+
+
+@pytest.mark.parametrize("case", _G["router"], ids=[c["name"] for c in _G["router"]])
+def test_router_hand_cases(case):
+    x, W = _one_hot_logits([_frac(s) for s in case["s"]])
+    b = np.array([float(_frac(v)) for v in case["bias"]], np.float32)
+    r = oracle.router(x, W, b, case["n_group"], case["topk_group"], case["k"],
+                      float(_frac(case["route_scale"])), case["mask_mode"])
+    assert r["idx"][0].tolist() == case["expect_idx"]
+    np.testing.assert_allclose(r["w"][0], [float(_frac(v)) for v in case["expect_w"]],
+                               rtol=2e-6, atol=0)
+
+
+@pytest.mark.parametrize("case", _G["dispatch"], ids=[c["name"] for c in _G["dispatch"]])
+def test_dispatch_hand_cases(case):
+    idx = np.array(case["idx"], np.int32)
+    counts, offsets, perm, inv = oracle.dispatch(idx, case["N_r"])
+    assert counts.tolist() == case["expect_counts"]
+    assert offsets.tolist() == case["expect_offsets"]
+    assert perm.tolist() == case["expect_perm"]
+    assert inv.tolist() == case["expect_inv"]
+    assert (perm // idx.shape[1]).tolist() == case["expect_tokens"]
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("case", _G["combine"], ids=[c["name"] for c in _G["combine"]])
+def test_combine_hand_cases(case, dtype):
+    def arr(v):
+        return np.array([[float(_frac(e)) for e in row] for row in v], np.float32)
+
+    E, shared = arr(case["E"]), arr(case["shared"])
+    if dtype == "bf16":  # every value in the case is exact in bf16
+        E = (E.view(np.uint32) >> 16).astype(np.uint16)
+        shared = (shared.view(np.uint32) >> 16).astype(np.uint16)
+    y, routed = oracle.combine(E, arr(case["w"]), np.array(case["inv"], np.int32),
+                               shared, case["k"])
+    assert routed.tolist() == arr(case["expect_routed"]).tolist()
+    assert y.tolist() == arr(case["expect_y"]).tolist()
+
+
+# --------------------------------------------------------------------------
+# Logits: BLAS (an independent library) on fp64 copies.
+
+def test_logits_match_blas():
+    rng = np.random.default_rng(10)
+    x, W, b = _rand_problem(rng, 37, 300, 24)
+    r = oracle.router(x, W, b, 4, 2, 3, 2.5, 0, want_logits=True)
+    ref = x.astype(np.float64) @ W.astype(np.float64).T
+    np.testing.assert_allclose(r["logits"], ref, rtol=1e-12, atol=1e-13)
+
+
+# --------------------------------------------------------------------------
+# Special case: one group and no bias reduces to plain top-k of the scores,
+# i.e. of the logits (sigmoid is monotone) -- the unbiased top-K_r form of
+# the DeepSeek-V3 "MoE Router" note.
+
+@pytest.mark.parametrize("use_none", [True, False])
+def test_unbiased_ungrouped_is_plain_topk(use_none):
+    rng = np.random.default_rng(11)
+    x, W, _ = _rand_problem(rng, 200, 64, 40)
+    b = None if use_none else np.zeros(40, np.float32)
+    k = 6
+    r = oracle.router(x, W, b, 1, 1, k, 1.0, 0, want_logits=True)
+    L = x.astype(np.float64) @ W.astype(np.float64).T
+    ref = np.argsort(-L, axis=1, kind="stable")[:, :k]
+    assert (r["idx"] == ref).all()
+    # renormalised gates: g = s / sum(s) over the K_r survivors (library expit)
+    s = expit(np.take_along_axis(L, ref, 1))
+    np.testing.assert_allclose(r["w"], s / s.sum(1, keepdims=True), rtol=1e-12)
+
+
+# --------------------------------------------------------------------------
+# Brute force on tiny inputs: the chosen experts maximise the sum of masked
+# scores over all k-subsets, where the mask keeps the topk_group groups that
+# maximise the sum of group scores, and a group score is the best pair sum
+# in the group.  Ties go to the lexicographically smallest index tuple.
+
+def _brute(c, G, Gk, k, mask_mode):
+    N = len(c)
+    S = N // G
+    if G > 1:
+        gs = [max(c[g * S + a] + c[g * S + b] for a, b in itertools.combinations(range(S), 2))
+              for g in range(G)]
+        keep = min(itertools.combinations(range(G), Gk),
+                   key=lambda sub: (-math.fsum(gs[g] for g in sub), sub))
+        fill = -math.inf if mask_mode == 0 else 0.0
+        m = [c[i] if (i // S) in keep else fill for i in range(N)]
+    else:
+        m = list(c)
+    best = min(itertools.combinations(range(N), k),
+               key=lambda sub: (-math.fsum(m[i] for i in sub), sub))
+    return set(best), m
+
+
+@pytest.mark.parametrize("N_r,G,Gk,k,mask_mode,bias_lo,bias_hi", [
+    (12, 1, 1, 4, 0, -0.1, 0.1),
+    (12, 2, 1, 3, 0, -0.1, 0.1),
+    (12, 3, 2, 4, 0, -0.1, 0.1),
+    (12, 4, 2, 3, 0, -0.1, 0.1),
+    (12, 4, 3, 4, 1, -0.1, 0.1),
+    (12, 4, 2, 4, 1, -1.5, -0.6),  # zero mask with negative biased scores
+    (12, 3, 1, 4, 1, -1.5, -0.6),  # k > group size: masked zeros must fill in
+    (8, 4, 2, 2, 0, -0.5, 0.5),
+    (10, 5, 2, 4, 0, -0.2, 0.2),
+    (9, 3, 3, 2, 0, -0.1, 0.1),
+])
+def test_router_brute_force(N_r, G, Gk, k, mask_mode, bias_lo, bias_hi):
+    rng = np.random.default_rng(1000 + N_r * 100 + G * 10 + Gk + k + mask_mode)
+    T = 300
+    x, W, _ = _rand_problem(rng, T, 16, N_r)
+    b = rng.uniform(bias_lo, bias_hi, N_r).astype(np.float32)
+    r = oracle.router(x, W, b, G, Gk, k, 2.5, mask_mode)
+    L = x.astype(np.float64) @ W.astype(np.float64).T
+    c = expit(L) + b.astype(np.float64)
+    for t in range(T):
+        want, m = _brute(list(c[t]), G, Gk, k, mask_mode)
+        got = r["idx"][t].tolist()
+        assert set(got) == want, (t, got, sorted(want))
+        # canonical slot order: masked score descending, index ascending
+        keys = [(-m[i], i) for i in got]
+        assert keys == sorted(keys)
+
+
+# --------------------------------------------------------------------------
+# Invariants the pages state.
+
+def _problem_v3(seed, T=400):
+    rng = np.random.default_rng(seed)
+    return _rand_problem(rng, T, 96, 64)
+
+
+def test_weights_sum_to_route_scale():
+    x, W, b = _problem_v3(1)
+    for scale in (1.0, 2.5, 2.827):
+        r = oracle.router(x, W, b, 8, 4, 8, scale, 0)
+        np.testing.assert_allclose(r["w"].sum(1), scale, rtol=1e-13)
+
+
+def test_weights_linear_in_route_scale():
+    x, W, b = _problem_v3(2)
+    r1 = oracle.router(x, W, b, 8, 4, 8, 1.25, 0)
+    r2 = oracle.router(x, W, b, 8, 4, 8, 2.5, 0)
+    assert (r1["idx"] == r2["idx"]).all()
+    assert (r2["w"] == 2.0 * r1["w"]).all()  # exact: scaling by a power of two
+
+
+def test_chosen_experts_in_at_most_topk_group_groups():
+    # node-limited routing: a token reaches at most topk_group groups
+    x, W, b = _problem_v3(3, T=2000)
+    for G, Gk in ((8, 4), (8, 1), (4, 2), (16, 3)):
+        r = oracle.router(x, W, b, G, Gk, min(8, Gk * (64 // G)), 2.5, 0)
+        S = 64 // G
+        ngroups = np.array([len(set((r["idx"][t] // S).tolist())) for t in range(len(x))])
+        assert ngroups.max() <= Gk
+
+
+def test_weights_use_unbiased_scores():
+    x, W, b = _problem_v3(4)
+    L = x.astype(np.float64) @ W.astype(np.float64).T
+    s = expit(L)
+    # a large bias on a few experts pulls them into the selection ...
+    b2 = b.copy()
+    b2[[3, 17, 40]] += 5.0
+    r = oracle.router(x, W, b2, 1, 1, 8, 2.5, 0)
+    assert all({3, 17, 40} <= set(row.tolist()) for row in r["idx"])
+    # ... but every weight is still route_scale * s / sum(s) of the unbiased s
+    sg = np.take_along_axis(s, r["idx"].astype(np.int64), 1)
+    np.testing.assert_allclose(r["w"], 2.5 * sg / sg.sum(1, keepdims=True), rtol=1e-12)
+
+
+def test_uniform_bias_shift_changes_nothing():
+    x, W, b = _problem_v3(5)
+    r1 = oracle.router(x, W, b, 8, 4, 8, 2.5, 0)
+    r2 = oracle.router(x, W, (b + np.float32(0.25)).astype(np.float32), 8, 4, 8, 2.5, 0)
+    ok = ~(oracle.near_tie(r1["margins"], 1e-9))
+    assert (r1["idx"][ok] == r2["idx"][ok]).all()
+    np.testing.assert_allclose(r1["w"][ok], r2["w"][ok], rtol=1e-15)
+
+
+def test_permutation_within_groups_is_equivariant():
+    x, W, b = _problem_v3(6)
+    G, S = 8, 8
+    rng = np.random.default_rng(7)
+    p = np.concatenate([g * S + rng.permutation(S) for g in range(G)])  # new i <- old p[i]
+    r1 = oracle.router(x, W, b, G, 4, 8, 2.5, 0)
+    r2 = oracle.router(x, W[p], b[p], G, 4, 8, 2.5, 0)
+    ok = ~oracle.order_tie(r1["margins"], 1e-12)
+    mapped = p[r2["idx"]]  # back to old expert ids
+    assert (mapped[ok] == r1["idx"][ok]).all()
+    np.testing.assert_allclose(r2["w"][ok], r1["w"][ok], rtol=1e-14)
+
+
+def test_margins_are_score_gaps():
+    x, W, b = _problem_v3(8, T=50)
+    k = 8
+    r = oracle.router(x, W, b, 1, 1, k, 2.5, 0)
+    c = expit(x.astype(np.float64) @ W.astype(np.float64).T) + b
+    srt = -np.sort(-c, axis=1)
+    np.testing.assert_allclose(r["margins"][:, 0], srt[:, k - 1] - srt[:, k], atol=1e-14)
+    assert np.isinf(r["margins"][:, 1]).all()
+    np.testing.assert_allclose(r["margins"][:, 2], np.diff(-srt[:, :k], axis=1).min(1),
+                               atol=1e-14)
+
+
+def test_router_rejects_bad_arguments():
+    x, W, b = _problem_v3(9, T=4)
+    with pytest.raises(ValueError):
+        oracle.router(x, W, b, 7, 2, 4, 2.5, 0)   # 64 % 7 != 0
+    with pytest.raises(ValueError):
+        oracle.router(x, W, b, 8, 9, 4, 2.5, 0)   # topk_group > n_group
+    with pytest.raises(ValueError):
+        oracle.router(x, W, b, 8, 1, 9, 2.5, 0)   # k > kept experts under -inf
+    with pytest.raises(ValueError):
+        oracle.router(x, W, b, 64, 2, 2, 2.5, 0)  # group of one expert
+
+
+# --------------------------------------------------------------------------
+# Dispatch against numpy (bincount, stable argsort).
+
+@pytest.mark.parametrize("skew", [False, True])
+def test_dispatch_matches_numpy(skew):
+    rng = np.random.default_rng(12)
+    T, k, N_r = 3000, 8, 256
+    if skew:
+        idx = np.where(rng.random((T, k)) < 0.9, rng.integers(0, 32, (T, k)),
+                       rng.integers(0, N_r, (T, k))).astype(np.int32)
+    else:
+        idx = rng.integers(0, N_r, (T, k)).astype(np.int32)
+    counts, offsets, perm, inv = oracle.dispatch(idx, N_r)
+    flat = idx.reshape(-1)
+    assert (counts == np.bincount(flat, minlength=N_r)).all()
+    assert offsets[0] == 0 and offsets[-1] == T * k
+    assert (np.diff(offsets) == counts).all()
+    assert (perm == np.argsort(flat, kind="stable")).all()
+    assert (inv[perm] == np.arange(T * k)).all()
+    assert (np.diff(flat[perm]) >= 0).all()
+
+
+def test_dispatch_rejects_out_of_range():
+    with pytest.raises(ValueError):
+        oracle.dispatch(np.array([[0, 5]], np.int32), 5)
+    with pytest.raises(ValueError):
+        oracle.dispatch(np.array([[0, -1]], np.int32), 5)
+
+
+# --------------------------------------------------------------------------
+# Gather against numpy fancy indexing.
+
+@pytest.mark.parametrize("dt", [np.float32, np.uint16])
+def test_gather_matches_fancy_indexing(dt):
+    rng = np.random.default_rng(13)
+    T, k, d = 50, 4, 33
+    x = rng.integers(0, 60000, (T, d)).astype(dt)
+    idx = rng.integers(0, 16, (T, k)).astype(np.int32)
+    _, _, perm, _ = oracle.dispatch(idx, 16)
+    xs = oracle.gather(x, k, perm)
+    assert (xs == x[perm // k]).all()
+    rows = np.array([0, 7, T * k - 1], np.int32)
+    assert (oracle.gather(x, k, perm, rows) == x[perm[rows] // k]).all()
+
+
+# --------------------------------------------------------------------------
+# bf16 rounding against torch's float32 -> bfloat16 cast (round to nearest
+# even), and the two ties that decide "to even".
+
+def test_round_bf16_matches_torch():
+    import torch
+    rng = np.random.default_rng(14)
+    v = np.concatenate([rng.standard_normal(100000) * 10.0 ** rng.integers(-30, 30, 100000),
+                        [1 + 2 ** -8, 1 + 3 * 2 ** -8, -(1 + 2 ** -8), 2.0 ** -130,
+                         3.3e38, -0.0]]).astype(np.float32)
+    got = oracle.round_bf16(v.astype(np.float64))
+    ref = torch.from_numpy(v).to(torch.bfloat16).to(torch.float32).numpy().astype(np.float64)
+    assert np.array_equal(got, ref)
+    assert got[-6] == 1.0 and got[-5] == 1 + 2 ** -6
+
+
+# --------------------------------------------------------------------------
+# Combine: closed forms.
+
+def test_combine_identity_experts_gives_route_scale_times_x():
+    """Experts = identity (E = gathered x rows), no shared expert:
+    y_t = sum_j w_tj x_t = route_scale * x_t since the weights sum to the
+    route scale ("Normalize weights" pages)."""
+    rng = np.random.default_rng(15)
+    x, W, b = _rand_problem(rng, 120, 64, 32)
+    r = oracle.router(x, W, b, 4, 2, 4, 2.5, 0)
+    w32 = r["w"].astype(np.float32)
+    _, _, perm, inv = oracle.dispatch(r["idx"], 32)
+    # fp32 rows: exact value of sum_j w_j x = x * sum_j w_j (fp32 weights)
+    y, _ = oracle.combine(oracle.gather(x, 4, perm), w32, inv, None, 4)
+    np.testing.assert_allclose(y, x.astype(np.float64) * w32.astype(np.float64).sum(1)[:, None],
+                               rtol=1e-14, atol=1e-300)
+    # bf16 rows: within half a bf16 ulp of the bf16-rounded route_scale * x
+    xb = (x.view(np.uint32) >> 16).astype(np.uint16)
+    xbf = (xb.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    yb, _ = oracle.combine(oracle.gather(xb, 4, perm), w32, inv, None, 4)
+    ulp = 2.0 ** (np.floor(np.log2(np.abs(2.5 * xbf) + 1e-300)) - 7)
+    assert (np.abs(yb - 2.5 * xbf) <= 0.5 * ulp + 1e-300).all()
+
+
+def test_combine_scatter_back_direction():
+    """One-hot weights pick one slot: y_t = E[inv[t*k + j0]] -- the row the
+    scatter-back new_x[idxs] = outs puts at slot (t, j0)."""
+    rng = np.random.default_rng(16)
+    T, k, N_r = 40, 3, 10
+    idx = np.stack([rng.permutation(N_r)[:k] for _ in range(T)]).astype(np.int32)
+    _, _, perm, inv = oracle.dispatch(idx, N_r)
+    E = np.repeat(np.arange(T * k, dtype=np.float32)[:, None], 2, 1)  # row i holds i
+    for j0 in range(k):
+        w = np.zeros((T, k), np.float32)
+        w[:, j0] = 1.0
+        y, _ = oracle.combine(E, w, inv, None, k)
+        assert (y[:, 0] == inv.reshape(T, k)[:, j0]).all()
+        # and perm is the inverse of inv: the sorted row came from slot t*k+j0
+        assert (perm[y[:, 0].astype(np.int64)] == np.arange(T) * k + j0).all()
+
+
+def test_combine_shared_add_rounds_twice():
+    """bf16 rows: routed sum rounded to bf16, then shared added and rounded
+    again (the two casts back to the row dtype)."""
+    T, k, d = 1, 1, 1
+    w = np.array([[1.0]], np.float32)
+    inv = np.array([0], np.int32)
+    one = np.array([[0x3F80]], np.uint16)                 # 1.0
+    tiny = np.array([[0x3B80]], np.uint16)                # 2^-8: half a ulp of 1.0
+    y, routed = oracle.combine(one, w, inv, tiny, k)
+    assert routed[0, 0] == 1.0 and y[0, 0] == 1.0          # tie -> even (1.0)
+    three = np.array([[0x3C40]], np.uint16)               # 3 * 2^-8 = 0.01171875
+    y, _ = oracle.combine(one, w, inv, three, k)
+    assert y[0, 0] == 1 + 2 ** -6                          # 1 + 1.5 ulp -> up to even
+
+
+def test_combine_routed_rounding_is_observable():
+    """Routed sum exactly halfway (1 + 2^-8) rounds to 1.0 before the shared
+    add; adding 2^-8 to the unrounded sum would reach 1 + 2^-7 instead."""
+    w = np.array([[1 + 2 ** -8]], np.float32)
+    one = np.array([[0x3F80]], np.uint16)                 # 1.0
+    tiny = np.array([[0x3B80]], np.uint16)                # 2^-8
+    y, routed = oracle.combine(one, w, np.array([0], np.int32), tiny, 1)
+    assert routed[0, 0] == 1.0
+    assert y[0, 0] == 1.0
