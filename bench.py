@@ -1,0 +1,432 @@
+"""Benchmark of the MoE routing hot path on B200: routed tokens/s.
+
+One step = the whole path over one batch of T tokens, every stage a libmr.so
+kernel launched through the C ABI on one stream:
+    router (3xTF32 tcgen05 GEMM + fused routing)  -> idx, w
+    dispatch (counts, offsets, stable perm, inv)   -> perm, inv
+    gather (token rows -> expert-sorted rows)      -> xs [T*k, d]
+    [expert FFNs are not part of the path: synthetic expert outputs E]
+    combine (weighted sum + shared add)            -> y [T, d]
+Default workload: the full DeepSeek-V3 routing + dispatch + combine batch
+(T=16384, d=7168, 256 experts in 8 groups keep 4, top-8, bf16 rows).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Multi-GPU (torchrun, one rank per GPU): every rank runs its own batch
+(replicas, weak scaling, no collective in the data path); value = all ranks'
+tokens / max-over-ranks device time.  --impl reference times the CPU oracle
+(rank 0 only) on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as wl  # noqa: E402
+
+METRIC = "routed tokens/sec (router+dispatch+combine) at 1 B200; % of roofline"
+UNIT = "tokens/s"
+
+# DRAM traffic per launch measured with ncu (dram__bytes_read.sum +
+# dram__bytes_write.sum) for the dominant kernel, keyed by the SHA-256 of the
+# source file it was built from; reported only while the source is unchanged.
+NCU_TRAFFIC = {}
+
+
+def _src_sha(rel):
+    with open(os.path.join(ROOT, rel), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+class Clocks:
+    """nvidia-smi sampling of SM clocks and throttle reasons (read-only)."""
+
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append({"sm": float(parts[2]), "max": float(parts[3]),
+                                 "hw": parts[5], "hwt": parts[6], "swt": parts[7],
+                                 "pcap": parts[8]})
+                except ValueError:
+                    continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        reasons = set()
+        for r in rows:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
+                              ("swt", "sw_thermal_slowdown"), ("pcap", "sw_power_cap")):
+                if r[key].lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": float(np.median([r["sm"] for r in rows])),
+                "sm_max_mhz": max(r["max"] for r in rows), "reasons": sorted(reasons),
+                "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (the reported baseline and the reference arm)
+
+def _oracle_sample(w: wl.Workload, n_tok: int, inputs):
+    """One pass of the oracle over n_tok tokens of the workload: router on
+    their rows, dispatch of their k*n_tok assignments, gather and combine of
+    their rows.  Returns the seconds it took."""
+    import oracle
+    x, W, b = inputs["x_f32"][:n_tok], inputs["W"], inputs["b"]
+    rows = inputs["x_rows"][:n_tok]
+    E, sh = inputs["E"][: n_tok * w.k], inputs["shared"][:n_tok]
+    t0 = time.perf_counter()
+    r = oracle.router(x, W, b, w.n_group, w.topk_group, w.k, w.route_scale, w.mask_mode)
+    _, _, perm, inv = oracle.dispatch(r["idx"], w.N_r)
+    oracle.gather(rows, w.k, perm)
+    oracle.combine(E, r["w"].astype(np.float32), inv, sh, w.k)
+    return time.perf_counter() - t0
+
+
+def _oracle_inputs(w: wl.Workload, n_tok: int):
+    sub = w.replace(T=n_tok)
+    d = wl.gen_router_inputs(w.replace(T=n_tok))
+    return {"x_f32": d["x_f32"], "W": d["W"], "b": d["b"],
+            "x_rows": d["x_bf16"] if w.io_dtype == "bf16" else d["x_f32"],
+            "E": wl.gen_E(sub), "shared": wl.gen_shared(sub)}
+
+
+def cpu_baseline(w: wl.Workload, target_s=12.0):
+    import oracle
+    probe = 32
+    cap = 4096
+    inp = _oracle_inputs(w, cap)
+    t = _oracle_sample(w, probe, inp)
+    n = int(min(cap, max(probe, probe * target_s / max(t, 1e-3))))
+    t = _oracle_sample(w, n, inp)
+    return {"value": n / t, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{n} tokens of {w.name} through the fp64 oracle (router, dispatch, "
+                      f"gather, combine), one pass, {t:.1f} s"}
+
+
+def run_reference(args, w: wl.Workload, rank: int):
+    if rank != 0:
+        return
+    import oracle
+    probe = _oracle_sample(w, 16, _oracle_inputs(w, 16))
+    per_step_s = 150.0 / max(1, args.steps + args.warmup)  # whole run within minutes
+    n = int(min(512, max(8, 16 * min(per_step_s, 6.0) / max(probe, 1e-3))))
+    inp = _oracle_inputs(w, n)
+    for _ in range(args.warmup):
+        _oracle_sample(w, n, inp)
+    times = [_oracle_sample(w, n, inp) for _ in range(args.steps)]
+    total = sum(times)
+    value = n * args.steps / total
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": _config(w, extra={"sample_tokens_per_step": n}),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.num_threads(),
+                         "kind": "oracle",
+                         "sample": f"{n} tokens of {w.name} per step (fp64 oracle: router, "
+                                   f"dispatch, gather, combine)"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def _config(w: wl.Workload, extra=None):
+    c = {"workload": w.name, "T": w.T, "d": w.d, "N_r": w.N_r, "n_group": w.n_group,
+         "topk_group": w.topk_group, "k": w.k, "route_scale": w.route_scale,
+         "mask": "-inf" if w.mask_mode == wl.MASK_NEG_INF else "zero",
+         "rows_dtype": w.io_dtype, "router_precision": "3xTF32 (tcgen05 kind::tf32)",
+         "l2": "inputs larger than L2 (x fp32 470 MB + E 1.88 GB + shared/y per step)",
+         "parallelism": "replicas (token batches per GPU, no collective)"}
+    if extra:
+        c.update(extra)
+    return c
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+
+def run_ours(args, w: wl.Workload, rank: int, world: int):
+    import torch
+    import torch.distributed as dist
+
+    import token_dispatch_fp32_b200 as mr
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.Stream(dev)
+
+    # inputs (seeded per rank; every rank routes its own batch)
+    wr = w.replace(seed=w.seed + 1000 * rank)
+    d = wl.gen_router_inputs(wr)
+    x32 = torch.from_numpy(d["x_f32"]).to(dev)
+    xb = torch.from_numpy(d["x_bf16"]).view(torch.bfloat16).to(dev)
+    Wd = torch.from_numpy(d["W"]).to(dev)
+    bd = torch.from_numpy(d["b"]).to(dev)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(wr.seed)
+    E = torch.randn((w.T * w.k, w.d), generator=gen, device=dev, dtype=torch.float32).to(
+        torch.bfloat16)
+    shared = torch.randn((w.T, w.d), generator=gen, device=dev, dtype=torch.float32).to(
+        torch.bfloat16)
+    idx = torch.empty((w.T, w.k), dtype=torch.int32, device=dev)
+    wt = torch.empty((w.T, w.k), dtype=torch.float32, device=dev)
+    counts = torch.empty(w.N_r, dtype=torch.int32, device=dev)
+    offsets = torch.empty(w.N_r + 1, dtype=torch.int32, device=dev)
+    perm = torch.empty(w.T * w.k, dtype=torch.int32, device=dev)
+    inv = torch.empty(w.T * w.k, dtype=torch.int32, device=dev)
+    xs = torch.empty((w.T * w.k, w.d), dtype=torch.bfloat16, device=dev)
+    y = torch.empty((w.T, w.d), dtype=torch.bfloat16, device=dev)
+    ws_r = torch.empty(max(4, mr.mr_router_workspace_size(w.T, w.d, w.N_r)), dtype=torch.uint8,
+                       device=dev)
+    ws_d = torch.empty(max(4, mr.mr_dispatch_workspace_size(w.T, w.k, w.N_r)),
+                       dtype=torch.uint8, device=dev)
+
+    names = ("router", "dispatch", "gather", "combine")
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        mr.mr_router_forward_ex(x32, Wd, bd, w.n_group, w.topk_group, w.k, w.route_scale,
+                                w.mask_mode, precision=mr.MR_PREC_3XTF32, idx_out=idx,
+                                w_out=wt, workspace=ws_r, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+        mr.mr_dispatch(idx, w.N_r, counts=counts, offsets=offsets, perm=perm, inv_perm=inv,
+                       workspace=ws_d, stream=stream)
+        if ev is not None:
+            ev[2].record(stream)
+        mr.mr_gather_rows(xb, w.k, perm=perm, inv_perm=inv, xs=xs, stream=stream)
+        if ev is not None:
+            ev[3].record(stream)
+        mr.mr_combine(E, wt, inv, shared, y=y, stream=stream)
+        if ev is not None:
+            ev[4].record(stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    assert mr.mr_get_error(stream) == mr.MR_OK
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    clocks = Clocks(local)
+    clocks.start()
+    barrier()
+    torch.cuda.synchronize(dev)
+    l0 = mr.mr_launch_count()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    launches = mr.mr_launch_count() - l0
+    barrier()
+    clk = clocks.stop()
+    ms = start.elapsed_time(end) / args.steps
+    stage_ms = {n: float(np.mean([e[j].elapsed_time(e[j + 1]) for e in evs]))
+                for j, n in enumerate(names)}
+    assert mr.mr_get_error(stream) == mr.MR_OK
+
+    t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_max = float(t.item())
+
+    # ---- end to end: pinned host inputs -> device -> path -> host result ----
+    e2e = None
+    if not args.no_e2e:
+        h_x32 = torch.empty_like(x32, device="cpu").pin_memory()
+        h_xb = torch.empty_like(xb, device="cpu").pin_memory()
+        h_E = torch.empty_like(E, device="cpu").pin_memory()
+        h_sh = torch.empty_like(shared, device="cpu").pin_memory()
+        h_y = torch.empty_like(y, device="cpu").pin_memory()
+        h_idx = torch.empty_like(idx, device="cpu").pin_memory()
+        h_w = torch.empty_like(wt, device="cpu").pin_memory()
+        for h, g in ((h_x32, x32), (h_xb, xb), (h_E, E), (h_sh, shared)):
+            h.copy_(g)
+        h2d = sum(t.numel() * t.element_size() for t in (h_x32, h_xb, h_E, h_sh))
+        d2h = sum(t.numel() * t.element_size() for t in (h_y, h_idx, h_w))
+
+        def e2e_step():
+            with torch.cuda.stream(stream):
+                x32.copy_(h_x32, non_blocking=True)
+                xb.copy_(h_xb, non_blocking=True)
+                E.copy_(h_E, non_blocking=True)
+                shared.copy_(h_sh, non_blocking=True)
+            step()
+            with torch.cuda.stream(stream):
+                h_y.copy_(y, non_blocking=True)
+                h_idx.copy_(idx, non_blocking=True)
+                h_w.copy_(wt, non_blocking=True)
+
+        n_e2e = max(2, min(args.steps, 10))
+        e2e_step()
+        torch.cuda.synchronize(dev)
+        barrier()
+        s0 = torch.cuda.Event(enable_timing=True)
+        s1 = torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        s1.record(stream)
+        torch.cuda.synchronize(dev)
+        e_ms = s0.elapsed_time(s1) / n_e2e
+        te = torch.tensor([e_ms], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        e2e = {"value": world * w.T / (float(te.item()) / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "steps": n_e2e}
+
+    if rank != 0:
+        return
+    peaks = _peaks()
+    T, dd, k, N = w.T, w.d, w.k, w.N_r
+    bytes_combine = T * (2 * k * dd + 4 * dd + 8 * k)          # E rows, shared, y, w, inv
+    bytes_gather = T * (2 * dd + 2 * k * dd + 4 * k)          # x row once, k copies, inv
+    bytes_router = T * (4 * dd + 8 * k) + 4 * N * dd + 4 * N  # x, idx/w, W, bias
+    flops_router = 2.0 * T * dd * N
+    comb_s = stage_ms["combine"] / 1e3
+    achieved = bytes_combine / comb_s / 1e9
+    traffic = None
+    ent = NCU_TRAFFIC.get("combine")
+    if ent and ent.get("src") == _src_sha("token_dispatch_fp32_b200/csrc/rows.cuh"):
+        traffic = ent["bytes"]
+    tf32_peak = peaks["bf16_tflops"] * 0.5  # nominal tf32 : bf16 dense ratio
+    stages = {
+        "router": {"ms": stage_ms["router"],
+                   "tflops_algorithmic": flops_router / (stage_ms["router"] / 1e3) / 1e12,
+                   "tflops_issued_3x": 3 * flops_router / (stage_ms["router"] / 1e3) / 1e12,
+                   "tf32_peak_tflops": tf32_peak,
+                   "frac_issued_of_tf32_peak": 3 * flops_router / (stage_ms["router"] / 1e3)
+                   / 1e12 / tf32_peak,
+                   "gbs": bytes_router / (stage_ms["router"] / 1e3) / 1e9},
+        "dispatch": {"ms": stage_ms["dispatch"]},
+        "gather": {"ms": stage_ms["gather"],
+                   "gbs": bytes_gather / (stage_ms["gather"] / 1e3) / 1e9,
+                   "frac_hbm": bytes_gather / (stage_ms["gather"] / 1e3) / 1e9 / peaks["hbm_gbs"]},
+        "combine": {"ms": stage_ms["combine"], "gbs": achieved,
+                    "frac_hbm": achieved / peaks["hbm_gbs"]},
+    }
+    line = {
+        "metric": METRIC, "value": world * T / (ms_max / 1e3), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic (seeded; x/W/b numpy PCG64, expert outputs and shared output "
+                "torch Philox on device)",
+        "config": _config(w),
+        "roofline": {"bound": "hbm", "kernel": "combine", "achieved": achieved,
+                     "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                     "traffic": traffic, "algorithmic_bytes": bytes_combine,
+                     "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json hbm_gbs)"
+                     if peaks["source"] == "measured" else "fallback 6650 GB/s"},
+        "stages": stages,
+        "gpu_launches": int(launches),
+        "clocks": clk,
+        "e2e": e2e,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w)
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", default=wl.V3_FULL.name, choices=[x.name for x in wl.ALL])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    w = wl.BY_NAME[args.workload]
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if args.impl == "reference":
+        run_reference(args, w, rank)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        run_ours(args, w, rank, world)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

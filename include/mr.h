@@ -1,0 +1,227 @@
+/*
+ * mr.h -- C ABI of libmr.so: the MoE routing hot path on NVIDIA B200 (sm_100a).
+ *
+ * The path, as the pages define it:
+ *
+ *   router    logits L = x . W^T in fp32, scores s = sigmoid(L), selection
+ *             scores c = s + bias, grouped selection (group score = sum of
+ *             the two largest c of the group, keep topk_group groups, mask
+ *             the rest), token top-k, weights = route_scale * s / (sum s +
+ *             1e-20) over the chosen experts.
+ *             (Kimi K2 "Normalize weights" page: formula G_i and the
+ *             MoEGate.forward excerpt; DeepSeek-V3.2-Exp "Normalize weights"
+ *             page: Gate.forward excerpt; DeepSeek-V3 "MoE Router" note:
+ *             affinity equation, bias, grouped routing, route_scale.)
+ *   dispatch  per-expert counts, expert offsets and the expert-sorted
+ *             permutation idxs = argsort(topk_idx.view(-1)) (stable).
+ *   gather    sorted_tokens = x[idxs // k].
+ *   combine   new_x[idxs] = expert outputs; y = sum_k w * new_x cast back to
+ *             the row dtype; y + shared-expert output.
+ *             (Kimi K2 "Add shared output" page: DeepseekV3MoE.forward and
+ *             moe_infer excerpts, formula Delta_ffn = y_routed + y_shared.)
+ *
+ * Conventions shared by every entry point
+ *  - All tensor pointers are caller-owned DEVICE pointers on the current
+ *    device, row-major and densely packed.  The library never allocates,
+ *    frees or synchronises (except mr_get_error, which must read the device).
+ *  - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy stream) and
+ *    runs asynchronously.  Arguments are validated on the host before any
+ *    launch; an invalid call launches nothing and returns a negative status.
+ *  - Index tensors are int32 (T*k < 2^31 is required and checked).
+ *  - T == 0 is valid and launches nothing.
+ *  - Device-side faults in the data (an expert id out of [0, N_r)) do not
+ *    trap: the kernel skips the entry and raises the sticky device flag that
+ *    mr_get_error() reports and clears.
+ *  - No exceptions cross the ABI.  Calls on different streams are
+ *    independent; the only shared state is that per-device error flag.
+ */
+#ifndef MR_H
+#define MR_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* cudaStream_t without including the CUDA runtime headers. */
+typedef struct CUstream_st *mr_stream_t;
+
+/* ---- status codes ------------------------------------------------------ */
+#define MR_OK 0
+#define MR_ERR_INVALID_ARG (-1) /* bad size, null pointer, inconsistent args  */
+#define MR_ERR_UNSUPPORTED (-2) /* valid but outside what the kernels support */
+#define MR_ERR_CUDA (-3)        /* a CUDA launch or query failed              */
+#define MR_ERR_DEVICE (-4)      /* device flag: bad expert id seen            */
+#define MR_ERR_TIMEOUT (-5)     /* device flag: a bounded wait gave up        */
+
+/* ---- element types of row tensors --------------------------------------- */
+#define MR_F32 0
+#define MR_BF16 1
+
+/* ---- mask value for the experts of dropped groups ------------------------
+ * MR_MASK_NEG_INF: -inf (DeepSeek-V3.2-Exp Gate.forward, masked_fill_ -inf);
+ * MR_MASK_ZERO:    0.0  (Kimi K2 / HF MoEGate.forward, masked_fill 0.0).   */
+#define MR_MASK_NEG_INF 0
+#define MR_MASK_ZERO 1
+
+/* ---- router arithmetic ----------------------------------------------------
+ * MR_PREC_3XTF32: tensor cores (tcgen05, kind::tf32), each fp32 operand split
+ *                 into a tf32 high part and a residual; hi*hi + hi*lo + lo*hi
+ *                 accumulate in fp32 (fp32-level accuracy).
+ * MR_PREC_TF32:   tensor cores, one tf32 product (about 1e-3 relative).
+ * MR_PREC_FFMA:   CUDA-core fp32 FMA (any shape; slowest).                   */
+#define MR_PREC_3XTF32 0
+#define MR_PREC_TF32 1
+#define MR_PREC_FFMA 2
+
+/* Library version, major*10000 + minor*100 + patch. */
+int mr_version(void);
+
+/* Static English text for a status code. */
+const char *mr_status_string(int status);
+
+/*
+ * mr_router_forward -- gate forward for T tokens.
+ *
+ * Computes, per token t, the k chosen experts and their weights exactly as
+ * the pages define them (see the file header).  Ties between equal selection
+ * scores (groups or experts) go to the lower index.  The k slots of a token
+ * are ordered by masked selection score descending, index ascending.
+ * When n_group == 1 the group step is skipped (it keeps every expert).
+ * A NULL bias means b = 0; the group score is still the top-2 sum.
+ *
+ *   x        [T, d] fp32 token rows (the fp32 cast of the hidden states).
+ *   W        [N_r, d] fp32 gate weight (nn.Linear layout, no Linear bias).
+ *   bias     [N_r] fp32 selection bias, or NULL.
+ *   n_group  groups; N_r % n_group == 0; group size >= 2 when n_group > 1.
+ *   topk_group  groups kept, 1 <= topk_group <= n_group.
+ *   k        experts per token, 1 <= k <= 8; with MR_MASK_NEG_INF and
+ *            n_group > 1 also k <= topk_group * (N_r / n_group).
+ *   route_scale  multiplier applied after renormalisation.
+ *   mask_mode    MR_MASK_NEG_INF or MR_MASK_ZERO.
+ *   idx_out  [T, k] int32 expert ids (written).
+ *   w_out    [T, k] fp32 weights (written).
+ *
+ * Limits: 1 <= N_r <= 512, n_group <= 32, d >= 1.  Uses 3xTF32 tensor-core
+ * arithmetic when d % 4 == 0 and N_r % 16 == 0, CUDA-core FMA otherwise.
+ * Needs no workspace.  Returns MR_OK or a negative status (nothing launched
+ * on an argument error).
+ */
+int mr_router_forward(const float *x, const float *W, const float *bias, int T,
+                      int d, int N_r, int n_group, int topk_group, int k,
+                      float route_scale, int mask_mode, int32_t *idx_out,
+                      float *w_out, mr_stream_t stream);
+
+/*
+ * mr_router_workspace_size -- bytes of device workspace that
+ * mr_router_forward_ex may use for T tokens (split-K partial logits of the
+ * small-batch path).  0 means no workspace is needed at this size.
+ */
+size_t mr_router_workspace_size(int T, int d, int N_r);
+
+/*
+ * mr_router_forward_ex -- mr_router_forward with explicit options.
+ *
+ *   x_dtype     MR_F32 ([T,d] fp32) or MR_BF16 ([T,d] bf16 hidden states;
+ *               widened to fp32 exactly inside the kernel, so the result is
+ *               identical to passing the fp32 cast).
+ *   precision   MR_PREC_3XTF32, MR_PREC_TF32 or MR_PREC_FFMA.
+ *   logits_out  [T, N_r] fp32 logits, or NULL (debug / verification only).
+ *   workspace   device buffer of workspace_bytes, or NULL.  With at least
+ *               mr_router_workspace_size(T, d, N_r) bytes, small batches use
+ *               the split-K path that spreads the weight read over all SMs.
+ * Returns MR_ERR_UNSUPPORTED when the requested precision cannot run this
+ * shape (tensor-core paths need d % 4 == 0 and N_r % 16 == 0).
+ */
+int mr_router_forward_ex(const void *x, int x_dtype, const float *W,
+                         const float *bias, int T, int d, int N_r, int n_group,
+                         int topk_group, int k, float route_scale,
+                         int mask_mode, int precision, int32_t *idx_out,
+                         float *w_out, float *logits_out, void *workspace,
+                         size_t workspace_bytes, mr_stream_t stream);
+
+/*
+ * mr_dispatch_workspace_size -- bytes of device workspace mr_dispatch needs.
+ */
+size_t mr_dispatch_workspace_size(int T, int k, int N_r);
+
+/*
+ * mr_dispatch -- moe_infer's dispatch bookkeeping (Kimi K2 "Add shared
+ * output" page, moe_infer: cnts.scatter_ / tokens_per_expert, idxs =
+ * topk_ids.view(-1).argsort(), the running start_idx/end_idx of the expert
+ * loop, and the inverse used by new_x[idxs] = outs).
+ *
+ *   idx       [T, k] int32 expert ids in [0, N_r).
+ *   counts    [N_r] int32: counts[e] = #{(t, j) : idx[t, j] == e}.
+ *   offsets   [N_r + 1] int32: exclusive prefix sum of counts.
+ *   perm      [T*k] int32: perm[i] = flat slot t*k + j of the i-th entry in
+ *             expert order; within an expert, ascending slot (stable), so
+ *             the token of sorted row i is perm[i] / k.
+ *   inv_perm  [T*k] int32 or NULL: inv_perm[perm[i]] = i.
+ *   workspace at least mr_dispatch_workspace_size(T, k, N_r) bytes; its
+ *             contents need no initialisation.
+ * Limits: 1 <= N_r <= 1024, 1 <= k <= 32.
+ * An id outside [0, N_r) is dropped: counts/offsets/perm cover the valid
+ * entries only, perm[offsets[N_r] ..] and the dropped slots' inv_perm are -1,
+ * and the device flag reports MR_ERR_DEVICE.
+ */
+int mr_dispatch(const int32_t *idx, int T, int k, int N_r, int32_t *counts,
+                int32_t *offsets, int32_t *perm, int32_t *inv_perm,
+                void *workspace, size_t workspace_bytes, mr_stream_t stream);
+
+/*
+ * mr_gather_rows -- sorted_tokens = x[idxs // k] (Kimi K2 "Add shared output"
+ * page, moe_infer).  Copies rows bit for bit.
+ *
+ *   x         [T, d] rows of `dtype` (MR_BF16 or MR_F32).
+ *   perm      [T*k] from mr_dispatch (used when inv_perm is NULL).
+ *   inv_perm  [T*k] from mr_dispatch or NULL.  When given, each token row is
+ *             read once and written to its k sorted positions.
+ *   xs        [T*k, d] output rows in expert-sorted order.
+ * Limits: 1 <= k <= 32.
+ */
+int mr_gather_rows(const void *x, int dtype, int T, int d, int k,
+                   const int32_t *perm, const int32_t *inv_perm, void *xs,
+                   mr_stream_t stream);
+
+/*
+ * mr_combine -- scatter-back, weighted combine and shared add (Kimi K2 "Add
+ * shared output" page: new_x[idxs] = outs, view(T,k,d) * topk_weight summed
+ * over k, cast back to the row dtype, then y + shared_experts(identity)).
+ *
+ *   expert_out [T*k, d] expert outputs in expert-sorted order (row i belongs
+ *              to slot perm[i]), `dtype` MR_BF16 or MR_F32.
+ *   w          [T, k] fp32 router weights.
+ *   inv_perm   [T*k] from mr_dispatch.
+ *   shared     [T, d] shared-expert output of `dtype`, or NULL.
+ *   y          [T, d] output of `dtype`.
+ * Per element: acc = sum_j w[t,j] * expert_out[inv_perm[t*k+j]] in fp32;
+ * bf16 rows: y = bf16(bf16(acc) + shared) (both roundings to nearest even);
+ * fp32 rows: y = acc + shared.
+ * Limits: 1 <= k <= 32.
+ */
+int mr_combine(const void *expert_out, int dtype, const float *w,
+               const int32_t *inv_perm, const void *shared, void *y, int T,
+               int d, int k, mr_stream_t stream);
+
+/*
+ * mr_launch_count -- number of kernels this library has launched in this
+ * process (all devices and streams), for accounting in benchmarks.
+ */
+uint64_t mr_launch_count(void);
+
+/*
+ * mr_get_error -- synchronise `stream`, then read and clear the current
+ * device's sticky error flag.  Returns MR_OK, MR_ERR_DEVICE (a bad expert id
+ * was seen), MR_ERR_TIMEOUT (a bounded wait inside a kernel gave up) or
+ * MR_ERR_CUDA (the synchronisation itself failed).
+ */
+int mr_get_error(mr_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MR_H */

@@ -1,0 +1,69 @@
+"""Gather (bit-exact) and combine (tolerance) parity on the GPU."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import token_dispatch_fp32_b200 as mr
+from parity import compare_combine, widen
+
+pytestmark = pytest.mark.gpu
+
+
+def _problem(T, d, k, N_r, dtype, seed, with_shared=True):
+    rng = np.random.default_rng(seed)
+    idx = np.stack([rng.permutation(N_r)[:k] for _ in range(T)]).astype(np.int32)
+    w = rng.uniform(0.05, 1.0, (T, k)).astype(np.float32)
+    w = (w / w.sum(1, keepdims=True) * np.float32(2.5)).astype(np.float32)
+    z = rng.standard_normal((T * k, d)).astype(np.float32)
+    sh = rng.standard_normal((T, d)).astype(np.float32) if with_shared else None
+    x = rng.standard_normal((T, d)).astype(np.float32)
+    if dtype == "bf16":
+        to = lambda a: None if a is None else (a.view(np.uint32) >> 16).astype(np.uint16)  # noqa
+        z, sh, x = to(z), to(sh), to(x)
+    return idx, w, z, sh, x
+
+
+def _dev(a):
+    t = torch.from_numpy(a)
+    return (t.view(torch.bfloat16) if a.dtype == np.uint16 else t).cuda()
+
+
+def _host(t):
+    if t.dtype == torch.bfloat16:
+        return t.view(torch.int16).cpu().numpy().view(np.uint16)
+    return t.cpu().numpy()
+
+
+ROW_CASES = [  # T, d, k, N_r, dtype
+    (300, 7168, 8, 256, "bf16"),
+    (257, 512, 4, 64, "f32"),
+    (100, 1001, 3, 40, "bf16"),   # odd row: element path
+    (64, 37, 2, 8, "f32"),        # ragged fp32 row
+    (1, 8, 1, 1, "bf16"),
+    (128, 64, 32, 64, "bf16"),    # k = 32
+]
+
+
+@pytest.mark.parametrize("T,d,k,N_r,dtype", ROW_CASES)
+@pytest.mark.parametrize("use_inv", [True, False], ids=["inv", "perm"])
+def test_gather_bit_exact(T, d, k, N_r, dtype, use_inv):
+    idx, _, _, _, x = _problem(T, d, k, N_r, dtype, seed=T * 7 + d)
+    _, _, perm, inv = oracle.dispatch(idx, N_r)
+    xs = mr.mr_gather_rows(_dev(x), k, perm=torch.from_numpy(perm).cuda(),
+                           inv_perm=torch.from_numpy(inv).cuda() if use_inv else None)
+    assert mr.mr_get_error() == mr.MR_OK
+    assert np.array_equal(_host(xs), oracle.gather(x, k, perm))
+
+
+@pytest.mark.parametrize("T,d,k,N_r,dtype", ROW_CASES)
+@pytest.mark.parametrize("with_shared", [True, False], ids=["shared", "noshared"])
+def test_combine_matches_oracle(T, d, k, N_r, dtype, with_shared):
+    idx, w, E, sh, _ = _problem(T, d, k, N_r, dtype, seed=T * 11 + d, with_shared=with_shared)
+    _, _, perm, inv = oracle.dispatch(idx, N_r)
+    y = mr.mr_combine(_dev(E), torch.from_numpy(w).cuda(), torch.from_numpy(inv).cuda(),
+                      None if sh is None else _dev(sh))
+    assert mr.mr_get_error() == mr.MR_OK
+    ry, rr = oracle.combine(E, w, inv, sh, k)
+    stats = compare_combine(widen(_host(y)), ry, rr, None if sh is None else widen(sh))
+    print(T, d, k, dtype, with_shared, stats)

@@ -1,0 +1,244 @@
+"""ctypes binding of libmr.so (include/mr.h): argument marshalling only.
+
+Every function here takes torch CUDA tensors, checks dtype/shape/contiguity,
+allocates missing outputs with torch (device memory is PyTorch's job), and
+calls the C entry point of the same name on the current torch stream.  No
+step of the routing path is computed in Python; there is no CPU fallback:
+if libmr.so is missing or a call fails, an exception is raised.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmr.so")
+
+MR_OK = 0
+MR_ERR_INVALID_ARG = -1
+MR_ERR_UNSUPPORTED = -2
+MR_ERR_CUDA = -3
+MR_ERR_DEVICE = -4
+MR_ERR_TIMEOUT = -5
+
+MR_F32 = 0
+MR_BF16 = 1
+MR_MASK_NEG_INF = 0
+MR_MASK_ZERO = 1
+MR_PREC_3XTF32 = 0
+MR_PREC_TF32 = 1
+MR_PREC_FFMA = 2
+
+_lib = None
+
+
+class MRError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} failed: status {status} ({status_string(status)})")
+
+
+def lib():
+    """The loaded libmr.so (raises ImportError when it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is not built; run "
+                              "`python -m token_dispatch_fp32_b200.build`")
+        L = C.CDLL(LIB_PATH)
+        p, i, f, sz = C.c_void_p, C.c_int, C.c_float, C.c_size_t
+        L.mr_version.restype = i
+        L.mr_status_string.argtypes = [i]
+        L.mr_status_string.restype = C.c_char_p
+        L.mr_router_forward.argtypes = [p, p, p, i, i, i, i, i, i, f, i, p, p, p]
+        L.mr_router_forward_ex.argtypes = [p, i, p, p, i, i, i, i, i, i, f, i, i, p, p, p, p,
+                                           sz, p]
+        L.mr_router_workspace_size.argtypes = [i, i, i]
+        L.mr_router_workspace_size.restype = sz
+        L.mr_dispatch_workspace_size.argtypes = [i, i, i]
+        L.mr_dispatch_workspace_size.restype = sz
+        L.mr_dispatch.argtypes = [p, i, i, i, p, p, p, p, p, sz, p]
+        L.mr_gather_rows.argtypes = [p, i, i, i, i, p, p, p, p]
+        L.mr_combine.argtypes = [p, i, p, p, p, p, i, i, i, p]
+        L.mr_get_error.argtypes = [p]
+        L.mr_launch_count.restype = C.c_uint64
+        for fn in ("mr_router_forward", "mr_router_forward_ex", "mr_dispatch",
+                   "mr_gather_rows", "mr_combine", "mr_get_error"):
+            getattr(L, fn).restype = i
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().mr_status_string(status).decode()
+
+
+def _check(fn: str, status: int) -> None:
+    if status != MR_OK:
+        raise MRError(fn, status)
+
+
+def _ptr(t):
+    return None if t is None else C.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return C.c_void_p(stream.cuda_stream)
+
+
+def _need(t, name, dtype=None, shape=None):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    return t
+
+
+def _row_dtype(t):
+    if t.dtype == torch.bfloat16:
+        return MR_BF16
+    if t.dtype == torch.float32:
+        return MR_F32
+    raise TypeError("row tensors must be bfloat16 or float32")
+
+
+def version() -> int:
+    return int(lib().mr_version())
+
+
+def mr_router_forward(x, W, bias, n_group, topk_group, k, route_scale, mask_mode,
+                      idx_out=None, w_out=None, stream=None):
+    """Gate forward (include/mr.h).  x [T,d] fp32, W [N_r,d] fp32, bias [N_r]
+    fp32 or None.  Returns (idx [T,k] int32, w [T,k] fp32)."""
+    _need(x, "x", torch.float32)
+    T, d = x.shape
+    _need(W, "W", torch.float32)
+    N_r = W.shape[0]
+    _need(W, "W", torch.float32, (N_r, d))
+    if bias is not None:
+        _need(bias, "bias", torch.float32, (N_r,))
+    idx_out = torch.empty((T, k), dtype=torch.int32, device=x.device) if idx_out is None else \
+        _need(idx_out, "idx_out", torch.int32, (T, k))
+    w_out = torch.empty((T, k), dtype=torch.float32, device=x.device) if w_out is None else \
+        _need(w_out, "w_out", torch.float32, (T, k))
+    _check("mr_router_forward", lib().mr_router_forward(
+        _ptr(x), _ptr(W), _ptr(bias), T, d, N_r, n_group, topk_group, k, float(route_scale),
+        mask_mode, _ptr(idx_out), _ptr(w_out), _stream(stream)))
+    return idx_out, w_out
+
+
+def mr_router_workspace_size(T, d, N_r) -> int:
+    return int(lib().mr_router_workspace_size(T, d, N_r))
+
+
+def mr_router_forward_ex(x, W, bias, n_group, topk_group, k, route_scale, mask_mode,
+                         precision=MR_PREC_3XTF32, idx_out=None, w_out=None, logits_out=None,
+                         workspace=None, stream=None):
+    """mr_router_forward with x dtype (fp32 or bf16), precision, optional
+    logits output and workspace.  Returns (idx, w)."""
+    _need(x, "x")
+    x_dtype = _row_dtype(x)
+    T, d = x.shape
+    N_r = W.shape[0]
+    _need(W, "W", torch.float32, (N_r, d))
+    if bias is not None:
+        _need(bias, "bias", torch.float32, (N_r,))
+    idx_out = torch.empty((T, k), dtype=torch.int32, device=x.device) if idx_out is None else \
+        _need(idx_out, "idx_out", torch.int32, (T, k))
+    w_out = torch.empty((T, k), dtype=torch.float32, device=x.device) if w_out is None else \
+        _need(w_out, "w_out", torch.float32, (T, k))
+    if logits_out is not None:
+        _need(logits_out, "logits_out", torch.float32, (T, N_r))
+    ws_bytes = 0
+    if workspace is not None:
+        _need(workspace, "workspace")
+        ws_bytes = workspace.numel() * workspace.element_size()
+    _check("mr_router_forward_ex", lib().mr_router_forward_ex(
+        _ptr(x), x_dtype, _ptr(W), _ptr(bias), T, d, N_r, n_group, topk_group, k,
+        float(route_scale), mask_mode, precision, _ptr(idx_out), _ptr(w_out), _ptr(logits_out),
+        _ptr(workspace), ws_bytes, _stream(stream)))
+    return idx_out, w_out
+
+
+def mr_dispatch_workspace_size(T, k, N_r) -> int:
+    return int(lib().mr_dispatch_workspace_size(T, k, N_r))
+
+
+def mr_dispatch(idx, N_r, counts=None, offsets=None, perm=None, inv_perm=None, workspace=None,
+                want_inv=True, stream=None):
+    """Dispatch bookkeeping.  idx [T,k] int32.  Returns (counts, offsets,
+    perm, inv_perm) as int32 tensors (inv_perm None when want_inv is False)."""
+    _need(idx, "idx", torch.int32)
+    T, k = idx.shape
+    dev = idx.device
+    counts = torch.empty(N_r, dtype=torch.int32, device=dev) if counts is None else \
+        _need(counts, "counts", torch.int32, (N_r,))
+    offsets = torch.empty(N_r + 1, dtype=torch.int32, device=dev) if offsets is None else \
+        _need(offsets, "offsets", torch.int32, (N_r + 1,))
+    perm = torch.empty(T * k, dtype=torch.int32, device=dev) if perm is None else \
+        _need(perm, "perm", torch.int32, (T * k,))
+    if inv_perm is None and want_inv:
+        inv_perm = torch.empty(T * k, dtype=torch.int32, device=dev)
+    elif inv_perm is not None:
+        _need(inv_perm, "inv_perm", torch.int32, (T * k,))
+    need = mr_dispatch_workspace_size(T, k, N_r)
+    if workspace is None:
+        workspace = torch.empty(max(need, 4), dtype=torch.uint8, device=dev)
+    _need(workspace, "workspace")
+    _check("mr_dispatch", lib().mr_dispatch(
+        _ptr(idx), T, k, N_r, _ptr(counts), _ptr(offsets), _ptr(perm), _ptr(inv_perm),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
+    return counts, offsets, perm, inv_perm
+
+
+def mr_gather_rows(x, k, perm=None, inv_perm=None, xs=None, stream=None):
+    """sorted rows xs [T*k, d] = x[perm // k] (x bf16 or fp32)."""
+    _need(x, "x")
+    T, d = x.shape
+    dt = _row_dtype(x)
+    if perm is not None:
+        _need(perm, "perm", torch.int32, (T * k,))
+    if inv_perm is not None:
+        _need(inv_perm, "inv_perm", torch.int32, (T * k,))
+    xs = torch.empty((T * k, d), dtype=x.dtype, device=x.device) if xs is None else \
+        _need(xs, "xs", x.dtype, (T * k, d))
+    _check("mr_gather_rows", lib().mr_gather_rows(
+        _ptr(x), dt, T, d, k, _ptr(perm), _ptr(inv_perm), _ptr(xs), _stream(stream)))
+    return xs
+
+
+def mr_combine(expert_out, w, inv_perm, shared=None, y=None, stream=None):
+    """y [T,d] = combine of expert_out [T*k,d] with w [T,k] (+ shared [T,d])."""
+    _need(w, "w", torch.float32)
+    T, k = w.shape
+    _need(expert_out, "expert_out")
+    d = expert_out.shape[1]
+    _need(expert_out, "expert_out", None, (T * k, d))
+    dt = _row_dtype(expert_out)
+    _need(inv_perm, "inv_perm", torch.int32, (T * k,))
+    if shared is not None:
+        _need(shared, "shared", expert_out.dtype, (T, d))
+    y = torch.empty((T, d), dtype=expert_out.dtype, device=expert_out.device) if y is None else \
+        _need(y, "y", expert_out.dtype, (T, d))
+    _check("mr_combine", lib().mr_combine(
+        _ptr(expert_out), dt, _ptr(w), _ptr(inv_perm), _ptr(shared), _ptr(y), T, d, k,
+        _stream(stream)))
+    return y
+
+
+def mr_launch_count() -> int:
+    """Kernels launched by libmr.so in this process so far."""
+    return int(lib().mr_launch_count())
+
+
+def mr_get_error(stream=None) -> int:
+    """Synchronise the stream and read/clear the device error flag (status)."""
+    return int(lib().mr_get_error(_stream(stream)))

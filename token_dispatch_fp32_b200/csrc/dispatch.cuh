@@ -1,0 +1,157 @@
+// dispatch.cuh -- moe_infer dispatch bookkeeping (Kimi K2 "Add shared output"
+// page, moe_infer): tokens_per_expert, the running expert offsets and the
+// stable expert-sorted permutation idxs = argsort(topk_ids.view(-1)), plus its
+// inverse.  A counting sort in three launches:
+//   1. count:   each CTA histograms a fixed chunk of the flat ids in shared
+//               memory with warp-aggregated atomics (__match_any_sync).
+//   2. scan:    one CTA turns the per-chunk histograms into counts, offsets
+//               and each chunk's starting position per expert.
+//   3. scatter: each CTA re-reads its chunk; each warp owns a contiguous
+//               sub-chunk, so (chunk base + warp prefix + in-warp rank) gives
+//               a stable position without any global atomics.
+#pragma once
+
+#include "mr_common.cuh"
+
+namespace mr {
+
+constexpr int kDispThreads = 256;
+constexpr int kDispWarps = kDispThreads / 32;
+constexpr int kDispChunk = 4096;                     // flat entries per CTA
+constexpr int kDispSub = kDispChunk / kDispWarps;    // entries per warp
+constexpr int kDispMaxExperts = 1024;
+
+__host__ __device__ inline long disp_num_chunks(long n) { return (n + kDispChunk - 1) / kDispChunk; }
+
+// Valid expert id, or -1 for one that is out of range (raises the flag once
+// per warp that sees it).
+__device__ __forceinline__ int disp_load(const int32_t* __restrict__ idx, long i, long n, int N_r,
+                                         bool* bad) {
+  if (i >= n) return -1;
+  const int e = idx[i];
+  if (e < 0 || e >= N_r) {
+    *bad = true;
+    return -1;
+  }
+  return e;
+}
+
+__global__ void __launch_bounds__(kDispThreads)
+    dispatch_count_kernel(const int32_t* __restrict__ idx, long n, int N_r,
+                          int32_t* __restrict__ chunk_hist) {
+  extern __shared__ int hist[];
+  for (int e = threadIdx.x; e < N_r; e += kDispThreads) hist[e] = 0;
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long base = (long)blockIdx.x * kDispChunk + (long)warp * kDispSub;
+  bool bad = false;
+  for (int r = 0; r < kDispSub; r += 32) {
+    const int e = disp_load(idx, base + r + lane, n, N_r, &bad);
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    if (e >= 0 && lane == __ffs(peers) - 1) atomicAdd(&hist[e], __popc(peers));
+  }
+  if (__any_sync(0xffffffffu, bad) && lane == 0) mr_raise(MR_FLAG_BAD_INDEX);
+  __syncthreads();
+  for (int e = threadIdx.x; e < N_r; e += kDispThreads)
+    chunk_hist[(long)blockIdx.x * N_r + e] = hist[e];
+}
+
+// One CTA of 1024 threads.  chunk_hist[c][e] is replaced by the position in
+// perm where chunk c's first entry of expert e goes.
+__global__ void __launch_bounds__(1024)
+    dispatch_scan_kernel(int32_t* __restrict__ chunk_hist, long nchunks, int N_r, long n,
+                         int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+                         int32_t* __restrict__ perm) {
+  __shared__ int warp_tot[32];
+  __shared__ int total_s;
+  const int e = threadIdx.x, lane = e & 31, warp = e >> 5;
+  int cnt = 0;
+  if (e < N_r)
+    for (long c = 0; c < nchunks; ++c) cnt += chunk_hist[c * N_r + e];
+  // exclusive scan of cnt over e (block of 1024 = 32 warps)
+  int incl = cnt;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += v;
+  }
+  if (lane == 31) warp_tot[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int t = warp_tot[lane];
+    int ti = t;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, ti, off);
+      if (lane >= off) ti += v;
+    }
+    warp_tot[lane] = ti - t;  // exclusive prefix of warp totals
+    if (lane == 31) total_s = ti;
+  }
+  __syncthreads();
+  const int excl = warp_tot[warp] + incl - cnt;
+  if (e < N_r) {
+    counts[e] = cnt;
+    offsets[e] = excl;
+    int run = excl;
+    for (long c = 0; c < nchunks; ++c) {
+      const int h = chunk_hist[c * N_r + e];
+      chunk_hist[c * N_r + e] = run;
+      run += h;
+    }
+  }
+  const int total = total_s;
+  if (e == 0) offsets[N_r] = total;
+  // slots of dropped (out-of-range) entries
+  for (long i = total + e; i < n; i += 1024) perm[i] = -1;
+}
+
+__global__ void __launch_bounds__(kDispThreads)
+    dispatch_scatter_kernel(const int32_t* __restrict__ idx, long n, int N_r,
+                            const int32_t* __restrict__ chunk_base, int32_t* __restrict__ perm,
+                            int32_t* __restrict__ inv) {
+  extern __shared__ int wbase[];  // [kDispWarps][N_r]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = threadIdx.x; i < kDispWarps * N_r; i += kDispThreads) wbase[i] = 0;
+  __syncthreads();
+  const long base = (long)blockIdx.x * kDispChunk + (long)warp * kDispSub;
+  int* mine = wbase + warp * N_r;
+  bool bad = false;
+  // per-warp histogram of this warp's sub-chunk
+  for (int r = 0; r < kDispSub; r += 32) {
+    const int e = disp_load(idx, base + r + lane, n, N_r, &bad);
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    if (e >= 0 && lane == __ffs(peers) - 1) mine[e] += __popc(peers);
+    __syncwarp();
+  }
+  __syncthreads();
+  // warp-exclusive prefix per expert, offset by this chunk's base
+  for (int e = threadIdx.x; e < N_r; e += kDispThreads) {
+    int run = chunk_base[(long)blockIdx.x * N_r + e];
+#pragma unroll
+    for (int w = 0; w < kDispWarps; ++w) {
+      const int h = wbase[w * N_r + e];
+      wbase[w * N_r + e] = run;
+      run += h;
+    }
+  }
+  __syncthreads();
+  const unsigned lt = (1u << lane) - 1u;
+  for (int r = 0; r < kDispSub; r += 32) {
+    const long i = base + r + lane;
+    const int e = disp_load(idx, i, n, N_r, &bad);
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    if (e >= 0) {
+      const int pos = mine[e] + __popc(peers & lt);
+      perm[pos] = (int32_t)i;
+      if (inv) inv[i] = pos;
+    } else if (i < n && inv) {
+      inv[i] = -1;
+    }
+    __syncwarp();
+    if (e >= 0 && lane == __ffs(peers) - 1) mine[e] += __popc(peers);
+    __syncwarp();
+  }
+}
+
+}  // namespace mr

@@ -1,0 +1,377 @@
+// mr.cu -- libmr.so: the extern "C" entry points declared in include/mr.h.
+//
+// Host code only validates arguments, builds TMA descriptors and launches the
+// kernels of this directory on the caller's stream; every step of the routing
+// path runs on the GPU.  Built as one translation unit for sm_100a.
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cmath>
+#include <mutex>
+
+#include "dispatch.cuh"
+#include "mr_common.cuh"
+#include "router_ffma.cuh"
+#include "router_tc.cuh"
+#include "rows.cuh"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+int g_num_sms[kMaxDevices];
+int g_cc_major[kMaxDevices];
+std::once_flag g_dev_once[kMaxDevices];
+
+// Properties of the current device, queried once per device.
+bool device_info(int* sms, int* cc_major) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
+  std::call_once(g_dev_once[dev], [dev] {
+    int v = 0;
+    g_num_sms[dev] = cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess ? v : 0;
+    g_cc_major[dev] = cudaDeviceGetAttribute(&v, cudaDevAttrComputeCapabilityMajor, dev) == cudaSuccess ? v : 0;
+  });
+  *sms = g_num_sms[dev];
+  *cc_major = g_cc_major[dev];
+  return *sms > 0;
+}
+
+std::atomic<uint64_t> g_launches{0};
+
+// Status of the launch just made (and count it).
+int launch_status() {
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? MR_OK : MR_ERR_CUDA;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ---- TMA descriptors -------------------------------------------------------
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  return g_encode;
+}
+
+// Row-major fp32 matrix [rows, cols], box [box_rows, box_cols], swizzled rows.
+bool make_map_f32(CUtensorMap* map, const float* base, uint64_t rows, uint64_t cols,
+                  uint32_t box_rows, uint32_t box_cols) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * sizeof(float)};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUtensorMapSwizzle sw =
+      box_cols * 4 == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(base), dims, strides,
+             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ---- router -----------------------------------------------------------------
+
+int validate_router(const void* x, int x_dtype, const float* W, int T, int d, int N_r,
+                    int n_group, int topk_group, int k, float route_scale, int mask_mode,
+                    int precision, const int32_t* idx_out, const float* w_out) {
+  if (T < 0 || d <= 0 || N_r <= 0 || n_group <= 0 || k <= 0) return MR_ERR_INVALID_ARG;
+  if (N_r % n_group != 0 || topk_group < 1 || topk_group > n_group || k > N_r)
+    return MR_ERR_INVALID_ARG;
+  if (n_group > 1 && N_r / n_group < 2) return MR_ERR_INVALID_ARG;
+  if (mask_mode != MR_MASK_NEG_INF && mask_mode != MR_MASK_ZERO) return MR_ERR_INVALID_ARG;
+  if (mask_mode == MR_MASK_NEG_INF && n_group > 1 && k > topk_group * (N_r / n_group))
+    return MR_ERR_INVALID_ARG;
+  if (x_dtype != MR_F32 && x_dtype != MR_BF16) return MR_ERR_INVALID_ARG;
+  if (precision != MR_PREC_3XTF32 && precision != MR_PREC_TF32 && precision != MR_PREC_FFMA)
+    return MR_ERR_INVALID_ARG;
+  if (!std::isfinite(route_scale)) return MR_ERR_INVALID_ARG;
+  if ((long long)T * k >= (1LL << 31) || (long long)T * d >= (1LL << 40)) return MR_ERR_INVALID_ARG;
+  if (T > 0 && (!x || !W || !idx_out || !w_out)) return MR_ERR_INVALID_ARG;
+  if (N_r > 512 || n_group > 32 || k > 8) return MR_ERR_UNSUPPORTED;
+  return MR_OK;
+}
+
+bool tc_shape_ok(const void* x, int x_dtype, const float* W, int d, int N_r) {
+  return x_dtype == MR_F32 && d % 4 == 0 && N_r % 16 == 0 && N_r >= 16 && aligned16(x) &&
+         aligned16(W);
+}
+
+template <int NJ, bool XBF16>
+int launch_ffma_nj(const void* x, const float* W, const float* bias, int T, int d, int N_r,
+                   int n_group, int topk_group, int k, float route_scale, int mask_mode,
+                   int32_t* idx_out, float* w_out, float* logits_out, cudaStream_t st) {
+  const size_t smem = mr::ffma_smem_bytes(NJ);
+  auto kern = mr::router_ffma_kernel<NJ, XBF16>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+      cudaSuccess)
+    return MR_ERR_CUDA;
+  const unsigned grid = (unsigned)((T + mr::kFfmaTokens - 1) / mr::kFfmaTokens);
+  kern<<<grid, mr::kFfmaThreads, smem, st>>>(x, W, bias, T, d, N_r, n_group, topk_group, k,
+                                              route_scale, mask_mode, idx_out, w_out, logits_out);
+  return launch_status();
+}
+
+template <bool XBF16>
+int launch_ffma(const void* x, const float* W, const float* bias, int T, int d, int N_r,
+                int n_group, int topk_group, int k, float route_scale, int mask_mode,
+                int32_t* idx_out, float* w_out, float* logits_out, cudaStream_t st) {
+  const int nj = (N_r + 31) / 32;
+#define MR_FFMA_CASE(NJV)                                                                       \
+  if (nj <= NJV)                                                                              \
+    return launch_ffma_nj<NJV, XBF16>(x, W, bias, T, d, N_r, n_group, topk_group, k,          \
+                                      route_scale, mask_mode, idx_out, w_out, logits_out, st);
+  MR_FFMA_CASE(1)
+  MR_FFMA_CASE(2)
+  MR_FFMA_CASE(4)
+  MR_FFMA_CASE(8)
+  MR_FFMA_CASE(12)
+  MR_FFMA_CASE(16)
+#undef MR_FFMA_CASE
+  return MR_ERR_UNSUPPORTED;
+}
+
+int launch_tc(const float* x, const float* W, const float* bias, int T, int d, int N_r,
+              int n_group, int topk_group, int k, float route_scale, int mask_mode, bool use3x,
+              int32_t* idx_out, float* w_out, float* logits_out, cudaStream_t st) {
+  const mr::tc::Plan plan = mr::tc::make_plan(N_r, 4);
+  if (plan.stages < 1) return MR_ERR_UNSUPPORTED;
+  const int n0 = N_r < 256 ? N_r : 256;
+  const int n1 = N_r - n0;
+  CUtensorMap mx, mw0, mw1;
+  if (!make_map_f32(&mx, x, (uint64_t)T, (uint64_t)d, mr::tc::BM, plan.BK)) return MR_ERR_CUDA;
+  if (!make_map_f32(&mw0, W, (uint64_t)N_r, (uint64_t)d, n0, plan.BK)) return MR_ERR_CUDA;
+  if (n1 > 0) {
+    if (!make_map_f32(&mw1, W, (uint64_t)N_r, (uint64_t)d, n1, plan.BK)) return MR_ERR_CUDA;
+  } else {
+    mw1 = mw0;
+  }
+  mr::tc::Params P;
+  P.T = T;
+  P.d = d;
+  P.N = N_r;
+  P.n_group = n_group;
+  P.topk_group = topk_group;
+  P.k = k;
+  P.mask_mode = mask_mode;
+  P.num_kc = (d + plan.BK - 1) / plan.BK;
+  P.use3x = use3x ? 1 : 0;
+  P.route_scale = route_scale;
+  P.bias = bias;
+  P.idx_out = idx_out;
+  P.w_out = w_out;
+  P.logits_out = logits_out;
+  const size_t smem = plan.total + 1024;
+  if (cudaFuncSetAttribute(mr::tc::router_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem) != cudaSuccess)
+    return MR_ERR_CUDA;
+  const unsigned grid = (unsigned)((T + mr::tc::BM - 1) / mr::tc::BM);
+  mr::tc::router_tc_kernel<<<grid, mr::tc::kThreads, smem, st>>>(mx, mw0, mw1, P);
+  return launch_status();
+}
+
+}  // namespace
+
+extern "C" {
+
+int mr_version(void) { return 100; }
+
+const char* mr_status_string(int status) {
+  switch (status) {
+    case MR_OK: return "ok";
+    case MR_ERR_INVALID_ARG: return "invalid argument";
+    case MR_ERR_UNSUPPORTED: return "unsupported shape, option or device";
+    case MR_ERR_CUDA: return "CUDA launch or query failed";
+    case MR_ERR_DEVICE: return "device flag: expert id out of range";
+    case MR_ERR_TIMEOUT: return "device flag: bounded wait timed out";
+    default: return "unknown status";
+  }
+}
+
+size_t mr_router_workspace_size(int T, int d, int N_r) {
+  (void)T;
+  (void)d;
+  (void)N_r;
+  return 0;
+}
+
+int mr_router_forward_ex(const void* x, int x_dtype, const float* W, const float* bias, int T,
+                         int d, int N_r, int n_group, int topk_group, int k, float route_scale,
+                         int mask_mode, int precision, int32_t* idx_out, float* w_out,
+                         float* logits_out, void* workspace, size_t workspace_bytes,
+                         mr_stream_t stream) {
+  (void)workspace;
+  (void)workspace_bytes;
+  int st = validate_router(x, x_dtype, W, T, d, N_r, n_group, topk_group, k, route_scale,
+                           mask_mode, precision, idx_out, w_out);
+  if (st != MR_OK || T == 0) return st;
+  int sms = 0, cc = 0;
+  if (!device_info(&sms, &cc)) return MR_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (precision == MR_PREC_FFMA) {
+    return x_dtype == MR_BF16
+               ? launch_ffma<true>(x, W, bias, T, d, N_r, n_group, topk_group, k, route_scale,
+                                   mask_mode, idx_out, w_out, logits_out, s)
+               : launch_ffma<false>(x, W, bias, T, d, N_r, n_group, topk_group, k, route_scale,
+                                    mask_mode, idx_out, w_out, logits_out, s);
+  }
+  if (cc != 10 || !tc_shape_ok(x, x_dtype, W, d, N_r)) return MR_ERR_UNSUPPORTED;
+  return launch_tc(static_cast<const float*>(x), W, bias, T, d, N_r, n_group, topk_group, k,
+                   route_scale, mask_mode, precision == MR_PREC_3XTF32, idx_out, w_out,
+                   logits_out, s);
+}
+
+int mr_router_forward(const float* x, const float* W, const float* bias, int T, int d, int N_r,
+                      int n_group, int topk_group, int k, float route_scale, int mask_mode,
+                      int32_t* idx_out, float* w_out, mr_stream_t stream) {
+  int st = validate_router(x, MR_F32, W, T, d, N_r, n_group, topk_group, k, route_scale,
+                           mask_mode, MR_PREC_3XTF32, idx_out, w_out);
+  if (st != MR_OK || T == 0) return st;
+  int sms = 0, cc = 0;
+  if (!device_info(&sms, &cc)) return MR_ERR_CUDA;
+  const int prec = (cc == 10 && tc_shape_ok(x, MR_F32, W, d, N_r)) ? MR_PREC_3XTF32 : MR_PREC_FFMA;
+  return mr_router_forward_ex(x, MR_F32, W, bias, T, d, N_r, n_group, topk_group, k, route_scale,
+                              mask_mode, prec, idx_out, w_out, nullptr, nullptr, 0, stream);
+}
+
+// ---- dispatch -----------------------------------------------------------------
+
+size_t mr_dispatch_workspace_size(int T, int k, int N_r) {
+  if (T <= 0 || k <= 0 || N_r <= 0) return 0;
+  return (size_t)mr::disp_num_chunks((long)T * k) * (size_t)N_r * sizeof(int32_t);
+}
+
+int mr_dispatch(const int32_t* idx, int T, int k, int N_r, int32_t* counts, int32_t* offsets,
+                int32_t* perm, int32_t* inv_perm, void* workspace, size_t workspace_bytes,
+                mr_stream_t stream) {
+  if (T < 0 || k <= 0 || N_r <= 0) return MR_ERR_INVALID_ARG;
+  if ((long long)T * k >= (1LL << 31)) return MR_ERR_INVALID_ARG;
+  if (k > 32 || N_r > mr::kDispMaxExperts) return MR_ERR_UNSUPPORTED;
+  if (!counts || !offsets) return MR_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (T == 0) {
+    if (cudaMemsetAsync(counts, 0, sizeof(int32_t) * N_r, s) != cudaSuccess ||
+        cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (N_r + 1), s) != cudaSuccess)
+      return MR_ERR_CUDA;
+    return MR_OK;
+  }
+  if (!idx || !perm || !workspace) return MR_ERR_INVALID_ARG;
+  if (workspace_bytes < mr_dispatch_workspace_size(T, k, N_r)) return MR_ERR_INVALID_ARG;
+  const long n = (long)T * k;
+  const long nchunks = mr::disp_num_chunks(n);
+  int32_t* hist = static_cast<int32_t*>(workspace);
+  mr::dispatch_count_kernel<<<(unsigned)nchunks, mr::kDispThreads, sizeof(int) * N_r, s>>>(
+      idx, n, N_r, hist);
+  if (launch_status() != MR_OK) return MR_ERR_CUDA;
+  mr::dispatch_scan_kernel<<<1, 1024, 0, s>>>(hist, nchunks, N_r, n, counts, offsets, perm);
+  if (launch_status() != MR_OK) return MR_ERR_CUDA;
+  const size_t smem = sizeof(int) * mr::kDispWarps * N_r;
+  if (smem > 48 * 1024 &&
+      cudaFuncSetAttribute(mr::dispatch_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem) != cudaSuccess)
+    return MR_ERR_CUDA;
+  mr::dispatch_scatter_kernel<<<(unsigned)nchunks, mr::kDispThreads, smem, s>>>(idx, n, N_r, hist,
+                                                                                perm, inv_perm);
+  return launch_status();
+}
+
+// ---- gather / combine -------------------------------------------------------
+
+int mr_gather_rows(const void* x, int dtype, int T, int d, int k, const int32_t* perm,
+                   const int32_t* inv_perm, void* xs, mr_stream_t stream) {
+  if (T < 0 || d <= 0 || k <= 0 || (dtype != MR_F32 && dtype != MR_BF16)) return MR_ERR_INVALID_ARG;
+  if ((long long)T * k >= (1LL << 31)) return MR_ERR_INVALID_ARG;
+  if (k > mr::kRowMaxK) return MR_ERR_UNSUPPORTED;
+  if (T == 0) return MR_OK;
+  if (!x || !xs || (!perm && !inv_perm)) return MR_ERR_INVALID_ARG;
+  int sms = 0, cc = 0;
+  if (!device_info(&sms, &cc)) return MR_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const long esz = dtype == MR_BF16 ? 2 : 4;
+  const long row_bytes = (long)d * esz;
+  const bool vec = row_bytes % 16 == 0 && aligned16(x) && aligned16(xs);
+  const long rows = (long)T * k;
+  const unsigned grid_t = (unsigned)std::min<long>(T, (long)sms * 32);
+  const unsigned grid_r = (unsigned)std::min<long>(rows, (long)sms * 32);
+  if (inv_perm) {
+    if (vec)
+      mr::gather_inv_kernel<uint4><<<grid_t, mr::kRowThreads, 0, s>>>(
+          static_cast<const uint4*>(x), T, row_bytes / 16, k, inv_perm, static_cast<uint4*>(xs));
+    else if (esz == 4)
+      mr::gather_inv_kernel<uint32_t><<<grid_t, mr::kRowThreads, 0, s>>>(
+          static_cast<const uint32_t*>(x), T, d, k, inv_perm, static_cast<uint32_t*>(xs));
+    else
+      mr::gather_inv_kernel<uint16_t><<<grid_t, mr::kRowThreads, 0, s>>>(
+          static_cast<const uint16_t*>(x), T, d, k, inv_perm, static_cast<uint16_t*>(xs));
+  } else {
+    if (vec)
+      mr::gather_perm_kernel<uint4><<<grid_r, mr::kRowThreads, 0, s>>>(
+          static_cast<const uint4*>(x), rows, row_bytes / 16, k, perm, static_cast<uint4*>(xs));
+    else if (esz == 4)
+      mr::gather_perm_kernel<uint32_t><<<grid_r, mr::kRowThreads, 0, s>>>(
+          static_cast<const uint32_t*>(x), rows, d, k, perm, static_cast<uint32_t*>(xs));
+    else
+      mr::gather_perm_kernel<uint16_t><<<grid_r, mr::kRowThreads, 0, s>>>(
+          static_cast<const uint16_t*>(x), rows, d, k, perm, static_cast<uint16_t*>(xs));
+  }
+  return launch_status();
+}
+
+int mr_combine(const void* expert_out, int dtype, const float* w, const int32_t* inv_perm,
+               const void* shared, void* y, int T, int d, int k, mr_stream_t stream) {
+  if (T < 0 || d <= 0 || k <= 0 || (dtype != MR_F32 && dtype != MR_BF16)) return MR_ERR_INVALID_ARG;
+  if ((long long)T * k >= (1LL << 31)) return MR_ERR_INVALID_ARG;
+  if (k > mr::kRowMaxK) return MR_ERR_UNSUPPORTED;
+  if (T == 0) return MR_OK;
+  if (!expert_out || !w || !inv_perm || !y) return MR_ERR_INVALID_ARG;
+  int sms = 0, cc = 0;
+  if (!device_info(&sms, &cc)) return MR_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const long esz = dtype == MR_BF16 ? 2 : 4;
+  const long row_bytes = (long)d * esz;
+  const bool vec = row_bytes % 16 == 0 && aligned16(expert_out) && aligned16(y) &&
+                   (!shared || aligned16(shared));
+  const unsigned grid = (unsigned)std::min<long>(T, (long)sms * 32);
+  if (vec && dtype == MR_BF16)
+    mr::combine_bf16_vec_kernel<<<grid, mr::kRowThreads, 0, s>>>(
+        static_cast<const uint4*>(expert_out), w, inv_perm, static_cast<const uint4*>(shared),
+        static_cast<uint4*>(y), T, row_bytes / 16, k);
+  else if (vec)
+    mr::combine_f32_vec_kernel<<<grid, mr::kRowThreads, 0, s>>>(
+        static_cast<const float4*>(expert_out), w, inv_perm, static_cast<const float4*>(shared),
+        static_cast<float4*>(y), T, row_bytes / 16, k);
+  else if (dtype == MR_BF16)
+    mr::combine_scalar_kernel<true><<<grid, mr::kRowThreads, 0, s>>>(expert_out, w, inv_perm,
+                                                                     shared, y, T, d, k);
+  else
+    mr::combine_scalar_kernel<false><<<grid, mr::kRowThreads, 0, s>>>(expert_out, w, inv_perm,
+                                                                      shared, y, T, d, k);
+  return launch_status();
+}
+
+// ---- device error flag ----------------------------------------------------
+
+uint64_t mr_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+int mr_get_error(mr_stream_t stream) {
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return MR_ERR_CUDA;
+  unsigned int flag = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&flag, g_mr_error_flag, sizeof(flag)) != cudaSuccess) return MR_ERR_CUDA;
+  if (flag == 0) return MR_OK;
+  if (cudaMemcpyToSymbol(g_mr_error_flag, &zero, sizeof(zero)) != cudaSuccess) return MR_ERR_CUDA;
+  return (flag & MR_FLAG_TIMEOUT) ? MR_ERR_TIMEOUT : MR_ERR_DEVICE;
+}
+
+}  // extern "C"

@@ -1,0 +1,223 @@
+// rows.cuh -- the HBM-bound row movers of the path.
+//
+// gather  (Kimi K2 "Add shared output" page, moe_infer: sorted_tokens =
+//          x[idxs // k]).  With the inverse permutation each token row is read
+//          once and written to its k sorted positions (read d, write k*d);
+//          with only perm each sorted row fetches its token row.
+// combine (same page: new_x[idxs] = outs, weighted sum over k, cast back,
+//          plus the shared expert's output).  Each token gathers its k expert
+//          rows through the inverse permutation -- the scatter-back is fused
+//          into the read -- accumulates in fp32, rounds to the row dtype,
+//          adds the shared row and rounds again.
+//
+// Rows move in 16-byte vectors when the row size allows (8 bf16 / 4 fp32),
+// element by element otherwise.  One CTA handles one token at a time
+// (grid-stride), so every row access is a contiguous, coalesced stream.
+#pragma once
+
+#include "mr_common.cuh"
+
+namespace mr {
+
+constexpr int kRowThreads = 128;
+constexpr int kRowUnroll = 4;
+constexpr int kRowMaxK = 32;
+
+template <typename V>
+__device__ __forceinline__ V ld_stream(const V* p) {
+  return __ldg(p);
+}
+template <>
+__device__ __forceinline__ uint16_t ld_stream<uint16_t>(const uint16_t* p) {
+  return *p;
+}
+
+// ---- gather ----------------------------------------------------------------
+
+template <typename V>
+__global__ void __launch_bounds__(kRowThreads)
+    gather_inv_kernel(const V* __restrict__ x, long T, long nvec, int k,
+                      const int32_t* __restrict__ inv, V* __restrict__ xs) {
+  __shared__ long dst[kRowMaxK];
+  for (long t = blockIdx.x; t < T; t += gridDim.x) {
+    if (threadIdx.x < k) dst[threadIdx.x] = inv[t * k + threadIdx.x];
+    __syncthreads();
+    const V* src = x + t * nvec;
+    for (long v0 = threadIdx.x; v0 < nvec; v0 += kRowUnroll * kRowThreads) {
+      V val[kRowUnroll];
+#pragma unroll
+      for (int u = 0; u < kRowUnroll; ++u) {
+        const long v = v0 + (long)u * kRowThreads;
+        if (v < nvec) val[u] = ld_stream(src + v);
+      }
+      for (int j = 0; j < k; ++j) {
+        const long r = dst[j];
+        if (r < 0) continue;
+        V* out = xs + r * nvec;
+#pragma unroll
+        for (int u = 0; u < kRowUnroll; ++u) {
+          const long v = v0 + (long)u * kRowThreads;
+          if (v < nvec) out[v] = val[u];
+        }
+      }
+    }
+    __syncthreads();
+  }
+}
+
+template <typename V>
+__global__ void __launch_bounds__(kRowThreads)
+    gather_perm_kernel(const V* __restrict__ x, long rows, long nvec, int k,
+                       const int32_t* __restrict__ perm, V* __restrict__ xs) {
+  for (long i = blockIdx.x; i < rows; i += gridDim.x) {
+    const long p = perm[i];
+    if (p < 0) continue;
+    const V* src = x + (p / k) * nvec;
+    V* out = xs + i * nvec;
+    for (long v = threadIdx.x; v < nvec; v += kRowThreads) out[v] = ld_stream(src + v);
+  }
+}
+
+// ---- combine ---------------------------------------------------------------
+
+__device__ __forceinline__ void bf16x2_unpack(uint32_t u, float& lo, float& hi) {
+  lo = __uint_as_float(u << 16);
+  hi = __uint_as_float(u & 0xffff0000u);
+}
+
+__device__ __forceinline__ uint32_t bf16x2_pack_rn(float lo, float hi) {
+  __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&p);
+}
+
+__device__ __forceinline__ float bf16_round(float v) {
+  return __bfloat162float(__float2bfloat16_rn(v));
+}
+
+// bf16 rows, 8 elements (one uint4) per vector.
+__global__ void __launch_bounds__(kRowThreads)
+    combine_bf16_vec_kernel(const uint4* __restrict__ E, const float* __restrict__ w,
+                            const int32_t* __restrict__ inv, const uint4* __restrict__ shared,
+                            uint4* __restrict__ y, long T, long nvec, int k) {
+  __shared__ long row[kRowMaxK];
+  __shared__ float wt[kRowMaxK];
+  for (long t = blockIdx.x; t < T; t += gridDim.x) {
+    if (threadIdx.x < k) {
+      row[threadIdx.x] = inv[t * k + threadIdx.x];
+      wt[threadIdx.x] = w[t * k + threadIdx.x];
+    }
+    __syncthreads();
+    for (long v = threadIdx.x; v < nvec; v += kRowThreads) {
+      float acc[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) acc[q] = 0.0f;
+#pragma unroll 8
+      for (int j = 0; j < k; ++j) {
+        const long r = row[j];
+        if (r < 0) continue;
+        const uint4 e = __ldg(E + r * nvec + v);
+        const float wj = wt[j];
+        float lo, hi;
+        bf16x2_unpack(e.x, lo, hi); acc[0] = fmaf(wj, lo, acc[0]); acc[1] = fmaf(wj, hi, acc[1]);
+        bf16x2_unpack(e.y, lo, hi); acc[2] = fmaf(wj, lo, acc[2]); acc[3] = fmaf(wj, hi, acc[3]);
+        bf16x2_unpack(e.z, lo, hi); acc[4] = fmaf(wj, lo, acc[4]); acc[5] = fmaf(wj, hi, acc[5]);
+        bf16x2_unpack(e.w, lo, hi); acc[6] = fmaf(wj, lo, acc[6]); acc[7] = fmaf(wj, hi, acc[7]);
+      }
+      uint4 o;
+      if (shared) {
+        const uint4 sv = __ldg(shared + t * nvec + v);
+        const uint32_t s4[4] = {sv.x, sv.y, sv.z, sv.w};
+        uint32_t r4[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          float slo, shi;
+          bf16x2_unpack(s4[q], slo, shi);
+          r4[q] = bf16x2_pack_rn(bf16_round(acc[2 * q]) + slo, bf16_round(acc[2 * q + 1]) + shi);
+        }
+        o = make_uint4(r4[0], r4[1], r4[2], r4[3]);
+      } else {
+        o = make_uint4(bf16x2_pack_rn(acc[0], acc[1]), bf16x2_pack_rn(acc[2], acc[3]),
+                       bf16x2_pack_rn(acc[4], acc[5]), bf16x2_pack_rn(acc[6], acc[7]));
+      }
+      y[t * nvec + v] = o;
+    }
+    __syncthreads();
+  }
+}
+
+// fp32 rows, 4 elements (one float4) per vector.
+__global__ void __launch_bounds__(kRowThreads)
+    combine_f32_vec_kernel(const float4* __restrict__ E, const float* __restrict__ w,
+                           const int32_t* __restrict__ inv, const float4* __restrict__ shared,
+                           float4* __restrict__ y, long T, long nvec, int k) {
+  __shared__ long row[kRowMaxK];
+  __shared__ float wt[kRowMaxK];
+  for (long t = blockIdx.x; t < T; t += gridDim.x) {
+    if (threadIdx.x < k) {
+      row[threadIdx.x] = inv[t * k + threadIdx.x];
+      wt[threadIdx.x] = w[t * k + threadIdx.x];
+    }
+    __syncthreads();
+    for (long v = threadIdx.x; v < nvec; v += kRowThreads) {
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int j = 0; j < k; ++j) {
+        const long r = row[j];
+        if (r < 0) continue;
+        const float4 e = __ldg(E + r * nvec + v);
+        const float wj = wt[j];
+        acc.x = fmaf(wj, e.x, acc.x);
+        acc.y = fmaf(wj, e.y, acc.y);
+        acc.z = fmaf(wj, e.z, acc.z);
+        acc.w = fmaf(wj, e.w, acc.w);
+      }
+      if (shared) {
+        const float4 s = __ldg(shared + t * nvec + v);
+        acc.x += s.x;
+        acc.y += s.y;
+        acc.z += s.z;
+        acc.w += s.w;
+      }
+      y[t * nvec + v] = acc;
+    }
+    __syncthreads();
+  }
+}
+
+// Any row size, element by element.
+template <bool BF16>
+__global__ void __launch_bounds__(kRowThreads)
+    combine_scalar_kernel(const void* __restrict__ Ev, const float* __restrict__ w,
+                          const int32_t* __restrict__ inv, const void* __restrict__ sharedv,
+                          void* __restrict__ yv, long T, long d, int k) {
+  __shared__ long row[kRowMaxK];
+  __shared__ float wt[kRowMaxK];
+  for (long t = blockIdx.x; t < T; t += gridDim.x) {
+    if (threadIdx.x < k) {
+      row[threadIdx.x] = inv[t * k + threadIdx.x];
+      wt[threadIdx.x] = w[t * k + threadIdx.x];
+    }
+    __syncthreads();
+    for (long c = threadIdx.x; c < d; c += kRowThreads) {
+      float acc = 0.0f;
+      for (int j = 0; j < k; ++j) {
+        const long r = row[j];
+        if (r < 0) continue;
+        const float e = BF16 ? mr_bf16_to_f32(static_cast<const uint16_t*>(Ev)[r * d + c])
+                             : static_cast<const float*>(Ev)[r * d + c];
+        acc = fmaf(wt[j], e, acc);
+      }
+      if (BF16) {
+        float out = bf16_round(acc);
+        if (sharedv) out = out + mr_bf16_to_f32(static_cast<const uint16_t*>(sharedv)[t * d + c]);
+        __nv_bfloat16 b = __float2bfloat16_rn(out);
+        static_cast<uint16_t*>(yv)[t * d + c] = *reinterpret_cast<uint16_t*>(&b);
+      } else {
+        if (sharedv) acc += static_cast<const float*>(sharedv)[t * d + c];
+        static_cast<float*>(yv)[t * d + c] = acc;
+      }
+    }
+    __syncthreads();
+  }
+}
+
+}  // namespace mr
