@@ -105,7 +105,9 @@ const char *mr_status_string(int status);
  *   w_out    [T, k] fp32 weights (written).
  *
  * Limits: 1 <= N_r <= 512, n_group <= 32, d >= 1.  Uses 3xTF32 tensor-core
- * arithmetic when d % 4 == 0 and N_r % 16 == 0, CUDA-core FMA otherwise.
+ * arithmetic when d % 4 == 0 and N_r % 16 == 0 (N_r % 32 == 0 above 256),
+ * CUDA-core FMA otherwise.  The environment variable MR_TC_CLUSTER=1 or 2
+ * pins how many CTAs share a 128-token tile (testing only).
  * Needs no workspace.  Returns MR_OK or a negative status (nothing launched
  * on an argument error).
  */
@@ -116,8 +118,11 @@ int mr_router_forward(const float *x, const float *W, const float *bias, int T,
 
 /*
  * mr_router_workspace_size -- bytes of device workspace that
- * mr_router_forward_ex may use for T tokens (split-K partial logits of the
- * small-batch path).  0 means no workspace is needed at this size.
+ * mr_router_forward_ex may use for T tokens on the current device: for
+ * T <= 256 the split-K partial logits of the small-batch path, about
+ * (number of SMs / ceil(N_r/128)) * T * N_r * 4 bytes; above that the
+ * tf32 residuals of W (N_r * d * 4 bytes), computed once per call so the
+ * fused kernel's CTAs do not each re-derive them.
  */
 size_t mr_router_workspace_size(int T, int d, int N_r);
 
@@ -130,10 +135,16 @@ size_t mr_router_workspace_size(int T, int d, int N_r);
  *   precision   MR_PREC_3XTF32, MR_PREC_TF32 or MR_PREC_FFMA.
  *   logits_out  [T, N_r] fp32 logits, or NULL (debug / verification only).
  *   workspace   device buffer of workspace_bytes, or NULL.  With at least
- *               mr_router_workspace_size(T, d, N_r) bytes, small batches use
- *               the split-K path that spreads the weight read over all SMs.
+ *               mr_router_workspace_size(T, d, N_r) bytes, batches of up to
+ *               256 tokens on the tensor-core precisions use the split-K path
+ *               (two launches: a K-sliced GEMM over all SMs writing partial
+ *               logits, then a reduce-and-route kernel); the result is the
+ *               same arithmetic, summed in a fixed order (deterministic).
+ *               Larger batches use it for W's tf32 residuals (one extra
+ *               launch); results are identical with or without it.
  * Returns MR_ERR_UNSUPPORTED when the requested precision cannot run this
- * shape (tensor-core paths need d % 4 == 0 and N_r % 16 == 0).
+ * shape (tensor-core paths need d % 4 == 0 and N_r % 16 == 0, or
+ * N_r % 32 == 0 when N_r > 256).
  */
 int mr_router_forward_ex(const void *x, int x_dtype, const float *W,
                          const float *bias, int T, int d, int N_r, int n_group,

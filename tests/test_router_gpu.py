@@ -73,6 +73,16 @@ def test_router_plain_tf32_logits(w):
     print(w.name, "tf32 logit max err", err.max())
 
 
+@pytest.mark.parametrize("cs", ["1", "2"])
+@pytest.mark.parametrize("w", [SMALL[1], SMALL[3], SMALL[4]], ids=lambda w: w.name)
+def test_router_cluster_size_pinned(w, cs, monkeypatch):
+    """Both tile shapes of the tensor-core kernel (one CTA with all experts,
+    or two CTAs splitting them) on the same inputs."""
+    monkeypatch.setenv("MR_TC_CLUSTER", cs)
+    idx, wt, logits = _run(w, mr.MR_PREC_3XTF32)
+    compare_router(idx, wt, oracle_router(w, np.arange(w.T)), logits)
+
+
 def test_router_default_entry_point_matches_ex():
     w = SMALL[1]
     a = _run(w, mr.MR_PREC_3XTF32, want_logits=False)
@@ -132,3 +142,90 @@ def test_router_full_size_sampled(w):
         S = w.N_r // w.n_group
         assert max(len(set(r)) for r in (idx // S).tolist()) <= w.topk_group
     print(w.name, stats)
+
+
+SPLITK = [
+    W("splitk_T1", T=1, d=7168, N_r=256, n_group=8, topk_group=4, k=8, route_scale=2.5,
+      mask_mode=0, seed=21),
+    W("splitk_T7_N384", T=7, d=7168, N_r=384, n_group=1, topk_group=1, k=8,
+      route_scale=2.827, mask_mode=1, seed=22),
+    W("splitk_T200_d1000", T=200, d=1000, N_r=256, n_group=8, topk_group=4, k=8,
+      route_scale=2.5, mask_mode=0, seed=23),
+    W("splitk_T256_N64", T=256, d=516, N_r=64, n_group=4, topk_group=2, k=4, route_scale=2.5,
+      mask_mode=1, seed=24, io_dtype="f32"),
+    wl.V3_DECODE,
+]
+
+
+@pytest.mark.parametrize("w", SPLITK, ids=[w.name for w in SPLITK])
+def test_router_splitk_small_batches(w):
+    """Batches of up to 256 tokens with a workspace take the split-K path
+    (K-sliced tensor-core GEMM over all SMs + reduce-and-route)."""
+    n = mr.mr_router_workspace_size(w.T, w.d, w.N_r)
+    assert n > 0
+    d = router_inputs(w)
+    ws = torch.empty(n, dtype=torch.uint8, device="cuda")
+    logits = torch.empty((w.T, w.N_r), dtype=torch.float32, device="cuda")
+    l0 = mr.mr_launch_count()
+    idx, wt = mr.mr_router_forward_ex(to_dev(d["x_f32"]), to_dev(d["W"]), to_dev(d["b"]),
+                                      w.n_group, w.topk_group, w.k, w.route_scale, w.mask_mode,
+                                      logits_out=logits, workspace=ws)
+    assert mr.mr_launch_count() - l0 == 2  # GEMM + reduce/route
+    assert mr.mr_get_error() == mr.MR_OK
+    ref = oracle_router(w, np.arange(w.T))
+    stats = compare_router(idx.cpu().numpy(), wt.cpu().numpy(), ref, logits.cpu().numpy())
+    print(w.name, stats)
+    # deterministic: slices are summed in a fixed order
+    idx2, wt2 = mr.mr_router_forward_ex(to_dev(d["x_f32"]), to_dev(d["W"]), to_dev(d["b"]),
+                                        w.n_group, w.topk_group, w.k, w.route_scale,
+                                        w.mask_mode, workspace=ws)
+    assert torch.equal(idx, idx2) and torch.equal(wt, wt2)
+
+
+def test_router_workspace_for_large_batches_holds_w_residuals():
+    assert mr.mr_router_workspace_size(4096, 7168, 256) == 4 * 7168 * 256
+
+
+@pytest.mark.parametrize("w", [SMALL[1], SMALL[2].replace(name="k2_like_T300", T=300),
+                               wl.V3_PREFILL], ids=lambda w: w.name)
+def test_router_with_precomputed_residuals_is_identical(w):
+    """Above 256 tokens a workspace makes the fused path read W's tf32
+    residuals precomputed (one extra launch); results are bit-identical."""
+    assert w.T > 256  # (smaller batches take the split-K path instead)
+    d = router_inputs(w)
+    args = (to_dev(d["x_f32"]), to_dev(d["W"]), to_dev(d["b"]), w.n_group, w.topk_group, w.k,
+            w.route_scale, w.mask_mode)
+    ws = torch.empty(mr.mr_router_workspace_size(w.T, w.d, w.N_r), dtype=torch.uint8,
+                     device="cuda")
+    l0 = mr.mr_launch_count()
+    a = mr.mr_router_forward_ex(*args, workspace=ws)
+    assert mr.mr_launch_count() - l0 == 2
+    b = mr.mr_router_forward_ex(*args)
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+    assert mr.mr_get_error() == mr.MR_OK
+
+
+def test_tf32_operand_low_bits_probe():
+    """The tensor core reads an fp32 operand of kind::tf32 with its 13 low
+    mantissa bits ignored (truncation).  The 3xTF32 kernels rely on it: the
+    staged fp32 tile serves as the hi operand and only lo = v - trunc(v) is
+    materialised."""
+    d, N = 32, 16
+    x = torch.zeros((1, d), device="cuda")
+    x[0, 0] = 1.0
+    ulp = 2.0 ** -10
+    vals = np.array([1.0 + j * ulp / 8 + 2.0 ** -22 for j in range(N)], np.float32)
+    W = torch.zeros((N, d), device="cuda")
+    W[:, 0] = torch.from_numpy(vals).cuda()
+    logits = torch.empty((1, N), device="cuda")
+    mr.mr_router_forward_ex(x, W, None, 1, 1, 1, 1.0, 0, precision=mr.MR_PREC_TF32,
+                            logits_out=logits)
+    got = logits.cpu().numpy()[0].astype(np.float64)
+    u = vals.view(np.uint32)
+    trunc = (u & np.uint32(0xFFFFE000)).view(np.float32).astype(np.float64)
+    rn = np.array([np.round(v / ulp) * ulp for v in vals.astype(np.float64)])
+    kind = "truncate" if np.array_equal(got, trunc) else "round" if np.array_equal(got, rn) \
+        else "other"
+    print("tf32 operand low bits:", kind, got[:10])
+    # The 3xTF32 kernels stage raw fp32 tiles as the hi operand and rely on it.
+    assert kind == "truncate"

@@ -17,7 +17,7 @@ namespace mr {
 
 constexpr int kDispThreads = 256;
 constexpr int kDispWarps = kDispThreads / 32;
-constexpr int kDispChunk = 4096;                     // flat entries per CTA
+constexpr int kDispChunk = 1024;                     // flat entries per CTA
 constexpr int kDispSub = kDispChunk / kDispWarps;    // entries per warp
 constexpr int kDispMaxExperts = 1024;
 
@@ -53,22 +53,41 @@ __global__ void __launch_bounds__(kDispThreads)
   if (__any_sync(0xffffffffu, bad) && lane == 0) mr_raise(MR_FLAG_BAD_INDEX);
   __syncthreads();
   for (int e = threadIdx.x; e < N_r; e += kDispThreads)
-    chunk_hist[(long)blockIdx.x * N_r + e] = hist[e];
+    chunk_hist[(long)blockIdx.x * N_r + e] = hist[e];  // chunk-major [chunk][expert]
 }
 
-// One CTA of 1024 threads.  chunk_hist[c][e] is replaced by the position in
-// perm where chunk c's first entry of expert e goes.
+// One CTA of 1024 threads; chunk_hist is [nchunks][N_r].  Q = 1024 / N_r
+// (rounded down to a power of two) threads share an expert, each owning a
+// contiguous range of chunks, so all loads of a phase are independent and
+// coalesced across experts.  Produces counts and offsets (block scan over the
+// expert totals) and replaces chunk_hist[c][e] by the position in perm where
+// chunk c's first entry of expert e goes.
 __global__ void __launch_bounds__(1024)
     dispatch_scan_kernel(int32_t* __restrict__ chunk_hist, long nchunks, int N_r, long n,
                          int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
                          int32_t* __restrict__ perm) {
+  __shared__ int part[1024];  // [q][e] partial sums
+  __shared__ int start_e[kDispMaxExperts];
   __shared__ int warp_tot[32];
   __shared__ int total_s;
-  const int e = threadIdx.x, lane = e & 31, warp = e >> 5;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  int Q = 1;
+  while (Q * 2 * N_r <= 1024) Q *= 2;
+  const int e = tid % N_r, q = tid / N_r;
+  const bool active = q < Q;
+  const long span = (nchunks + Q - 1) / Q;
+  const long c_lo = active ? q * span : 0;
+  const long c_hi = active ? (c_lo + span < nchunks ? c_lo + span : nchunks) : 0;
+  // 1. partial sums over this thread's chunk range
+  int sum = 0;
+#pragma unroll 8
+  for (long c = c_lo; c < c_hi; ++c) sum += chunk_hist[c * N_r + e];
+  if (active) part[q * N_r + e] = sum;
+  __syncthreads();
+  // 2. expert totals and their exclusive scan (thread t = expert t)
   int cnt = 0;
-  if (e < N_r)
-    for (long c = 0; c < nchunks; ++c) cnt += chunk_hist[c * N_r + e];
-  // exclusive scan of cnt over e (block of 1024 = 32 warps)
+  if (tid < N_r)
+    for (int qq = 0; qq < Q; ++qq) cnt += part[qq * N_r + tid];
   int incl = cnt;
 #pragma unroll
   for (int off = 1; off < 32; off <<= 1) {
@@ -78,32 +97,39 @@ __global__ void __launch_bounds__(1024)
   if (lane == 31) warp_tot[warp] = incl;
   __syncthreads();
   if (warp == 0) {
-    int t = warp_tot[lane];
+    const int t = warp_tot[lane];
     int ti = t;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
       const int v = __shfl_up_sync(0xffffffffu, ti, off);
       if (lane >= off) ti += v;
     }
-    warp_tot[lane] = ti - t;  // exclusive prefix of warp totals
+    warp_tot[lane] = ti - t;
     if (lane == 31) total_s = ti;
   }
   __syncthreads();
-  const int excl = warp_tot[warp] + incl - cnt;
-  if (e < N_r) {
-    counts[e] = cnt;
-    offsets[e] = excl;
-    int run = excl;
-    for (long c = 0; c < nchunks; ++c) {
+  if (tid < N_r) {
+    const int excl = warp_tot[warp] + incl - cnt;
+    counts[tid] = cnt;
+    offsets[tid] = excl;
+    start_e[tid] = excl;
+  }
+  __syncthreads();
+  // 3. starting position of each chunk: expert start + earlier ranges + running sum
+  if (active) {
+    int run = start_e[e];
+    for (int qq = 0; qq < q; ++qq) run += part[qq * N_r + e];
+#pragma unroll 8
+    for (long c = c_lo; c < c_hi; ++c) {
       const int h = chunk_hist[c * N_r + e];
       chunk_hist[c * N_r + e] = run;
       run += h;
     }
   }
   const int total = total_s;
-  if (e == 0) offsets[N_r] = total;
+  if (tid == 0) offsets[N_r] = total;
   // slots of dropped (out-of-range) entries
-  for (long i = total + e; i < n; i += 1024) perm[i] = -1;
+  for (long i = total + tid; i < n; i += 1024) perm[i] = -1;
 }
 
 __global__ void __launch_bounds__(kDispThreads)

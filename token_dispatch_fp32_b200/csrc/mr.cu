@@ -6,12 +6,14 @@
 #include <cudaTypedefs.h>
 
 #include <atomic>
+#include <cstdlib>
 #include <cmath>
 #include <mutex>
 
 #include "dispatch.cuh"
 #include "mr_common.cuh"
 #include "router_ffma.cuh"
+#include "router_splitk.cuh"
 #include "router_tc.cuh"
 #include "rows.cuh"
 
@@ -103,9 +105,11 @@ int validate_router(const void* x, int x_dtype, const float* W, int T, int d, in
   return MR_OK;
 }
 
+// Tensor-core path: rows of 16-byte multiples for TMA, experts per CTA a
+// multiple of 16 (the MMA's N granularity for M = 128).
 bool tc_shape_ok(const void* x, int x_dtype, const float* W, int d, int N_r) {
-  return x_dtype == MR_F32 && d % 4 == 0 && N_r % 16 == 0 && N_r >= 16 && aligned16(x) &&
-         aligned16(W);
+  const bool n_ok = N_r <= 256 ? (N_r % 16 == 0 && N_r >= 16) : (N_r % 32 == 0);
+  return x_dtype == MR_F32 && d % 4 == 0 && n_ok && aligned16(x) && aligned16(W);
 }
 
 template <int NJ, bool XBF16>
@@ -142,31 +146,135 @@ int launch_ffma(const void* x, const float* W, const float* bias, int T, int d, 
   return MR_ERR_UNSUPPORTED;
 }
 
+// ---- small-batch (split-K) router ---------------------------------------
+
+constexpr int kSplitKMaxT = 256;  // batches up to one MMA N of tokens
+
+struct SplitKShape {
+  int NT, TT, MT, KC, KS;
+  size_t ws_bytes;
+};
+
+SplitKShape splitk_shape(int T, int d, int N_r, int sms) {
+  SplitKShape k;
+  k.NT = ((T + 15) / 16) * 16;
+  if (k.NT > mr::sk::kMaxNT) k.NT = mr::sk::kMaxNT;
+  k.TT = (T + k.NT - 1) / k.NT;
+  k.MT = (N_r + mr::tc::BM - 1) / mr::tc::BM;
+  k.KC = (d + mr::tc::BK - 1) / mr::tc::BK;
+  int ks = sms / (k.MT * k.TT);
+  if (ks < 1) ks = 1;
+  if (ks > k.KC) ks = k.KC;
+  k.KS = ks;
+  k.ws_bytes = (size_t)k.KS * (size_t)T * (size_t)N_r * sizeof(float);
+  return k;
+}
+
+bool splitk_applies(int T, int N_r) { return T > 0 && T <= kSplitKMaxT && N_r <= 512; }
+
+template <int NJ>
+int launch_reduce_nj(const float* part, int KS, int T, int N_r, const float* bias, int n_group,
+                     int topk_group, int k, float route_scale, int mask_mode, int32_t* idx_out,
+                     float* w_out, float* logits_out, cudaStream_t st) {
+  mr::sk::router_reduce_route_kernel<NJ><<<T, 256, 0, st>>>(part, KS, T, N_r, bias, n_group,
+                                                             topk_group, k, route_scale,
+                                                             mask_mode, idx_out, w_out,
+                                                             logits_out);
+  return launch_status();
+}
+
+int launch_splitk(const float* x, const float* W, const float* bias, int T, int d, int N_r,
+                  int n_group, int topk_group, int k, float route_scale, int mask_mode,
+                  bool use3x, int32_t* idx_out, float* w_out, float* logits_out, void* ws,
+                  int sms, cudaStream_t st) {
+  const SplitKShape sh = splitk_shape(T, d, N_r, sms);
+  const mr::sk::Plan plan = mr::sk::make_plan(sh.NT, (sh.KC + sh.KS - 1) / sh.KS);
+  CUtensorMap mw, mx;
+  if (!make_map_f32(&mw, W, (uint64_t)N_r, (uint64_t)d, mr::tc::BM, mr::tc::BK)) return MR_ERR_CUDA;
+  if (!make_map_f32(&mx, x, (uint64_t)T, (uint64_t)d, sh.NT, mr::tc::BK)) return MR_ERR_CUDA;
+  mr::sk::Params P;
+  P.T = T;
+  P.d = d;
+  P.N = N_r;
+  P.NT = sh.NT;
+  P.KS = sh.KS;
+  P.num_kc = sh.KC;
+  P.use3x = use3x ? 1 : 0;
+  P.part = static_cast<float*>(ws);
+  const size_t smem = plan.total + 1024;
+  if (cudaFuncSetAttribute(mr::sk::router_splitk_gemm_kernel,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return MR_ERR_CUDA;
+  mr::sk::router_splitk_gemm_kernel<<<dim3(sh.KS, sh.MT, sh.TT), mr::sk::kThreads, smem, st>>>(
+      mw, mx, P);
+  if (launch_status() != MR_OK) return MR_ERR_CUDA;
+  const int nj = (N_r + 31) / 32;
+#define MR_RED_CASE(NJV)                                                                      \
+  if (nj <= NJV)                                                                              \
+    return launch_reduce_nj<NJV>(P.part, sh.KS, T, N_r, bias, n_group, topk_group, k,          \
+                                 route_scale, mask_mode, idx_out, w_out, logits_out, st);
+  MR_RED_CASE(2)
+  MR_RED_CASE(4)
+  MR_RED_CASE(8)
+  MR_RED_CASE(12)
+  MR_RED_CASE(16)
+#undef MR_RED_CASE
+  return MR_ERR_UNSUPPORTED;
+}
+
+// Experts per CTA: all of them, or half per CTA of a 2-CTA cluster when
+// N_r > 256 (TMEM holds two accumulation buffers of at most 256 columns) or
+// when a split doubles the CTA count of a small batch.
+int tc_cluster_size(int T, int N_r, int sms) {
+  if (N_r > 256) return 2;
+  // MR_TC_CLUSTER=1|2 pins the choice (used by the tests to cover both).
+  if (const char* env = getenv("MR_TC_CLUSTER")) {
+    if (env[0] == '1') return 1;
+    if (env[0] == '2' && N_r % 32 == 0) return 2;
+  }
+  const int tiles = (T + mr::tc::BM - 1) / mr::tc::BM;
+  return (N_r % 32 == 0 && 2 * tiles <= sms) ? 2 : 1;
+}
+
+// W's residuals [N_r, d] fp32, precomputed into the workspace by the fused path.
+size_t wlo_bytes(int d, int N_r) { return (size_t)N_r * (size_t)d * sizeof(float); }
+
 int launch_tc(const float* x, const float* W, const float* bias, int T, int d, int N_r,
               int n_group, int topk_group, int k, float route_scale, int mask_mode, bool use3x,
-              int32_t* idx_out, float* w_out, float* logits_out, cudaStream_t st) {
-  const mr::tc::Plan plan = mr::tc::make_plan(N_r, 4);
-  if (plan.stages < 1) return MR_ERR_UNSUPPORTED;
-  const int n0 = N_r < 256 ? N_r : 256;
-  const int n1 = N_r - n0;
-  CUtensorMap mx, mw0, mw1;
-  if (!make_map_f32(&mx, x, (uint64_t)T, (uint64_t)d, mr::tc::BM, plan.BK)) return MR_ERR_CUDA;
-  if (!make_map_f32(&mw0, W, (uint64_t)N_r, (uint64_t)d, n0, plan.BK)) return MR_ERR_CUDA;
-  if (n1 > 0) {
-    if (!make_map_f32(&mw1, W, (uint64_t)N_r, (uint64_t)d, n1, plan.BK)) return MR_ERR_CUDA;
+              int32_t* idx_out, float* w_out, float* logits_out, float* wlo, int sms,
+              cudaStream_t st) {
+  const int CS = tc_cluster_size(T, N_r, sms);
+  const int NL = N_r / CS;
+  const mr::tc::Plan plan = mr::tc::make_plan(NL);
+  if (plan.stages < 2 || mr::tc::exchange_bytes(n_group) > plan.stages * plan.stage_bytes)
+    return MR_ERR_UNSUPPORTED;
+  CUtensorMap mx, mw, mwlo;
+  if (!make_map_f32(&mx, x, (uint64_t)T, (uint64_t)d, mr::tc::BM, mr::tc::BK)) return MR_ERR_CUDA;
+  if (!make_map_f32(&mw, W, (uint64_t)N_r, (uint64_t)d, NL, mr::tc::BK)) return MR_ERR_CUDA;
+  const bool use_wlo = use3x && wlo != nullptr;
+  if (use_wlo) {
+    const long n4 = (long)N_r * d / 4;
+    mr::tc::split_residual_kernel<<<(unsigned)std::min<long>((n4 + 255) / 256, (long)sms * 8), 256,
+                                    0, st>>>(reinterpret_cast<const float4*>(W),
+                                             reinterpret_cast<float4*>(wlo), n4);
+    if (launch_status() != MR_OK) return MR_ERR_CUDA;
+    if (!make_map_f32(&mwlo, wlo, (uint64_t)N_r, (uint64_t)d, NL, mr::tc::BK)) return MR_ERR_CUDA;
   } else {
-    mw1 = mw0;
+    mwlo = mw;
   }
   mr::tc::Params P;
   P.T = T;
   P.d = d;
   P.N = N_r;
+  P.NL = NL;
+  P.CS = CS;
   P.n_group = n_group;
   P.topk_group = topk_group;
   P.k = k;
   P.mask_mode = mask_mode;
-  P.num_kc = (d + plan.BK - 1) / plan.BK;
+  P.num_kc = (d + mr::tc::BK - 1) / mr::tc::BK;
   P.use3x = use3x ? 1 : 0;
+  P.wlo = use_wlo ? 1 : 0;
   P.route_scale = route_scale;
   P.bias = bias;
   P.idx_out = idx_out;
@@ -176,8 +284,29 @@ int launch_tc(const float* x, const float* W, const float* bias, int T, int d, i
   if (cudaFuncSetAttribute(mr::tc::router_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem) != cudaSuccess)
     return MR_ERR_CUDA;
-  const unsigned grid = (unsigned)((T + mr::tc::BM - 1) / mr::tc::BM);
-  mr::tc::router_tc_kernel<<<grid, mr::tc::kThreads, smem, st>>>(mx, mw0, mw1, P);
+  if (CS > 1 && cudaFuncSetAttribute(mr::tc::router_tc_kernel,
+                                     cudaFuncAttributeNonPortableClusterSizeAllowed, 0) !=
+                    cudaSuccess)
+    return MR_ERR_CUDA;
+  const unsigned tiles = (unsigned)((T + mr::tc::BM - 1) / mr::tc::BM);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(tiles * CS);
+  cfg.blockDim = dim3(mr::tc::kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = CS;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, mr::tc::router_tc_kernel, mx, mw, mwlo, P);
+  if (e != cudaSuccess) {
+    (void)cudaGetLastError();
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return MR_ERR_CUDA;
+  }
   return launch_status();
 }
 
@@ -200,10 +329,11 @@ const char* mr_status_string(int status) {
 }
 
 size_t mr_router_workspace_size(int T, int d, int N_r) {
-  (void)T;
-  (void)d;
-  (void)N_r;
-  return 0;
+  if (T <= 0 || d <= 0 || N_r <= 0 || N_r > 512) return 0;
+  if (!splitk_applies(T, N_r)) return wlo_bytes(d, N_r);
+  int sms = 0, cc = 0;
+  if (!device_info(&sms, &cc)) return 0;
+  return splitk_shape(T, d, N_r, sms).ws_bytes;
 }
 
 int mr_router_forward_ex(const void* x, int x_dtype, const float* W, const float* bias, int T,
@@ -211,8 +341,6 @@ int mr_router_forward_ex(const void* x, int x_dtype, const float* W, const float
                          int mask_mode, int precision, int32_t* idx_out, float* w_out,
                          float* logits_out, void* workspace, size_t workspace_bytes,
                          mr_stream_t stream) {
-  (void)workspace;
-  (void)workspace_bytes;
   int st = validate_router(x, x_dtype, W, T, d, N_r, n_group, topk_group, k, route_scale,
                            mask_mode, precision, idx_out, w_out);
   if (st != MR_OK || T == 0) return st;
@@ -227,9 +355,17 @@ int mr_router_forward_ex(const void* x, int x_dtype, const float* W, const float
                                     mask_mode, idx_out, w_out, logits_out, s);
   }
   if (cc != 10 || !tc_shape_ok(x, x_dtype, W, d, N_r)) return MR_ERR_UNSUPPORTED;
+  if (workspace && splitk_applies(T, N_r) &&
+      workspace_bytes >= splitk_shape(T, d, N_r, sms).ws_bytes)
+    return launch_splitk(static_cast<const float*>(x), W, bias, T, d, N_r, n_group, topk_group,
+                         k, route_scale, mask_mode, precision == MR_PREC_3XTF32, idx_out, w_out,
+                         logits_out, workspace, sms, s);
+  float* wlo = (workspace && aligned16(workspace) && workspace_bytes >= wlo_bytes(d, N_r))
+                   ? static_cast<float*>(workspace)
+                   : nullptr;
   return launch_tc(static_cast<const float*>(x), W, bias, T, d, N_r, n_group, topk_group, k,
                    route_scale, mask_mode, precision == MR_PREC_3XTF32, idx_out, w_out,
-                   logits_out, s);
+                   logits_out, wlo, sms, s);
 }
 
 int mr_router_forward(const float* x, const float* W, const float* bias, int T, int d, int N_r,

@@ -1,26 +1,44 @@
 // router_tc.cuh -- fused gate GEMM + routing on the 5th-generation tensor cores.
 //
-// One CTA owns a tile of 128 tokens and ALL N_r experts, so a token's logits
-// never leave the chip: the accumulator lives in tensor memory (TMEM lane =
-// token, column = expert) and the routing epilogue reads it back directly.
+// A cluster of CS CTAs (CS = 1, or 2 when the experts are split) owns a tile
+// of 128 tokens; CTA r of the cluster owns experts [r*NL, (r+1)*NL), NL <= 256.
+// A token's logits never go to HBM: they accumulate in tensor memory (TMEM
+// lane = token, column = expert) and the routing epilogue reads them back.
 //
-//   warp 0       TMA producer: x tile [128 x BK] and W tile [N_r x BK] per
-//                stage (fp32, hardware swizzle), completion on an mbarrier.
-//   warp 1       TMEM owner and MMA issuer (one thread): tcgen05.mma
-//                kind::tf32, M=128, N=N_r (two MMAs when N_r > 256).
-//   warps 2..5   3xTF32 split while the main loop runs: each staged fp32 value
-//                v becomes hi = v with the low 13 mantissa bits cleared (exact
-//                in tf32) and lo = v - hi (exact in fp32), so
-//                x.w ~= hi.hi + hi.lo + lo.hi with fp32 accumulation.
-//                Afterwards the same warps are the epilogue: warp w reads TMEM
-//                lanes 32*(w%4).. with tcgen05.ld and routes its token in
-//                registers (sigmoid, bias, group top-2, group top-k, top-8
-//                insertion with lower-index tie-break, renormalise, scale).
+//   warp 0      TMA producer: x tile [128 x 32] and W tile [NL x 32] fp32 per
+//               stage (128-byte hardware swizzle), completion on an mbarrier.
+//   warp 1      TMEM owner and MMA issuer (one elected thread):
+//               tcgen05.mma.cta_group::1.kind::tf32, M = 128, N = NL.
+//   warps 2..9  "workers":
+//               (a) 3xTF32 split of every staged fp32 value v into
+//                   hi = v with the low 13 mantissa bits cleared (exact in
+//                   tf32) and lo = v - hi (exact in fp32); the MMA issues
+//                   hi*hi + hi*lo + lo*hi into one fp32 accumulator.  The
+//                   tensor core ignores those 13 bits of a tf32 operand, so
+//                   the staged tile serves as hi unchanged and only lo is
+//                   written; W's residuals may instead come precomputed (TMA);
+//                   lo(x)*hi(W) is skipped when a stage's x residuals are all
+//                   zero (tf32-exact activations, e.g. bf16 hidden states);
+//               (b) promotion: the tensor core adds each product into its
+//                   fp32 accumulator rounding toward zero, so one accumulator
+//                   over all d would drift by ~1 ulp per MMA.  The K loop is
+//                   cut into intervals of kPromote chunks that alternate
+//                   between two TMEM buffers; each finished interval is added
+//                   into fp32 registers (round to nearest) while the tensor
+//                   core fills the other buffer.  Interval errors change sign
+//                   from interval to interval and no longer accumulate.
+//               (c) epilogue: the register sums go back to TMEM, then warp w
+//                   (w = 2..5) routes the 32 tokens of TMEM lanes 32*(w%4)..:
+//                   sigmoid, bias, per-group top-2, group top-k, a top-8
+//                   insertion list with lower-index tie-break, renormalise and
+//                   scale.  With CS = 2 the two CTAs exchange per-group top-2
+//                   pairs and top-8 lists through distributed shared memory.
 //
 // Arithmetic follows the pages (Kimi K2 "Normalize weights" page,
 // MoEGate.forward; DeepSeek-V3.2-Exp "Normalize weights" page, Gate.forward).
 // Every mbarrier wait is bounded (MR_WAIT_LIMIT_NS); on expiry the CTA raises
-// MR_FLAG_TIMEOUT, stops issuing work, drains its MMAs and frees its TMEM.
+// MR_FLAG_TIMEOUT, stops issuing work, drains its own copies and MMAs, still
+// takes part in every cluster barrier, and frees its TMEM.
 #pragma once
 
 #include <cuda.h>
@@ -31,14 +49,19 @@ namespace mr {
 namespace tc {
 
 constexpr int BM = 128;
-constexpr int kThreads = 192;
-constexpr int kMaxN = 512;
+constexpr int BK = 32;                        // fp32 along K per stage (128-byte rows)
+constexpr int kWorkers = 8;                   // worker warps 2..9
+constexpr int kThreads = 64 + 32 * kWorkers;  // 320
+constexpr int kPromote = 128 / BK;            // K chunks per accumulation interval (128 K)
+constexpr int kMaxNL = 256;
 constexpr int kMaxGroups = 32;
 constexpr int kTopMax = 8;
-constexpr size_t kSmemBudget = 232448;  // 227 KB opt-in per CTA
+constexpr int kMaxStages = 6;
+constexpr uint32_t kSmemBudget = 232448;      // 227 KB opt-in per CTA
 
 struct Params {
-  int T, d, N, n_group, topk_group, k, mask_mode, num_kc, use3x;
+  int T, d, N, NL, CS, n_group, topk_group, k, mask_mode, num_kc, use3x;
+  int wlo;  // W residuals W - trunc_tf32(W) arrive by TMA (map_wlo) instead of being split here
   float route_scale;
   const float* bias;
   int32_t* idx_out;
@@ -48,31 +71,32 @@ struct Params {
 
 // Shared-memory plan, identical on host and device.
 struct Plan {
-  int BK, stages;
+  int stages;
   uint32_t a_bytes, b_bytes, hi_bytes, stage_bytes;
-  uint32_t bar_off, misc_off, bias_off, gs_off, total;
+  uint32_t bar_off, misc_off, bias_off, total;
 };
 
 __host__ __device__ inline uint32_t align_up(uint32_t v, uint32_t a) { return (v + a - 1) / a * a; }
 
-__host__ __device__ inline Plan make_plan(int N, int stages_cap) {
+__host__ __device__ inline Plan make_plan(int NL) {
   Plan p;
-  p.BK = (N <= 256) ? 32 : 16;
-  p.a_bytes = BM * p.BK * 4;
-  p.b_bytes = N * p.BK * 4;
-  p.hi_bytes = p.a_bytes + p.b_bytes;          // [A | B] of one kind (hi or lo)
+  p.a_bytes = BM * BK * 4;
+  p.b_bytes = NL * BK * 4;
+  p.hi_bytes = p.a_bytes + p.b_bytes;  // [A | B] of one kind (hi or lo)
   p.stage_bytes = align_up(2 * p.hi_bytes, 1024);
-  const uint32_t extras = 1024 /*align slack*/ + 256 /*barriers*/ + 64 + 4 * kMaxN +
-                          4 * kMaxGroups * BM;
+  const uint32_t extras = 1024 /*align slack*/ + 512 /*barriers*/ + 256 + 4 * 2 * kMaxNL;
   int s = (int)((kSmemBudget - extras) / p.stage_bytes);
-  if (s > stages_cap) s = stages_cap;
-  p.stages = s;
+  p.stages = s > kMaxStages ? kMaxStages : s;
   p.bar_off = p.stages * p.stage_bytes;
-  p.misc_off = p.bar_off + 256;
-  p.bias_off = p.misc_off + 64;
-  p.gs_off = p.bias_off + 4 * kMaxN;
-  p.total = p.gs_off + 4 * kMaxGroups * BM;
+  p.misc_off = p.bar_off + 512;
+  p.bias_off = p.misc_off + 256;
+  p.total = p.bias_off + 4 * 2 * kMaxNL;
   return p;
+}
+
+// Bytes of epilogue exchange space (aliases the stage ring after the K loop).
+__host__ __device__ inline uint32_t exchange_bytes(int G) {
+  return 4u * (2u * G * BM + 3u * kTopMax * BM);
 }
 
 // ---- PTX wrappers ----------------------------------------------------------
@@ -144,20 +168,44 @@ __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
-// UMMA shared-memory descriptor, K-major operand, swizzled rows of BK fp32.
-__device__ __forceinline__ uint64_t make_desc(uint32_t saddr, int BK) {
-  const uint64_t sbo = (BK == 32) ? 1024u : 512u;      // 8 rows x row bytes
-  const uint64_t layout = (BK == 32) ? 2u : 4u;        // SWIZZLE_128B / SWIZZLE_64B
+__device__ __forceinline__ void workers_sync() {
+  asm volatile("bar.sync 1, %0;" ::"r"(32 * kWorkers) : "memory");
+}
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// Whole-cluster barrier; every thread of every CTA in the cluster calls it
+// the same number of times, with its warp converged (.aligned).
+__device__ __forceinline__ void cluster_sync_all() {
+  __syncwarp();
+  asm volatile("barrier.cluster.arrive.aligned;\n\tbarrier.cluster.wait.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ float ld_peer_f32(const float* local, uint32_t peer) {
+  uint32_t ra, v;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(smem_u32(local)), "r"(peer));
+  asm volatile("ld.shared::cluster.b32 %0, [%1];" : "=r"(v) : "r"(ra) : "memory");
+  return __uint_as_float(v);
+}
+
+// UMMA shared-memory descriptor: K-major operand, rows of BK fp32 (128 bytes),
+// 128-byte swizzle, 8-row groups 8 * 128 bytes apart.
+__device__ __forceinline__ uint64_t make_desc(uint32_t saddr) {
+  static_assert(BK == 32, "descriptor written for 128-byte rows");
   uint64_t d = 0;
   d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
-  d |= (uint64_t)1u << 16;                              // LBO (unused when swizzled)
-  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
-  d |= (uint64_t)1u << 46;                              // descriptor version (sm_100)
-  d |= layout << 61;
+  d |= (uint64_t)1u << 16;                      // LBO (unused when swizzled)
+  d |= (uint64_t)(1024u >> 4) << 32;            // SBO
+  d |= (uint64_t)1u << 46;                      // descriptor version (sm_100)
+  d |= (uint64_t)2u << 61;                      // SWIZZLE_128B
   return d;
 }
 
-// Instruction descriptor: D fp32, A/B tf32, both K-major, M=128, N=n.
+// Instruction descriptor: D fp32, A/B tf32, both K-major, M = 128, N = n.
 __device__ __forceinline__ uint32_t make_idesc(int n) {
   return (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(n >> 3) << 17) |
          ((uint32_t)(BM >> 4) << 24);
@@ -179,22 +227,31 @@ __device__ __forceinline__ void mma_commit(uint32_t bar) {
       : "memory");
 }
 
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
-  uint32_t r[32];
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
   asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
       : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
         "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
-        "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
-        "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
-        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
-        "=r"(r[31])
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
       : "r"(taddr));
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
-  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+      "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+      "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+      "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+      "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+      "r"(__float_as_uint(v[15]))
+      : "memory");
 }
 
 // Keep the best 8 (value desc, index asc).  Candidates arrive in increasing
@@ -228,40 +285,46 @@ struct Top8 {
 
 __global__ void __launch_bounds__(kThreads, 1)
     router_tc_kernel(const __grid_constant__ CUtensorMap map_x,
-                     const __grid_constant__ CUtensorMap map_w0,
-                     const __grid_constant__ CUtensorMap map_w1, const Params P) {
+                     const __grid_constant__ CUtensorMap map_w,
+                     const __grid_constant__ CUtensorMap map_wlo, const Params P) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const Plan plan = make_plan(P.N, 4);
-  const int BK = plan.BK, STAGES = plan.stages;
+  const int NL = P.NL;
+  const Plan plan = make_plan(NL);
+  const int STAGES = plan.stages;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t crank = P.CS > 1 ? cluster_rank() : 0u;
+  const int tile = blockIdx.x / P.CS;
+  const int col0 = (int)crank * NL;  // first global expert of this CTA
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + plan.bar_off);
-  // bars[0..S) full, [S..2S) converted, [2S..3S) empty, [3S] accumulator ready
+  // [0,S) full  [S,2S) converted  [2S,3S) empty  3S+{0,1} acc full
+  // 3S+{2,3} acc free  3S+4 MMA drained
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + plan.misc_off);
   volatile int* abort = reinterpret_cast<volatile int*>(smem + plan.misc_off + 8);
+  // xnz[s][w]: worker warp w saw a nonzero x residual in stage s this round
+  volatile uint32_t* xnz = reinterpret_cast<volatile uint32_t*>(smem + plan.misc_off + 32);
   float* bias_s = reinterpret_cast<float*>(smem + plan.bias_off);
-  float* gs_s = reinterpret_cast<float*>(smem + plan.gs_off);
 
   const uint32_t smem0 = smem_u32(smem);
-  auto bar_full = [&](int s) { return smem_u32(&bars[s]); };
-  auto bar_conv = [&](int s) { return smem_u32(&bars[STAGES + s]); };
-  auto bar_empty = [&](int s) { return smem_u32(&bars[2 * STAGES + s]); };
-  const uint32_t bar_acc = smem_u32(&bars[3 * STAGES]);
-
-  const int N = P.N;
-  const int n0 = N < 256 ? N : 256;
-  const int n1 = N - n0;
-  const uint32_t tmem_cols = N <= 32 ? 32 : N <= 64 ? 64 : N <= 128 ? 128 : N <= 256 ? 256 : 512;
+  auto bar = [&](int i) { return smem_u32(&bars[i]); };
+  const int B_FULL = 0, B_CONV = STAGES, B_EMPTY = 2 * STAGES, B_ACCF = 3 * STAGES,
+            B_ACCE = 3 * STAGES + 2, B_DRAIN = 3 * STAGES + 4;
+  const uint32_t tmem_cols = 2 * NL <= 32 ? 32 : 2 * NL <= 64 ? 64 : 2 * NL <= 128 ? 128
+                           : 2 * NL <= 256 ? 256 : 512;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(bar_full(s), 1);
-      mbar_init(bar_conv(s), 128);
-      mbar_init(bar_empty(s), 1);
+      mbar_init(bar(B_FULL + s), 1);
+      mbar_init(bar(B_CONV + s), 32 * kWorkers);
+      mbar_init(bar(B_EMPTY + s), 1);
     }
-    mbar_init(bar_acc, 1);
+    mbar_init(bar(B_ACCF + 0), 1);
+    mbar_init(bar(B_ACCF + 1), 1);
+    mbar_init(bar(B_ACCE + 0), 32 * kWorkers);
+    mbar_init(bar(B_ACCE + 1), 32 * kWorkers);
+    mbar_init(bar(B_DRAIN), 1);
     *abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -272,186 +335,330 @@ __global__ void __launch_bounds__(kThreads, 1)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
-  for (int e = threadIdx.x; e < N; e += kThreads) bias_s[e] = P.bias ? P.bias[e] : 0.0f;
+  for (int e = threadIdx.x; e < NL; e += kThreads)
+    bias_s[e] = P.bias ? P.bias[col0 + e] : 0.0f;
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  const int m0 = blockIdx.x * BM;
+  const int m0 = tile * BM;
   const int KC = P.num_kc;
+  const int J = (KC + kPromote - 1) / kPromote;  // accumulation intervals
 
   if (warp == 0) {
     // ---------------- TMA producer ----------------
     if (lane == 0) {
-      const uint32_t tx = (uint32_t)(BM + N) * BK * 4;
+      const uint32_t tx = (uint32_t)(BM + (P.wlo ? 2 : 1) * NL) * BK * 4;
       int issued = 0;
       for (int kc = 0; kc < KC; ++kc) {
         const int s = kc % STAGES;
-        if (kc >= STAGES && !mbar_wait(bar_empty(s), ((kc / STAGES) - 1) & 1, abort)) break;
+        if (kc >= STAGES && !mbar_wait(bar(B_EMPTY + s), ((kc / STAGES) - 1) & 1, abort)) break;
         ++issued;
         const uint32_t base = smem0 + s * plan.stage_bytes;
-        mbar_arrive_expect_tx(bar_full(s), tx);
-        tma_load_2d(base, &map_x, bar_full(s), kc * BK, m0);
-        tma_load_2d(base + plan.a_bytes, &map_w0, bar_full(s), kc * BK, 0);
-        if (n1 > 0)
-          tma_load_2d(base + plan.a_bytes + (uint32_t)n0 * BK * 4, &map_w1, bar_full(s), kc * BK,
-                      n0);
+        mbar_arrive_expect_tx(bar(B_FULL + s), tx);
+        tma_load_2d(base, &map_x, bar(B_FULL + s), kc * BK, m0);
+        tma_load_2d(base + plan.a_bytes, &map_w, bar(B_FULL + s), kc * BK, col0);
+        if (P.wlo)
+          tma_load_2d(base + plan.hi_bytes + plan.a_bytes, &map_wlo, bar(B_FULL + s), kc * BK,
+                      col0);
       }
-      // Before the CTA may exit, every copy it issued must have landed (on the
+      // Every copy this CTA issued must land before the CTA may exit (on the
       // normal path these waits succeed at once).
       for (int kc = issued - STAGES < 0 ? 0 : issued - STAGES; kc < issued; ++kc)
-        mbar_wait(bar_full(kc % STAGES), (kc / STAGES) & 1, abort, true);
+        mbar_wait(bar(B_FULL + kc % STAGES), (kc / STAGES) & 1, abort, true);
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
-      const uint32_t id0 = make_idesc(n0);
-      const uint32_t id1 = n1 > 0 ? make_idesc(n1) : 0u;
-      const uint32_t b1_off = (uint32_t)n0 * BK * 4;
+      const uint32_t idesc = make_idesc(NL);
       for (int kc = 0; kc < KC; ++kc) {
         const int s = kc % STAGES;
-        const uint32_t ph = (kc / STAGES) & 1;
-        if (!mbar_wait(P.use3x ? bar_conv(s) : bar_full(s), ph, abort)) break;
+        const int j = kc / kPromote, b = j & 1;
+        const bool first = (kc % kPromote) == 0;
+        if (first && j >= 2 && !mbar_wait(bar(B_ACCE + b), ((j >> 1) - 1) & 1, abort)) break;
+        if (!mbar_wait(P.use3x ? bar(B_CONV + s) : bar(B_FULL + s), (kc / STAGES) & 1, abort))
+          break;
         tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(b * NL);
         const uint32_t a_hi = smem0 + s * plan.stage_bytes;
         const uint32_t b_hi = a_hi + plan.a_bytes;
         const uint32_t a_lo = a_hi + plan.hi_bytes;
         const uint32_t b_lo = b_hi + plan.hi_bytes;
+        // lo(x) * hi(W) adds exact zeros when every x residual of the stage
+        // is 0 (x already tf32-exact, e.g. bf16 activations): skip it.
+        bool x_lo = false;
+        if (P.use3x)
+#pragma unroll
+          for (int w = 0; w < kWorkers; ++w) x_lo |= xnz[s * kWorkers + w] != 0u;
+#pragma unroll
         for (int kk = 0; kk < BK / 8; ++kk) {
           const uint32_t ko = kk * 32;  // 8 tf32 = 32 bytes along K
-          const uint32_t acc0 = (kc > 0 || kk > 0) ? 1u : 0u;
-          const uint64_t dah = make_desc(a_hi + ko, BK), dbh = make_desc(b_hi + ko, BK);
-          mma_tf32(tmem_base, dah, dbh, id0, acc0);
-          if (n1 > 0) mma_tf32(tmem_base + n0, dah, make_desc(b_hi + b1_off + ko, BK), id1, acc0);
+          const uint32_t acc0 = (!first || kk > 0) ? 1u : 0u;
+          const uint64_t dah = make_desc(a_hi + ko), dbh = make_desc(b_hi + ko);
+          mma_tf32(d_tmem, dah, dbh, idesc, acc0);
           if (P.use3x) {
-            const uint64_t dal = make_desc(a_lo + ko, BK), dbl = make_desc(b_lo + ko, BK);
-            mma_tf32(tmem_base, dah, dbl, id0, 1u);
-            mma_tf32(tmem_base, dal, dbh, id0, 1u);
-            if (n1 > 0) {
-              mma_tf32(tmem_base + n0, dah, make_desc(b_lo + b1_off + ko, BK), id1, 1u);
-              mma_tf32(tmem_base + n0, dal, make_desc(b_hi + b1_off + ko, BK), id1, 1u);
+            mma_tf32(d_tmem, dah, make_desc(b_lo + ko), idesc, 1u);
+            if (x_lo) mma_tf32(d_tmem, make_desc(a_lo + ko), dbh, idesc, 1u);
+          }
+        }
+        mma_commit(bar(B_EMPTY + s));
+        if ((kc % kPromote) == kPromote - 1 || kc == KC - 1) mma_commit(bar(B_ACCF + b));
+      }
+      // Track every MMA issued so far; waited on before TMEM is released.
+      mma_commit(bar(B_DRAIN));
+      mbar_wait(bar(B_DRAIN), 0, abort, true);
+    }
+  } else {
+    // ---------------- workers: split, promotion ----------------
+    const int wt = threadIdx.x - 64;  // 0..255
+    const int q = warp & 3;           // TMEM lane quarter
+    const int h = (warp - 2) >> 2;    // column half
+    const int n16 = NL / 16;
+    const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+    float acc[8][16];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+      for (int c = 0; c < 16; ++c) acc[i][c] = 0.0f;
+    int promoted = 0;
+    bool ok = true;
+
+    auto promote = [&](int j) {
+      const int b = j & 1;
+      if (!mbar_wait(bar(B_ACCF + b), (j >> 1) & 1, abort)) {
+        ok = false;
+        return;
+      }
+      tc_fence_after();
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int c = h + 2 * i;
+        if (c < n16) {
+          float v[16];
+          tmem_ld16(tmem_base + lane_off + (uint32_t)(b * NL + c * 16), v);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) acc[i][e] += v[e];
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar(B_ACCE + b));
+      ++promoted;
+    };
+
+    const int n4a = (int)(plan.a_bytes / 16);  // the x part of [A | B]
+    const int n4 = P.wlo ? n4a : (int)(plan.hi_bytes / 16);
+    for (int kc = 0; kc < KC && ok; ++kc) {
+      if (P.use3x) {
+        const int s = kc % STAGES;
+        if (!mbar_wait(bar(B_FULL + s), (kc / STAGES) & 1, abort)) {
+          ok = false;
+          break;
+        }
+        // The tensor core reads a kind::tf32 operand with its 13 low mantissa
+        // bits ignored (truncation), so the staged fp32 tile already is the
+        // hi part; only the residual lo = v - trunc(v) is written.
+        const float4* hi = reinterpret_cast<const float4*>(smem + s * plan.stage_bytes);
+        float4* lo = reinterpret_cast<float4*>(smem + s * plan.stage_bytes + plan.hi_bytes);
+        uint32_t nz = 0;
+        for (int i = wt; i < n4; i += 32 * kWorkers) {
+          const float4 v = hi[i];
+          float4 l;
+          l.x = v.x - __uint_as_float(__float_as_uint(v.x) & 0xFFFFE000u);
+          l.y = v.y - __uint_as_float(__float_as_uint(v.y) & 0xFFFFE000u);
+          l.z = v.z - __uint_as_float(__float_as_uint(v.z) & 0xFFFFE000u);
+          l.w = v.w - __uint_as_float(__float_as_uint(v.w) & 0xFFFFE000u);
+          lo[i] = l;
+          if (i < n4a)
+            nz |= __float_as_uint(l.x) | __float_as_uint(l.y) | __float_as_uint(l.z) |
+                  __float_as_uint(l.w);
+        }
+        const bool any_nz = __any_sync(0xffffffffu, (nz << 1) != 0u);  // ignore -0.0
+        if (lane == 0) xnz[s * kWorkers + (warp - 2)] = any_nz ? 1u : 0u;
+        fence_proxy_async();
+        mbar_arrive(bar(B_CONV + s));
+      }
+      // promote the interval before the one the tensor core is working on
+      if ((kc % kPromote) == kPromote - 1 && kc / kPromote >= 1) promote(kc / kPromote - 1);
+    }
+    while (ok && promoted < J) promote(promoted);
+    ok = __all_sync(0xffffffffu, ok);
+
+    // final sums back to TMEM buffer 0 for the routing epilogue
+    if (ok) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int c = h + 2 * i;
+        if (c < n16) tmem_st16(tmem_base + lane_off + (uint32_t)(c * 16), acc[i]);
+      }
+      asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    workers_sync();
+    tc_fence_after();
+    if (*abort) ok = false;
+    ok = __all_sync(0xffffffffu, ok);
+
+    // ---------------- routing epilogue ----------------
+    if (warp < 6) {
+      const int row = q * 32 + lane;
+      const long tok = (long)m0 + row;
+      const int G = P.n_group, S = P.N / G;
+      const int cs = P.CS;
+      // exchange space aliases the (now idle) stage ring
+      float* exA1 = reinterpret_cast<float*>(smem);             // [G][BM]
+      float* exA2 = exA1 + G * BM;                               // [G][BM]
+      float* exV = exA2 + G * BM;                                // [8][BM]
+      float* exS = exV + kTopMax * BM;                           // [8][BM]
+      int* exI = reinterpret_cast<int*>(exS + kTopMax * BM);     // [8][BM]
+      float v[16];
+
+      if (ok && P.logits_out) {
+        for (int c = 0; c < n16; ++c) {
+          tmem_ld16(tmem_base + lane_off + (uint32_t)(c * 16), v);  // whole warp
+          if (tok < P.T)
+#pragma unroll
+            for (int e = 0; e < 16; ++e) P.logits_out[tok * P.N + col0 + c * 16 + e] = v[e];
+        }
+      }
+
+      // pass 1: per-group top-2 of the biased scores over this CTA's experts
+      uint32_t kept = 0xffffffffu;
+      if (G > 1) {
+        for (int g = 0; g < G; ++g) {
+          exA1[g * BM + row] = -INFINITY;
+          exA2[g * BM + row] = -INFINITY;
+        }
+        if (ok) {
+          float a1 = -INFINITY, a2 = -INFINITY;
+          int g = col0 / S, next_b = (g + 1) * S;
+          for (int c = 0; c < n16; ++c) {
+            tmem_ld16(tmem_base + lane_off + (uint32_t)(c * 16), v);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const int e = col0 + c * 16 + i;
+              if (e == next_b) {
+                exA1[g * BM + row] = a1;
+                exA2[g * BM + row] = a2;
+                ++g;
+                next_b += S;
+                a1 = -INFINITY;
+                a2 = -INFINITY;
+              }
+              const float cval = mr_sigmoid(v[i]) + bias_s[e - col0];
+              if (cval > a1) {
+                a2 = a1;
+                a1 = cval;
+              } else if (cval > a2) {
+                a2 = cval;
+              }
+            }
+          }
+          exA1[g * BM + row] = a1;
+          exA2[g * BM + row] = a2;
+        }
+      }
+      if (cs > 1) {
+        cluster_sync_all();  // #1: group pairs visible to the peer
+      }
+      if (G > 1) {
+        float gs[kMaxGroups];
+#pragma unroll
+        for (int g = 0; g < kMaxGroups; ++g) {
+          if (g < G) {
+            float a1 = exA1[g * BM + row], a2 = exA2[g * BM + row];
+            if (cs > 1) {
+              const float b1 = ld_peer_f32(&exA1[g * BM + row], crank ^ 1u);
+              const float b2 = ld_peer_f32(&exA2[g * BM + row], crank ^ 1u);
+              if (a1 >= b1) {
+                a2 = fmaxf(a2, b1);
+              } else {
+                a2 = fmaxf(a1, b2);
+                a1 = b1;
+              }
+            }
+            gs[g] = a1 + a2;
+          }
+        }
+        kept = 0;
+        for (int r = 0; r < P.topk_group; ++r) {
+          float bv = -INFINITY;
+          int bg = -1;
+#pragma unroll
+          for (int g = 0; g < kMaxGroups; ++g) {
+            if (g < G && !((kept >> g) & 1u) && (bg < 0 || gs[g] > bv)) {
+              bv = gs[g];
+              bg = g;
+            }
+          }
+          kept |= 1u << bg;
+        }
+      }
+
+      // pass 2: this CTA's top-8 over the masked scores
+      Top8 top;
+      top.init();
+      if (ok) {
+        const bool zero_fill = (G > 1) && (P.mask_mode == MR_MASK_ZERO);
+        int g = col0 / S, next_b = (g + 1) * S;
+        for (int c = 0; c < n16; ++c) {
+          tmem_ld16(tmem_base + lane_off + (uint32_t)(c * 16), v);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int e = col0 + c * 16 + i;
+            if (e == next_b) {
+              ++g;
+              next_b += S;
+            }
+            const bool keep = G == 1 || ((kept >> g) & 1u);
+            if (keep) {
+              const float s = mr_sigmoid(v[i]);
+              const float cval = s + bias_s[e - col0];
+              if (cval > top.v[kTopMax - 1]) top.push(cval, e, s);
+            } else if (zero_fill && 0.0f > top.v[kTopMax - 1]) {
+              top.push(0.0f, e, mr_sigmoid(v[i]));
             }
           }
         }
-        mma_commit(bar_empty(s));
       }
-      // Always commit the accumulator barrier, also after an abort, so the
-      // epilogue can wait for every issued MMA to finish before TMEM is freed.
-      mma_commit(bar_acc);
-    }
-  } else {
-    // ---------------- 3xTF32 split, then epilogue ----------------
-    const int ct = threadIdx.x - 64;  // 0..127
-    if (P.use3x) {
-      const int n4 = (int)(plan.hi_bytes / 16);
-      for (int kc = 0; kc < KC; ++kc) {
-        const int s = kc % STAGES;
-        if (!mbar_wait(bar_full(s), (kc / STAGES) & 1, abort)) break;
-        float4* hi = reinterpret_cast<float4*>(smem + s * plan.stage_bytes);
-        float4* lo = reinterpret_cast<float4*>(smem + s * plan.stage_bytes + plan.hi_bytes);
-        for (int i = ct; i < n4; i += 128) {
-          float4 v = hi[i], h, l;
-          h.x = __uint_as_float(__float_as_uint(v.x) & 0xFFFFE000u); l.x = v.x - h.x;
-          h.y = __uint_as_float(__float_as_uint(v.y) & 0xFFFFE000u); l.y = v.y - h.y;
-          h.z = __uint_as_float(__float_as_uint(v.z) & 0xFFFFE000u); l.z = v.z - h.z;
-          h.w = __uint_as_float(__float_as_uint(v.w) & 0xFFFFE000u); l.w = v.w - h.w;
-          hi[i] = h;
-          lo[i] = l;
-        }
-        fence_proxy_async();
-        mbar_arrive(bar_conv(s));
-      }
-    }
-
-    // ---------------- epilogue: one thread = one token ----------------
-    const bool ok = __all_sync(0xffffffffu, mbar_wait(bar_acc, 0, abort));
-    tc_fence_after();
-    const int q = warp & 3;
-    const int row = q * 32 + lane;
-    const long tok = (long)m0 + row;
-    const uint32_t trow = tmem_base + ((uint32_t)(q * 32) << 16);
-    const int G = P.n_group, S = N / G;
-    float v[32];
-
-    if (ok && P.logits_out) {
-      for (int c0 = 0; c0 < N; c0 += 32) {
-        tmem_ld32(trow + c0, v);
-        if (tok < P.T)
+      if (cs > 1) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) P.logits_out[tok * N + c0 + i] = v[i];
-      }
-    }
-
-    uint32_t kept = 0xffffffffu;
-    if (ok && G > 1) {
-      // pass 1: group scores = sum of the two largest biased scores
-      float a1 = -INFINITY, a2 = -INFINITY;
-      int g = 0, next_b = S;
-      for (int c0 = 0; c0 < N; c0 += 32) {
-        tmem_ld32(trow + c0, v);
+        for (int j = 0; j < kTopMax; ++j) {
+          exV[j * BM + row] = top.v[j];
+          exS[j * BM + row] = top.s[j];
+          exI[j * BM + row] = top.i[j];
+        }
+        cluster_sync_all();  // #2: top-8 lists visible to the peer
+        if (crank == 0) {
+          // merge the two sorted lists (value desc, index asc)
+          float pv[kTopMax], ps[kTopMax];
+          int pi[kTopMax];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int e = c0 + i;
-          if (e == next_b) {
-            gs_s[g * BM + row] = a1 + a2;
-            ++g;
-            next_b += S;
-            a1 = -INFINITY;
-            a2 = -INFINITY;
+          for (int j = 0; j < kTopMax; ++j) {
+            pv[j] = ld_peer_f32(&exV[j * BM + row], 1u);
+            ps[j] = ld_peer_f32(&exS[j * BM + row], 1u);
+            pi[j] = __float_as_int(ld_peer_f32(reinterpret_cast<float*>(&exI[j * BM + row]), 1u));
           }
-          const float c = mr_sigmoid(v[i]) + bias_s[e];
-          if (c > a1) {
-            a2 = a1;
-            a1 = c;
-          } else if (c > a2) {
-            a2 = c;
-          }
-        }
-      }
-      gs_s[g * BM + row] = a1 + a2;
-      // keep topk_group groups (lower group index on ties)
-      kept = 0;
-      for (int r = 0; r < P.topk_group; ++r) {
-        float bv = -INFINITY;
-        int bg = -1;
-        for (int gg = 0; gg < G; ++gg) {
-          const float gv = gs_s[gg * BM + row];
-          if (!((kept >> gg) & 1u) && (bg < 0 || gv > bv)) {
-            bv = gv;
-            bg = gg;
-          }
-        }
-        kept |= 1u << bg;
-      }
-    }
-
-    if (ok) {
-      // pass 2: token top-k over the masked scores
-      Top8 top;
-      top.init();
-      const bool zero_fill = (G > 1) && (P.mask_mode == MR_MASK_ZERO);
-      int g = 0, next_b = S;
-      for (int c0 = 0; c0 < N; c0 += 32) {
-        tmem_ld32(trow + c0, v);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int e = c0 + i;
-          if (e == next_b) {
-            ++g;
-            next_b += S;
-          }
-          const bool keep = (kept >> g) & 1u;
-          if (keep) {
-            const float s = mr_sigmoid(v[i]);
-            const float c = s + bias_s[e];
-            if (c > top.v[kTopMax - 1]) top.push(c, e, s);
-          } else if (zero_fill && 0.0f > top.v[kTopMax - 1]) {
-            top.push(0.0f, e, mr_sigmoid(v[i]));
-          }
+          for (int j = 0; j < kTopMax; ++j)
+            if (mr_better(pv[j], pi[j], top.v[kTopMax - 1], top.i[kTopMax - 1])) {
+              // insert (pv, pi) keeping (value desc, index asc)
+              top.v[kTopMax - 1] = pv[j];
+              top.s[kTopMax - 1] = ps[j];
+              top.i[kTopMax - 1] = pi[j];
+#pragma unroll
+              for (int t = kTopMax - 1; t > 0; --t) {
+                if (mr_better(top.v[t], top.i[t], top.v[t - 1], top.i[t - 1])) {
+                  const float tv = top.v[t]; top.v[t] = top.v[t - 1]; top.v[t - 1] = tv;
+                  const float ts = top.s[t]; top.s[t] = top.s[t - 1]; top.s[t - 1] = ts;
+                  const int ti = top.i[t]; top.i[t] = top.i[t - 1]; top.i[t - 1] = ti;
+                }
+              }
+            }
         }
+        cluster_sync_all();  // #3: the peer's lists have been read
       }
-      if (tok < P.T) {
+      if (ok && crank == 0 && tok < P.T) {
         float den = 0.0f;
 #pragma unroll
         for (int j = 0; j < kTopMax; ++j)
@@ -468,6 +675,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
+  // Threads that take no part in the routing epilogue still join its three
+  // cluster barriers, so a cluster always completes them.
+  if (P.CS > 1 && !(warp >= 2 && warp < 6)) {
+    cluster_sync_all();
+    cluster_sync_all();
+    cluster_sync_all();
+  }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -476,6 +690,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
                  "r"(tmem_cols)
                  : "memory");
+  }
+}
+
+// W_lo = W - trunc_tf32(W), once per call, so the router's CTAs stream the
+// residuals by TMA instead of each re-deriving them in shared memory.
+__global__ void __launch_bounds__(256) split_residual_kernel(const float4* __restrict__ W,
+                                                             float4* __restrict__ Wlo, long n4) {
+  for (long i = blockIdx.x * 256L + threadIdx.x; i < n4; i += (long)gridDim.x * 256) {
+    const float4 v = __ldg(W + i);
+    float4 l;
+    l.x = v.x - __uint_as_float(__float_as_uint(v.x) & 0xFFFFE000u);
+    l.y = v.y - __uint_as_float(__float_as_uint(v.y) & 0xFFFFE000u);
+    l.z = v.z - __uint_as_float(__float_as_uint(v.z) & 0xFFFFE000u);
+    l.w = v.w - __uint_as_float(__float_as_uint(v.w) & 0xFFFFE000u);
+    Wlo[i] = l;
   }
 }
 
