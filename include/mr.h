@@ -183,6 +183,46 @@ int mr_dispatch(const int32_t *idx, int T, int k, int N_r, int32_t *counts,
                 void *workspace, size_t workspace_bytes, mr_stream_t stream);
 
 /*
+ * mr_dispatch_noalloc -- mr_dispatch for callers that cannot allocate device
+ * memory when they dispatch.  The pages have no counterpart to this entry
+ * point; it exists for the runtime around the path, not for the method.
+ *
+ * Some callers hold a stream and their input/output tensors but may not call
+ * cudaMalloc (or any allocating routine) at that point: a serving loop whose
+ * device memory is planned before requests start and treats an allocation
+ * mid-request as an error (cudaMalloc can synchronise the device and fragment
+ * a planned pool), or a plug-in running inside another framework's runtime,
+ * which owns all device memory and hands the plug-in only tensors and a
+ * stream.  Such a caller cannot provide mr_dispatch's workspace.  This entry
+ * point takes the same inputs and outputs as mr_dispatch and computes the
+ * same results, with the workspace taken from a fixed array compiled into
+ * libmr.so instead.
+ *
+ * Limits: everything mr_dispatch allows, and additionally
+ * mr_dispatch_workspace_size(T, k, N_r) <= mr_dispatch_noalloc_max_workspace()
+ * (1 MiB: ceil(T*k / 1024) * N_r <= 262144, e.g. T*k up to 1,048,576 entries
+ * at N_r = 256).  Larger sizes return MR_ERR_UNSUPPORTED before any launch;
+ * use mr_dispatch with a workspace for them.
+ *
+ * The fixed array: every GPU that loads libmr.so holds one 1 MiB copy until
+ * the process exits.  The first call on a device looks up the array's device
+ * address (once per device, with that device current), so make that first
+ * call before capturing a stream into a CUDA graph.  The entry point itself
+ * calls no cudaMalloc, cudaFree or other allocating routine.  All calls on a
+ * device share the one array, and it keeps whatever the last call left in
+ * it: nothing in it needs to start at zero (each call rewrites every entry it
+ * later reads), but calls that may overlap on the GPU -- on different streams
+ * without ordering between them -- race on it and must be serialised by the
+ * caller.
+ */
+int mr_dispatch_noalloc(const int32_t *idx, int T, int k, int N_r,
+                        int32_t *counts, int32_t *offsets, int32_t *perm,
+                        int32_t *inv_perm, mr_stream_t stream);
+
+/* Size in bytes of the fixed scratch array mr_dispatch_noalloc uses. */
+size_t mr_dispatch_noalloc_max_workspace(void);
+
+/*
  * mr_gather_rows -- sorted_tokens = x[idxs // k] (Kimi K2 "Add shared output"
  * page, moe_infer).  Copies rows bit for bit.
  *

@@ -60,11 +60,13 @@ def lib():
         L.mr_dispatch_workspace_size.argtypes = [i, i, i]
         L.mr_dispatch_workspace_size.restype = sz
         L.mr_dispatch.argtypes = [p, i, i, i, p, p, p, p, p, sz, p]
+        L.mr_dispatch_noalloc.argtypes = [p, i, i, i, p, p, p, p, p]
+        L.mr_dispatch_noalloc_max_workspace.restype = sz
         L.mr_gather_rows.argtypes = [p, i, i, i, i, p, p, p, p]
         L.mr_combine.argtypes = [p, i, p, p, p, p, i, i, i, p]
         L.mr_get_error.argtypes = [p]
         L.mr_launch_count.restype = C.c_uint64
-        for fn in ("mr_router_forward", "mr_router_forward_ex", "mr_dispatch",
+        for fn in ("mr_router_forward", "mr_router_forward_ex", "mr_dispatch", "mr_dispatch_noalloc",
                    "mr_gather_rows", "mr_combine", "mr_get_error"):
             getattr(L, fn).restype = i
         _lib = L
@@ -197,6 +199,28 @@ def mr_dispatch(idx, N_r, counts=None, offsets=None, perm=None, inv_perm=None, w
         _ptr(idx), T, k, N_r, _ptr(counts), _ptr(offsets), _ptr(perm), _ptr(inv_perm),
         _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
     return counts, offsets, perm, inv_perm
+
+
+def mr_dispatch_noalloc(idx, N_r, counts, offsets, perm, inv_perm=None, stream=None):
+    """Dispatch into caller-provided outputs with no workspace argument: the C
+    entry point uses a fixed scratch array inside libmr.so and allocates
+    nothing (for callers that may not allocate device memory at dispatch
+    time).  Outputs must be preallocated int32 CUDA tensors."""
+    _need(idx, "idx", torch.int32)
+    T, k = idx.shape
+    _need(counts, "counts", torch.int32, (N_r,))
+    _need(offsets, "offsets", torch.int32, (N_r + 1,))
+    _need(perm, "perm", torch.int32, (T * k,))
+    if inv_perm is not None:
+        _need(inv_perm, "inv_perm", torch.int32, (T * k,))
+    _check("mr_dispatch_noalloc", lib().mr_dispatch_noalloc(
+        _ptr(idx), T, k, N_r, _ptr(counts), _ptr(offsets), _ptr(perm), _ptr(inv_perm),
+        _stream(stream)))
+    return counts, offsets, perm, inv_perm
+
+
+def mr_dispatch_noalloc_max_workspace() -> int:
+    return int(lib().mr_dispatch_noalloc_max_workspace())
 
 
 def mr_gather_rows(x, k, perm=None, inv_perm=None, xs=None, stream=None):

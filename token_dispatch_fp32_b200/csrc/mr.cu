@@ -422,6 +422,67 @@ int mr_dispatch(const int32_t* idx, int T, int k, int N_r, int32_t* counts, int3
   return launch_status();
 }
 
+// ---- dispatch without allocation ---------------------------------------------
+//
+// Scratch of mr_dispatch_noalloc: a fixed array in the library's device image.
+// Every device that loads the library holds one copy until the process exits.
+// Host code may not use the symbol as a pointer; its device address is looked
+// up once per device (with that device current) by noalloc_scratch().
+constexpr size_t kNoAllocScratchBytes = size_t(1) << 20;
+static __device__ __align__(256) int32_t g_dispatch_scratch[kNoAllocScratchBytes / sizeof(int32_t)];
+
+int32_t* g_noalloc_ptr[kMaxDevices];
+std::once_flag g_noalloc_once[kMaxDevices];
+
+int32_t* noalloc_scratch() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::call_once(g_noalloc_once[dev], [dev] {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_dispatch_scratch);
+    g_noalloc_ptr[dev] = e == cudaSuccess ? static_cast<int32_t*>(p) : nullptr;
+  });
+  return g_noalloc_ptr[dev];
+}
+
+size_t mr_dispatch_noalloc_max_workspace(void) { return kNoAllocScratchBytes; }
+
+int mr_dispatch_noalloc(const int32_t* idx, int T, int k, int N_r, int32_t* counts,
+                        int32_t* offsets, int32_t* perm, int32_t* inv_perm, mr_stream_t stream) {
+  if (T < 0 || k <= 0 || N_r <= 0) return MR_ERR_INVALID_ARG;
+  if ((long long)T * k >= (1LL << 31)) return MR_ERR_INVALID_ARG;
+  if (k > 32 || N_r > mr::kDispMaxExperts) return MR_ERR_UNSUPPORTED;
+  if (!counts || !offsets) return MR_ERR_INVALID_ARG;
+  if (mr_dispatch_workspace_size(T, k, N_r) > kNoAllocScratchBytes) return MR_ERR_UNSUPPORTED;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (T == 0) {
+    if (cudaMemsetAsync(counts, 0, sizeof(int32_t) * N_r, s) != cudaSuccess ||
+        cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (N_r + 1), s) != cudaSuccess)
+      return MR_ERR_CUDA;
+    return MR_OK;
+  }
+  if (!idx || !perm) return MR_ERR_INVALID_ARG;
+  int32_t* hist = noalloc_scratch();
+  if (!hist) return MR_ERR_CUDA;
+  // Same kernels as mr_dispatch.  The count kernel writes every histogram
+  // entry the later kernels read, so the scratch needs no clearing.
+  const long n = (long)T * k;
+  const long nchunks = mr::disp_num_chunks(n);
+  mr::dispatch_count_kernel<<<(unsigned)nchunks, mr::kDispThreads, sizeof(int) * N_r, s>>>(
+      idx, n, N_r, hist);
+  if (launch_status() != MR_OK) return MR_ERR_CUDA;
+  mr::dispatch_scan_kernel<<<1, 1024, 0, s>>>(hist, nchunks, N_r, n, counts, offsets, perm);
+  if (launch_status() != MR_OK) return MR_ERR_CUDA;
+  const size_t smem = sizeof(int) * mr::kDispWarps * N_r;
+  if (smem > 48 * 1024 &&
+      cudaFuncSetAttribute(mr::dispatch_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem) != cudaSuccess)
+    return MR_ERR_CUDA;
+  mr::dispatch_scatter_kernel<<<(unsigned)nchunks, mr::kDispThreads, smem, s>>>(idx, n, N_r, hist,
+                                                                                perm, inv_perm);
+  return launch_status();
+}
+
 // ---- gather / combine -------------------------------------------------------
 
 int mr_gather_rows(const void* x, int dtype, int T, int d, int k, const int32_t* perm,
