@@ -42,7 +42,11 @@ UNIT = "tokens/s"
 # DRAM traffic per launch measured with ncu (dram__bytes_read.sum +
 # dram__bytes_write.sum) for the dominant kernel, keyed by the SHA-256 of the
 # source file it was built from; reported only while the source is unchanged.
-NCU_TRAFFIC = {}
+NCU_TRAFFIC = {
+    # ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum on the full V3
+    # workload (T=16384): 2.12 GB read + 223.83 MB written per launch.
+    "combine": {"src": "d0f0dabc6a463fef", "bytes": 2.12e9 + 223.83e6},
+}
 
 
 def _src_sha(rel):
@@ -358,7 +362,7 @@ def run_ours(args, w: wl.Workload, rank: int, world: int):
     achieved = bytes_combine / comb_s / 1e9
     traffic = None
     ent = NCU_TRAFFIC.get("combine")
-    if ent and ent.get("src") == _src_sha("token_dispatch_fp32_b200/csrc/rows.cuh"):
+    if ent and ent.get("src") == _src_sha("token_dispatch_fp32_b200/csrc/combine.cuh"):
         traffic = ent["bytes"]
     tf32_peak = peaks["bf16_tflops"] * 0.5  # nominal tf32 : bf16 dense ratio
     stages = {

@@ -1,84 +1,15 @@
-// rows.cuh -- the HBM-bound row movers of the path.
-//
-// gather  (Kimi K2 "Add shared output" page, moe_infer: sorted_tokens =
-//          x[idxs // k]).  With the inverse permutation each token row is read
-//          once and written to its k sorted positions (read d, write k*d);
-//          with only perm each sorted row fetches its token row.
-// combine (same page: new_x[idxs] = outs, weighted sum over k, cast back,
-//          plus the shared expert's output).  Each token gathers its k expert
-//          rows through the inverse permutation -- the scatter-back is fused
-//          into the read -- accumulates in fp32, rounds to the row dtype,
-//          adds the shared row and rounds again.
-//
-// Rows move in 16-byte vectors when the row size allows (8 bf16 / 4 fp32),
-// element by element otherwise.  One CTA handles one token at a time
-// (grid-stride), so every row access is a contiguous, coalesced stream.
+// combine.cuh -- scatter-back, weighted combine and shared add (Kimi K2 "Add
+// shared output" page: new_x[idxs] = outs, weighted sum over k, cast back to
+// the row dtype, plus the shared expert's output).  Each token gathers its k
+// expert rows through the inverse permutation -- the scatter-back is fused
+// into the read -- accumulates in fp32 (FMA, slot order), rounds to the row
+// dtype, adds the shared row and rounds again (bf16, nearest-even).  One CTA
+// per token (grid-stride), 16-byte vectors when the row size allows.
 #pragma once
 
-#include "mr_common.cuh"
+#include "rows_common.cuh"
 
 namespace mr {
-
-constexpr int kRowThreads = 128;
-constexpr int kRowUnroll = 4;
-constexpr int kRowMaxK = 32;
-
-template <typename V>
-__device__ __forceinline__ V ld_stream(const V* p) {
-  return __ldg(p);
-}
-template <>
-__device__ __forceinline__ uint16_t ld_stream<uint16_t>(const uint16_t* p) {
-  return *p;
-}
-
-// ---- gather ----------------------------------------------------------------
-
-template <typename V>
-__global__ void __launch_bounds__(kRowThreads)
-    gather_inv_kernel(const V* __restrict__ x, long T, long nvec, int k,
-                      const int32_t* __restrict__ inv, V* __restrict__ xs) {
-  __shared__ long dst[kRowMaxK];
-  for (long t = blockIdx.x; t < T; t += gridDim.x) {
-    if (threadIdx.x < k) dst[threadIdx.x] = inv[t * k + threadIdx.x];
-    __syncthreads();
-    const V* src = x + t * nvec;
-    for (long v0 = threadIdx.x; v0 < nvec; v0 += kRowUnroll * kRowThreads) {
-      V val[kRowUnroll];
-#pragma unroll
-      for (int u = 0; u < kRowUnroll; ++u) {
-        const long v = v0 + (long)u * kRowThreads;
-        if (v < nvec) val[u] = ld_stream(src + v);
-      }
-      for (int j = 0; j < k; ++j) {
-        const long r = dst[j];
-        if (r < 0) continue;
-        V* out = xs + r * nvec;
-#pragma unroll
-        for (int u = 0; u < kRowUnroll; ++u) {
-          const long v = v0 + (long)u * kRowThreads;
-          if (v < nvec) out[v] = val[u];
-        }
-      }
-    }
-    __syncthreads();
-  }
-}
-
-template <typename V>
-__global__ void __launch_bounds__(kRowThreads)
-    gather_perm_kernel(const V* __restrict__ x, long rows, long nvec, int k,
-                       const int32_t* __restrict__ perm, V* __restrict__ xs) {
-  for (long i = blockIdx.x; i < rows; i += gridDim.x) {
-    const long p = perm[i];
-    if (p < 0) continue;
-    const V* src = x + (p / k) * nvec;
-    V* out = xs + i * nvec;
-    for (long v = threadIdx.x; v < nvec; v += kRowThreads) out[v] = ld_stream(src + v);
-  }
-}
-
-// ---- combine ---------------------------------------------------------------
 
 __device__ __forceinline__ void bf16x2_unpack(uint32_t u, float& lo, float& hi) {
   lo = __uint_as_float(u << 16);

@@ -1,0 +1,56 @@
+// gather.cuh -- sorted_tokens = x[idxs // k] (Kimi K2 "Add shared output"
+// page, moe_infer).  With the inverse permutation each token row is read once
+// and written to its k expert-sorted positions (read d, write k*d elements);
+// with only perm each sorted row fetches its token row.  One CTA per token
+// (grid-stride), 16-byte vectors when the row size allows, elements otherwise.
+#pragma once
+
+#include "rows_common.cuh"
+
+namespace mr {
+
+template <typename V>
+__global__ void __launch_bounds__(kRowThreads)
+    gather_inv_kernel(const V* __restrict__ x, long T, long nvec, int k,
+                      const int32_t* __restrict__ inv, V* __restrict__ xs) {
+  __shared__ long dst[kRowMaxK];
+  for (long t = blockIdx.x; t < T; t += gridDim.x) {
+    if (threadIdx.x < k) dst[threadIdx.x] = inv[t * k + threadIdx.x];
+    __syncthreads();
+    const V* src = x + t * nvec;
+    for (long v0 = threadIdx.x; v0 < nvec; v0 += kRowUnroll * kRowThreads) {
+      V val[kRowUnroll];
+#pragma unroll
+      for (int u = 0; u < kRowUnroll; ++u) {
+        const long v = v0 + (long)u * kRowThreads;
+        if (v < nvec) val[u] = ld_stream(src + v);
+      }
+      for (int j = 0; j < k; ++j) {
+        const long r = dst[j];
+        if (r < 0) continue;
+        V* out = xs + r * nvec;
+#pragma unroll
+        for (int u = 0; u < kRowUnroll; ++u) {
+          const long v = v0 + (long)u * kRowThreads;
+          if (v < nvec) out[v] = val[u];
+        }
+      }
+    }
+    __syncthreads();
+  }
+}
+
+template <typename V>
+__global__ void __launch_bounds__(kRowThreads)
+    gather_perm_kernel(const V* __restrict__ x, long rows, long nvec, int k,
+                       const int32_t* __restrict__ perm, V* __restrict__ xs) {
+  for (long i = blockIdx.x; i < rows; i += gridDim.x) {
+    const long p = perm[i];
+    if (p < 0) continue;
+    const V* src = x + (p / k) * nvec;
+    V* out = xs + i * nvec;
+    for (long v = threadIdx.x; v < nvec; v += kRowThreads) out[v] = ld_stream(src + v);
+  }
+}
+
+}  // namespace mr

@@ -15,7 +15,8 @@
 #include "router_ffma.cuh"
 #include "router_splitk.cuh"
 #include "router_tc.cuh"
-#include "rows.cuh"
+#include "combine.cuh"
+#include "gather.cuh"
 
 namespace {
 
