@@ -200,8 +200,11 @@ def _config(w: wl.Workload, extra=None):
     c = {"workload": w.name, "T": w.T, "d": w.d, "N_r": w.N_r, "n_group": w.n_group,
          "topk_group": w.topk_group, "k": w.k, "route_scale": w.route_scale,
          "mask": "-inf" if w.mask_mode == wl.MASK_NEG_INF else "zero",
-         "rows_dtype": w.io_dtype, "router_precision": "3xTF32 (tcgen05 kind::tf32)",
-         "l2": "inputs larger than L2 (x fp32 470 MB + E 1.88 GB + shared/y per step)",
+         "rows_dtype": w.io_dtype,
+         "router_precision": ("bf16x3: bf16 rows x three bf16 planes of W, exact products, "
+                              "fp32 accumulation (tcgen05 kind::f16)")
+         if w.io_dtype == wl.BF16 else "3xTF32 (tcgen05 kind::tf32)",
+         "l2": "inputs larger than L2 (x 235 MB + E 1.88 GB + shared 235 MB per step)",
          "parallelism": "replicas (token batches per GPU, no collective)"}
     if extra:
         c.update(extra)
@@ -225,37 +228,44 @@ def run_ours(args, w: wl.Workload, rank: int, world: int):
     # inputs (seeded per rank; every rank routes its own batch)
     wr = w.replace(seed=w.seed + 1000 * rank)
     d = wl.gen_router_inputs(wr)
+    bf16_rows = w.io_dtype == wl.BF16
     x32 = torch.from_numpy(d["x_f32"]).to(dev)
-    xb = torch.from_numpy(d["x_bf16"]).view(torch.bfloat16).to(dev)
+    xb = torch.from_numpy(d["x_bf16"]).view(torch.bfloat16).to(dev) if bf16_rows else x32
+    row_t = torch.bfloat16 if bf16_rows else torch.float32
     Wd = torch.from_numpy(d["W"]).to(dev)
     bd = torch.from_numpy(d["b"]).to(dev)
     gen = torch.Generator(device=dev)
     gen.manual_seed(wr.seed)
-    E = torch.randn((w.T * w.k, w.d), generator=gen, device=dev, dtype=torch.float32).to(
-        torch.bfloat16)
-    shared = torch.randn((w.T, w.d), generator=gen, device=dev, dtype=torch.float32).to(
-        torch.bfloat16)
+    E = torch.randn((w.T * w.k, w.d), generator=gen, device=dev, dtype=torch.float32).to(row_t)
+    shared = torch.randn((w.T, w.d), generator=gen, device=dev, dtype=torch.float32).to(row_t)
     idx = torch.empty((w.T, w.k), dtype=torch.int32, device=dev)
     wt = torch.empty((w.T, w.k), dtype=torch.float32, device=dev)
     counts = torch.empty(w.N_r, dtype=torch.int32, device=dev)
     offsets = torch.empty(w.N_r + 1, dtype=torch.int32, device=dev)
     perm = torch.empty(w.T * w.k, dtype=torch.int32, device=dev)
     inv = torch.empty(w.T * w.k, dtype=torch.int32, device=dev)
-    xs = torch.empty((w.T * w.k, w.d), dtype=torch.bfloat16, device=dev)
-    y = torch.empty((w.T, w.d), dtype=torch.bfloat16, device=dev)
+    xs = torch.empty((w.T * w.k, w.d), dtype=row_t, device=dev)
+    y = torch.empty((w.T, w.d), dtype=row_t, device=dev)
     ws_r = torch.empty(max(4, mr.mr_router_workspace_size(w.T, w.d, w.N_r)), dtype=torch.uint8,
                        device=dev)
     ws_d = torch.empty(max(4, mr.mr_dispatch_workspace_size(w.T, w.k, w.N_r)),
                        dtype=torch.uint8, device=dev)
 
     names = ("router", "dispatch", "gather", "combine")
+    # The router reads the hidden states as stored (bf16 rows: the bf16x3
+    # tensor-core decomposition, exact products); fp32 rows take 3xTF32.
+    router_x = xb
+    router_prec = mr.MR_PREC_BF16X3 if bf16_rows else mr.MR_PREC_3XTF32
+
+    def router(xin, prec):
+        mr.mr_router_forward_ex(xin, Wd, bd, w.n_group, w.topk_group, w.k, w.route_scale,
+                                w.mask_mode, precision=prec, idx_out=idx, w_out=wt,
+                                workspace=ws_r, stream=stream)
 
     def step(ev=None):
         if ev is not None:
             ev[0].record(stream)
-        mr.mr_router_forward_ex(x32, Wd, bd, w.n_group, w.topk_group, w.k, w.route_scale,
-                                w.mask_mode, precision=mr.MR_PREC_3XTF32, idx_out=idx,
-                                w_out=wt, workspace=ws_r, stream=stream)
+        router(router_x, router_prec)
         if ev is not None:
             ev[1].record(stream)
         mr.mr_dispatch(idx, w.N_r, counts=counts, offsets=offsets, perm=perm, inv_perm=inv,
@@ -299,6 +309,21 @@ def run_ours(args, w: wl.Workload, rank: int, world: int):
                 for j, n in enumerate(names)}
     assert mr.mr_get_error(stream) == mr.MR_OK
 
+    # For reference, the router on the fp32 cast of the same rows (3xTF32),
+    # timed alone outside the step.
+    alt_ms = None
+    if bf16_rows:
+        for _ in range(3):
+            router(x32, mr.MR_PREC_3XTF32)
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n_alt = max(5, min(50, args.steps))
+        a0.record(stream)
+        for _ in range(n_alt):
+            router(x32, mr.MR_PREC_3XTF32)
+        a1.record(stream)
+        torch.cuda.synchronize(dev)
+        alt_ms = a0.elapsed_time(a1) / n_alt
+
     t = torch.tensor([ms], dtype=torch.float64, device=dev)
     if world > 1:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -307,21 +332,21 @@ def run_ours(args, w: wl.Workload, rank: int, world: int):
     # ---- end to end: pinned host inputs -> device -> path -> host result ----
     e2e = None
     if not args.no_e2e:
-        h_x32 = torch.empty_like(x32, device="cpu").pin_memory()
+        # inputs of one step: the token rows (as stored), the synthetic
+        # expert outputs and the shared-expert output; W and b stay resident
         h_xb = torch.empty_like(xb, device="cpu").pin_memory()
         h_E = torch.empty_like(E, device="cpu").pin_memory()
         h_sh = torch.empty_like(shared, device="cpu").pin_memory()
         h_y = torch.empty_like(y, device="cpu").pin_memory()
         h_idx = torch.empty_like(idx, device="cpu").pin_memory()
         h_w = torch.empty_like(wt, device="cpu").pin_memory()
-        for h, g in ((h_x32, x32), (h_xb, xb), (h_E, E), (h_sh, shared)):
+        for h, g in ((h_xb, xb), (h_E, E), (h_sh, shared)):
             h.copy_(g)
-        h2d = sum(t.numel() * t.element_size() for t in (h_x32, h_xb, h_E, h_sh))
+        h2d = sum(t.numel() * t.element_size() for t in (h_xb, h_E, h_sh))
         d2h = sum(t.numel() * t.element_size() for t in (h_y, h_idx, h_w))
 
         def e2e_step():
             with torch.cuda.stream(stream):
-                x32.copy_(h_x32, non_blocking=True)
                 xb.copy_(h_xb, non_blocking=True)
                 E.copy_(h_E, non_blocking=True)
                 shared.copy_(h_sh, non_blocking=True)
@@ -354,9 +379,10 @@ def run_ours(args, w: wl.Workload, rank: int, world: int):
         return
     peaks = _peaks()
     T, dd, k, N = w.T, w.d, w.k, w.N_r
-    bytes_combine = T * (2 * k * dd + 4 * dd + 8 * k)          # E rows, shared, y, w, inv
-    bytes_gather = T * (2 * dd + 2 * k * dd + 4 * k)          # x row once, k copies, inv
-    bytes_router = T * (4 * dd + 8 * k) + 4 * N * dd + 4 * N  # x, idx/w, W, bias
+    rb = 2 if bf16_rows else 4                                 # row element bytes
+    bytes_combine = T * (rb * k * dd + 2 * rb * dd + 8 * k)   # E rows, shared, y, w, inv
+    bytes_gather = T * (rb * dd + rb * k * dd + 4 * k)        # x row once, k copies, inv
+    bytes_router = T * (rb * dd + 8 * k) + 4 * N * dd + 4 * N  # x, idx/w, W, bias
     flops_router = 2.0 * T * dd * N
     comb_s = stage_ms["combine"] / 1e3
     achieved = bytes_combine / comb_s / 1e9
@@ -364,15 +390,22 @@ def run_ours(args, w: wl.Workload, rank: int, world: int):
     ent = NCU_TRAFFIC.get("combine")
     if ent and ent.get("src") == _src_sha("token_dispatch_fp32_b200/csrc/combine.cuh"):
         traffic = ent["bytes"]
-    tf32_peak = peaks["bf16_tflops"] * 0.5  # nominal tf32 : bf16 dense ratio
+    # Tensor work the router issues: three products per multiply-add, either
+    # bf16 (bf16x3) or tf32 (3xTF32, tf32 peak = bf16 peak x 0.5 nominal).
+    r_s = stage_ms["router"] / 1e3
+    issue_peak = peaks["bf16_tflops"] * (1.0 if bf16_rows else 0.5)
     stages = {
         "router": {"ms": stage_ms["router"],
-                   "tflops_algorithmic": flops_router / (stage_ms["router"] / 1e3) / 1e12,
-                   "tflops_issued_3x": 3 * flops_router / (stage_ms["router"] / 1e3) / 1e12,
-                   "tf32_peak_tflops": tf32_peak,
-                   "frac_issued_of_tf32_peak": 3 * flops_router / (stage_ms["router"] / 1e3)
-                   / 1e12 / tf32_peak,
-                   "gbs": bytes_router / (stage_ms["router"] / 1e3) / 1e9},
+                   "arithmetic": "bf16x3 (bf16 rows, W in three bf16 planes, exact products, "
+                                 "fp32 accumulation)" if bf16_rows else "3xTF32",
+                   "ms_3xtf32_on_fp32_cast": alt_ms,
+                   "tflops_algorithmic": flops_router / r_s / 1e12,
+                   "tflops_issued": 3 * flops_router / r_s / 1e12,
+                   "issue_peak_tflops": issue_peak,
+                   "issue_peak_kind": "bf16 dense (measured)" if bf16_rows
+                                      else "tf32 dense = 0.5 x measured bf16",
+                   "frac_issued_of_peak": 3 * flops_router / r_s / 1e12 / issue_peak,
+                   "gbs": bytes_router / r_s / 1e9},
         "dispatch": {"ms": stage_ms["dispatch"]},
         "gather": {"ms": stage_ms["gather"],
                    "gbs": bytes_gather / (stage_ms["gather"] / 1e3) / 1e9,

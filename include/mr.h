@@ -71,10 +71,17 @@ typedef struct CUstream_st *mr_stream_t;
  *                 into a tf32 high part and a residual; hi*hi + hi*lo + lo*hi
  *                 accumulate in fp32 (fp32-level accuracy).
  * MR_PREC_TF32:   tensor cores, one tf32 product (about 1e-3 relative).
- * MR_PREC_FFMA:   CUDA-core fp32 FMA (any shape; slowest).                   */
+ * MR_PREC_FFMA:   CUDA-core fp32 FMA (any shape; slowest).
+ * MR_PREC_BF16X3: for bf16 activations (x_dtype MR_BF16): W is split once
+ *                 per call into three bf16 planes W1 + W2 + W3 (equal to W
+ *                 within 2^-24 relative), and x*W1 + x*W2 + x*W3 run as
+ *                 bf16 tensor-core products, each exact in fp32, with fp32
+ *                 accumulation: fp32-level accuracy at half the tensor time
+ *                 and half the activation bytes of 3xTF32.                  */
 #define MR_PREC_3XTF32 0
 #define MR_PREC_TF32 1
 #define MR_PREC_FFMA 2
+#define MR_PREC_BF16X3 3
 
 /* Library version, major*10000 + minor*100 + patch. */
 int mr_version(void);
@@ -118,21 +125,25 @@ int mr_router_forward(const float *x, const float *W, const float *bias, int T,
 
 /*
  * mr_router_workspace_size -- bytes of device workspace that
- * mr_router_forward_ex may use for T tokens on the current device: for
- * T <= 256 the split-K partial logits of the small-batch path, about
- * (number of SMs / ceil(N_r/128)) * T * N_r * 4 bytes; above that the
- * tf32 residuals of W (N_r * d * 4 bytes), computed once per call so the
- * fused kernel's CTAs do not each re-derive them.
+ * mr_router_forward_ex may use for T tokens on the current device: the
+ * largest of W's three bf16 planes (3 * N_r * d * 2 bytes, bf16 activations),
+ * W's tf32 residuals (N_r * d * 4 bytes, fp32 activations; both computed once
+ * per call so the fused kernel's CTAs do not each re-derive them) and, for
+ * T <= 256, the split-K partial logits of the small-batch path (about
+ * (number of SMs / ceil(N_r/128)) * T * N_r * 4 bytes).
  */
 size_t mr_router_workspace_size(int T, int d, int N_r);
 
 /*
  * mr_router_forward_ex -- mr_router_forward with explicit options.
  *
- *   x_dtype     MR_F32 ([T,d] fp32) or MR_BF16 ([T,d] bf16 hidden states;
- *               widened to fp32 exactly inside the kernel, so the result is
- *               identical to passing the fp32 cast).
- *   precision   MR_PREC_3XTF32, MR_PREC_TF32 or MR_PREC_FFMA.
+ *   x_dtype     MR_F32 ([T,d] fp32) or MR_BF16 ([T,d] bf16 hidden states,
+ *               whose fp32 cast is exact).
+ *   precision   MR_PREC_3XTF32, MR_PREC_TF32, MR_PREC_FFMA or MR_PREC_BF16X3.
+ *               With MR_BF16 activations the tensor-core precisions (3XTF32
+ *               or BF16X3) both run the bf16x3 decomposition, which needs a
+ *               workspace of mr_router_workspace_size bytes (W's planes);
+ *               MR_PREC_FFMA computes the fp32 cast on CUDA cores.
  *   logits_out  [T, N_r] fp32 logits, or NULL (debug / verification only).
  *   workspace   device buffer of workspace_bytes, or NULL.  With at least
  *               mr_router_workspace_size(T, d, N_r) bytes, batches of up to

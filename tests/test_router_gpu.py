@@ -182,8 +182,9 @@ def test_router_splitk_small_batches(w):
     assert torch.equal(idx, idx2) and torch.equal(wt, wt2)
 
 
-def test_router_workspace_for_large_batches_holds_w_residuals():
-    assert mr.mr_router_workspace_size(4096, 7168, 256) == 4 * 7168 * 256
+def test_router_workspace_for_large_batches_holds_w_planes():
+    # three bf16 planes of W (which also covers W's fp32 tf32-residuals)
+    assert mr.mr_router_workspace_size(4096, 7168, 256) == 3 * 2 * 7168 * 256
 
 
 @pytest.mark.parametrize("w", [SMALL[1], SMALL[2].replace(name="k2_like_T300", T=300),
@@ -229,3 +230,66 @@ def test_tf32_operand_low_bits_probe():
     print("tf32 operand low bits:", kind, got[:10])
     # The 3xTF32 kernels stage raw fp32 tiles as the hi operand and rely on it.
     assert kind == "truncate"
+
+
+BF16X3 = [
+    SMALL[1],                                              # V3-like, ragged T and K tail
+    SMALL[2].replace(name="k2_like_T300", T=300),          # 384 experts, 2-CTA split
+    W("bf16x3_N16_T77", T=77, d=64, N_r=16, n_group=2, topk_group=1, k=3, route_scale=2.5,
+      mask_mode=0, seed=31),
+    W("bf16x3_N320_G10_T140", T=140, d=304, N_r=320, n_group=10, topk_group=3, k=5,
+      route_scale=2.5, mask_mode=1, seed=32, bias_lo=-0.8, bias_hi=-0.2),
+    W("bf16x3_no_bias_T129", T=129, d=256, N_r=64, n_group=8, topk_group=3, k=6,
+      route_scale=1.0, mask_mode=0, seed=33, with_bias=False),
+]
+
+
+def _run_bf16x3(w, precision=mr.MR_PREC_BF16X3, logits=True):
+    d = router_inputs(w)
+    ws = torch.empty(mr.mr_router_workspace_size(w.T, w.d, w.N_r), dtype=torch.uint8,
+                     device="cuda")
+    lg = torch.empty((w.T, w.N_r), dtype=torch.float32, device="cuda") if logits else None
+    idx, wt = mr.mr_router_forward_ex(to_dev(d["x_bf16"], "bf16"), to_dev(d["W"]),
+                                      to_dev(d["b"]), w.n_group, w.topk_group, w.k,
+                                      w.route_scale, w.mask_mode, precision=precision,
+                                      logits_out=lg, workspace=ws)
+    assert mr.mr_get_error() == mr.MR_OK
+    return idx.cpu().numpy(), wt.cpu().numpy(), None if lg is None else lg.cpu().numpy()
+
+
+@pytest.mark.parametrize("w", BF16X3, ids=[w.name for w in BF16X3])
+def test_router_bf16x3_small_all_tokens(w):
+    """bf16 activations: W split into three bf16 planes, exact products,
+    fp32 accumulation -- same tolerances as the fp32 path."""
+    assert w.io_dtype == "bf16"
+    idx, wt, logits = _run_bf16x3(w)
+    stats = compare_router(idx, wt, oracle_router(w, np.arange(w.T)), logits)
+    print(w.name, "bf16x3", stats)
+
+
+@pytest.mark.parametrize("cs", ["1", "2"])
+def test_router_bf16x3_cluster_size_pinned(cs, monkeypatch):
+    monkeypatch.setenv("MR_TC_CLUSTER", cs)
+    w = SMALL[1]
+    idx, wt, logits = _run_bf16x3(w)
+    compare_router(idx, wt, oracle_router(w, np.arange(w.T)), logits)
+
+
+@pytest.mark.parametrize("w", [wl.V3_PREFILL, wl.K2_PREFILL, wl.V3_FULL],
+                         ids=lambda w: w.name)
+def test_router_bf16x3_full_size_sampled(w):
+    idx, wt, logits = _run_bf16x3(w)
+    tok = sample_tokens(w.T, 256, seed=w.seed + 7)
+    stats = compare_router(idx[tok], wt[tok], oracle_router(w, tok), logits[tok])
+    np.testing.assert_allclose(wt.sum(1), w.route_scale, rtol=2e-6)
+    print(w.name, "bf16x3", stats)
+
+
+def test_router_bf16_input_needs_workspace_on_tensor_cores():
+    w = SMALL[1]
+    d = router_inputs(w)
+    with pytest.raises(mr.MRError) as e:
+        mr.mr_router_forward_ex(to_dev(d["x_bf16"], "bf16"), to_dev(d["W"]), to_dev(d["b"]),
+                                w.n_group, w.topk_group, w.k, w.route_scale, w.mask_mode,
+                                precision=mr.MR_PREC_BF16X3)
+    assert e.value.status == mr.MR_ERR_UNSUPPORTED

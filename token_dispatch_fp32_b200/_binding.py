@@ -30,6 +30,7 @@ MR_MASK_ZERO = 1
 MR_PREC_3XTF32 = 0
 MR_PREC_TF32 = 1
 MR_PREC_FFMA = 2
+MR_PREC_BF16X3 = 3
 
 _lib = None
 

@@ -68,6 +68,20 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return g_encode;
 }
 
+// Row-major bf16 matrix [rows, cols], box [box_rows, 32] (64-byte rows, 64-byte swizzle).
+bool make_map_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                   uint32_t box_rows) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * 2};
+  const cuuint32_t box[2] = {32, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Row-major fp32 matrix [rows, cols], box [box_rows, box_cols], swizzled rows.
 bool make_map_f32(CUtensorMap* map, const float* base, uint64_t rows, uint64_t cols,
                   uint32_t box_rows, uint32_t box_cols) {
@@ -97,7 +111,8 @@ int validate_router(const void* x, int x_dtype, const float* W, int T, int d, in
   if (mask_mode == MR_MASK_NEG_INF && n_group > 1 && k > topk_group * (N_r / n_group))
     return MR_ERR_INVALID_ARG;
   if (x_dtype != MR_F32 && x_dtype != MR_BF16) return MR_ERR_INVALID_ARG;
-  if (precision != MR_PREC_3XTF32 && precision != MR_PREC_TF32 && precision != MR_PREC_FFMA)
+  if (precision != MR_PREC_3XTF32 && precision != MR_PREC_TF32 && precision != MR_PREC_FFMA &&
+      precision != MR_PREC_BF16X3)
     return MR_ERR_INVALID_ARG;
   if (!std::isfinite(route_scale)) return MR_ERR_INVALID_ARG;
   if ((long long)T * k >= (1LL << 31) || (long long)T * d >= (1LL << 40)) return MR_ERR_INVALID_ARG;
@@ -239,20 +254,37 @@ int tc_cluster_size(int T, int N_r, int sms) {
 
 // W's residuals [N_r, d] fp32, precomputed into the workspace by the fused path.
 size_t wlo_bytes(int d, int N_r) { return (size_t)N_r * (size_t)d * sizeof(float); }
+// W's three bf16 planes [3, N_r, d] for bf16 activations.
+size_t planes_bytes(int d, int N_r) { return 3 * (size_t)N_r * (size_t)d * 2; }
 
-int launch_tc(const float* x, const float* W, const float* bias, int T, int d, int N_r,
+// x fp32 with tf32 arithmetic (use3x: 3xTF32), or x bf16 with W as three
+// bf16 planes (bf16x3, planes written into `ws` here).
+int launch_tc(const void* x, const float* W, const float* bias, int T, int d, int N_r,
               int n_group, int topk_group, int k, float route_scale, int mask_mode, bool use3x,
-              int32_t* idx_out, float* w_out, float* logits_out, float* wlo, int sms,
-              cudaStream_t st) {
+              bool bf16x3, int32_t* idx_out, float* w_out, float* logits_out, float* wlo,
+              void* ws, int sms, cudaStream_t st) {
   const int CS = tc_cluster_size(T, N_r, sms);
   const int NL = N_r / CS;
-  const mr::tc::Plan plan = mr::tc::make_plan(NL);
+  const mr::tc::Plan plan = mr::tc::make_plan(NL, bf16x3);
   if (plan.stages < 2 || mr::tc::exchange_bytes(n_group) > plan.stages * plan.stage_bytes)
     return MR_ERR_UNSUPPORTED;
   CUtensorMap mx, mw, mwlo;
-  if (!make_map_f32(&mx, x, (uint64_t)T, (uint64_t)d, mr::tc::BM, mr::tc::BK)) return MR_ERR_CUDA;
-  if (!make_map_f32(&mw, W, (uint64_t)N_r, (uint64_t)d, NL, mr::tc::BK)) return MR_ERR_CUDA;
-  const bool use_wlo = use3x && wlo != nullptr;
+  const bool use_wlo = !bf16x3 && use3x && wlo != nullptr;
+  if (bf16x3) {
+    const long n = (long)N_r * d;
+    __nv_bfloat16* planes = static_cast<__nv_bfloat16*>(ws);
+    mr::tc::split_planes_kernel<<<(unsigned)std::min<long>((n + 255) / 256, (long)sms * 8), 256, 0,
+                                  st>>>(W, planes, n);
+    if (launch_status() != MR_OK) return MR_ERR_CUDA;
+    if (!make_map_bf16(&mx, x, (uint64_t)T, (uint64_t)d, mr::tc::BM)) return MR_ERR_CUDA;
+    if (!make_map_bf16(&mw, planes, 3 * (uint64_t)N_r, (uint64_t)d, NL)) return MR_ERR_CUDA;
+    mwlo = mw;
+  } else {
+    if (!make_map_f32(&mx, static_cast<const float*>(x), (uint64_t)T, (uint64_t)d, mr::tc::BM,
+                      mr::tc::BK))
+      return MR_ERR_CUDA;
+    if (!make_map_f32(&mw, W, (uint64_t)N_r, (uint64_t)d, NL, mr::tc::BK)) return MR_ERR_CUDA;
+  }
   if (use_wlo) {
     const long n4 = (long)N_r * d / 4;
     mr::tc::split_residual_kernel<<<(unsigned)std::min<long>((n4 + 255) / 256, (long)sms * 8), 256,
@@ -260,7 +292,7 @@ int launch_tc(const float* x, const float* W, const float* bias, int T, int d, i
                                              reinterpret_cast<float4*>(wlo), n4);
     if (launch_status() != MR_OK) return MR_ERR_CUDA;
     if (!make_map_f32(&mwlo, wlo, (uint64_t)N_r, (uint64_t)d, NL, mr::tc::BK)) return MR_ERR_CUDA;
-  } else {
+  } else if (!bf16x3) {
     mwlo = mw;
   }
   mr::tc::Params P;
@@ -276,6 +308,7 @@ int launch_tc(const float* x, const float* W, const float* bias, int T, int d, i
   P.num_kc = (d + mr::tc::BK - 1) / mr::tc::BK;
   P.use3x = use3x ? 1 : 0;
   P.wlo = use_wlo ? 1 : 0;
+  P.bf16x3 = bf16x3 ? 1 : 0;
   P.route_scale = route_scale;
   P.bias = bias;
   P.idx_out = idx_out;
@@ -331,10 +364,13 @@ const char* mr_status_string(int status) {
 
 size_t mr_router_workspace_size(int T, int d, int N_r) {
   if (T <= 0 || d <= 0 || N_r <= 0 || N_r > 512) return 0;
-  if (!splitk_applies(T, N_r)) return wlo_bytes(d, N_r);
-  int sms = 0, cc = 0;
-  if (!device_info(&sms, &cc)) return 0;
-  return splitk_shape(T, d, N_r, sms).ws_bytes;
+  size_t need = planes_bytes(d, N_r);  // >= W residuals (fp32 x, fused path)
+  if (splitk_applies(T, N_r)) {
+    int sms = 0, cc = 0;
+    if (!device_info(&sms, &cc)) return 0;
+    need = std::max(need, splitk_shape(T, d, N_r, sms).ws_bytes);
+  }
+  return need;
 }
 
 int mr_router_forward_ex(const void* x, int x_dtype, const float* W, const float* bias, int T,
@@ -355,6 +391,15 @@ int mr_router_forward_ex(const void* x, int x_dtype, const float* W, const float
                : launch_ffma<false>(x, W, bias, T, d, N_r, n_group, topk_group, k, route_scale,
                                     mask_mode, idx_out, w_out, logits_out, s);
   }
+  if (x_dtype == MR_BF16 || precision == MR_PREC_BF16X3) {
+    // bf16 activations on tensor cores: W as three bf16 planes (workspace)
+    if (x_dtype != MR_BF16 || precision == MR_PREC_TF32 || cc != 10 || d % 8 != 0 ||
+        !tc_shape_ok(x, MR_F32, W, d, N_r) || !workspace || !aligned16(workspace) ||
+        workspace_bytes < planes_bytes(d, N_r))
+      return MR_ERR_UNSUPPORTED;
+    return launch_tc(x, W, bias, T, d, N_r, n_group, topk_group, k, route_scale, mask_mode, true,
+                     true, idx_out, w_out, logits_out, nullptr, workspace, sms, s);
+  }
   if (cc != 10 || !tc_shape_ok(x, x_dtype, W, d, N_r)) return MR_ERR_UNSUPPORTED;
   if (workspace && splitk_applies(T, N_r) &&
       workspace_bytes >= splitk_shape(T, d, N_r, sms).ws_bytes)
@@ -364,9 +409,9 @@ int mr_router_forward_ex(const void* x, int x_dtype, const float* W, const float
   float* wlo = (workspace && aligned16(workspace) && workspace_bytes >= wlo_bytes(d, N_r))
                    ? static_cast<float*>(workspace)
                    : nullptr;
-  return launch_tc(static_cast<const float*>(x), W, bias, T, d, N_r, n_group, topk_group, k,
-                   route_scale, mask_mode, precision == MR_PREC_3XTF32, idx_out, w_out,
-                   logits_out, wlo, sms, s);
+  return launch_tc(x, W, bias, T, d, N_r, n_group, topk_group, k, route_scale, mask_mode,
+                   precision == MR_PREC_3XTF32, false, idx_out, w_out, logits_out, wlo, nullptr,
+                   sms, s);
 }
 
 int mr_router_forward(const float* x, const float* W, const float* bias, int T, int d, int N_r,

@@ -49,7 +49,7 @@ namespace mr {
 namespace tc {
 
 constexpr int BM = 128;
-constexpr int BK = 32;                        // fp32 along K per stage (128-byte rows)
+constexpr int BK = 32;                        // K elements per stage (fp32: 128-byte rows)
 constexpr int kWorkers = 8;                   // worker warps 2..9
 constexpr int kThreads = 64 + 32 * kWorkers;  // 320
 constexpr int kPromote = 128 / BK;            // K chunks per accumulation interval (128 K)
@@ -62,6 +62,9 @@ constexpr uint32_t kSmemBudget = 232448;      // 227 KB opt-in per CTA
 struct Params {
   int T, d, N, NL, CS, n_group, topk_group, k, mask_mode, num_kc, use3x;
   int wlo;  // W residuals W - trunc_tf32(W) arrive by TMA (map_wlo) instead of being split here
+  // bf16x3: x is bf16 and W arrives as three bf16 planes W1 + W2 + W3 (map_w
+  // over [3*N, d]); every product x*Wi is exact in fp32 (kind::f16 MMA).
+  int bf16x3;
   float route_scale;
   const float* bias;
   int32_t* idx_out;
@@ -78,19 +81,24 @@ struct Plan {
 
 __host__ __device__ inline uint32_t align_up(uint32_t v, uint32_t a) { return (v + a - 1) / a * a; }
 
-__host__ __device__ inline Plan make_plan(int NL) {
+// Stage layout.  tf32: [x | W] fp32 tiles (hi) followed by their residuals
+// (lo), 128-byte rows.  bf16x3: [x | W1 | W2 | W3] bf16 tiles, 64-byte rows.
+__host__ __device__ inline Plan make_plan(int NL, bool bf16x3 = false) {
   Plan p;
-  p.a_bytes = BM * BK * 4;
-  p.b_bytes = NL * BK * 4;
-  p.hi_bytes = p.a_bytes + p.b_bytes;  // [A | B] of one kind (hi or lo)
-  p.stage_bytes = align_up(2 * p.hi_bytes, 1024);
-  const uint32_t extras = 1024 /*align slack*/ + 512 /*barriers*/ + 256 + 4 * 2 * kMaxNL;
+  const int esz = bf16x3 ? 2 : 4;
+  p.a_bytes = BM * BK * esz;
+  p.b_bytes = NL * BK * esz;
+  p.hi_bytes = p.a_bytes + (bf16x3 ? 3 : 1) * p.b_bytes;
+  p.stage_bytes = align_up((bf16x3 ? 1 : 2) * p.hi_bytes, 1024);
+  // after the ring: 256 B of mbarriers, 256 B of flags, the CTA's bias slice;
+  // the launch adds 1 KB so the ring can start on a 1024-byte boundary
+  const uint32_t extras = 1024 + 256 + 256 + 4 * kMaxNL;
   int s = (int)((kSmemBudget - extras) / p.stage_bytes);
   p.stages = s > kMaxStages ? kMaxStages : s;
   p.bar_off = p.stages * p.stage_bytes;
-  p.misc_off = p.bar_off + 512;
+  p.misc_off = p.bar_off + 256;
   p.bias_off = p.misc_off + 256;
-  p.total = p.bias_off + 4 * 2 * kMaxNL;
+  p.total = p.bias_off + 4 * kMaxNL;
   return p;
 }
 
@@ -205,10 +213,38 @@ __device__ __forceinline__ uint64_t make_desc(uint32_t saddr) {
   return d;
 }
 
+// Same for bf16 operands: rows of BK bf16 (64 bytes), 64-byte swizzle, 8-row
+// groups 8 * 64 bytes apart.
+__device__ __forceinline__ uint64_t make_desc_sw64(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)1u << 16;                      // LBO (unused when swizzled)
+  d |= (uint64_t)(512u >> 4) << 32;             // SBO
+  d |= (uint64_t)1u << 46;                      // descriptor version (sm_100)
+  d |= (uint64_t)4u << 61;                      // SWIZZLE_64B
+  return d;
+}
+
 // Instruction descriptor: D fp32, A/B tf32, both K-major, M = 128, N = n.
 __device__ __forceinline__ uint32_t make_idesc(int n) {
   return (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(n >> 3) << 17) |
          ((uint32_t)(BM >> 4) << 24);
+}
+
+// Instruction descriptor: D fp32, A/B bf16, both K-major, M = 128, N = n.
+__device__ __forceinline__ uint32_t make_idesc_bf16(int n) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) |
+         ((uint32_t)(BM >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_bf16(uint32_t dtmem, uint64_t adesc, uint64_t bdesc,
+                                         uint32_t idesc, uint32_t accum) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(dtmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accum)
+      : "memory");
 }
 
 __device__ __forceinline__ void mma_tf32(uint32_t dtmem, uint64_t adesc, uint64_t bdesc,
@@ -291,7 +327,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int NL = P.NL;
-  const Plan plan = make_plan(NL);
+  const bool bf16x3 = P.bf16x3 != 0;
+  const Plan plan = make_plan(NL, bf16x3);
   const int STAGES = plan.stages;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t crank = P.CS > 1 ? cluster_rank() : 0u;
@@ -349,7 +386,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ---------------- TMA producer ----------------
     if (lane == 0) {
-      const uint32_t tx = (uint32_t)(BM + (P.wlo ? 2 : 1) * NL) * BK * 4;
+      const uint32_t tx = bf16x3 ? plan.hi_bytes
+                                 : (uint32_t)(BM + (P.wlo ? 2 : 1) * NL) * BK * 4;
       int issued = 0;
       for (int kc = 0; kc < KC; ++kc) {
         const int s = kc % STAGES;
@@ -358,10 +396,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t base = smem0 + s * plan.stage_bytes;
         mbar_arrive_expect_tx(bar(B_FULL + s), tx);
         tma_load_2d(base, &map_x, bar(B_FULL + s), kc * BK, m0);
-        tma_load_2d(base + plan.a_bytes, &map_w, bar(B_FULL + s), kc * BK, col0);
-        if (P.wlo)
-          tma_load_2d(base + plan.hi_bytes + plan.a_bytes, &map_wlo, bar(B_FULL + s), kc * BK,
-                      col0);
+        if (bf16x3) {
+#pragma unroll
+          for (int pl = 0; pl < 3; ++pl)
+            tma_load_2d(base + plan.a_bytes + pl * plan.b_bytes, &map_w, bar(B_FULL + s),
+                        kc * BK, pl * P.N + col0);
+        } else {
+          tma_load_2d(base + plan.a_bytes, &map_w, bar(B_FULL + s), kc * BK, col0);
+          if (P.wlo)
+            tma_load_2d(base + plan.hi_bytes + plan.a_bytes, &map_wlo, bar(B_FULL + s), kc * BK,
+                        col0);
+        }
       }
       // Every copy this CTA issued must land before the CTA may exit (on the
       // normal path these waits succeed at once).
@@ -371,16 +416,32 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
-      const uint32_t idesc = make_idesc(NL);
+      const uint32_t idesc = bf16x3 ? make_idesc_bf16(NL) : make_idesc(NL);
       for (int kc = 0; kc < KC; ++kc) {
         const int s = kc % STAGES;
         const int j = kc / kPromote, b = j & 1;
         const bool first = (kc % kPromote) == 0;
         if (first && j >= 2 && !mbar_wait(bar(B_ACCE + b), ((j >> 1) - 1) & 1, abort)) break;
-        if (!mbar_wait(P.use3x ? bar(B_CONV + s) : bar(B_FULL + s), (kc / STAGES) & 1, abort))
+        if (!mbar_wait((P.use3x && !bf16x3) ? bar(B_CONV + s) : bar(B_FULL + s),
+                       (kc / STAGES) & 1, abort))
           break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(b * NL);
+        if (bf16x3) {
+          const uint32_t a = smem0 + s * plan.stage_bytes;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint32_t ko = kk * 32;  // 16 bf16 = 32 bytes along K
+            const uint64_t da = make_desc_sw64(a + ko);
+#pragma unroll
+            for (int pl = 0; pl < 3; ++pl)
+              mma_bf16(d_tmem, da, make_desc_sw64(a + plan.a_bytes + pl * plan.b_bytes + ko),
+                       idesc, (!first || kk > 0 || pl > 0) ? 1u : 0u);
+          }
+          mma_commit(bar(B_EMPTY + s));
+          if ((kc % kPromote) == kPromote - 1 || kc == KC - 1) mma_commit(bar(B_ACCF + b));
+          continue;
+        }
         const uint32_t a_hi = smem0 + s * plan.stage_bytes;
         const uint32_t b_hi = a_hi + plan.a_bytes;
         const uint32_t a_lo = a_hi + plan.hi_bytes;
@@ -449,7 +510,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int n4a = (int)(plan.a_bytes / 16);  // the x part of [A | B]
     const int n4 = P.wlo ? n4a : (int)(plan.hi_bytes / 16);
     for (int kc = 0; kc < KC && ok; ++kc) {
-      if (P.use3x) {
+      if (P.use3x && !bf16x3) {
         const int s = kc % STAGES;
         if (!mbar_wait(bar(B_FULL + s), (kc / STAGES) & 1, abort)) {
           ok = false;
@@ -705,6 +766,24 @@ __global__ void __launch_bounds__(256) split_residual_kernel(const float4* __res
     l.z = v.z - __uint_as_float(__float_as_uint(v.z) & 0xFFFFE000u);
     l.w = v.w - __uint_as_float(__float_as_uint(v.w) & 0xFFFFE000u);
     Wlo[i] = l;
+  }
+}
+
+// W -> three bf16 planes with W1 + W2 + W3 = W to within 2^-24 relative:
+// W1 = bf16(W), W2 = bf16(W - W1), W3 = bf16(W - W1 - W2) (round to nearest
+// even; each difference is exact in fp32).  Planes stacked as [3][N_r*d].
+__global__ void __launch_bounds__(256) split_planes_kernel(const float* __restrict__ W,
+                                                           __nv_bfloat16* __restrict__ planes,
+                                                           long n) {
+  for (long i = blockIdx.x * 256L + threadIdx.x; i < n; i += (long)gridDim.x * 256) {
+    const float w = __ldg(W + i);
+    const __nv_bfloat16 p1 = __float2bfloat16_rn(w);
+    const float r1 = w - __bfloat162float(p1);
+    const __nv_bfloat16 p2 = __float2bfloat16_rn(r1);
+    const float r2 = r1 - __bfloat162float(p2);
+    planes[i] = p1;
+    planes[n + i] = p2;
+    planes[2 * n + i] = __float2bfloat16_rn(r2);
   }
 }
 
