@@ -24,8 +24,12 @@ __device__ __forceinline__ uint64_t mr_globaltimer_ns() {
 // Bounded waits give up after this long (then raise MR_FLAG_TIMEOUT).
 #define MR_WAIT_LIMIT_NS 1000000000ull
 
-// s = sigmoid(L) in fp32 (Kimi K2 "Normalize weights" page: logits.sigmoid()).
-__device__ __forceinline__ float mr_sigmoid(float L) { return 1.0f / (1.0f + expf(-L)); }
+// s = sigmoid(L) = 1 / (1 + e^-L) in fp32 (Kimi K2 "Normalize weights" page:
+// logits.sigmoid()), with CUDA's fast exponential and division intrinsics: a
+// few ulp for the O(1) logits of a router, and L -> -inf gives 0, L -> +inf 1.
+__device__ __forceinline__ float mr_sigmoid(float L) {
+  return __fdividef(1.0f, 1.0f + __expf(-L));
+}
 
 // Total order used by every top-k: larger value first, lower index on ties.
 __device__ __forceinline__ bool mr_better(float va, int ia, float vb, int ib) {

@@ -102,9 +102,10 @@ __host__ __device__ inline Plan make_plan(int NL, bool bf16x3 = false) {
   return p;
 }
 
-// Bytes of epilogue exchange space (aliases the stage ring after the K loop).
+// Bytes of epilogue exchange space (aliases the stage ring after the K loop):
+// per column half, group top-2 pairs and top-8 lists of 128 tokens.
 __host__ __device__ inline uint32_t exchange_bytes(int G) {
-  return 4u * (2u * G * BM + 3u * kTopMax * BM);
+  return 4u * 2u * (2u * G * BM + 3u * kTopMax * BM);
 }
 
 // ---- PTX wrappers ----------------------------------------------------------
@@ -560,22 +561,40 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (*abort) ok = false;
     ok = __all_sync(0xffffffffu, ok);
 
-    // ---------------- routing epilogue ----------------
-    if (warp < 6) {
+    // ---------------- routing epilogue: all 8 workers ----------------
+    // Warps w and w+4 read the same 32 TMEM lanes (tokens); half h of the
+    // pair takes chunks [h*nh, (h+1)*nh) of this CTA's expert columns.  Group
+    // top-2 pairs and top-8 lists of the halves (and, with CS = 2, of the peer
+    // CTA's halves) meet in shared memory, so every routing step runs on two
+    // warps per SM sub-partition.
+    {
       const int row = q * 32 + lane;
       const long tok = (long)m0 + row;
       const int G = P.n_group, S = P.N / G;
       const int cs = P.CS;
+      const int nh = (n16 + 1) / 2;
+      const int c_beg = h * nh, c_end = (c_beg + nh < n16) ? c_beg + nh : n16;
       // exchange space aliases the (now idle) stage ring
-      float* exA1 = reinterpret_cast<float*>(smem);             // [G][BM]
-      float* exA2 = exA1 + G * BM;                               // [G][BM]
-      float* exV = exA2 + G * BM;                                // [8][BM]
-      float* exS = exV + kTopMax * BM;                           // [8][BM]
-      int* exI = reinterpret_cast<int*>(exS + kTopMax * BM);     // [8][BM]
-      float v[16];
+      float* exA1 = reinterpret_cast<float*>(smem);             // [2][G][BM]
+      float* exA2 = exA1 + 2 * G * BM;                           // [2][G][BM]
+      float* exV = exA2 + 2 * G * BM;                            // [2][8][BM]
+      float* exS = exV + 2 * kTopMax * BM;                       // [2][8][BM]
+      int* exI = reinterpret_cast<int*>(exS + 2 * kTopMax * BM); // [2][8][BM]
+      float v[16], bv[16];
+      auto load_bias = [&](int c) {
+        const float4* b4 = reinterpret_cast<const float4*>(bias_s + c * 16);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float4 t = b4[i];
+          bv[4 * i] = t.x;
+          bv[4 * i + 1] = t.y;
+          bv[4 * i + 2] = t.z;
+          bv[4 * i + 3] = t.w;
+        }
+      };
 
       if (ok && P.logits_out) {
-        for (int c = 0; c < n16; ++c) {
+        for (int c = c_beg; c < c_end; ++c) {
           tmem_ld16(tmem_base + lane_off + (uint32_t)(c * 16), v);  // whole warp
           if (tok < P.T)
 #pragma unroll
@@ -583,30 +602,35 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
 
-      // pass 1: per-group top-2 of the biased scores over this CTA's experts
+      // pass 1: s = sigmoid(L) back into TMEM; per-group top-2 of c = s + b
       uint32_t kept = 0xffffffffu;
       if (G > 1) {
         for (int g = 0; g < G; ++g) {
-          exA1[g * BM + row] = -INFINITY;
-          exA2[g * BM + row] = -INFINITY;
+          exA1[(h * G + g) * BM + row] = -INFINITY;
+          exA2[(h * G + g) * BM + row] = -INFINITY;
         }
-        if (ok) {
+        if (ok && c_beg < c_end) {
           float a1 = -INFINITY, a2 = -INFINITY;
-          int g = col0 / S, next_b = (g + 1) * S;
-          for (int c = 0; c < n16; ++c) {
-            tmem_ld16(tmem_base + lane_off + (uint32_t)(c * 16), v);
+          int g = (col0 + c_beg * 16) / S, next_b = (g + 1) * S;
+          for (int c = c_beg; c < c_end; ++c) {
+            const uint32_t ta = tmem_base + lane_off + (uint32_t)(c * 16);
+            tmem_ld16(ta, v);
+            load_bias(c);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) v[i] = mr_sigmoid(v[i]);
+            tmem_st16(ta, v);
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
               const int e = col0 + c * 16 + i;
               if (e == next_b) {
-                exA1[g * BM + row] = a1;
-                exA2[g * BM + row] = a2;
+                exA1[(h * G + g) * BM + row] = a1;
+                exA2[(h * G + g) * BM + row] = a2;
                 ++g;
                 next_b += S;
                 a1 = -INFINITY;
                 a2 = -INFINITY;
               }
-              const float cval = mr_sigmoid(v[i]) + bias_s[e - col0];
+              const float cval = v[i] + bv[i];
               if (cval > a1) {
                 a2 = a1;
                 a1 = cval;
@@ -615,22 +639,32 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
             }
           }
-          exA1[g * BM + row] = a1;
-          exA2[g * BM + row] = a2;
+          asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+          exA1[(h * G + g) * BM + row] = a1;
+          exA2[(h * G + g) * BM + row] = a2;
         }
       }
-      if (cs > 1) {
-        cluster_sync_all();  // #1: group pairs visible to the peer
-      }
+      workers_sync();
+      if (cs > 1) cluster_sync_all();  // #1: group pairs visible to the peer
       if (G > 1) {
         float gs[kMaxGroups];
 #pragma unroll
         for (int g = 0; g < kMaxGroups; ++g) {
           if (g < G) {
-            float a1 = exA1[g * BM + row], a2 = exA2[g * BM + row];
-            if (cs > 1) {
-              const float b1 = ld_peer_f32(&exA1[g * BM + row], crank ^ 1u);
-              const float b2 = ld_peer_f32(&exA2[g * BM + row], crank ^ 1u);
+            // top-2 of the union of the halves' (and the peer's) pairs
+            float a1 = -INFINITY, a2 = -INFINITY;
+#pragma unroll
+            for (int src = 0; src < 4; ++src) {
+              if (src >= 2 && cs == 1) break;
+              const int hh = src & 1;
+              float b1, b2;
+              if (src < 2) {
+                b1 = exA1[(hh * G + g) * BM + row];
+                b2 = exA2[(hh * G + g) * BM + row];
+              } else {
+                b1 = ld_peer_f32(&exA1[(hh * G + g) * BM + row], crank ^ 1u);
+                b2 = ld_peer_f32(&exA2[(hh * G + g) * BM + row], crank ^ 1u);
+              }
               if (a1 >= b1) {
                 a2 = fmaxf(a2, b1);
               } else {
@@ -643,12 +677,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         kept = 0;
         for (int r = 0; r < P.topk_group; ++r) {
-          float bv = -INFINITY;
+          float bv2 = -INFINITY;
           int bg = -1;
 #pragma unroll
           for (int g = 0; g < kMaxGroups; ++g) {
-            if (g < G && !((kept >> g) & 1u) && (bg < 0 || gs[g] > bv)) {
-              bv = gs[g];
+            if (g < G && !((kept >> g) & 1u) && (bg < 0 || gs[g] > bv2)) {
+              bv2 = gs[g];
               bg = g;
             }
           }
@@ -656,14 +690,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
 
-      // pass 2: this CTA's top-8 over the masked scores
+      // pass 2: top-8 of this half's masked scores
       Top8 top;
       top.init();
-      if (ok) {
+      if (ok && c_beg < c_end) {
         const bool zero_fill = (G > 1) && (P.mask_mode == MR_MASK_ZERO);
-        int g = col0 / S, next_b = (g + 1) * S;
-        for (int c = 0; c < n16; ++c) {
+        int g = (col0 + c_beg * 16) / S, next_b = (g + 1) * S;
+        for (int c = c_beg; c < c_end; ++c) {
           tmem_ld16(tmem_base + lane_off + (uint32_t)(c * 16), v);
+          load_bias(c);
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             const int e = col0 + c * 16 + i;
@@ -672,41 +707,49 @@ __global__ void __launch_bounds__(kThreads, 1)
               next_b += S;
             }
             const bool keep = G == 1 || ((kept >> g) & 1u);
+            // with groups, pass 1 left s in TMEM; otherwise v holds logits
             if (keep) {
-              const float s = mr_sigmoid(v[i]);
-              const float cval = s + bias_s[e - col0];
-              if (cval > top.v[kTopMax - 1]) top.push(cval, e, s);
+              const float sv = G > 1 ? v[i] : mr_sigmoid(v[i]);
+              const float cval = sv + bv[i];
+              if (cval > top.v[kTopMax - 1]) top.push(cval, e, sv);
             } else if (zero_fill && 0.0f > top.v[kTopMax - 1]) {
-              top.push(0.0f, e, mr_sigmoid(v[i]));
+              top.push(0.0f, e, v[i]);
             }
           }
         }
       }
-      if (cs > 1) {
 #pragma unroll
-        for (int j = 0; j < kTopMax; ++j) {
-          exV[j * BM + row] = top.v[j];
-          exS[j * BM + row] = top.s[j];
-          exI[j * BM + row] = top.i[j];
-        }
-        cluster_sync_all();  // #2: top-8 lists visible to the peer
-        if (crank == 0) {
-          // merge the two sorted lists (value desc, index asc)
-          float pv[kTopMax], ps[kTopMax];
-          int pi[kTopMax];
+      for (int j = 0; j < kTopMax; ++j) {
+        exV[(h * kTopMax + j) * BM + row] = top.v[j];
+        exS[(h * kTopMax + j) * BM + row] = top.s[j];
+        exI[(h * kTopMax + j) * BM + row] = top.i[j];
+      }
+      workers_sync();
+      if (cs > 1) cluster_sync_all();  // #2: top-8 lists visible to the peer
+      if (h == 0 && crank == 0) {
+        // merge the other half's list, then the peer CTA's two lists
+#pragma unroll 1
+        for (int src = 1; src < 4; ++src) {
+          if (src >= 2 && cs == 1) break;
+          const int hh = src & 1;
 #pragma unroll
           for (int j = 0; j < kTopMax; ++j) {
-            pv[j] = ld_peer_f32(&exV[j * BM + row], 1u);
-            ps[j] = ld_peer_f32(&exS[j * BM + row], 1u);
-            pi[j] = __float_as_int(ld_peer_f32(reinterpret_cast<float*>(&exI[j * BM + row]), 1u));
-          }
-#pragma unroll
-          for (int j = 0; j < kTopMax; ++j)
-            if (mr_better(pv[j], pi[j], top.v[kTopMax - 1], top.i[kTopMax - 1])) {
-              // insert (pv, pi) keeping (value desc, index asc)
-              top.v[kTopMax - 1] = pv[j];
-              top.s[kTopMax - 1] = ps[j];
-              top.i[kTopMax - 1] = pi[j];
+            const int o = (hh * kTopMax + j) * BM + row;
+            float pv, ps;
+            int pi;
+            if (src < 2) {
+              pv = exV[o];
+              ps = exS[o];
+              pi = exI[o];
+            } else {
+              pv = ld_peer_f32(&exV[o], 1u);
+              ps = ld_peer_f32(&exS[o], 1u);
+              pi = __float_as_int(ld_peer_f32(reinterpret_cast<float*>(&exI[o]), 1u));
+            }
+            if (mr_better(pv, pi, top.v[kTopMax - 1], top.i[kTopMax - 1])) {
+              top.v[kTopMax - 1] = pv;
+              top.s[kTopMax - 1] = ps;
+              top.i[kTopMax - 1] = pi;
 #pragma unroll
               for (int t = kTopMax - 1; t > 0; --t) {
                 if (mr_better(top.v[t], top.i[t], top.v[t - 1], top.i[t - 1])) {
@@ -716,29 +759,30 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
               }
             }
+          }
         }
-        cluster_sync_all();  // #3: the peer's lists have been read
-      }
-      if (ok && crank == 0 && tok < P.T) {
-        float den = 0.0f;
+        if (ok && tok < P.T) {
+          float den = 0.0f;
 #pragma unroll
-        for (int j = 0; j < kTopMax; ++j)
-          if (j < P.k) den += top.s[j];
-        den += 1e-20f;
+          for (int j = 0; j < kTopMax; ++j)
+            if (j < P.k) den += top.s[j];
+          den += 1e-20f;
 #pragma unroll
-        for (int j = 0; j < kTopMax; ++j) {
-          if (j < P.k) {
-            P.idx_out[tok * P.k + j] = top.i[j];
-            P.w_out[tok * P.k + j] = (top.s[j] / den) * P.route_scale;
+          for (int j = 0; j < kTopMax; ++j) {
+            if (j < P.k) {
+              P.idx_out[tok * P.k + j] = top.i[j];
+              P.w_out[tok * P.k + j] = (top.s[j] / den) * P.route_scale;
+            }
           }
         }
       }
+      if (cs > 1) cluster_sync_all();  // #3: the peer's lists have been read
     }
   }
 
   // Threads that take no part in the routing epilogue still join its three
   // cluster barriers, so a cluster always completes them.
-  if (P.CS > 1 && !(warp >= 2 && warp < 6)) {
+  if (P.CS > 1 && warp < 2) {
     cluster_sync_all();
     cluster_sync_all();
     cluster_sync_all();
