@@ -212,6 +212,30 @@ def _config(w: wl.Workload, extra=None):
 
 
 # ---------------------------------------------------------------------------
+# Multi-rank host logic (replicas): each rank routes its own seeded batch; the
+# step time is the max over ranks; the value counts every rank's tokens.
+
+def rank_workload(w: wl.Workload, rank: int) -> wl.Workload:
+    """The batch rank `rank` routes: the same shapes, its own seed."""
+    return w.replace(seed=w.seed + 1000 * rank)
+
+
+def max_over_ranks(ms: float, world: int, device=None) -> float:
+    """Max of a per-rank time over all ranks (all_reduce MAX when world > 1)."""
+    import torch
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_tokens_per_s(world: int, T: int, ms_max: float) -> float:
+    """Whole-job throughput: all ranks' tokens over the slowest rank's time."""
+    return world * T / (ms_max / 1e3)
+
+
+# ---------------------------------------------------------------------------
 # GPU arm
 
 def run_ours(args, w: wl.Workload, rank: int, world: int):
@@ -226,7 +250,7 @@ def run_ours(args, w: wl.Workload, rank: int, world: int):
     stream = torch.cuda.Stream(dev)
 
     # inputs (seeded per rank; every rank routes its own batch)
-    wr = w.replace(seed=w.seed + 1000 * rank)
+    wr = rank_workload(w, rank)
     d = wl.gen_router_inputs(wr)
     bf16_rows = w.io_dtype == wl.BF16
     x32 = torch.from_numpy(d["x_f32"]).to(dev)
@@ -324,10 +348,7 @@ def run_ours(args, w: wl.Workload, rank: int, world: int):
         torch.cuda.synchronize(dev)
         alt_ms = a0.elapsed_time(a1) / n_alt
 
-    t = torch.tensor([ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_max = float(t.item())
+    ms_max = max_over_ranks(ms, world, dev)
 
     # ---- end to end: pinned host inputs -> device -> path -> host result ----
     e2e = None
@@ -368,10 +389,8 @@ def run_ours(args, w: wl.Workload, rank: int, world: int):
         s1.record(stream)
         torch.cuda.synchronize(dev)
         e_ms = s0.elapsed_time(s1) / n_e2e
-        te = torch.tensor([e_ms], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
-        e2e = {"value": world * w.T / (float(te.item()) / 1e3), "unit": UNIT,
+        e2e = {"value": aggregate_tokens_per_s(world, w.T, max_over_ranks(e_ms, world, dev)),
+               "unit": UNIT,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "steps": n_e2e}
 
@@ -414,7 +433,8 @@ def run_ours(args, w: wl.Workload, rank: int, world: int):
                     "frac_hbm": achieved / peaks["hbm_gbs"]},
     }
     line = {
-        "metric": METRIC, "value": world * T / (ms_max / 1e3), "unit": UNIT, "n_gpus": world,
+        "metric": METRIC, "value": aggregate_tokens_per_s(world, T, ms_max), "unit": UNIT,
+        "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic (seeded; x/W/b numpy PCG64, expert outputs and shared output "

@@ -113,8 +113,10 @@ const char *mr_status_string(int status);
  *
  * Limits: 1 <= N_r <= 512, n_group <= 32, d >= 1.  Uses 3xTF32 tensor-core
  * arithmetic when d % 4 == 0 and N_r % 16 == 0 (N_r % 32 == 0 above 256),
- * CUDA-core FMA otherwise.  The environment variable MR_TC_CLUSTER=1 or 2
- * pins how many CTAs share a 128-token tile (testing only).
+ * CUDA-core FMA otherwise.  The environment variable MR_TC_CLUSTER=1, 2 or
+ * P pins how CTAs share the work of a 128-token tile (testing only): one CTA
+ * with all experts, two CTAs splitting the experts, or (bf16x3) two CTAs
+ * running one 256-token tensor-core MMA.
  * Needs no workspace.  Returns MR_OK or a negative status (nothing launched
  * on an argument error).
  */

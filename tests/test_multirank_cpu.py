@@ -1,0 +1,67 @@
+"""The multi-rank host logic of the benchmark (replicas, weak scaling) on
+CPU ranks over gloo, world size 2: per-rank batches differ, the step time is
+the max over ranks on every rank, and the value counts all ranks' tokens.
+The reference arm runs on rank 0 only."""
+import os
+import socket
+import subprocess
+import sys
+
+import numpy as np
+import pytest
+import torch.multiprocessing as tmp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+import workloads as wl  # noqa: E402
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, times, out_dir):
+    import datetime
+
+    import torch.distributed as dist
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank,
+                            world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        ms_max = bench.max_over_ranks(times[rank], world)
+        wr = bench.rank_workload(wl.TINY, rank)
+        x = wl.gen_router_inputs(wr)["x_f32"]
+        np.save(os.path.join(out_dir, f"x{rank}.npy"), x)
+        with open(os.path.join(out_dir, f"r{rank}.txt"), "w") as f:
+            f.write(f"{ms_max!r} {bench.aggregate_tokens_per_s(world, wr.T, ms_max)!r}")
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_ranks_max_and_aggregate(tmp_path):
+    world, times = 2, [1.25, 3.5]
+    tmp.spawn(_rank_main, args=(world, _free_port(), times, str(tmp_path)), nprocs=world,
+              join=True)
+    res = [open(tmp_path / f"r{r}.txt").read().split() for r in range(world)]
+    for ms, val in res:
+        assert float(ms) == max(times)
+        assert float(val) == pytest.approx(world * wl.TINY.T / (max(times) / 1e3))
+    x0, x1 = (np.load(tmp_path / f"x{r}.npy") for r in range(world))
+    assert x0.shape == x1.shape and not np.array_equal(x0, x1)
+
+
+def test_single_rank_is_identity():
+    assert bench.max_over_ranks(2.0, 1) == 2.0
+    assert bench.rank_workload(wl.TINY, 0) == wl.TINY
+    assert bench.aggregate_tokens_per_s(1, 1000, 2.0) == pytest.approx(5e5)
+
+
+def test_reference_arm_other_ranks_exit_without_work():
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
+    p = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--gpus", "2", "--steps", "3", "--warmup", "3"], env=env,
+                       capture_output=True, text=True, timeout=120)
+    assert p.returncode == 0 and p.stdout.strip() == ""

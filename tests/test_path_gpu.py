@@ -27,11 +27,21 @@ def run_path(w: wl.Workload, E_dev, shared_dev):
     d = router_inputs(w)
     x32 = to_dev(d["x_f32"])
     x_rows = to_dev(d["x_bf16"], "bf16") if w.io_dtype == "bf16" else x32
+    # outputs start as values no kernel writes: a skipped element cannot pass
+    # on the stale result of an earlier call
+    fill = lambda shape, dt, v: torch.full(shape, v, dtype=dt, device="cuda")  # noqa: E731
+    T, k, N, dd = w.T, w.k, w.N_r, w.d
     idx, wt = mr.mr_router_forward(x32, to_dev(d["W"]), to_dev(d["b"]), w.n_group,
-                                   w.topk_group, w.k, w.route_scale, w.mask_mode)
-    counts, offsets, perm, inv = mr.mr_dispatch(idx, w.N_r)
-    xs = mr.mr_gather_rows(x_rows, w.k, perm=perm, inv_perm=inv)
-    y = mr.mr_combine(E_dev if E_dev is not None else xs, wt, inv, shared_dev)
+                                   w.topk_group, w.k, w.route_scale, w.mask_mode,
+                                   idx_out=fill((T, k), torch.int32, -1),
+                                   w_out=fill((T, k), torch.float32, float("nan")))
+    counts, offsets, perm, inv = mr.mr_dispatch(
+        idx, N, counts=fill((N,), torch.int32, -7), offsets=fill((N + 1,), torch.int32, -7),
+        perm=fill((T * k,), torch.int32, -7), inv_perm=fill((T * k,), torch.int32, -7))
+    xs = mr.mr_gather_rows(x_rows, w.k, perm=perm, inv_perm=inv,
+                           xs=fill((T * k, dd), x_rows.dtype, float("nan")))
+    y = mr.mr_combine(E_dev if E_dev is not None else xs, wt, inv, shared_dev,
+                      y=fill((T, dd), x_rows.dtype, float("nan")))
     assert mr.mr_get_error() == mr.MR_OK
     return dict(idx=idx, w=wt, counts=counts, offsets=offsets, perm=perm, inv=inv, xs=xs, y=y,
                 x_rows=x_rows)

@@ -33,20 +33,28 @@ SMALL = [
 FULL = [wl.V3_PREFILL, wl.K2_PREFILL, wl.V3_DECODE, wl.V3_FULL]
 
 
+def _poisoned(T, k):
+    """Output buffers filled with values no kernel writes, so a token the
+    kernel skips cannot pass on a stale result of an earlier call."""
+    return (torch.full((T, k), -1, dtype=torch.int32, device="cuda"),
+            torch.full((T, k), float("nan"), dtype=torch.float32, device="cuda"))
+
+
 def _run(w, precision, x_dtype="f32", want_logits=True, api="ex"):
     d = router_inputs(w)
+    io, wo = _poisoned(w.T, w.k)
     x = to_dev(d["x_bf16"], "bf16") if x_dtype == "bf16" else to_dev(d["x_f32"])
     Wd, b = to_dev(d["W"]), to_dev(d["b"])
     if api == "plain":
         idx, wt = mr.mr_router_forward(x, Wd, b, w.n_group, w.topk_group, w.k, w.route_scale,
-                                       w.mask_mode)
+                                       w.mask_mode, idx_out=io, w_out=wo)
         logits = None
     else:
-        logits = torch.empty((w.T, w.N_r), dtype=torch.float32, device="cuda") \
+        logits = torch.full((w.T, w.N_r), float("nan"), device="cuda") \
             if want_logits else None
         idx, wt = mr.mr_router_forward_ex(x, Wd, b, w.n_group, w.topk_group, w.k,
                                           w.route_scale, w.mask_mode, precision=precision,
-                                          logits_out=logits)
+                                          idx_out=io, w_out=wo, logits_out=logits)
     torch.cuda.synchronize()
     assert mr.mr_get_error() == mr.MR_OK
     return idx.cpu().numpy(), wt.cpu().numpy(), None if logits is None else logits.cpu().numpy()
@@ -165,11 +173,12 @@ def test_router_splitk_small_batches(w):
     assert n > 0
     d = router_inputs(w)
     ws = torch.empty(n, dtype=torch.uint8, device="cuda")
-    logits = torch.empty((w.T, w.N_r), dtype=torch.float32, device="cuda")
+    logits = torch.full((w.T, w.N_r), float("nan"), device="cuda")
+    io, wo = _poisoned(w.T, w.k)
     l0 = mr.mr_launch_count()
     idx, wt = mr.mr_router_forward_ex(to_dev(d["x_f32"]), to_dev(d["W"]), to_dev(d["b"]),
                                       w.n_group, w.topk_group, w.k, w.route_scale, w.mask_mode,
-                                      logits_out=logits, workspace=ws)
+                                      idx_out=io, w_out=wo, logits_out=logits, workspace=ws)
     assert mr.mr_launch_count() - l0 == 2  # GEMM + reduce/route
     assert mr.mr_get_error() == mr.MR_OK
     ref = oracle_router(w, np.arange(w.T))
@@ -248,11 +257,12 @@ def _run_bf16x3(w, precision=mr.MR_PREC_BF16X3, logits=True):
     d = router_inputs(w)
     ws = torch.empty(mr.mr_router_workspace_size(w.T, w.d, w.N_r), dtype=torch.uint8,
                      device="cuda")
-    lg = torch.empty((w.T, w.N_r), dtype=torch.float32, device="cuda") if logits else None
+    lg = torch.full((w.T, w.N_r), float("nan"), device="cuda") if logits else None
+    io, wo = _poisoned(w.T, w.k)
     idx, wt = mr.mr_router_forward_ex(to_dev(d["x_bf16"], "bf16"), to_dev(d["W"]),
                                       to_dev(d["b"]), w.n_group, w.topk_group, w.k,
                                       w.route_scale, w.mask_mode, precision=precision,
-                                      logits_out=lg, workspace=ws)
+                                      idx_out=io, w_out=wo, logits_out=lg, workspace=ws)
     assert mr.mr_get_error() == mr.MR_OK
     return idx.cpu().numpy(), wt.cpu().numpy(), None if lg is None else lg.cpu().numpy()
 
@@ -267,10 +277,13 @@ def test_router_bf16x3_small_all_tokens(w):
     print(w.name, "bf16x3", stats)
 
 
-@pytest.mark.parametrize("cs", ["1", "2"])
-def test_router_bf16x3_cluster_size_pinned(cs, monkeypatch):
+@pytest.mark.parametrize("cs", ["1", "2", "P"])
+@pytest.mark.parametrize("w", [SMALL[1], BF16X3[4]], ids=lambda w: w.name)
+def test_router_bf16x3_cluster_size_pinned(w, cs, monkeypatch):
+    """Every way the bf16x3 kernel can cover a tile: one CTA, two CTAs
+    splitting the experts, or a 2-SM pair running one M = 256 MMA (T = 300
+    and 129 give an odd tile count, so a pair's second tile lies past T)."""
     monkeypatch.setenv("MR_TC_CLUSTER", cs)
-    w = SMALL[1]
     idx, wt, logits = _run_bf16x3(w)
     compare_router(idx, wt, oracle_router(w, np.arange(w.T)), logits)
 

@@ -42,6 +42,8 @@ ROW_CASES = [  # T, d, k, N_r, dtype
     (64, 37, 2, 8, "f32"),        # ragged fp32 row
     (1, 8, 1, 1, "bf16"),
     (128, 64, 32, 64, "bf16"),    # k = 32
+    (2000, 7168, 8, 256, "bf16"),  # several tokens per CTA: the row ring wraps
+    (1500, 4096, 6, 64, "f32"),
 ]
 
 
@@ -67,3 +69,28 @@ def test_combine_matches_oracle(T, d, k, N_r, dtype, with_shared):
     ry, rr = oracle.combine(E, w, inv, sh, k)
     stats = compare_combine(widen(_host(y)), ry, rr, None if sh is None else widen(sh))
     print(T, d, k, dtype, with_shared, stats)
+
+
+@pytest.mark.parametrize("d,dtype", [(7168, "bf16"), (512, "f32"), (1001, "bf16")])
+def test_gather_skips_dropped_slots(d, dtype):
+    """Slots whose inverse entry is -1 (assignments dispatch dropped) write
+    nothing: their sorted rows keep what was there, every other row is the
+    token's row."""
+    T, k, N_r = 700, 4, 32
+    idx, _, _, _, x = _problem(T, d, k, N_r, dtype, seed=11)
+    _, _, perm, inv = oracle.dispatch(idx, N_r)
+    rng = np.random.default_rng(5)
+    drop = rng.random(T * k) < 0.1
+    inv_d = np.where(drop, -1, inv).astype(np.int32)
+    poison = np.full((T * k, d), 0x7FC1 if dtype == "bf16" else np.nan,
+                     dtype=np.uint16 if dtype == "bf16" else np.float32)
+    xs = _dev(poison.copy())
+    mr.mr_gather_rows(_dev(x), k, perm=torch.from_numpy(perm).cuda(),
+                      inv_perm=torch.from_numpy(inv_d).cuda(), xs=xs)
+    assert mr.mr_get_error() == mr.MR_OK
+    got = _host(xs)
+    want = oracle.gather(x, k, perm)
+    kept_rows = np.sort(inv[~drop])
+    dropped_rows = np.sort(inv[drop])
+    assert np.array_equal(got[kept_rows], want[kept_rows])
+    assert np.array_equal(got[dropped_rows].view(np.uint8), poison[dropped_rows].view(np.uint8))

@@ -3,6 +3,9 @@
 // and written to its k expert-sorted positions (read d, write k*d elements);
 // with only perm each sorted row fetches its token row.  One CTA per token
 // (grid-stride), 16-byte vectors when the row size allows, elements otherwise.
+// (A copy-engine variant -- cp.async.bulk row loads into a shared-memory ring
+// and k bulk stores per row -- measured no faster on the full DeepSeek-V3
+// batch, so the plain vector copy stays.)
 #pragma once
 
 #include "rows_common.cuh"

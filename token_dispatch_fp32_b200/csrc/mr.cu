@@ -238,18 +238,30 @@ int launch_splitk(const float* x, const float* W, const float* bias, int T, int 
   return MR_ERR_UNSUPPORTED;
 }
 
-// Experts per CTA: all of them, or half per CTA of a 2-CTA cluster when
-// N_r > 256 (TMEM holds two accumulation buffers of at most 256 columns) or
-// when a split doubles the CTA count of a small batch.
-int tc_cluster_size(int T, int N_r, int sms) {
-  if (N_r > 256) return 2;
-  // MR_TC_CLUSTER=1|2 pins the choice (used by the tests to cover both).
+// How CTAs share a 128-token tile of the fused router:
+//  - CS = 2 splits the experts over a 2-CTA cluster: always when N_r > 256
+//    (TMEM holds two accumulation buffers of at most 256 columns), and when
+//    it at least doubles the CTA count of a small batch;
+//  - pair: bf16x3 with N_r <= 256 on large batches; two CTAs run one M = 256
+//    MMA over consecutive tiles and each stages half of W.
+// MR_TC_CLUSTER = 1, 2 or P pins the choice (used by the tests to cover each).
+struct TcShape {
+  int CS;
+  bool pair;
+};
+
+TcShape tc_shape(int T, int N_r, int sms, bool bf16x3) {
+  if (N_r > 256) return {2, false};
+  const bool pair_ok = bf16x3 && N_r % 32 == 0;
   if (const char* env = getenv("MR_TC_CLUSTER")) {
-    if (env[0] == '1') return 1;
-    if (env[0] == '2' && N_r % 32 == 0) return 2;
+    if (env[0] == '1') return {1, false};
+    if (env[0] == '2' && N_r % 32 == 0) return {2, false};
+    if ((env[0] == 'P' || env[0] == 'p') && pair_ok) return {1, true};
   }
   const int tiles = (T + mr::tc::BM - 1) / mr::tc::BM;
-  return (N_r % 32 == 0 && 2 * tiles <= sms) ? 2 : 1;
+  if (N_r % 32 == 0 && 2 * tiles <= sms) return {2, false};
+  if (pair_ok && tiles >= 2) return {1, true};
+  return {1, false};
 }
 
 // W's residuals [N_r, d] fp32, precomputed into the workspace by the fused path.
@@ -263,11 +275,17 @@ int launch_tc(const void* x, const float* W, const float* bias, int T, int d, in
               int n_group, int topk_group, int k, float route_scale, int mask_mode, bool use3x,
               bool bf16x3, int32_t* idx_out, float* w_out, float* logits_out, float* wlo,
               void* ws, int sms, cudaStream_t st) {
-  const int CS = tc_cluster_size(T, N_r, sms);
+  TcShape shp = tc_shape(T, N_r, sms, bf16x3);
+  auto fits = [&](const TcShape& t) {
+    const mr::tc::Plan p = mr::tc::make_plan(N_r / t.CS, bf16x3, t.pair);
+    return p.stages >= 2 && mr::tc::epilogue_smem_bytes(n_group) <= p.stages * p.stage_bytes;
+  };
+  if (!fits(shp) && shp.pair) shp = {1, false};  // a pair's ring is half the size
+  if (!fits(shp)) return MR_ERR_UNSUPPORTED;
+  const int CS = shp.CS;
+  const bool pair = shp.pair;
   const int NL = N_r / CS;
-  const mr::tc::Plan plan = mr::tc::make_plan(NL, bf16x3);
-  if (plan.stages < 2 || mr::tc::exchange_bytes(n_group) > plan.stages * plan.stage_bytes)
-    return MR_ERR_UNSUPPORTED;
+  const mr::tc::Plan plan = mr::tc::make_plan(NL, bf16x3, pair);
   CUtensorMap mx, mw, mwlo;
   const bool use_wlo = !bf16x3 && use3x && wlo != nullptr;
   if (bf16x3) {
@@ -277,7 +295,8 @@ int launch_tc(const void* x, const float* W, const float* bias, int T, int d, in
                                   st>>>(W, planes, n);
     if (launch_status() != MR_OK) return MR_ERR_CUDA;
     if (!make_map_bf16(&mx, x, (uint64_t)T, (uint64_t)d, mr::tc::BM)) return MR_ERR_CUDA;
-    if (!make_map_bf16(&mw, planes, 3 * (uint64_t)N_r, (uint64_t)d, NL)) return MR_ERR_CUDA;
+    if (!make_map_bf16(&mw, planes, 3 * (uint64_t)N_r, (uint64_t)d, pair ? NL / 2 : NL))
+      return MR_ERR_CUDA;
     mwlo = mw;
   } else {
     if (!make_map_f32(&mx, static_cast<const float*>(x), (uint64_t)T, (uint64_t)d, mr::tc::BM,
@@ -309,20 +328,20 @@ int launch_tc(const void* x, const float* W, const float* bias, int T, int d, in
   P.use3x = use3x ? 1 : 0;
   P.wlo = use_wlo ? 1 : 0;
   P.bf16x3 = bf16x3 ? 1 : 0;
+  P.pair = pair ? 1 : 0;
   P.route_scale = route_scale;
   P.bias = bias;
   P.idx_out = idx_out;
   P.w_out = w_out;
   P.logits_out = logits_out;
   const size_t smem = plan.total + 1024;
-  if (cudaFuncSetAttribute(mr::tc::router_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)smem) != cudaSuccess)
+  auto kern = pair ? mr::tc::router_tc_kernel<true> : mr::tc::router_tc_kernel<false>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+      cudaSuccess)
     return MR_ERR_CUDA;
-  if (CS > 1 && cudaFuncSetAttribute(mr::tc::router_tc_kernel,
-                                     cudaFuncAttributeNonPortableClusterSizeAllowed, 0) !=
-                    cudaSuccess)
-    return MR_ERR_CUDA;
-  const unsigned tiles = (unsigned)((T + mr::tc::BM - 1) / mr::tc::BM);
+  unsigned tiles = (unsigned)((T + mr::tc::BM - 1) / mr::tc::BM);
+  if (pair) tiles = (tiles + 1) / 2 * 2;  // a pair's second tile may be past T
+  const unsigned cluster = (CS > 1 || pair) ? 2u : 1u;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(tiles * CS);
   cfg.blockDim = dim3(mr::tc::kThreads);
@@ -330,12 +349,12 @@ int launch_tc(const void* x, const float* W, const float* bias, int T, int d, in
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = CS;
+  attr[0].val.clusterDim.x = cluster;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, mr::tc::router_tc_kernel, mx, mw, mwlo, P);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, mx, mw, mwlo, P);
   if (e != cudaSuccess) {
     (void)cudaGetLastError();
     g_launches.fetch_add(1, std::memory_order_relaxed);

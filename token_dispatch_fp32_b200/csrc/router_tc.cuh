@@ -5,34 +5,40 @@
 // A token's logits never go to HBM: they accumulate in tensor memory (TMEM
 // lane = token, column = expert) and the routing epilogue reads them back.
 //
-//   warp 0      TMA producer: x tile [128 x 32] and W tile [NL x 32] fp32 per
-//               stage (128-byte hardware swizzle), completion on an mbarrier.
-//   warp 1      TMEM owner and MMA issuer (one elected thread):
-//               tcgen05.mma.cta_group::1.kind::tf32, M = 128, N = NL.
-//   warps 2..9  "workers":
-//               (a) 3xTF32 split of every staged fp32 value v into
-//                   hi = v with the low 13 mantissa bits cleared (exact in
-//                   tf32) and lo = v - hi (exact in fp32); the MMA issues
-//                   hi*hi + hi*lo + lo*hi into one fp32 accumulator.  The
-//                   tensor core ignores those 13 bits of a tf32 operand, so
-//                   the staged tile serves as hi unchanged and only lo is
-//                   written; W's residuals may instead come precomputed (TMA);
-//                   lo(x)*hi(W) is skipped when a stage's x residuals are all
-//                   zero (tf32-exact activations, e.g. bf16 hidden states);
-//               (b) promotion: the tensor core adds each product into its
-//                   fp32 accumulator rounding toward zero, so one accumulator
-//                   over all d would drift by ~1 ulp per MMA.  The K loop is
-//                   cut into intervals of kPromote chunks that alternate
-//                   between two TMEM buffers; each finished interval is added
-//                   into fp32 registers (round to nearest) while the tensor
-//                   core fills the other buffer.  Interval errors change sign
-//                   from interval to interval and no longer accumulate.
-//               (c) epilogue: the register sums go back to TMEM, then warp w
-//                   (w = 2..5) routes the 32 tokens of TMEM lanes 32*(w%4)..:
-//                   sigmoid, bias, per-group top-2, group top-k, a top-8
-//                   insertion list with lower-index tie-break, renormalise and
-//                   scale.  With CS = 2 the two CTAs exchange per-group top-2
-//                   pairs and top-8 lists through distributed shared memory.
+//   warp 0      TMA producer: x tile [128 x BK] and W tile [NL x BK] per
+//               stage (hardware swizzle), completion on an mbarrier.
+//   warp 1      TMEM owner and MMA issuer (one elected thread), M = 128 (or
+//               M = 256 over a CTA pair, cta_group::2), N = NL.
+//   warps 2..9  "workers".
+//
+// Two ways to get fp32-accurate logits from the tensor cores:
+//   3xTF32 (fp32 x): every staged fp32 value v splits into hi = v with the
+//     low 13 mantissa bits cleared (exact in tf32) and lo = v - hi (exact in
+//     fp32); kind::tf32 MMAs issue hi*hi + hi*lo + lo*hi.  The tensor core
+//     ignores those 13 bits of a tf32 operand, so the staged tile serves as hi
+//     unchanged and the workers only write lo; W's residuals may instead come
+//     precomputed (TMA); lo(x)*hi(W) is skipped when a stage's x residuals are
+//     all zero.
+//   bf16x3 (bf16 x): W is stored once as three bf16 planes W1 + W2 + W3 that
+//     sum to W exactly (24 significant bits); kind::f16 MMAs issue x*W1 +
+//     x*W2 + x*W3, each product exact in fp32 -- the fp32 dot product of the
+//     stored bf16 activations with the fp32 weights, up to accumulation order.
+//
+// Promotion: the tensor core adds each product into its fp32 accumulator
+// rounding toward zero, so one accumulator over all d would drift by ~1 ulp per
+// MMA.  The K loop is cut into intervals of 128 K that alternate between two
+// TMEM buffers; the workers add each finished interval into fp32 registers
+// (round to nearest) while the tensor core fills the other buffer.
+//
+// Routing epilogue (all 8 workers; the sums go back to TMEM first): warps w
+// and w+4 read the same 32 TMEM lanes (tokens), each half of the expert
+// columns.  Pass 1 turns logits into s = sigmoid(L) in place and keeps the
+// per-group top-2 of c = s + b (branch-free); the halves' pairs (and, with
+// CS = 2, the peer CTA's through distributed shared memory) meet in shared
+// memory and the topk_group best groups are kept.  Pass 2 forms each chunk's
+// 16 masked candidates and inserts only those above the current 8th into a
+// sorted top-8 list (lower index first on ties); the halves' lists (and the
+// peer's) are merged bitonically; then renormalise and scale.
 //
 // Arithmetic follows the pages (Kimi K2 "Normalize weights" page,
 // MoEGate.forward; DeepSeek-V3.2-Exp "Normalize weights" page, Gate.forward).
@@ -56,7 +62,7 @@ constexpr int kPromote = 128 / BK;            // K chunks per accumulation inter
 constexpr int kMaxNL = 256;
 constexpr int kMaxGroups = 32;
 constexpr int kTopMax = 8;
-constexpr int kMaxStages = 6;
+constexpr int kMaxStages = 8;
 constexpr uint32_t kSmemBudget = 232448;      // 227 KB opt-in per CTA
 
 struct Params {
@@ -65,6 +71,11 @@ struct Params {
   // bf16x3: x is bf16 and W arrives as three bf16 planes W1 + W2 + W3 (map_w
   // over [3*N, d]); every product x*Wi is exact in fp32 (kind::f16 MMA).
   int bf16x3;
+  // pair (bf16x3, N <= 256): the cluster's two CTAs own consecutive 128-token
+  // tiles and run one M = 256 MMA (cta_group::2) issued by CTA 0; each CTA
+  // stages its own x tile and half of W's rows, and keeps its own 128 tokens
+  // x all N experts in its TMEM.
+  int pair;
   float route_scale;
   const float* bias;
   int32_t* idx_out;
@@ -83,11 +94,11 @@ __host__ __device__ inline uint32_t align_up(uint32_t v, uint32_t a) { return (v
 
 // Stage layout.  tf32: [x | W] fp32 tiles (hi) followed by their residuals
 // (lo), 128-byte rows.  bf16x3: [x | W1 | W2 | W3] bf16 tiles, 64-byte rows.
-__host__ __device__ inline Plan make_plan(int NL, bool bf16x3 = false) {
+__host__ __device__ inline Plan make_plan(int NL, bool bf16x3 = false, bool pair = false) {
   Plan p;
   const int esz = bf16x3 ? 2 : 4;
   p.a_bytes = BM * BK * esz;
-  p.b_bytes = NL * BK * esz;
+  p.b_bytes = (pair ? NL / 2 : NL) * BK * esz;
   p.hi_bytes = p.a_bytes + (bf16x3 ? 3 : 1) * p.b_bytes;
   p.stage_bytes = align_up((bf16x3 ? 1 : 2) * p.hi_bytes, 1024);
   // after the ring: 256 B of mbarriers, 256 B of flags, the CTA's bias slice;
@@ -103,9 +114,13 @@ __host__ __device__ inline Plan make_plan(int NL, bool bf16x3 = false) {
 }
 
 // Bytes of epilogue exchange space (aliases the stage ring after the K loop):
-// per column half, group top-2 pairs and top-8 lists of 128 tokens.
+// per column half, group top-2 pairs and top-8 lists of 128 tokens; followed
+// by the pass-2 candidate scratch (16 scores and 16 s per worker thread).
 __host__ __device__ inline uint32_t exchange_bytes(int G) {
   return 4u * 2u * (2u * G * BM + 3u * kTopMax * BM);
+}
+__host__ __device__ inline uint32_t epilogue_smem_bytes(int G) {
+  return exchange_bytes(G) + 4u * 2u * 16u * 32u * kWorkers;
 }
 
 // ---- PTX wrappers ----------------------------------------------------------
@@ -165,6 +180,29 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1)
       : "memory");
+}
+
+// The same copy for a 2-SM pair: completes on an mbarrier given by its
+// shared::cluster address, which may be the peer CTA's.
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map,
+                                                 uint32_t bar_cluster, int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(c0), "r"(c1)
+      : "memory");
+}
+
+// shared::cluster address of `local` in CTA `rank` of this cluster.
+__device__ __forceinline__ uint32_t cluster_addr(uint32_t local, uint32_t rank) {
+  uint32_t ra;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(local), "r"(rank));
+  return ra;
+}
+
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster)
+               : "memory");
 }
 
 __device__ __forceinline__ void fence_proxy_async() {
@@ -232,10 +270,10 @@ __device__ __forceinline__ uint32_t make_idesc(int n) {
          ((uint32_t)(BM >> 4) << 24);
 }
 
-// Instruction descriptor: D fp32, A/B bf16, both K-major, M = 128, N = n.
-__device__ __forceinline__ uint32_t make_idesc_bf16(int n) {
+// Instruction descriptor: D fp32, A/B bf16, both K-major, M = m, N = n.
+__device__ __forceinline__ uint32_t make_idesc_bf16(int n, int m = BM) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) |
-         ((uint32_t)(BM >> 4) << 24);
+         ((uint32_t)(m >> 4) << 24);
 }
 
 __device__ __forceinline__ void mma_bf16(uint32_t dtmem, uint64_t adesc, uint64_t bdesc,
@@ -255,6 +293,26 @@ __device__ __forceinline__ void mma_tf32(uint32_t dtmem, uint64_t adesc, uint64_
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(dtmem),
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accum)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_bf16_pair(uint32_t dtmem, uint64_t adesc, uint64_t bdesc,
+                                              uint32_t idesc, uint32_t accum) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(dtmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accum)
+      : "memory");
+}
+
+// Arrive on the barrier at this offset in both CTAs of the pair once every
+// pair MMA issued so far has completed.
+__device__ __forceinline__ void mma_commit_pair(uint32_t bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], %1;" ::"r"(bar),
+      "h"((uint16_t)3)
       : "memory");
 }
 
@@ -305,6 +363,35 @@ struct Top8 {
       i[j] = 0x7fffffff;
     }
   }
+  // Keep the better (value desc, index asc) of slots a and b in a.
+  __device__ __forceinline__ void order(int a, int b) {
+    if (mr_better(v[b], i[b], v[a], i[a])) {
+      const float tv = v[a]; v[a] = v[b]; v[b] = tv;
+      const float ts = s[a]; s[a] = s[b]; s[b] = ts;
+      const int ti = i[a]; i[a] = i[b]; i[b] = ti;
+    }
+  }
+  // Merge another sorted list into this one, keeping the best 8: taking the
+  // better of (this[j], other[7-j]) leaves the 8 best as a bitonic sequence,
+  // which three half-cleaner rounds sort (all indices static, no branches
+  // beyond the selects).
+  __device__ __forceinline__ void merge(const float (&ov)[kTopMax], const float (&os)[kTopMax],
+                                        const int (&oi)[kTopMax]) {
+#pragma unroll
+    for (int j = 0; j < kTopMax; ++j) {
+      const int r = kTopMax - 1 - j;
+      if (mr_better(ov[r], oi[r], v[j], i[j])) {
+        v[j] = ov[r];
+        s[j] = os[r];
+        i[j] = oi[r];
+      }
+    }
+#pragma unroll
+    for (int d = kTopMax / 2; d > 0; d >>= 1)
+#pragma unroll
+      for (int j = 0; j < kTopMax; ++j)
+        if ((j & d) == 0) order(j, j + d);
+  }
   __device__ __forceinline__ void push(float cv, int ci, float cs) {
     v[kTopMax - 1] = cv;
     i[kTopMax - 1] = ci;
@@ -320,6 +407,7 @@ struct Top8 {
   }
 };
 
+template <bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
     router_tc_kernel(const __grid_constant__ CUtensorMap map_x,
                      const __grid_constant__ CUtensorMap map_w,
@@ -329,12 +417,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int NL = P.NL;
   const bool bf16x3 = P.bf16x3 != 0;
-  const Plan plan = make_plan(NL, bf16x3);
+  // The 2-SM instructions exist only in the PAIR instantiation: a kernel that
+  // contains them must be launched in clusters of two.
+  constexpr bool pair = PAIR;
+  const Plan plan = make_plan(NL, bf16x3, pair);
   const int STAGES = plan.stages;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t crank = P.CS > 1 ? cluster_rank() : 0u;
-  const int tile = blockIdx.x / P.CS;
-  const int col0 = (int)crank * NL;  // first global expert of this CTA
+  const uint32_t crank = (P.CS > 1 || pair) ? cluster_rank() : 0u;
+  const int tile = pair ? (int)blockIdx.x : (int)blockIdx.x / P.CS;
+  const int col0 = pair ? 0 : (int)crank * NL;  // first expert of this CTA's accumulator
+  const bool leader = !pair || crank == 0;       // issues the MMAs
+  const int wrow0 = pair ? (int)crank * (NL / 2) : col0;  // first W row this CTA stages
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + plan.bar_off);
   // [0,S) full  [S,2S) converted  [2S,3S) empty  3S+{0,1} acc full
@@ -360,19 +453,29 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(bar(B_ACCF + 0), 1);
     mbar_init(bar(B_ACCF + 1), 1);
-    mbar_init(bar(B_ACCE + 0), 32 * kWorkers);
-    mbar_init(bar(B_ACCE + 1), 32 * kWorkers);
+    mbar_init(bar(B_ACCE + 0), (pair ? 2 : 1) * 32 * kWorkers);  // both CTAs' workers
+    mbar_init(bar(B_ACCE + 1), (pair ? 2 : 1) * 32 * kWorkers);
     mbar_init(bar(B_DRAIN), 1);
     *abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                     smem_u32(tmem_slot)),
-                 "r"(tmem_cols)
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    if constexpr (PAIR) {
+      asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                       smem_u32(tmem_slot)),
+                   "r"(tmem_cols)
+                   : "memory");
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+    } else {
+      asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                       smem_u32(tmem_slot)),
+                   "r"(tmem_cols)
+                   : "memory");
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
   }
+  // pair: barriers must be initialised in both CTAs before any remote use
+  if (pair) cluster_sync_all();
   for (int e = threadIdx.x; e < NL; e += kThreads)
     bias_s[e] = P.bias ? P.bias[col0 + e] : 0.0f;
   tc_fence_before();
@@ -395,6 +498,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (kc >= STAGES && !mbar_wait(bar(B_EMPTY + s), ((kc / STAGES) - 1) & 1, abort)) break;
         ++issued;
         const uint32_t base = smem0 + s * plan.stage_bytes;
+        if constexpr (PAIR) {
+          // both CTAs' copies complete on CTA 0's full barrier
+          const uint32_t fb = cluster_addr(bar(B_FULL + s), 0);
+          if (leader) mbar_arrive_expect_tx(bar(B_FULL + s), 2 * tx);
+          tma_load_2d_pair(base, &map_x, fb, kc * BK, m0);
+#pragma unroll
+          for (int pl = 0; pl < 3; ++pl)
+            tma_load_2d_pair(base + plan.a_bytes + pl * plan.b_bytes, &map_w, fb, kc * BK,
+                             pl * P.N + wrow0);
+          continue;
+        }
         mbar_arrive_expect_tx(bar(B_FULL + s), tx);
         tma_load_2d(base, &map_x, bar(B_FULL + s), kc * BK, m0);
         if (bf16x3) {
@@ -410,14 +524,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       // Every copy this CTA issued must land before the CTA may exit (on the
-      // normal path these waits succeed at once).
-      for (int kc = issued - STAGES < 0 ? 0 : issued - STAGES; kc < issued; ++kc)
-        mbar_wait(bar(B_FULL + kc % STAGES), (kc / STAGES) & 1, abort, true);
+      // normal path these waits succeed at once).  A pair's copies complete
+      // on CTA 0's barriers: CTA 0 drains them, CTA 1 is held by the final
+      // cluster barrier until then.
+      if (leader)
+        for (int kc = issued - STAGES < 0 ? 0 : issued - STAGES; kc < issued; ++kc)
+          mbar_wait(bar(B_FULL + kc % STAGES), (kc / STAGES) & 1, abort, true);
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
-    if (lane == 0) {
-      const uint32_t idesc = bf16x3 ? make_idesc_bf16(NL) : make_idesc(NL);
+    if (lane == 0 && !leader) {
+      // CTA 1 of a pair: CTA 0's MMAs write this CTA's TMEM; wait for them
+      mbar_wait(bar(B_DRAIN), 0, abort, true);
+    } else if (lane == 0) {
+      const uint32_t idesc = bf16x3 ? make_idesc_bf16(NL, pair ? 2 * BM : BM) : make_idesc(NL);
       for (int kc = 0; kc < KC; ++kc) {
         const int s = kc % STAGES;
         const int j = kc / kPromote, b = j & 1;
@@ -435,12 +555,23 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t ko = kk * 32;  // 16 bf16 = 32 bytes along K
             const uint64_t da = make_desc_sw64(a + ko);
 #pragma unroll
-            for (int pl = 0; pl < 3; ++pl)
-              mma_bf16(d_tmem, da, make_desc_sw64(a + plan.a_bytes + pl * plan.b_bytes + ko),
-                       idesc, (!first || kk > 0 || pl > 0) ? 1u : 0u);
+            for (int pl = 0; pl < 3; ++pl) {
+              const uint64_t db = make_desc_sw64(a + plan.a_bytes + pl * plan.b_bytes + ko);
+              const uint32_t acc = (!first || kk > 0 || pl > 0) ? 1u : 0u;
+              if constexpr (PAIR)
+                mma_bf16_pair(d_tmem, da, db, idesc, acc);
+              else
+                mma_bf16(d_tmem, da, db, idesc, acc);
+            }
           }
-          mma_commit(bar(B_EMPTY + s));
-          if ((kc % kPromote) == kPromote - 1 || kc == KC - 1) mma_commit(bar(B_ACCF + b));
+          const bool iv_end = (kc % kPromote) == kPromote - 1 || kc == KC - 1;
+          if constexpr (PAIR) {
+            mma_commit_pair(bar(B_EMPTY + s));
+            if (iv_end) mma_commit_pair(bar(B_ACCF + b));
+          } else {
+            mma_commit(bar(B_EMPTY + s));
+            if (iv_end) mma_commit(bar(B_ACCF + b));
+          }
           continue;
         }
         const uint32_t a_hi = smem0 + s * plan.stage_bytes;
@@ -468,7 +599,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if ((kc % kPromote) == kPromote - 1 || kc == KC - 1) mma_commit(bar(B_ACCF + b));
       }
       // Track every MMA issued so far; waited on before TMEM is released.
-      mma_commit(bar(B_DRAIN));
+      if constexpr (PAIR)
+        mma_commit_pair(bar(B_DRAIN));
+      else
+        mma_commit(bar(B_DRAIN));
       mbar_wait(bar(B_DRAIN), 0, abort, true);
     }
   } else {
@@ -504,7 +638,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(bar(B_ACCE + b));
+      if (PAIR && !leader)
+        mbar_arrive_cluster(cluster_addr(bar(B_ACCE + b), 0));
+      else
+        mbar_arrive(bar(B_ACCE + b));
       ++promoted;
     };
 
@@ -631,12 +768,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 a2 = -INFINITY;
               }
               const float cval = v[i] + bv[i];
-              if (cval > a1) {
-                a2 = a1;
-                a1 = cval;
-              } else if (cval > a2) {
-                a2 = cval;
-              }
+              a2 = fmaxf(a2, fminf(a1, cval));  // top-2 of the values seen
+              a1 = fmaxf(a1, cval);
             }
           }
           asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
@@ -690,15 +823,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
 
-      // pass 2: top-8 of this half's masked scores
+      // pass 2: top-8 of this half's masked scores.  Per chunk, the 16
+      // candidate scores are formed branch-free and only those beating the
+      // current 8th enter a compact insertion loop; they are staged in shared
+      // memory (idle stage ring) so the loop can index them.
       Top8 top;
       top.init();
       if (ok && c_beg < c_end) {
         const bool zero_fill = (G > 1) && (P.mask_mode == MR_MASK_ZERO);
+        float* scrC = reinterpret_cast<float*>(smem + exchange_bytes(G));  // [16][256]
+        float* scrS = scrC + 16 * 32 * kWorkers;                            // [16][256]
         int g = (col0 + c_beg * 16) / S, next_b = (g + 1) * S;
         for (int c = c_beg; c < c_end; ++c) {
           tmem_ld16(tmem_base + lane_off + (uint32_t)(c * 16), v);
           load_bias(c);
+          const float thr = top.v[kTopMax - 1];
+          uint32_t m = 0;
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             const int e = col0 + c * 16 + i;
@@ -708,12 +848,24 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             const bool keep = G == 1 || ((kept >> g) & 1u);
             // with groups, pass 1 left s in TMEM; otherwise v holds logits
-            if (keep) {
-              const float sv = G > 1 ? v[i] : mr_sigmoid(v[i]);
-              const float cval = sv + bv[i];
-              if (cval > top.v[kTopMax - 1]) top.push(cval, e, sv);
-            } else if (zero_fill && 0.0f > top.v[kTopMax - 1]) {
-              top.push(0.0f, e, v[i]);
+            const float sv = G > 1 ? v[i] : mr_sigmoid(v[i]);
+            const float cval = keep ? sv + bv[i] : (zero_fill ? 0.0f : -INFINITY);
+            v[i] = sv;
+            bv[i] = cval;
+            m |= (cval > thr ? 1u : 0u) << i;
+          }
+          if (m) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              scrC[i * 32 * kWorkers + wt] = bv[i];
+              scrS[i * 32 * kWorkers + wt] = v[i];
+            }
+            while (m) {
+              const int i = __ffs(m) - 1;
+              m &= m - 1;
+              const float cval = scrC[i * 32 * kWorkers + wt];
+              if (cval > top.v[kTopMax - 1])
+                top.push(cval, col0 + c * 16 + i, scrS[i * 32 * kWorkers + wt]);
             }
           }
         }
@@ -726,40 +878,29 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       workers_sync();
       if (cs > 1) cluster_sync_all();  // #2: top-8 lists visible to the peer
-      if (h == 0 && crank == 0) {
-        // merge the other half's list, then the peer CTA's two lists
+      if (h == 0 && (PAIR || crank == 0)) {
+        // merge the other half's list, then (experts split over the cluster)
+        // the peer CTA's two lists; a pair's CTAs each own their tokens
 #pragma unroll 1
         for (int src = 1; src < 4; ++src) {
           if (src >= 2 && cs == 1) break;
           const int hh = src & 1;
+          float pv[kTopMax], ps[kTopMax];
+          int pi[kTopMax];
 #pragma unroll
           for (int j = 0; j < kTopMax; ++j) {
             const int o = (hh * kTopMax + j) * BM + row;
-            float pv, ps;
-            int pi;
             if (src < 2) {
-              pv = exV[o];
-              ps = exS[o];
-              pi = exI[o];
+              pv[j] = exV[o];
+              ps[j] = exS[o];
+              pi[j] = exI[o];
             } else {
-              pv = ld_peer_f32(&exV[o], 1u);
-              ps = ld_peer_f32(&exS[o], 1u);
-              pi = __float_as_int(ld_peer_f32(reinterpret_cast<float*>(&exI[o]), 1u));
-            }
-            if (mr_better(pv, pi, top.v[kTopMax - 1], top.i[kTopMax - 1])) {
-              top.v[kTopMax - 1] = pv;
-              top.s[kTopMax - 1] = ps;
-              top.i[kTopMax - 1] = pi;
-#pragma unroll
-              for (int t = kTopMax - 1; t > 0; --t) {
-                if (mr_better(top.v[t], top.i[t], top.v[t - 1], top.i[t - 1])) {
-                  const float tv = top.v[t]; top.v[t] = top.v[t - 1]; top.v[t - 1] = tv;
-                  const float ts = top.s[t]; top.s[t] = top.s[t - 1]; top.s[t - 1] = ts;
-                  const int ti = top.i[t]; top.i[t] = top.i[t - 1]; top.i[t - 1] = ti;
-                }
-              }
+              pv[j] = ld_peer_f32(&exV[o], 1u);
+              ps[j] = ld_peer_f32(&exS[o], 1u);
+              pi[j] = __float_as_int(ld_peer_f32(reinterpret_cast<float*>(&exI[o]), 1u));
             }
           }
+          top.merge(pv, ps, pi);
         }
         if (ok && tok < P.T) {
           float den = 0.0f;
@@ -789,12 +930,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
+  // pair: neither CTA leaves while the other may still read its shared memory
+  // (CTA 0's MMAs read CTA 1's tiles), arrive on its barriers or copy into it
+  if (pair) cluster_sync_all();
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
-                 "r"(tmem_cols)
-                 : "memory");
+    if constexpr (PAIR)
+      asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                   "r"(tmem_cols)
+                   : "memory");
+    else
+      asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                   "r"(tmem_cols)
+                   : "memory");
   }
 }
 
