@@ -119,8 +119,11 @@ __host__ __device__ inline Plan make_plan(int NL, bool bf16x3 = false, bool pair
 __host__ __device__ inline uint32_t exchange_bytes(int G) {
   return 4u * 2u * (2u * G * BM + 3u * kTopMax * BM);
 }
+// Per-thread candidate buffer of the top-k scan (value, score, index):
+// kCandCap slots plus one slot that absorbs the stores of non-candidates.
+constexpr int kCandCap = 16;
 __host__ __device__ inline uint32_t epilogue_smem_bytes(int G) {
-  return exchange_bytes(G) + 4u * 2u * 16u * 32u * kWorkers;
+  return exchange_bytes(G) + 4u * 3u * (kCandCap + 1) * 32u * kWorkers;
 }
 
 // ---- PTX wrappers ----------------------------------------------------------
@@ -336,6 +339,33 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// Two 16-column loads (columns at ta and tb) and their wait in one asm
+// statement, so one TMEM round trip serves 32 columns and no output register
+// is visible to the compiler before the data has arrived.
+__device__ __forceinline__ void tmem_ld16x2(uint32_t ta, uint32_t tb, float (&va)[16],
+                                            float (&vb)[16]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%32];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%33];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+        "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+        "=r"(r[31])
+      : "r"(ta), "r"(tb)
+      : "memory");
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    va[i] = __uint_as_float(r[i]);
+    vb[i] = __uint_as_float(r[16 + i]);
+  }
+}
+
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
@@ -406,6 +436,65 @@ struct Top8 {
     }
   }
 };
+
+// Group choice of one token (one thread): the group score is the sum of the
+// two best biased scores of the group, over the top-2 pairs that this CTA's
+// two column halves (and, with CS = 2, the peer CTA's) left in exA1/exA2
+// [half][group][row]; the topk_group best groups are kept (lower index first
+// on ties), by counting for each group how many groups beat it.  tau: the
+// smallest second-best score of the kept groups when 2*topk_group >= k.
+template <int MAXG>
+__device__ __forceinline__ void select_groups(int G, int topk_group, int k, int cs, uint32_t crank,
+                                              const float* exA1, const float* exA2, int row,
+                                              uint32_t& kept, float& tau) {
+  float ga1[MAXG], ga2[MAXG];
+#pragma unroll
+  for (int g = 0; g < MAXG; ++g) {
+    float a1 = -INFINITY, a2 = -INFINITY;
+    if (g < G) {
+#pragma unroll
+      for (int src = 0; src < 4; ++src) {
+        if (src >= 2 && cs == 1) break;
+        const int hh = src & 1;
+        float b1, b2;
+        if (src < 2) {
+          b1 = exA1[(hh * G + g) * BM + row];
+          b2 = exA2[(hh * G + g) * BM + row];
+        } else {
+          b1 = ld_peer_f32(&exA1[(hh * G + g) * BM + row], crank ^ 1u);
+          b2 = ld_peer_f32(&exA2[(hh * G + g) * BM + row], crank ^ 1u);
+        }
+        // top-2 of the union of two top-2 pairs
+        const float hi = fmaxf(a1, b1);
+        a2 = fmaxf(fminf(a1, b1), fmaxf(a2, b2));
+        a1 = hi;
+      }
+    }
+    ga1[g] = a1;
+    ga2[g] = a2;
+  }
+  kept = 0;
+  float t = INFINITY;
+#pragma unroll
+  for (int g = 0; g < MAXG; ++g) {
+    if (g < G) {
+      const float sg = ga1[g] + ga2[g];
+      int rank = 0;
+#pragma unroll
+      for (int o = 0; o < MAXG; ++o) {
+        if (o < G && o != g) {
+          const float so = ga1[o] + ga2[o];
+          rank += (so > sg || (so == sg && o < g)) ? 1 : 0;
+        }
+      }
+      if (rank < topk_group) {
+        kept |= 1u << g;
+        t = fminf(t, ga2[g]);
+      }
+    }
+  }
+  tau = (2 * topk_group >= k) ? t : -INFINITY;
+}
 
 template <bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -717,7 +806,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       float* exV = exA2 + 2 * G * BM;                            // [2][8][BM]
       float* exS = exV + 2 * kTopMax * BM;                       // [2][8][BM]
       int* exI = reinterpret_cast<int*>(exS + 2 * kTopMax * BM); // [2][8][BM]
-      float v[16], bv[16];
+      float v[16], v2[16], bv[16];
       auto load_bias = [&](int c) {
         const float4* b4 = reinterpret_cast<const float4*>(bias_s + c * 16);
 #pragma unroll
@@ -732,6 +821,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
       if (ok && P.logits_out) {
         for (int c = c_beg; c < c_end; ++c) {
+          __syncwarp();
           tmem_ld16(tmem_base + lane_off + (uint32_t)(c * 16), v);  // whole warp
           if (tok < P.T)
 #pragma unroll
@@ -749,13 +839,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok && c_beg < c_end) {
           float a1 = -INFINITY, a2 = -INFINITY;
           int g = (col0 + c_beg * 16) / S, next_b = (g + 1) * S;
-          for (int c = c_beg; c < c_end; ++c) {
-            const uint32_t ta = tmem_base + lane_off + (uint32_t)(c * 16);
-            tmem_ld16(ta, v);
+          auto body1 = [&](int c, float(&x)[16]) {
             load_bias(c);
 #pragma unroll
-            for (int i = 0; i < 16; ++i) v[i] = mr_sigmoid(v[i]);
-            tmem_st16(ta, v);
+            for (int i = 0; i < 16; ++i) x[i] = mr_sigmoid(x[i]);
+            tmem_st16(tmem_base + lane_off + (uint32_t)(c * 16), x);
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
               const int e = col0 + c * 16 + i;
@@ -767,10 +855,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                 a1 = -INFINITY;
                 a2 = -INFINITY;
               }
-              const float cval = v[i] + bv[i];
+              const float cval = x[i] + bv[i];
               a2 = fmaxf(a2, fminf(a1, cval));  // top-2 of the values seen
               a1 = fmaxf(a1, cval);
             }
+          };
+          // two chunks per TMEM round trip (the second load of an odd tail
+          // re-reads the first chunk and is ignored)
+          for (int c = c_beg; c < c_end; c += 2) {
+            const int c2 = c + 1 < c_end ? c + 1 : c;
+            tmem_ld16x2(tmem_base + lane_off + (uint32_t)(c * 16),
+                        tmem_base + lane_off + (uint32_t)(c2 * 16), v, v2);
+            body1(c, v);
+            if (c2 != c) body1(c2, v2);
           }
           asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
           exA1[(h * G + g) * BM + row] = a1;
@@ -779,63 +876,42 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       workers_sync();
       if (cs > 1) cluster_sync_all();  // #1: group pairs visible to the peer
+      // Group choice from the merged per-group top-2 pairs, and a lower
+      // bound tau on the k-th best masked score: the kept groups' top-2
+      // values are 2*topk_group distinct candidates, so when that is >= k
+      // the k-th best of all candidates is >= the smallest of them.
+      float tau = -INFINITY;
       if (G > 1) {
-        float gs[kMaxGroups];
-#pragma unroll
-        for (int g = 0; g < kMaxGroups; ++g) {
-          if (g < G) {
-            // top-2 of the union of the halves' (and the peer's) pairs
-            float a1 = -INFINITY, a2 = -INFINITY;
-#pragma unroll
-            for (int src = 0; src < 4; ++src) {
-              if (src >= 2 && cs == 1) break;
-              const int hh = src & 1;
-              float b1, b2;
-              if (src < 2) {
-                b1 = exA1[(hh * G + g) * BM + row];
-                b2 = exA2[(hh * G + g) * BM + row];
-              } else {
-                b1 = ld_peer_f32(&exA1[(hh * G + g) * BM + row], crank ^ 1u);
-                b2 = ld_peer_f32(&exA2[(hh * G + g) * BM + row], crank ^ 1u);
-              }
-              if (a1 >= b1) {
-                a2 = fmaxf(a2, b1);
-              } else {
-                a2 = fmaxf(a1, b2);
-                a1 = b1;
-              }
-            }
-            gs[g] = a1 + a2;
-          }
-        }
-        kept = 0;
-        for (int r = 0; r < P.topk_group; ++r) {
-          float bv2 = -INFINITY;
-          int bg = -1;
-#pragma unroll
-          for (int g = 0; g < kMaxGroups; ++g) {
-            if (g < G && !((kept >> g) & 1u) && (bg < 0 || gs[g] > bv2)) {
-              bv2 = gs[g];
-              bg = g;
-            }
-          }
-          kept |= 1u << bg;
-        }
+        if (G <= 8)
+          select_groups<8>(G, P.topk_group, P.k, cs, crank, exA1, exA2, row, kept, tau);
+        else
+          select_groups<kMaxGroups>(G, P.topk_group, P.k, cs, crank, exA1, exA2, row, kept, tau);
       }
 
-      // pass 2: top-8 of this half's masked scores.  Per chunk, the 16
-      // candidate scores are formed branch-free and only those beating the
-      // current 8th enter a compact insertion loop; they are staged in shared
-      // memory (idle stage ring) so the loop can index them.
+      // pass 2: top-8 of this half's masked scores.  A score enters only if
+      // it is >= tau and beats the list's current 8th; such candidates are
+      // appended (in index order) to this thread's buffer in shared memory
+      // and inserted into the sorted list when the buffer fills and at the
+      // end, so the serial insertion runs ~k times per token, not once per
+      // score that beats a running threshold.
       Top8 top;
       top.init();
       if (ok && c_beg < c_end) {
         const bool zero_fill = (G > 1) && (P.mask_mode == MR_MASK_ZERO);
-        float* scrC = reinterpret_cast<float*>(smem + exchange_bytes(G));  // [16][256]
-        float* scrS = scrC + 16 * 32 * kWorkers;                            // [16][256]
+        float* bufV = reinterpret_cast<float*>(smem + exchange_bytes(G));  // [kCandCap][256]
+        float* bufS = bufV + (kCandCap + 1) * 32 * kWorkers;
+        int* bufI = reinterpret_cast<int*>(bufS + (kCandCap + 1) * 32 * kWorkers);
+        int cnt = 0;
+        auto flush = [&]() {
+          for (int j = 0; j < cnt; ++j) {
+            const float cv = bufV[j * 32 * kWorkers + wt];
+            if (cv > top.v[kTopMax - 1])
+              top.push(cv, bufI[j * 32 * kWorkers + wt], bufS[j * 32 * kWorkers + wt]);
+          }
+          cnt = 0;
+        };
         int g = (col0 + c_beg * 16) / S, next_b = (g + 1) * S;
-        for (int c = c_beg; c < c_end; ++c) {
-          tmem_ld16(tmem_base + lane_off + (uint32_t)(c * 16), v);
+        auto body2 = [&](int c, float(&x)[16]) {
           load_bias(c);
           const float thr = top.v[kTopMax - 1];
           uint32_t m = 0;
@@ -847,28 +923,37 @@ __global__ void __launch_bounds__(kThreads, 1)
               next_b += S;
             }
             const bool keep = G == 1 || ((kept >> g) & 1u);
-            // with groups, pass 1 left s in TMEM; otherwise v holds logits
-            const float sv = G > 1 ? v[i] : mr_sigmoid(v[i]);
+            // with groups, pass 1 left s in TMEM; otherwise x holds logits
+            const float sv = G > 1 ? x[i] : mr_sigmoid(x[i]);
             const float cval = keep ? sv + bv[i] : (zero_fill ? 0.0f : -INFINITY);
-            v[i] = sv;
+            x[i] = sv;
             bv[i] = cval;
-            m |= (cval > thr ? 1u : 0u) << i;
+            m |= (cval >= tau && cval > thr ? 1u : 0u) << i;
           }
-          if (m) {
+          if (cnt + __popc(m) > kCandCap) flush();
+          // branch-free append in index order; non-candidates write the
+          // spare slot kCandCap
+          int p = cnt;
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              scrC[i * 32 * kWorkers + wt] = bv[i];
-              scrS[i * 32 * kWorkers + wt] = v[i];
-            }
-            while (m) {
-              const int i = __ffs(m) - 1;
-              m &= m - 1;
-              const float cval = scrC[i * 32 * kWorkers + wt];
-              if (cval > top.v[kTopMax - 1])
-                top.push(cval, col0 + c * 16 + i, scrS[i * 32 * kWorkers + wt]);
-            }
+          for (int i = 0; i < 16; ++i) {
+            const bool bit = (m >> i) & 1u;
+            const int slot = (bit ? p : kCandCap) * 32 * kWorkers + wt;
+            bufV[slot] = bv[i];
+            bufS[slot] = x[i];
+            bufI[slot] = col0 + c * 16 + i;
+            p += bit ? 1 : 0;
           }
+          cnt = p;
+        };
+        for (int c = c_beg; c < c_end; c += 2) {
+          __syncwarp();  // the buffer flush diverges; tcgen05.ld is .aligned
+          const int c2 = c + 1 < c_end ? c + 1 : c;
+          tmem_ld16x2(tmem_base + lane_off + (uint32_t)(c * 16),
+                      tmem_base + lane_off + (uint32_t)(c2 * 16), v, v2);
+          body2(c, v);
+          if (c2 != c) body2(c2, v2);
         }
+        flush();
       }
 #pragma unroll
       for (int j = 0; j < kTopMax; ++j) {
