@@ -29,6 +29,11 @@ SMALL = [
       mask_mode=0, seed=17, io_dtype="f32"),
     W("N320_G10_T140", T=140, d=300, N_r=320, n_group=10, topk_group=3, k=5,
       route_scale=2.5, mask_mode=1, seed=18, io_dtype="f32"),
+    # every biased score < 0 = the masked groups' fill: the top-k is mostly
+    # masked experts (ties at 0.0 resolved by index), and the kept groups'
+    # top-2 bound lies below every candidate
+    W("zero_mask_all_negative_T200", T=200, d=256, N_r=256, n_group=8, topk_group=4, k=8,
+      route_scale=2.5, mask_mode=1, seed=19, bias_lo=-1.5, bias_hi=-1.1, io_dtype="f32"),
 ]
 FULL = [wl.V3_PREFILL, wl.K2_PREFILL, wl.V3_DECODE, wl.V3_FULL]
 
@@ -250,6 +255,8 @@ BF16X3 = [
       route_scale=2.5, mask_mode=1, seed=32, bias_lo=-0.8, bias_hi=-0.2),
     W("bf16x3_no_bias_T129", T=129, d=256, N_r=64, n_group=8, topk_group=3, k=6,
       route_scale=1.0, mask_mode=0, seed=33, with_bias=False),
+    W("bf16x3_zero_mask_all_negative_T300", T=300, d=512, N_r=256, n_group=8, topk_group=4,
+      k=8, route_scale=2.5, mask_mode=1, seed=34, bias_lo=-1.5, bias_hi=-1.1),
 ]
 
 

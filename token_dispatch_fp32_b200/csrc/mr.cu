@@ -242,8 +242,11 @@ int launch_splitk(const float* x, const float* W, const float* bias, int T, int 
 //  - CS = 2 splits the experts over a 2-CTA cluster: always when N_r > 256
 //    (TMEM holds two accumulation buffers of at most 256 columns), and when
 //    it at least doubles the CTA count of a small batch;
-//  - pair: bf16x3 with N_r <= 256 on large batches; two CTAs run one M = 256
-//    MMA over consecutive tiles and each stages half of W.
+//  - otherwise one CTA per tile.
+// pair (bf16x3, N_r <= 256): two CTAs run one M = 256 MMA over consecutive
+// tiles and each stages half of W.  It is only taken when pinned: on the
+// full DeepSeek-V3 batch (T = 16384) it measured 5 us slower than one CTA
+// per tile (188 vs 182 us).
 // MR_TC_CLUSTER = 1, 2 or P pins the choice (used by the tests to cover each).
 struct TcShape {
   int CS;
@@ -260,7 +263,6 @@ TcShape tc_shape(int T, int N_r, int sms, bool bf16x3) {
   }
   const int tiles = (T + mr::tc::BM - 1) / mr::tc::BM;
   if (N_r % 32 == 0 && 2 * tiles <= sms) return {2, false};
-  if (pair_ok && tiles >= 2) return {1, true};
   return {1, false};
 }
 

@@ -542,8 +542,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(bar(B_ACCF + 0), 1);
     mbar_init(bar(B_ACCF + 1), 1);
-    mbar_init(bar(B_ACCE + 0), (pair ? 2 : 1) * 32 * kWorkers);  // both CTAs' workers
-    mbar_init(bar(B_ACCE + 1), (pair ? 2 : 1) * 32 * kWorkers);
+    // one arrival per worker warp (of both CTAs in a pair)
+    mbar_init(bar(B_ACCE + 0), (pair ? 2 : 1) * kWorkers);
+    mbar_init(bar(B_ACCE + 1), (pair ? 2 : 1) * kWorkers);
     mbar_init(bar(B_DRAIN), 1);
     *abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -716,21 +717,37 @@ __global__ void __launch_bounds__(kThreads, 1)
         return;
       }
       tc_fence_after();
+      // chunks h, h+2, ..., two per TMEM round trip
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
+      for (int i = 0; i < 8; i += 2) {
         const int c = h + 2 * i;
-        if (c < n16) {
-          float v[16];
-          tmem_ld16(tmem_base + lane_off + (uint32_t)(b * NL + c * 16), v);
+        if (c + 2 < n16) {
+          float v0[16], v1[16];
+          tmem_ld16x2(tmem_base + lane_off + (uint32_t)(b * NL + c * 16),
+                      tmem_base + lane_off + (uint32_t)(b * NL + (c + 2) * 16), v0, v1);
 #pragma unroll
-          for (int e = 0; e < 16; ++e) acc[i][e] += v[e];
+          for (int e = 0; e < 16; ++e) {
+            acc[i][e] += v0[e];
+            acc[i + 1][e] += v1[e];
+          }
+        } else if (c < n16) {
+          float v0[16];
+          tmem_ld16(tmem_base + lane_off + (uint32_t)(b * NL + c * 16), v0);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) acc[i][e] += v0[e];
         }
       }
+      // Every lane's loads have completed (tcgen05.wait::ld); one elected
+      // arrival per warp releases the buffer to the MMA issuer (a pair's
+      // CTA 1 arrives on CTA 0's barrier, a cluster-scope release).
       tc_fence_before();
-      if (PAIR && !leader)
-        mbar_arrive_cluster(cluster_addr(bar(B_ACCE + b), 0));
-      else
-        mbar_arrive(bar(B_ACCE + b));
+      __syncwarp();
+      if (lane == 0) {
+        if (PAIR && !leader)
+          mbar_arrive_cluster(cluster_addr(bar(B_ACCE + b), 0));
+        else
+          mbar_arrive(bar(B_ACCE + b));
+      }
       ++promoted;
     };
 
