@@ -350,6 +350,46 @@ def run_ours(args, w: wl.Workload, rank: int, world: int):
 
     ms_max = max_over_ranks(ms, world, dev)
 
+    # The decode-size router (one position x batch 64), timed alone: W read
+    # once per call by the split-K kernel over all SMs, then reduce-and-route.
+    decode = None
+    if args.workload == wl.V3_FULL.name:
+        wd = wl.V3_DECODE
+        dd_in = wl.gen_router_inputs(wd)
+        dx = torch.from_numpy(dd_in["x_bf16"]).view(torch.bfloat16).to(dev)
+        dW = torch.from_numpy(dd_in["W"]).to(dev)
+        db = torch.from_numpy(dd_in["b"]).to(dev)
+        didx = torch.empty((wd.T, wd.k), dtype=torch.int32, device=dev)
+        dwt = torch.empty((wd.T, wd.k), dtype=torch.float32, device=dev)
+        dws = torch.empty(max(4, mr.mr_router_workspace_size(wd.T, wd.d, wd.N_r)),
+                          dtype=torch.uint8, device=dev)
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)  # > L2
+
+        def dstep():
+            mr.mr_router_forward_ex(dx, dW, db, wd.n_group, wd.topk_group, wd.k, wd.route_scale,
+                                    wd.mask_mode, precision=mr.MR_PREC_BF16X3, idx_out=didx,
+                                    w_out=dwt, workspace=dws, stream=stream)
+
+        for _ in range(5):
+            dstep()
+        n_dec = 100
+        tot = 0.0
+        for _ in range(n_dec):  # W comes from HBM every call: L2 flushed between calls
+            with torch.cuda.stream(stream):
+                flush.fill_(1)
+            d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            d0.record(stream)
+            dstep()
+            d1.record(stream)
+            d1.synchronize()
+            tot += d0.elapsed_time(d1)
+        dus = tot / n_dec * 1e3
+        dbytes = 4 * wd.N_r * wd.d + 2 * wd.T * wd.d + 4 * wd.N_r + 8 * wd.T * wd.k
+        decode = {"workload": wd.name, "us": dus, "launches_per_call": 2,
+                  "algorithmic_bytes": dbytes, "gbs": dbytes / (dus * 1e-6) / 1e9,
+                  "l2": "flushed before every call (256 MB write)"}
+        assert mr.mr_get_error(stream) == mr.MR_OK
+
     # ---- end to end: pinned host inputs -> device -> path -> host result ----
     e2e = None
     if not args.no_e2e:
@@ -432,6 +472,9 @@ def run_ours(args, w: wl.Workload, rank: int, world: int):
         "combine": {"ms": stage_ms["combine"], "gbs": achieved,
                     "frac_hbm": achieved / peaks["hbm_gbs"]},
     }
+    if decode is not None:
+        decode["frac_hbm"] = decode["gbs"] / peaks["hbm_gbs"]
+        stages["decode_router"] = decode
     line = {
         "metric": METRIC, "value": aggregate_tokens_per_s(world, T, ms_max), "unit": UNIT,
         "n_gpus": world,

@@ -170,30 +170,46 @@ SPLITK = [
 ]
 
 
-@pytest.mark.parametrize("w", SPLITK, ids=[w.name for w in SPLITK])
-def test_router_splitk_small_batches(w):
+SPLITK_CASES = [(w, "f32") for w in SPLITK] + [(w, "bf16") for w in SPLITK
+                                                if w.io_dtype == "bf16"]
+
+
+@pytest.mark.parametrize("w,rows", SPLITK_CASES, ids=[f"{w.name}-{r}" for w, r in SPLITK_CASES])
+def test_router_splitk_small_batches(w, rows):
     """Batches of up to 256 tokens with a workspace take the split-K path
-    (K-sliced tensor-core GEMM over all SMs + reduce-and-route)."""
+    (K-sliced tensor-core GEMM over all SMs, cluster reduction, reduce-and-
+    route), for fp32 rows and for bf16 rows (staged as bf16, widened in
+    shared memory).  d = 7168 and 1000 reduce the K slices in clusters of 8;
+    d = 516 has too few K chunks for that and writes every slice."""
     n = mr.mr_router_workspace_size(w.T, w.d, w.N_r)
     assert n > 0
     d = router_inputs(w)
+    x = to_dev(d["x_bf16"], "bf16") if rows == "bf16" else to_dev(d["x_f32"])
     ws = torch.empty(n, dtype=torch.uint8, device="cuda")
     logits = torch.full((w.T, w.N_r), float("nan"), device="cuda")
     io, wo = _poisoned(w.T, w.k)
     l0 = mr.mr_launch_count()
-    idx, wt = mr.mr_router_forward_ex(to_dev(d["x_f32"]), to_dev(d["W"]), to_dev(d["b"]),
+    idx, wt = mr.mr_router_forward_ex(x, to_dev(d["W"]), to_dev(d["b"]),
                                       w.n_group, w.topk_group, w.k, w.route_scale, w.mask_mode,
                                       idx_out=io, w_out=wo, logits_out=logits, workspace=ws)
     assert mr.mr_launch_count() - l0 == 2  # GEMM + reduce/route
     assert mr.mr_get_error() == mr.MR_OK
     ref = oracle_router(w, np.arange(w.T))
     stats = compare_router(idx.cpu().numpy(), wt.cpu().numpy(), ref, logits.cpu().numpy())
-    print(w.name, stats)
+    print(w.name, rows, stats)
     # deterministic: slices are summed in a fixed order
-    idx2, wt2 = mr.mr_router_forward_ex(to_dev(d["x_f32"]), to_dev(d["W"]), to_dev(d["b"]),
+    idx2, wt2 = mr.mr_router_forward_ex(x, to_dev(d["W"]), to_dev(d["b"]),
                                         w.n_group, w.topk_group, w.k, w.route_scale,
                                         w.mask_mode, workspace=ws)
     assert torch.equal(idx, idx2) and torch.equal(wt, wt2)
+    if rows == "bf16":
+        # the same logits as the fp32 cast of the rows, bit for bit: both
+        # stage the same fp32 values and a bf16 row has no tf32 residual
+        lf = torch.full_like(logits, float("nan"))
+        mr.mr_router_forward_ex(to_dev(d["x_f32"]), to_dev(d["W"]), to_dev(d["b"]), w.n_group,
+                                w.topk_group, w.k, w.route_scale, w.mask_mode,
+                                logits_out=lf, workspace=ws)
+        assert torch.equal(lf, logits)
 
 
 def test_router_workspace_for_large_batches_holds_w_planes():
@@ -285,11 +301,11 @@ def test_router_bf16x3_small_all_tokens(w):
 
 
 @pytest.mark.parametrize("cs", ["1", "2", "P"])
-@pytest.mark.parametrize("w", [SMALL[1], BF16X3[4]], ids=lambda w: w.name)
+@pytest.mark.parametrize("w", [SMALL[1], BF16X3[5]], ids=lambda w: w.name)
 def test_router_bf16x3_cluster_size_pinned(w, cs, monkeypatch):
     """Every way the bf16x3 kernel can cover a tile: one CTA, two CTAs
     splitting the experts, or a 2-SM pair running one M = 256 MMA (T = 300
-    and 129 give an odd tile count, so a pair's second tile lies past T)."""
+    gives an odd tile count, so a pair's second tile lies past T)."""
     monkeypatch.setenv("MR_TC_CLUSTER", cs)
     idx, wt, logits = _run_bf16x3(w)
     compare_router(idx, wt, oracle_router(w, np.arange(w.T)), logits)

@@ -70,7 +70,7 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 
 // Row-major bf16 matrix [rows, cols], box [box_rows, 32] (64-byte rows, 64-byte swizzle).
 bool make_map_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
-                   uint32_t box_rows) {
+                   uint32_t box_rows, bool swizzle = true) {
   auto enc = tensor_map_encoder();
   if (!enc) return false;
   const cuuint64_t dims[2] = {cols, rows};
@@ -78,7 +78,8 @@ bool make_map_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t c
   const cuuint32_t box[2] = {32, box_rows};
   const cuuint32_t estr[2] = {1, 1};
   return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
-             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             swizzle ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_NONE,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -167,11 +168,51 @@ int launch_ffma(const void* x, const float* W, const float* bias, int T, int d, 
 constexpr int kSplitKMaxT = 256;  // batches up to one MMA N of tokens
 
 struct SplitKShape {
-  int NT, TT, MT, KC, KS;
+  int NT, TT, MT, KC, KS, CL;
   size_t ws_bytes;
 };
 
-SplitKShape splitk_shape(int T, int d, int N_r, int sms) {
+// Clusters of kCluster split-K CTAs that fit on the device at once (a cluster
+// must sit inside one GPC, so fewer than sms / kCluster may); 0 if unknown.
+int splitk_max_clusters(size_t smem) {
+  static std::mutex mu;
+  static int cache_dev[16], cache_n[16];
+  static size_t cache_smem[16];
+  static int used = 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  std::lock_guard<std::mutex> lock(mu);
+  for (int i = 0; i < used; ++i)
+    if (cache_dev[i] == dev && cache_smem[i] == smem) return cache_n[i];
+  if (cudaFuncSetAttribute(mr::sk::router_splitk_gemm_kernel,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return 0;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(mr::sk::kCluster);
+  cfg.blockDim = dim3(mr::sk::kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = mr::sk::kCluster;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, mr::sk::router_splitk_gemm_kernel, &cfg) != cudaSuccess) {
+    (void)cudaGetLastError();
+    n = 0;
+  }
+  if (used < 16) {
+    cache_dev[used] = dev;
+    cache_smem[used] = smem;
+    cache_n[used] = n;
+    ++used;
+  }
+  return n;
+}
+
+SplitKShape splitk_shape(int T, int d, int N_r, int sms, bool x_bf16) {
   SplitKShape k;
   k.NT = ((T + 15) / 16) * 16;
   if (k.NT > mr::sk::kMaxNT) k.NT = mr::sk::kMaxNT;
@@ -181,8 +222,21 @@ SplitKShape splitk_shape(int T, int d, int N_r, int sms) {
   int ks = sms / (k.MT * k.TT);
   if (ks < 1) ks = 1;
   if (ks > k.KC) ks = k.KC;
+  // slices reduced in clusters of kCluster through distributed shared memory
+  k.CL = 1;
+  if (ks >= 2 * mr::sk::kCluster) {
+    // as many clusters as fit at once (one wave), kCluster slices each
+    const mr::sk::Plan pl = mr::sk::make_plan(k.NT, (k.KC + ks - 1) / ks, x_bf16);
+    int per_tile = ks / mr::sk::kCluster;
+    const int fit = splitk_max_clusters(pl.total + 1024);
+    if (fit > 0 && per_tile * k.MT * k.TT > fit) per_tile = fit / (k.MT * k.TT);
+    if (per_tile >= 2) {
+      ks = per_tile * mr::sk::kCluster;
+      k.CL = mr::sk::kCluster;
+    }
+  }
   k.KS = ks;
-  k.ws_bytes = (size_t)k.KS * (size_t)T * (size_t)N_r * sizeof(float);
+  k.ws_bytes = (size_t)(k.KS / k.CL) * (size_t)T * (size_t)N_r * sizeof(float);
   return k;
 }
 
@@ -192,42 +246,83 @@ template <int NJ>
 int launch_reduce_nj(const float* part, int KS, int T, int N_r, const float* bias, int n_group,
                      int topk_group, int k, float route_scale, int mask_mode, int32_t* idx_out,
                      float* w_out, float* logits_out, cudaStream_t st) {
-  mr::sk::router_reduce_route_kernel<NJ><<<T, 256, 0, st>>>(part, KS, T, N_r, bias, n_group,
-                                                             topk_group, k, route_scale,
-                                                             mask_mode, idx_out, w_out,
-                                                             logits_out);
-  return launch_status();
+  // programmatic dependent of the GEMM: launched while the GEMM drains, it
+  // waits (griddepcontrol.wait) for the GEMM's results before reading them
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)T);
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, mr::sk::router_reduce_route_kernel<NJ>, part, KS,
+                                           T, N_r, bias, n_group, topk_group, k, route_scale,
+                                           mask_mode, idx_out, w_out, logits_out);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  if (e != cudaSuccess) {
+    (void)cudaGetLastError();
+    return MR_ERR_CUDA;
+  }
+  return MR_OK;
 }
 
-int launch_splitk(const float* x, const float* W, const float* bias, int T, int d, int N_r,
-                  int n_group, int topk_group, int k, float route_scale, int mask_mode,
+int launch_splitk(const void* x, bool x_bf16, const float* W, const float* bias, int T, int d,
+                  int N_r, int n_group, int topk_group, int k, float route_scale, int mask_mode,
                   bool use3x, int32_t* idx_out, float* w_out, float* logits_out, void* ws,
                   int sms, cudaStream_t st) {
-  const SplitKShape sh = splitk_shape(T, d, N_r, sms);
-  const mr::sk::Plan plan = mr::sk::make_plan(sh.NT, (sh.KC + sh.KS - 1) / sh.KS);
+  const SplitKShape sh = splitk_shape(T, d, N_r, sms, x_bf16);
+  const mr::sk::Plan plan = mr::sk::make_plan(sh.NT, (sh.KC + sh.KS - 1) / sh.KS, x_bf16);
   CUtensorMap mw, mx;
   if (!make_map_f32(&mw, W, (uint64_t)N_r, (uint64_t)d, mr::tc::BM, mr::tc::BK)) return MR_ERR_CUDA;
-  if (!make_map_f32(&mx, x, (uint64_t)T, (uint64_t)d, sh.NT, mr::tc::BK)) return MR_ERR_CUDA;
+  if (x_bf16) {
+    if (!make_map_bf16(&mx, x, (uint64_t)T, (uint64_t)d, sh.NT, /*swizzle=*/false))
+      return MR_ERR_CUDA;
+  } else if (!make_map_f32(&mx, static_cast<const float*>(x), (uint64_t)T, (uint64_t)d, sh.NT,
+                           mr::tc::BK)) {
+    return MR_ERR_CUDA;
+  }
   mr::sk::Params P;
   P.T = T;
   P.d = d;
   P.N = N_r;
   P.NT = sh.NT;
   P.KS = sh.KS;
+  P.CL = sh.CL;
   P.num_kc = sh.KC;
   P.use3x = use3x ? 1 : 0;
+  P.x_bf16 = x_bf16 ? 1 : 0;
   P.part = static_cast<float*>(ws);
   const size_t smem = plan.total + 1024;
   if (cudaFuncSetAttribute(mr::sk::router_splitk_gemm_kernel,
                            cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return MR_ERR_CUDA;
-  mr::sk::router_splitk_gemm_kernel<<<dim3(sh.KS, sh.MT, sh.TT), mr::sk::kThreads, smem, st>>>(
-      mw, mx, P);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)sh.KS, (unsigned)sh.MT, (unsigned)sh.TT);
+  cfg.blockDim = dim3(mr::sk::kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)sh.CL;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, mr::sk::router_splitk_gemm_kernel, mw, mx, P);
+  if (e != cudaSuccess) {
+    (void)cudaGetLastError();
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return MR_ERR_CUDA;
+  }
   if (launch_status() != MR_OK) return MR_ERR_CUDA;
+  const int KSr = sh.KS / sh.CL;
   const int nj = (N_r + 31) / 32;
 #define MR_RED_CASE(NJV)                                                                      \
   if (nj <= NJV)                                                                              \
-    return launch_reduce_nj<NJV>(P.part, sh.KS, T, N_r, bias, n_group, topk_group, k,          \
+    return launch_reduce_nj<NJV>(P.part, KSr, T, N_r, bias, n_group, topk_group, k,            \
                                  route_scale, mask_mode, idx_out, w_out, logits_out, st);
   MR_RED_CASE(2)
   MR_RED_CASE(4)
@@ -389,7 +484,8 @@ size_t mr_router_workspace_size(int T, int d, int N_r) {
   if (splitk_applies(T, N_r)) {
     int sms = 0, cc = 0;
     if (!device_info(&sms, &cc)) return 0;
-    need = std::max(need, splitk_shape(T, d, N_r, sms).ws_bytes);
+    need = std::max(need, std::max(splitk_shape(T, d, N_r, sms, false).ws_bytes,
+                                   splitk_shape(T, d, N_r, sms, true).ws_bytes));
   }
   return need;
 }
@@ -412,6 +508,15 @@ int mr_router_forward_ex(const void* x, int x_dtype, const float* W, const float
                : launch_ffma<false>(x, W, bias, T, d, N_r, n_group, topk_group, k, route_scale,
                                     mask_mode, idx_out, w_out, logits_out, s);
   }
+  // Small batches (decode): split-K over all SMs, fp32 W read directly, for
+  // either row type (3xTF32; a bf16 row needs no residual).
+  if (cc == 10 && workspace && aligned16(workspace) && splitk_applies(T, N_r) &&
+      tc_shape_ok(x, MR_F32, W, d, N_r) && (x_dtype == MR_F32 || d % 8 == 0) &&
+      !(precision == MR_PREC_BF16X3 && x_dtype != MR_BF16) &&
+      workspace_bytes >= splitk_shape(T, d, N_r, sms, x_dtype == MR_BF16).ws_bytes)
+    return launch_splitk(x, x_dtype == MR_BF16, W, bias, T, d, N_r, n_group, topk_group, k,
+                         route_scale, mask_mode, precision != MR_PREC_TF32, idx_out, w_out,
+                         logits_out, workspace, sms, s);
   if (x_dtype == MR_BF16 || precision == MR_PREC_BF16X3) {
     // bf16 activations on tensor cores: W as three bf16 planes (workspace)
     if (x_dtype != MR_BF16 || precision == MR_PREC_TF32 || cc != 10 || d % 8 != 0 ||
@@ -422,11 +527,6 @@ int mr_router_forward_ex(const void* x, int x_dtype, const float* W, const float
                      true, idx_out, w_out, logits_out, nullptr, workspace, sms, s);
   }
   if (cc != 10 || !tc_shape_ok(x, x_dtype, W, d, N_r)) return MR_ERR_UNSUPPORTED;
-  if (workspace && splitk_applies(T, N_r) &&
-      workspace_bytes >= splitk_shape(T, d, N_r, sms).ws_bytes)
-    return launch_splitk(static_cast<const float*>(x), W, bias, T, d, N_r, n_group, topk_group,
-                         k, route_scale, mask_mode, precision == MR_PREC_3XTF32, idx_out, w_out,
-                         logits_out, workspace, sms, s);
   float* wlo = (workspace && aligned16(workspace) && workspace_bytes >= wlo_bytes(d, N_r))
                    ? static_cast<float*>(workspace)
                    : nullptr;

@@ -168,3 +168,150 @@ __device__ __forceinline__ void mr_route_token_warp(const float* __restrict__ L,
     w_out[lane] = (my_s / den) * route_scale;
   }
 }
+
+// The same routing with short dependency chains, for groups that are whole
+// 32-expert columns of the lane layout (N_r / n_group a multiple of 32) or no
+// groups, and k <= 32:
+//   * every group's top-2 pair is reduced across the warp in one butterfly
+//     (the groups' chains interleave) and the kept groups are found by
+//     counting, for each group, the groups that beat it;
+//   * tau = the k-th best of the 32 lane maxima of the masked scores: those
+//     are k distinct experts, so the token's k-th best is >= tau;
+//   * the scores >= tau (at least k, usually little more) are compacted into
+//     `scratch` (warp-private shared memory, 96 words) and each one's place is
+//     the number of candidates that beat it (value desc, index asc).
+// More than 32 candidates (ties at the 0.0 fill, or tau = -inf) or other group
+// shapes take mr_route_token_warp.  Results are those of mr_route_token_warp
+// except for the order in which the k unbiased scores are summed.
+template <int NJ>
+__device__ __forceinline__ void mr_route_token_warp_fast(const float* __restrict__ L,
+                                                         const float* __restrict__ bias, int N_r,
+                                                         int n_group, int topk_group, int k,
+                                                         float route_scale, int mask_mode,
+                                                         int32_t* __restrict__ idx_out,
+                                                         float* __restrict__ w_out,
+                                                         float* scratch) {
+  const int lane = threadIdx.x & 31;
+  const int S = N_r / n_group;
+  if (k > 32 || (n_group > 1 && (S % 32 != 0 || n_group > NJ))) {
+    mr_route_token_warp<NJ>(L, bias, N_r, n_group, topk_group, k, route_scale, mask_mode,
+                            idx_out, w_out);
+    return;
+  }
+  float s[NJ], m[NJ];
+#pragma unroll
+  for (int j = 0; j < NJ; ++j) {
+    const int e = lane + 32 * j;
+    if (e < N_r) {
+      s[j] = mr_sigmoid(L[e]);
+      m[j] = s[j] + (bias ? bias[e] : 0.0f);
+    } else {
+      s[j] = 0.0f;
+      m[j] = -INFINITY;
+    }
+  }
+  if (n_group > 1) {
+    const int jpg = S / 32;  // lane slots j per group: group of slot j is j / jpg
+    int gj[NJ];
+#pragma unroll
+    for (int j = 0; j < NJ; ++j) gj[j] = jpg == 1 ? j : j / jpg;
+    float a1[NJ], a2[NJ];
+#pragma unroll
+    for (int g = 0; g < NJ; ++g) {
+      a1[g] = -INFINITY;
+      a2[g] = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < NJ; ++j) {
+        if (gj[j] == g) {
+          a2[g] = fmaxf(a2[g], fminf(a1[g], m[j]));
+          a1[g] = fmaxf(a1[g], m[j]);
+        }
+      }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+#pragma unroll
+      for (int g = 0; g < NJ; ++g) {
+        const float b1 = __shfl_xor_sync(0xffffffffu, a1[g], off);
+        const float b2 = __shfl_xor_sync(0xffffffffu, a2[g], off);
+        const float hi = fmaxf(a1[g], b1);
+        a2[g] = fmaxf(fminf(a1[g], b1), fmaxf(a2[g], b2));
+        a1[g] = hi;
+      }
+    }
+    uint32_t kept = 0;
+#pragma unroll
+    for (int g = 0; g < NJ; ++g) {
+      if (g < n_group) {
+        const float sg = a1[g] + a2[g];
+        int rank = 0;
+#pragma unroll
+        for (int o = 0; o < NJ; ++o) {
+          const float so = a1[o] + a2[o];
+          if (o < n_group && o != g) rank += (so > sg || (so == sg && o < g)) ? 1 : 0;
+        }
+        if (rank < topk_group) kept |= 1u << g;
+      }
+    }
+    const float fill = (mask_mode == MR_MASK_NEG_INF) ? -INFINITY : 0.0f;
+#pragma unroll
+    for (int j = 0; j < NJ; ++j)
+      if (lane + 32 * j < N_r && !((kept >> gj[j]) & 1u)) m[j] = fill;
+  }
+  // tau: the k-th best lane maximum (ties: lower lane first)
+  float lm = -INFINITY;
+#pragma unroll
+  for (int j = 0; j < NJ; ++j) lm = fmaxf(lm, m[j]);
+  int lr = 0;
+#pragma unroll
+  for (int o = 0; o < 32; ++o) {
+    const float v = __shfl_sync(0xffffffffu, lm, o);
+    lr += (v > lm || (v == lm && o < lane)) ? 1 : 0;
+  }
+  const uint32_t at = __ballot_sync(0xffffffffu, lr == k - 1);
+  const float tau = __shfl_sync(0xffffffffu, lm, __ffs(at) - 1);
+  // candidates: valid experts with masked score >= tau, compacted in slot order
+  uint32_t bal[NJ];
+  int n = 0;
+#pragma unroll
+  for (int j = 0; j < NJ; ++j) {
+    bal[j] = __ballot_sync(0xffffffffu, lane + 32 * j < N_r && m[j] >= tau);
+    n += __popc(bal[j]);
+  }
+  if (n > 32) {
+    mr_route_token_warp<NJ>(L, bias, N_r, n_group, topk_group, k, route_scale, mask_mode,
+                            idx_out, w_out);
+    return;
+  }
+  int base = 0;
+#pragma unroll
+  for (int j = 0; j < NJ; ++j) {
+    if ((bal[j] >> lane) & 1u) {
+      const int slot = base + __popc(bal[j] & ((1u << lane) - 1u));
+      scratch[slot] = m[j];
+      scratch[32 + slot] = s[j];
+      scratch[64 + slot] = __int_as_float(lane + 32 * j);
+    }
+    base += __popc(bal[j]);
+  }
+  __syncwarp();
+  float cv = -INFINITY, cs = 0.0f;
+  int ci = 0x7fffffff, rank = 32;
+  if (lane < n) {
+    cv = scratch[lane];
+    cs = scratch[32 + lane];
+    ci = __float_as_int(scratch[64 + lane]);
+    rank = 0;
+    for (int o = 0; o < n; ++o)
+      rank += mr_better(scratch[o], __float_as_int(scratch[64 + o]), cv, ci) ? 1 : 0;
+  }
+  float den = rank < k ? cs : 0.0f;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) den += __shfl_xor_sync(0xffffffffu, den, off);
+  den += 1e-20f;
+  if (rank < k) {
+    idx_out[rank] = ci;
+    w_out[rank] = (cs / den) * route_scale;
+  }
+  __syncwarp();  // scratch may be reused by the caller's next token
+}

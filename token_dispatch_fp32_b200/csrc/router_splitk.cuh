@@ -1,19 +1,30 @@
 // router_splitk.cuh -- gate GEMM for small batches (decode): split-K over all
-// SMs on the tensor cores, then a reduce-and-route kernel.
+// SMs on the tensor cores, a cluster reduction through distributed shared
+// memory, then a reduce-and-route kernel.
 //
 // With T of order 64 the fused kernel would give the weight read to one or two
 // SMs.  Here the roles of the operands are swapped so the 128-row MMA tile
 // runs over experts: A = W rows [128 experts x K], B = x rows [NT tokens x K],
 // D = logits^T [128 experts (TMEM lanes) x NT tokens (columns)], and the K
 // loop is split into KS slices, one CTA per (slice, expert tile, token tile),
-// so every SM streams a share of W.  Operands get the same 3xTF32 split as the
-// fused kernel; a slice spans only a few K chunks, so its accumulator stays
-// small and the tensor core's round-toward-zero accumulation costs nothing
-// measurable (partials are summed in fp32 with round-to-nearest afterwards).
-// Each CTA writes its fp32 partial logits to the workspace
-// part[slice][token][expert]; router_reduce_route_kernel sums the slices in
-// slice order (deterministic) and routes every token with one warp
-// (mr_route_token_warp).
+// so every SM streams a share of W once.
+//
+// Arithmetic: 3xTF32 on the staged fp32 values (the tensor core reads a tf32
+// operand with its 13 low mantissa bits ignored, so a staged tile serves as hi
+// and only lo = v - trunc(v) is written): W_hi*x_hi + W_lo*x_hi + W_hi*x_lo.
+// bf16 activations are staged by TMA as bf16 and widened into the fp32 B tile
+// by the workers; a bf16 value is exact in tf32, so x_lo = 0 and its MMA is
+// skipped.  A slice spans only a few K chunks, so the tensor core's
+// round-toward-zero accumulation stays within a few ulp.
+//
+// Reduction: the CL CTAs of a cluster hold consecutive K slices of the same
+// (expert tile, token tile).  Each copies its partial tile from TMEM to shared
+// memory; after a cluster barrier CTA r sums rows [r*NT/CL, (r+1)*NT/CL) of
+// the CL partials in rank order (deterministic) through distributed shared
+// memory and writes them to part[ks / CL][token][expert].  A second cluster
+// barrier keeps every CTA's shared memory alive until its peers have read it.
+// router_reduce_route_kernel (launched as a programmatic dependent of the
+// GEMM) sums the KS / CL slices in order and routes every token with one warp.
 #pragma once
 
 #include "router_tc.cuh"
@@ -23,28 +34,34 @@ namespace sk {
 
 using namespace mr::tc;
 
-constexpr int kThreads = 192;   // warp 0 TMA, warp 1 MMA, warps 2..5 split + epilogue
+constexpr int kWorkersSk = 8;   // worker warps 2..9
+constexpr int kThreads = 64 + 32 * kWorkersSk;  // warp 0 TMA, warp 1 MMA, then workers
 constexpr int kMaxNT = 256;     // tokens per CTA (MMA N)
+constexpr int kCluster = 8;     // CTAs per cluster reduction (when KS allows)
 
 struct Params {
-  int T, d, N, NT, KS, num_kc, use3x;
-  float* part;  // [KS][T][N]
+  int T, d, N, NT, KS, CL, num_kc, use3x, x_bf16;
+  float* part;  // [KS / CL][T][N]
 };
 
 struct Plan {
   int stages;
-  uint32_t a_bytes, b_bytes, hi_bytes, stage_bytes, bar_off, misc_off, total;
+  uint32_t a_bytes, b_bytes, hi_bytes, xs_bytes, stage_bytes, bar_off, misc_off, total;
 };
 
-__host__ __device__ inline Plan make_plan(int NT, int max_chunks) {
+// Stage: [A hi (W) | B hi (x fp32)] [A lo | B lo] [x bf16 staging].
+__host__ __device__ inline Plan make_plan(int NT, int max_chunks, bool x_bf16) {
   Plan p;
   p.a_bytes = BM * BK * 4;                 // 128 experts
   p.b_bytes = NT * BK * 4;                 // NT tokens
   p.hi_bytes = p.a_bytes + p.b_bytes;
-  p.stage_bytes = align_up(2 * p.hi_bytes, 1024);
+  p.xs_bytes = x_bf16 ? NT * BK * 2 : 0;
+  p.stage_bytes = align_up(2 * p.hi_bytes + p.xs_bytes, 1024);
   int s = (int)((kSmemBudget - 1024 - 512 - 64) / p.stage_bytes);
   if (s > kMaxStages) s = kMaxStages;
   if (s > max_chunks) s = max_chunks < 1 ? 1 : max_chunks;
+  // the reduction buffer [NT][128] fp32 aliases the ring after the K loop
+  while (s * p.stage_bytes < (uint32_t)NT * BM * 4) ++s;
   p.stages = s;
   p.bar_off = p.stages * p.stage_bytes;
   p.misc_off = p.bar_off + 512;
@@ -54,6 +71,13 @@ __host__ __device__ inline Plan make_plan(int NT, int max_chunks) {
 
 __host__ __device__ inline int slice_begin(int ks, int KS, int KC) {
   return (int)(((long)ks * KC) / KS);
+}
+
+// Byte offset of fp32 element (row, k) of a K-major tile with 128-byte rows
+// and the 128-byte swizzle (16-byte chunk c of row r sits at chunk c ^ (r % 8)).
+__device__ __forceinline__ uint32_t sw128_f32(int row, int k) {
+  return (uint32_t)(row >> 3) * 1024u + (uint32_t)(row & 7) * 128u +
+         ((uint32_t)((k >> 2) ^ (row & 7)) << 4) + (uint32_t)(k & 3) * 4u;
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -66,9 +90,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int c_beg = slice_begin(ks, P.KS, P.num_kc), c_end = slice_begin(ks + 1, P.KS, P.num_kc);
   const int NC = c_end - c_beg;
   const int NT = P.NT;
-  const Plan plan = make_plan(NT, (P.num_kc + P.KS - 1) / P.KS);
+  const bool xb = P.x_bf16 != 0;
+  const bool conv = P.use3x || xb;  // the workers touch every stage
+  const Plan plan = make_plan(NT, (P.num_kc + P.KS - 1) / P.KS, xb);
   const int STAGES = plan.stages;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int CL = P.CL;
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + plan.bar_off);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + plan.misc_off);
@@ -78,10 +105,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int B_FULL = 0, B_CONV = STAGES, B_EMPTY = 2 * STAGES, B_ACC = 3 * STAGES;
   const uint32_t tmem_cols = NT <= 32 ? 32 : NT <= 64 ? 64 : NT <= 128 ? 128 : 256;
 
+  // the reduce-and-route grid may be scheduled now: it waits for this grid's
+  // completion (griddepcontrol.wait) before reading anything
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (threadIdx.x == 0) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_w)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_x)) : "memory");
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(bar(B_FULL + s), 1);
-      mbar_init(bar(B_CONV + s), 128);
+      mbar_init(bar(B_CONV + s), kWorkersSk);  // one elected arrival per worker warp
       mbar_init(bar(B_EMPTY + s), 1);
     }
     mbar_init(bar(B_ACC), 1);
@@ -99,10 +131,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  bool ok = true;
 
   if (warp == 0) {
     if (lane == 0) {
-      const uint32_t tx = (uint32_t)(BM + NT) * BK * 4;
+      const uint32_t tx = plan.a_bytes + (xb ? plan.xs_bytes : plan.b_bytes);
       int issued = 0;
       for (int i = 0; i < NC; ++i) {
         const int s = i % STAGES, kc = c_beg + i;
@@ -111,7 +144,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t base = smem0 + s * plan.stage_bytes;
         mbar_arrive_expect_tx(bar(B_FULL + s), tx);
         tma_load_2d(base, &map_w, bar(B_FULL + s), kc * BK, mt * BM);
-        tma_load_2d(base + plan.a_bytes, &map_x, bar(B_FULL + s), kc * BK, tt * NT);
+        tma_load_2d(xb ? base + 2 * plan.hi_bytes : base + plan.a_bytes, &map_x, bar(B_FULL + s),
+                    kc * BK, tt * NT);
       }
       for (int i = issued - STAGES < 0 ? 0 : issued - STAGES; i < issued; ++i)
         mbar_wait(bar(B_FULL + i % STAGES), (i / STAGES) & 1, abort, true);
@@ -121,7 +155,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t idesc = make_idesc(NT);
       for (int i = 0; i < NC; ++i) {
         const int s = i % STAGES;
-        if (!mbar_wait(P.use3x ? bar(B_CONV + s) : bar(B_FULL + s), (i / STAGES) & 1, abort))
+        if (!mbar_wait(conv ? bar(B_CONV + s) : bar(B_FULL + s), (i / STAGES) & 1, abort))
           break;
         tc_fence_after();
         const uint32_t a_hi = smem0 + s * plan.stage_bytes;
@@ -135,8 +169,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t dah = make_desc(a_hi + ko), dbh = make_desc(b_hi + ko);
           mma_tf32(tmem_base, dah, dbh, idesc, acc0);
           if (P.use3x) {
-            mma_tf32(tmem_base, dah, make_desc(b_lo + ko), idesc, 1u);
-            mma_tf32(tmem_base, make_desc(a_lo + ko), dbh, idesc, 1u);
+            mma_tf32(tmem_base, make_desc(a_lo + ko), dbh, idesc, 1u);   // W_lo * x
+            if (!xb) mma_tf32(tmem_base, dah, make_desc(b_lo + ko), idesc, 1u);  // W * x_lo
           }
         }
         mma_commit(bar(B_EMPTY + s));
@@ -144,48 +178,113 @@ __global__ void __launch_bounds__(kThreads, 1)
       mma_commit(bar(B_ACC));
     }
   } else {
-    const int ct = threadIdx.x - 64;  // 0..127
-    if (P.use3x) {
-      const int n4 = (int)(plan.hi_bytes / 16);
+    const int ct = threadIdx.x - 64;  // 0 .. 32 * kWorkersSk - 1
+    constexpr int kW = 32 * kWorkersSk;
+    if (conv) {
       for (int i = 0; i < NC; ++i) {
         const int s = i % STAGES;
         if (!mbar_wait(bar(B_FULL + s), (i / STAGES) & 1, abort)) break;
-        // staged fp32 = hi (the tensor core truncates tf32 operands); write lo
-        const float4* hi = reinterpret_cast<const float4*>(smem + s * plan.stage_bytes);
-        float4* lo = reinterpret_cast<float4*>(smem + s * plan.stage_bytes + plan.hi_bytes);
-        for (int j = ct; j < n4; j += 128) {
-          const float4 v = hi[j];
-          float4 l;
-          l.x = v.x - __uint_as_float(__float_as_uint(v.x) & 0xFFFFE000u);
-          l.y = v.y - __uint_as_float(__float_as_uint(v.y) & 0xFFFFE000u);
-          l.z = v.z - __uint_as_float(__float_as_uint(v.z) & 0xFFFFE000u);
-          l.w = v.w - __uint_as_float(__float_as_uint(v.w) & 0xFFFFE000u);
-          lo[j] = l;
+        uint8_t* st = smem + s * plan.stage_bytes;
+        if (xb) {
+          // widen the bf16 x tile [NT][32] into the swizzled fp32 B tile
+          const uint16_t* xs = reinterpret_cast<const uint16_t*>(st + 2 * plan.hi_bytes);
+          uint8_t* bh = st + plan.a_bytes;
+          for (int j = ct; j < NT * BK; j += kW) {
+            const int r = j / BK, kk = j % BK;
+            *reinterpret_cast<float*>(bh + sw128_f32(r, kk)) = mr_bf16_to_f32(xs[j]);
+          }
         }
+        if (P.use3x) {
+          // lo = v - trunc_tf32(v) of W (and of fp32 x), same layout
+          const int n4 = (int)((xb ? plan.a_bytes : plan.hi_bytes) / 16);
+          const float4* hi = reinterpret_cast<const float4*>(st);
+          float4* lo = reinterpret_cast<float4*>(st + plan.hi_bytes);
+          for (int j = ct; j < n4; j += kW) {
+            const float4 v = hi[j];
+            float4 l;
+            l.x = v.x - __uint_as_float(__float_as_uint(v.x) & 0xFFFFE000u);
+            l.y = v.y - __uint_as_float(__float_as_uint(v.y) & 0xFFFFE000u);
+            l.z = v.z - __uint_as_float(__float_as_uint(v.z) & 0xFFFFE000u);
+            l.w = v.w - __uint_as_float(__float_as_uint(v.w) & 0xFFFFE000u);
+            lo[j] = l;
+          }
+        }
+        // each thread's generic-proxy writes are made visible to the tensor
+        // core's async proxy, then one lane per warp releases the stage
         fence_proxy_async();
-        mbar_arrive(bar(B_CONV + s));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(B_CONV + s));
       }
     }
     // The accumulator barrier is always committed (also after an abort), so
     // this wait drains every MMA before TMEM is released.
-    const bool ok = __all_sync(0xffffffffu, mbar_wait(bar(B_ACC), 0, abort, true)) && !*abort;
+    ok = __all_sync(0xffffffffu, mbar_wait(bar(B_ACC), 0, abort, true)) && !*abort;
     tc_fence_after();
     const int q = warp & 3;
-    const int e = mt * BM + q * 32 + lane;  // expert of this TMEM lane
+    const int hf = (warp - 2) >> 2;  // warps w and w+4 share lanes, split the columns
+    const int el = q * 32 + lane;  // expert (within the tile) of this TMEM lane
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+    float* red = reinterpret_cast<float*>(smem);  // [NT][128], aliases the idle ring
     float v[16];
-    for (int c = 0; c < NT / 16; ++c) {
+    const int nc = NT / 16, ch = (nc + 1) / 2;
+    for (int c = hf * ch; c < nc && c < (hf + 1) * ch; ++c) {
       tmem_ld16(tmem_base + lane_off + (uint32_t)(c * 16), v);  // whole warp
+      if (CL > 1) {
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const int t = tt * NT + c * 16 + j;
-        if (ok && t < P.T && e < P.N) P.part[((long)ks * P.T + t) * P.N + e] = v[j];
+        for (int j = 0; j < 16; ++j) red[(c * 16 + j) * BM + el] = v[j];
+      } else {
+        const int e = mt * BM + el;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const int t = tt * NT + c * 16 + j;
+          if (ok && t < P.T && e < P.N) P.part[((long)ks * P.T + t) * P.N + e] = v[j];
+        }
       }
     }
   }
 
   tc_fence_before();
   __syncthreads();
+  if (CL > 1) {
+    // every thread of the cluster takes both barriers, whatever happened above
+    cluster_sync_all();
+    const uint32_t rank = cluster_rank();
+    const int rows = NT / CL;  // tokens reduced by this CTA
+    const float* red = reinterpret_cast<const float*>(smem);
+    // a CTA that gave up on a wait (abort flag) leaves no valid partial
+    for (int src = 0; src < CL; ++src)
+      ok = ok && __float_as_int(ld_peer_f32(reinterpret_cast<const float*>(
+                                                const_cast<const int*>(abort)),
+                                            (uint32_t)src)) == 0;
+    for (int j = threadIdx.x; j < rows * (BM / 4); j += kThreads) {
+      const int tl = (int)rank * rows + j / (BM / 4), el = (j % (BM / 4)) * 4;
+      // CL == kCluster here: all loads in flight before the first add
+      float4 o[kCluster];
+#pragma unroll
+      for (int src = 0; src < kCluster; ++src)
+        o[src] = ld_peer_f32x4(&red[tl * BM + el], (uint32_t)src);
+      float4 acc = o[0];
+#pragma unroll
+      for (int src = 1; src < kCluster; ++src) {
+        acc.x += o[src].x;
+        acc.y += o[src].y;
+        acc.z += o[src].z;
+        acc.w += o[src].w;
+      }
+      const int t = tt * NT + tl, e = mt * BM + el;
+      if (ok && t < P.T && e < P.N) {
+        float* dst = P.part + ((long)(ks / CL) * P.T + t) * P.N + e;
+        if (e + 3 < P.N) {
+          *reinterpret_cast<float4*>(dst) = acc;
+        } else {
+          dst[0] = acc.x;
+          if (e + 1 < P.N) dst[1] = acc.y;
+          if (e + 2 < P.N) dst[2] = acc.z;
+        }
+      }
+    }
+    cluster_sync_all();
+  }
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
@@ -196,7 +295,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // One CTA per token: sum the KS partial logits of each expert in slice order,
-// then route the token with one warp.
+// then route the token with one warp.  Launched as a programmatic dependent of
+// the GEMM: it waits for that grid's results before reading them.
 template <int NJ>
 __global__ void __launch_bounds__(256)
     router_reduce_route_kernel(const float* __restrict__ part, int KS, int T, int N_r,
@@ -204,6 +304,11 @@ __global__ void __launch_bounds__(256)
                                float route_scale, int mask_mode, int32_t* __restrict__ idx_out,
                                float* __restrict__ w_out, float* __restrict__ logits_out) {
   __shared__ float L[32 * NJ];
+  __shared__ float bs[32 * NJ];
+  __shared__ float scratch[96];
+  // the bias does not come from the GEMM: fetch it while the GEMM runs
+  for (int e = threadIdx.x; e < N_r; e += blockDim.x) bs[e] = bias ? bias[e] : 0.0f;
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int t = blockIdx.x;
   for (int e = threadIdx.x; e < N_r; e += blockDim.x) {
     float acc = 0.0f;
@@ -216,8 +321,8 @@ __global__ void __launch_bounds__(256)
   }
   __syncthreads();
   if (threadIdx.x < 32)
-    mr_route_token_warp<NJ>(L, bias, N_r, n_group, topk_group, k, route_scale, mask_mode,
-                            idx_out + (long)t * k, w_out + (long)t * k);
+    mr_route_token_warp_fast<NJ>(L, bs, N_r, n_group, topk_group, k, route_scale, mask_mode,
+                                 idx_out + (long)t * k, w_out + (long)t * k, scratch);
 }
 
 }  // namespace sk

@@ -235,6 +235,18 @@ __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.aligned;\n\tbarrier.cluster.wait.aligned;" ::: "memory");
 }
 
+// 16 bytes from the same offset in CTA `peer`'s shared memory (16-byte aligned).
+__device__ __forceinline__ float4 ld_peer_f32x4(const float* local, uint32_t peer) {
+  uint32_t ra;
+  float4 v;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(smem_u32(local)), "r"(peer));
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(ra)
+               : "memory");
+  return v;
+}
+
 __device__ __forceinline__ float ld_peer_f32(const float* local, uint32_t peer) {
   uint32_t ra, v;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(smem_u32(local)), "r"(peer));
@@ -537,7 +549,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(bar(B_FULL + s), 1);
-      mbar_init(bar(B_CONV + s), 32 * kWorkers);
+      mbar_init(bar(B_CONV + s), kWorkers);  // one elected arrival per worker warp
       mbar_init(bar(B_EMPTY + s), 1);
     }
     mbar_init(bar(B_ACCF + 0), 1);
@@ -780,8 +792,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const bool any_nz = __any_sync(0xffffffffu, (nz << 1) != 0u);  // ignore -0.0
         if (lane == 0) xnz[s * kWorkers + (warp - 2)] = any_nz ? 1u : 0u;
+        // each thread's residual writes become visible to the async proxy;
+        // then one lane per warp releases the stage
         fence_proxy_async();
-        mbar_arrive(bar(B_CONV + s));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(B_CONV + s));
       }
       // promote the interval before the one the tensor core is working on
       if ((kc % kPromote) == kPromote - 1 && kc / kPromote >= 1) promote(kc / kPromote - 1);
