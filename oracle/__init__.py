@@ -51,6 +51,9 @@ def _load():
         p = C.c_void_p
         lib.mo_router.argtypes = [p, p, p, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int,
                                   C.c_int, C.c_double, C.c_int, p, p, p, p, C.c_int]
+        lib.mo_router2.argtypes = [p, p, p, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int,
+                                   C.c_int, C.c_double, C.c_int, C.c_int, C.c_int, C.c_int,
+                                   p, p, p, p, C.c_int]
         lib.mo_dispatch.argtypes = [p, C.c_int, C.c_int, C.c_int, p, p, p, p]
         lib.mo_gather.argtypes = [p, C.c_long, C.c_int, C.c_int, p, p, C.c_long, p]
         lib.mo_round_bf16.argtypes = [C.c_double]
@@ -71,12 +74,17 @@ def num_threads() -> int:
 
 
 def router(x, W, b, n_group, topk_group, k, route_scale, mask_mode,
-           want_logits=False, threads=0) -> dict:
+           want_logits=False, threads=0, score="sigmoid", group_score="top2",
+           eps=True) -> dict:
     """Gate forward for every row of x (Kimi K2 "Normalize weights" page,
     MoEGate.forward; DeepSeek-V3.2-Exp "Normalize weights" page,
     Gate.forward; DeepSeek-V3 "MoE Router" note, "How it works").
 
     x [T,d] fp32 values, W [N_r,d] fp32, b [N_r] fp32 or None.
+    Variants (DeepSeek-V3.2-Exp Gate.forward): score="softmax" (softmax over
+    all experts; the weights are the scaled scores, not renormalised),
+    group_score="max" (a group's largest biased score instead of its top-2
+    sum), eps=False (renormalise by the plain sum).
     Returns idx [T,k] int32 in canonical order (masked biased score
     descending, index ascending), w [T,k] float64, margins [T,3] float64
     (selection, group, slot-order margins) and optionally logits [T,N_r].
@@ -92,9 +100,11 @@ def router(x, W, b, n_group, topk_group, k, route_scale, mask_mode,
     w = np.empty((T, k), np.float64)
     margins = np.empty((T, 3), np.float64)
     logits = np.empty((T, N_r), np.float64) if want_logits else None
-    rc = lib.mo_router(_ptr(x), _ptr(W), _ptr(b), T, d, N_r, n_group, topk_group, k,
-                       float(route_scale), mask_mode, _ptr(idx), _ptr(w), _ptr(logits),
-                       _ptr(margins), threads)
+    assert score in ("sigmoid", "softmax") and group_score in ("top2", "max")
+    rc = lib.mo_router2(_ptr(x), _ptr(W), _ptr(b), T, d, N_r, n_group, topk_group, k,
+                        float(route_scale), mask_mode, int(score == "softmax"),
+                        int(group_score == "max"), int(bool(eps)), _ptr(idx), _ptr(w),
+                        _ptr(logits), _ptr(margins), threads)
     if rc != 0:
         raise ValueError(f"oracle router rejected the arguments (rc={rc})")
     return {"idx": idx, "w": w, "margins": margins, "logits": logits}

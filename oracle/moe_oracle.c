@@ -87,10 +87,21 @@ static int mo_cmp_double_desc(const void *pa, const void *pb)
  * margins[2] = smallest gap between consecutive selected masked scores
  *              (+inf for k = 1): decides the order of the k slots.
  */
+/* Scoring variants of the DeepSeek-V3.2-Exp "Normalize weights" page
+ * (Gate.forward): softmax scores over all N_r experts, which are then used as
+ * weights without renormalisation; the group score as the group's largest
+ * biased score (the page's choice when there is no bias); renormalisation
+ * without the 1e-20 of the Kimi K2 code. */
+typedef struct {
+    int softmax;    /* 0: s = sigmoid(L); 1: s = softmax(L), weights not renormalised */
+    int group_max;  /* 0: group score = sum of the two largest; 1: the largest */
+    int eps;        /* 1: renormalise by sum + 1e-20 (Kimi K2); 0: by the sum */
+} mo_variant;
+
 static void mo_router_token(const float *xt, const float *W, const float *bias,
                             int d, int N_r, int n_group, int topk_group, int k,
-                            double route_scale, int mask_mode, int32_t *idx,
-                            double *w, double *logits, double *margins,
+                            double route_scale, int mask_mode, mo_variant var,
+                            int32_t *idx, double *w, double *logits, double *margins,
                             double *L, double *s, double *m, mo_pair *ord,
                             double *tmp, mo_pair *gord, double *gs)
 {
@@ -101,17 +112,32 @@ static void mo_router_token(const float *xt, const float *W, const float *bias,
         for (int j = 0; j < d; ++j)
             acc += (double)xt[j] * (double)wi[j];
         L[i] = acc;
-        s[i] = 1.0 / (1.0 + exp(-acc));
-        m[i] = s[i] + (bias ? (double)bias[i] : 0.0);
+        if (!var.softmax)
+            s[i] = 1.0 / (1.0 + exp(-acc));
         if (logits) logits[i] = acc;
     }
+    if (var.softmax) {
+        /* softmax over all experts, shifted by the largest logit */
+        double mx = L[0], sum = 0.0;
+        for (int i = 1; i < N_r; ++i)
+            if (L[i] > mx) mx = L[i];
+        for (int i = 0; i < N_r; ++i)
+            sum += exp(L[i] - mx);
+        for (int i = 0; i < N_r; ++i)
+            s[i] = exp(L[i] - mx) / sum;
+    }
+    for (int i = 0; i < N_r; ++i)
+        m[i] = s[i] + (bias ? (double)bias[i] : 0.0);
 
     double m_grp = INFINITY;
     if (n_group > 1) {
         for (int g = 0; g < n_group; ++g) {
             memcpy(tmp, m + (size_t)g * S, sizeof(double) * S);
             qsort(tmp, S, sizeof(double), mo_cmp_double_desc);
-            gs[g] = tmp[0] + tmp[1];
+            if (var.group_max)
+                gs[g] = tmp[0];
+            else
+                gs[g] = tmp[0] + tmp[1];
             gord[g].v = gs[g];
             gord[g].i = g;
         }
@@ -136,9 +162,14 @@ static void mo_router_token(const float *xt, const float *W, const float *bias,
         idx[j] = ord[j].i;
         den += s[ord[j].i];
     }
-    den += 1e-20;
-    for (int j = 0; j < k; ++j)
-        w[j] = route_scale * (s[ord[j].i] / den);
+    if (var.eps)
+        den += 1e-20;
+    for (int j = 0; j < k; ++j) {
+        if (var.softmax)
+            w[j] = route_scale * s[ord[j].i];  /* softmax: not renormalised */
+        else
+            w[j] = route_scale * (s[ord[j].i] / den);
+    }
 
     if (margins) {
         double m_tok = INFINITY;
@@ -155,11 +186,12 @@ static void mo_router_token(const float *xt, const float *W, const float *bias,
     }
 }
 
-int mo_router(const float *x, const float *W, const float *bias, int T, int d,
-              int N_r, int n_group, int topk_group, int k, double route_scale,
-              int mask_mode, int32_t *idx, double *w, double *logits,
-              double *margins, int nthreads)
+int mo_router2(const float *x, const float *W, const float *bias, int T, int d,
+               int N_r, int n_group, int topk_group, int k, double route_scale,
+               int mask_mode, int softmax, int group_max, int eps, int32_t *idx,
+               double *w, double *logits, double *margins, int nthreads)
 {
+    const mo_variant var = {softmax != 0, group_max != 0, eps != 0};
     if (T < 0 || d <= 0 || N_r <= 0 || n_group <= 0 || N_r % n_group != 0 ||
         topk_group <= 0 || topk_group > n_group || k <= 0 || k > N_r ||
         (n_group > 1 && N_r / n_group < 2) || (mask_mode != 0 && mask_mode != 1) ||
@@ -189,7 +221,7 @@ int mo_router(const float *x, const float *W, const float *bias, int T, int d,
 #endif
             for (int t = 0; t < T; ++t)
                 mo_router_token(x + (size_t)t * d, W, bias, d, N_r, n_group,
-                                topk_group, k, route_scale, mask_mode,
+                                topk_group, k, route_scale, mask_mode, var,
                                 idx + (size_t)t * k, w + (size_t)t * k,
                                 logits ? logits + (size_t)t * N_r : NULL,
                                 margins ? margins + (size_t)t * 3 : NULL, L, s,
@@ -199,6 +231,17 @@ int mo_router(const float *x, const float *W, const float *bias, int T, int d,
     }
     (void)nthreads;
     return bad ? MO_ERR_ARG : MO_OK;
+}
+
+/* The Kimi K2 / DeepSeek-V3 gate: sigmoid scores, top-2 group sums,
+ * renormalisation with + 1e-20. */
+int mo_router(const float *x, const float *W, const float *bias, int T, int d,
+              int N_r, int n_group, int topk_group, int k, double route_scale,
+              int mask_mode, int32_t *idx, double *w, double *logits,
+              double *margins, int nthreads)
+{
+    return mo_router2(x, W, bias, T, d, N_r, n_group, topk_group, k, route_scale,
+                      mask_mode, 0, 0, 1, idx, w, logits, margins, nthreads);
 }
 
 /* ------------------------------------------------------------------ */

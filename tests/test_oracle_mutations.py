@@ -30,6 +30,11 @@ MUTATIONS = {
     "bf16_round_half_up": ("double r = nearbyint(ldexp(fabs(v), -q));",
                            "double r = floor(ldexp(fabs(v), -q) + 0.5);"),
     "logit_sign_flip": ("s[i] = 1.0 / (1.0 + exp(-acc));", "s[i] = 1.0 / (1.0 + exp(acc));"),
+    "softmax_renormalised": ("w[j] = route_scale * s[ord[j].i];  /* softmax: not renormalised */",
+                             "w[j] = route_scale * (s[ord[j].i] / den);"),
+    "softmax_not_shifted_sum": ("sum += exp(L[i] - mx);", "sum += exp(L[i]);"),
+    "group_max_is_pair_sum": ("gs[g] = tmp[0];\n            else", "gs[g] = tmp[0] + tmp[1];\n            else"),
+    "epsilon_always_added": ("    if (var.eps)\n        den += 1e-20;", "    den += 1e-20;"),
 }
 
 

@@ -389,3 +389,109 @@ def test_combine_routed_rounding_is_observable():
     y, routed = oracle.combine(one, w, np.array([0], np.int32), tiny, 1)
     assert routed[0, 0] == 1.0
     assert y[0, 0] == 1.0
+
+
+# --------------------------------------------------------------------------
+# Scoring variants (DeepSeek-V3.2-Exp "Normalize weights" page, Gate.forward):
+# softmax scores used as weights without renormalisation, the group's largest
+# biased score as its group score, renormalisation without the 1e-20.
+
+def _softmax64(L):
+    z = L - L.max(axis=1, keepdims=True)
+    e = np.exp(z)
+    return e / e.sum(axis=1, keepdims=True)
+
+
+def test_softmax_all_experts_gives_scaled_softmax():
+    """G = 1, no bias, k = N_r: every expert is chosen and its weight is
+    route_scale * softmax(L) (scipy's softmax on BLAS logits), summing to the
+    route scale."""
+    from scipy.special import softmax
+    rng = np.random.default_rng(71)
+    x, W, _ = _rand_problem(rng, 64, 48, 12)
+    r = oracle.router(x, W, None, 1, 1, 12, 2.5, 0, score="softmax")
+    L = x.astype(np.float64) @ W.astype(np.float64).T
+    ref = 2.5 * softmax(L, axis=1)
+    for t in range(64):
+        got = np.zeros(12)
+        got[r["idx"][t]] = r["w"][t]
+        np.testing.assert_allclose(got, ref[t], rtol=1e-12, atol=1e-15)
+    np.testing.assert_allclose(r["w"].sum(1), 2.5, rtol=1e-12)
+
+
+def test_softmax_weights_are_not_renormalised():
+    """k < N_r: the top-k of softmax(L) are the top-k logits (softmax is
+    monotone) and their weights are the scaled scores themselves, so they sum
+    to less than the route scale."""
+    rng = np.random.default_rng(72)
+    x, W, _ = _rand_problem(rng, 200, 32, 16)
+    r = oracle.router(x, W, None, 1, 1, 4, 2.5, 0, score="softmax")
+    L = x.astype(np.float64) @ W.astype(np.float64).T
+    p = _softmax64(L)
+    want = np.argsort(-L, axis=1, kind="stable")[:, :4]
+    assert np.array_equal(r["idx"], want)
+    np.testing.assert_allclose(r["w"], 2.5 * np.take_along_axis(p, want, 1), rtol=1e-12)
+    assert (r["w"].sum(1) < 2.5 - 1e-6).all()
+
+
+@pytest.mark.parametrize("group_score", ["top2", "max"])
+@pytest.mark.parametrize("score", ["sigmoid", "softmax"])
+def test_variants_brute_force(score, group_score):
+    """Brute force on tiny inputs for each scoring variant: scores from the
+    closed forms (expit / softmax of BLAS logits), group scores as the best
+    pair sum or the best single score, then the best k-subset."""
+    rng = np.random.default_rng(73 + 2 * (score == "softmax") + (group_score == "max"))
+    T, N_r, G, Gk, k = 250, 12, 4, 2, 3
+    x, W, _ = _rand_problem(rng, T, 16, N_r)
+    b = rng.uniform(-0.05, 0.05, N_r).astype(np.float32)
+    r = oracle.router(x, W, b, G, Gk, k, 2.5, 0, score=score, group_score=group_score)
+    L = x.astype(np.float64) @ W.astype(np.float64).T
+    s = expit(L) if score == "sigmoid" else _softmax64(L)
+    c = s + b.astype(np.float64)
+    S = N_r // G
+    for t in range(T):
+        if group_score == "top2":
+            want, _ = _brute(list(c[t]), G, Gk, k, 0)
+        else:
+            gs = [max(c[t, g * S:(g + 1) * S]) for g in range(G)]
+            keep = min(itertools.combinations(range(G), Gk),
+                       key=lambda sub: (-math.fsum(gs[g] for g in sub), sub))
+            m = [c[t, i] if (i // S) in keep else -math.inf for i in range(N_r)]
+            want = set(min(itertools.combinations(range(N_r), k),
+                           key=lambda sub: (-math.fsum(m[i] for i in sub), sub)))
+        assert set(r["idx"][t].tolist()) == want, (t, r["idx"][t], sorted(want))
+        sel = s[t, r["idx"][t]]
+        w = 2.5 * sel if score == "softmax" else 2.5 * sel / (sel.sum() + 1e-20)
+        np.testing.assert_allclose(r["w"][t], w, rtol=1e-12)
+
+
+def test_group_max_differs_from_top2_sum():
+    """A token whose best single score and best pair sum sit in different
+    groups: the two group scores keep different groups."""
+    # group 0: (0.9, 0.1)  -> max 0.9, pair 1.0; group 1: (0.6, 0.55) -> max 0.6, pair 1.15
+    x, W = _one_hot_logits(["0.9", "0.1", "0.6", "0.55"])
+    top2 = oracle.router(x, W, None, 2, 1, 1, 1.0, 0)
+    amax = oracle.router(x, W, None, 2, 1, 1, 1.0, 0, group_score="max")
+    assert top2["idx"][0].tolist() == [2]
+    assert amax["idx"][0].tolist() == [0]
+
+
+def test_renormalisation_epsilon_only_matters_when_scores_underflow():
+    """With or without the 1e-20 the weights agree for ordinary scores; when
+    every chosen sigmoid score underflows to 0 the epsilon gives 0 weights and
+    the plain sum gives 0/0."""
+    rng = np.random.default_rng(74)
+    x, W, b = _rand_problem(rng, 100, 32, 16)
+    a = oracle.router(x, W, b, 4, 2, 4, 2.5, 0)
+    n = oracle.router(x, W, b, 4, 2, 4, 2.5, 0, eps=False)
+    assert np.array_equal(a["idx"], n["idx"])
+    np.testing.assert_allclose(a["w"], n["w"], rtol=1e-15)
+    # logits of -1000: exp(1000) overflows, sigmoid is exactly 0
+    xz = np.zeros((1, 4), np.float32)
+    xz[0, 0] = 1.0
+    Wz = np.zeros((8, 4), np.float32)
+    Wz[:, 0] = -1000.0
+    az = oracle.router(xz, Wz, None, 1, 1, 2, 2.5, 0)
+    nz = oracle.router(xz, Wz, None, 1, 1, 2, 2.5, 0, eps=False)
+    assert (az["w"] == 0).all()
+    assert np.isnan(nz["w"]).all()
