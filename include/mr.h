@@ -83,6 +83,24 @@ typedef struct CUstream_st *mr_stream_t;
 #define MR_PREC_FFMA 2
 #define MR_PREC_BF16X3 3
 
+/* ---- scoring variants (flags of mr_router_forward_ex2) --------------------
+ * From the DeepSeek-V3.2-Exp "Normalize weights" page (Gate.forward):
+ * MR_SCORE_SOFTMAX  s = softmax(L) over all N_r experts instead of sigmoid;
+ *                   the chosen experts' weights are route_scale * s, not
+ *                   renormalised.
+ * MR_GROUP_MAX      group score = the group's largest biased score (the
+ *                   page's choice when there is no bias) instead of the sum
+ *                   of its two largest.
+ * MR_NORM_NO_EPS    renormalise by the plain sum of the k scores (the page)
+ *                   instead of sum + 1e-20 (Kimi K2 MoEGate.forward); the two
+ *                   differ only when every chosen score underflows.
+ * The page's gate is MR_NORM_NO_EPS, plus MR_GROUP_MAX when there is no bias,
+ * plus MR_SCORE_SOFTMAX for score_func "softmax".  0 is the Kimi K2 /
+ * DeepSeek-V3 gate of mr_router_forward.                                    */
+#define MR_SCORE_SOFTMAX 1
+#define MR_GROUP_MAX 2
+#define MR_NORM_NO_EPS 4
+
 /* Library version, major*10000 + minor*100 + patch. */
 int mr_version(void);
 
@@ -150,9 +168,10 @@ size_t mr_router_workspace_size(int T, int d, int N_r);
  *   workspace   device buffer of workspace_bytes, or NULL.  With at least
  *               mr_router_workspace_size(T, d, N_r) bytes, batches of up to
  *               256 tokens on the tensor-core precisions use the split-K path
- *               (two launches: a K-sliced GEMM over all SMs writing partial
- *               logits, then a reduce-and-route kernel); the result is the
- *               same arithmetic, summed in a fixed order (deterministic).
+ *               for fp32 and bf16 rows alike (two launches: a K-sliced 3xTF32
+ *               GEMM over all SMs whose slices are summed in clusters, then a
+ *               reduce-and-route kernel); the result is the same arithmetic,
+ *               summed in a fixed order (deterministic).
  *               Larger batches use it for W's tf32 residuals (one extra
  *               launch); results are identical with or without it.
  * Returns MR_ERR_UNSUPPORTED when the requested precision cannot run this
@@ -165,6 +184,21 @@ int mr_router_forward_ex(const void *x, int x_dtype, const float *W,
                          int mask_mode, int precision, int32_t *idx_out,
                          float *w_out, float *logits_out, void *workspace,
                          size_t workspace_bytes, mr_stream_t stream);
+
+/*
+ * mr_router_forward_ex2 -- mr_router_forward_ex with the scoring variants of
+ * the DeepSeek-V3.2-Exp "Normalize weights" page (Gate.forward): `flags` is
+ * a combination of MR_SCORE_SOFTMAX, MR_GROUP_MAX and MR_NORM_NO_EPS (0 gives
+ * mr_router_forward_ex).  Every path (fused tensor-core, split-K, CUDA-core)
+ * supports every combination; other bits give MR_ERR_INVALID_ARG.
+ */
+int mr_router_forward_ex2(const void *x, int x_dtype, const float *W,
+                          const float *bias, int T, int d, int N_r, int n_group,
+                          int topk_group, int k, float route_scale,
+                          int mask_mode, int precision, int flags,
+                          int32_t *idx_out, float *w_out, float *logits_out,
+                          void *workspace, size_t workspace_bytes,
+                          mr_stream_t stream);
 
 /*
  * mr_dispatch_workspace_size -- bytes of device workspace mr_dispatch needs.

@@ -83,6 +83,17 @@ def test_router_ex_validation():
                                   None, 0, None) == mr.MR_ERR_INVALID_ARG
 
 
+def test_router_ex2_rejects_unknown_flags():
+    L = mr.lib()
+    p = C.c_void_p(16)
+    for flags in (8, 16, -1):
+        assert L.mr_router_forward_ex2(p, 0, p, None, 4, 64, 64, 8, 4, 8, 2.5, 0, 0, flags, p, p,
+                                       None, None, 0, None) == mr.MR_ERR_INVALID_ARG
+    # the known flags pass flag validation and then fail on the bad dtype
+    assert L.mr_router_forward_ex2(p, 7, p, None, 4, 64, 64, 8, 4, 8, 2.5, 0, 0, 7, p, p,
+                                   None, None, 0, None) == mr.MR_ERR_INVALID_ARG
+
+
 def test_dispatch_validation():
     L = mr.lib()
     p = C.c_void_p(16)

@@ -329,3 +329,103 @@ def test_router_bf16_input_needs_workspace_on_tensor_cores():
                                 w.n_group, w.topk_group, w.k, w.route_scale, w.mask_mode,
                                 precision=mr.MR_PREC_BF16X3)
     assert e.value.status == mr.MR_ERR_UNSUPPORTED
+
+
+# --------------------------------------------------------------------------
+# Scoring variants of the DeepSeek-V3.2-Exp Gate (softmax scores without
+# renormalisation, largest-score group score, no 1e-20), on every path.
+
+VARIANTS = {
+    "softmax": (mr.MR_SCORE_SOFTMAX, dict(score="softmax")),
+    "group_max": (mr.MR_GROUP_MAX, dict(group_score="max")),
+    "no_eps": (mr.MR_NORM_NO_EPS, dict(eps=False)),
+    "v32_softmax_nobias": (mr.MR_SCORE_SOFTMAX | mr.MR_GROUP_MAX | mr.MR_NORM_NO_EPS,
+                           dict(score="softmax", group_score="max", eps=False)),
+}
+
+VAR_W = [
+    W("var_v3_T300", T=300, d=512, N_r=256, n_group=8, topk_group=4, k=8, route_scale=2.5,
+      mask_mode=0, seed=41),
+    W("var_k2_T260", T=260, d=256, N_r=384, n_group=1, topk_group=1, k=8, route_scale=2.827,
+      mask_mode=1, seed=42),
+    W("var_zero_mask_T200", T=200, d=256, N_r=128, n_group=4, topk_group=2, k=6, route_scale=2.5,
+      mask_mode=1, seed=43, bias_lo=-0.6, bias_hi=0.1),
+]
+
+
+def _variant_ref(w, tok, okw, no_bias):
+    d = router_inputs(w)
+    b = None if no_bias else d["b"]
+    return oracle.router(d["x_f32"][tok], d["W"], b, w.n_group, w.topk_group, w.k,
+                         w.route_scale, w.mask_mode, want_logits=True, **okw)
+
+
+def _variant_run(w, flags, rows, precision, no_bias, ws=True):
+    d = router_inputs(w)
+    x = to_dev(d["x_bf16"], "bf16") if rows == "bf16" else to_dev(d["x_f32"])
+    b = None if no_bias else to_dev(d["b"])
+    wsb = torch.empty(mr.mr_router_workspace_size(w.T, w.d, w.N_r), dtype=torch.uint8,
+                      device="cuda") if ws else None
+    lg = torch.full((w.T, w.N_r), float("nan"), device="cuda")
+    io, wo = _poisoned(w.T, w.k)
+    idx, wt = mr.mr_router_forward_ex(x, to_dev(d["W"]), b, w.n_group, w.topk_group, w.k,
+                                      w.route_scale, w.mask_mode, precision=precision,
+                                      idx_out=io, w_out=wo, logits_out=lg, workspace=wsb,
+                                      flags=flags)
+    assert mr.mr_get_error() == mr.MR_OK
+    return idx.cpu().numpy(), wt.cpu().numpy(), lg.cpu().numpy()
+
+
+@pytest.mark.parametrize("var", sorted(VARIANTS))
+@pytest.mark.parametrize("path", ["fused_bf16x3", "fused_3xtf32", "splitk_bf16", "ffma"])
+@pytest.mark.parametrize("w", VAR_W, ids=[w.name for w in VAR_W])
+def test_router_scoring_variants(w, path, var):
+    flags, okw = VARIANTS[var]
+    no_bias = var == "v32_softmax_nobias"
+    if path == "splitk_bf16":
+        w = w.replace(T=100)
+    tok = np.arange(w.T)
+    rows = "f32" if path in ("fused_3xtf32",) else "bf16"
+    prec = {"fused_bf16x3": mr.MR_PREC_BF16X3, "fused_3xtf32": mr.MR_PREC_3XTF32,
+            "splitk_bf16": mr.MR_PREC_BF16X3, "ffma": mr.MR_PREC_FFMA}[path]
+    if path == "ffma":
+        w = w.replace(T=96)
+        tok = np.arange(w.T)
+    idx, wt, lg = _variant_run(w, flags, rows, prec, no_bias, ws=path != "ffma")
+    ref = _variant_ref(w, tok, okw, no_bias)
+    # softmax scores are O(1/N_r), so the absolute 1e-5 near-tie band (made for
+    # O(1) sigmoid scores) holds a few percent of the tokens; they are still
+    # counted and excluded from the exact comparison only
+    tie_frac = 0.05 if okw.get("score") == "softmax" else 0.01
+    stats = compare_router(idx, wt, ref, lg, allow_tie_frac=tie_frac)
+    if var in ("softmax", "v32_softmax_nobias"):
+        assert (wt.sum(1) < w.route_scale).all()  # not renormalised
+    else:
+        np.testing.assert_allclose(wt.sum(1), w.route_scale, rtol=2e-6)
+    print(w.name, path, var, stats)
+
+
+@pytest.mark.parametrize("cs", ["1", "2", "P"])
+def test_router_softmax_every_tile_shape(cs, monkeypatch):
+    """Softmax needs each token's largest logit and sum of exponentials over
+    all experts: over the two column halves, and with CS = 2 over the two
+    CTAs that split the experts."""
+    monkeypatch.setenv("MR_TC_CLUSTER", cs)
+    w = VAR_W[0]
+    flags, okw = VARIANTS["softmax"]
+    idx, wt, lg = _variant_run(w, flags, "bf16", mr.MR_PREC_BF16X3, False)
+    compare_router(idx, wt, _variant_ref(w, np.arange(w.T), okw, False), lg, allow_tie_frac=0.05)
+
+
+def test_router_no_eps_underflow_gives_nan_like_the_page():
+    """Every chosen sigmoid score underflows to 0: with the 1e-20 the weights
+    are 0, without it 0/0 -- both as the oracle computes them."""
+    T, d, N = 4, 64, 64
+    x = torch.zeros((T, d), device="cuda")
+    x[:, 0] = 1.0
+    Wt = torch.zeros((N, d), device="cuda")
+    Wt[:, 0] = -1000.0
+    for flags, want_nan in ((0, False), (mr.MR_NORM_NO_EPS, True)):
+        _, wt = mr.mr_router_forward_ex(x, Wt, None, 1, 1, 4, 2.5, 0, flags=flags)
+        got = wt.cpu().numpy()
+        assert np.isnan(got).all() if want_nan else (got == 0).all()

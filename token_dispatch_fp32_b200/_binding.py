@@ -31,6 +31,9 @@ MR_PREC_3XTF32 = 0
 MR_PREC_TF32 = 1
 MR_PREC_FFMA = 2
 MR_PREC_BF16X3 = 3
+MR_SCORE_SOFTMAX = 1
+MR_GROUP_MAX = 2
+MR_NORM_NO_EPS = 4
 
 _lib = None
 
@@ -56,6 +59,8 @@ def lib():
         L.mr_router_forward.argtypes = [p, p, p, i, i, i, i, i, i, f, i, p, p, p]
         L.mr_router_forward_ex.argtypes = [p, i, p, p, i, i, i, i, i, i, f, i, i, p, p, p, p,
                                            sz, p]
+        L.mr_router_forward_ex2.argtypes = [p, i, p, p, i, i, i, i, i, i, f, i, i, i, p, p, p,
+                                            p, sz, p]
         L.mr_router_workspace_size.argtypes = [i, i, i]
         L.mr_router_workspace_size.restype = sz
         L.mr_dispatch_workspace_size.argtypes = [i, i, i]
@@ -144,9 +149,10 @@ def mr_router_workspace_size(T, d, N_r) -> int:
 
 def mr_router_forward_ex(x, W, bias, n_group, topk_group, k, route_scale, mask_mode,
                          precision=MR_PREC_3XTF32, idx_out=None, w_out=None, logits_out=None,
-                         workspace=None, stream=None):
+                         workspace=None, stream=None, flags=0):
     """mr_router_forward with x dtype (fp32 or bf16), precision, optional
-    logits output and workspace.  Returns (idx, w)."""
+    logits output and workspace; flags != 0 (MR_SCORE_SOFTMAX, MR_GROUP_MAX,
+    MR_NORM_NO_EPS) calls mr_router_forward_ex2.  Returns (idx, w)."""
     _need(x, "x")
     x_dtype = _row_dtype(x)
     T, d = x.shape
@@ -164,10 +170,16 @@ def mr_router_forward_ex(x, W, bias, n_group, topk_group, k, route_scale, mask_m
     if workspace is not None:
         _need(workspace, "workspace")
         ws_bytes = workspace.numel() * workspace.element_size()
-    _check("mr_router_forward_ex", lib().mr_router_forward_ex(
-        _ptr(x), x_dtype, _ptr(W), _ptr(bias), T, d, N_r, n_group, topk_group, k,
-        float(route_scale), mask_mode, precision, _ptr(idx_out), _ptr(w_out), _ptr(logits_out),
-        _ptr(workspace), ws_bytes, _stream(stream)))
+    if flags:
+        _check("mr_router_forward_ex2", lib().mr_router_forward_ex2(
+            _ptr(x), x_dtype, _ptr(W), _ptr(bias), T, d, N_r, n_group, topk_group, k,
+            float(route_scale), mask_mode, precision, int(flags), _ptr(idx_out), _ptr(w_out),
+            _ptr(logits_out), _ptr(workspace), ws_bytes, _stream(stream)))
+    else:
+        _check("mr_router_forward_ex", lib().mr_router_forward_ex(
+            _ptr(x), x_dtype, _ptr(W), _ptr(bias), T, d, N_r, n_group, topk_group, k,
+            float(route_scale), mask_mode, precision, _ptr(idx_out), _ptr(w_out),
+            _ptr(logits_out), _ptr(workspace), ws_bytes, _stream(stream)))
     return idx_out, w_out
 
 

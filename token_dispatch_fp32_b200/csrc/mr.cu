@@ -132,7 +132,8 @@ bool tc_shape_ok(const void* x, int x_dtype, const float* W, int d, int N_r) {
 template <int NJ, bool XBF16>
 int launch_ffma_nj(const void* x, const float* W, const float* bias, int T, int d, int N_r,
                    int n_group, int topk_group, int k, float route_scale, int mask_mode,
-                   int32_t* idx_out, float* w_out, float* logits_out, cudaStream_t st) {
+                   int flags, int32_t* idx_out, float* w_out, float* logits_out,
+                   cudaStream_t st) {
   const size_t smem = mr::ffma_smem_bytes(NJ);
   auto kern = mr::router_ffma_kernel<NJ, XBF16>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
@@ -140,19 +141,21 @@ int launch_ffma_nj(const void* x, const float* W, const float* bias, int T, int 
     return MR_ERR_CUDA;
   const unsigned grid = (unsigned)((T + mr::kFfmaTokens - 1) / mr::kFfmaTokens);
   kern<<<grid, mr::kFfmaThreads, smem, st>>>(x, W, bias, T, d, N_r, n_group, topk_group, k,
-                                              route_scale, mask_mode, idx_out, w_out, logits_out);
+                                              route_scale, mask_mode, flags, idx_out, w_out,
+                                              logits_out);
   return launch_status();
 }
 
 template <bool XBF16>
 int launch_ffma(const void* x, const float* W, const float* bias, int T, int d, int N_r,
-                int n_group, int topk_group, int k, float route_scale, int mask_mode,
+                int n_group, int topk_group, int k, float route_scale, int mask_mode, int flags,
                 int32_t* idx_out, float* w_out, float* logits_out, cudaStream_t st) {
   const int nj = (N_r + 31) / 32;
 #define MR_FFMA_CASE(NJV)                                                                       \
   if (nj <= NJV)                                                                              \
     return launch_ffma_nj<NJV, XBF16>(x, W, bias, T, d, N_r, n_group, topk_group, k,          \
-                                      route_scale, mask_mode, idx_out, w_out, logits_out, st);
+                                      route_scale, mask_mode, flags, idx_out, w_out,          \
+                                      logits_out, st);
   MR_FFMA_CASE(1)
   MR_FFMA_CASE(2)
   MR_FFMA_CASE(4)
@@ -244,8 +247,8 @@ bool splitk_applies(int T, int N_r) { return T > 0 && T <= kSplitKMaxT && N_r <=
 
 template <int NJ>
 int launch_reduce_nj(const float* part, int KS, int T, int N_r, const float* bias, int n_group,
-                     int topk_group, int k, float route_scale, int mask_mode, int32_t* idx_out,
-                     float* w_out, float* logits_out, cudaStream_t st) {
+                     int topk_group, int k, float route_scale, int mask_mode, int flags,
+                     int32_t* idx_out, float* w_out, float* logits_out, cudaStream_t st) {
   // programmatic dependent of the GEMM: launched while the GEMM drains, it
   // waits (griddepcontrol.wait) for the GEMM's results before reading them
   cudaLaunchConfig_t cfg = {};
@@ -260,7 +263,7 @@ int launch_reduce_nj(const float* part, int KS, int T, int N_r, const float* bia
   cfg.numAttrs = 1;
   const cudaError_t e = cudaLaunchKernelEx(&cfg, mr::sk::router_reduce_route_kernel<NJ>, part, KS,
                                            T, N_r, bias, n_group, topk_group, k, route_scale,
-                                           mask_mode, idx_out, w_out, logits_out);
+                                           mask_mode, flags, idx_out, w_out, logits_out);
   g_launches.fetch_add(1, std::memory_order_relaxed);
   if (e != cudaSuccess) {
     (void)cudaGetLastError();
@@ -271,8 +274,8 @@ int launch_reduce_nj(const float* part, int KS, int T, int N_r, const float* bia
 
 int launch_splitk(const void* x, bool x_bf16, const float* W, const float* bias, int T, int d,
                   int N_r, int n_group, int topk_group, int k, float route_scale, int mask_mode,
-                  bool use3x, int32_t* idx_out, float* w_out, float* logits_out, void* ws,
-                  int sms, cudaStream_t st) {
+                  int flags, bool use3x, int32_t* idx_out, float* w_out, float* logits_out,
+                  void* ws, int sms, cudaStream_t st) {
   const SplitKShape sh = splitk_shape(T, d, N_r, sms, x_bf16);
   const mr::sk::Plan plan = mr::sk::make_plan(sh.NT, (sh.KC + sh.KS - 1) / sh.KS, x_bf16);
   CUtensorMap mw, mx;
@@ -323,7 +326,7 @@ int launch_splitk(const void* x, bool x_bf16, const float* W, const float* bias,
 #define MR_RED_CASE(NJV)                                                                      \
   if (nj <= NJV)                                                                              \
     return launch_reduce_nj<NJV>(P.part, KSr, T, N_r, bias, n_group, topk_group, k,            \
-                                 route_scale, mask_mode, idx_out, w_out, logits_out, st);
+                                 route_scale, mask_mode, flags, idx_out, w_out, logits_out, st);
   MR_RED_CASE(2)
   MR_RED_CASE(4)
   MR_RED_CASE(8)
@@ -369,9 +372,9 @@ size_t planes_bytes(int d, int N_r) { return 3 * (size_t)N_r * (size_t)d * 2; }
 // x fp32 with tf32 arithmetic (use3x: 3xTF32), or x bf16 with W as three
 // bf16 planes (bf16x3, planes written into `ws` here).
 int launch_tc(const void* x, const float* W, const float* bias, int T, int d, int N_r,
-              int n_group, int topk_group, int k, float route_scale, int mask_mode, bool use3x,
-              bool bf16x3, int32_t* idx_out, float* w_out, float* logits_out, float* wlo,
-              void* ws, int sms, cudaStream_t st) {
+              int n_group, int topk_group, int k, float route_scale, int mask_mode, int flags,
+              bool use3x, bool bf16x3, int32_t* idx_out, float* w_out, float* logits_out,
+              float* wlo, void* ws, int sms, cudaStream_t st) {
   TcShape shp = tc_shape(T, N_r, sms, bf16x3);
   auto fits = [&](const TcShape& t) {
     const mr::tc::Plan p = mr::tc::make_plan(N_r / t.CS, bf16x3, t.pair);
@@ -421,6 +424,7 @@ int launch_tc(const void* x, const float* W, const float* bias, int T, int d, in
   P.topk_group = topk_group;
   P.k = k;
   P.mask_mode = mask_mode;
+  P.flags = flags;
   P.num_kc = (d + mr::tc::BK - 1) / mr::tc::BK;
   P.use3x = use3x ? 1 : 0;
   P.wlo = use_wlo ? 1 : 0;
@@ -432,7 +436,11 @@ int launch_tc(const void* x, const float* W, const float* bias, int T, int d, in
   P.w_out = w_out;
   P.logits_out = logits_out;
   const size_t smem = plan.total + 1024;
-  auto kern = pair ? mr::tc::router_tc_kernel<true> : mr::tc::router_tc_kernel<false>;
+  const bool sm = (flags & MR_SCORE_SOFTMAX) != 0;
+  auto kern = pair ? (sm ? mr::tc::router_tc_kernel<true, true>
+                         : mr::tc::router_tc_kernel<true, false>)
+                   : (sm ? mr::tc::router_tc_kernel<false, true>
+                         : mr::tc::router_tc_kernel<false, false>);
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
       cudaSuccess)
     return MR_ERR_CUDA;
@@ -490,11 +498,12 @@ size_t mr_router_workspace_size(int T, int d, int N_r) {
   return need;
 }
 
-int mr_router_forward_ex(const void* x, int x_dtype, const float* W, const float* bias, int T,
-                         int d, int N_r, int n_group, int topk_group, int k, float route_scale,
-                         int mask_mode, int precision, int32_t* idx_out, float* w_out,
-                         float* logits_out, void* workspace, size_t workspace_bytes,
-                         mr_stream_t stream) {
+int mr_router_forward_ex2(const void* x, int x_dtype, const float* W, const float* bias, int T,
+                          int d, int N_r, int n_group, int topk_group, int k, float route_scale,
+                          int mask_mode, int precision, int flags, int32_t* idx_out,
+                          float* w_out, float* logits_out, void* workspace,
+                          size_t workspace_bytes, mr_stream_t stream) {
+  if (flags & ~(MR_SCORE_SOFTMAX | MR_GROUP_MAX | MR_NORM_NO_EPS)) return MR_ERR_INVALID_ARG;
   int st = validate_router(x, x_dtype, W, T, d, N_r, n_group, topk_group, k, route_scale,
                            mask_mode, precision, idx_out, w_out);
   if (st != MR_OK || T == 0) return st;
@@ -504,9 +513,9 @@ int mr_router_forward_ex(const void* x, int x_dtype, const float* W, const float
   if (precision == MR_PREC_FFMA) {
     return x_dtype == MR_BF16
                ? launch_ffma<true>(x, W, bias, T, d, N_r, n_group, topk_group, k, route_scale,
-                                   mask_mode, idx_out, w_out, logits_out, s)
+                                   mask_mode, flags, idx_out, w_out, logits_out, s)
                : launch_ffma<false>(x, W, bias, T, d, N_r, n_group, topk_group, k, route_scale,
-                                    mask_mode, idx_out, w_out, logits_out, s);
+                                    mask_mode, flags, idx_out, w_out, logits_out, s);
   }
   // Small batches (decode): split-K over all SMs, fp32 W read directly, for
   // either row type (3xTF32; a bf16 row needs no residual).
@@ -515,7 +524,7 @@ int mr_router_forward_ex(const void* x, int x_dtype, const float* W, const float
       !(precision == MR_PREC_BF16X3 && x_dtype != MR_BF16) &&
       workspace_bytes >= splitk_shape(T, d, N_r, sms, x_dtype == MR_BF16).ws_bytes)
     return launch_splitk(x, x_dtype == MR_BF16, W, bias, T, d, N_r, n_group, topk_group, k,
-                         route_scale, mask_mode, precision != MR_PREC_TF32, idx_out, w_out,
+                         route_scale, mask_mode, flags, precision != MR_PREC_TF32, idx_out, w_out,
                          logits_out, workspace, sms, s);
   if (x_dtype == MR_BF16 || precision == MR_PREC_BF16X3) {
     // bf16 activations on tensor cores: W as three bf16 planes (workspace)
@@ -523,16 +532,26 @@ int mr_router_forward_ex(const void* x, int x_dtype, const float* W, const float
         !tc_shape_ok(x, MR_F32, W, d, N_r) || !workspace || !aligned16(workspace) ||
         workspace_bytes < planes_bytes(d, N_r))
       return MR_ERR_UNSUPPORTED;
-    return launch_tc(x, W, bias, T, d, N_r, n_group, topk_group, k, route_scale, mask_mode, true,
-                     true, idx_out, w_out, logits_out, nullptr, workspace, sms, s);
+    return launch_tc(x, W, bias, T, d, N_r, n_group, topk_group, k, route_scale, mask_mode, flags,
+                     true, true, idx_out, w_out, logits_out, nullptr, workspace, sms, s);
   }
   if (cc != 10 || !tc_shape_ok(x, x_dtype, W, d, N_r)) return MR_ERR_UNSUPPORTED;
   float* wlo = (workspace && aligned16(workspace) && workspace_bytes >= wlo_bytes(d, N_r))
                    ? static_cast<float*>(workspace)
                    : nullptr;
-  return launch_tc(x, W, bias, T, d, N_r, n_group, topk_group, k, route_scale, mask_mode,
+  return launch_tc(x, W, bias, T, d, N_r, n_group, topk_group, k, route_scale, mask_mode, flags,
                    precision == MR_PREC_3XTF32, false, idx_out, w_out, logits_out, wlo, nullptr,
                    sms, s);
+}
+
+int mr_router_forward_ex(const void* x, int x_dtype, const float* W, const float* bias, int T,
+                         int d, int N_r, int n_group, int topk_group, int k, float route_scale,
+                         int mask_mode, int precision, int32_t* idx_out, float* w_out,
+                         float* logits_out, void* workspace, size_t workspace_bytes,
+                         mr_stream_t stream) {
+  return mr_router_forward_ex2(x, x_dtype, W, bias, T, d, N_r, n_group, topk_group, k,
+                               route_scale, mask_mode, precision, 0, idx_out, w_out, logits_out,
+                               workspace, workspace_bytes, stream);
 }
 
 int mr_router_forward(const float* x, const float* W, const float* bias, int T, int d, int N_r,

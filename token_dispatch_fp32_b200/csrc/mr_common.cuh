@@ -41,6 +41,48 @@ __device__ __forceinline__ float mr_bf16_to_f32(uint16_t b) {
 }
 
 // ---------------------------------------------------------------------------
+// Scores and weights, with the scoring variants of the DeepSeek-V3.2-Exp
+// "Normalize weights" page (Gate.forward): MR_SCORE_SOFTMAX takes
+// s = softmax(L) over all experts and uses the scaled scores as weights
+// without renormalisation; otherwise s = sigmoid(L) and the weights are
+// renormalised by the sum of the k scores, + 1e-20 unless MR_NORM_NO_EPS.
+
+// Scores of the lane's experts e = lane + 32*j (0 past N_r).
+template <int NJ>
+__device__ __forceinline__ void mr_scores_warp(const float* __restrict__ L, int N_r, int flags,
+                                               float (&s)[NJ]) {
+  const int lane = threadIdx.x & 31;
+  if (flags & MR_SCORE_SOFTMAX) {
+    float mx = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < NJ; ++j)
+      if (lane + 32 * j < N_r) mx = fmaxf(mx, L[lane + 32 * j]);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    float sum = 0.0f;
+#pragma unroll
+    for (int j = 0; j < NJ; ++j) {
+      s[j] = lane + 32 * j < N_r ? __expf(L[lane + 32 * j] - mx) : 0.0f;
+      sum += s[j];
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+#pragma unroll
+    for (int j = 0; j < NJ; ++j) s[j] = s[j] / sum;
+  } else {
+#pragma unroll
+    for (int j = 0; j < NJ; ++j) s[j] = lane + 32 * j < N_r ? mr_sigmoid(L[lane + 32 * j]) : 0.0f;
+  }
+}
+
+// Weight of a chosen expert with score s_j; den = the sum of the k scores.
+__device__ __forceinline__ float mr_weight(float s_j, float den, float route_scale, int flags) {
+  if (flags & MR_SCORE_SOFTMAX) return s_j * route_scale;
+  if (!(flags & MR_NORM_NO_EPS)) den += 1e-20f;
+  return (s_j / den) * route_scale;
+}
+
+// ---------------------------------------------------------------------------
 // Warp-cooperative routing of one token from its N_r logits.
 //
 // Lane `l` owns experts e = l + 32*j, j < NJ (N_r <= 32*NJ).  Steps, in the
@@ -58,20 +100,19 @@ __device__ __forceinline__ void mr_route_token_warp(const float* __restrict__ L,
                                                     int n_group, int topk_group, int k,
                                                     float route_scale, int mask_mode,
                                                     int32_t* __restrict__ idx_out,
-                                                    float* __restrict__ w_out) {
+                                                    float* __restrict__ w_out, int flags = 0) {
   const int lane = threadIdx.x & 31;
   const int S = N_r / n_group;
   float s[NJ], m[NJ];
   int grp[NJ];
+  mr_scores_warp<NJ>(L, N_r, flags, s);
 #pragma unroll
   for (int j = 0; j < NJ; ++j) {
     const int e = lane + 32 * j;
     if (e < N_r) {
-      s[j] = mr_sigmoid(L[e]);
       m[j] = s[j] + (bias ? bias[e] : 0.0f);
       grp[j] = e / S;
     } else {
-      s[j] = 0.0f;
       m[j] = -INFINITY;
       grp[j] = -1;
     }
@@ -105,7 +146,7 @@ __device__ __forceinline__ void mr_route_token_warp(const float* __restrict__ L,
           a1 = b1;
         }
       }
-      if (lane == g) gs_mine = a1 + a2;
+      if (lane == g) gs_mine = (flags & MR_GROUP_MAX) ? a1 : a1 + a2;
     }
     uint32_t kept = 0;
     for (int r = 0; r < topk_group; ++r) {
@@ -162,10 +203,9 @@ __device__ __forceinline__ void mr_route_token_warp(const float* __restrict__ L,
     }
     den += bs;
   }
-  den += 1e-20f;
   if (lane < k) {
     idx_out[lane] = my_idx;
-    w_out[lane] = (my_s / den) * route_scale;
+    w_out[lane] = mr_weight(my_s, den, route_scale, flags);
   }
 }
 
@@ -190,25 +230,20 @@ __device__ __forceinline__ void mr_route_token_warp_fast(const float* __restrict
                                                          float route_scale, int mask_mode,
                                                          int32_t* __restrict__ idx_out,
                                                          float* __restrict__ w_out,
-                                                         float* scratch) {
+                                                         float* scratch, int flags = 0) {
   const int lane = threadIdx.x & 31;
   const int S = N_r / n_group;
   if (k > 32 || (n_group > 1 && (S % 32 != 0 || n_group > NJ))) {
     mr_route_token_warp<NJ>(L, bias, N_r, n_group, topk_group, k, route_scale, mask_mode,
-                            idx_out, w_out);
+                            idx_out, w_out, flags);
     return;
   }
   float s[NJ], m[NJ];
+  mr_scores_warp<NJ>(L, N_r, flags, s);
 #pragma unroll
   for (int j = 0; j < NJ; ++j) {
     const int e = lane + 32 * j;
-    if (e < N_r) {
-      s[j] = mr_sigmoid(L[e]);
-      m[j] = s[j] + (bias ? bias[e] : 0.0f);
-    } else {
-      s[j] = 0.0f;
-      m[j] = -INFINITY;
-    }
+    m[j] = e < N_r ? s[j] + (bias ? bias[e] : 0.0f) : -INFINITY;
   }
   if (n_group > 1) {
     const int jpg = S / 32;  // lane slots j per group: group of slot j is j / jpg
@@ -241,13 +276,14 @@ __device__ __forceinline__ void mr_route_token_warp_fast(const float* __restrict
     }
     uint32_t kept = 0;
 #pragma unroll
+    const bool gmax = (flags & MR_GROUP_MAX) != 0;
     for (int g = 0; g < NJ; ++g) {
       if (g < n_group) {
-        const float sg = a1[g] + a2[g];
+        const float sg = gmax ? a1[g] : a1[g] + a2[g];
         int rank = 0;
 #pragma unroll
         for (int o = 0; o < NJ; ++o) {
-          const float so = a1[o] + a2[o];
+          const float so = gmax ? a1[o] : a1[o] + a2[o];
           if (o < n_group && o != g) rank += (so > sg || (so == sg && o < g)) ? 1 : 0;
         }
         if (rank < topk_group) kept |= 1u << g;
@@ -280,7 +316,7 @@ __device__ __forceinline__ void mr_route_token_warp_fast(const float* __restrict
   }
   if (n > 32) {
     mr_route_token_warp<NJ>(L, bias, N_r, n_group, topk_group, k, route_scale, mask_mode,
-                            idx_out, w_out);
+                            idx_out, w_out, flags);
     return;
   }
   int base = 0;
@@ -308,10 +344,9 @@ __device__ __forceinline__ void mr_route_token_warp_fast(const float* __restrict
   float den = rank < k ? cs : 0.0f;
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) den += __shfl_xor_sync(0xffffffffu, den, off);
-  den += 1e-20f;
   if (rank < k) {
     idx_out[rank] = ci;
-    w_out[rank] = (cs / den) * route_scale;
+    w_out[rank] = mr_weight(cs, den, route_scale, flags);
   }
   __syncwarp();  // scratch may be reused by the caller's next token
 }

@@ -21,7 +21,7 @@ template <int NJ, bool XBF16>
 __global__ void __launch_bounds__(kFfmaThreads)
     router_ffma_kernel(const void* __restrict__ xv, const float* __restrict__ W,
                        const float* __restrict__ bias, int T, int d, int N_r, int n_group,
-                       int topk_group, int k, float route_scale, int mask_mode,
+                       int topk_group, int k, float route_scale, int mask_mode, int flags,
                        int32_t* __restrict__ idx_out, float* __restrict__ w_out,
                        float* __restrict__ logits_out) {
   constexpr int NP = 32 * NJ;       // padded expert count
@@ -97,7 +97,7 @@ __global__ void __launch_bounds__(kFfmaThreads)
     const long gt = t0 + tok;
     if (gt < T)
       mr_route_token_warp<NJ>(Ls + tok * LLD, bias, N_r, n_group, topk_group, k, route_scale,
-                              mask_mode, idx_out + gt * k, w_out + gt * k);
+                              mask_mode, idx_out + gt * k, w_out + gt * k, flags);
   }
 }
 

@@ -301,8 +301,9 @@ template <int NJ>
 __global__ void __launch_bounds__(256)
     router_reduce_route_kernel(const float* __restrict__ part, int KS, int T, int N_r,
                                const float* __restrict__ bias, int n_group, int topk_group, int k,
-                               float route_scale, int mask_mode, int32_t* __restrict__ idx_out,
-                               float* __restrict__ w_out, float* __restrict__ logits_out) {
+                               float route_scale, int mask_mode, int flags,
+                               int32_t* __restrict__ idx_out, float* __restrict__ w_out,
+                               float* __restrict__ logits_out) {
   __shared__ float L[32 * NJ];
   __shared__ float bs[32 * NJ];
   __shared__ float scratch[96];
@@ -322,7 +323,7 @@ __global__ void __launch_bounds__(256)
   __syncthreads();
   if (threadIdx.x < 32)
     mr_route_token_warp_fast<NJ>(L, bs, N_r, n_group, topk_group, k, route_scale, mask_mode,
-                                 idx_out + (long)t * k, w_out + (long)t * k, scratch);
+                                 idx_out + (long)t * k, w_out + (long)t * k, scratch, flags);
 }
 
 }  // namespace sk

@@ -76,6 +76,7 @@ struct Params {
   // stages its own x tile and half of W's rows, and keeps its own 128 tokens
   // x all N experts in its TMEM.
   int pair;
+  int flags;  // MR_SCORE_SOFTMAX | MR_GROUP_MAX | MR_NORM_NO_EPS
   float route_scale;
   const float* bias;
   int32_t* idx_out;
@@ -117,7 +118,7 @@ __host__ __device__ inline Plan make_plan(int NL, bool bf16x3 = false, bool pair
 // per column half, group top-2 pairs and top-8 lists of 128 tokens; followed
 // by the pass-2 candidate scratch (16 scores and 16 s per worker thread).
 __host__ __device__ inline uint32_t exchange_bytes(int G) {
-  return 4u * 2u * (2u * G * BM + 3u * kTopMax * BM);
+  return 4u * 2u * (2u * G * BM + 3u * kTopMax * BM + 2u * BM);
 }
 // Per-thread candidate buffer of the top-k scan (value, score, index):
 // kCandCap slots plus one slot that absorbs the stores of non-candidates.
@@ -458,7 +459,7 @@ struct Top8 {
 template <int MAXG>
 __device__ __forceinline__ void select_groups(int G, int topk_group, int k, int cs, uint32_t crank,
                                               const float* exA1, const float* exA2, int row,
-                                              uint32_t& kept, float& tau) {
+                                              bool gmax, uint32_t& kept, float& tau) {
   float ga1[MAXG], ga2[MAXG];
 #pragma unroll
   for (int g = 0; g < MAXG; ++g) {
@@ -490,12 +491,12 @@ __device__ __forceinline__ void select_groups(int G, int topk_group, int k, int 
 #pragma unroll
   for (int g = 0; g < MAXG; ++g) {
     if (g < G) {
-      const float sg = ga1[g] + ga2[g];
+      const float sg = gmax ? ga1[g] : ga1[g] + ga2[g];
       int rank = 0;
 #pragma unroll
       for (int o = 0; o < MAXG; ++o) {
         if (o < G && o != g) {
-          const float so = ga1[o] + ga2[o];
+          const float so = gmax ? ga1[o] : ga1[o] + ga2[o];
           rank += (so > sg || (so == sg && o < g)) ? 1 : 0;
         }
       }
@@ -508,7 +509,9 @@ __device__ __forceinline__ void select_groups(int G, int topk_group, int k, int 
   tau = (2 * topk_group >= k) ? t : -INFINITY;
 }
 
-template <bool PAIR>
+// SOFTMAX: the MR_SCORE_SOFTMAX instantiation (its two statistics passes and
+// cluster barriers are compiled out of the sigmoid kernel).
+template <bool PAIR, bool SOFTMAX>
 __global__ void __launch_bounds__(kThreads, 1)
     router_tc_kernel(const __grid_constant__ CUtensorMap map_x,
                      const __grid_constant__ CUtensorMap map_w,
@@ -838,6 +841,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       float* exV = exA2 + 2 * G * BM;                            // [2][8][BM]
       float* exS = exV + 2 * kTopMax * BM;                       // [2][8][BM]
       int* exI = reinterpret_cast<int*>(exS + 2 * kTopMax * BM); // [2][8][BM]
+      float* exM = reinterpret_cast<float*>(exI + 2 * kTopMax * BM);  // [2][BM] row max
+      float* exZ = exM + 2 * BM;                                 // [2][BM] sum of exp
+      constexpr bool softmax = SOFTMAX;
       float v[16], v2[16], bv[16];
       auto load_bias = [&](int c) {
         const float4* b4 = reinterpret_cast<const float4*>(bias_s + c * 16);
@@ -861,21 +867,73 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
 
-      // pass 1: s = sigmoid(L) back into TMEM; per-group top-2 of c = s + b
-      uint32_t kept = 0xffffffffu;
-      if (G > 1) {
-        for (int g = 0; g < G; ++g) {
-          exA1[(h * G + g) * BM + row] = -INFINITY;
-          exA2[(h * G + g) * BM + row] = -INFINITY;
+      // softmax scores need the row's largest logit and its sum of
+      // exponentials over all experts (both halves; with CS = 2 the peer's)
+      float smx = 0.0f, sinv = 1.0f;
+      if constexpr (softmax) {
+        float mx = -INFINITY;
+        if (ok)
+          for (int c = c_beg; c < c_end; c += 2) {
+            const int c2 = c + 1 < c_end ? c + 1 : c;
+            tmem_ld16x2(tmem_base + lane_off + (uint32_t)(c * 16),
+                        tmem_base + lane_off + (uint32_t)(c2 * 16), v, v2);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) mx = fmaxf(mx, fmaxf(v[i], v2[i]));
+          }
+        exM[h * BM + row] = mx;
+        workers_sync();
+        if (cs > 1) cluster_sync_all();  // softmax #a: row maxima visible
+        smx = fmaxf(exM[row], exM[BM + row]);
+        if (cs > 1) smx = fmaxf(smx, fmaxf(ld_peer_f32(&exM[row], crank ^ 1u),
+                                           ld_peer_f32(&exM[BM + row], crank ^ 1u)));
+        float z = 0.0f;
+        if (ok)
+          for (int c = c_beg; c < c_end; c += 2) {
+            const int c2 = c + 1 < c_end ? c + 1 : c;
+            tmem_ld16x2(tmem_base + lane_off + (uint32_t)(c * 16),
+                        tmem_base + lane_off + (uint32_t)(c2 * 16), v, v2);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) z += __expf(v[i] - smx);
+            if (c2 != c)
+#pragma unroll
+              for (int i = 0; i < 16; ++i) z += __expf(v2[i] - smx);
+          }
+        exZ[h * BM + row] = z;
+        workers_sync();
+        if (cs > 1) cluster_sync_all();  // softmax #b: partial sums visible
+        // the CTA that owns experts [0, NL) adds first: both CTAs of a
+        // cluster form the same sum
+        float zsum = exZ[row] + exZ[BM + row];
+        if (cs > 1) {
+          const float zp = ld_peer_f32(&exZ[row], crank ^ 1u) + ld_peer_f32(&exZ[BM + row], crank ^ 1u);
+          zsum = crank == 0 ? zsum + zp : zp + zsum;
         }
+        sinv = 1.0f / zsum;
+      }
+
+      // pass 1: s = sigmoid(L) (or softmax) back into TMEM; per-group top-2
+      // of c = s + b
+      uint32_t kept = 0xffffffffu;
+      if (G > 1 || softmax) {
+        if (G > 1)
+          for (int g = 0; g < G; ++g) {
+            exA1[(h * G + g) * BM + row] = -INFINITY;
+            exA2[(h * G + g) * BM + row] = -INFINITY;
+          }
         if (ok && c_beg < c_end) {
           float a1 = -INFINITY, a2 = -INFINITY;
           int g = (col0 + c_beg * 16) / S, next_b = (g + 1) * S;
           auto body1 = [&](int c, float(&x)[16]) {
             load_bias(c);
+            if constexpr (softmax) {
 #pragma unroll
-            for (int i = 0; i < 16; ++i) x[i] = mr_sigmoid(x[i]);
+              for (int i = 0; i < 16; ++i) x[i] = __expf(x[i] - smx) * sinv;
+            } else {
+#pragma unroll
+              for (int i = 0; i < 16; ++i) x[i] = mr_sigmoid(x[i]);
+            }
             tmem_st16(tmem_base + lane_off + (uint32_t)(c * 16), x);
+            if (G == 1) return;
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
               const int e = col0 + c * 16 + i;
@@ -902,8 +960,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (c2 != c) body1(c2, v2);
           }
           asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-          exA1[(h * G + g) * BM + row] = a1;
-          exA2[(h * G + g) * BM + row] = a2;
+          if (G > 1) {
+            exA1[(h * G + g) * BM + row] = a1;
+            exA2[(h * G + g) * BM + row] = a2;
+          }
         }
       }
       workers_sync();
@@ -914,10 +974,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       // the k-th best of all candidates is >= the smallest of them.
       float tau = -INFINITY;
       if (G > 1) {
+        const bool gmax = (P.flags & MR_GROUP_MAX) != 0;
         if (G <= 8)
-          select_groups<8>(G, P.topk_group, P.k, cs, crank, exA1, exA2, row, kept, tau);
+          select_groups<8>(G, P.topk_group, P.k, cs, crank, exA1, exA2, row, gmax, kept, tau);
         else
-          select_groups<kMaxGroups>(G, P.topk_group, P.k, cs, crank, exA1, exA2, row, kept, tau);
+          select_groups<kMaxGroups>(G, P.topk_group, P.k, cs, crank, exA1, exA2, row, gmax, kept,
+                                    tau);
       }
 
       // pass 2: top-8 of this half's masked scores.  A score enters only if
@@ -955,8 +1017,8 @@ __global__ void __launch_bounds__(kThreads, 1)
               next_b += S;
             }
             const bool keep = G == 1 || ((kept >> g) & 1u);
-            // with groups, pass 1 left s in TMEM; otherwise x holds logits
-            const float sv = G > 1 ? x[i] : mr_sigmoid(x[i]);
+            // pass 1 (groups or softmax) left s in TMEM; otherwise x holds logits
+            const float sv = (G > 1 || softmax) ? x[i] : mr_sigmoid(x[i]);
             const float cval = keep ? sv + bv[i] : (zero_fill ? 0.0f : -INFINITY);
             x[i] = sv;
             bv[i] = cval;
@@ -1024,12 +1086,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int j = 0; j < kTopMax; ++j)
             if (j < P.k) den += top.s[j];
-          den += 1e-20f;
 #pragma unroll
           for (int j = 0; j < kTopMax; ++j) {
             if (j < P.k) {
               P.idx_out[tok * P.k + j] = top.i[j];
-              P.w_out[tok * P.k + j] = (top.s[j] / den) * P.route_scale;
+              P.w_out[tok * P.k + j] = mr_weight(top.s[j], den, P.route_scale, P.flags);
             }
           }
         }
@@ -1038,12 +1099,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
-  // Threads that take no part in the routing epilogue still join its three
-  // cluster barriers, so a cluster always completes them.
+  // Threads that take no part in the routing epilogue still join its cluster
+  // barriers (three; five with softmax scores), so a cluster always completes
+  // them.
   if (P.CS > 1 && warp < 2) {
-    cluster_sync_all();
-    cluster_sync_all();
-    cluster_sync_all();
+    const int n_sync = SOFTMAX ? 5 : 3;
+    for (int i = 0; i < n_sync; ++i) cluster_sync_all();
   }
   tc_fence_before();
   __syncthreads();
