@@ -201,7 +201,9 @@ int mr_router_forward_ex2(const void *x, int x_dtype, const float *W,
                           mr_stream_t stream);
 
 /*
- * mr_dispatch_workspace_size -- bytes of device workspace mr_dispatch needs.
+ * mr_dispatch_workspace_size -- bytes of device workspace mr_dispatch needs:
+ * 16 + ceil(T*k / 1024) * N_r * 4 + N_r * 4 (a barrier word, per-chunk
+ * expert histograms, expert totals).
  */
 size_t mr_dispatch_workspace_size(int T, int k, int N_r);
 
@@ -220,6 +222,11 @@ size_t mr_dispatch_workspace_size(int T, int k, int N_r);
  *   inv_perm  [T*k] int32 or NULL: inv_perm[perm[i]] = i.
  *   workspace at least mr_dispatch_workspace_size(T, k, N_r) bytes; its
  *             contents need no initialisation.
+ * One cooperative kernel (histogram, per-expert chunk prefix, offsets and
+ * stable scatter, separated by two grid barriers whose waits are bounded)
+ * preceded by a 4-byte memset of the barrier word, when one CTA per
+ * 1024-entry chunk fits on the device at once; three kernels otherwise.
+ * Calls on different streams need different workspaces.
  * Limits: 1 <= N_r <= 1024, 1 <= k <= 32.
  * An id outside [0, N_r) is dropped: counts/offsets/perm cover the valid
  * entries only, perm[offsets[N_r] ..] and the dropped slots' inv_perm are -1,
@@ -246,10 +253,11 @@ int mr_dispatch(const int32_t *idx, int T, int k, int N_r, int32_t *counts,
  * libmr.so instead.
  *
  * Limits: everything mr_dispatch allows, and additionally
- * mr_dispatch_workspace_size(T, k, N_r) <= mr_dispatch_noalloc_max_workspace()
+ * ceil(T*k / 1024) * N_r * 4 <= mr_dispatch_noalloc_max_workspace()
  * (1 MiB: ceil(T*k / 1024) * N_r <= 262144, e.g. T*k up to 1,048,576 entries
  * at N_r = 256).  Larger sizes return MR_ERR_UNSUPPORTED before any launch;
- * use mr_dispatch with a workspace for them.
+ * use mr_dispatch with a workspace for them.  (It runs the three-kernel
+ * counting sort.)
  *
  * The fixed array: every GPU that loads libmr.so holds one 1 MiB copy until
  * the process exits.  The first call on a device looks up the array's device

@@ -98,7 +98,7 @@ def test_dispatch_validation():
     L = mr.lib()
     p = C.c_void_p(16)
     ws = L.mr_dispatch_workspace_size(100, 8, 256)
-    assert ws == 4 * 256  # one chunk of 1024 entries
+    assert ws == 16 + 4 * 256 + 4 * 256  # barrier word, one chunk of 1024 entries, totals
     assert L.mr_dispatch(p, 100, 0, 256, p, p, p, p, p, ws, None) == mr.MR_ERR_INVALID_ARG
     assert L.mr_dispatch(p, 100, 8, 0, p, p, p, p, p, ws, None) == mr.MR_ERR_INVALID_ARG
     assert L.mr_dispatch(p, 100, 8, 256, p, p, p, p, p, ws - 1, None) == mr.MR_ERR_INVALID_ARG

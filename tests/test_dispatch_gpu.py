@@ -1,5 +1,7 @@
 """Dispatch parity on the GPU: counts, offsets, perm and inv_perm bit-exact
-against the oracle (stable argsort reading of idxs = argsort(topk_ids))."""
+against the oracle (stable argsort reading of idxs = argsort(topk_ids)), for
+the one-launch cooperative kernel and, beyond what fits at once, the
+three-kernel counting sort."""
 import numpy as np
 import pytest
 import torch
@@ -41,6 +43,7 @@ CASES = [
     ("uniform", 5000, 32, 1024),            # largest k and N_r
     ("one_expert", 3000, 4, 64),            # every entry in one segment
     ("uniform", 64, 1, 1),
+    ("skewed", 200000, 8, 256),             # more chunks than fit at once: three kernels
 ]
 
 

@@ -180,4 +180,199 @@ __global__ void __launch_bounds__(kDispThreads)
   }
 }
 
+// ---------------------------------------------------------------------------
+// The same counting sort in ONE cooperative launch (every CTA resident):
+//   phase 1  CTA c histograms chunk c (as dispatch_count_kernel);
+//   barrier
+//   phase 2  CTA j owns experts [j*E, (j+1)*E): their totals, and each chunk's
+//            exclusive prefix within the expert's column (in place);
+//   barrier
+//   phase 3  every CTA scans the expert totals (offsets), CTA 0 writes counts,
+//            offsets and the dropped slots' -1, and CTA c scatters chunk c (as
+//            dispatch_scatter_kernel) from base offsets[e] + prefix[c][e].
+// The barrier counter lives in the workspace and is zeroed before the launch;
+// each wait is bounded (MR_WAIT_LIMIT_NS): a CTA that gives up raises
+// MR_FLAG_TIMEOUT and skips the remaining phases.
+struct DispFusedWs {
+  int* barrier;      // 1 int (zeroed by the host before the launch)
+  int32_t* hist;     // [nchunks][N_r]
+  int32_t* totals;   // [N_r]
+};
+
+__device__ __forceinline__ bool disp_grid_barrier(int* counter, int target) {
+  __shared__ int ok_s;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int ok = 1;
+    __threadfence();
+    atomicAdd(counter, 1);
+    uint64_t t0 = 0;
+    for (uint32_t it = 0;; ++it) {
+      int v;
+      asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(counter) : "memory");
+      if (v >= target) break;
+      if (it == 0) t0 = mr_globaltimer_ns();
+      if ((it & 63u) == 63u && mr_globaltimer_ns() - t0 > MR_WAIT_LIMIT_NS) {
+        mr_raise(MR_FLAG_TIMEOUT);
+        ok = 0;
+        break;
+      }
+      __nanosleep(64);
+    }
+    ok_s = ok;
+  }
+  __syncthreads();
+  return ok_s != 0;
+}
+
+__global__ void __launch_bounds__(kDispThreads)
+    dispatch_fused_kernel(const int32_t* __restrict__ idx, long n, int N_r, DispFusedWs ws,
+                          int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+                          int32_t* __restrict__ perm, int32_t* __restrict__ inv) {
+  extern __shared__ int sm[];  // max(kDispThreads, kDispWarps * N_r) ints, reused by the phases
+  __shared__ int start_s[kDispMaxExperts];
+  __shared__ int warp_tot[kDispWarps];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
+  const int nchunks = gridDim.x, c = blockIdx.x;
+  const long base = (long)c * kDispChunk + (long)warp * kDispSub;
+  bool bad = false;
+
+  // ---- phase 1: chunk histogram
+  for (int e = tid; e < N_r; e += kDispThreads) sm[e] = 0;
+  __syncthreads();
+  for (int r = 0; r < kDispSub; r += 32) {
+    const int e = disp_load(idx, base + r + lane, n, N_r, &bad);
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    if (e >= 0 && lane == __ffs(peers) - 1) atomicAdd(&sm[e], __popc(peers));
+  }
+  if (__any_sync(0xffffffffu, bad) && lane == 0) mr_raise(MR_FLAG_BAD_INDEX);
+  __syncthreads();
+  for (int e = tid; e < N_r; e += kDispThreads) ws.hist[(long)c * N_r + e] = sm[e];
+  if (!disp_grid_barrier(ws.barrier, nchunks)) return;
+
+  // ---- phase 2: this CTA's experts: totals and per-chunk exclusive prefix
+  {
+    const int E = (N_r + nchunks - 1) / nchunks;  // experts per CTA
+    const int e0 = c * E, e_end = e0 + E < N_r ? e0 + E : N_r;
+    if (E > kDispThreads / 2) {
+      // few chunks: one thread per expert, serial over the chunks
+      for (int e = e0 + tid; e < e_end; e += kDispThreads) {
+        int run = 0;
+        for (long cc = 0; cc < nchunks; ++cc) {
+          const int h = __ldcg(&ws.hist[cc * N_r + e]);
+          ws.hist[cc * N_r + e] = run;
+          run += h;
+        }
+        ws.totals[e] = run;
+      }
+    } else {
+      // Q >= 2 threads per expert, each a contiguous range of chunks
+      int Q = 1;
+      while (Q * 2 * E <= kDispThreads) Q *= 2;
+      const int el = tid % E, q = tid / E;
+      const int e = e0 + el;
+      const bool active = q < Q && e < e_end;
+      const long span = ((long)nchunks + Q - 1) / Q;
+      const long c_lo = active ? q * span : 0;
+      const long c_hi = active ? (c_lo + span < nchunks ? c_lo + span : nchunks) : 0;
+      int sum = 0;
+      for (long cc = c_lo; cc < c_hi; ++cc) sum += __ldcg(&ws.hist[cc * N_r + e]);
+      if (q < Q) sm[q * E + el] = sum;
+      __syncthreads();
+      if (active) {
+        int run = 0;
+        for (int qq = 0; qq < q; ++qq) run += sm[qq * E + el];
+        if (q == Q - 1) ws.totals[e] = run + sum;
+        for (long cc = c_lo; cc < c_hi; ++cc) {
+          const int h = __ldcg(&ws.hist[cc * N_r + e]);
+          ws.hist[cc * N_r + e] = run;
+          run += h;
+        }
+      }
+    }
+  }
+  if (!disp_grid_barrier(ws.barrier, 2 * nchunks)) return;
+
+  // ---- phase 3a: expert offsets (every CTA; exclusive scan of the totals)
+  {
+    constexpr int kPer = kDispMaxExperts / kDispThreads;  // 4
+    int v[kPer], loc = 0;
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      const int e = tid * kPer + j;
+      v[j] = e < N_r ? __ldcg(&ws.totals[e]) : 0;
+      loc += v[j];
+    }
+    int incl = loc;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += t;
+    }
+    if (lane == 31) warp_tot[warp] = incl;
+    __syncthreads();
+    int wex = 0;
+    for (int w = 0; w < warp; ++w) wex += warp_tot[w];
+    int run = wex + incl - loc;
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      const int e = tid * kPer + j;
+      if (e < N_r) {
+        start_s[e] = run;
+        if (c == 0) {
+          counts[e] = v[j];
+          offsets[e] = run;
+        }
+      }
+      run += v[j];
+    }
+    __syncthreads();
+    if (c == 0) {
+      int total = 0;
+      for (int w = 0; w < kDispWarps; ++w) total += warp_tot[w];
+      if (tid == 0) offsets[N_r] = total;
+      for (long i = total + tid; i < n; i += kDispThreads) perm[i] = -1;  // dropped slots
+    }
+  }
+
+  // ---- phase 3b: stable scatter of this chunk
+  int* wbase = sm;  // [kDispWarps][N_r]
+  for (int i = tid; i < kDispWarps * N_r; i += kDispThreads) wbase[i] = 0;
+  __syncthreads();
+  int* mine = wbase + warp * N_r;
+  for (int r = 0; r < kDispSub; r += 32) {
+    const int e = disp_load(idx, base + r + lane, n, N_r, &bad);
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    if (e >= 0 && lane == __ffs(peers) - 1) mine[e] += __popc(peers);
+    __syncwarp();
+  }
+  __syncthreads();
+  for (int e = tid; e < N_r; e += kDispThreads) {
+    int run = start_s[e] + __ldcg(&ws.hist[(long)c * N_r + e]);
+#pragma unroll
+    for (int w = 0; w < kDispWarps; ++w) {
+      const int h = wbase[w * N_r + e];
+      wbase[w * N_r + e] = run;
+      run += h;
+    }
+  }
+  __syncthreads();
+  const unsigned lt = (1u << lane) - 1u;
+  for (int r = 0; r < kDispSub; r += 32) {
+    const long i = base + r + lane;
+    const int e = disp_load(idx, i, n, N_r, &bad);
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    if (e >= 0) {
+      const int pos = mine[e] + __popc(peers & lt);
+      perm[pos] = (int32_t)i;
+      if (inv) inv[i] = pos;
+    } else if (i < n && inv) {
+      inv[i] = -1;
+    }
+    __syncwarp();
+    if (e >= 0 && lane == __ffs(peers) - 1) mine[e] += __popc(peers);
+    __syncwarp();
+  }
+}
+
 }  // namespace mr

@@ -569,9 +569,15 @@ int mr_router_forward(const float* x, const float* W, const float* bias, int T, 
 
 // ---- dispatch -----------------------------------------------------------------
 
+// Chunk histograms of the three-kernel dispatch: [nchunks][N_r] int32.
+size_t disp_hist_bytes(int T, int k, int N_r) {
+  return (size_t)mr::disp_num_chunks((long)T * k) * (size_t)N_r * sizeof(int32_t);
+}
+
 size_t mr_dispatch_workspace_size(int T, int k, int N_r) {
   if (T <= 0 || k <= 0 || N_r <= 0) return 0;
-  return (size_t)mr::disp_num_chunks((long)T * k) * (size_t)N_r * sizeof(int32_t);
+  // fused kernel: barrier counter (16 bytes), chunk histograms, expert totals
+  return 16 + disp_hist_bytes(T, k, N_r) + (size_t)N_r * sizeof(int32_t);
 }
 
 int mr_dispatch(const int32_t* idx, int T, int k, int N_r, int32_t* counts, int32_t* offsets,
@@ -592,6 +598,32 @@ int mr_dispatch(const int32_t* idx, int T, int k, int N_r, int32_t* counts, int3
   if (workspace_bytes < mr_dispatch_workspace_size(T, k, N_r)) return MR_ERR_INVALID_ARG;
   const long n = (long)T * k;
   const long nchunks = mr::disp_num_chunks(n);
+  int sms = 0, cc = 0;
+  if (!device_info(&sms, &cc)) return MR_ERR_CUDA;
+  // One cooperative launch when every chunk's CTA can be resident at once.
+  const size_t fsmem = sizeof(int) * std::max(mr::kDispThreads, mr::kDispWarps * N_r);
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, mr::dispatch_fused_kernel,
+                                                    mr::kDispThreads, fsmem) != cudaSuccess)
+    per_sm = 0;
+  if ((long)per_sm * sms >= nchunks) {
+    mr::DispFusedWs wsd;
+    wsd.barrier = static_cast<int*>(workspace);
+    wsd.hist = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + 16);
+    wsd.totals = wsd.hist + nchunks * N_r;
+    if (cudaMemsetAsync(wsd.barrier, 0, sizeof(int), s) != cudaSuccess) return MR_ERR_CUDA;
+    void* args[] = {const_cast<int32_t**>(&idx), const_cast<long*>(&n), &N_r, &wsd, &counts,
+                    &offsets, &perm, &inv_perm};
+    const cudaError_t e = cudaLaunchCooperativeKernel(
+        reinterpret_cast<const void*>(mr::dispatch_fused_kernel), dim3((unsigned)nchunks),
+        dim3(mr::kDispThreads), args, fsmem, s);
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    if (e != cudaSuccess) {
+      (void)cudaGetLastError();
+      return MR_ERR_CUDA;
+    }
+    return MR_OK;
+  }
   int32_t* hist = static_cast<int32_t*>(workspace);
   mr::dispatch_count_kernel<<<(unsigned)nchunks, mr::kDispThreads, sizeof(int) * N_r, s>>>(
       idx, n, N_r, hist);
@@ -639,7 +671,7 @@ int mr_dispatch_noalloc(const int32_t* idx, int T, int k, int N_r, int32_t* coun
   if ((long long)T * k >= (1LL << 31)) return MR_ERR_INVALID_ARG;
   if (k > 32 || N_r > mr::kDispMaxExperts) return MR_ERR_UNSUPPORTED;
   if (!counts || !offsets) return MR_ERR_INVALID_ARG;
-  if (mr_dispatch_workspace_size(T, k, N_r) > kNoAllocScratchBytes) return MR_ERR_UNSUPPORTED;
+  if (disp_hist_bytes(T, k, N_r) > kNoAllocScratchBytes) return MR_ERR_UNSUPPORTED;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (T == 0) {
     if (cudaMemsetAsync(counts, 0, sizeof(int32_t) * N_r, s) != cudaSuccess ||
