@@ -452,13 +452,17 @@ int launch_tc(const void* x, const float* W, const float* bias, int T, int d, in
   cfg.blockDim = dim3(mr::tc::kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = cluster;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  // programmatic dependent of the preceding kernel (the W split): the router
+  // CTAs set up while it runs, then wait for it (griddepcontrol.wait)
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, mx, mw, mwlo, P);
   if (e != cudaSuccess) {
     (void)cudaGetLastError();

@@ -550,6 +550,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                            : 2 * NL <= 256 ? 256 : 512;
 
   if (threadIdx.x == 0) {
+    // the descriptors live in the kernel parameters: fetch them during set-up
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_x)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_w)) : "memory");
+    if (P.wlo)
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_wlo))
+                   : "memory");
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(bar(B_FULL + s), 1);
       mbar_init(bar(B_CONV + s), kWorkers);  // one elected arrival per worker warp
@@ -581,6 +587,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   // pair: barriers must be initialised in both CTAs before any remote use
   if (pair) cluster_sync_all();
+  // Launched as a programmatic dependent: the set-up above overlaps the
+  // preceding kernel (W's planes or residuals); no global input is read
+  // before that grid has completed.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   for (int e = threadIdx.x; e < NL; e += kThreads)
     bias_s[e] = P.bias ? P.bias[col0 + e] : 0.0f;
   tc_fence_before();
@@ -1129,6 +1139,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 // residuals by TMA instead of each re-deriving them in shared memory.
 __global__ void __launch_bounds__(256) split_residual_kernel(const float4* __restrict__ W,
                                                              float4* __restrict__ Wlo, long n4) {
+  // the router grid (a programmatic dependent) may be scheduled now; it
+  // waits for this grid's completion before it reads anything
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   for (long i = blockIdx.x * 256L + threadIdx.x; i < n4; i += (long)gridDim.x * 256) {
     const float4 v = __ldg(W + i);
     float4 l;
@@ -1146,6 +1159,7 @@ __global__ void __launch_bounds__(256) split_residual_kernel(const float4* __res
 __global__ void __launch_bounds__(256) split_planes_kernel(const float* __restrict__ W,
                                                            __nv_bfloat16* __restrict__ planes,
                                                            long n) {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   for (long i = blockIdx.x * 256L + threadIdx.x; i < n; i += (long)gridDim.x * 256) {
     const float w = __ldg(W + i);
     const __nv_bfloat16 p1 = __float2bfloat16_rn(w);
