@@ -319,6 +319,19 @@ int mr_combine(const void *expert_out, int dtype, const float *w,
 uint64_t mr_launch_count(void);
 
 /*
+ * mr_selftest_bounded_wait -- exercises the failure path of the library's
+ * bounded waits without a GPU fault: one small kernel waits on something that
+ * nothing completes -- which = 0: an mbarrier phase (the wait of the
+ * tensor-core router kernels); which = 1: a grid barrier that only one of two
+ * CTAs reaches (the wait of the cooperative dispatch kernel).  The wait gives
+ * up after the library's limit (1 s), raises the device flag and the kernel
+ * returns; mr_get_error then reports MR_ERR_TIMEOUT and the context stays
+ * usable.  The pages have no counterpart to this entry point (it is a test
+ * hook).  Returns MR_ERR_INVALID_ARG for another `which`.
+ */
+int mr_selftest_bounded_wait(int which, mr_stream_t stream);
+
+/*
  * mr_get_error -- synchronise `stream`, then read and clear the current
  * device's sticky error flag.  Returns MR_OK, MR_ERR_DEVICE (a bad expert id
  * was seen), MR_ERR_TIMEOUT (a bounded wait inside a kernel gave up) or

@@ -118,3 +118,7 @@ def test_rows_validation():
     assert L.mr_combine(p, 1, None, p, None, p, 10, 64, 8, None) == mr.MR_ERR_INVALID_ARG
     assert L.mr_combine(p, 1, p, p, None, p, 10, 0, 8, None) == mr.MR_ERR_INVALID_ARG
     assert L.mr_combine(None, 1, None, None, None, None, 0, 64, 8, None) == mr.MR_OK
+
+
+def test_selftest_rejects_unknown_case():
+    assert mr.lib().mr_selftest_bounded_wait(7, None) == mr.MR_ERR_INVALID_ARG

@@ -71,6 +71,7 @@ def lib():
         L.mr_gather_rows.argtypes = [p, i, i, i, i, p, p, p, p]
         L.mr_combine.argtypes = [p, i, p, p, p, p, i, i, i, p]
         L.mr_get_error.argtypes = [p]
+        L.mr_selftest_bounded_wait.argtypes = [i, p]
         L.mr_launch_count.restype = C.c_uint64
         for fn in ("mr_router_forward", "mr_router_forward_ex", "mr_dispatch", "mr_dispatch_noalloc",
                    "mr_gather_rows", "mr_combine", "mr_get_error"):

@@ -472,9 +472,45 @@ int launch_tc(const void* x, const float* W, const float* bias, int T, int d, in
   return launch_status();
 }
 
+// Bounded-wait self test (see mr_selftest_bounded_wait).
+__global__ void selftest_mbar_wait_kernel() {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_s;
+  if (threadIdx.x == 0) {
+    abort_s = 0;
+    mr::tc::mbar_init(mr::tc::smem_u32(&bar), 1);  // nothing ever arrives
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    mr::tc::mbar_wait(mr::tc::smem_u32(&bar), 0, &abort_s);  // gives up, raises the flag
+  }
+}
+
+__global__ void selftest_grid_barrier_kernel(int* counter) {
+  // only CTA 0 arrives; its target counts two CTAs
+  if (blockIdx.x == 0) mr::disp_grid_barrier(counter, 2);
+}
+
 }  // namespace
 
 extern "C" {
+
+int mr_selftest_bounded_wait(int which, mr_stream_t stream) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (which == 0) {
+    selftest_mbar_wait_kernel<<<1, 32, 0, s>>>();
+    return launch_status();
+  }
+  if (which == 1) {
+    int* counter = nullptr;
+    if (cudaMallocAsync(&counter, sizeof(int), s) != cudaSuccess) return MR_ERR_CUDA;
+    if (cudaMemsetAsync(counter, 0, sizeof(int), s) != cudaSuccess) return MR_ERR_CUDA;
+    selftest_grid_barrier_kernel<<<1, 32, 0, s>>>(counter);
+    const int st = launch_status();
+    if (cudaFreeAsync(counter, s) != cudaSuccess) return MR_ERR_CUDA;
+    return st;
+  }
+  return MR_ERR_INVALID_ARG;
+}
+
 
 int mr_version(void) { return 100; }
 
