@@ -44,8 +44,9 @@ UNIT = "tokens/s"
 # source file it was built from; reported only while the source is unchanged.
 NCU_TRAFFIC = {
     # ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum on the full V3
-    # workload (T=16384): 2.12 GB read + 223.83 MB written per launch.
-    "combine": {"src": "d0f0dabc6a463fef", "bytes": 2.12e9 + 223.83e6},
+    # workload (T=16384), 64 CTAs per SM: 2.115 GB read + 223.80 MB written
+    # per launch.
+    "combine": {"src": "d0f0dabc6a463fef", "bytes": 2.115008768e9 + 223.802368e6},
 }
 
 

