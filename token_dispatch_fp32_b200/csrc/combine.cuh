@@ -70,7 +70,7 @@ __global__ void __launch_bounds__(kRowThreads)
         o = make_uint4(bf16x2_pack_rn(acc[0], acc[1]), bf16x2_pack_rn(acc[2], acc[3]),
                        bf16x2_pack_rn(acc[4], acc[5]), bf16x2_pack_rn(acc[6], acc[7]));
       }
-      y[t * nvec + v] = o;
+      st_stream(y + t * nvec + v, o);
     }
     __syncthreads();
   }
@@ -108,7 +108,7 @@ __global__ void __launch_bounds__(kRowThreads)
         acc.z += s.z;
         acc.w += s.w;
       }
-      y[t * nvec + v] = acc;
+      st_stream(y + t * nvec + v, acc);
     }
     __syncthreads();
   }

@@ -20,4 +20,15 @@ __device__ __forceinline__ uint16_t ld_stream<uint16_t>(const uint16_t* p) {
   return *p;
 }
 
+// Store of an output row that is not read again by this kernel: streaming
+// (evict-first) for the vector and word types.
+template <typename V>
+__device__ __forceinline__ void st_stream(V* p, const V& v) {
+  __stcs(p, v);
+}
+template <>
+__device__ __forceinline__ void st_stream<uint16_t>(uint16_t* p, const uint16_t& v) {
+  *p = v;
+}
+
 }  // namespace mr
