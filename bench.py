@@ -129,19 +129,21 @@ class Clocks:
 # ---------------------------------------------------------------------------
 # CPU oracle timing (the reported baseline and the reference arm)
 
-def _oracle_sample(w: wl.Workload, n_tok: int, inputs):
+def _oracle_sample(w: wl.Workload, n_tok: int, inputs, threads=0):
     """One pass of the oracle over n_tok tokens of the workload: router on
     their rows, dispatch of their k*n_tok assignments, gather and combine of
-    their rows.  Returns the seconds it took."""
+    their rows (threads = 0: every host thread).  Returns the seconds it
+    took."""
     import oracle
     x, W, b = inputs["x_f32"][:n_tok], inputs["W"], inputs["b"]
     rows = inputs["x_rows"][:n_tok]
     E, sh = inputs["E"][: n_tok * w.k], inputs["shared"][:n_tok]
     t0 = time.perf_counter()
-    r = oracle.router(x, W, b, w.n_group, w.topk_group, w.k, w.route_scale, w.mask_mode)
+    r = oracle.router(x, W, b, w.n_group, w.topk_group, w.k, w.route_scale, w.mask_mode,
+                      threads=threads)
     _, _, perm, inv = oracle.dispatch(r["idx"], w.N_r)
     oracle.gather(rows, w.k, perm)
-    oracle.combine(E, r["w"].astype(np.float32), inv, sh, w.k)
+    oracle.combine(E, r["w"].astype(np.float32), inv, sh, w.k, threads=threads)
     return time.perf_counter() - t0
 
 
@@ -153,7 +155,7 @@ def _oracle_inputs(w: wl.Workload, n_tok: int):
             "E": wl.gen_E(sub), "shared": wl.gen_shared(sub)}
 
 
-def cpu_baseline(w: wl.Workload, target_s=12.0):
+def cpu_baseline(w: wl.Workload, target_s=15.0):
     """The oracle on a bounded sample of the workload: passes over the same
     `cap` tokens until about target_s seconds of CPU work have run."""
     import oracle
@@ -163,10 +165,15 @@ def cpu_baseline(w: wl.Workload, target_s=12.0):
     n = int(min(cap, max(64, 64 * target_s / max(t, 1e-3))))
     passes = max(1, int(round(target_s / max(t * n / 64, 1e-3))))
     total = sum(_oracle_sample(w, n, inp) for _ in range(passes))
+    # the same oracle on one host thread, over a quarter of the sample
+    n1 = max(16, n // 4)
+    t1 = _oracle_sample(w, n1, inp, threads=1)
     return {"value": n * passes / total, "unit": UNIT, "cores": oracle.num_threads(),
             "kind": "oracle",
+            "value_single_thread": n1 / t1,
             "sample": f"{passes} pass(es) over {n} tokens of {w.name} through the fp64 oracle "
-                      f"(router, dispatch, gather, combine), {total:.1f} s"}
+                      f"(router, dispatch, gather, combine), {total:.1f} s; single thread: "
+                      f"{n1} tokens, {t1:.1f} s"}
 
 
 def run_reference(args, w: wl.Workload, rank: int):
