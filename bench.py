@@ -194,7 +194,8 @@ def run_reference(args, w: wl.Workload, rank: int):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": _config(w, extra={"sample_tokens_per_step": n}),
+        "config": _config(w, extra={"sample_tokens_per_step": n,
+                                    "router_precision": "fp64 oracle (CPU)"}),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.num_threads(),
                          "kind": "oracle",
                          "sample": f"{n} tokens of {w.name} per step (fp64 oracle: router, "
