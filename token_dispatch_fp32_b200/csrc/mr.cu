@@ -391,8 +391,8 @@ int launch_tc(const void* x, const float* W, const float* bias, int T, int d, in
   if (bf16x3) {
     const long n = (long)N_r * d;
     __nv_bfloat16* planes = static_cast<__nv_bfloat16*>(ws);
-    mr::tc::split_planes_kernel<<<(unsigned)std::min<long>((n + 255) / 256, (long)sms * 8), 256, 0,
-                                  st>>>(W, planes, n);
+    mr::tc::split_planes_kernel<<<(unsigned)std::min<long>((n / 8 + 255) / 256 + 1, (long)sms * 8),
+                                  256, 0, st>>>(W, planes, n);
     if (launch_status() != MR_OK) return MR_ERR_CUDA;
     if (!make_map_bf16(&mx, x, (uint64_t)T, (uint64_t)d, mr::tc::BM)) return MR_ERR_CUDA;
     if (!make_map_bf16(&mw, planes, 3 * (uint64_t)N_r, (uint64_t)d, pair ? NL / 2 : NL))

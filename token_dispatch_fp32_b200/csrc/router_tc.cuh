@@ -1156,19 +1156,44 @@ __global__ void __launch_bounds__(256) split_residual_kernel(const float4* __res
 // W -> three bf16 planes with W1 + W2 + W3 = W to within 2^-24 relative:
 // W1 = bf16(W), W2 = bf16(W - W1), W3 = bf16(W - W1 - W2) (round to nearest
 // even; each difference is exact in fp32).  Planes stacked as [3][N_r*d].
+__device__ __forceinline__ void split3(float w, __nv_bfloat16& p1, __nv_bfloat16& p2,
+                                       __nv_bfloat16& p3) {
+  p1 = __float2bfloat16_rn(w);
+  const float r1 = w - __bfloat162float(p1);
+  p2 = __float2bfloat16_rn(r1);
+  const float r2 = r1 - __bfloat162float(p2);
+  p3 = __float2bfloat16_rn(r2);
+}
+
+// Eight weights per thread (two 16-byte loads, one 16-byte store per plane)
+// when n % 8 == 0 and the pointers are 16-byte aligned; one otherwise.
 __global__ void __launch_bounds__(256) split_planes_kernel(const float* __restrict__ W,
                                                            __nv_bfloat16* __restrict__ planes,
                                                            long n) {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  const bool vec = (n % 8) == 0 && (reinterpret_cast<uintptr_t>(W) % 16) == 0 &&
+                   (reinterpret_cast<uintptr_t>(planes) % 16) == 0;
+  if (vec) {
+    const long n8 = n / 8;
+    for (long i = blockIdx.x * 256L + threadIdx.x; i < n8; i += (long)gridDim.x * 256) {
+      const float4 a = __ldg(reinterpret_cast<const float4*>(W) + 2 * i);
+      const float4 b = __ldg(reinterpret_cast<const float4*>(W) + 2 * i + 1);
+      const float w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+      __align__(16) __nv_bfloat16 p[3][8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) split3(w[e], p[0][e], p[1][e], p[2][e]);
+#pragma unroll
+      for (int pl = 0; pl < 3; ++pl)
+        reinterpret_cast<uint4*>(planes + pl * n)[i] = *reinterpret_cast<const uint4*>(p[pl]);
+    }
+    return;
+  }
   for (long i = blockIdx.x * 256L + threadIdx.x; i < n; i += (long)gridDim.x * 256) {
-    const float w = __ldg(W + i);
-    const __nv_bfloat16 p1 = __float2bfloat16_rn(w);
-    const float r1 = w - __bfloat162float(p1);
-    const __nv_bfloat16 p2 = __float2bfloat16_rn(r1);
-    const float r2 = r1 - __bfloat162float(p2);
+    __nv_bfloat16 p1, p2, p3;
+    split3(__ldg(W + i), p1, p2, p3);
     planes[i] = p1;
     planes[n + i] = p2;
-    planes[2 * n + i] = __float2bfloat16_rn(r2);
+    planes[2 * n + i] = p3;
   }
 }
 
