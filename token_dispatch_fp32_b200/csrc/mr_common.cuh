@@ -275,8 +275,8 @@ __device__ __forceinline__ void mr_route_token_warp_fast(const float* __restrict
       }
     }
     uint32_t kept = 0;
-#pragma unroll
     const bool gmax = (flags & MR_GROUP_MAX) != 0;
+#pragma unroll
     for (int g = 0; g < NJ; ++g) {
       if (g < n_group) {
         const float sg = gmax ? a1[g] : a1[g] + a2[g];

@@ -608,9 +608,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t tx = bf16x3 ? plan.hi_bytes
                                  : (uint32_t)(BM + (P.wlo ? 2 : 1) * NL) * BK * 4;
       int issued = 0;
-      for (int kc = 0; kc < KC; ++kc) {
-        const int s = kc % STAGES;
-        if (kc >= STAGES && !mbar_wait(bar(B_EMPTY + s), ((kc / STAGES) - 1) & 1, abort)) break;
+      // stage s of the ring and the parity ph of its current round, kept
+      // incrementally (no division by the run-time stage count per chunk)
+      int s = 0;
+      uint32_t ph = 0;
+      for (int kc = 0; kc < KC; ++kc, (++s == STAGES ? (s = 0, ph ^= 1u) : 0u)) {
+        if (kc >= STAGES && !mbar_wait(bar(B_EMPTY + s), ph ^ 1u, abort)) break;
         ++issued;
         const uint32_t base = smem0 + s * plan.stage_bytes;
         if constexpr (PAIR) {
@@ -653,13 +656,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait(bar(B_DRAIN), 0, abort, true);
     } else if (lane == 0) {
       const uint32_t idesc = bf16x3 ? make_idesc_bf16(NL, pair ? 2 * BM : BM) : make_idesc(NL);
-      for (int kc = 0; kc < KC; ++kc) {
-        const int s = kc % STAGES;
+      int s = 0;
+      uint32_t ph = 0;  // stage and round parity, kept incrementally
+      for (int kc = 0; kc < KC; ++kc, (++s == STAGES ? (s = 0, ph ^= 1u) : 0u)) {
         const int j = kc / kPromote, b = j & 1;
         const bool first = (kc % kPromote) == 0;
         if (first && j >= 2 && !mbar_wait(bar(B_ACCE + b), ((j >> 1) - 1) & 1, abort)) break;
-        if (!mbar_wait((P.use3x && !bf16x3) ? bar(B_CONV + s) : bar(B_FULL + s),
-                       (kc / STAGES) & 1, abort))
+        if (!mbar_wait((P.use3x && !bf16x3) ? bar(B_CONV + s) : bar(B_FULL + s), ph, abort))
           break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(b * NL);
@@ -778,10 +781,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const int n4a = (int)(plan.a_bytes / 16);  // the x part of [A | B]
     const int n4 = P.wlo ? n4a : (int)(plan.hi_bytes / 16);
-    for (int kc = 0; kc < KC && ok; ++kc) {
+    int s = 0;
+    uint32_t ph = 0;
+    for (int kc = 0; kc < KC && ok; ++kc, (++s == STAGES ? (s = 0, ph ^= 1u) : 0u)) {
       if (P.use3x && !bf16x3) {
-        const int s = kc % STAGES;
-        if (!mbar_wait(bar(B_FULL + s), (kc / STAGES) & 1, abort)) {
+        if (!mbar_wait(bar(B_FULL + s), ph, abort)) {
           ok = false;
           break;
         }
