@@ -119,7 +119,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar(B_ACC), 1);
     *abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
+  // The producer (thread 0) fills the whole ring before the block-wide
+  // barrier: the first loads are in flight while TMEM is being allocated.
+  const uint32_t tx = plan.a_bytes + (xb ? plan.xs_bytes : plan.b_bytes);
+  const int pre = NC < STAGES ? NC : STAGES;
+  auto issue = [&](int i) {
+    const int s = i % STAGES, kc = c_beg + i;
+    const uint32_t base = smem0 + s * plan.stage_bytes;
+    mbar_arrive_expect_tx(bar(B_FULL + s), tx);
+    tma_load_2d(base, &map_w, bar(B_FULL + s), kc * BK, mt * BM);
+    tma_load_2d(xb ? base + 2 * plan.hi_bytes : base + plan.a_bytes, &map_x, bar(B_FULL + s),
+                kc * BK, tt * NT);
+  };
+  if (threadIdx.x == 0)
+    for (int i = 0; i < pre; ++i) issue(i);
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      smem_u32(tmem_slot)),
@@ -135,17 +150,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     if (lane == 0) {
-      const uint32_t tx = plan.a_bytes + (xb ? plan.xs_bytes : plan.b_bytes);
-      int issued = 0;
-      for (int i = 0; i < NC; ++i) {
-        const int s = i % STAGES, kc = c_beg + i;
-        if (i >= STAGES && !mbar_wait(bar(B_EMPTY + s), ((i / STAGES) - 1) & 1, abort)) break;
+      int issued = pre;
+      for (int i = pre; i < NC; ++i) {
+        if (!mbar_wait(bar(B_EMPTY + i % STAGES), ((i / STAGES) - 1) & 1, abort)) break;
         ++issued;
-        const uint32_t base = smem0 + s * plan.stage_bytes;
-        mbar_arrive_expect_tx(bar(B_FULL + s), tx);
-        tma_load_2d(base, &map_w, bar(B_FULL + s), kc * BK, mt * BM);
-        tma_load_2d(xb ? base + 2 * plan.hi_bytes : base + plan.a_bytes, &map_x, bar(B_FULL + s),
-                    kc * BK, tt * NT);
+        issue(i);
       }
       for (int i = issued - STAGES < 0 ? 0 : issued - STAGES; i < issued; ++i)
         mbar_wait(bar(B_FULL + i % STAGES), (i / STAGES) & 1, abort, true);
@@ -251,11 +260,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t rank = cluster_rank();
     const int rows = NT / CL;  // tokens reduced by this CTA
     const float* red = reinterpret_cast<const float*>(smem);
-    // a CTA that gave up on a wait (abort flag) leaves no valid partial
-    for (int src = 0; src < CL; ++src)
-      ok = ok && __float_as_int(ld_peer_f32(reinterpret_cast<const float*>(
-                                                const_cast<const int*>(abort)),
-                                            (uint32_t)src)) == 0;
+    // a CTA that gave up on a wait (abort flag) leaves no valid partial; the
+    // CL flags are loaded together (independent remote loads), then combined
+    int fl[kCluster];
+#pragma unroll
+    for (int src = 0; src < kCluster; ++src)
+      fl[src] = src < CL ? __float_as_int(ld_peer_f32(
+                               reinterpret_cast<const float*>(const_cast<const int*>(abort)),
+                               (uint32_t)src))
+                         : 0;
+    int bad = 0;
+#pragma unroll
+    for (int src = 0; src < kCluster; ++src) bad |= fl[src];
+    ok = ok && bad == 0;
     for (int j = threadIdx.x; j < rows * (BM / 4); j += kThreads) {
       const int tl = (int)rank * rows + j / (BM / 4), el = (j % (BM / 4)) * 4;
       // CL == kCluster here: all loads in flight before the first add
@@ -294,11 +311,144 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// Shared state of route_token_cta.
+struct CtaRouteSmem {
+  float a1[8], a2[8];  // per-warp top-2 of the biased scores (distinct experts)
+  float tau;           // lower bound on the token's k-th best masked score
+  uint32_t kept;       // bit g: group g kept
+  int cnt[8];          // candidates per warp
+  float cm[32], cs[32];
+  int ci[32];
+};
+
+// Routing of one token by a CTA of 256 threads, thread e owning expert e
+// (N_r <= 256, sigmoid scores; groups that are whole warps, or no groups).
+// The steps and their order are those of mr_route_token_warp_fast, with the
+// per-lane loops of one warp spread over eight warps:
+//   * each warp reduces the top-2 pair of its 32 biased scores;
+//   * warp 0 merges the pairs of each group into its score (top-2 sum, or
+//     the best), keeps topk_group groups by counting the groups that beat
+//     each one (lower group on ties), and takes tau = the k-th best of the
+//     kept warps' pairs -- k distinct experts, so the token's k-th best
+//     masked score is >= tau;
+//   * the experts with masked score >= tau are compacted in expert order and
+//     each one's place is the number of candidates that beat it (value desc,
+//     index asc); the k best write their slots.
+// Returns false, having written nothing, when there are more than 32
+// candidates (ties at the 0.0 fill, or fewer than k finite pair values); the
+// caller then routes with the one-warp routine.  Every thread of the CTA
+// calls it (it synchronises the CTA).
+__device__ __forceinline__ bool route_token_cta(float Lv, const float* __restrict__ bs, int N_r,
+                                                int n_group, int topk_group, int k,
+                                                float route_scale, int mask_mode, int flags,
+                                                int32_t* __restrict__ idx_out,
+                                                float* __restrict__ w_out, CtaRouteSmem& sm) {
+  const int e = threadIdx.x, warp = e >> 5, lane = e & 31;
+  const bool valid = e < N_r;
+  const float s = valid ? mr_sigmoid(Lv) : 0.0f;
+  const float c = valid ? s + bs[e] : -INFINITY;
+  float a1 = c, a2 = -INFINITY;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    const float b1 = __shfl_xor_sync(0xffffffffu, a1, off);
+    const float b2 = __shfl_xor_sync(0xffffffffu, a2, off);
+    const float hi = fmaxf(a1, b1);
+    a2 = fmaxf(fminf(a1, b1), fmaxf(a2, b2));
+    a1 = hi;
+  }
+  if (lane == 0) {
+    sm.a1[warp] = a1;
+    sm.a2[warp] = a2;
+  }
+  __syncthreads();
+  const int nw = (N_r + 31) / 32;                           // warps that hold experts
+  const int q = n_group > 1 ? (N_r / n_group) / 32 : nw;    // warps per group
+  if (warp == 0) {
+    uint32_t kept = 1u;
+    if (n_group > 1) {
+      float g1 = -INFINITY, g2 = -INFINITY;
+      if (lane < n_group) {
+        for (int i = 0; i < q; ++i) {
+          const float b1 = sm.a1[lane * q + i], b2 = sm.a2[lane * q + i];
+          const float hi = fmaxf(g1, b1);
+          g2 = fmaxf(fminf(g1, b1), fmaxf(g2, b2));
+          g1 = hi;
+        }
+      }
+      const float gsc = (flags & MR_GROUP_MAX) ? g1 : g1 + g2;
+      int rank = 0;
+      for (int o = 0; o < n_group; ++o) {
+        const float so = __shfl_sync(0xffffffffu, gsc, o);
+        rank += (so > gsc || (so == gsc && o < lane)) ? 1 : 0;
+      }
+      kept = __ballot_sync(0xffffffffu, lane < n_group && rank < topk_group);
+    }
+    const int w = lane >> 1;
+    float v = -INFINITY;
+    if (lane < 2 * nw && ((kept >> (w / q)) & 1u)) v = (lane & 1) ? sm.a2[w] : sm.a1[w];
+    int r = 0;
+    for (int o = 0; o < 2 * nw; ++o) {
+      const float vo = __shfl_sync(0xffffffffu, v, o);
+      r += (vo > v || (vo == v && o < lane)) ? 1 : 0;
+    }
+    const uint32_t at = __ballot_sync(0xffffffffu, lane < 2 * nw && r == k - 1);
+    const float tau = at ? __shfl_sync(0xffffffffu, v, __ffs(at) - 1) : -INFINITY;
+    if (lane == 0) {
+      sm.kept = kept;
+      sm.tau = tau;
+    }
+  }
+  __syncthreads();
+  // fewer than k finite pair values: no bound, every expert is a candidate
+  if (sm.tau == -INFINITY && N_r > 32) return false;
+  const float fill = (mask_mode == MR_MASK_NEG_INF) ? -INFINITY : 0.0f;
+  const float m = !valid ? -INFINITY : ((sm.kept >> (warp / q)) & 1u) ? c : fill;
+  const bool cand = valid && m >= sm.tau;
+  const uint32_t bal = __ballot_sync(0xffffffffu, cand);
+  if (lane == 0) sm.cnt[warp] = __popc(bal);
+  __syncthreads();
+  int base = 0, n = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int ni = sm.cnt[i];
+    base += i < warp ? ni : 0;
+    n += ni;
+  }
+  if (n > 32) return false;  // the same n in every thread
+  if (cand) {
+    const int slot = base + __popc(bal & ((1u << lane) - 1u));
+    sm.cm[slot] = m;
+    sm.cs[slot] = s;
+    sm.ci[slot] = e;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    float cv = -INFINITY, cs = 0.0f;
+    int ci = 0x7fffffff, rank = 32;
+    if (lane < n) {
+      cv = sm.cm[lane];
+      cs = sm.cs[lane];
+      ci = sm.ci[lane];
+      rank = 0;
+      for (int o = 0; o < n; ++o) rank += mr_better(sm.cm[o], sm.ci[o], cv, ci) ? 1 : 0;
+    }
+    float den = rank < k ? cs : 0.0f;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) den += __shfl_xor_sync(0xffffffffu, den, off);
+    if (rank < k) {
+      idx_out[rank] = ci;
+      w_out[rank] = mr_weight(cs, den, route_scale, flags);
+    }
+  }
+  return true;
+}
+
 // One CTA per token: sum the KS partial logits of each expert in slice order,
-// then route the token with one warp.  Launched as a programmatic dependent of
-// the GEMM: it waits for that grid's results before reading them.
+// then route the token (route_token_cta where its shape allows, else one
+// warp).  Launched as a programmatic dependent of the GEMM: it waits for that
+// grid's results before reading them.
 template <int NJ>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 1)
     router_reduce_route_kernel(const float* __restrict__ part, int KS, int T, int N_r,
                                const float* __restrict__ bias, int n_group, int topk_group, int k,
                                float route_scale, int mask_mode, int flags,
@@ -307,10 +457,12 @@ __global__ void __launch_bounds__(256)
   __shared__ float L[32 * NJ];
   __shared__ float bs[32 * NJ];
   __shared__ float scratch[96];
+  __shared__ CtaRouteSmem rs;
   // the bias does not come from the GEMM: fetch it while the GEMM runs
   for (int e = threadIdx.x; e < N_r; e += blockDim.x) bs[e] = bias ? bias[e] : 0.0f;
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const int t = blockIdx.x;
+  float mine = 0.0f;  // the logit of expert threadIdx.x
   for (int e = threadIdx.x; e < N_r; e += blockDim.x) {
     float acc = 0.0f;
     const float* p = part + (long)t * N_r + e;
@@ -318,9 +470,15 @@ __global__ void __launch_bounds__(256)
 #pragma unroll 8
     for (int s = 0; s < KS; ++s) acc += p[s * stride];
     L[e] = acc;
+    if (e == (int)threadIdx.x) mine = acc;
     if (logits_out) logits_out[(long)t * N_r + e] = acc;
   }
   __syncthreads();
+  const bool cta = blockDim.x == 256 && N_r <= 256 && !(flags & MR_SCORE_SOFTMAX) &&
+                   (n_group == 1 || (N_r % n_group == 0 && (N_r / n_group) % 32 == 0));
+  if (cta && route_token_cta(mine, bs, N_r, n_group, topk_group, k, route_scale, mask_mode, flags,
+                             idx_out + (long)t * k, w_out + (long)t * k, rs))
+    return;
   if (threadIdx.x < 32)
     mr_route_token_warp_fast<NJ>(L, bs, N_r, n_group, topk_group, k, route_scale, mask_mode,
                                  idx_out + (long)t * k, w_out + (long)t * k, scratch, flags);
