@@ -212,6 +212,49 @@ def test_router_splitk_small_batches(w, rows):
         assert torch.equal(lf, logits)
 
 
+# Routing shapes of the decode reduce-and-route kernel: whole-CTA routing
+# with groups of 1, 2 and 4 warps or none, a partial last warp, a single warp,
+# and the cases that hand the token to the one-warp routine (the kept groups'
+# top-2 pairs give fewer than k values; ties at the 0.0 fill of masked
+# experts beat the bound).
+ROUTE_SHAPES = [
+    W("route_g4_two_warps_per_group", T=96, d=512, N_r=256, n_group=4, topk_group=2, k=8,
+      route_scale=2.5, mask_mode=0, seed=61),
+    W("route_g2_four_warps_per_group", T=96, d=512, N_r=256, n_group=2, topk_group=1, k=6,
+      route_scale=1.0, mask_mode=0, seed=62),
+    W("route_no_groups_N256_zero_fill", T=96, d=512, N_r=256, n_group=1, topk_group=1, k=8,
+      route_scale=2.827, mask_mode=1, seed=63),
+    W("route_no_groups_N208", T=96, d=512, N_r=208, n_group=1, topk_group=1, k=8,
+      route_scale=1.0, mask_mode=0, seed=64),
+    W("route_no_groups_N32", T=96, d=512, N_r=32, n_group=1, topk_group=1, k=4,
+      route_scale=1.0, mask_mode=0, seed=65),
+    W("route_g8_keep2_too_few_pairs", T=96, d=512, N_r=256, n_group=8, topk_group=2, k=8,
+      route_scale=2.5, mask_mode=0, seed=66),
+    W("route_zero_fill_negative_bias", T=96, d=512, N_r=256, n_group=8, topk_group=4, k=8,
+      route_scale=2.5, mask_mode=1, seed=67, bias_lo=-0.95, bias_hi=-0.8),
+]
+
+
+@pytest.mark.parametrize("w", ROUTE_SHAPES, ids=[w.name for w in ROUTE_SHAPES])
+def test_router_splitk_routing_shapes(w):
+    """Every token of each routing shape of the split-K path against the
+    oracle (expert sets exact outside near-ties, weights within tolerance)."""
+    d = router_inputs(w)
+    ws = torch.empty(mr.mr_router_workspace_size(w.T, w.d, w.N_r), dtype=torch.uint8,
+                     device="cuda")
+    logits = torch.full((w.T, w.N_r), float("nan"), device="cuda")
+    io, wo = _poisoned(w.T, w.k)
+    l0 = mr.mr_launch_count()
+    idx, wt = mr.mr_router_forward_ex(to_dev(d["x_f32"]), to_dev(d["W"]), to_dev(d["b"]),
+                                      w.n_group, w.topk_group, w.k, w.route_scale, w.mask_mode,
+                                      idx_out=io, w_out=wo, logits_out=logits, workspace=ws)
+    assert mr.mr_launch_count() - l0 == 2  # the split-K GEMM + reduce-and-route
+    assert mr.mr_get_error() == mr.MR_OK
+    ref = oracle_router(w, np.arange(w.T))
+    stats = compare_router(idx.cpu().numpy(), wt.cpu().numpy(), ref, logits.cpu().numpy())
+    print(w.name, stats)
+
+
 def test_router_workspace_for_large_batches_holds_w_planes():
     # three bf16 planes of W (which also covers W's fp32 tf32-residuals)
     assert mr.mr_router_workspace_size(4096, 7168, 256) == 3 * 2 * 7168 * 256
