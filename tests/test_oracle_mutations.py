@@ -35,6 +35,16 @@ MUTATIONS = {
     "softmax_not_shifted_sum": ("sum += exp(L[i] - mx);", "sum += exp(L[i]);"),
     "group_max_is_pair_sum": ("gs[g] = tmp[0];\n            else", "gs[g] = tmp[0] + tmp[1];\n            else"),
     "epsilon_always_added": ("    if (var.eps)\n        den += 1e-20;", "    den += 1e-20;"),
+    "one_group_too_few_kept": ("for (int r = topk_group; r < n_group; ++r) {",
+                               "for (int r = topk_group - 1; r < n_group; ++r) {"),
+    "margin_sign_flip": ("m_tok = ord[k - 1].v - ord[k].v;", "m_tok = ord[k].v - ord[k - 1].v;"),
+    "offsets_start_at_first_count": ("offsets[0] = 0;", "offsets[0] = counts[0];"),
+    "gather_token_is_slot_mod_k": ("long tok = perm[slot] / k;", "long tok = perm[slot] % k;"),
+    "combine_weights_reversed": ("acc += (double)w[t * k + j] * mo_load(E, dtype, row * d + c);",
+                                 "acc += (double)w[t * k + (k - 1 - j)] * "
+                                 "mo_load(E, dtype, row * d + c);"),
+    "combine_row_of_token_not_slot": ("long row = inv[t * k + j];", "long row = inv[t + j];"),
+    "final_sum_not_rounded": ("                if (dtype == 1) y = mo_round_bf16(y);\n", ""),
 }
 
 
@@ -52,4 +62,6 @@ def test_pins_catch_mutation(name, tmp_path):
     r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
                         os.path.join(ROOT, "tests", "test_oracle_pins.py")],
                        cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
-    assert r.returncode != 0, f"pins did not catch '{name}':\n{r.stdout[-2000:]}"
+    # exit status 1: a pin failed (not a crash, a usage error or no tests)
+    assert r.returncode == 1, (f"pins did not catch '{name}' (status {r.returncode}):\n"
+                               f"{r.stdout[-2000:]}")
