@@ -24,7 +24,8 @@
 // memory and writes them to part[ks / CL][token][expert].  A second cluster
 // barrier keeps every CTA's shared memory alive until its peers have read it.
 // router_reduce_route_kernel (launched as a programmatic dependent of the
-// GEMM) sums the KS / CL slices in order and routes every token with one warp.
+// GEMM) sums the KS / CL slices in order and routes each token with the whole
+// CTA (route_token_cta), or with one warp for the shapes that does not cover.
 #pragma once
 
 #include "router_tc.cuh"
