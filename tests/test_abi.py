@@ -4,6 +4,8 @@ host-side argument validation rejects bad calls before touching the GPU
 import ctypes as C
 import os
 import re
+import shutil
+import subprocess
 
 import pytest
 
@@ -31,10 +33,43 @@ def test_library_exports_every_declared_symbol():
         assert hasattr(lib, fn), fn
 
 
-def test_library_is_sm100a_and_has_no_oracle_dependency():
-    path = mr._binding.LIB_PATH
-    data = open(path, "rb").read()
-    assert b"liboracle" not in data and b"mo_router" not in data
+def test_library_has_no_oracle_dependency():
+    """The product library neither links the oracle nor carries its entry
+    points (ELF dynamic section and exported symbols)."""
+    lib = mr.lib()
+    for sym in ("mo_router", "mo_router2", "mo_dispatch", "mo_gather", "mo_combine"):
+        assert not hasattr(lib, sym), sym
+    readelf = shutil.which("readelf")
+    if readelf is None:
+        pytest.skip("readelf not available")
+    dyn = subprocess.run([readelf, "-d", mr._binding.LIB_PATH], capture_output=True, text=True,
+                         check=True).stdout
+    needed = re.findall(r"\(NEEDED\)\s+Shared library: \[([^\]]+)\]", dyn)
+    assert needed and not any("oracle" in n for n in needed), needed
+
+
+def header_parameter_counts():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    out = {}
+    for name, args in re.findall(r"\b(mr_[a-z0-9_]+)\s*\(([^;{]*?)\)\s*;", text):
+        args = " ".join(args.split())
+        out[name] = 0 if args in ("", "void") else len(args.split(","))
+    return out
+
+
+def test_binding_marshals_the_declared_arguments():
+    """Each ctypes prototype of the binding has as many arguments as the
+    header's declaration (an ABI drift would pass garbage, not fail)."""
+    lib = mr.lib()
+    counts = header_parameter_counts()
+    assert set(counts) == set(declared_functions())
+    for name, n in counts.items():
+        argtypes = getattr(lib, name).argtypes
+        if argtypes is None:
+            assert n == 0, f"{name}: {n} parameters declared, no prototype in the binding"
+        else:
+            assert len(argtypes) == n, f"{name}: header {n}, binding {len(argtypes)}"
 
 
 def test_version_and_status_strings():
