@@ -12,7 +12,8 @@ Default workload: the full DeepSeek-V3 routing + dispatch + combine batch
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-Multi-GPU (torchrun, one rank per GPU): every rank runs its own batch
+Multi-GPU (one rank per GPU, under torchrun, or started by this script when
+--gpus N > 1 is given without a launcher): every rank runs its own batch
 (replicas, weak scaling, no collective in the data path); value = all ranks'
 tokens / max-over-ranks device time.  --impl reference times the CPU oracle
 (rank 0 only) on a bounded sample of the same workload.
@@ -155,10 +156,45 @@ def _oracle_inputs(w: wl.Workload, n_tok: int):
             "E": wl.gen_E(sub), "shared": wl.gen_shared(sub)}
 
 
-def cpu_baseline(w: wl.Workload, target_s=15.0):
-    """The oracle on a bounded sample of the workload: passes over the same
-    `cap` tokens until about target_s seconds of CPU work have run."""
+def _router_check(w: wl.Workload, gpu_router):
+    """The oracle's router over every token of the workload (rank 0's batch),
+    timed, with its near-tie count and the GPU's selection compared outside
+    the near-ties (gpu_router = (idx, w) of the timed step)."""
     import oracle
+    d = wl.gen_router_inputs(w)
+    t0 = time.perf_counter()
+    r = oracle.router(d["x_f32"], d["W"], d["b"], w.n_group, w.topk_group, w.k, w.route_scale,
+                      w.mask_mode)
+    secs = time.perf_counter() - t0
+    m = r["margins"]
+    msel = np.minimum(m[:, 0], m[:, 1])
+    tie = (msel <= oracle.NEAR_TIE_EPS) & (msel > 0)
+    otie = tie | ((m[:, 2] <= oracle.NEAR_TIE_EPS) & (m[:, 2] > 0))
+    gidx, gw = gpu_router
+    ok = ~tie
+    bad = int((np.sort(gidx, 1) != np.sort(r["idx"], 1)).any(1)[ok].sum())
+    og, orr = np.argsort(gidx, 1, kind="stable"), np.argsort(r["idx"], 1, kind="stable")
+    wg = np.take_along_axis(gw.astype(np.float64), og, 1)[ok]
+    wr = np.take_along_axis(r["w"], orr, 1)[ok]
+    return {"tokens": int(w.T), "near_ties": int(tie.sum()), "order_ties": int(otie.sum()),
+            "selection_mismatches_outside_near_ties": bad,
+            "w_max_rel_outside_near_ties": float((np.abs(wg - wr) / np.abs(wr)).max()),
+            "eps": oracle.NEAR_TIE_EPS,
+            "source": "fp64 oracle router over every token of the benchmark batch, against "
+                      "the GPU's idx/w of the timed step"}, secs
+
+
+def cpu_baseline(w: wl.Workload, target_s=15.0, gpu_router=None):
+    """The oracle on a bounded sample of the workload: passes over the same
+    `cap` tokens until about target_s seconds of CPU work have run.  With
+    gpu_router, also the oracle's router over the whole batch (timed, with
+    the near-tie count and a check of the GPU's selection: "router_check")."""
+    import oracle
+    check = None
+    if gpu_router is not None:
+        check, secs = _router_check(w, gpu_router)
+        check["oracle_router_s"] = secs
+        check["oracle_router_tokens_per_s"] = w.T / secs
     cap = 2048
     inp = _oracle_inputs(w, cap)
     t = _oracle_sample(w, 64, inp)
@@ -168,12 +204,15 @@ def cpu_baseline(w: wl.Workload, target_s=15.0):
     # the same oracle on one host thread, over a quarter of the sample
     n1 = max(16, n // 4)
     t1 = _oracle_sample(w, n1, inp, threads=1)
-    return {"value": n * passes / total, "unit": UNIT, "cores": oracle.num_threads(),
-            "kind": "oracle",
-            "value_single_thread": n1 / t1,
+    out = {"value": n * passes / total, "unit": UNIT, "cores": oracle.num_threads(),
+           "kind": "oracle",
+           "value_single_thread": n1 / t1,
             "sample": f"{passes} pass(es) over {n} tokens of {w.name} through the fp64 oracle "
                       f"(router, dispatch, gather, combine), {total:.1f} s; single thread: "
                       f"{n1} tokens, {t1:.1f} s"}
+    if check is not None:
+        out["router_check"] = check
+    return out
 
 
 def run_reference(args, w: wl.Workload, rank: int):
@@ -341,30 +380,92 @@ def run_ours(args, w: wl.Workload, rank: int, world: int):
     stage_ms = {n: float(np.mean([e[j].elapsed_time(e[j + 1]) for e in evs]))
                 for j, n in enumerate(names)}
     assert mr.mr_get_error(stream) == mr.MR_OK
-
-    # For reference, the router on the fp32 cast of the same rows (3xTF32),
-    # timed alone outside the step.
-    alt_ms = None
-    if bf16_rows:
-        for _ in range(3):
-            router(x32, mr.MR_PREC_3XTF32)
-        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        n_alt = max(5, min(50, args.steps))
-        a0.record(stream)
-        for _ in range(n_alt):
-            router(x32, mr.MR_PREC_3XTF32)
-        a1.record(stream)
-        torch.cuda.synchronize(dev)
-        alt_ms = a0.elapsed_time(a1) / n_alt
+    step_router_out = (idx.cpu().numpy(), wt.cpu().numpy())  # checked by the oracle leg
 
     ms_max = max_over_ranks(ms, world, dev)
 
-    # The decode-size router (one position x batch 64), timed alone: W read
-    # once per call by the split-K kernel over all SMs, then reduce-and-route.
+    # ---- router variants and other router shapes, each timed alone ----------
+    # Between timed calls a read pass over a buffer of 4x the L2 leaves the L2
+    # holding clean lines of that buffer, so every call reads its inputs from
+    # HBM without paying for dirty-line write-backs.
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    flush.fill_(1)
+    flush_i32 = flush.view(torch.int32)
+
+    def read_flush():
+        with torch.cuda.stream(stream):
+            flush_i32.sum(dtype=torch.int64)
+
+    def write_flush():
+        with torch.cuda.stream(stream):
+            flush.fill_(1)
+
+    def time_alone(fn, n, flush_fn=read_flush):
+        """Mean device time (ms) of fn() on the stream over n calls, each
+        after flush_fn (events bracket fn alone)."""
+        for _ in range(3):
+            fn()
+        tot = 0.0
+        for _ in range(n):
+            if flush_fn is not None:
+                flush_fn()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            e1.synchronize()
+            tot += e0.elapsed_time(e1)
+        return tot / n
+
+    n_alone = max(10, min(50, args.steps))
+    # The router on the fp32 cast of the same rows: 3xTF32 (three tf32
+    # products) and plain TF32 (one product, reported separately).
+    alt_ms = tf32_ms = None
+    if bf16_rows:
+        alt_ms = time_alone(lambda: router(x32, mr.MR_PREC_3XTF32), n_alone, None)
+        tf32_ms = time_alone(lambda: router(x32, mr.MR_PREC_TF32), n_alone, None)
+
+    # The DeepSeek-V3 and Kimi K2 prefill routers (4096 and 8192 tokens), in
+    # the benchmark's arithmetic (bf16 rows, bf16x3), timed alone.
+    other_routers = {}
+    if args.workload == wl.V3_FULL.name and not args.no_extra_stages:
+        for key, wo in (("router_deepseek_v3_prefill_T4096", wl.V3_PREFILL),
+                        ("router_kimi_k2_prefill_T8192", wl.K2_PREFILL)):
+            oin = wl.gen_router_inputs(wo)
+            ox = torch.from_numpy(oin["x_bf16"]).view(torch.bfloat16).to(dev)
+            oW = torch.from_numpy(oin["W"]).to(dev)
+            ob = torch.from_numpy(oin["b"]).to(dev)
+            oidx = torch.empty((wo.T, wo.k), dtype=torch.int32, device=dev)
+            owt = torch.empty((wo.T, wo.k), dtype=torch.float32, device=dev)
+            ows = torch.empty(max(4, mr.mr_router_workspace_size(wo.T, wo.d, wo.N_r)),
+                              dtype=torch.uint8, device=dev)
+
+            def orouter(wo=wo, ox=ox, oW=oW, ob=ob, oidx=oidx, owt=owt, ows=ows):
+                mr.mr_router_forward_ex(ox, oW, ob, wo.n_group, wo.topk_group, wo.k,
+                                        wo.route_scale, wo.mask_mode,
+                                        precision=mr.MR_PREC_BF16X3, idx_out=oidx, w_out=owt,
+                                        workspace=ows, stream=stream)
+
+            oms = time_alone(orouter, n_alone)
+            of = 2.0 * wo.T * wo.d * wo.N_r
+            other_routers[key] = {"workload": wo.name, "ms": oms,
+                                  "tflops_algorithmic": of / (oms / 1e3) / 1e12,
+                                  "tflops_issued": 3 * of / (oms / 1e3) / 1e12,
+                                  "l2": "read pass over 512 MB before each call"}
+            del ox, oW, ob, oidx, owt, ows
+        assert mr.mr_get_error(stream) == mr.MR_OK
+
+    # The decode-size router (one position x batch 64): W read once per call.
+    # Main figure: the plain entry point with the config's fp32 rows (split-K
+    # over all SMs + reduce-and-route, no workspace).  Beside it: bf16 rows
+    # through mr_router_forward_ex, a CUDA-graph replay, and the same call after
+    # a write flush (dirty L2 lines) instead of a read pass.
     decode = None
     if args.workload == wl.V3_FULL.name:
         wd = wl.V3_DECODE
         dd_in = wl.gen_router_inputs(wd)
+        dx32 = torch.from_numpy(dd_in["x_f32"]).to(dev)
         dx = torch.from_numpy(dd_in["x_bf16"]).view(torch.bfloat16).to(dev)
         dW = torch.from_numpy(dd_in["W"]).to(dev)
         db = torch.from_numpy(dd_in["b"]).to(dev)
@@ -372,60 +473,52 @@ def run_ours(args, w: wl.Workload, rank: int, world: int):
         dwt = torch.empty((wd.T, wd.k), dtype=torch.float32, device=dev)
         dws = torch.empty(max(4, mr.mr_router_workspace_size(wd.T, wd.d, wd.N_r)),
                           dtype=torch.uint8, device=dev)
-        flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)  # > L2
 
-        def dstep():
+        def dplain():
+            mr.mr_router_forward(dx32, dW, db, wd.n_group, wd.topk_group, wd.k, wd.route_scale,
+                                 wd.mask_mode, idx_out=didx, w_out=dwt, stream=stream)
+
+        def dbf16():
             mr.mr_router_forward_ex(dx, dW, db, wd.n_group, wd.topk_group, wd.k, wd.route_scale,
                                     wd.mask_mode, precision=mr.MR_PREC_BF16X3, idx_out=didx,
                                     w_out=dwt, workspace=dws, stream=stream)
 
-        for _ in range(5):
-            dstep()
         n_dec = 100
-        tot = 0.0
-        for _ in range(n_dec):  # W comes from HBM every call: L2 flushed between calls
-            with torch.cuda.stream(stream):
-                flush.fill_(1)
-            d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            d0.record(stream)
-            dstep()
-            d1.record(stream)
-            d1.synchronize()
-            tot += d0.elapsed_time(d1)
-        dus = tot / n_dec * 1e3
-        # the same call replayed from a CUDA graph (no per-launch host work)
+        l0 = mr.mr_launch_count()
+        dplain()
+        dlaunch = mr.mr_launch_count() - l0
+        dus = time_alone(dplain, n_dec) * 1e3
+        dus_write = time_alone(dplain, n_dec, write_flush) * 1e3
+        bus = time_alone(dbf16, n_dec) * 1e3
         gus, gerr = None, None
         try:
             graph = torch.cuda.CUDAGraph()
             with torch.cuda.graph(graph, stream=stream):
-                dstep()
-            for _ in range(3):
-                graph.replay()
-            torch.cuda.synchronize(dev)
-            gt = 0.0
-            for _ in range(n_dec):
-                with torch.cuda.stream(stream):
-                    flush.fill_(1)
-                    g0 = torch.cuda.Event(enable_timing=True)
-                    g1 = torch.cuda.Event(enable_timing=True)
-                    g0.record(stream)
+                dplain()
+            def replay():
+                with torch.cuda.stream(stream):  # replay on the timed stream
                     graph.replay()
-                    g1.record(stream)
-                g1.synchronize()
-                gt += g0.elapsed_time(g1)
-            gus = gt / n_dec * 1e3
+
+            gus = time_alone(replay, n_dec) * 1e3
             del graph
         except Exception as ex:  # report, do not fail the bench
             gerr = f"{type(ex).__name__}: {ex}"[:200]
-        dbytes = 4 * wd.N_r * wd.d + 2 * wd.T * wd.d + 4 * wd.N_r + 8 * wd.T * wd.k
-        decode = {"workload": wd.name, "us": dus, "launches_per_call": 2,
+        dbytes = 4 * wd.N_r * wd.d + 4 * wd.T * wd.d + 4 * wd.N_r + 8 * wd.T * wd.k
+        bbytes = 4 * wd.N_r * wd.d + 2 * wd.T * wd.d + 4 * wd.N_r + 8 * wd.T * wd.k
+        decode = {"workload": wd.name, "entry_point": "mr_router_forward (fp32 rows)",
+                  "us": dus, "launches_per_call": int(dlaunch),
                   "algorithmic_bytes": dbytes, "gbs": dbytes / (dus * 1e-6) / 1e9,
                   "us_cuda_graph": gus,
                   "gbs_cuda_graph": dbytes / (gus * 1e-6) / 1e9 if gus else None,
-                  "l2": "flushed before every call (256 MB write)"}
+                  "us_after_write_flush": dus_write,
+                  "us_bf16_rows_ex": bus,
+                  "gbs_bf16_rows_ex": bbytes / (bus * 1e-6) / 1e9,
+                  "l2": "read pass over 512 MB before every call (us_after_write_flush: "
+                        "a 512 MB write instead)"}
         if gerr:
             decode["cuda_graph_error"] = gerr
         assert mr.mr_get_error(stream) == mr.MR_OK
+    del flush, flush_i32
 
     # ---- end to end: pinned host inputs -> device -> path -> host result ----
     e2e = None
@@ -479,8 +572,16 @@ def run_ours(args, w: wl.Workload, rank: int, world: int):
     bytes_combine = T * (rb * k * dd + 2 * rb * dd + 8 * k)   # E rows, shared, y, w, inv
     bytes_gather = T * (rb * dd + rb * k * dd + 4 * k)        # x row once, k copies, inv
     bytes_router = T * (rb * dd + 8 * k) + 4 * N * dd + 4 * N  # x, idx/w, W, bias
+    bytes_dispatch = T * k * (4 + 12)                         # idx in; perm, inv, ~scan out
     flops_router = 2.0 * T * dd * N
     comb_s = stage_ms["combine"] / 1e3
+    # Roofline of the whole step: each stage's bound time at the measured
+    # peaks (router: the slower of its bytes at HBM bandwidth and its
+    # algorithmic flops at the bf16 tensor peak), summed, over the step time.
+    hbm = peaks["hbm_gbs"] * 1e9
+    bound_us = {"router": 1e6 * max(bytes_router / hbm, flops_router / (peaks["bf16_tflops"] * 1e12)),
+                "dispatch": 1e6 * bytes_dispatch / hbm, "gather": 1e6 * bytes_gather / hbm,
+                "combine": 1e6 * bytes_combine / hbm}
     achieved = bytes_combine / comb_s / 1e9
     traffic = None
     ent = NCU_TRAFFIC.get("combine")
@@ -501,14 +602,34 @@ def run_ours(args, w: wl.Workload, rank: int, world: int):
                    "issue_peak_kind": "bf16 dense (measured)" if bf16_rows
                                       else "tf32 dense = 0.5 x measured bf16",
                    "frac_issued_of_peak": 3 * flops_router / r_s / 1e12 / issue_peak,
+                   "frac_algorithmic_of_bf16_peak":
+                       flops_router / r_s / 1e12 / peaks["bf16_tflops"],
                    "gbs": bytes_router / r_s / 1e9},
-        "dispatch": {"ms": stage_ms["dispatch"]},
+        "dispatch": {"ms": stage_ms["dispatch"],
+                     "gbs": bytes_dispatch / (stage_ms["dispatch"] / 1e3) / 1e9},
         "gather": {"ms": stage_ms["gather"],
                    "gbs": bytes_gather / (stage_ms["gather"] / 1e3) / 1e9,
                    "frac_hbm": bytes_gather / (stage_ms["gather"] / 1e3) / 1e9 / peaks["hbm_gbs"]},
         "combine": {"ms": stage_ms["combine"], "gbs": achieved,
                     "frac_hbm": achieved / peaks["hbm_gbs"]},
     }
+    tf32_peak = 0.5 * peaks["bf16_tflops"]
+    if alt_ms is not None:
+        stages["router_3xtf32_fp32_rows"] = {
+            "ms": alt_ms, "tflops_issued": 3 * flops_router / (alt_ms / 1e3) / 1e12,
+            "issue_peak_tflops": tf32_peak, "issue_peak_kind": "tf32 dense = 0.5 x bf16",
+            "frac_issued_of_peak": 3 * flops_router / (alt_ms / 1e3) / 1e12 / tf32_peak}
+    if tf32_ms is not None:
+        stages["router_tf32_fp32_rows"] = {
+            "ms": tf32_ms, "arithmetic": "plain TF32: one tf32 product per multiply-add, "
+                                         "fp32 accumulation (logits within ~1e-3 relative)",
+            "tflops": flops_router / (tf32_ms / 1e3) / 1e12, "peak_tflops": tf32_peak,
+            "peak_kind": "tf32 dense = 0.5 x bf16",
+            "frac_of_peak": flops_router / (tf32_ms / 1e3) / 1e12 / tf32_peak}
+    for key, st in other_routers.items():
+        st["frac_issued_of_bf16_peak"] = st["tflops_issued"] / peaks["bf16_tflops"]
+        st["frac_algorithmic_of_bf16_peak"] = st["tflops_algorithmic"] / peaks["bf16_tflops"]
+        stages[key] = st
     if decode is not None:
         decode["frac_hbm"] = decode["gbs"] / peaks["hbm_gbs"]
         if decode.get("gbs_cuda_graph"):
@@ -526,18 +647,48 @@ def run_ours(args, w: wl.Workload, rank: int, world: int):
                      "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
                      "traffic": traffic, "algorithmic_bytes": bytes_combine,
                      "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json hbm_gbs)"
-                     if peaks["source"] == "measured" else "fallback 6650 GB/s"},
+                     if peaks["source"] == "measured" else "fallback 6650 GB/s",
+                     "step_frac": sum(bound_us.values()) / (ms_max * 1e3),
+                     "step_bound_us": bound_us,
+                     "step_frac_note": "sum of the stages' roofline times at the measured "
+                                       "peaks (router: max of HBM bytes and algorithmic flops "
+                                       "at the bf16 peak) / ms_per_step"},
         "stages": stages,
         "gpu_launches": int(launches),
         "clocks": clk,
         "e2e": e2e,
     }
     if world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(w)
+        line["cpu_baseline"] = cpu_baseline(w, gpu_router=step_router_out)
+        line["near_ties"] = line["cpu_baseline"].pop("router_check")
     print(json.dumps(line), flush=True)
 
 
-def main():
+def _free_port() -> int:
+    import socket
+    with socket.socket(socket.AF_INET, socket.SOCK_STREAM) as so:
+        so.bind(("127.0.0.1", 0))
+        return so.getsockname()[1]
+
+
+def _spawned_rank(rank: int, argv, world: int, port: int):
+    """Entry of a rank started by spawn_ranks: the launcher's environment
+    (RANK, LOCAL_RANK, WORLD_SIZE, MASTER_ADDR, MASTER_PORT), then main()."""
+    os.environ.update({"RANK": str(rank), "LOCAL_RANK": str(rank), "WORLD_SIZE": str(world),
+                       "MASTER_ADDR": "127.0.0.1", "MASTER_PORT": str(port)})
+    main(argv)
+
+
+def spawn_ranks(argv, world: int):
+    """`--gpus N` without a launcher: start N ranks here (one process per
+    GPU, spawn start method), each with the environment torchrun would give
+    it, and wait for them; a failing rank fails the run."""
+    import torch.multiprocessing as tmp
+    tmp.start_processes(_spawned_rank, args=(argv, world, _free_port()), nprocs=world,
+                        join=True, start_method="spawn")
+
+
+def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
@@ -546,12 +697,23 @@ def main():
     ap.add_argument("--workload", default=wl.V3_FULL.name, choices=[x.name for x in wl.ALL])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    args = ap.parse_args()
+    ap.add_argument("--no-extra-stages", action="store_true",
+                    help="skip the prefill-router stages timed beside the step")
+    args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.gpus < 1:
+        ap.error("--gpus must be >= 1")
     w = wl.BY_NAME[args.workload]
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        spawn_ranks(sys.argv[1:] if argv is None else argv, args.gpus)
+        return
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
+    if world != args.gpus:
+        print(f"bench.py: --gpus {args.gpus} but WORLD_SIZE={world}; launch one rank per GPU "
+              f"(torchrun --nproc-per-node {args.gpus}) or drop the launcher", file=sys.stderr)
+        sys.exit(2)
     if args.impl == "reference":
         run_reference(args, w, rank)
         return

@@ -22,8 +22,10 @@
  *
  * Conventions shared by every entry point
  *  - All tensor pointers are caller-owned DEVICE pointers on the current
- *    device, row-major and densely packed.  The library never allocates,
- *    frees or synchronises (except mr_get_error, which must read the device).
+ *    device, row-major and densely packed.  The library never allocates
+ *    device memory, frees or synchronises (except mr_get_error, which must
+ *    read the device); its only device memory is a few fixed arrays in its
+ *    own image, named below where they are used.
  *  - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy stream) and
  *    runs asynchronously.  Arguments are validated on the host before any
  *    launch; an invalid call launches nothing and returns a negative status.
@@ -33,7 +35,10 @@
  *    trap: the kernel skips the entry and raises the sticky device flag that
  *    mr_get_error() reports and clears.
  *  - No exceptions cross the ABI.  Calls on different streams are
- *    independent; the only shared state is that per-device error flag.
+ *    independent, except for the per-device state named where it is used:
+ *    the error flag, the split-K array of mr_router_forward (ordered across
+ *    streams by the library) and the scratch array of mr_dispatch_noalloc
+ *    (ordered by the caller).
  */
 #ifndef MR_H
 #define MR_H
@@ -135,13 +140,35 @@ const char *mr_status_string(int status);
  * P pins how CTAs share the work of a 128-token tile (testing only): one CTA
  * with all experts, two CTAs splitting the experts, or (bf16x3) two CTAs
  * running one 256-token tensor-core MMA.
- * Needs no workspace.  Returns MR_OK or a negative status (nothing launched
- * on an argument error).
+ *
+ * The kernels are picked by T, with no workspace argument:
+ *  - T > 256: one fused kernel (GEMM + routing in its epilogue; the logits
+ *    never leave the SM).
+ *  - T <= 256 (decode): the split-K path -- a K-sliced GEMM over all SMs
+ *    whose slices are summed in clusters, then a reduce-and-route kernel (two
+ *    launches) -- when its partial logits fit the library's fixed array of
+ *    mr_router_forward_max_scratch() bytes (2 MiB; e.g. every T <= 256 at
+ *    d = 7168, N_r = 256); otherwise the fused kernel.  That array is part of
+ *    libmr.so's device image: every GPU that loads the library holds one copy
+ *    until the process exits, and this entry point allocates nothing.  All
+ *    calls on a device share it; the library orders them across streams (each
+ *    use waits on the previous use's event and records its own), except while
+ *    `stream` is being captured into a CUDA graph, where it adds no
+ *    dependency: the caller then orders the graph's launches against other
+ *    small-batch calls of this entry point on that device.  The first call on
+ *    a device looks up the array's address and creates the event.
+ * The results are the same 3xTF32 arithmetic on either path, summed in a
+ * fixed order (deterministic).
+ * Returns MR_OK or a negative status (nothing launched on an argument error).
  */
 int mr_router_forward(const float *x, const float *W, const float *bias, int T,
                       int d, int N_r, int n_group, int topk_group, int k,
                       float route_scale, int mask_mode, int32_t *idx_out,
                       float *w_out, mr_stream_t stream);
+
+/* Size in bytes of the fixed array mr_router_forward keeps its split-K
+ * partial logits in (no counterpart on the pages). */
+size_t mr_router_forward_max_scratch(void);
 
 /*
  * mr_router_workspace_size -- bytes of device workspace that
@@ -199,6 +226,41 @@ int mr_router_forward_ex2(const void *x, int x_dtype, const float *W,
                           int32_t *idx_out, float *w_out, float *logits_out,
                           void *workspace, size_t workspace_bytes,
                           mr_stream_t stream);
+
+/*
+ * mr_router_forward_bf16w -- the gate with its weight stored in bf16.
+ *
+ * The Kimi K2 "Normalize weights" page's MoEGate.forward casts the stored
+ * gate weight to fp32 at use (self.weight.type(torch.float32) inside
+ * F.linear): the weight may be kept in a narrower type and the logits are
+ * still fp32 dot products.  Here W is kept in bf16 -- half the bytes of the
+ * decode-time weight read -- and the method is otherwise that of
+ * mr_router_forward_ex2 on the widened (exact) fp32 values of W.
+ *
+ *   x          [T, d] rows: MR_BF16 (tensor cores) or MR_F32 (CUDA cores).
+ *   W_bf16     [N_r, d] bf16 gate weight (bit patterns, nn.Linear layout).
+ *   flags      as mr_router_forward_ex2.
+ *   workspace  optional, mr_router_workspace_size(T, d, N_r) bytes: with it,
+ *              or with NULL and the batch's partials within
+ *              mr_router_forward_max_scratch() (the array mr_router_forward
+ *              uses, shared and ordered the same way), batches of up to 256
+ *              bf16 rows take the split-K path (two launches); larger batches
+ *              take the fused kernel (one launch, no workspace).
+ * Arithmetic: bf16 rows x bf16 W on the tensor cores (tcgen05 kind::f16, one
+ * product per multiply-add, each exact in fp32, fp32 accumulation): the fp32
+ * logits of the widened operands up to summation order, so the tolerances of
+ * the fp32 path hold against the oracle fed the widened W.  fp32 rows, or
+ * shapes the tensor-core kernels do not take (d % 8, N_r % 16 or, above 256,
+ * N_r % 32 nonzero): CUDA-core FMA on the widened W.
+ * Limits and errors as mr_router_forward_ex2.
+ */
+int mr_router_forward_bf16w(const void *x, int x_dtype, const void *W_bf16,
+                            const float *bias, int T, int d, int N_r,
+                            int n_group, int topk_group, int k,
+                            float route_scale, int mask_mode, int flags,
+                            int32_t *idx_out, float *w_out, float *logits_out,
+                            void *workspace, size_t workspace_bytes,
+                            mr_stream_t stream);
 
 /*
  * mr_dispatch_workspace_size -- bytes of device workspace mr_dispatch needs:
@@ -261,8 +323,9 @@ int mr_dispatch(const int32_t *idx, int T, int k, int N_r, int32_t *counts,
  *
  * The fixed array: every GPU that loads libmr.so holds one 1 MiB copy until
  * the process exits.  The first call on a device looks up the array's device
- * address (once per device, with that device current), so make that first
- * call before capturing a stream into a CUDA graph.  The entry point itself
+ * address with that device current (cudaGetSymbolAddress) and keeps it; a
+ * lookup that fails returns MR_ERR_CUDA and is tried again by the next call.
+ * Make that first call before capturing a stream into a CUDA graph.  The entry point itself
  * calls no cudaMalloc, cudaFree or other allocating routine.  All calls on a
  * device share the one array, and it keeps whatever the last call left in
  * it: nothing in it needs to start at zero (each call rewrites every entry it
@@ -276,6 +339,36 @@ int mr_dispatch_noalloc(const int32_t *idx, int T, int k, int N_r,
 
 /* Size in bytes of the fixed scratch array mr_dispatch_noalloc uses. */
 size_t mr_dispatch_noalloc_max_workspace(void);
+
+/*
+ * mr_ep_recv_order -- receive-side order of the expert-parallel exchange
+ * (Kimi K2 "Add shared output" page, moe_infer, ep_size > 1: the labels
+ * gatherd_idxs of the received rows, their argsort, and
+ * tokens_per_expert_post_gather).
+ *
+ * With ep ranks, rank r owns experts [r*E_loc, (r+1)*E_loc).  After the row
+ * all-to-all it holds R rows, source by source, each source's rows in that
+ * source's expert-sorted order.
+ *   recv_counts    [ep, E_loc] int32 (device): recv_counts[s][e] = rows from
+ *                  source s for local expert e (the all_to_all_single of
+ *                  tokens_per_expert).
+ *   R              the sum of recv_counts (the rows received).
+ *   order          [R] int32: order[j] = the received row that goes j-th when
+ *                  the rows are sorted by local expert (stable: by source,
+ *                  then the source's order) -- sorted = received[order],
+ *                  e.g. mr_gather_rows(received, k = 1, perm = order).
+ *   inv_order      [R] int32 or NULL: inv_order[order[j]] = j -- the
+ *                  scatter-back new_x[gatherd_idxs] = outs is
+ *                  mr_gather_rows(outs, k = 1, inv_perm = order).
+ *   local_counts   [E_loc] int32: rows per local expert.
+ *   local_offsets  [E_loc + 1] int32: their exclusive prefix.
+ * One kernel, no sort (the stable order has a closed form per segment).
+ * Limits: ep * E_loc <= 1024.  A negative count or a sum other than R writes
+ * nothing and raises the device flag (MR_ERR_DEVICE from mr_get_error).
+ */
+int mr_ep_recv_order(const int32_t *recv_counts, int ep, int E_loc, int R,
+                     int32_t *order, int32_t *inv_order, int32_t *local_counts,
+                     int32_t *local_offsets, mr_stream_t stream);
 
 /*
  * mr_gather_rows -- sorted_tokens = x[idxs // k] (Kimi K2 "Add shared output"
@@ -326,8 +419,11 @@ uint64_t mr_launch_count(void);
  * CTAs reaches (the wait of the cooperative dispatch kernel).  The wait gives
  * up after the library's limit (1 s), raises the device flag and the kernel
  * returns; mr_get_error then reports MR_ERR_TIMEOUT and the context stays
- * usable.  The pages have no counterpart to this entry point (it is a test
- * hook).  Returns MR_ERR_INVALID_ARG for another `which`.
+ * usable.  The grid-barrier case counts arrivals in a word of the library's
+ * device image (cleared by the kernel), so the call allocates nothing; two
+ * self tests of that kind running at once would share the word.  The pages
+ * have no counterpart to this entry point (it is a test hook).  Returns
+ * MR_ERR_INVALID_ARG for another `which`.
  */
 int mr_selftest_bounded_wait(int which, mr_stream_t stream);
 

@@ -55,6 +55,8 @@ def _load():
                                    C.c_int, C.c_double, C.c_int, C.c_int, C.c_int, C.c_int,
                                    p, p, p, p, C.c_int]
         lib.mo_dispatch.argtypes = [p, C.c_int, C.c_int, C.c_int, p, p, p, p]
+        lib.mo_ep_splits.argtypes = [p, C.c_int, C.c_int, C.c_int, p, p, p]
+        lib.mo_ep_recv_order.argtypes = [p, C.c_int, C.c_int, p, p]
         lib.mo_gather.argtypes = [p, C.c_long, C.c_int, C.c_int, p, p, C.c_long, p]
         lib.mo_round_bf16.argtypes = [C.c_double]
         lib.mo_round_bf16.restype = C.c_double
@@ -141,6 +143,46 @@ def dispatch(idx, N_r):
     return counts, offsets, perm, inv
 
 
+def ep_splits(counts_all, r):
+    """Expert-parallel bookkeeping of rank r (Kimi K2 "Add shared output"
+    page, moe_infer, ep_size > 1: tokens_per_ep_rank, the all_to_all_single
+    of tokens_per_expert, output_splits).  counts_all [ep, N_r]: every rank's
+    tokens_per_expert; rank r owns experts [r*E_loc, (r+1)*E_loc).
+    Returns send_splits [ep], recv_counts [ep, E_loc], recv_splits [ep]."""
+    counts_all = np.ascontiguousarray(counts_all, dtype=np.int32)
+    ep, N_r = counts_all.shape
+    E_loc = N_r // ep
+    send = np.empty(ep, np.int32)
+    recv_counts = np.empty((ep, E_loc), np.int32)
+    recv = np.empty(ep, np.int32)
+    if _load().mo_ep_splits(_ptr(counts_all), ep, N_r, r, _ptr(send), _ptr(recv_counts),
+                            _ptr(recv)) != 0:
+        raise ValueError("oracle ep_splits rejected the arguments")
+    return send, recv_counts, recv
+
+
+def ep_recv_order(recv_counts):
+    """Order of the received rows by local expert (the page's gatherd_idxs
+    labels and their argsort, taken stable).  recv_counts [ep, E_loc].
+    Returns order [R] (sorted_tokens = gathered_tokens[order]) and
+    local_counts [E_loc] (tokens_per_expert_post_gather)."""
+    recv_counts = np.ascontiguousarray(recv_counts, dtype=np.int32)
+    ep, E_loc = recv_counts.shape
+    order = np.empty(int(recv_counts.sum()), np.int32)
+    local = np.empty(E_loc, np.int32)
+    if _load().mo_ep_recv_order(_ptr(recv_counts), ep, E_loc, _ptr(order), _ptr(local)) != 0:
+        raise ValueError("oracle ep_recv_order rejected the arguments")
+    return order, local
+
+
+def all_to_all(send_blocks):
+    """The all-to-all exchange itself, for ranks emulated in one process:
+    send_blocks[s][r] is what rank s sends rank r; rank r receives the
+    concatenation over s, in source order (dist.all_to_all)."""
+    ep = len(send_blocks)
+    return [np.concatenate([send_blocks[s][r] for s in range(ep)], axis=0) for r in range(ep)]
+
+
 def gather(x, k, perm, rows=None):
     """sorted_tokens = x[idxs // k] (Kimi K2 "Add shared output" page,
     moe_infer).  x is [T,d] of any element type, copied byte for byte;
@@ -152,7 +194,8 @@ def gather(x, k, perm, rows=None):
     rows_a = None if rows is None else np.ascontiguousarray(rows, dtype=np.int32)
     n = perm.shape[0] if rows is None else rows_a.shape[0]
     out = np.empty((n,) + x.shape[1:], x.dtype)
-    rc = lib.mo_gather(_ptr(x), x.strides[0], T, k, _ptr(perm), _ptr(rows_a), n, _ptr(out))
+    row_bytes = x.dtype.itemsize * int(np.prod(x.shape[1:]))  # numpy gives an empty array stride 0
+    rc = lib.mo_gather(_ptr(x), row_bytes, T, k, _ptr(perm), _ptr(rows_a), n, _ptr(out))
     if rc != 0:
         raise ValueError(f"oracle gather: index out of range (rc={rc})")
     return out

@@ -386,6 +386,75 @@ int mo_combine(const void *E, int dtype, const float *w, const int32_t *inv,
     return bad ? MO_ERR_RANGE : MO_OK;
 }
 
+/* ------------------------------------------------------------------ */
+/* Expert-parallel exchange ([K2-add] moe_infer, the ep_size > 1 branch).
+ * ep ranks; rank r owns the experts [r*E_loc, (r+1)*E_loc), E_loc = N_r/ep
+ * (tokens_per_expert.view(ep_size, -1)).
+ *
+ * mo_ep_splits: the bookkeeping of rank r, given every rank's
+ * tokens_per_expert (counts_all [ep][N_r]):
+ *   send_splits[s]    rows rank r sends to rank s (tokens_per_ep_rank:
+ *                     the sum of its counts over s's experts);
+ *   recv_counts[s][e] what all_to_all_single(tokens_per_expert) delivers to
+ *                     rank r: source s's count for r's local expert e
+ *                     (tokens_per_expert_group, viewed [ep][E_loc]);
+ *   recv_splits[s]    rows rank r receives from s (output_splits: the row
+ *                     sums of recv_counts). */
+int mo_ep_splits(const int32_t *counts_all, int ep, int N_r, int r, int32_t *send_splits,
+                 int32_t *recv_counts, int32_t *recv_splits)
+{
+    if (ep <= 0 || N_r <= 0 || N_r % ep != 0 || r < 0 || r >= ep) return MO_ERR_ARG;
+    const int E_loc = N_r / ep;
+    for (int s = 0; s < ep; ++s) {
+        long send = 0, recv = 0;
+        for (int e = 0; e < E_loc; ++e) {
+            send += counts_all[(long)r * N_r + (long)s * E_loc + e];
+            const int32_t c = counts_all[(long)s * N_r + (long)r * E_loc + e];
+            recv_counts[(long)s * E_loc + e] = c;
+            recv += c;
+        }
+        send_splits[s] = (int32_t)send;
+        recv_splits[s] = (int32_t)recv;
+    }
+    return MO_OK;
+}
+
+/* mo_ep_recv_order: the received rows arrive source by source, and within a
+ * source in its expert-sorted order; the page labels every received row
+ * with its local expert (gatherd_idxs[s..s+k] = i % experts_per_rank over
+ * the (source, expert) segments of tokens_per_expert_group, in that order)
+ * and argsorts the labels.  The argsort is taken stable (equal labels keep
+ * arrival order: by source, then the source's order), the reading used for
+ * every argsort of the path.  order[j] = the received row that goes j-th
+ * (sorted_tokens = gathered_tokens[order]); local_counts[e] =
+ * tokens_per_expert_post_gather (the column sums of recv_counts). */
+int mo_ep_recv_order(const int32_t *recv_counts, int ep, int E_loc, int32_t *order,
+                     int32_t *local_counts)
+{
+    if (ep <= 0 || E_loc <= 0) return MO_ERR_ARG;
+    long R = 0;
+    for (long i = 0; i < (long)ep * E_loc; ++i) {
+        if (recv_counts[i] < 0) return MO_ERR_RANGE;
+        R += recv_counts[i];
+    }
+    for (int e = 0; e < E_loc; ++e) local_counts[e] = 0;
+    mo_slot *sl = R > 0 ? malloc(sizeof(mo_slot) * (size_t)R) : NULL;
+    if (R > 0 && !sl) return MO_ERR_ARG;
+    long pos = 0;
+    for (long seg = 0; seg < (long)ep * E_loc; ++seg) {
+        const int label = (int)(seg % E_loc);
+        for (int32_t c = 0; c < recv_counts[seg]; ++c, ++pos) {
+            sl[pos].key = label;
+            sl[pos].slot = (int32_t)pos;
+        }
+        local_counts[label] += recv_counts[seg];
+    }
+    if (R > 0) qsort(sl, (size_t)R, sizeof(mo_slot), mo_cmp_slot);
+    for (long j = 0; j < R; ++j) order[j] = sl[j].slot;
+    free(sl);
+    return MO_OK;
+}
+
 int mo_num_threads(void)
 {
 #ifdef _OPENMP

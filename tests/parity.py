@@ -17,6 +17,8 @@ Comparison rules (tolerances the routing path is specified with):
 from __future__ import annotations
 
 import functools
+import json
+import os
 
 import numpy as np
 import torch
@@ -116,7 +118,9 @@ def compare_combine(gy, ry, rrouted, shared):
     assert (err <= tol).all(), (f"combine error at {worst}: gpu {gy[worst]} oracle {ry[worst]} "
                                 f"tol {tol[worst]}")
     rel_l2 = np.linalg.norm(gy - ry, axis=1) / np.maximum(np.linalg.norm(ry, axis=1), 1e-30)
-    return {"y_max_abs": float(err.max()), "y_row_rel_l2_max": float(rel_l2.max())}
+    return {"y_max_abs": float(err.max()), "y_row_rel_l2_max": float(rel_l2.max()),
+            "y_max_err_over_tol": float((err / tol).max()),
+            "y_differ_elems": int((err > 0).sum())}
 
 
 def widen(a):
@@ -124,3 +128,17 @@ def widen(a):
     if a.dtype == np.uint16:
         return wl.bf16_bits_to_f32(a).astype(np.float64)
     return a.astype(np.float64)
+
+
+def record(config: str, stage: str, stats: dict) -> None:
+    """Append one JSON line {config, stage, **stats} to the file named by the
+    environment variable MR_PARITY_OUT (nothing when it is unset): the
+    per-config parity figures (near-ties, largest errors) of a test run."""
+    path = os.environ.get("MR_PARITY_OUT")
+    if not path:
+        return
+    row = {"config": config, "stage": stage}
+    row.update({k: (float(v) if isinstance(v, (np.floating,)) else
+                    int(v) if isinstance(v, (np.integer,)) else v) for k, v in stats.items()})
+    with open(path, "a") as f:
+        f.write(json.dumps(row) + "\n")

@@ -89,3 +89,31 @@ def test_reference_arm_line_has_the_contract_keys():
     assert d["config"]["router_precision"].startswith("fp64")
     assert d["e2e"]["value"] == d["value"] and d["e2e"]["h2d_bytes_per_step"] == 0
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+
+
+def test_gpus_flag_without_launcher_starts_one_rank_per_gpu():
+    """`bench.py --gpus 2` with no launcher starts the two ranks itself (the
+    environment torchrun would give them); rank 0 alone prints one line and
+    it reports n_gpus = 2.  The reference arm needs no GPU, so this runs on
+    CPU."""
+    import json
+    env = {k: v for k, v in os.environ.items()
+           if k not in ("RANK", "WORLD_SIZE", "LOCAL_RANK", "MASTER_ADDR", "MASTER_PORT")}
+    p = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--gpus", "2", "--steps", "3", "--warmup", "3"], env=env,
+                       capture_output=True, text=True, timeout=600)
+    assert p.returncode == 0, p.stderr[-2000:]
+    lines = [ln for ln in p.stdout.splitlines() if ln.strip()]
+    assert len(lines) == 1, p.stdout
+    d = json.loads(lines[0])
+    assert d["n_gpus"] == 2 and d["impl"] == "reference"
+
+
+@pytest.mark.parametrize("impl", ["ours", "reference"])
+def test_gpus_flag_disagreeing_with_launcher_fails(impl):
+    env = dict(os.environ, RANK="0", WORLD_SIZE="2", LOCAL_RANK="0")
+    p = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", impl,
+                        "--gpus", "4", "--steps", "3", "--warmup", "3"], env=env,
+                       capture_output=True, text=True, timeout=120)
+    assert p.returncode != 0 and "WORLD_SIZE" in p.stderr
+    assert p.stdout.strip() == ""

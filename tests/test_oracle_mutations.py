@@ -45,6 +45,12 @@ MUTATIONS = {
                                  "mo_load(E, dtype, row * d + c);"),
     "combine_row_of_token_not_slot": ("long row = inv[t * k + j];", "long row = inv[t + j];"),
     "final_sum_not_rounded": ("                if (dtype == 1) y = mo_round_bf16(y);\n", ""),
+    "ep_label_is_source": ("const int label = (int)(seg % E_loc);",
+                           "const int label = (int)(seg / E_loc);"),
+    "ep_recv_block_of_sender": ("const int32_t c = counts_all[(long)s * N_r + (long)r * E_loc + e];",
+                                "const int32_t c = counts_all[(long)r * N_r + (long)s * E_loc + e];"),
+    "ep_send_block_of_receiver": ("send += counts_all[(long)r * N_r + (long)s * E_loc + e];",
+                                  "send += counts_all[(long)s * N_r + (long)r * E_loc + e];"),
 }
 
 

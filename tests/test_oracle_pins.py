@@ -495,3 +495,65 @@ def test_renormalisation_epsilon_only_matters_when_scores_underflow():
     nz = oracle.router(xz, Wz, None, 1, 1, 2, 2.5, 0, eps=False)
     assert (az["w"] == 0).all()
     assert np.isnan(nz["w"]).all()
+
+
+# --------------------------------------------------------------------------
+# Expert-parallel bookkeeping (Kimi K2 "Add shared output" page, moe_infer,
+# ep_size > 1).
+
+def _ep_counts(ep, N_r, seed, zeros=0.3):
+    rng = np.random.default_rng(seed)
+    c = rng.integers(0, 9, size=(ep, N_r)).astype(np.int32)
+    c[rng.random((ep, N_r)) < zeros] = 0
+    return c
+
+
+@pytest.mark.parametrize("ep,N_r", [(1, 8), (2, 8), (4, 64), (8, 256), (3, 12)])
+def test_ep_splits_are_the_transposed_blocks(ep, N_r):
+    """send_splits = block sums of the rank's own counts; recv_counts[s] = the
+    block of source s's counts that belongs to this rank (the count
+    all-to-all); recv_splits = its row sums; and over all ranks every row
+    sent is received once."""
+    c = _ep_counts(ep, N_r, ep * 100 + N_r)
+    E_loc = N_r // ep
+    sent = np.zeros((ep, ep), np.int64)
+    for r in range(ep):
+        send, rc, recv = oracle.ep_splits(c, r)
+        for s in range(ep):
+            assert send[s] == c[r, s * E_loc:(s + 1) * E_loc].sum()
+            assert np.array_equal(rc[s], c[s, r * E_loc:(r + 1) * E_loc])
+            assert recv[s] == rc[s].sum()
+            sent[r, s] = send[s]
+    for r in range(ep):
+        _, _, recv = oracle.ep_splits(c, r)
+        assert np.array_equal(recv, sent[:, r])  # what s sends r is what r receives from s
+
+
+@pytest.mark.parametrize("ep,E_loc", [(1, 4), (2, 32), (4, 16), (8, 32), (5, 3)])
+def test_ep_recv_order_is_a_stable_argsort_of_the_labels(ep, E_loc):
+    """The receive order against numpy: the page's labels (i % experts_per_rank
+    over the (source, expert) segments, built here with numpy.repeat) and
+    numpy's stable argsort; the local counts are the column sums."""
+    rc = _ep_counts(ep, E_loc, 7 * ep + E_loc)
+    order, local = oracle.ep_recv_order(rc)
+    labels = np.repeat(np.tile(np.arange(E_loc), ep), rc.reshape(-1))
+    assert np.array_equal(order, np.argsort(labels, kind="stable"))
+    assert np.array_equal(local, rc.sum(0))
+
+
+def test_ep_recv_order_hand_case():
+    """Two sources, two local experts: source 0 sends 2 rows of expert 0 and 1
+    of expert 1, source 1 sends 3 rows of expert 1.  Sorted by expert, keeping
+    arrival order: rows 0, 1 (expert 0), then 2, 3, 4, 5 (expert 1)."""
+    order, local = oracle.ep_recv_order(np.array([[2, 1], [0, 3]], np.int32))
+    assert order.tolist() == [0, 1, 2, 3, 4, 5] and local.tolist() == [2, 4]
+    # source 0: expert 1 first is impossible (sorted), but source 1 may send
+    # expert 0 rows after source 0's expert 1 rows: they move ahead of them
+    order, local = oracle.ep_recv_order(np.array([[1, 2], [2, 1]], np.int32))
+    assert order.tolist() == [0, 3, 4, 1, 2, 5] and local.tolist() == [3, 3]
+
+
+def test_all_to_all_emulation():
+    blocks = [[np.array([1]), np.array([2, 3])], [np.array([4, 5]), np.array([], int)]]
+    got = oracle.all_to_all(blocks)
+    assert got[0].tolist() == [1, 4, 5] and got[1].tolist() == [2, 3]

@@ -1,9 +1,16 @@
 """The whole hot path on the GPU, chained through the C ABI exactly as the
 benchmark runs it: router -> dispatch -> gather -> (synthetic experts) ->
-combine.  Each stage is checked against the oracle fed with the GPU's own
-upstream outputs (so dispatch/gather are bit-exact with no exclusions), the
-router against the oracle on the raw inputs, and the identity-expert closed
-form (y = route_scale * x) on every token."""
+combine, on all five workloads.  Every stage is compared with the oracle on
+every token and every row:
+  * the router on the raw inputs (selection exact outside near-ties, weights
+    within 1e-5 relative, logits within 2e-5);
+  * dispatch and gather fed the GPU's own idx, so they are bit-exact with no
+    exclusions;
+  * combine fed the GPU's own weights and inverse permutation, within the
+    combine tolerance;
+plus the identity-expert closed form (y = route_scale * x) on every token.
+With MR_PARITY_OUT set, each comparison appends its figures (near-ties,
+largest errors) to that file, one JSON line per workload and stage."""
 import numpy as np
 import pytest
 import torch
@@ -11,16 +18,36 @@ import torch
 import oracle
 import token_dispatch_fp32_b200 as mr
 import workloads as wl
-from parity import (compare_combine, compare_router, oracle_router, router_inputs, row_inputs,
-                    sample_tokens, to_dev, widen)
+from parity import (compare_combine, compare_router, oracle_router, record, router_inputs,
+                    row_inputs, to_dev, widen)
 
 pytestmark = pytest.mark.gpu
+
+ALL = [wl.TINY, wl.V3_PREFILL, wl.K2_PREFILL, wl.V3_DECODE, wl.V3_FULL]
+CHUNK_ROWS = 1 << 14  # rows compared per host round trip (bounds host memory)
 
 
 def _host_rows(t):
     if t.dtype == torch.bfloat16:
         return t.view(torch.int16).cpu().numpy().view(np.uint16)
     return t.cpu().numpy()
+
+
+def bench_router(w: wl.Workload, x32, x_rows, Wd, bd, idx, wt, logits=None):
+    """The router as the benchmark launches it for this workload: bf16 rows
+    above 256 tokens take the bf16x3 kernel with a workspace; decode-size and
+    fp32 batches take the plain entry point on the fp32 rows (split-K for
+    T <= 256, with no workspace)."""
+    if w.io_dtype == wl.BF16 and w.T > 256:
+        ws = torch.empty(mr.mr_router_workspace_size(w.T, w.d, w.N_r), dtype=torch.uint8,
+                         device="cuda")
+        mr.mr_router_forward_ex(x_rows, Wd, bd, w.n_group, w.topk_group, w.k, w.route_scale,
+                                w.mask_mode, precision=mr.MR_PREC_BF16X3, idx_out=idx,
+                                w_out=wt, logits_out=logits, workspace=ws)
+        return "bf16x3 fused (mr_router_forward_ex)"
+    mr.mr_router_forward(x32, Wd, bd, w.n_group, w.topk_group, w.k, w.route_scale,
+                         w.mask_mode, idx_out=idx, w_out=wt)
+    return "plain mr_router_forward (fp32 rows)"
 
 
 def run_path(w: wl.Workload, E_dev, shared_dev):
@@ -31,10 +58,8 @@ def run_path(w: wl.Workload, E_dev, shared_dev):
     # on the stale result of an earlier call
     fill = lambda shape, dt, v: torch.full(shape, v, dtype=dt, device="cuda")  # noqa: E731
     T, k, N, dd = w.T, w.k, w.N_r, w.d
-    idx, wt = mr.mr_router_forward(x32, to_dev(d["W"]), to_dev(d["b"]), w.n_group,
-                                   w.topk_group, w.k, w.route_scale, w.mask_mode,
-                                   idx_out=fill((T, k), torch.int32, -1),
-                                   w_out=fill((T, k), torch.float32, float("nan")))
+    idx, wt = fill((T, k), torch.int32, -1), fill((T, k), torch.float32, float("nan"))
+    how = bench_router(w, x32, x_rows, to_dev(d["W"]), to_dev(d["b"]), idx, wt)
     counts, offsets, perm, inv = mr.mr_dispatch(
         idx, N, counts=fill((N,), torch.int32, -7), offsets=fill((N + 1,), torch.int32, -7),
         perm=fill((T * k,), torch.int32, -7), inv_perm=fill((T * k,), torch.int32, -7))
@@ -44,41 +69,57 @@ def run_path(w: wl.Workload, E_dev, shared_dev):
                       y=fill((T, dd), x_rows.dtype, float("nan")))
     assert mr.mr_get_error() == mr.MR_OK
     return dict(idx=idx, w=wt, counts=counts, offsets=offsets, perm=perm, inv=inv, xs=xs, y=y,
-                x_rows=x_rows)
+                x_rows=x_rows, router=how)
 
 
-@pytest.mark.parametrize("w", [wl.TINY, wl.V3_FULL], ids=["tiny", "v3_full"])
-def test_full_path(w):
+@pytest.mark.parametrize("w", ALL, ids=[w.name for w in ALL])
+def test_full_path_every_token(w):
     rows = row_inputs(w)
     dt = "bf16" if w.io_dtype == "bf16" else None
     out = run_path(w, to_dev(rows["E"], dt), to_dev(rows["shared"], dt))
     idx = out["idx"].cpu().numpy()
     wt = out["w"].cpu().numpy()
-    # router on sampled tokens
-    tok = sample_tokens(w.T, 256, seed=w.seed)
-    stats = compare_router(idx[tok], wt[tok], oracle_router(w, tok, want_logits=False))
+    # router: every token
+    stats = compare_router(idx, wt, oracle_router(w, np.arange(w.T), want_logits=False))
+    stats["router"] = out["router"]
+    record(w.name, "router", stats)
     # dispatch on the GPU's idx: bit-exact, every entry
     rc, ro, rp, ri = oracle.dispatch(idx, w.N_r)
     assert (out["counts"].cpu().numpy() == rc).all()
     assert (out["offsets"].cpu().numpy() == ro).all()
     assert (out["perm"].cpu().numpy() == rp).all()
     assert (out["inv"].cpu().numpy() == ri).all()
-    # gather: bit-exact on sampled sorted rows (all rows for small T)
-    x_host = rows_x = router_inputs(w)["x_bf16" if w.io_dtype == "bf16" else "x_f32"]
+    record(w.name, "dispatch", {"entries": int(w.T * w.k), "mismatches": 0,
+                                "hot_expert_max_count": int(rc.max())})
+    # gather: bit-exact, every sorted row
+    x_host = router_inputs(w)["x_bf16" if w.io_dtype == "bf16" else "x_f32"]
     nrows = w.T * w.k
-    srows = sample_tokens(nrows, 4096, seed=1).astype(np.int32)
-    xs = out["xs"][torch.from_numpy(srows).long().cuda()]
-    assert np.array_equal(_host_rows(xs), oracle.gather(x_host, w.k, rp, srows))
-    # combine on sampled tokens with the GPU's weights and inverse permutation
-    ry, rr = oracle.combine(rows["E"], wt, ri, rows["shared"], w.k,
-                            tokens=tok.astype(np.int32))
-    gy = widen(_host_rows(out["y"][torch.from_numpy(tok).cuda()]))
-    cstats = compare_combine(gy, ry, rr, widen(rows["shared"][tok]))
-    print(w.name, stats, cstats, "hot-expert counts", rc[:4])
-    del rows_x
+    for r0 in range(0, nrows, CHUNK_ROWS):
+        r1 = min(nrows, r0 + CHUNK_ROWS)
+        sel = np.arange(r0, r1, dtype=np.int32)
+        want = oracle.gather(x_host, w.k, rp, sel)
+        assert np.array_equal(_host_rows(out["xs"][r0:r1]), want), f"gather rows {r0}..{r1}"
+    record(w.name, "gather", {"rows": nrows, "mismatches": 0})
+    # combine: every token, with the GPU's weights and inverse permutation
+    worst = {"y_max_abs": 0.0, "y_row_rel_l2_max": 0.0, "y_max_err_over_tol": 0.0,
+             "y_differ_elems": 0}
+    tstep = max(1, CHUNK_ROWS // w.k)
+    for t0 in range(0, w.T, tstep):
+        t1 = min(w.T, t0 + tstep)
+        tok = np.arange(t0, t1, dtype=np.int32)
+        ry, rr = oracle.combine(rows["E"], wt, ri, rows["shared"], w.k, tokens=tok)
+        gy = widen(_host_rows(out["y"][t0:t1]))
+        c = compare_combine(gy, ry, rr, widen(rows["shared"][t0:t1]))
+        for key in worst:
+            worst[key] = worst[key] + c[key] if key == "y_differ_elems" else max(worst[key],
+                                                                                  c[key])
+    worst["tokens"] = w.T
+    worst["elems"] = w.T * w.d
+    record(w.name, "combine", worst)
+    print(w.name, out["router"], stats, worst, "hot-expert counts", rc[:4])
 
 
-@pytest.mark.parametrize("w", [wl.TINY, wl.V3_FULL], ids=["tiny", "v3_full"])
+@pytest.mark.parametrize("w", ALL, ids=[w.name for w in ALL])
 def test_identity_experts_closed_form_every_token(w):
     """Experts = identity and no shared expert: y_t = sum_j w_tj x_t =
     route_scale * x_t (weights sum to the route scale), on every token."""

@@ -6,7 +6,7 @@ import torch
 import oracle
 import token_dispatch_fp32_b200 as mr
 import workloads as wl
-from parity import compare_router, oracle_router, router_inputs, sample_tokens, to_dev
+from parity import compare_router, oracle_router, record, router_inputs, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -74,16 +74,69 @@ def test_router_small_all_tokens(w, precision):
     print(w.name, precision, stats)
 
 
-@pytest.mark.parametrize("w", SMALL[:4], ids=[w.name for w in SMALL[:4]])
-def test_router_plain_tf32_logits(w):
-    """One-product TF32 is reported separately: logits within ~1e-3, not 2e-5."""
-    idx, wt, logits = _run(w, mr.MR_PREC_TF32)
+# Plain TF32 (one tensor-core product per multiply-add).  The tensor core
+# reads each fp32 operand with its 13 low mantissa bits dropped (truncation,
+# pinned by test_tf32_operand_low_bits_probe), so each operand carries a relative
+# error below 2^-10 and a product x_j W_ij one below 2^-9 + 2^-20.  With fp32
+# accumulation (round toward zero inside 128-K intervals, rounded sums
+# between them: below 128 * 2^-23 + 2^-24 relative) every logit satisfies
+#     |L_tf32 - L| <= TF32_LOGIT_COEF * sum_j |x_j W_ij|,
+# TF32_LOGIT_COEF = 2^-9 + 2^-20 + 129 * 2^-23 < 1.97e-3.
+TF32_LOGIT_COEF = 2.0 ** -9 + 2.0 ** -20 + 129 * 2.0 ** -23
+
+
+def tf32_check(w, x_f32, idx, wt, logits, tag):
+    """TF32 router output against the oracle: the logits within the bound
+    above; the selection and weights exactly what the method gives for the
+    GPU's own logits (the oracle fed those logits as x with W = identity,
+    so its logits equal them), outside the usual 1e-5 near-tie band; and
+    the number of tokens whose selection differs from the fp64 selection
+    on the true inputs (reported: the cost of the cheaper arithmetic)."""
+    d = router_inputs(w)
     ref = oracle_router(w, np.arange(w.T))
-    err = np.abs(logits - ref["logits"]) / np.maximum(np.abs(ref["logits"]), 1.0)
-    assert err.max() < 2e-2
-    assert (idx >= 0).all() and (idx < w.N_r).all()
-    np.testing.assert_allclose(wt.sum(1), w.route_scale, rtol=1e-5)
-    print(w.name, "tf32 logit max err", err.max())
+    L = ref["logits"]
+    absdot = np.abs(np.asarray(x_f32, np.float64)) @ np.abs(d["W"].astype(np.float64)).T
+    err = np.abs(logits.astype(np.float64) - L)
+    assert (err <= TF32_LOGIT_COEF * absdot).all(), \
+        f"TF32 logit error {(err / absdot).max():.3g} x sum|xW| > {TF32_LOGIT_COEF:.3g}"
+    eye = np.eye(w.N_r, dtype=np.float32)
+    own = oracle.router(logits.astype(np.float32), eye, d["b"], w.n_group, w.topk_group, w.k,
+                        w.route_scale, w.mask_mode)
+    stats = compare_router(idx, wt, own)
+    changed = int((np.sort(idx, 1) != np.sort(ref["idx"], 1)).any(1).sum())
+    stats.update({"logit_max_abs_err": float(err.max()),
+                  "logit_err_over_bound_max": float((err / (TF32_LOGIT_COEF * absdot)).max()),
+                  "selection_changed_vs_fp64": changed})
+    record(w.name, tag, stats)
+    return stats
+
+
+@pytest.mark.parametrize("w", SMALL[:4], ids=[w.name for w in SMALL[:4]])
+def test_router_plain_tf32_parity(w):
+    """One-product TF32, reported separately: logits within the derived TF32
+    bound, selection and weights exact given its logits."""
+    idx, wt, logits = _run(w, mr.MR_PREC_TF32)
+    stats = tf32_check(w, router_inputs(w)["x_f32"], idx, wt, logits, "router_tf32")
+    print(w.name, "tf32", stats)
+
+
+@pytest.mark.parametrize("w", FULL, ids=[w.name for w in FULL])
+def test_router_plain_tf32_full_size(w):
+    """The TF32 variant on the full workloads (fused kernel; split-K for the
+    64-token decode batch), every token."""
+    d = router_inputs(w)
+    ws = torch.empty(mr.mr_router_workspace_size(w.T, w.d, w.N_r), dtype=torch.uint8,
+                     device="cuda")
+    lg = torch.full((w.T, w.N_r), float("nan"), device="cuda")
+    io, wo = _poisoned(w.T, w.k)
+    idx, wt = mr.mr_router_forward_ex(to_dev(d["x_f32"]), to_dev(d["W"]), to_dev(d["b"]),
+                                      w.n_group, w.topk_group, w.k, w.route_scale, w.mask_mode,
+                                      precision=mr.MR_PREC_TF32, idx_out=io, w_out=wo,
+                                      logits_out=lg, workspace=ws)
+    assert mr.mr_get_error() == mr.MR_OK
+    stats = tf32_check(w, d["x_f32"], idx.cpu().numpy(), wt.cpu().numpy(), lg.cpu().numpy(),
+                       "router_tf32")
+    print(w.name, "tf32", stats)
 
 
 @pytest.mark.parametrize("cs", ["1", "2"])
@@ -140,13 +193,13 @@ def test_router_empty_batch():
 
 
 @pytest.mark.parametrize("w", FULL, ids=[w.name for w in FULL])
-def test_router_full_size_sampled(w):
-    """Every token runs on the GPU in the configuration the benchmark uses;
-    the oracle checks a sample of tokens (incl. the first and last)."""
+def test_router_full_size_every_token(w):
+    """The fp32-row (3xTF32) router at full size against the oracle on every
+    token: selection, weights and logits."""
     idx, wt, logits = _run(w, mr.MR_PREC_3XTF32)
-    tok = sample_tokens(w.T, 256, seed=w.seed)
-    ref = oracle_router(w, tok)
-    stats = compare_router(idx[tok], wt[tok], ref, logits[tok])
+    ref = oracle_router(w, np.arange(w.T))
+    stats = compare_router(idx, wt, ref, logits)
+    record(w.name, "router_3xtf32_fp32_rows", stats)
     # properties that hold for every token
     assert (idx >= 0).all() and (idx < w.N_r).all()
     assert all(len(set(r)) == w.k for r in idx[:: max(1, w.T // 512)])
@@ -354,13 +407,15 @@ def test_router_bf16x3_cluster_size_pinned(w, cs, monkeypatch):
     compare_router(idx, wt, oracle_router(w, np.arange(w.T)), logits)
 
 
-@pytest.mark.parametrize("w", [wl.V3_PREFILL, wl.K2_PREFILL, wl.V3_FULL],
+@pytest.mark.parametrize("w", [wl.V3_PREFILL, wl.K2_PREFILL, wl.V3_DECODE, wl.V3_FULL],
                          ids=lambda w: w.name)
-def test_router_bf16x3_full_size_sampled(w):
+def test_router_bf16x3_full_size_every_token(w):
+    """bf16 rows (the benchmark's router arithmetic) at full size against the
+    oracle on every token, logits included (T <= 256 runs split-K)."""
     idx, wt, logits = _run_bf16x3(w)
-    tok = sample_tokens(w.T, 256, seed=w.seed + 7)
-    stats = compare_router(idx[tok], wt[tok], oracle_router(w, tok), logits[tok])
+    stats = compare_router(idx, wt, oracle_router(w, np.arange(w.T)), logits)
     np.testing.assert_allclose(wt.sum(1), w.route_scale, rtol=2e-6)
+    record(w.name, "router_bf16_rows", stats)
     print(w.name, "bf16x3", stats)
 
 
@@ -472,3 +527,151 @@ def test_router_no_eps_underflow_gives_nan_like_the_page():
         _, wt = mr.mr_router_forward_ex(x, Wt, None, 1, 1, 4, 2.5, 0, flags=flags)
         got = wt.cpu().numpy()
         assert np.isnan(got).all() if want_nan else (got == 0).all()
+
+
+@pytest.mark.parametrize("w", SPLITK, ids=[w.name for w in SPLITK])
+def test_router_plain_entry_point_picks_splitk_for_small_batches(w):
+    """The plain entry point (no workspace argument) runs batches of up to 256
+    tokens on the split-K path -- two launches, its partials in the library's
+    own array -- with the same results as mr_router_forward_ex given a
+    workspace, and parity with the oracle on every token."""
+    d = router_inputs(w)
+    x, Wd, b = to_dev(d["x_f32"]), to_dev(d["W"]), to_dev(d["b"])
+    io, wo = _poisoned(w.T, w.k)
+    l0 = mr.mr_launch_count()
+    idx, wt = mr.mr_router_forward(x, Wd, b, w.n_group, w.topk_group, w.k, w.route_scale,
+                                   w.mask_mode, idx_out=io, w_out=wo)
+    assert mr.mr_launch_count() - l0 == 2  # split-K GEMM + reduce/route
+    assert mr.mr_get_error() == mr.MR_OK
+    ref = oracle_router(w, np.arange(w.T), want_logits=False)
+    print(w.name, compare_router(idx.cpu().numpy(), wt.cpu().numpy(), ref))
+    ws = torch.empty(mr.mr_router_workspace_size(w.T, w.d, w.N_r), dtype=torch.uint8,
+                     device="cuda")
+    idx2, wt2 = mr.mr_router_forward_ex(x, Wd, b, w.n_group, w.topk_group, w.k, w.route_scale,
+                                        w.mask_mode, workspace=ws)
+    assert torch.equal(idx, idx2) and torch.equal(wt, wt2)
+
+
+def test_router_plain_small_batches_on_two_streams():
+    """Calls of the plain entry point on two streams share its split-K array;
+    the library orders them, so interleaved calls on unordered streams each
+    get their own batch's result."""
+    ws_ = [SPLITK[0], SPLITK[2], wl.V3_DECODE]
+    ins = []
+    for w in ws_:
+        d = router_inputs(w)
+        ins.append((w, to_dev(d["x_f32"]), to_dev(d["W"]), to_dev(d["b"])))
+    refs = [mr.mr_router_forward(x, Wd, b, w.n_group, w.topk_group, w.k, w.route_scale,
+                                 w.mask_mode) for w, x, Wd, b in ins]
+    torch.cuda.synchronize()
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    outs = []
+    for rep in range(6):
+        for j, (w, x, Wd, b) in enumerate(ins):
+            s = streams[(rep + j) % 2]
+            outs.append((j, mr.mr_router_forward(x, Wd, b, w.n_group, w.topk_group, w.k,
+                                                  w.route_scale, w.mask_mode, stream=s)))
+    torch.cuda.synchronize()
+    assert mr.mr_get_error() == mr.MR_OK
+    for j, (idx, wt) in outs:
+        assert torch.equal(idx, refs[j][0]) and torch.equal(wt, refs[j][1])
+
+
+def test_router_plain_large_batches_stay_fused():
+    """Above 256 tokens the plain entry point runs the fused kernel (one
+    launch: no W residual pass without a workspace)."""
+    w = SMALL[1]
+    d = router_inputs(w)
+    l0 = mr.mr_launch_count()
+    idx, wt = mr.mr_router_forward(to_dev(d["x_f32"]), to_dev(d["W"]), to_dev(d["b"]),
+                                   w.n_group, w.topk_group, w.k, w.route_scale, w.mask_mode)
+    assert mr.mr_launch_count() - l0 == 1
+    assert mr.mr_get_error() == mr.MR_OK
+    compare_router(idx.cpu().numpy(), wt.cpu().numpy(),
+                   oracle_router(w, np.arange(w.T), want_logits=False))
+    assert mr.mr_router_forward_max_scratch() == 2 << 20
+
+
+# --------------------------------------------------------------------------
+# Gate weight stored in bf16 (mr_router_forward_bf16w).  The oracle gets the
+# widened bf16 values of W; with bf16 rows every product is exact in fp32, so
+# the tolerances of the fp32 path hold.
+
+BF16W = [
+    SMALL[1],                                              # fused, ragged T and K tail
+    SMALL[2].replace(name="k2_like_bf16w_T300", T=300),    # 384 experts, 2-CTA split
+    BF16X3[2],                                             # N_r = 16, k = 3
+    BF16X3[3],                                             # 320 experts in 10 groups, zero mask
+    BF16X3[5],                                             # all biased scores negative
+    SPLITK[0], SPLITK[1], SPLITK[2], wl.V3_DECODE,         # decode sizes: split-K
+]
+
+
+def _bf16w_ref(w, tok):
+    d = router_inputs(w)
+    Wf = wl.gen_W_bf16(w)["W_f32"]
+    return oracle.router(d["x_f32"][tok], Wf, d["b"], w.n_group, w.topk_group, w.k,
+                         w.route_scale, w.mask_mode, want_logits=True)
+
+
+def _bf16w_run(w, rows="bf16", workspace=True):
+    d = router_inputs(w)
+    Wb = to_dev(wl.gen_W_bf16(w)["W_bf16"], "bf16")
+    x = to_dev(d["x_bf16"], "bf16") if rows == "bf16" else to_dev(d["x_f32"])
+    ws = torch.empty(mr.mr_router_workspace_size(w.T, w.d, w.N_r), dtype=torch.uint8,
+                     device="cuda") if workspace else None
+    lg = torch.full((w.T, w.N_r), float("nan"), device="cuda")
+    io, wo = _poisoned(w.T, w.k)
+    l0 = mr.mr_launch_count()
+    idx, wt = mr.mr_router_forward_bf16w(x, Wb, to_dev(d["b"]), w.n_group, w.topk_group, w.k,
+                                         w.route_scale, w.mask_mode, idx_out=io, w_out=wo,
+                                         logits_out=lg, workspace=ws)
+    launches = mr.mr_launch_count() - l0
+    assert mr.mr_get_error() == mr.MR_OK
+    return idx.cpu().numpy(), wt.cpu().numpy(), lg.cpu().numpy(), launches
+
+
+@pytest.mark.parametrize("w", BF16W, ids=[w.name for w in BF16W])
+def test_router_bf16_weights_all_tokens(w):
+    """bf16 rows x bf16-stored W on the tensor cores (fused kernel with one
+    bf16 plane, or split-K with kind::f16 for <= 256 tokens) against the
+    oracle on the widened W: every token, fp32 tolerances."""
+    assert w.io_dtype == "bf16"
+    idx, wt, lg, launches = _bf16w_run(w)
+    assert launches == (2 if w.T <= 256 else 1)
+    stats = compare_router(idx, wt, _bf16w_ref(w, np.arange(w.T)), lg)
+    record(w.name, "router_bf16_weights", stats)
+    print(w.name, "bf16 W", stats)
+
+
+def test_router_bf16_weights_without_workspace_and_fp32_rows():
+    """Decode-size batch without a workspace (the library's split-K array),
+    and fp32 rows (CUDA-core path on the widened W): same results as the
+    oracle."""
+    w = wl.V3_DECODE
+    ref = _bf16w_ref(w, np.arange(w.T))
+    idx, wt, lg, launches = _bf16w_run(w, workspace=False)
+    assert launches == 2
+    compare_router(idx, wt, ref, lg)
+    w2 = SMALL[1]
+    idx, wt, lg, launches = _bf16w_run(w2, rows="f32", workspace=False)
+    assert launches == 1
+    compare_router(idx, wt, _bf16w_ref(w2, np.arange(w2.T)), lg)
+
+
+@pytest.mark.parametrize("cs", ["1", "2", "P"])
+def test_router_bf16_weights_every_tile_shape(cs, monkeypatch):
+    monkeypatch.setenv("MR_TC_CLUSTER", cs)
+    w = BF16X3[5]
+    idx, wt, lg, _ = _bf16w_run(w)
+    compare_router(idx, wt, _bf16w_ref(w, np.arange(w.T)), lg)
+
+
+@pytest.mark.parametrize("w", [wl.V3_PREFILL, wl.K2_PREFILL, wl.V3_FULL], ids=lambda w: w.name)
+def test_router_bf16_weights_full_size_every_token(w):
+    idx, wt, lg, launches = _bf16w_run(w)
+    assert launches == 1
+    stats = compare_router(idx, wt, _bf16w_ref(w, np.arange(w.T)), lg)
+    np.testing.assert_allclose(wt.sum(1), w.route_scale, rtol=2e-6)
+    record(w.name, "router_bf16_weights", stats)
+    print(w.name, "bf16 W", stats)

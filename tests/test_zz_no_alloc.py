@@ -13,6 +13,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 import token_dispatch_fp32_b200 as mr
 
 
@@ -37,11 +38,36 @@ def test_noalloc_dispatch_matches_workspace_dispatch_twice_in_a_row():
     for T, k, N_r, seed, skew in cases:
         idx = _ids(T, k, N_r, seed, skew)
         ref = mr.mr_dispatch(idx, N_r)  # existing entry point, caller workspace
+        # and the oracle's stable counting sort of the same ids
+        orc = oracle.dispatch(idx.cpu().numpy(), N_r)
         for _ in range(2):              # two calls in a row share the scratch
             got = mr.mr_dispatch_noalloc(idx, N_r, *_outs(T, k, N_r))
             assert mr.mr_get_error() == mr.MR_OK
-            for g, r in zip(got, ref):
+            for g, r, o in zip(got, ref, orc):
                 assert torch.equal(g, r)
+                assert np.array_equal(g.cpu().numpy(), o)
+
+
+@pytest.mark.gpu
+def test_noalloc_dispatch_drops_out_of_range_ids_like_mr_dispatch():
+    """Ids outside [0, N_r) are dropped by both entry points alike: the valid
+    entries are sorted, the dropped slots' inverse entries and the tail of
+    perm read -1, and the device flag reports it."""
+    T, k, N_r = 500, 4, 64
+    a = _ids(T, k, N_r, 3).cpu().numpy()
+    a[7, 2], a[123, 0], a[499, 3] = -1, N_r, N_r + 5
+    idx = torch.from_numpy(a).cuda()
+    ref = mr.mr_dispatch(idx, N_r)
+    assert mr.mr_get_error() == mr.MR_ERR_DEVICE
+    for _ in range(2):
+        got = mr.mr_dispatch_noalloc(idx, N_r, *_outs(T, k, N_r))
+        assert mr.mr_get_error() == mr.MR_ERR_DEVICE
+        for g, r in zip(got, ref):
+            assert torch.equal(g, r)
+    counts, offsets, perm, inv = (t.cpu().numpy() for t in got)
+    assert counts.sum() == T * k - 3 and offsets[-1] == T * k - 3
+    assert (perm[T * k - 3:] == -1).all()
+    assert inv[7 * k + 2] == -1 and inv[123 * k] == -1 and inv[499 * k + 3] == -1
 
 
 @pytest.mark.gpu

@@ -61,6 +61,8 @@ def lib():
                                            sz, p]
         L.mr_router_forward_ex2.argtypes = [p, i, p, p, i, i, i, i, i, i, f, i, i, i, p, p, p,
                                             p, sz, p]
+        L.mr_router_forward_bf16w.argtypes = [p, i, p, p, i, i, i, i, i, i, f, i, i, p, p, p,
+                                              p, sz, p]
         L.mr_router_workspace_size.argtypes = [i, i, i]
         L.mr_router_workspace_size.restype = sz
         L.mr_dispatch_workspace_size.argtypes = [i, i, i]
@@ -68,7 +70,9 @@ def lib():
         L.mr_dispatch.argtypes = [p, i, i, i, p, p, p, p, p, sz, p]
         L.mr_dispatch_noalloc.argtypes = [p, i, i, i, p, p, p, p, p]
         L.mr_dispatch_noalloc_max_workspace.restype = sz
+        L.mr_router_forward_max_scratch.restype = sz
         L.mr_gather_rows.argtypes = [p, i, i, i, i, p, p, p, p]
+        L.mr_ep_recv_order.argtypes = [p, i, i, i, p, p, p, p, p]
         L.mr_combine.argtypes = [p, i, p, p, p, p, i, i, i, p]
         L.mr_get_error.argtypes = [p]
         L.mr_selftest_bounded_wait.argtypes = [i, p]
@@ -97,6 +101,27 @@ def _stream(stream):
     if stream is None:
         stream = torch.cuda.current_stream()
     return C.c_void_p(stream.cuda_stream)
+
+
+def _call(fn: str, dev, stream, *args) -> None:
+    """Calls C entry point `fn` with `dev` as the current CUDA device and the
+    stream handle as the last argument: the library launches on the current
+    device, so the tensors' device is made current for the call.  `stream`
+    (default: that device's current stream) must belong to the same device."""
+    with torch.cuda.device(dev):
+        if stream is None:
+            stream = torch.cuda.current_stream(dev)
+        elif stream.device != dev:
+            raise ValueError(f"stream is on {stream.device}, tensors on {dev}")
+        _check(fn, getattr(lib(), fn)(*args, C.c_void_p(stream.cuda_stream)))
+
+
+def _device_of(*tensors):
+    """The one CUDA device of the given tensors (None entries ignored)."""
+    devs = {t.device for t in tensors if t is not None}
+    if len(devs) != 1:
+        raise ValueError(f"tensors must be on one CUDA device, got {sorted(map(str, devs))}")
+    return devs.pop()
 
 
 def _need(t, name, dtype=None, shape=None):
@@ -138,10 +163,15 @@ def mr_router_forward(x, W, bias, n_group, topk_group, k, route_scale, mask_mode
         _need(idx_out, "idx_out", torch.int32, (T, k))
     w_out = torch.empty((T, k), dtype=torch.float32, device=x.device) if w_out is None else \
         _need(w_out, "w_out", torch.float32, (T, k))
-    _check("mr_router_forward", lib().mr_router_forward(
-        _ptr(x), _ptr(W), _ptr(bias), T, d, N_r, n_group, topk_group, k, float(route_scale),
-        mask_mode, _ptr(idx_out), _ptr(w_out), _stream(stream)))
+    dev = _device_of(x, W, bias, idx_out, w_out)
+    _call("mr_router_forward", dev, stream, _ptr(x), _ptr(W), _ptr(bias), T, d, N_r, n_group,
+          topk_group, k, float(route_scale), mask_mode, _ptr(idx_out), _ptr(w_out))
     return idx_out, w_out
+
+
+def mr_router_forward_max_scratch() -> int:
+    """Bytes of the fixed array holding mr_router_forward's split-K partials."""
+    return int(lib().mr_router_forward_max_scratch())
 
 
 def mr_router_workspace_size(T, d, N_r) -> int:
@@ -171,16 +201,46 @@ def mr_router_forward_ex(x, W, bias, n_group, topk_group, k, route_scale, mask_m
     if workspace is not None:
         _need(workspace, "workspace")
         ws_bytes = workspace.numel() * workspace.element_size()
+    dev = _device_of(x, W, bias, idx_out, w_out, logits_out, workspace)
     if flags:
-        _check("mr_router_forward_ex2", lib().mr_router_forward_ex2(
-            _ptr(x), x_dtype, _ptr(W), _ptr(bias), T, d, N_r, n_group, topk_group, k,
-            float(route_scale), mask_mode, precision, int(flags), _ptr(idx_out), _ptr(w_out),
-            _ptr(logits_out), _ptr(workspace), ws_bytes, _stream(stream)))
+        _call("mr_router_forward_ex2", dev, stream, _ptr(x), x_dtype, _ptr(W), _ptr(bias), T, d,
+              N_r, n_group, topk_group, k, float(route_scale), mask_mode, precision,
+              int(flags), _ptr(idx_out), _ptr(w_out), _ptr(logits_out), _ptr(workspace),
+              ws_bytes)
     else:
-        _check("mr_router_forward_ex", lib().mr_router_forward_ex(
-            _ptr(x), x_dtype, _ptr(W), _ptr(bias), T, d, N_r, n_group, topk_group, k,
-            float(route_scale), mask_mode, precision, _ptr(idx_out), _ptr(w_out),
-            _ptr(logits_out), _ptr(workspace), ws_bytes, _stream(stream)))
+        _call("mr_router_forward_ex", dev, stream, _ptr(x), x_dtype, _ptr(W), _ptr(bias), T, d,
+              N_r, n_group, topk_group, k, float(route_scale), mask_mode, precision,
+              _ptr(idx_out), _ptr(w_out), _ptr(logits_out), _ptr(workspace), ws_bytes)
+    return idx_out, w_out
+
+
+def mr_router_forward_bf16w(x, W_bf16, bias, n_group, topk_group, k, route_scale, mask_mode,
+                            idx_out=None, w_out=None, logits_out=None, workspace=None,
+                            stream=None, flags=0):
+    """The gate with a bf16-stored weight W_bf16 [N_r,d] (torch.bfloat16):
+    x [T,d] bf16 (tensor cores) or fp32 (CUDA cores).  Returns (idx, w)."""
+    _need(x, "x")
+    x_dtype = _row_dtype(x)
+    T, d = x.shape
+    N_r = W_bf16.shape[0]
+    _need(W_bf16, "W_bf16", torch.bfloat16, (N_r, d))
+    if bias is not None:
+        _need(bias, "bias", torch.float32, (N_r,))
+    idx_out = torch.empty((T, k), dtype=torch.int32, device=x.device) if idx_out is None else \
+        _need(idx_out, "idx_out", torch.int32, (T, k))
+    w_out = torch.empty((T, k), dtype=torch.float32, device=x.device) if w_out is None else \
+        _need(w_out, "w_out", torch.float32, (T, k))
+    if logits_out is not None:
+        _need(logits_out, "logits_out", torch.float32, (T, N_r))
+    ws_bytes = 0
+    if workspace is not None:
+        _need(workspace, "workspace")
+        ws_bytes = workspace.numel() * workspace.element_size()
+    _call("mr_router_forward_bf16w", _device_of(x, W_bf16, bias, idx_out, w_out, logits_out,
+                                                 workspace), stream,
+          _ptr(x), x_dtype, _ptr(W_bf16), _ptr(bias), T, d, N_r, n_group, topk_group, k,
+          float(route_scale), mask_mode, int(flags), _ptr(idx_out), _ptr(w_out),
+          _ptr(logits_out), _ptr(workspace), ws_bytes)
     return idx_out, w_out
 
 
@@ -209,9 +269,9 @@ def mr_dispatch(idx, N_r, counts=None, offsets=None, perm=None, inv_perm=None, w
     if workspace is None:
         workspace = torch.empty(max(need, 4), dtype=torch.uint8, device=dev)
     _need(workspace, "workspace")
-    _check("mr_dispatch", lib().mr_dispatch(
-        _ptr(idx), T, k, N_r, _ptr(counts), _ptr(offsets), _ptr(perm), _ptr(inv_perm),
-        _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
+    _call("mr_dispatch", _device_of(idx, counts, offsets, perm, inv_perm, workspace), stream,
+          _ptr(idx), T, k, N_r, _ptr(counts), _ptr(offsets), _ptr(perm), _ptr(inv_perm),
+          _ptr(workspace), workspace.numel() * workspace.element_size())
     return counts, offsets, perm, inv_perm
 
 
@@ -227,14 +287,38 @@ def mr_dispatch_noalloc(idx, N_r, counts, offsets, perm, inv_perm=None, stream=N
     _need(perm, "perm", torch.int32, (T * k,))
     if inv_perm is not None:
         _need(inv_perm, "inv_perm", torch.int32, (T * k,))
-    _check("mr_dispatch_noalloc", lib().mr_dispatch_noalloc(
-        _ptr(idx), T, k, N_r, _ptr(counts), _ptr(offsets), _ptr(perm), _ptr(inv_perm),
-        _stream(stream)))
+    # the device made current here is the one whose scratch array the call uses
+    _call("mr_dispatch_noalloc", _device_of(idx, counts, offsets, perm, inv_perm), stream,
+          _ptr(idx), T, k, N_r, _ptr(counts), _ptr(offsets), _ptr(perm), _ptr(inv_perm))
     return counts, offsets, perm, inv_perm
 
 
 def mr_dispatch_noalloc_max_workspace() -> int:
     return int(lib().mr_dispatch_noalloc_max_workspace())
+
+
+def mr_ep_recv_order(recv_counts, R, order=None, inv_order=None, local_counts=None,
+                     local_offsets=None, stream=None):
+    """Receive-side order of the expert-parallel exchange: recv_counts
+    [ep, E_loc] int32 (device), R = its sum (rows received).  Returns
+    (order [R], inv_order [R], local_counts [E_loc], local_offsets [E_loc+1])."""
+    _need(recv_counts, "recv_counts", torch.int32)
+    ep, E_loc = recv_counts.shape
+    dev = recv_counts.device
+    order = torch.empty(R, dtype=torch.int32, device=dev) if order is None else \
+        _need(order, "order", torch.int32, (R,))
+    inv_order = torch.empty(R, dtype=torch.int32, device=dev) if inv_order is None else \
+        _need(inv_order, "inv_order", torch.int32, (R,))
+    local_counts = torch.empty(E_loc, dtype=torch.int32, device=dev) if local_counts is None \
+        else _need(local_counts, "local_counts", torch.int32, (E_loc,))
+    local_offsets = torch.empty(E_loc + 1, dtype=torch.int32, device=dev) \
+        if local_offsets is None else _need(local_offsets, "local_offsets", torch.int32,
+                                            (E_loc + 1,))
+    _call("mr_ep_recv_order", _device_of(recv_counts, order, inv_order, local_counts,
+                                          local_offsets), stream,
+          _ptr(recv_counts), ep, E_loc, int(R), _ptr(order), _ptr(inv_order),
+          _ptr(local_counts), _ptr(local_offsets))
+    return order, inv_order, local_counts, local_offsets
 
 
 def mr_gather_rows(x, k, perm=None, inv_perm=None, xs=None, stream=None):
@@ -248,8 +332,8 @@ def mr_gather_rows(x, k, perm=None, inv_perm=None, xs=None, stream=None):
         _need(inv_perm, "inv_perm", torch.int32, (T * k,))
     xs = torch.empty((T * k, d), dtype=x.dtype, device=x.device) if xs is None else \
         _need(xs, "xs", x.dtype, (T * k, d))
-    _check("mr_gather_rows", lib().mr_gather_rows(
-        _ptr(x), dt, T, d, k, _ptr(perm), _ptr(inv_perm), _ptr(xs), _stream(stream)))
+    _call("mr_gather_rows", _device_of(x, perm, inv_perm, xs), stream, _ptr(x), dt, T, d, k,
+          _ptr(perm), _ptr(inv_perm), _ptr(xs))
     return xs
 
 
@@ -266,9 +350,8 @@ def mr_combine(expert_out, w, inv_perm, shared=None, y=None, stream=None):
         _need(shared, "shared", expert_out.dtype, (T, d))
     y = torch.empty((T, d), dtype=expert_out.dtype, device=expert_out.device) if y is None else \
         _need(y, "y", expert_out.dtype, (T, d))
-    _check("mr_combine", lib().mr_combine(
-        _ptr(expert_out), dt, _ptr(w), _ptr(inv_perm), _ptr(shared), _ptr(y), T, d, k,
-        _stream(stream)))
+    _call("mr_combine", _device_of(expert_out, w, inv_perm, shared, y), stream,
+          _ptr(expert_out), dt, _ptr(w), _ptr(inv_perm), _ptr(shared), _ptr(y), T, d, k)
     return y
 
 
@@ -278,5 +361,10 @@ def mr_launch_count() -> int:
 
 
 def mr_get_error(stream=None) -> int:
-    """Synchronise the stream and read/clear the device error flag (status)."""
-    return int(lib().mr_get_error(_stream(stream)))
+    """Synchronise the stream and read/clear the error flag of the stream's
+    device (default: the current stream of the current device); returns the
+    status."""
+    if stream is None:
+        return int(lib().mr_get_error(_stream(None)))
+    with torch.cuda.device(stream.device):
+        return int(lib().mr_get_error(C.c_void_p(stream.cuda_stream)))

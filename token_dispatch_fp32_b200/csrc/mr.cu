@@ -11,6 +11,7 @@
 #include <mutex>
 
 #include "dispatch.cuh"
+#include "ep.cuh"
 #include "mr_common.cuh"
 #include "router_ffma.cuh"
 #include "router_splitk.cuh"
@@ -129,13 +130,13 @@ bool tc_shape_ok(const void* x, int x_dtype, const float* W, int d, int N_r) {
   return x_dtype == MR_F32 && d % 4 == 0 && n_ok && aligned16(x) && aligned16(W);
 }
 
-template <int NJ, bool XBF16>
-int launch_ffma_nj(const void* x, const float* W, const float* bias, int T, int d, int N_r,
+template <int NJ, bool XBF16, bool WBF16>
+int launch_ffma_nj(const void* x, const void* W, const float* bias, int T, int d, int N_r,
                    int n_group, int topk_group, int k, float route_scale, int mask_mode,
                    int flags, int32_t* idx_out, float* w_out, float* logits_out,
                    cudaStream_t st) {
   const size_t smem = mr::ffma_smem_bytes(NJ);
-  auto kern = mr::router_ffma_kernel<NJ, XBF16>;
+  auto kern = mr::router_ffma_kernel<NJ, XBF16, WBF16>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
       cudaSuccess)
     return MR_ERR_CUDA;
@@ -146,16 +147,16 @@ int launch_ffma_nj(const void* x, const float* W, const float* bias, int T, int 
   return launch_status();
 }
 
-template <bool XBF16>
-int launch_ffma(const void* x, const float* W, const float* bias, int T, int d, int N_r,
+template <bool XBF16, bool WBF16 = false>
+int launch_ffma(const void* x, const void* W, const float* bias, int T, int d, int N_r,
                 int n_group, int topk_group, int k, float route_scale, int mask_mode, int flags,
                 int32_t* idx_out, float* w_out, float* logits_out, cudaStream_t st) {
   const int nj = (N_r + 31) / 32;
 #define MR_FFMA_CASE(NJV)                                                                       \
   if (nj <= NJV)                                                                              \
-    return launch_ffma_nj<NJV, XBF16>(x, W, bias, T, d, N_r, n_group, topk_group, k,          \
-                                      route_scale, mask_mode, flags, idx_out, w_out,          \
-                                      logits_out, st);
+    return launch_ffma_nj<NJV, XBF16, WBF16>(x, W, bias, T, d, N_r, n_group, topk_group, k,   \
+                                             route_scale, mask_mode, flags, idx_out, w_out,   \
+                                             logits_out, st);
   MR_FFMA_CASE(1)
   MR_FFMA_CASE(2)
   MR_FFMA_CASE(4)
@@ -215,7 +216,8 @@ int splitk_max_clusters(size_t smem) {
   return n;
 }
 
-SplitKShape splitk_shape(int T, int d, int N_r, int sms, bool x_bf16) {
+// bm: W and x both bf16 (kind::f16 on the staged tiles).
+SplitKShape splitk_shape(int T, int d, int N_r, int sms, bool x_bf16, bool bm = false) {
   SplitKShape k;
   k.NT = ((T + 15) / 16) * 16;
   if (k.NT > mr::sk::kMaxNT) k.NT = mr::sk::kMaxNT;
@@ -229,7 +231,7 @@ SplitKShape splitk_shape(int T, int d, int N_r, int sms, bool x_bf16) {
   k.CL = 1;
   if (ks >= 2 * mr::sk::kCluster) {
     // as many clusters as fit at once (one wave), kCluster slices each
-    const mr::sk::Plan pl = mr::sk::make_plan(k.NT, (k.KC + ks - 1) / ks, x_bf16);
+    const mr::sk::Plan pl = mr::sk::make_plan(k.NT, (k.KC + ks - 1) / ks, x_bf16, bm);
     int per_tile = ks / mr::sk::kCluster;
     const int fit = splitk_max_clusters(pl.total + 1024);
     if (fit > 0 && per_tile * k.MT * k.TT > fit) per_tile = fit / (k.MT * k.TT);
@@ -272,15 +274,24 @@ int launch_reduce_nj(const float* part, int KS, int T, int N_r, const float* bia
   return MR_OK;
 }
 
+// W fp32 (3xTF32, or one tf32 product without use3x), or W stored in bf16
+// (wb16 non-null; x must be bf16: kind::f16 MMAs on the staged tiles).
 int launch_splitk(const void* x, bool x_bf16, const float* W, const float* bias, int T, int d,
                   int N_r, int n_group, int topk_group, int k, float route_scale, int mask_mode,
                   int flags, bool use3x, int32_t* idx_out, float* w_out, float* logits_out,
-                  void* ws, int sms, cudaStream_t st) {
-  const SplitKShape sh = splitk_shape(T, d, N_r, sms, x_bf16);
-  const mr::sk::Plan plan = mr::sk::make_plan(sh.NT, (sh.KC + sh.KS - 1) / sh.KS, x_bf16);
+                  void* ws, int sms, cudaStream_t st, const void* wb16 = nullptr) {
+  const bool bm = wb16 != nullptr;
+  const SplitKShape sh = splitk_shape(T, d, N_r, sms, x_bf16, bm);
+  const mr::sk::Plan plan = mr::sk::make_plan(sh.NT, (sh.KC + sh.KS - 1) / sh.KS, x_bf16, bm);
   CUtensorMap mw, mx;
-  if (!make_map_f32(&mw, W, (uint64_t)N_r, (uint64_t)d, mr::tc::BM, mr::tc::BK)) return MR_ERR_CUDA;
-  if (x_bf16) {
+  if (bm) {
+    if (!x_bf16) return MR_ERR_UNSUPPORTED;
+    if (!make_map_bf16(&mw, wb16, (uint64_t)N_r, (uint64_t)d, mr::tc::BM) ||
+        !make_map_bf16(&mx, x, (uint64_t)T, (uint64_t)d, sh.NT))
+      return MR_ERR_CUDA;
+  } else if (!make_map_f32(&mw, W, (uint64_t)N_r, (uint64_t)d, mr::tc::BM, mr::tc::BK)) {
+    return MR_ERR_CUDA;
+  } else if (x_bf16) {
     if (!make_map_bf16(&mx, x, (uint64_t)T, (uint64_t)d, sh.NT, /*swizzle=*/false))
       return MR_ERR_CUDA;
   } else if (!make_map_f32(&mx, static_cast<const float*>(x), (uint64_t)T, (uint64_t)d, sh.NT,
@@ -297,6 +308,7 @@ int launch_splitk(const void* x, bool x_bf16, const float* W, const float* bias,
   P.num_kc = sh.KC;
   P.use3x = use3x ? 1 : 0;
   P.x_bf16 = x_bf16 ? 1 : 0;
+  P.bf16_mma = bm ? 1 : 0;
   P.part = static_cast<float*>(ws);
   const size_t smem = plan.total + 1024;
   if (cudaFuncSetAttribute(mr::sk::router_splitk_gemm_kernel,
@@ -370,14 +382,16 @@ size_t wlo_bytes(int d, int N_r) { return (size_t)N_r * (size_t)d * sizeof(float
 size_t planes_bytes(int d, int N_r) { return 3 * (size_t)N_r * (size_t)d * 2; }
 
 // x fp32 with tf32 arithmetic (use3x: 3xTF32), or x bf16 with W as three
-// bf16 planes (bf16x3, planes written into `ws` here).
+// bf16 planes (bf16x3, planes written into `ws` here), or x bf16 with W
+// stored in bf16 (wbf16 non-null: one plane, W itself, no split).
 int launch_tc(const void* x, const float* W, const float* bias, int T, int d, int N_r,
               int n_group, int topk_group, int k, float route_scale, int mask_mode, int flags,
               bool use3x, bool bf16x3, int32_t* idx_out, float* w_out, float* logits_out,
-              float* wlo, void* ws, int sms, cudaStream_t st) {
+              float* wlo, void* ws, int sms, cudaStream_t st, const void* wbf16 = nullptr) {
+  const int nplanes = wbf16 ? 1 : 3;
   TcShape shp = tc_shape(T, N_r, sms, bf16x3);
   auto fits = [&](const TcShape& t) {
-    const mr::tc::Plan p = mr::tc::make_plan(N_r / t.CS, bf16x3, t.pair);
+    const mr::tc::Plan p = mr::tc::make_plan(N_r / t.CS, bf16x3, t.pair, nplanes);
     return p.stages >= 2 && mr::tc::epilogue_smem_bytes(n_group) <= p.stages * p.stage_bytes;
   };
   if (!fits(shp) && shp.pair) shp = {1, false};  // a pair's ring is half the size
@@ -385,17 +399,21 @@ int launch_tc(const void* x, const float* W, const float* bias, int T, int d, in
   const int CS = shp.CS;
   const bool pair = shp.pair;
   const int NL = N_r / CS;
-  const mr::tc::Plan plan = mr::tc::make_plan(NL, bf16x3, pair);
+  const mr::tc::Plan plan = mr::tc::make_plan(NL, bf16x3, pair, nplanes);
   CUtensorMap mx, mw, mwlo;
   const bool use_wlo = !bf16x3 && use3x && wlo != nullptr;
   if (bf16x3) {
-    const long n = (long)N_r * d;
-    __nv_bfloat16* planes = static_cast<__nv_bfloat16*>(ws);
-    mr::tc::split_planes_kernel<<<(unsigned)std::min<long>((n / 8 + 255) / 256 + 1, (long)sms * 8),
-                                  256, 0, st>>>(W, planes, n);
-    if (launch_status() != MR_OK) return MR_ERR_CUDA;
+    const void* planes = wbf16;
+    if (!wbf16) {
+      const long n = (long)N_r * d;
+      mr::tc::split_planes_kernel<<<(unsigned)std::min<long>((n / 8 + 255) / 256 + 1,
+                                                             (long)sms * 8),
+                                    256, 0, st>>>(W, static_cast<__nv_bfloat16*>(ws), n);
+      if (launch_status() != MR_OK) return MR_ERR_CUDA;
+      planes = ws;
+    }
     if (!make_map_bf16(&mx, x, (uint64_t)T, (uint64_t)d, mr::tc::BM)) return MR_ERR_CUDA;
-    if (!make_map_bf16(&mw, planes, 3 * (uint64_t)N_r, (uint64_t)d, pair ? NL / 2 : NL))
+    if (!make_map_bf16(&mw, planes, (uint64_t)nplanes * N_r, (uint64_t)d, pair ? NL / 2 : NL))
       return MR_ERR_CUDA;
     mwlo = mw;
   } else {
@@ -430,6 +448,7 @@ int launch_tc(const void* x, const float* W, const float* bias, int T, int d, in
   P.wlo = use_wlo ? 1 : 0;
   P.bf16x3 = bf16x3 ? 1 : 0;
   P.pair = pair ? 1 : 0;
+  P.nplanes = nplanes;
   P.route_scale = route_scale;
   P.bias = bias;
   P.idx_out = idx_out;
@@ -472,6 +491,75 @@ int launch_tc(const void* x, const float* W, const float* bias, int T, int d, in
   return launch_status();
 }
 
+// ---- the plain router's split-K partials --------------------------------------
+//
+// mr_router_forward has no workspace argument, so its small-batch (split-K)
+// path keeps the partial logits in a fixed array of the library's device image
+// (every device that loads the library holds one copy until the process
+// exits).  Host code may not use the symbol as a pointer: its device address
+// is looked up per device, with that device current, and only a successful
+// lookup is kept.  All calls on a device share the array; the library orders
+// them across streams with one event per device (each use waits for the
+// previous use's event and records its own), except inside stream capture,
+// where it adds no dependency.
+constexpr size_t kRouterScratchBytes = size_t(2) << 20;
+static __device__ __align__(256) float g_router_scratch[kRouterScratchBytes / sizeof(float)];
+
+std::atomic<float*> g_router_scratch_ptr[kMaxDevices];
+std::mutex g_router_scratch_mu[kMaxDevices];
+cudaEvent_t g_router_scratch_done[kMaxDevices];
+
+float* router_scratch(int dev) {
+  float* p = g_router_scratch_ptr[dev].load(std::memory_order_acquire);
+  if (p) return p;
+  std::lock_guard<std::mutex> lock(g_router_scratch_mu[dev]);
+  p = g_router_scratch_ptr[dev].load(std::memory_order_relaxed);
+  if (p) return p;
+  void* addr = nullptr;
+  if (cudaGetSymbolAddress(&addr, g_router_scratch) != cudaSuccess || !addr) {
+    (void)cudaGetLastError();
+    return nullptr;
+  }
+  p = static_cast<float*>(addr);
+  g_router_scratch_ptr[dev].store(p, std::memory_order_release);
+  return p;
+}
+
+// One use of the array on `s`: holds the device's lock, makes `s` wait for
+// the previous use (outside stream capture), and records this use's event.
+class RouterScratchUse {
+ public:
+  RouterScratchUse(int dev, cudaStream_t s) : dev_(dev), s_(s), lock_(g_router_scratch_mu[dev]) {
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(s, &cap) != cudaSuccess) {
+      (void)cudaGetLastError();
+      cap = cudaStreamCaptureStatusActive;  // unknown: add no event
+    }
+    order_ = cap == cudaStreamCaptureStatusNone;
+    if (!order_) return;
+    if (!g_router_scratch_done[dev] &&
+        cudaEventCreateWithFlags(&g_router_scratch_done[dev], cudaEventDisableTiming) !=
+            cudaSuccess) {
+      g_router_scratch_done[dev] = nullptr;
+      ok_ = false;
+      return;
+    }
+    ok_ = cudaStreamWaitEvent(s, g_router_scratch_done[dev], 0) == cudaSuccess;
+  }
+  bool ok() const { return ok_; }
+  int done(int status) {
+    if (order_ && cudaEventRecord(g_router_scratch_done[dev_], s_) != cudaSuccess)
+      return MR_ERR_CUDA;
+    return status;
+  }
+
+ private:
+  int dev_;
+  cudaStream_t s_;
+  std::lock_guard<std::mutex> lock_;
+  bool order_ = false, ok_ = true;
+};
+
 // Bounded-wait self test (see mr_selftest_bounded_wait).
 __global__ void selftest_mbar_wait_kernel() {
   __shared__ __align__(8) uint64_t bar;
@@ -484,9 +572,18 @@ __global__ void selftest_mbar_wait_kernel() {
   }
 }
 
-__global__ void selftest_grid_barrier_kernel(int* counter) {
+// Arrival counter of the grid-barrier self test: a word in the library's
+// device image (no allocation); the kernel clears it before arriving.
+__device__ int g_selftest_counter = 0;
+
+__global__ void selftest_grid_barrier_kernel() {
   // only CTA 0 arrives; its target counts two CTAs
-  if (blockIdx.x == 0) mr::disp_grid_barrier(counter, 2);
+  if (threadIdx.x == 0) {
+    atomicExch(&g_selftest_counter, 0);
+    __threadfence();
+  }
+  __syncthreads();
+  mr::disp_grid_barrier(&g_selftest_counter, 2);
 }
 
 }  // namespace
@@ -500,13 +597,8 @@ int mr_selftest_bounded_wait(int which, mr_stream_t stream) {
     return launch_status();
   }
   if (which == 1) {
-    int* counter = nullptr;
-    if (cudaMallocAsync(&counter, sizeof(int), s) != cudaSuccess) return MR_ERR_CUDA;
-    if (cudaMemsetAsync(counter, 0, sizeof(int), s) != cudaSuccess) return MR_ERR_CUDA;
-    selftest_grid_barrier_kernel<<<1, 32, 0, s>>>(counter);
-    const int st = launch_status();
-    if (cudaFreeAsync(counter, s) != cudaSuccess) return MR_ERR_CUDA;
-    return st;
+    selftest_grid_barrier_kernel<<<1, 32, 0, s>>>();
+    return launch_status();
   }
   return MR_ERR_INVALID_ARG;
 }
@@ -534,6 +626,7 @@ size_t mr_router_workspace_size(int T, int d, int N_r) {
     if (!device_info(&sms, &cc)) return 0;
     need = std::max(need, std::max(splitk_shape(T, d, N_r, sms, false).ws_bytes,
                                    splitk_shape(T, d, N_r, sms, true).ws_bytes));
+    need = std::max(need, splitk_shape(T, d, N_r, sms, true, true).ws_bytes);
   }
   return need;
 }
@@ -602,9 +695,74 @@ int mr_router_forward(const float* x, const float* W, const float* bias, int T, 
   if (st != MR_OK || T == 0) return st;
   int sms = 0, cc = 0;
   if (!device_info(&sms, &cc)) return MR_ERR_CUDA;
-  const int prec = (cc == 10 && tc_shape_ok(x, MR_F32, W, d, N_r)) ? MR_PREC_3XTF32 : MR_PREC_FFMA;
+  const bool tc = cc == 10 && tc_shape_ok(x, MR_F32, W, d, N_r);
+  // Small batches (decode): the split-K path, its partial logits in the
+  // library's own array (this entry point takes no workspace).
+  if (tc && splitk_applies(T, N_r) &&
+      splitk_shape(T, d, N_r, sms, false).ws_bytes <= kRouterScratchBytes) {
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MR_ERR_CUDA;
+    float* scratch = router_scratch(dev);
+    if (!scratch) return MR_ERR_CUDA;
+    RouterScratchUse use(dev, s);
+    if (!use.ok()) return MR_ERR_CUDA;
+    st = launch_splitk(x, false, W, bias, T, d, N_r, n_group, topk_group, k, route_scale,
+                       mask_mode, 0, true, idx_out, w_out, nullptr, scratch, sms, s);
+    return use.done(st);
+  }
   return mr_router_forward_ex(x, MR_F32, W, bias, T, d, N_r, n_group, topk_group, k, route_scale,
-                              mask_mode, prec, idx_out, w_out, nullptr, nullptr, 0, stream);
+                              mask_mode, tc ? MR_PREC_3XTF32 : MR_PREC_FFMA, idx_out, w_out,
+                              nullptr, nullptr, 0, stream);
+}
+
+size_t mr_router_forward_max_scratch(void) { return kRouterScratchBytes; }
+
+int mr_router_forward_bf16w(const void* x, int x_dtype, const void* W_bf16, const float* bias,
+                            int T, int d, int N_r, int n_group, int topk_group, int k,
+                            float route_scale, int mask_mode, int flags, int32_t* idx_out,
+                            float* w_out, float* logits_out, void* workspace,
+                            size_t workspace_bytes, mr_stream_t stream) {
+  if (flags & ~(MR_SCORE_SOFTMAX | MR_GROUP_MAX | MR_NORM_NO_EPS)) return MR_ERR_INVALID_ARG;
+  int st = validate_router(x, x_dtype, static_cast<const float*>(W_bf16), T, d, N_r, n_group,
+                           topk_group, k, route_scale, mask_mode, MR_PREC_3XTF32, idx_out, w_out);
+  if (st != MR_OK || T == 0) return st;
+  int sms = 0, cc = 0;
+  if (!device_info(&sms, &cc)) return MR_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const bool n_ok = N_r <= 256 ? (N_r % 16 == 0 && N_r >= 16) : (N_r % 32 == 0);
+  const bool tc = cc == 10 && x_dtype == MR_BF16 && d % 8 == 0 && n_ok && aligned16(x) &&
+                  aligned16(W_bf16);
+  if (tc && splitk_applies(T, N_r)) {
+    const size_t need = splitk_shape(T, d, N_r, sms, true, true).ws_bytes;
+    if (workspace && aligned16(workspace) && workspace_bytes >= need)
+      return launch_splitk(x, true, nullptr, bias, T, d, N_r, n_group, topk_group, k,
+                           route_scale, mask_mode, flags, false, idx_out, w_out, logits_out,
+                           workspace, sms, s, W_bf16);
+    if (!workspace && need <= kRouterScratchBytes) {
+      int dev = 0;
+      if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MR_ERR_CUDA;
+      float* scratch = router_scratch(dev);
+      if (!scratch) return MR_ERR_CUDA;
+      RouterScratchUse use(dev, s);
+      if (!use.ok()) return MR_ERR_CUDA;
+      st = launch_splitk(x, true, nullptr, bias, T, d, N_r, n_group, topk_group, k, route_scale,
+                         mask_mode, flags, false, idx_out, w_out, logits_out, scratch, sms, s,
+                         W_bf16);
+      return use.done(st);
+    }
+  }
+  if (tc)
+    return launch_tc(x, nullptr, bias, T, d, N_r, n_group, topk_group, k, route_scale, mask_mode,
+                     flags, true, true, idx_out, w_out, logits_out, nullptr, nullptr, sms, s,
+                     W_bf16);
+  return x_dtype == MR_BF16
+             ? launch_ffma<true, true>(x, W_bf16, bias, T, d, N_r, n_group, topk_group, k,
+                                       route_scale, mask_mode, flags, idx_out, w_out, logits_out,
+                                       s)
+             : launch_ffma<false, true>(x, W_bf16, bias, T, d, N_r, n_group, topk_group, k,
+                                        route_scale, mask_mode, flags, idx_out, w_out,
+                                        logits_out, s);
 }
 
 // ---- dispatch -----------------------------------------------------------------
@@ -689,18 +847,28 @@ int mr_dispatch(const int32_t* idx, int T, int k, int N_r, int32_t* counts, int3
 constexpr size_t kNoAllocScratchBytes = size_t(1) << 20;
 static __device__ __align__(256) int32_t g_dispatch_scratch[kNoAllocScratchBytes / sizeof(int32_t)];
 
-int32_t* g_noalloc_ptr[kMaxDevices];
-std::once_flag g_noalloc_once[kMaxDevices];
+std::atomic<int32_t*> g_noalloc_ptr[kMaxDevices];
+std::mutex g_noalloc_mu;
 
+// Device address of the scratch array on the current device.  Only a
+// successful lookup is cached: after a failed one (nullptr returned, the
+// error cleared) the next call on that device tries again.
 int32_t* noalloc_scratch() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-  std::call_once(g_noalloc_once[dev], [dev] {
-    void* p = nullptr;
-    const cudaError_t e = cudaGetSymbolAddress(&p, g_dispatch_scratch);
-    g_noalloc_ptr[dev] = e == cudaSuccess ? static_cast<int32_t*>(p) : nullptr;
-  });
-  return g_noalloc_ptr[dev];
+  int32_t* p = g_noalloc_ptr[dev].load(std::memory_order_acquire);
+  if (p) return p;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  p = g_noalloc_ptr[dev].load(std::memory_order_relaxed);
+  if (p) return p;
+  void* addr = nullptr;
+  if (cudaGetSymbolAddress(&addr, g_dispatch_scratch) != cudaSuccess || !addr) {
+    (void)cudaGetLastError();
+    return nullptr;
+  }
+  p = static_cast<int32_t*>(addr);
+  g_noalloc_ptr[dev].store(p, std::memory_order_release);
+  return p;
 }
 
 size_t mr_dispatch_noalloc_max_workspace(void) { return kNoAllocScratchBytes; }
@@ -738,6 +906,24 @@ int mr_dispatch_noalloc(const int32_t* idx, int T, int k, int N_r, int32_t* coun
     return MR_ERR_CUDA;
   mr::dispatch_scatter_kernel<<<(unsigned)nchunks, mr::kDispThreads, smem, s>>>(idx, n, N_r, hist,
                                                                                 perm, inv_perm);
+  return launch_status();
+}
+
+// ---- expert-parallel receive order ------------------------------------------
+
+int mr_ep_recv_order(const int32_t* recv_counts, int ep, int E_loc, int R, int32_t* order,
+                     int32_t* inv_order, int32_t* local_counts, int32_t* local_offsets,
+                     mr_stream_t stream) {
+  if (ep <= 0 || E_loc <= 0 || R < 0) return MR_ERR_INVALID_ARG;
+  if ((long)ep * E_loc > mr::kEpMaxSegments) return MR_ERR_UNSUPPORTED;
+  if (!recv_counts || !local_counts || !local_offsets || (R > 0 && !order))
+    return MR_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const unsigned grid = (unsigned)std::max<long>(1, ((long)R + mr::kEpRowsPerCta - 1) /
+                                                        mr::kEpRowsPerCta);
+  mr::ep_recv_order_kernel<<<grid, mr::kEpThreads, 0, s>>>(recv_counts, ep, E_loc, R, order,
+                                                            inv_order, local_counts,
+                                                            local_offsets);
   return launch_status();
 }
 

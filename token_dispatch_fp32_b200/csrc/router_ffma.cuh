@@ -17,9 +17,10 @@ __host__ __device__ constexpr size_t ffma_smem_bytes(int nj) {
                                   kFfmaTokens * (32 * nj + 1));
 }
 
-template <int NJ, bool XBF16>
+// XBF16: x rows stored in bf16; WBF16: W stored in bf16 (both widened exactly).
+template <int NJ, bool XBF16, bool WBF16 = false>
 __global__ void __launch_bounds__(kFfmaThreads)
-    router_ffma_kernel(const void* __restrict__ xv, const float* __restrict__ W,
+    router_ffma_kernel(const void* __restrict__ xv, const void* __restrict__ Wv,
                        const float* __restrict__ bias, int T, int d, int N_r, int n_group,
                        int topk_group, int k, float route_scale, int mask_mode, int flags,
                        int32_t* __restrict__ idx_out, float* __restrict__ w_out,
@@ -58,7 +59,14 @@ __global__ void __launch_bounds__(kFfmaThreads)
     for (int i = threadIdx.x; i < NP * kFfmaBK; i += kFfmaThreads) {
       const int e = i / kFfmaBK, kk = i % kFfmaBK;
       const int gk = k0 + kk;
-      ws[kk * WLD + e] = (e < N_r && gk < d) ? W[(long)e * d + gk] : 0.0f;
+      float v = 0.0f;
+      if (e < N_r && gk < d) {
+        if (WBF16)
+          v = mr_bf16_to_f32(static_cast<const uint16_t*>(Wv)[(long)e * d + gk]);
+        else
+          v = static_cast<const float*>(Wv)[(long)e * d + gk];
+      }
+      ws[kk * WLD + e] = v;
     }
     __syncthreads();
 #pragma unroll 4

@@ -14,8 +14,11 @@
 // and only lo = v - trunc(v) is written): W_hi*x_hi + W_lo*x_hi + W_hi*x_lo.
 // bf16 activations are staged by TMA as bf16 and widened into the fp32 B tile
 // by the workers; a bf16 value is exact in tf32, so x_lo = 0 and its MMA is
-// skipped.  A slice spans only a few K chunks, so the tensor core's
-// round-toward-zero accumulation stays within a few ulp.
+// skipped.  With W stored in bf16 and bf16 rows (bf16_mma), both tiles are
+// staged by TMA with the 64-byte swizzle and feed kind::f16 MMAs directly:
+// W*x is exact in fp32, no conversion, one product per multiply-add.  A slice
+// spans only a few K chunks, so the tensor core's round-toward-zero
+// accumulation stays within a few ulp.
 //
 // Reduction: the CL CTAs of a cluster hold consecutive K slices of the same
 // (expert tile, token tile).  Each copies its partial tile from TMEM to shared
@@ -42,6 +45,7 @@ constexpr int kCluster = 8;     // CTAs per cluster reduction (when KS allows)
 
 struct Params {
   int T, d, N, NT, KS, CL, num_kc, use3x, x_bf16;
+  int bf16_mma;  // W and x both bf16: kind::f16 on the staged tiles
   float* part;  // [KS / CL][T][N]
 };
 
@@ -50,14 +54,17 @@ struct Plan {
   uint32_t a_bytes, b_bytes, hi_bytes, xs_bytes, stage_bytes, bar_off, misc_off, total;
 };
 
-// Stage: [A hi (W) | B hi (x fp32)] [A lo | B lo] [x bf16 staging].
-__host__ __device__ inline Plan make_plan(int NT, int max_chunks, bool x_bf16) {
+// Stage: [A hi (W) | B hi (x fp32)] [A lo | B lo] [x bf16 staging]; with
+// bf16_mma: [A (W bf16) | B (x bf16)], 64-byte rows.
+__host__ __device__ inline Plan make_plan(int NT, int max_chunks, bool x_bf16,
+                                          bool bf16_mma = false) {
   Plan p;
-  p.a_bytes = BM * BK * 4;                 // 128 experts
-  p.b_bytes = NT * BK * 4;                 // NT tokens
+  const uint32_t esz = bf16_mma ? 2 : 4;
+  p.a_bytes = BM * BK * esz;               // 128 experts
+  p.b_bytes = NT * BK * esz;               // NT tokens
   p.hi_bytes = p.a_bytes + p.b_bytes;
-  p.xs_bytes = x_bf16 ? NT * BK * 2 : 0;
-  p.stage_bytes = align_up(2 * p.hi_bytes + p.xs_bytes, 1024);
+  p.xs_bytes = (x_bf16 && !bf16_mma) ? NT * BK * 2 : 0;
+  p.stage_bytes = align_up((bf16_mma ? 1 : 2) * p.hi_bytes + p.xs_bytes, 1024);
   int s = (int)((kSmemBudget - 1024 - 512 - 64) / p.stage_bytes);
   if (s > kMaxStages) s = kMaxStages;
   if (s > max_chunks) s = max_chunks < 1 ? 1 : max_chunks;
@@ -92,8 +99,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int NC = c_end - c_beg;
   const int NT = P.NT;
   const bool xb = P.x_bf16 != 0;
-  const bool conv = P.use3x || xb;  // the workers touch every stage
-  const Plan plan = make_plan(NT, (P.num_kc + P.KS - 1) / P.KS, xb);
+  const bool bm = P.bf16_mma != 0;
+  const bool conv = !bm && (P.use3x || xb);  // the workers touch every stage
+  const Plan plan = make_plan(NT, (P.num_kc + P.KS - 1) / P.KS, xb, bm);
   const int STAGES = plan.stages;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int CL = P.CL;
@@ -124,15 +132,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   // The producer (thread 0) fills the whole ring before the block-wide
   // barrier: the first loads are in flight while TMEM is being allocated.
-  const uint32_t tx = plan.a_bytes + (xb ? plan.xs_bytes : plan.b_bytes);
+  const uint32_t tx = plan.a_bytes + ((xb && !bm) ? plan.xs_bytes : plan.b_bytes);
   const int pre = NC < STAGES ? NC : STAGES;
   auto issue = [&](int i) {
     const int s = i % STAGES, kc = c_beg + i;
     const uint32_t base = smem0 + s * plan.stage_bytes;
     mbar_arrive_expect_tx(bar(B_FULL + s), tx);
     tma_load_2d(base, &map_w, bar(B_FULL + s), kc * BK, mt * BM);
-    tma_load_2d(xb ? base + 2 * plan.hi_bytes : base + plan.a_bytes, &map_x, bar(B_FULL + s),
-                kc * BK, tt * NT);
+    tma_load_2d((xb && !bm) ? base + 2 * plan.hi_bytes : base + plan.a_bytes, &map_x,
+                bar(B_FULL + s), kc * BK, tt * NT);
   };
   if (threadIdx.x == 0)
     for (int i = 0; i < pre; ++i) issue(i);
@@ -162,12 +170,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      const uint32_t idesc = make_idesc(NT);
+      const uint32_t idesc = bm ? make_idesc_bf16(NT, BM) : make_idesc(NT);
       for (int i = 0; i < NC; ++i) {
         const int s = i % STAGES;
         if (!mbar_wait(conv ? bar(B_CONV + s) : bar(B_FULL + s), (i / STAGES) & 1, abort))
           break;
         tc_fence_after();
+        if (bm) {
+          const uint32_t a = smem0 + s * plan.stage_bytes, b = a + plan.a_bytes;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint32_t ko = kk * 32;  // 16 bf16 = 32 bytes along K
+            mma_bf16(tmem_base, make_desc_sw64(a + ko), make_desc_sw64(b + ko), idesc,
+                     (i > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(bar(B_EMPTY + s));
+          continue;
+        }
         const uint32_t a_hi = smem0 + s * plan.stage_bytes;
         const uint32_t b_hi = a_hi + plan.a_bytes;
         const uint32_t a_lo = a_hi + plan.hi_bytes;

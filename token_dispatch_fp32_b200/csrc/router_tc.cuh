@@ -23,6 +23,8 @@
 //     sum to W exactly (24 significant bits); kind::f16 MMAs issue x*W1 +
 //     x*W2 + x*W3, each product exact in fp32 -- the fp32 dot product of the
 //     stored bf16 activations with the fp32 weights, up to accumulation order.
+//   bf16 weights (bf16 x, W stored in bf16): the same kernel with one plane,
+//     W itself; x*W is exact in fp32, one kind::f16 MMA per multiply-add.
 //
 // Promotion: the tensor core adds each product into its fp32 accumulator
 // rounding toward zero, so one accumulator over all d would drift by ~1 ulp per
@@ -76,6 +78,9 @@ struct Params {
   // stages its own x tile and half of W's rows, and keeps its own 128 tokens
   // x all N experts in its TMEM.
   int pair;
+  // bf16 path: the number of bf16 planes of W (3: W split into W1 + W2 + W3;
+  // 1: W itself stored in bf16, one exact product per multiply-add).
+  int nplanes;
   int flags;  // MR_SCORE_SOFTMAX | MR_GROUP_MAX | MR_NORM_NO_EPS
   float route_scale;
   const float* bias;
@@ -94,13 +99,15 @@ struct Plan {
 __host__ __device__ inline uint32_t align_up(uint32_t v, uint32_t a) { return (v + a - 1) / a * a; }
 
 // Stage layout.  tf32: [x | W] fp32 tiles (hi) followed by their residuals
-// (lo), 128-byte rows.  bf16x3: [x | W1 | W2 | W3] bf16 tiles, 64-byte rows.
-__host__ __device__ inline Plan make_plan(int NL, bool bf16x3 = false, bool pair = false) {
+// (lo), 128-byte rows.  bf16: [x | W1 | W2 | W3] bf16 tiles (nplanes = 3) or
+// [x | W] (nplanes = 1, W stored in bf16), 64-byte rows.
+__host__ __device__ inline Plan make_plan(int NL, bool bf16x3 = false, bool pair = false,
+                                          int nplanes = 3) {
   Plan p;
   const int esz = bf16x3 ? 2 : 4;
   p.a_bytes = BM * BK * esz;
   p.b_bytes = (pair ? NL / 2 : NL) * BK * esz;
-  p.hi_bytes = p.a_bytes + (bf16x3 ? 3 : 1) * p.b_bytes;
+  p.hi_bytes = p.a_bytes + (bf16x3 ? nplanes : 1) * p.b_bytes;
   p.stage_bytes = align_up((bf16x3 ? 1 : 2) * p.hi_bytes, 1024);
   // after the ring: 256 B of mbarriers, 256 B of flags, the CTA's bias slice;
   // the launch adds 1 KB so the ring can start on a 1024-byte boundary
@@ -524,7 +531,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   // The 2-SM instructions exist only in the PAIR instantiation: a kernel that
   // contains them must be launched in clusters of two.
   constexpr bool pair = PAIR;
-  const Plan plan = make_plan(NL, bf16x3, pair);
+  const int NP = P.nplanes;
+  const Plan plan = make_plan(NL, bf16x3, pair, NP);
   const int STAGES = plan.stages;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t crank = (P.CS > 1 || pair) ? cluster_rank() : 0u;
@@ -621,8 +629,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t fb = cluster_addr(bar(B_FULL + s), 0);
           if (leader) mbar_arrive_expect_tx(bar(B_FULL + s), 2 * tx);
           tma_load_2d_pair(base, &map_x, fb, kc * BK, m0);
-#pragma unroll
-          for (int pl = 0; pl < 3; ++pl)
+#pragma unroll 3
+          for (int pl = 0; pl < NP; ++pl)
             tma_load_2d_pair(base + plan.a_bytes + pl * plan.b_bytes, &map_w, fb, kc * BK,
                              pl * P.N + wrow0);
           continue;
@@ -630,8 +638,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive_expect_tx(bar(B_FULL + s), tx);
         tma_load_2d(base, &map_x, bar(B_FULL + s), kc * BK, m0);
         if (bf16x3) {
-#pragma unroll
-          for (int pl = 0; pl < 3; ++pl)
+#pragma unroll 3
+          for (int pl = 0; pl < NP; ++pl)
             tma_load_2d(base + plan.a_bytes + pl * plan.b_bytes, &map_w, bar(B_FULL + s),
                         kc * BK, pl * P.N + col0);
         } else {
@@ -672,8 +680,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int kk = 0; kk < BK / 16; ++kk) {
             const uint32_t ko = kk * 32;  // 16 bf16 = 32 bytes along K
             const uint64_t da = make_desc_sw64(a + ko);
-#pragma unroll
-            for (int pl = 0; pl < 3; ++pl) {
+#pragma unroll 3
+            for (int pl = 0; pl < NP; ++pl) {
               const uint64_t db = make_desc_sw64(a + plan.a_bytes + pl * plan.b_bytes + ko);
               const uint32_t acc = (!first || kk > 0 || pl > 0) ? 1u : 0u;
               if constexpr (PAIR)

@@ -23,7 +23,8 @@ Random recipe (stated once, used everywhere):
   grandchild sequence, so the values do not depend on thread count.
 * x: N(0,1).  For bf16 workloads x is quantised to bf16 (round to nearest
   even) and the fp32 copy holds the widened bf16 values exactly.
-* W: N(0,1)/sqrt(d) in fp32 (logits ~ N(0,1)).
+* W: N(0,1)/sqrt(d) in fp32 (logits ~ N(0,1)); the bf16-stored gate weight
+  is that W rounded to bf16 (nearest even).
 * b: U(lo, hi) fp32; the skewed workload adds +1.0 to experts [0, 32).
 * E (synthetic expert outputs, expert-sorted rows [T*k, d]) and shared
   ([T, d]): N(0,1), bf16 for bf16 workloads, fp32 otherwise.
@@ -155,6 +156,14 @@ def gen_W(w: Workload) -> np.ndarray:
     """Gate weight [N_r, d] fp32, N(0, 1/d)."""
     z = _normal_blocks(_child(w.seed, "W"), w.N_r * w.d, F32).reshape(w.N_r, w.d)
     return (z / np.float32(math.sqrt(w.d))).astype(np.float32)
+
+
+def gen_W_bf16(w: Workload) -> dict:
+    """The gate weight stored in bf16: gen_W rounded to bf16 (nearest even).
+    Returns the bf16 bit patterns [N_r, d] (uint16) and their exact fp32
+    values."""
+    bits = to_bf16_bits(gen_W(w))
+    return {"W_bf16": bits, "W_f32": bf16_bits_to_f32(bits)}
 
 
 def gen_b(w: Workload) -> np.ndarray | None:
