@@ -286,6 +286,71 @@ def aggregate_tokens_per_s(world: int, T: int, ms_max: float) -> float:
 # ---------------------------------------------------------------------------
 # GPU arm
 
+def run_router_only(args, w: wl.Workload):
+    """The router stage alone on the workload (a profiling aid: ncu captures
+    of the router run this), in the benchmark's launch configuration: bf16
+    rows above 256 tokens through mr_router_forward_ex (bf16x3, workspace);
+    otherwise the plain entry point on fp32 rows.  --router-weights bf16
+    times mr_router_forward_bf16w instead.  Prints one JSON line."""
+    import torch
+
+    import token_dispatch_fp32_b200 as mr
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.Stream(dev)
+    d = wl.gen_router_inputs(w)
+    bf16_rows = w.io_dtype == wl.BF16
+    x32 = torch.from_numpy(d["x_f32"]).to(dev)
+    xb = torch.from_numpy(d["x_bf16"]).view(torch.bfloat16).to(dev) if bf16_rows else None
+    Wd = torch.from_numpy(d["W"]).to(dev)
+    Wb = torch.from_numpy(wl.gen_W_bf16(w)["W_bf16"]).view(torch.bfloat16).to(dev)
+    bd = torch.from_numpy(d["b"]).to(dev)
+    idx = torch.empty((w.T, w.k), dtype=torch.int32, device=dev)
+    wt = torch.empty((w.T, w.k), dtype=torch.float32, device=dev)
+    ws = torch.empty(max(4, mr.mr_router_workspace_size(w.T, w.d, w.N_r)), dtype=torch.uint8,
+                     device=dev)
+    if args.router_weights == "bf16":
+        how = "mr_router_forward_bf16w (bf16 rows, bf16 W)"
+
+        def call():
+            mr.mr_router_forward_bf16w(xb if bf16_rows else x32, Wb, bd, w.n_group, w.topk_group,
+                                       w.k, w.route_scale, w.mask_mode, idx_out=idx, w_out=wt,
+                                       workspace=ws, stream=stream)
+    elif bf16_rows and w.T > 256:
+        how = "mr_router_forward_ex (bf16 rows, bf16x3)"
+
+        def call():
+            mr.mr_router_forward_ex(xb, Wd, bd, w.n_group, w.topk_group, w.k, w.route_scale,
+                                    w.mask_mode, precision=mr.MR_PREC_BF16X3, idx_out=idx,
+                                    w_out=wt, workspace=ws, stream=stream)
+    else:
+        how = "mr_router_forward (fp32 rows)"
+
+        def call():
+            mr.mr_router_forward(x32, Wd, bd, w.n_group, w.topk_group, w.k, w.route_scale,
+                                 w.mask_mode, idx_out=idx, w_out=wt, stream=stream)
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    l0 = mr.mr_launch_count()
+    e0.record(stream)
+    for _ in range(args.steps):
+        call()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    assert mr.mr_get_error(stream) == mr.MR_OK
+    ms = e0.elapsed_time(e1) / args.steps
+    fl = 2.0 * w.T * w.d * w.N_r
+    print(json.dumps({"only": "router", "workload": w.name, "entry_point": how,
+                      "ms": ms, "steps": args.steps, "warmup": args.warmup,
+                      "launches_per_call": (mr.mr_launch_count() - l0) / args.steps,
+                      "tflops_algorithmic": fl / (ms / 1e3) / 1e12,
+                      "tc_cluster_pin": os.environ.get("MR_TC_CLUSTER"),
+                      "l2": "back-to-back calls (inputs of the full workloads exceed L2)"}),
+          flush=True)
+
+
 def run_ours(args, w: wl.Workload, rank: int, world: int):
     import torch
     import torch.distributed as dist
@@ -454,6 +519,47 @@ def run_ours(args, w: wl.Workload, rank: int, world: int):
                                   "tflops_issued": 3 * of / (oms / 1e3) / 1e12,
                                   "l2": "read pass over 512 MB before each call"}
             del ox, oW, ob, oidx, owt, ows
+        assert mr.mr_get_error(stream) == mr.MR_OK
+
+    # One synthetic expert layer (d -> 2048, the DeepSeek-V3 expert width) over
+    # the expert-sorted rows of the DeepSeek-V3 prefill batch, with the row
+    # gather fused into the grouped GEMM; beside it the unfused pair (the
+    # sorted rows written by mr_gather_rows, then the same GEMM reading them
+    # through an identity permutation).
+    expert = None
+    if args.workload == wl.V3_FULL.name and not args.no_extra_stages:
+        we, n_out = wl.V3_PREFILL, 2048
+        ein = wl.gen_router_inputs(we)
+        ex = torch.from_numpy(ein["x_bf16"]).view(torch.bfloat16).to(dev)
+        ews = torch.empty(max(4, mr.mr_router_workspace_size(we.T, we.d, we.N_r)),
+                          dtype=torch.uint8, device=dev)
+        eidx, ewt = mr.mr_router_forward_ex(ex, torch.from_numpy(ein["W"]).to(dev),
+                                            torch.from_numpy(ein["b"]).to(dev), we.n_group,
+                                            we.topk_group, we.k, we.route_scale, we.mask_mode,
+                                            precision=mr.MR_PREC_BF16X3, workspace=ews,
+                                            stream=stream)
+        ecounts, eoff, eperm, einv = mr.mr_dispatch(eidx, we.N_r, stream=stream)
+        eW = torch.from_numpy(wl.gen_expert_W(we, n_out)).view(torch.bfloat16).to(dev)
+        eout = torch.empty((we.T * we.k, n_out), dtype=torch.bfloat16, device=dev)
+        exs = torch.empty((we.T * we.k, we.d), dtype=torch.bfloat16, device=dev)
+        ident = torch.arange(we.T * we.k, dtype=torch.int32, device=dev)
+
+        def fused():
+            mr.mr_expert_gemm_gather(ex, we.k, eperm, eoff, eW, out=eout, stream=stream)
+
+        def unfused():
+            mr.mr_gather_rows(ex, we.k, perm=eperm, inv_perm=einv, xs=exs, stream=stream)
+            mr.mr_expert_gemm_gather(exs, 1, ident, eoff, eW, out=eout, stream=stream)
+
+        fms = time_alone(fused, n_alone)
+        ums = time_alone(unfused, n_alone)
+        ef = 2.0 * we.T * we.k * we.d * n_out
+        expert = {"workload": we.name, "n_out": n_out, "ms": fms,
+                  "tflops": ef / (fms / 1e3) / 1e12, "ms_unfused_gather_then_gemm": ums,
+                  "rows": we.T * we.k,
+                  "saved_bytes": 2 * 2 * we.T * we.k * we.d,
+                  "l2": "read pass over 512 MB before each call"}
+        del ex, ews, eW, eout, exs
         assert mr.mr_get_error(stream) == mr.MR_OK
 
     # The decode-size router (one position x batch 64): W read once per call.
@@ -630,6 +736,9 @@ def run_ours(args, w: wl.Workload, rank: int, world: int):
         st["frac_issued_of_bf16_peak"] = st["tflops_issued"] / peaks["bf16_tflops"]
         st["frac_algorithmic_of_bf16_peak"] = st["tflops_algorithmic"] / peaks["bf16_tflops"]
         stages[key] = st
+    if expert is not None:
+        expert["frac_of_bf16_peak"] = expert["tflops"] / peaks["bf16_tflops"]
+        stages["expert_gemm_gather_deepseek_v3_prefill_T4096"] = expert
     if decode is not None:
         decode["frac_hbm"] = decode["gbs"] / peaks["hbm_gbs"]
         if decode.get("gbs_cuda_graph"):
@@ -699,6 +808,10 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra-stages", action="store_true",
                     help="skip the prefill-router stages timed beside the step")
+    ap.add_argument("--only", choices=("router",), default=None,
+                    help="time one stage alone (a profiling aid; no bench line)")
+    ap.add_argument("--router-weights", choices=("f32", "bf16"), default="f32",
+                    help="with --only router: the gate weight's stored type")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -716,6 +829,9 @@ def main(argv=None):
         sys.exit(2)
     if args.impl == "reference":
         run_reference(args, w, rank)
+        return
+    if args.only == "router":
+        run_router_only(args, w)
         return
     if world > 1:
         import datetime

@@ -371,6 +371,34 @@ int mr_ep_recv_order(const int32_t *recv_counts, int ep, int E_loc, int R,
                      int32_t *local_offsets, mr_stream_t stream);
 
 /*
+ * mr_expert_gemm_gather -- one expert layer over the expert-sorted rows, with
+ * the row gather fused into the GEMM (Kimi K2 "Add shared output" page,
+ * moe_infer: sorted_tokens = x[idxs // k], then
+ * expert(sorted_tokens[start_idx:end_idx]) for each expert).
+ *
+ * The expert is one linear map per expert with caller-supplied (synthetic)
+ * weights; the sorted row j belongs to expert e(j), the e with
+ * offsets[e] <= j < offsets[e + 1], and
+ *     out[j][n] = sum_c x[perm[j] / k][c] * W_exp[e(j)][n][c].
+ * The gathered rows are never written: each 128-row block of an expert's
+ * segment is loaded from x by tensor-memory-access gathers (four rows per
+ * copy, the rows taken from perm).  bf16 operands, each product exact, fp32
+ * accumulation in tensor memory, rounded to bf16 (nearest even) on output.
+ *
+ *   x        [T, d] bf16 token rows.
+ *   perm     [T*k] int32, offsets [N_r + 1] int32: from mr_dispatch.
+ *   W_exp    [N_r, n_out, d] bf16 (nn.Linear layout per expert).
+ *   out      [T*k, n_out] bf16 in expert-sorted order; rows from offsets[N_r]
+ *            on (dropped ids) are not written.
+ * Limits: d % 8 == 0, n_out % 16 == 0, N_r <= 1024, 16-byte aligned x, W_exp
+ * and out (else MR_ERR_UNSUPPORTED).  One kernel; no workspace.
+ */
+int mr_expert_gemm_gather(const void *x, const int32_t *perm,
+                          const int32_t *offsets, const void *W_exp, int T,
+                          int d, int k, int N_r, int n_out, void *out,
+                          mr_stream_t stream);
+
+/*
  * mr_gather_rows -- sorted_tokens = x[idxs // k] (Kimi K2 "Add shared output"
  * page, moe_infer).  Copies rows bit for bit.
  *

@@ -55,6 +55,8 @@ def _load():
                                    C.c_int, C.c_double, C.c_int, C.c_int, C.c_int, C.c_int,
                                    p, p, p, p, C.c_int]
         lib.mo_dispatch.argtypes = [p, C.c_int, C.c_int, C.c_int, p, p, p, p]
+        lib.mo_expert_gemm.argtypes = [p, C.c_int, C.c_int, C.c_int, p, p, C.c_int, p,
+                                       C.c_int, p, C.c_long, p, C.c_int]
         lib.mo_ep_splits.argtypes = [p, C.c_int, C.c_int, C.c_int, p, p, p]
         lib.mo_ep_recv_order.argtypes = [p, C.c_int, C.c_int, p, p]
         lib.mo_gather.argtypes = [p, C.c_long, C.c_int, C.c_int, p, p, C.c_long, p]
@@ -181,6 +183,31 @@ def all_to_all(send_blocks):
     concatenation over s, in source order (dist.all_to_all)."""
     ep = len(send_blocks)
     return [np.concatenate([send_blocks[s][r] for s in range(ep)], axis=0) for r in range(ep)]
+
+
+def expert_gemm(x_bits, k, perm, offsets, W_bits, rows=None, threads=0):
+    """One expert layer over the expert-sorted rows (Kimi K2 "Add shared
+    output" page, moe_infer: expert(sorted_tokens[start_idx:end_idx]) for
+    each expert), the expert a linear map with synthetic weights:
+    out[j] = x[perm[j] // k] . W[e(j)]^T in binary64, e(j) the expert whose
+    segment [offsets[e], offsets[e+1]) holds sorted row j.  x_bits [T,d] and
+    W_bits [N_r, n_out, d] are bf16 bit patterns (uint16); rows selects
+    sorted rows (all when None).  Returns float64 [n_rows, n_out]."""
+    x_bits = np.ascontiguousarray(x_bits, dtype=np.uint16)
+    W_bits = np.ascontiguousarray(W_bits, dtype=np.uint16)
+    perm = np.ascontiguousarray(perm, dtype=np.int32)
+    offsets = np.ascontiguousarray(offsets, dtype=np.int32)
+    T, d = x_bits.shape
+    N_r, n_out, dw = W_bits.shape
+    assert dw == d and offsets.shape == (N_r + 1,)
+    rows_a = None if rows is None else np.ascontiguousarray(rows, dtype=np.int32)
+    n = int(offsets[-1]) if rows is None else rows_a.shape[0]
+    out = np.empty((n, n_out), np.float64)
+    rc = _load().mo_expert_gemm(_ptr(x_bits), T, d, k, _ptr(perm), _ptr(offsets), N_r,
+                                _ptr(W_bits), n_out, _ptr(rows_a), n, _ptr(out), threads)
+    if rc != 0:
+        raise ValueError(f"oracle expert_gemm: index out of range (rc={rc})")
+    return out
 
 
 def gather(x, k, perm, rows=None):

@@ -455,6 +455,46 @@ int mo_ep_recv_order(const int32_t *recv_counts, int ep, int E_loc, int32_t *ord
     return MO_OK;
 }
 
+/* ------------------------------------------------------------------ */
+/* One expert layer on the expert-sorted rows ([K2-add] moe_infer: for each
+ * expert i, expert_out = expert(sorted_tokens[start_idx:end_idx])), the
+ * expert being one linear map with synthetic weights: the sorted row j
+ * (token perm[j] / k, expert e with offsets[e] <= j < offsets[e+1]) gives
+ * out[j][n] = sum_c x[token][c] * W[e][n][c], in binary64 from the bf16
+ * values of x [T][d] and W [N_r][n_out][d] (bf16 bit patterns).  rows
+ * selects a subset of sorted rows (NULL: all offsets[N_r]); out is
+ * [n_rows][n_out].  The dot products are plain sequential loops. */
+int mo_expert_gemm(const uint16_t *x, int T, int d, int k, const int32_t *perm,
+                   const int32_t *offsets, int N_r, const uint16_t *W, int n_out,
+                   const int32_t *rows, long n_rows, double *out, int nthreads)
+{
+    if (T < 0 || d <= 0 || k <= 0 || N_r <= 0 || n_out <= 0) return MO_ERR_ARG;
+    const long total = offsets[N_r];
+    int bad = 0;
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#pragma omp parallel for schedule(dynamic, 4) reduction(| : bad)
+#endif
+    for (long r = 0; r < n_rows; ++r) {
+        const long j = rows ? rows[r] : r;
+        if (j < 0 || j >= total || perm[j] < 0 || perm[j] / k >= T) {
+            bad = 1;
+            continue;
+        }
+        int e = 0;
+        while (offsets[e + 1] <= j) ++e;  /* the expert whose segment holds j */
+        const long tok = perm[j] / k;
+        for (int n = 0; n < n_out; ++n) {
+            double acc = 0.0;
+            for (int c = 0; c < d; ++c)
+                acc += mo_load(x, 1, tok * d + c) * mo_load(W, 1, ((long)e * n_out + n) * d + c);
+            out[r * n_out + n] = acc;
+        }
+    }
+    (void)nthreads;
+    return bad ? MO_ERR_RANGE : MO_OK;
+}
+
 int mo_num_threads(void)
 {
 #ifdef _OPENMP

@@ -9,8 +9,9 @@ Comparison rules (tolerances the routing path is specified with):
   * weights: within 1e-5 relative of the oracle (matched by expert id).
   * logits: |dL| <= 2e-5 * max(|L|, 1).
   * dispatch and gather: bit-exact.
-  * combine: |dy| <= 1e-2 * max(|y|, |routed|, |shared|) + 1e-5; the
-    absolute term bounds the fp32 accumulation error of k fused multiply-adds
+  * combine: |dy| <= 1e-2 * max(|y|, |routed|, |shared|) + 1e-5, plus one
+    bf16 ulp of the routed sum for bf16 rows (compare_combine); the 1e-5
+    bounds the fp32 accumulation error of k fused multiply-adds
     (k * 2^-24 * sum_j |w_j e_j| <= 8 * 6e-8 * 15 for N(0,1) rows and weights
     summing to <= 2.827), which a bf16 rounding boundary can expose.
 """
@@ -107,20 +108,39 @@ def compare_router(gidx, gw, ref, glogits=None, logit_tol=LOGIT_TOL, allow_tie_f
     return stats
 
 
-def compare_combine(gy, ry, rrouted, shared):
-    """gy: GPU y as float64 numpy; ry/rrouted from the oracle; shared float64 or None."""
+def bf16_ulp(a):
+    """Spacing of bf16 values at |a| (8 significant bits): 2^(e - 8) for
+    |a| = m * 2^e, 0.5 <= m < 1; the subnormal spacing 2^-133 at the bottom."""
+    a = np.abs(np.asarray(a, np.float64))
+    _, e = np.frexp(a)
+    return np.where(a == 0, 2.0 ** -133, np.ldexp(1.0, np.maximum(e - 8, -133)))
+
+
+def compare_combine(gy, ry, rrouted, shared, bf16=True):
+    """gy: GPU y as float64 numpy; ry/rrouted from the oracle; shared float64 or None.
+
+    bf16 rows: the pages round the fp32 routed sum to bf16, then round the
+    sum with the shared row again.  The GPU's fp32 sum differs from the exact
+    sum by far less than half a bf16 ulp, yet where the exact value sits on a
+    rounding boundary the first rounding can land one bf16 ulp of the routed
+    sum away from the oracle's, and the second rounding can add one ulp of y
+    (< 2^-7 |y|, inside the relative term).  Hence the tolerance
+    1e-2 * max(|y|, |routed|, |shared|) + ulp_bf16(routed) + 1e-5."""
     scale = np.maximum(np.abs(ry), np.abs(rrouted))
     if shared is not None:
         scale = np.maximum(scale, np.abs(shared))
     err = np.abs(gy - ry)
     tol = Y_RTOL * scale + Y_ATOL
+    if bf16:
+        tol = tol + bf16_ulp(rrouted)
     worst = np.unravel_index(np.argmax(err - tol), err.shape)
     assert (err <= tol).all(), (f"combine error at {worst}: gpu {gy[worst]} oracle {ry[worst]} "
                                 f"tol {tol[worst]}")
     rel_l2 = np.linalg.norm(gy - ry, axis=1) / np.maximum(np.linalg.norm(ry, axis=1), 1e-30)
     return {"y_max_abs": float(err.max()), "y_row_rel_l2_max": float(rel_l2.max()),
             "y_max_err_over_tol": float((err / tol).max()),
-            "y_differ_elems": int((err > 0).sum())}
+            "y_differ_elems": int((err > 0).sum()),
+            "y_beyond_1e-2_rel": int((err > Y_RTOL * scale + Y_ATOL).sum())}
 
 
 def widen(a):

@@ -1,0 +1,107 @@
+"""One expert layer over the expert-sorted rows with the row gather fused into
+the GEMM (mr_expert_gemm_gather; Kimi K2 "Add shared output" page, moe_infer:
+sorted_tokens = x[idxs // k], expert(sorted_tokens[start_idx:end_idx])),
+against the oracle's binary64 restatement.
+
+Tolerance: each bf16 x bf16 product is exact in fp32; the tensor core adds
+them into an fp32 accumulator rounding toward zero, one rounding per
+16-deep MMA step, so the accumulated value is within (d/16 + 2) * 2^-23 *
+sum_c |x_c W_c| of the exact dot product; the result is then rounded to bf16,
+which can land one bf16 ulp away where the exact value sits on a rounding
+boundary.  Hence |out - exact| <= ulp_bf16(exact) + (d/16 + 2) 2^-23 sum|xW|.
+Rows past the expert segments (dropped ids) must stay untouched."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import token_dispatch_fp32_b200 as mr
+import workloads as wl
+from parity import bf16_ulp, record
+
+pytestmark = pytest.mark.gpu
+
+
+def _ids(T, k, N_r, seed, skew):
+    rng = np.random.default_rng(seed)
+    if skew:
+        return np.where(rng.random((T, k)) < 0.7, rng.integers(0, 8, (T, k)),
+                        rng.integers(0, N_r, (T, k))).astype(np.int32)
+    return np.stack([rng.permutation(N_r)[:k] for _ in range(T)]).astype(np.int32)
+
+
+def _dev_bits(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).view(torch.bfloat16).cuda()
+
+
+CASES = [
+    # T, d, N_r, k, n_out, skew, n_check (None: every row)
+    (100, 256, 16, 4, 256, False, None),
+    (257, 200, 32, 3, 144, True, None),      # K tail (200 % 32), partial N tile
+    (64, 7168, 256, 8, 512, False, None),    # decode-size batch, most experts one block
+    (1000, 512, 64, 8, 256, True, None),     # skewed: experts with many blocks
+    (4096, 7168, 256, 8, 2048, False, 768),  # DeepSeek-V3 prefill batch, sampled rows
+]
+
+
+@pytest.mark.parametrize("T,d,N_r,k,n_out,skew,n_check", CASES,
+                         ids=[f"T{c[0]}_d{c[1]}_E{c[2]}_n{c[4]}" for c in CASES])
+def test_expert_gemm_gather_matches_oracle(T, d, N_r, k, n_out, skew, n_check):
+    w = wl.Workload(f"expert_T{T}_d{d}", T=T, d=d, N_r=N_r, n_group=1, topk_group=1, k=k,
+                    route_scale=1.0, mask_mode=0, seed=T + d + N_r)
+    rng = np.random.default_rng(w.seed)
+    x = wl.to_bf16_bits(rng.standard_normal((T, d)).astype(np.float32))
+    W = wl.gen_expert_W(w, n_out)
+    idx = _ids(T, k, N_r, w.seed, skew)
+    counts, offsets, perm, inv = oracle.dispatch(idx, N_r)
+    out = torch.full((T * k, n_out), float("nan"), dtype=torch.bfloat16, device="cuda")
+    mr.mr_expert_gemm_gather(_dev_bits(x), k, torch.from_numpy(perm).cuda(),
+                             torch.from_numpy(offsets).cuda(), _dev_bits(W), out=out)
+    assert mr.mr_get_error() == mr.MR_OK
+    if n_check is None:
+        rows = np.arange(T * k, dtype=np.int32)
+    else:  # spread over the experts, with every segment's first and last row
+        ends = np.concatenate([offsets[:-1], offsets[1:] - 1])
+        ends = ends[(ends >= 0) & (ends < T * k)]
+        rows = np.unique(np.concatenate([ends, rng.choice(T * k, n_check, replace=False)]))
+        rows = rows.astype(np.int32)
+    ref = oracle.expert_gemm(x, k, perm, offsets, W, rows=rows)
+    got = out.view(torch.int16).cpu().numpy().view(np.uint16)[rows]
+    got = wl.bf16_bits_to_f32(got).astype(np.float64)
+    xf = np.abs(wl.bf16_bits_to_f32(x).astype(np.float64))
+    Wf = np.abs(wl.bf16_bits_to_f32(W).astype(np.float64))
+    e_of = np.searchsorted(offsets, rows, side="right") - 1
+    absdot = np.stack([xf[perm[j] // k] @ Wf[e].T for j, e in zip(rows, e_of)])
+    tol = bf16_ulp(ref) + (d / 16 + 2) * 2.0 ** -23 * absdot
+    err = np.abs(got - ref)
+    assert np.isfinite(got).all()
+    worst = np.unravel_index(np.argmax(err - tol), err.shape)
+    assert (err <= tol).all(), f"row {rows[worst[0]]} col {worst[1]}: {got[worst]} vs {ref[worst]}"
+    stats = {"rows_checked": int(len(rows)), "rows": int(T * k), "max_abs_err": float(err.max()),
+             "max_err_over_tol": float((err / tol).max()),
+             "differ_from_rounded_exact": int((got != oracle.round_bf16(ref)).sum())}
+    record(w.name, "expert_gemm_gather", stats)
+    print(w.name, stats)
+
+
+def test_expert_gemm_gather_leaves_dropped_rows_alone():
+    """Ids outside [0, N_r) are dropped by the dispatch; the rows past
+    offsets[N_r] keep whatever the output held."""
+    T, d, N_r, k, n_out = 50, 64, 8, 2, 32
+    rng = np.random.default_rng(5)
+    idx = _ids(T, k, N_r, 5, False)
+    idx[3, 1] = N_r + 2
+    idx_d = torch.from_numpy(idx).cuda()
+    counts, offsets, perm, inv = mr.mr_dispatch(idx_d, N_r)
+    assert mr.mr_get_error() == mr.MR_ERR_DEVICE
+    x = wl.to_bf16_bits(rng.standard_normal((T, d)).astype(np.float32))
+    W = wl.to_bf16_bits(rng.standard_normal((N_r, n_out, d)).astype(np.float32) * 0.1)
+    out = torch.full((T * k, n_out), 7.0, dtype=torch.bfloat16, device="cuda")
+    mr.mr_expert_gemm_gather(_dev_bits(x), k, perm, offsets, _dev_bits(W), out=out)
+    assert mr.mr_get_error() == mr.MR_OK
+    n_valid = int(offsets[-1])
+    assert n_valid == T * k - 1
+    assert (out[n_valid:].float() == 7.0).all()
+    ref = oracle.expert_gemm(x, k, perm.cpu().numpy(), offsets.cpu().numpy(), W)
+    got = out[:n_valid].float().cpu().numpy().astype(np.float64)
+    assert (np.abs(got - ref) <= bf16_ulp(ref) + 1e-3).all()

@@ -45,6 +45,10 @@ MUTATIONS = {
                                  "mo_load(E, dtype, row * d + c);"),
     "combine_row_of_token_not_slot": ("long row = inv[t * k + j];", "long row = inv[t + j];"),
     "final_sum_not_rounded": ("                if (dtype == 1) y = mo_round_bf16(y);\n", ""),
+    "expert_gemm_segment_off_by_one": ("while (offsets[e + 1] <= j) ++e;",
+                                       "while (offsets[e + 1] < j) ++e;"),
+    "expert_gemm_row_is_slot": ("const long tok = perm[j] / k;\n        for (int n = 0;",
+                                "const long tok = perm[j] % T;\n        for (int n = 0;"),
     "ep_label_is_source": ("const int label = (int)(seg % E_loc);",
                            "const int label = (int)(seg / E_loc);"),
     "ep_recv_block_of_sender": ("const int32_t c = counts_all[(long)s * N_r + (long)r * E_loc + e];",

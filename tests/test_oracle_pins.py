@@ -16,6 +16,7 @@ import pytest
 from scipy.special import expit
 
 import oracle
+import workloads as wl
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "hand_cases.json")
 
@@ -557,3 +558,39 @@ def test_all_to_all_emulation():
     blocks = [[np.array([1]), np.array([2, 3])], [np.array([4, 5]), np.array([], int)]]
     got = oracle.all_to_all(blocks)
     assert got[0].tolist() == [1, 4, 5] and got[1].tolist() == [2, 3]
+
+
+# --------------------------------------------------------------------------
+# One expert layer over the expert-sorted rows (the grouped GEMM the gather
+# feeds), against numpy's matmul on fancy-indexed rows, per expert segment.
+
+@pytest.mark.parametrize("skew", [False, True])
+def test_expert_gemm_matches_numpy_per_segment(skew):
+    rng = np.random.default_rng(11 + skew)
+    T, d, N_r, k, n_out = 37, 48, 8, 3, 20
+    if skew:
+        idx = np.where(rng.random((T, k)) < 0.8, 2, rng.integers(0, N_r, (T, k)))
+    else:
+        idx = np.stack([rng.permutation(N_r)[:k] for _ in range(T)])
+    counts, offsets, perm, inv = oracle.dispatch(idx.astype(np.int32), N_r)
+    x = wl.to_bf16_bits(rng.standard_normal((T, d)).astype(np.float32))
+    W = wl.to_bf16_bits(rng.standard_normal((N_r, n_out, d)).astype(np.float32))
+    got = oracle.expert_gemm(x, k, perm, offsets, W)
+    xf = wl.bf16_bits_to_f32(x).astype(np.float64)
+    Wf = wl.bf16_bits_to_f32(W).astype(np.float64)
+    for e in range(N_r):
+        seg = slice(offsets[e], offsets[e + 1])
+        want = xf[perm[seg] // k] @ Wf[e].T
+        assert np.allclose(got[seg], want, rtol=1e-12, atol=1e-12), e
+    rows = np.array([0, offsets[3], T * k - 1], np.int32)
+    assert np.array_equal(oracle.expert_gemm(x, k, perm, offsets, W, rows=rows), got[rows])
+
+
+def test_expert_gemm_hand_case():
+    """Two tokens, two experts, k = 1: token 0 -> expert 1, token 1 -> expert 0.
+    Sorted rows: (token 1, expert 0), (token 0, expert 1)."""
+    x = wl.to_bf16_bits(np.array([[1.0, 2.0], [3.0, -1.0]], np.float32))
+    W = wl.to_bf16_bits(np.array([[[1.0, 0.0]], [[0.5, 0.25]]], np.float32))  # [2,1,2]
+    counts, offsets, perm, inv = oracle.dispatch(np.array([[1], [0]], np.int32), 2)
+    got = oracle.expert_gemm(x, 1, perm, offsets, W)
+    assert got.tolist() == [[3.0], [1.0]]  # 3*1 + -1*0 ; 1*0.5 + 2*0.25

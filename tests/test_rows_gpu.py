@@ -67,7 +67,8 @@ def test_combine_matches_oracle(T, d, k, N_r, dtype, with_shared):
                       None if sh is None else _dev(sh))
     assert mr.mr_get_error() == mr.MR_OK
     ry, rr = oracle.combine(E, w, inv, sh, k)
-    stats = compare_combine(widen(_host(y)), ry, rr, None if sh is None else widen(sh))
+    stats = compare_combine(widen(_host(y)), ry, rr, None if sh is None else widen(sh),
+                            bf16=dtype == "bf16")
     print(T, d, k, dtype, with_shared, stats)
 
 

@@ -73,6 +73,7 @@ def lib():
         L.mr_router_forward_max_scratch.restype = sz
         L.mr_gather_rows.argtypes = [p, i, i, i, i, p, p, p, p]
         L.mr_ep_recv_order.argtypes = [p, i, i, i, p, p, p, p, p]
+        L.mr_expert_gemm_gather.argtypes = [p, p, p, p, i, i, i, i, i, p, p]
         L.mr_combine.argtypes = [p, i, p, p, p, p, i, i, i, p]
         L.mr_get_error.argtypes = [p]
         L.mr_selftest_bounded_wait.argtypes = [i, p]
@@ -319,6 +320,26 @@ def mr_ep_recv_order(recv_counts, R, order=None, inv_order=None, local_counts=No
           _ptr(recv_counts), ep, E_loc, int(R), _ptr(order), _ptr(inv_order),
           _ptr(local_counts), _ptr(local_offsets))
     return order, inv_order, local_counts, local_offsets
+
+
+def mr_expert_gemm_gather(x, k, perm, offsets, W_exp, out=None, stream=None):
+    """One linear expert layer over the expert-sorted rows with the row
+    gather fused in: out [T*k, n_out] bf16, row j = x[perm[j] // k] .
+    W_exp[e(j)]^T.  x [T,d] bf16, perm [T*k], offsets [N_r+1] int32 (from
+    mr_dispatch), W_exp [N_r, n_out, d] bf16."""
+    _need(x, "x", torch.bfloat16)
+    T, d = x.shape
+    _need(perm, "perm", torch.int32, (T * k,))
+    _need(W_exp, "W_exp", torch.bfloat16)
+    N_r, n_out, dw = W_exp.shape
+    if dw != d:
+        raise ValueError(f"W_exp is [N_r, n_out, {dw}], x rows have {d} columns")
+    _need(offsets, "offsets", torch.int32, (N_r + 1,))
+    out = torch.empty((T * k, n_out), dtype=torch.bfloat16, device=x.device) if out is None \
+        else _need(out, "out", torch.bfloat16, (T * k, n_out))
+    _call("mr_expert_gemm_gather", _device_of(x, perm, offsets, W_exp, out), stream,
+          _ptr(x), _ptr(perm), _ptr(offsets), _ptr(W_exp), T, d, k, N_r, n_out, _ptr(out))
+    return out
 
 
 def mr_gather_rows(x, k, perm=None, inv_perm=None, xs=None, stream=None):

@@ -1,0 +1,229 @@
+// expert_gemm.cuh -- one expert layer over the expert-sorted rows with the
+// row gather fused into the GEMM (Kimi K2 "Add shared output" page, moe_infer:
+// sorted_tokens = x[idxs // k], then expert(sorted_tokens[start_idx:end_idx])
+// for each expert).
+//
+// The expert is one linear map per expert (synthetic weights W[e] [n_out, d],
+// bf16, nn.Linear layout): out[j] = x[perm[j] / k] . W[e(j)]^T for the sorted
+// row j, e(j) the expert whose segment [offsets[e], offsets[e+1]) holds j.
+// The gathered rows are never written to memory: the A tile of a 128-row
+// block of an expert's segment is loaded straight from the token rows x by
+// TMA tile::gather4 (four rows per copy, their indices taken from the
+// permutation), and the B tile from W[e].  tcgen05 kind::f16, M = 128,
+// N = 256, fp32 accumulation in TMEM, rounded to bf16 on the way out.
+//
+//   warp 0      producer: all 32 lanes issue the gather4 copies of a stage
+//               (lane l: rows 4l..4l+3), lane 0 also the W tile.
+//   warp 1      TMEM owner and MMA issuer (one elected thread).
+//   warps 2..5  epilogue: TMEM lanes -> bf16 -> global (one row per thread).
+//
+// Grid: x = 128-row blocks over all experts (an upper bound from the host;
+// each CTA finds its expert and block from the offsets, surplus CTAs exit),
+// y = 256-column blocks of n_out.  Every mbarrier wait is bounded.
+#pragma once
+
+#include "router_tc.cuh"
+
+namespace mr {
+namespace eg {
+
+using namespace mr::tc;
+
+constexpr int kBN = 256;                    // output columns per CTA (MMA N)
+constexpr int kThreads = 192;               // producer, MMA, 4 epilogue warps
+constexpr int kStages = 8;
+constexpr uint32_t kABytes = BM * BK * 2;   // 128 rows x 32 bf16
+constexpr uint32_t kBBytes = kBN * BK * 2;  // 256 rows x 32 bf16
+constexpr uint32_t kStageBytes = kABytes + kBBytes;
+constexpr uint32_t kBarOff = kStages * kStageBytes;
+constexpr uint32_t kSmemBytes = kBarOff + 256 + 4 * BM + 64 + 1024;
+
+struct Params {
+  int T, d, k, N_r, n_out;
+  const int32_t* perm;
+  const int32_t* offsets;
+  __nv_bfloat16* out;  // [offsets[N_r], n_out]
+};
+
+__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                            int col, int r0, int r1, int r2, int r3) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(col), "r"(r0), "r"(r1), "r"(r2),
+      "r"(r3)
+      : "memory");
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    expert_gemm_gather_kernel(const __grid_constant__ CUtensorMap map_x,
+                              const __grid_constant__ CUtensorMap map_w, const Params P) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kBarOff);
+  int* tok_s = reinterpret_cast<int*>(smem + kBarOff + 256);      // [128] token of each row
+  int* misc = reinterpret_cast<int*>(smem + kBarOff + 256 + 4 * BM);
+  volatile int* abort = reinterpret_cast<volatile int*>(misc + 4);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc + 6);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t smem0 = smem_u32(smem);
+  auto bar = [&](int i) { return smem_u32(&bars[i]); };
+  const int B_FULL = 0, B_EMPTY = kStages, B_ACC = 2 * kStages;
+
+  // ---- which expert and which 128-row block of its segment -----------------
+  // blocks of expert e: ceil(count_e / 128); a CTA-wide exclusive scan of
+  // them over the experts (thread i owns experts [i*c, (i+1)*c))
+  {
+    const int c = (P.N_r + kThreads - 1) / kThreads;
+    const int e0 = tid * c, e1 = e0 + c < P.N_r ? e0 + c : P.N_r;
+    int mine = 0;
+    for (int e = e0; e < e1; ++e) mine += (P.offsets[e + 1] - P.offsets[e] + BM - 1) / BM;
+    int x = mine;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, x, off);
+      if (lane >= off) x += y;
+    }
+    __shared__ int wsum[kThreads / 32];
+    if (lane == 31) wsum[warp] = x;
+    if (tid == 0) misc[0] = -1;
+    __syncthreads();
+    int before = x - mine;
+    for (int w = 0; w < warp; ++w) before += wsum[w];
+    const int t = blockIdx.x;
+    if (t >= before && t < before + mine) {
+      int acc = before;
+      for (int e = e0; e < e1; ++e) {
+        const int nb = (P.offsets[e + 1] - P.offsets[e] + BM - 1) / BM;
+        if (t < acc + nb) {
+          misc[0] = e;
+          misc[1] = t - acc;
+          break;
+        }
+        acc += nb;
+      }
+    }
+    __syncthreads();
+  }
+  const int e = misc[0];
+  if (e < 0) return;  // past the last block: every thread leaves together
+  const int row0 = P.offsets[e] + misc[1] * BM;
+  const int row_end = P.offsets[e + 1];
+  const int n0 = blockIdx.y * kBN;
+  const int KC = (P.d + BK - 1) / BK;
+
+  if (tid < BM) {
+    const int j = row0 + tid;
+    // rows past the segment load some valid token row; their results are dropped
+    tok_s[tid] = j < row_end ? P.perm[j] / P.k : P.perm[row0] / P.k;
+  }
+  if (tid == 0) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_x)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_w)) : "memory");
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(bar(B_FULL + s), 1);
+      mbar_init(bar(B_EMPTY + s), 1);
+    }
+    mbar_init(bar(B_ACC), 1);
+    *abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_slot)),
+                 "r"(kBN)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ---- producer: 32 gather4 copies (one per lane) + the W tile ----------
+    const int r0 = tok_s[4 * lane], r1 = tok_s[4 * lane + 1], r2 = tok_s[4 * lane + 2],
+              r3 = tok_s[4 * lane + 3];
+    int s = 0;
+    uint32_t ph = 0;
+    int issued = 0;
+    for (int kc = 0; kc < KC; ++kc, (++s == kStages ? (s = 0, ph ^= 1u) : 0u)) {
+      bool go = true;
+      if (lane == 0 && kc >= kStages) go = mbar_wait(bar(B_EMPTY + s), ph ^ 1u, abort);
+      go = __shfl_sync(0xffffffffu, go, 0);
+      if (!go) break;
+      const uint32_t base = smem0 + s * kStageBytes;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(bar(B_FULL + s), kStageBytes);
+        tma_load_2d(base + kABytes, &map_w, bar(B_FULL + s), kc * BK, e * P.n_out + n0);
+      }
+      __syncwarp();
+      tma_gather4(base + (uint32_t)lane * 4u * (BK * 2), &map_x, bar(B_FULL + s), kc * BK, r0,
+                  r1, r2, r3);
+      ++issued;
+    }
+    // every copy this CTA issued lands before the CTA may exit
+    if (lane == 0)
+      for (int kc = issued - kStages < 0 ? 0 : issued - kStages; kc < issued; ++kc)
+        mbar_wait(bar(B_FULL + kc % kStages), (kc / kStages) & 1, abort, true);
+  } else if (warp == 1) {
+    // ---- MMA issuer -------------------------------------------------------
+    if (lane == 0) {
+      const uint32_t idesc = make_idesc_bf16(kBN, BM);
+      int s = 0;
+      uint32_t ph = 0;
+      for (int kc = 0; kc < KC; ++kc, (++s == kStages ? (s = 0, ph ^= 1u) : 0u)) {
+        if (!mbar_wait(bar(B_FULL + s), ph, abort)) break;
+        tc_fence_after();
+        const uint32_t a = smem0 + s * kStageBytes, b = a + kABytes;
+#pragma unroll
+        for (int kk = 0; kk < BK / 16; ++kk)
+          mma_bf16(tmem_base, make_desc_sw64(a + kk * 32), make_desc_sw64(b + kk * 32), idesc,
+                   (kc > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(bar(B_EMPTY + s));
+      }
+      // always committed (also after an abort): drains every MMA before the
+      // epilogue reads TMEM and before TMEM is released
+      mma_commit(bar(B_ACC));
+    }
+    __syncwarp();
+  } else {
+    // ---- epilogue: warp w reads TMEM lanes 32*(w % 4).., one row per lane --
+    const int q = warp & 3;
+    const int r = q * 32 + lane;
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(bar(B_ACC), 0, abort, true)) && !*abort;
+    tc_fence_after();
+    const int j = row0 + r;
+    const bool store = ok && j < row_end;
+    const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+    __nv_bfloat16* dst = P.out + (long)j * P.n_out + n0;
+    for (int c = 0; c < kBN / 16; ++c) {
+      float v[16];
+      tmem_ld16(tmem_base + lane_off + (uint32_t)(c * 16), v);  // whole warp
+      if (store && n0 + c * 16 < P.n_out) {
+        uint4 pk[2];
+        uint32_t* w = reinterpret_cast<uint32_t*>(pk);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+          w[i] = *reinterpret_cast<const uint32_t*>(&h);
+        }
+        uint4* o = reinterpret_cast<uint4*>(dst + c * 16);
+        o[0] = pk[0];
+        o[1] = pk[1];
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                 "r"(kBN)
+                 : "memory");
+  }
+}
+
+}  // namespace eg
+}  // namespace mr

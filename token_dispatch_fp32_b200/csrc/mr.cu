@@ -12,6 +12,7 @@
 
 #include "dispatch.cuh"
 #include "ep.cuh"
+#include "expert_gemm.cuh"
 #include "mr_common.cuh"
 #include "router_ffma.cuh"
 #include "router_splitk.cuh"
@@ -448,7 +449,6 @@ int launch_tc(const void* x, const float* W, const float* bias, int T, int d, in
   P.wlo = use_wlo ? 1 : 0;
   P.bf16x3 = bf16x3 ? 1 : 0;
   P.pair = pair ? 1 : 0;
-  P.nplanes = nplanes;
   P.route_scale = route_scale;
   P.bias = bias;
   P.idx_out = idx_out;
@@ -456,10 +456,15 @@ int launch_tc(const void* x, const float* W, const float* bias, int T, int d, in
   P.logits_out = logits_out;
   const size_t smem = plan.total + 1024;
   const bool sm = (flags & MR_SCORE_SOFTMAX) != 0;
-  auto kern = pair ? (sm ? mr::tc::router_tc_kernel<true, true>
-                         : mr::tc::router_tc_kernel<true, false>)
-                   : (sm ? mr::tc::router_tc_kernel<false, true>
-                         : mr::tc::router_tc_kernel<false, false>);
+  auto kern = nplanes == 1
+                  ? (pair ? (sm ? mr::tc::router_tc_kernel<true, true, 1>
+                                : mr::tc::router_tc_kernel<true, false, 1>)
+                          : (sm ? mr::tc::router_tc_kernel<false, true, 1>
+                                : mr::tc::router_tc_kernel<false, false, 1>))
+                  : (pair ? (sm ? mr::tc::router_tc_kernel<true, true, 3>
+                                : mr::tc::router_tc_kernel<true, false, 3>)
+                          : (sm ? mr::tc::router_tc_kernel<false, true, 3>
+                                : mr::tc::router_tc_kernel<false, false, 3>));
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
       cudaSuccess)
     return MR_ERR_CUDA;
@@ -924,6 +929,58 @@ int mr_ep_recv_order(const int32_t* recv_counts, int ep, int E_loc, int R, int32
   mr::ep_recv_order_kernel<<<grid, mr::kEpThreads, 0, s>>>(recv_counts, ep, E_loc, R, order,
                                                             inv_order, local_counts,
                                                             local_offsets);
+  return launch_status();
+}
+
+// ---- expert layer with the row gather fused in -------------------------------
+
+int mr_expert_gemm_gather(const void* x, const int32_t* perm, const int32_t* offsets,
+                          const void* W_exp, int T, int d, int k, int N_r, int n_out, void* out,
+                          mr_stream_t stream) {
+  if (T < 0 || d <= 0 || k <= 0 || N_r <= 0 || n_out <= 0) return MR_ERR_INVALID_ARG;
+  if ((long long)T * k >= (1LL << 31) || (long long)N_r * n_out >= (1LL << 31))
+    return MR_ERR_INVALID_ARG;
+  if (T == 0) return MR_OK;
+  if (!x || !perm || !offsets || !W_exp || !out) return MR_ERR_INVALID_ARG;
+  int sms = 0, cc = 0;
+  if (!device_info(&sms, &cc)) return MR_ERR_CUDA;
+  if (cc != 10 || d % 8 != 0 || n_out % 16 != 0 || N_r > mr::kDispMaxExperts ||
+      !aligned16(x) || !aligned16(W_exp) || !aligned16(out))
+    return MR_ERR_UNSUPPORTED;
+  auto enc = tensor_map_encoder();
+  if (!enc) return MR_ERR_CUDA;
+  CUtensorMap mx, mw;
+  {
+    // token rows, one-row boxes: each tile::gather4 copy fetches four of them
+    const cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)T};
+    const cuuint64_t strides[1] = {(cuuint64_t)d * 2};
+    const cuuint32_t box[2] = {32, 1};
+    const cuuint32_t estr[2] = {1, 1};
+    if (enc(&mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return MR_ERR_CUDA;
+  }
+  if (!make_map_bf16(&mw, W_exp, (uint64_t)N_r * n_out, (uint64_t)d, mr::eg::kBN))
+    return MR_ERR_CUDA;
+  mr::eg::Params P;
+  P.T = T;
+  P.d = d;
+  P.k = k;
+  P.N_r = N_r;
+  P.n_out = n_out;
+  P.perm = perm;
+  P.offsets = offsets;
+  P.out = static_cast<__nv_bfloat16*>(out);
+  const size_t smem = mr::eg::kSmemBytes;
+  if (cudaFuncSetAttribute(mr::eg::expert_gemm_gather_kernel,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return MR_ERR_CUDA;
+  // at most ceil(T*k / 128) + N_r blocks of 128 sorted rows; surplus CTAs exit
+  const unsigned gx = (unsigned)(((long)T * k + mr::tc::BM - 1) / mr::tc::BM + N_r);
+  const unsigned gy = (unsigned)((n_out + mr::eg::kBN - 1) / mr::eg::kBN);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  mr::eg::expert_gemm_gather_kernel<<<dim3(gx, gy), mr::eg::kThreads, smem, s>>>(mx, mw, P);
   return launch_status();
 }
 

@@ -78,9 +78,6 @@ struct Params {
   // stages its own x tile and half of W's rows, and keeps its own 128 tokens
   // x all N experts in its TMEM.
   int pair;
-  // bf16 path: the number of bf16 planes of W (3: W split into W1 + W2 + W3;
-  // 1: W itself stored in bf16, one exact product per multiply-add).
-  int nplanes;
   int flags;  // MR_SCORE_SOFTMAX | MR_GROUP_MAX | MR_NORM_NO_EPS
   float route_scale;
   const float* bias;
@@ -518,7 +515,9 @@ __device__ __forceinline__ void select_groups(int G, int topk_group, int k, int 
 
 // SOFTMAX: the MR_SCORE_SOFTMAX instantiation (its two statistics passes and
 // cluster barriers are compiled out of the sigmoid kernel).
-template <bool PAIR, bool SOFTMAX>
+// NPL: bf16 planes of W (3: bf16x3; 1: W stored in bf16; the tf32 paths
+// ignore it).  A compile-time count keeps the MMA issue loop fully unrolled.
+template <bool PAIR, bool SOFTMAX, int NPL = 3>
 __global__ void __launch_bounds__(kThreads, 1)
     router_tc_kernel(const __grid_constant__ CUtensorMap map_x,
                      const __grid_constant__ CUtensorMap map_w,
@@ -531,7 +530,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // The 2-SM instructions exist only in the PAIR instantiation: a kernel that
   // contains them must be launched in clusters of two.
   constexpr bool pair = PAIR;
-  const int NP = P.nplanes;
+  constexpr int NP = NPL;
   const Plan plan = make_plan(NL, bf16x3, pair, NP);
   const int STAGES = plan.stages;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -629,7 +628,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t fb = cluster_addr(bar(B_FULL + s), 0);
           if (leader) mbar_arrive_expect_tx(bar(B_FULL + s), 2 * tx);
           tma_load_2d_pair(base, &map_x, fb, kc * BK, m0);
-#pragma unroll 3
+#pragma unroll
           for (int pl = 0; pl < NP; ++pl)
             tma_load_2d_pair(base + plan.a_bytes + pl * plan.b_bytes, &map_w, fb, kc * BK,
                              pl * P.N + wrow0);
@@ -638,7 +637,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive_expect_tx(bar(B_FULL + s), tx);
         tma_load_2d(base, &map_x, bar(B_FULL + s), kc * BK, m0);
         if (bf16x3) {
-#pragma unroll 3
+#pragma unroll
           for (int pl = 0; pl < NP; ++pl)
             tma_load_2d(base + plan.a_bytes + pl * plan.b_bytes, &map_w, bar(B_FULL + s),
                         kc * BK, pl * P.N + col0);
@@ -680,7 +679,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int kk = 0; kk < BK / 16; ++kk) {
             const uint32_t ko = kk * 32;  // 16 bf16 = 32 bytes along K
             const uint64_t da = make_desc_sw64(a + ko);
-#pragma unroll 3
+#pragma unroll
             for (int pl = 0; pl < NP; ++pl) {
               const uint64_t db = make_desc_sw64(a + plan.a_bytes + pl * plan.b_bytes + ko);
               const uint32_t acc = (!first || kk > 0 || pl > 0) ? 1u : 0u;

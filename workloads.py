@@ -97,7 +97,7 @@ V3_FULL = Workload("deepseek_v3_full_route_dispatch_combine_T16384", T=16384,
 ALL = [TINY, V3_PREFILL, K2_PREFILL, V3_DECODE, V3_FULL]
 BY_NAME = {w.name: w for w in ALL}
 
-_TENSORS = ("x", "W", "b", "E", "shared")
+_TENSORS = ("x", "W", "b", "E", "shared", "expert_W")
 
 
 def to_bf16_bits(a: np.ndarray) -> np.ndarray:
@@ -164,6 +164,14 @@ def gen_W_bf16(w: Workload) -> dict:
     values."""
     bits = to_bf16_bits(gen_W(w))
     return {"W_bf16": bits, "W_f32": bf16_bits_to_f32(bits)}
+
+
+def gen_expert_W(w: Workload, n_out: int) -> np.ndarray:
+    """Synthetic expert weights [N_r, n_out, d] as bf16 bit patterns:
+    N(0, 1/d) rounded to bf16 (a linear expert layer; no trained weights)."""
+    z = _normal_blocks(_child(w.seed, "expert_W"), w.N_r * n_out * w.d, F32)
+    return to_bf16_bits((z / np.float32(math.sqrt(w.d))).astype(np.float32)).reshape(
+        w.N_r, n_out, w.d)
 
 
 def gen_b(w: Workload) -> np.ndarray | None:
