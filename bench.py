@@ -351,6 +351,54 @@ def run_router_only(args, w: wl.Workload):
           flush=True)
 
 
+def run_expert_only(args, w: wl.Workload):
+    """The gather-fused expert layer alone (a profiling aid): route and
+    dispatch the workload, then time mr_expert_gemm_gather with --n-out
+    output columns per expert.  Prints one JSON line."""
+    import torch
+
+    import token_dispatch_fp32_b200 as mr
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.Stream(dev)
+    d = wl.gen_router_inputs(w)
+    xb = torch.from_numpy(d["x_bf16"]).view(torch.bfloat16).to(dev)
+    ws = torch.empty(max(4, mr.mr_router_workspace_size(w.T, w.d, w.N_r)), dtype=torch.uint8,
+                     device=dev)
+    idx, _ = mr.mr_router_forward_ex(xb, torch.from_numpy(d["W"]).to(dev),
+                                     torch.from_numpy(d["b"]).to(dev), w.n_group, w.topk_group,
+                                     w.k, w.route_scale, w.mask_mode,
+                                     precision=mr.MR_PREC_BF16X3, workspace=ws, stream=stream)
+    _, offsets, perm, _ = mr.mr_dispatch(idx, w.N_r, stream=stream)
+    eW = torch.from_numpy(wl.gen_expert_W(w, args.n_out)).view(torch.bfloat16).to(dev)
+    out = torch.empty((w.T * w.k, args.n_out), dtype=torch.bfloat16, device=dev)
+    eWp = mr.mr_expert_pack_weights(eW, stream=stream) if args.expert_weights == "packed" \
+        else None
+
+    def call():
+        if eWp is not None:
+            mr.mr_expert_gemm_gather_packed(xb, w.k, perm, offsets, eWp, w.N_r, args.n_out,
+                                            out=out, stream=stream)
+        else:
+            mr.mr_expert_gemm_gather(xb, w.k, perm, offsets, eW, out=out, stream=stream)
+
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        call()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    assert mr.mr_get_error(stream) == mr.MR_OK
+    ms = e0.elapsed_time(e1) / args.steps
+    fl = 2.0 * w.T * w.k * w.d * args.n_out
+    print(json.dumps({"only": "expert", "workload": w.name, "n_out": args.n_out, "ms": ms,
+                      "weights": args.expert_weights,
+                      "tflops": fl / (ms / 1e3) / 1e12, "steps": args.steps}), flush=True)
+
+
 def run_ours(args, w: wl.Workload, rank: int, world: int):
     import torch
     import torch.distributed as dist
@@ -544,22 +592,36 @@ def run_ours(args, w: wl.Workload, rank: int, world: int):
         exs = torch.empty((we.T * we.k, we.d), dtype=torch.bfloat16, device=dev)
         ident = torch.arange(we.T * we.k, dtype=torch.int32, device=dev)
 
+        # the expert weights are packed once, as at weight-load time
+        eWp = mr.mr_expert_pack_weights(eW, stream=stream)
+
         def fused():
+            mr.mr_expert_gemm_gather_packed(ex, we.k, eperm, eoff, eWp, we.N_r, n_out, out=eout,
+                                            stream=stream)
+
+        def fused_plain_layout():
             mr.mr_expert_gemm_gather(ex, we.k, eperm, eoff, eW, out=eout, stream=stream)
 
         def unfused():
             mr.mr_gather_rows(ex, we.k, perm=eperm, inv_perm=einv, xs=exs, stream=stream)
-            mr.mr_expert_gemm_gather(exs, 1, ident, eoff, eW, out=eout, stream=stream)
+            mr.mr_expert_gemm_gather_packed(exs, 1, ident, eoff, eWp, we.N_r, n_out, out=eout,
+                                            stream=stream)
 
         fms = time_alone(fused, n_alone)
+        pms = time_alone(fused_plain_layout, max(3, n_alone // 4))
         ums = time_alone(unfused, n_alone)
         ef = 2.0 * we.T * we.k * we.d * n_out
+        wbytes = 2 * we.N_r * n_out * we.d
         expert = {"workload": we.name, "n_out": n_out, "ms": fms,
-                  "tflops": ef / (fms / 1e3) / 1e12, "ms_unfused_gather_then_gemm": ums,
-                  "rows": we.T * we.k,
+                  "tflops": ef / (fms / 1e3) / 1e12,
+                  "weights": "packed tiles (mr_expert_pack_weights, once, outside the timing)",
+                  "ms_plain_weight_layout": pms,
+                  "ms_unfused_gather_then_gemm": ums, "rows": we.T * we.k,
+                  "expert_weight_bytes": wbytes,
+                  "hbm_bound_ms": None,
                   "saved_bytes": 2 * 2 * we.T * we.k * we.d,
                   "l2": "read pass over 512 MB before each call"}
-        del ex, ews, eW, eout, exs
+        del ex, ews, eW, eWp, eout, exs
         assert mr.mr_get_error(stream) == mr.MR_OK
 
     # The decode-size router (one position x batch 64): W read once per call.
@@ -738,6 +800,11 @@ def run_ours(args, w: wl.Workload, rank: int, world: int):
         stages[key] = st
     if expert is not None:
         expert["frac_of_bf16_peak"] = expert["tflops"] / peaks["bf16_tflops"]
+        # every expert's weights read once from HBM, against the tensor time
+        expert["hbm_bound_ms"] = expert["expert_weight_bytes"] / (peaks["hbm_gbs"] * 1e9) * 1e3
+        expert["roofline_ms"] = max(expert["hbm_bound_ms"], 2.0 * expert["rows"] * 7168 *
+                                    expert["n_out"] / (peaks["bf16_tflops"] * 1e12) * 1e3)
+        expert["frac_of_roofline"] = expert["roofline_ms"] / expert["ms"]
         stages["expert_gemm_gather_deepseek_v3_prefill_T4096"] = expert
     if decode is not None:
         decode["frac_hbm"] = decode["gbs"] / peaks["hbm_gbs"]
@@ -808,7 +875,11 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra-stages", action="store_true",
                     help="skip the prefill-router stages timed beside the step")
-    ap.add_argument("--only", choices=("router",), default=None,
+    ap.add_argument("--expert-weights", choices=("packed", "plain"), default="packed",
+                    help="with --only expert: the expert weights' layout")
+    ap.add_argument("--n-out", type=int, default=2048,
+                    help="with --only expert: output columns of the expert layer")
+    ap.add_argument("--only", choices=("router", "expert"), default=None,
                     help="time one stage alone (a profiling aid; no bench line)")
     ap.add_argument("--router-weights", choices=("f32", "bf16"), default="f32",
                     help="with --only router: the gate weight's stored type")
@@ -832,6 +903,9 @@ def main(argv=None):
         return
     if args.only == "router":
         run_router_only(args, w)
+        return
+    if args.only == "expert":
+        run_expert_only(args, w)
         return
     if world > 1:
         import datetime

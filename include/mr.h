@@ -399,6 +399,30 @@ int mr_expert_gemm_gather(const void *x, const int32_t *perm,
                           mr_stream_t stream);
 
 /*
+ * mr_expert_packed_bytes / mr_expert_pack_weights /
+ * mr_expert_gemm_gather_packed -- the same expert layer with its weights
+ * re-laid once (at weight-load time) so each tile the GEMM stages is one
+ * contiguous block: W_exp [N_r, n_out, d] is cut into tiles of 256 output
+ * rows x 64 K columns, tile (e, nt, kc) stored as a [256][64] bf16 block at
+ * block index (e * ceil(n_out/256) + nt) * ceil(d/64) + kc, zero-padded past
+ * n_out and d, each 128-byte row's 16-byte chunks permuted into the
+ * 128-byte-swizzled order the tensor core reads (chunk c of row r at
+ * position c ^ (r % 8)), so one bulk copy stages a tile.  The pages have no
+ * counterpart (a storage layout, not a step of the method); results are
+ * bit-identical to mr_expert_gemm_gather.
+ * mr_expert_pack_weights writes mr_expert_packed_bytes(N_r, n_out, d) bytes
+ * (caller-owned, 16-byte aligned; d % 8 == 0).
+ */
+size_t mr_expert_packed_bytes(int N_r, int n_out, int d);
+int mr_expert_pack_weights(const void *W_exp, int N_r, int n_out, int d,
+                           void *W_packed, size_t packed_bytes,
+                           mr_stream_t stream);
+int mr_expert_gemm_gather_packed(const void *x, const int32_t *perm,
+                                 const int32_t *offsets, const void *W_packed,
+                                 int T, int d, int k, int N_r, int n_out,
+                                 void *out, mr_stream_t stream);
+
+/*
  * mr_gather_rows -- sorted_tokens = x[idxs // k] (Kimi K2 "Add shared output"
  * page, moe_infer).  Copies rows bit for bit.
  *

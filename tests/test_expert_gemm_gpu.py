@@ -44,9 +44,15 @@ CASES = [
 ]
 
 
+@pytest.mark.parametrize("bk", ["64", "32"])
 @pytest.mark.parametrize("T,d,N_r,k,n_out,skew,n_check", CASES,
                          ids=[f"T{c[0]}_d{c[1]}_E{c[2]}_n{c[4]}" for c in CASES])
-def test_expert_gemm_gather_matches_oracle(T, d, N_r, k, n_out, skew, n_check):
+def test_expert_gemm_gather_matches_oracle(T, d, N_r, k, n_out, skew, n_check, bk,
+                                           monkeypatch):
+    """Both K-chunk widths: 64 bf16 (128-byte rows, the default) and 32."""
+    monkeypatch.setenv("MR_EG_BK", bk)
+    if bk == "32" and n_check is not None:
+        pytest.skip("the full-size case runs with the default width")
     w = wl.Workload(f"expert_T{T}_d{d}", T=T, d=d, N_r=N_r, n_group=1, topk_group=1, k=k,
                     route_scale=1.0, mask_mode=0, seed=T + d + N_r)
     rng = np.random.default_rng(w.seed)
@@ -80,7 +86,7 @@ def test_expert_gemm_gather_matches_oracle(T, d, N_r, k, n_out, skew, n_check):
     stats = {"rows_checked": int(len(rows)), "rows": int(T * k), "max_abs_err": float(err.max()),
              "max_err_over_tol": float((err / tol).max()),
              "differ_from_rounded_exact": int((got != oracle.round_bf16(ref)).sum())}
-    record(w.name, "expert_gemm_gather", stats)
+    record(w.name, f"expert_gemm_gather_bk{bk}", stats)
     print(w.name, stats)
 
 
@@ -105,3 +111,23 @@ def test_expert_gemm_gather_leaves_dropped_rows_alone():
     ref = oracle.expert_gemm(x, k, perm.cpu().numpy(), offsets.cpu().numpy(), W)
     got = out[:n_valid].float().cpu().numpy().astype(np.float64)
     assert (np.abs(got - ref) <= bf16_ulp(ref) + 1e-3).all()
+
+
+@pytest.mark.parametrize("T,d,N_r,k,n_out", [(257, 200, 32, 3, 144), (300, 7168, 64, 8, 512),
+                                             (100, 520, 16, 4, 256)])
+def test_expert_gemm_packed_weights_bit_identical(T, d, N_r, k, n_out):
+    """The packed weight layout changes only where the weights are read:
+    the results equal the plain layout's bit for bit (K tails and partial
+    output tiles included)."""
+    w = wl.Workload(f"expert_packed_T{T}", T=T, d=d, N_r=N_r, n_group=1, topk_group=1, k=k,
+                    route_scale=1.0, mask_mode=0, seed=3 * T + d)
+    rng = np.random.default_rng(w.seed)
+    x = _dev_bits(wl.to_bf16_bits(rng.standard_normal((T, d)).astype(np.float32)))
+    W = _dev_bits(wl.gen_expert_W(w, n_out))
+    counts, offsets, perm, inv = mr.mr_dispatch(torch.from_numpy(_ids(T, k, N_r, w.seed, True))
+                                                .cuda(), N_r)
+    plain = mr.mr_expert_gemm_gather(x, k, perm, offsets, W)
+    Wp = mr.mr_expert_pack_weights(W)
+    packed = mr.mr_expert_gemm_gather_packed(x, k, perm, offsets, Wp, N_r, n_out)
+    assert mr.mr_get_error() == mr.MR_OK
+    assert torch.equal(plain.view(torch.int16), packed.view(torch.int16))

@@ -675,3 +675,49 @@ def test_router_bf16_weights_full_size_every_token(w):
     np.testing.assert_allclose(wt.sum(1), w.route_scale, rtol=2e-6)
     record(w.name, "router_bf16_weights", stats)
     print(w.name, "bf16 W", stats)
+
+
+# --------------------------------------------------------------------------
+# K-split clusters: 2 or 4 CTAs share one 128-token tile's K loop and meet
+# through distributed shared memory (the default for batches with few tiles).
+
+@pytest.mark.parametrize("ks", ["K2", "K4"])
+@pytest.mark.parametrize("path", ["3xtf32", "tf32", "bf16x3", "bf16w", "softmax"])
+def test_router_ksplit_shapes(ks, path, monkeypatch):
+    monkeypatch.setenv("MR_TC_CLUSTER", ks)
+    if path == "3xtf32":
+        w = SMALL[1]  # T = 300: ragged last tile, d = 1000: K tail
+        idx, wt, lg = _run(w, mr.MR_PREC_3XTF32)
+        compare_router(idx, wt, oracle_router(w, np.arange(w.T)), lg)
+    elif path == "tf32":
+        w = SMALL[3]
+        idx, wt, lg = _run(w, mr.MR_PREC_TF32)
+        tf32_check(w, router_inputs(w)["x_f32"], idx, wt, lg, "router_tf32_ksplit")
+    elif path == "bf16x3":
+        w = BF16X3[5]  # zero mask, every biased score negative
+        idx, wt, lg = _run_bf16x3(w)
+        compare_router(idx, wt, oracle_router(w, np.arange(w.T)), lg)
+    elif path == "bf16w":
+        w = BF16X3[0]
+        idx, wt, lg, launches = _bf16w_run(w)
+        assert launches == 1
+        compare_router(idx, wt, _bf16w_ref(w, np.arange(w.T)), lg)
+    else:
+        w = VAR_W[0]
+        flags, okw = VARIANTS["softmax"]
+        idx, wt, lg = _variant_run(w, flags, "bf16", mr.MR_PREC_BF16X3, False)
+        compare_router(idx, wt, _variant_ref(w, np.arange(w.T), okw, False), lg,
+                       allow_tie_frac=0.05)
+
+
+def test_router_ksplit_is_deterministic_and_matches_one_cta():
+    """The K-split sums the slices in a fixed order: repeated calls agree bit
+    for bit, and the selection equals one CTA per tile's (the logits may
+    differ in the last bits: the summation order differs)."""
+    w = wl.V3_PREFILL.replace(name="v3_T1000", T=1000)
+    a = _run_bf16x3(w)
+    b = _run_bf16x3(w)
+    for u, v in zip(a, b):
+        assert np.array_equal(u, v)
+    ref = oracle_router(w, np.arange(w.T))
+    compare_router(a[0], a[1], ref, a[2])

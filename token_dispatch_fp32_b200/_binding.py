@@ -74,6 +74,10 @@ def lib():
         L.mr_gather_rows.argtypes = [p, i, i, i, i, p, p, p, p]
         L.mr_ep_recv_order.argtypes = [p, i, i, i, p, p, p, p, p]
         L.mr_expert_gemm_gather.argtypes = [p, p, p, p, i, i, i, i, i, p, p]
+        L.mr_expert_gemm_gather_packed.argtypes = [p, p, p, p, i, i, i, i, i, p, p]
+        L.mr_expert_packed_bytes.argtypes = [i, i, i]
+        L.mr_expert_packed_bytes.restype = sz
+        L.mr_expert_pack_weights.argtypes = [p, i, i, i, p, sz, p]
         L.mr_combine.argtypes = [p, i, p, p, p, p, i, i, i, p]
         L.mr_get_error.argtypes = [p]
         L.mr_selftest_bounded_wait.argtypes = [i, p]
@@ -339,6 +343,35 @@ def mr_expert_gemm_gather(x, k, perm, offsets, W_exp, out=None, stream=None):
         else _need(out, "out", torch.bfloat16, (T * k, n_out))
     _call("mr_expert_gemm_gather", _device_of(x, perm, offsets, W_exp, out), stream,
           _ptr(x), _ptr(perm), _ptr(offsets), _ptr(W_exp), T, d, k, N_r, n_out, _ptr(out))
+    return out
+
+
+def mr_expert_pack_weights(W_exp, stream=None):
+    """W_exp [N_r, n_out, d] bf16 -> the packed tile layout (a flat bf16
+    tensor) that mr_expert_gemm_gather_packed reads."""
+    _need(W_exp, "W_exp", torch.bfloat16)
+    N_r, n_out, d = W_exp.shape
+    n = int(lib().mr_expert_packed_bytes(N_r, n_out, d))
+    Wp = torch.empty(n // 2, dtype=torch.bfloat16, device=W_exp.device)
+    _call("mr_expert_pack_weights", _device_of(W_exp, Wp), stream, _ptr(W_exp), N_r, n_out, d,
+          _ptr(Wp), n)
+    return Wp
+
+
+def mr_expert_gemm_gather_packed(x, k, perm, offsets, W_packed, N_r, n_out, out=None,
+                                 stream=None):
+    """mr_expert_gemm_gather with packed weights (mr_expert_pack_weights)."""
+    _need(x, "x", torch.bfloat16)
+    T, d = x.shape
+    _need(perm, "perm", torch.int32, (T * k,))
+    _need(offsets, "offsets", torch.int32, (N_r + 1,))
+    _need(W_packed, "W_packed", torch.bfloat16)
+    if W_packed.numel() * 2 < int(lib().mr_expert_packed_bytes(N_r, n_out, d)):
+        raise ValueError("W_packed is smaller than mr_expert_packed_bytes")
+    out = torch.empty((T * k, n_out), dtype=torch.bfloat16, device=x.device) if out is None \
+        else _need(out, "out", torch.bfloat16, (T * k, n_out))
+    _call("mr_expert_gemm_gather_packed", _device_of(x, perm, offsets, W_packed, out), stream,
+          _ptr(x), _ptr(perm), _ptr(offsets), _ptr(W_packed), T, d, k, N_r, n_out, _ptr(out))
     return out
 
 

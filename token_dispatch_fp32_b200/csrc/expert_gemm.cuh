@@ -10,7 +10,8 @@
 // block of an expert's segment is loaded straight from the token rows x by
 // TMA tile::gather4 (four rows per copy, their indices taken from the
 // permutation), and the B tile from W[e].  tcgen05 kind::f16, M = 128,
-// N = 256, fp32 accumulation in TMEM, rounded to bf16 on the way out.
+// N = 256, fp32 accumulation in TMEM, rounded to bf16 on the way out.  K is
+// staged in chunks of 32 or 64 bf16 (BKE: 64- or 128-byte rows).
 //
 //   warp 0      producer: all 32 lanes issue the gather4 copies of a stage
 //               (lane l: rows 4l..4l+3), lane 0 also the W tile.
@@ -31,19 +32,37 @@ using namespace mr::tc;
 
 constexpr int kBN = 256;                    // output columns per CTA (MMA N)
 constexpr int kThreads = 192;               // producer, MMA, 4 epilogue warps
-constexpr int kStages = 8;
-constexpr uint32_t kABytes = BM * BK * 2;   // 128 rows x 32 bf16
-constexpr uint32_t kBBytes = kBN * BK * 2;  // 256 rows x 32 bf16
-constexpr uint32_t kStageBytes = kABytes + kBBytes;
-constexpr uint32_t kBarOff = kStages * kStageBytes;
-constexpr uint32_t kSmemBytes = kBarOff + 256 + 4 * BM + 64 + 1024;
+
+// Shared-memory plan for K chunks of BKE bf16 (32: 64-byte rows, 64-byte
+// swizzle; 64: 128-byte rows, 128-byte swizzle).
+template <int BKE>
+struct EgPlan {
+  static constexpr int kStages = BKE == 32 ? 8 : 4;
+  static constexpr uint32_t kABytes = BM * BKE * 2;   // 128 gathered rows
+  static constexpr uint32_t kBBytes = kBN * BKE * 2;  // 256 weight rows
+  static constexpr uint32_t kStageBytes = kABytes + kBBytes;
+  static constexpr uint32_t kBarOff = kStages * kStageBytes;
+  static constexpr uint32_t kSmemBytes = kBarOff + 256 + 4 * BM + 64 + 1024;
+};
 
 struct Params {
   int T, d, k, N_r, n_out;
   const int32_t* perm;
   const int32_t* offsets;
+  const __nv_bfloat16* w_packed;  // packed weights (PACKED only)
   __nv_bfloat16* out;  // [offsets[N_r], n_out]
 };
+
+// One contiguous global -> shared copy completing on an mbarrier (16-byte
+// aligned addresses, a multiple of 16 bytes).
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
+                                          uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(dst),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+      : "memory");
+}
 
 __device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap* map, uint32_t bar,
                                             int col, int r0, int r1, int r2, int r3) {
@@ -55,9 +74,23 @@ __device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
+// Packed weight layout (PACKED): W[e] cut into tiles of 256 output rows x 64
+// K columns, tile (e, nt, kc) stored as one contiguous 32 KB block at block
+// index (e * NT + nt) * KC + kc (NT = ceil(n_out / 256), KC = ceil(d / 64);
+// rows past n_out and columns past d are zero), its bytes already in the
+// order the tensor core reads a 128-byte-swizzled K-major tile (16-byte
+// chunk c of row r at chunk c ^ (r % 8) of that row).  A stage's weight tile
+// is then one bulk copy of 32 contiguous KB instead of 256 row requests of
+// 128 bytes.
+template <int BKE, bool PACKED = false>
 __global__ void __launch_bounds__(kThreads, 1)
     expert_gemm_gather_kernel(const __grid_constant__ CUtensorMap map_x,
                               const __grid_constant__ CUtensorMap map_w, const Params P) {
+  static_assert(!PACKED || BKE == 64, "the packed layout has 64-column tiles");
+  using PL = EgPlan<BKE>;
+  constexpr int kStages = PL::kStages;
+  constexpr uint32_t kABytes = PL::kABytes, kStageBytes = PL::kStageBytes,
+                     kBarOff = PL::kBarOff;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -111,7 +144,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int row0 = P.offsets[e] + misc[1] * BM;
   const int row_end = P.offsets[e + 1];
   const int n0 = blockIdx.y * kBN;
-  const int KC = (P.d + BK - 1) / BK;
+  const int KC = (P.d + BKE - 1) / BKE;
 
   if (tid < BM) {
     const int j = row0 + tid;
@@ -156,10 +189,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t base = smem0 + s * kStageBytes;
       if (lane == 0) {
         mbar_arrive_expect_tx(bar(B_FULL + s), kStageBytes);
-        tma_load_2d(base + kABytes, &map_w, bar(B_FULL + s), kc * BK, e * P.n_out + n0);
+        if constexpr (PACKED)
+          bulk_load(base + kABytes,
+                    P.w_packed + ((long)(e * (int)gridDim.y + (int)blockIdx.y) * KC + kc) *
+                                     (kBN * 64),
+                    PL::kBBytes, bar(B_FULL + s));
+        else
+          tma_load_2d(base + kABytes, &map_w, bar(B_FULL + s), kc * BKE, e * P.n_out + n0);
       }
       __syncwarp();
-      tma_gather4(base + (uint32_t)lane * 4u * (BK * 2), &map_x, bar(B_FULL + s), kc * BK, r0,
+      tma_gather4(base + (uint32_t)lane * 4u * (BKE * 2), &map_x, bar(B_FULL + s), kc * BKE, r0,
                   r1, r2, r3);
       ++issued;
     }
@@ -178,9 +217,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint32_t a = smem0 + s * kStageBytes, b = a + kABytes;
 #pragma unroll
-        for (int kk = 0; kk < BK / 16; ++kk)
-          mma_bf16(tmem_base, make_desc_sw64(a + kk * 32), make_desc_sw64(b + kk * 32), idesc,
-                   (kc > 0 || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < BKE / 16; ++kk) {
+          // 16 bf16 = 32 bytes along K; 64- or 128-byte swizzled rows
+          const uint64_t da = BKE == 32 ? make_desc_sw64(a + kk * 32) : make_desc(a + kk * 32);
+          const uint64_t db = BKE == 32 ? make_desc_sw64(b + kk * 32) : make_desc(b + kk * 32);
+          mma_bf16(tmem_base, da, db, idesc, (kc > 0 || kk > 0) ? 1u : 0u);
+        }
         mma_commit(bar(B_EMPTY + s));
       }
       // always committed (also after an abort): drains every MMA before the
@@ -222,6 +264,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
                  "r"(kBN)
                  : "memory");
+  }
+}
+
+// W [N_r][n_out][d] -> the packed layout above (swizzled within each row),
+// eight bf16 (16 bytes) per thread and step; d % 8 == 0.
+__global__ void __launch_bounds__(256)
+    expert_pack_kernel(const uint4* __restrict__ W, uint4* __restrict__ Wp, int n_out, int d,
+                       int NT, int KC, long n_vec) {
+  const int cv = 64 / 8;  // 16-byte vectors per packed row
+  for (long o = (long)blockIdx.x * blockDim.x + threadIdx.x; o < n_vec;
+       o += (long)gridDim.x * blockDim.x) {
+    const int c8o = (int)(o % cv);  // 16-byte chunk position in the packed row
+    const int r = (int)((o / cv) % kBN);
+    const int c8 = c8o ^ (r & 7);   // the K chunk stored there (128-byte swizzle)
+    const long blk = o / ((long)cv * kBN);
+    const int kc = (int)(blk % KC);
+    const int nt = (int)((blk / KC) % NT);
+    const long e = blk / ((long)KC * NT);
+    const int n = nt * kBN + r, col = kc * 64 + c8 * 8;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (n < n_out && col < d) v = W[((e * n_out + n) * (long)d + col) / 8];
+    Wp[o] = v;
   }
 }
 

@@ -350,31 +350,44 @@ int launch_splitk(const void* x, bool x_bf16, const float* W, const float* bias,
 }
 
 // How CTAs share a 128-token tile of the fused router:
+//  - ks = 2 or 4 (N_r <= 256): a cluster of ks CTAs splits the K loop of the
+//    tile (partial sums meet through distributed shared memory), taken while
+//    ks times the tile count still fits the SMs and every CTA keeps at least
+//    eight K chunks: the DeepSeek-V3 prefill batch (32 tiles) runs on 128
+//    CTAs instead of 32;
 //  - CS = 2 splits the experts over a 2-CTA cluster: always when N_r > 256
-//    (TMEM holds two accumulation buffers of at most 256 columns), and when
-//    it at least doubles the CTA count of a small batch;
-//  - otherwise one CTA per tile.
+//    (TMEM holds two accumulation buffers of at most 256 columns);
+//  - otherwise one CTA per tile (the full 16384-token batch: 128 tiles).
 // pair (bf16x3, N_r <= 256): two CTAs run one M = 256 MMA over consecutive
 // tiles and each stages half of W.  It is only taken when pinned: on the
 // full DeepSeek-V3 batch (T = 16384) it measured 5 us slower than one CTA
 // per tile (188 vs 182 us).
-// MR_TC_CLUSTER = 1, 2 or P pins the choice (used by the tests to cover each).
+// MR_TC_CLUSTER = 1, 2, P, K2 or K4 pins the choice (used by the tests to
+// cover each).
 struct TcShape {
   int CS;
   bool pair;
+  int ks;
 };
 
-TcShape tc_shape(int T, int N_r, int sms, bool bf16x3) {
-  if (N_r > 256) return {2, false};
+TcShape tc_shape(int T, int N_r, int sms, bool bf16x3, int num_kc) {
+  if (N_r > 256) return {2, false, 1};
   const bool pair_ok = bf16x3 && N_r % 32 == 0;
   if (const char* env = getenv("MR_TC_CLUSTER")) {
-    if (env[0] == '1') return {1, false};
-    if (env[0] == '2' && N_r % 32 == 0) return {2, false};
-    if ((env[0] == 'P' || env[0] == 'p') && pair_ok) return {1, true};
+    if (env[0] == '1') return {1, false, 1};
+    if (env[0] == '2' && N_r % 32 == 0) return {2, false, 1};
+    if ((env[0] == 'P' || env[0] == 'p') && pair_ok) return {1, true, 1};
+    if ((env[0] == 'K' || env[0] == 'k') && (env[1] == '2' || env[1] == '4')) {
+      const int ks = env[1] - '0';
+      if (num_kc >= ks) return {1, false, ks};
+    }
   }
   const int tiles = (T + mr::tc::BM - 1) / mr::tc::BM;
-  if (N_r % 32 == 0 && 2 * tiles <= sms) return {2, false};
-  return {1, false};
+  int ks = 1;
+  while (ks < 4 && 2 * ks * tiles <= sms && num_kc >= 8 * 2 * ks) ks *= 2;
+  if (ks > 1) return {1, false, ks};
+  if (N_r % 32 == 0 && 2 * tiles <= sms) return {2, false, 1};
+  return {1, false, 1};
 }
 
 // W's residuals [N_r, d] fp32, precomputed into the workspace by the fused path.
@@ -390,12 +403,15 @@ int launch_tc(const void* x, const float* W, const float* bias, int T, int d, in
               bool use3x, bool bf16x3, int32_t* idx_out, float* w_out, float* logits_out,
               float* wlo, void* ws, int sms, cudaStream_t st, const void* wbf16 = nullptr) {
   const int nplanes = wbf16 ? 1 : 3;
-  TcShape shp = tc_shape(T, N_r, sms, bf16x3);
+  const int num_kc = (d + mr::tc::BK - 1) / mr::tc::BK;
+  TcShape shp = tc_shape(T, N_r, sms, bf16x3, num_kc);
   auto fits = [&](const TcShape& t) {
     const mr::tc::Plan p = mr::tc::make_plan(N_r / t.CS, bf16x3, t.pair, nplanes);
-    return p.stages >= 2 && mr::tc::epilogue_smem_bytes(n_group) <= p.stages * p.stage_bytes;
+    const uint32_t ring = p.stages * p.stage_bytes;
+    const uint32_t xk = t.ks > 1 ? (uint32_t)mr::tc::BM * (N_r + 4) * 4 : 0;  // K-split partials
+    return p.stages >= 2 && mr::tc::epilogue_smem_bytes(n_group) <= ring && xk <= ring;
   };
-  if (!fits(shp) && shp.pair) shp = {1, false};  // a pair's ring is half the size
+  if (!fits(shp) && (shp.pair || shp.ks > 1)) shp = {1, false, 1};  // a pair's ring is half
   if (!fits(shp)) return MR_ERR_UNSUPPORTED;
   const int CS = shp.CS;
   const bool pair = shp.pair;
@@ -449,6 +465,7 @@ int launch_tc(const void* x, const float* W, const float* bias, int T, int d, in
   P.wlo = use_wlo ? 1 : 0;
   P.bf16x3 = bf16x3 ? 1 : 0;
   P.pair = pair ? 1 : 0;
+  P.ksplit = shp.ks;
   P.route_scale = route_scale;
   P.bias = bias;
   P.idx_out = idx_out;
@@ -470,9 +487,9 @@ int launch_tc(const void* x, const float* W, const float* bias, int T, int d, in
     return MR_ERR_CUDA;
   unsigned tiles = (unsigned)((T + mr::tc::BM - 1) / mr::tc::BM);
   if (pair) tiles = (tiles + 1) / 2 * 2;  // a pair's second tile may be past T
-  const unsigned cluster = (CS > 1 || pair) ? 2u : 1u;
+  const unsigned cluster = (CS > 1 || pair) ? 2u : (unsigned)shp.ks;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(tiles * CS);
+  cfg.gridDim = dim3(tiles * CS * shp.ks);
   cfg.blockDim = dim3(mr::tc::kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
@@ -934,35 +951,59 @@ int mr_ep_recv_order(const int32_t* recv_counts, int ep, int E_loc, int R, int32
 
 // ---- expert layer with the row gather fused in -------------------------------
 
-int mr_expert_gemm_gather(const void* x, const int32_t* perm, const int32_t* offsets,
-                          const void* W_exp, int T, int d, int k, int N_r, int n_out, void* out,
-                          mr_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// Shared by the plain and the packed-weight entry points.
+int launch_expert_gemm(const void* x, const int32_t* perm, const int32_t* offsets,
+                       const void* W, bool packed, int T, int d, int k, int N_r, int n_out,
+                       void* out, cudaStream_t s) {
   if (T < 0 || d <= 0 || k <= 0 || N_r <= 0 || n_out <= 0) return MR_ERR_INVALID_ARG;
   if ((long long)T * k >= (1LL << 31) || (long long)N_r * n_out >= (1LL << 31))
     return MR_ERR_INVALID_ARG;
   if (T == 0) return MR_OK;
-  if (!x || !perm || !offsets || !W_exp || !out) return MR_ERR_INVALID_ARG;
+  if (!x || !perm || !offsets || !W || !out) return MR_ERR_INVALID_ARG;
   int sms = 0, cc = 0;
   if (!device_info(&sms, &cc)) return MR_ERR_CUDA;
   if (cc != 10 || d % 8 != 0 || n_out % 16 != 0 || N_r > mr::kDispMaxExperts ||
-      !aligned16(x) || !aligned16(W_exp) || !aligned16(out))
+      !aligned16(x) || !aligned16(W) || !aligned16(out))
     return MR_ERR_UNSUPPORTED;
   auto enc = tensor_map_encoder();
   if (!enc) return MR_ERR_CUDA;
+  // K chunk: 64 bf16 (128-byte rows) unless MR_EG_BK=32 pins 32 (64-byte
+  // rows); the packed layout always has 64-column tiles
+  const char* bk_env = getenv("MR_EG_BK");
+  const int bke = (!packed && bk_env && bk_env[0] == '3') ? 32 : 64;
+  const CUtensorMapSwizzle sw = bke == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
+  const int NT = (n_out + mr::eg::kBN - 1) / mr::eg::kBN;
+  const int KC64 = (d + 63) / 64;
   CUtensorMap mx, mw;
   {
     // token rows, one-row boxes: each tile::gather4 copy fetches four of them
     const cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)T};
     const cuuint64_t strides[1] = {(cuuint64_t)d * 2};
-    const cuuint32_t box[2] = {32, 1};
+    const cuuint32_t box[2] = {(cuuint32_t)bke, 1};
     const cuuint32_t estr[2] = {1, 1};
     if (enc(&mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return MR_ERR_CUDA;
   }
-  if (!make_map_bf16(&mw, W_exp, (uint64_t)N_r * n_out, (uint64_t)d, mr::eg::kBN))
-    return MR_ERR_CUDA;
+  {
+    // nn.Linear layout [N_r * n_out, d], or the packed blocks as [rows, 64]
+    const cuuint64_t cols = packed ? 64 : (cuuint64_t)d;
+    const cuuint64_t rows =
+        packed ? (cuuint64_t)N_r * NT * KC64 * mr::eg::kBN : (cuuint64_t)N_r * n_out;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {cols * 2};
+    const cuuint32_t box[2] = {(cuuint32_t)bke, (cuuint32_t)mr::eg::kBN};
+    const cuuint32_t estr[2] = {1, 1};
+    if (enc(&mw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(W), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return MR_ERR_CUDA;
+  }
   mr::eg::Params P;
   P.T = T;
   P.d = d;
@@ -971,17 +1012,57 @@ int mr_expert_gemm_gather(const void* x, const int32_t* perm, const int32_t* off
   P.n_out = n_out;
   P.perm = perm;
   P.offsets = offsets;
+  P.w_packed = packed ? static_cast<const __nv_bfloat16*>(W) : nullptr;
   P.out = static_cast<__nv_bfloat16*>(out);
-  const size_t smem = mr::eg::kSmemBytes;
-  if (cudaFuncSetAttribute(mr::eg::expert_gemm_gather_kernel,
-                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+  auto kern = packed ? mr::eg::expert_gemm_gather_kernel<64, true>
+                     : (bke == 32 ? mr::eg::expert_gemm_gather_kernel<32, false>
+                                  : mr::eg::expert_gemm_gather_kernel<64, false>);
+  const size_t smem = bke == 32 ? mr::eg::EgPlan<32>::kSmemBytes : mr::eg::EgPlan<64>::kSmemBytes;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+      cudaSuccess)
     return MR_ERR_CUDA;
   // at most ceil(T*k / 128) + N_r blocks of 128 sorted rows; surplus CTAs exit
   const unsigned gx = (unsigned)(((long)T * k + mr::tc::BM - 1) / mr::tc::BM + N_r);
-  const unsigned gy = (unsigned)((n_out + mr::eg::kBN - 1) / mr::eg::kBN);
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  mr::eg::expert_gemm_gather_kernel<<<dim3(gx, gy), mr::eg::kThreads, smem, s>>>(mx, mw, P);
+  kern<<<dim3(gx, (unsigned)NT), mr::eg::kThreads, smem, s>>>(mx, mw, P);
   return launch_status();
+}
+
+}  // namespace
+
+extern "C" {
+
+int mr_expert_gemm_gather(const void* x, const int32_t* perm, const int32_t* offsets,
+                          const void* W_exp, int T, int d, int k, int N_r, int n_out, void* out,
+                          mr_stream_t stream) {
+  return launch_expert_gemm(x, perm, offsets, W_exp, false, T, d, k, N_r, n_out, out,
+                            reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t mr_expert_packed_bytes(int N_r, int n_out, int d) {
+  if (N_r <= 0 || n_out <= 0 || d <= 0) return 0;
+  return (size_t)N_r * ((n_out + 255) / 256) * ((d + 63) / 64) * 256 * 64 * 2;
+}
+
+int mr_expert_pack_weights(const void* W_exp, int N_r, int n_out, int d, void* W_packed,
+                           size_t packed_bytes, mr_stream_t stream) {
+  if (N_r <= 0 || n_out <= 0 || d <= 0 || !W_exp || !W_packed) return MR_ERR_INVALID_ARG;
+  if (packed_bytes < mr_expert_packed_bytes(N_r, n_out, d)) return MR_ERR_INVALID_ARG;
+  if (d % 8 != 0 || !aligned16(W_exp) || !aligned16(W_packed)) return MR_ERR_UNSUPPORTED;
+  int sms = 0, cc = 0;
+  if (!device_info(&sms, &cc)) return MR_ERR_CUDA;
+  const int NT = (n_out + 255) / 256, KC = (d + 63) / 64;
+  const long n_vec = (long)(mr_expert_packed_bytes(N_r, n_out, d) / 16);
+  const unsigned grid = (unsigned)std::min<long>((n_vec + 255) / 256, (long)sms * 16);
+  mr::eg::expert_pack_kernel<<<grid, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint4*>(W_exp), static_cast<uint4*>(W_packed), n_out, d, NT, KC, n_vec);
+  return launch_status();
+}
+
+int mr_expert_gemm_gather_packed(const void* x, const int32_t* perm, const int32_t* offsets,
+                                 const void* W_packed, int T, int d, int k, int N_r, int n_out,
+                                 void* out, mr_stream_t stream) {
+  return launch_expert_gemm(x, perm, offsets, W_packed, true, T, d, k, N_r, n_out, out,
+                            reinterpret_cast<cudaStream_t>(stream));
 }
 
 // ---- gather / combine -------------------------------------------------------

@@ -78,6 +78,12 @@ struct Params {
   // stages its own x tile and half of W's rows, and keeps its own 128 tokens
   // x all N experts in its TMEM.
   int pair;
+  // ksplit (CS = 1, not pair): a cluster of ksplit CTAs shares one 128-token
+  // tile, CTA r taking K chunks [r*num_kc/ksplit, (r+1)*num_kc/ksplit); their
+  // fp32 partial sums meet through distributed shared memory, summed in rank
+  // order by the CTA that owns each lane quarter (quarter q % ksplit == r),
+  // and only that CTA writes the quarter's tokens.
+  int ksplit;
   int flags;  // MR_SCORE_SOFTMAX | MR_GROUP_MAX | MR_NORM_NO_EPS
   float route_scale;
   const float* bias;
@@ -534,9 +540,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const Plan plan = make_plan(NL, bf16x3, pair, NP);
   const int STAGES = plan.stages;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t crank = (P.CS > 1 || pair) ? cluster_rank() : 0u;
-  const int tile = pair ? (int)blockIdx.x : (int)blockIdx.x / P.CS;
-  const int col0 = pair ? 0 : (int)crank * NL;  // first expert of this CTA's accumulator
+  const int KSP = P.ksplit;
+  const uint32_t crank = (P.CS > 1 || pair || KSP > 1) ? cluster_rank() : 0u;
+  const int tile = pair ? (int)blockIdx.x : (int)blockIdx.x / (P.CS * KSP);
+  const int col0 = (pair || KSP > 1) ? 0 : (int)crank * NL;  // first expert of the accumulator
   const bool leader = !pair || crank == 0;       // issues the MMAs
   const int wrow0 = pair ? (int)crank * (NL / 2) : col0;  // first W row this CTA stages
 
@@ -606,7 +613,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem_base = *tmem_slot;
 
   const int m0 = tile * BM;
-  const int KC = P.num_kc;
+  // this CTA's K chunks: all of them, or its share of a K-split cluster
+  const int kc0 = KSP > 1 ? (int)(((long)crank * P.num_kc) / KSP) : 0;
+  const int KC = KSP > 1 ? (int)(((long)(crank + 1) * P.num_kc) / KSP) - kc0 : P.num_kc;
   const int J = (KC + kPromote - 1) / kPromote;  // accumulation intervals
 
   if (warp == 0) {
@@ -627,24 +636,24 @@ __global__ void __launch_bounds__(kThreads, 1)
           // both CTAs' copies complete on CTA 0's full barrier
           const uint32_t fb = cluster_addr(bar(B_FULL + s), 0);
           if (leader) mbar_arrive_expect_tx(bar(B_FULL + s), 2 * tx);
-          tma_load_2d_pair(base, &map_x, fb, kc * BK, m0);
+          tma_load_2d_pair(base, &map_x, fb, (kc0 + kc) * BK, m0);
 #pragma unroll
           for (int pl = 0; pl < NP; ++pl)
-            tma_load_2d_pair(base + plan.a_bytes + pl * plan.b_bytes, &map_w, fb, kc * BK,
+            tma_load_2d_pair(base + plan.a_bytes + pl * plan.b_bytes, &map_w, fb, (kc0 + kc) * BK,
                              pl * P.N + wrow0);
           continue;
         }
         mbar_arrive_expect_tx(bar(B_FULL + s), tx);
-        tma_load_2d(base, &map_x, bar(B_FULL + s), kc * BK, m0);
+        tma_load_2d(base, &map_x, bar(B_FULL + s), (kc0 + kc) * BK, m0);
         if (bf16x3) {
 #pragma unroll
           for (int pl = 0; pl < NP; ++pl)
             tma_load_2d(base + plan.a_bytes + pl * plan.b_bytes, &map_w, bar(B_FULL + s),
-                        kc * BK, pl * P.N + col0);
+                        (kc0 + kc) * BK, pl * P.N + col0);
         } else {
-          tma_load_2d(base + plan.a_bytes, &map_w, bar(B_FULL + s), kc * BK, col0);
+          tma_load_2d(base + plan.a_bytes, &map_w, bar(B_FULL + s), (kc0 + kc) * BK, col0);
           if (P.wlo)
-            tma_load_2d(base + plan.hi_bytes + plan.a_bytes, &map_wlo, bar(B_FULL + s), kc * BK,
+            tma_load_2d(base + plan.hi_bytes + plan.a_bytes, &map_wlo, bar(B_FULL + s), (kc0 + kc) * BK,
                         col0);
         }
       }
@@ -828,6 +837,64 @@ __global__ void __launch_bounds__(kThreads, 1)
     while (ok && promoted < J) promote(promoted);
     ok = __all_sync(0xffffffffu, ok);
 
+    // K-split: the ksplit CTAs of the cluster hold partial sums over their K
+    // chunks.  Each writes its partials to its (now idle) ring, [BM][NL + 4]
+    // fp32 (the pad keeps a warp's rows on distinct banks); after a cluster
+    // barrier the owner of each lane quarter (q % ksplit == rank) sums the
+    // ksplit partials of its rows in rank order (the same order whichever CTA
+    // owns them), and a second barrier keeps every ring alive until its
+    // readers are done.  The other quarters' rows keep their partials; their
+    // routing below runs but writes nothing.
+    const bool own_q = KSP == 1 || (q % KSP) == (int)crank;
+    if (KSP > 1) {
+      const int row = q * 32 + lane;
+      const int NLp = NL + 4;
+      float* xpart = reinterpret_cast<float*>(smem);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int c = h + 2 * i;
+        if (c < n16) {
+          float4* d4 = reinterpret_cast<float4*>(&xpart[row * NLp + c * 16]);
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            d4[j] = make_float4(acc[i][4 * j], acc[i][4 * j + 1], acc[i][4 * j + 2],
+                                acc[i][4 * j + 3]);
+        }
+      }
+      if (!ok && lane == 0) *abort = 1;
+      cluster_sync_all();  // K-split #1: partials and abort flags visible
+      int bad = 0;
+      for (int r = 0; r < KSP; ++r)
+        bad |= __float_as_int(
+            ld_peer_f32(reinterpret_cast<const float*>(const_cast<const int*>(abort)), (uint32_t)r));
+      ok = ok && bad == 0;
+      if (own_q && ok) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int c = h + 2 * i;
+          if (c < n16) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const float* src = &xpart[row * NLp + c * 16 + 4 * j];
+              float4 sum = ld_peer_f32x4(src, 0u);
+              for (int r = 1; r < KSP; ++r) {
+                const float4 v = ld_peer_f32x4(src, (uint32_t)r);
+                sum.x += v.x;
+                sum.y += v.y;
+                sum.z += v.z;
+                sum.w += v.w;
+              }
+              acc[i][4 * j] = sum.x;
+              acc[i][4 * j + 1] = sum.y;
+              acc[i][4 * j + 2] = sum.z;
+              acc[i][4 * j + 3] = sum.w;
+            }
+          }
+        }
+      }
+      cluster_sync_all();  // K-split #2: every peer has read this CTA's partials
+    }
+
     // final sums back to TMEM buffer 0 for the routing epilogue
     if (ok) {
 #pragma unroll
@@ -882,7 +949,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c = c_beg; c < c_end; ++c) {
           __syncwarp();
           tmem_ld16(tmem_base + lane_off + (uint32_t)(c * 16), v);  // whole warp
-          if (tok < P.T)
+          if (tok < P.T && own_q)
 #pragma unroll
             for (int e = 0; e < 16; ++e) P.logits_out[tok * P.N + col0 + c * 16 + e] = v[e];
         }
@@ -1078,9 +1145,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       workers_sync();
       if (cs > 1) cluster_sync_all();  // #2: top-8 lists visible to the peer
-      if (h == 0 && (PAIR || crank == 0)) {
+      if (h == 0 && (PAIR || cs == 1 || crank == 0)) {
         // merge the other half's list, then (experts split over the cluster)
-        // the peer CTA's two lists; a pair's CTAs each own their tokens
+        // the peer CTA's two lists; a pair's CTAs each own their tokens, and
+        // so do a K-split cluster's (by lane quarter, own_q)
 #pragma unroll 1
         for (int src = 1; src < 4; ++src) {
           if (src >= 2 && cs == 1) break;
@@ -1102,7 +1170,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           top.merge(pv, ps, pi);
         }
-        if (ok && tok < P.T) {
+        if (ok && tok < P.T && own_q) {
           float den = 0.0f;
 #pragma unroll
           for (int j = 0; j < kTopMax; ++j)
@@ -1126,6 +1194,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (P.CS > 1 && warp < 2) {
     const int n_sync = SOFTMAX ? 5 : 3;
     for (int i = 0; i < n_sync; ++i) cluster_sync_all();
+  }
+  // ... and the two barriers of the K-split exchange
+  if (KSP > 1 && warp < 2) {
+    cluster_sync_all();
+    cluster_sync_all();
   }
   tc_fence_before();
   __syncthreads();
