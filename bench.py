@@ -374,13 +374,17 @@ def run_expert_only(args, w: wl.Workload):
     out = torch.empty((w.T * w.k, args.n_out), dtype=torch.bfloat16, device=dev)
     eWp = mr.mr_expert_pack_weights(eW, stream=stream) if args.expert_weights == "packed" \
         else None
+    rows, rperm = xb, perm
+    if args.expert_rows == "sorted":  # the rows materialised first; the GEMM alone is timed
+        rows = mr.mr_gather_rows(xb, w.k, perm=perm, stream=stream)
+        rperm = None
 
     def call():
         if eWp is not None:
-            mr.mr_expert_gemm_gather_packed(xb, w.k, perm, offsets, eWp, w.N_r, args.n_out,
+            mr.mr_expert_gemm_gather_packed(rows, w.k, rperm, offsets, eWp, w.N_r, args.n_out,
                                             out=out, stream=stream)
         else:
-            mr.mr_expert_gemm_gather(xb, w.k, perm, offsets, eW, out=out, stream=stream)
+            mr.mr_expert_gemm_gather(rows, w.k, rperm, offsets, eW, out=out, stream=stream)
 
     for _ in range(args.warmup):
         call()
@@ -395,7 +399,7 @@ def run_expert_only(args, w: wl.Workload):
     ms = e0.elapsed_time(e1) / args.steps
     fl = 2.0 * w.T * w.k * w.d * args.n_out
     print(json.dumps({"only": "expert", "workload": w.name, "n_out": args.n_out, "ms": ms,
-                      "weights": args.expert_weights,
+                      "weights": args.expert_weights, "rows": args.expert_rows,
                       "tflops": fl / (ms / 1e3) / 1e12, "steps": args.steps}), flush=True)
 
 
@@ -590,7 +594,6 @@ def run_ours(args, w: wl.Workload, rank: int, world: int):
         eW = torch.from_numpy(wl.gen_expert_W(we, n_out)).view(torch.bfloat16).to(dev)
         eout = torch.empty((we.T * we.k, n_out), dtype=torch.bfloat16, device=dev)
         exs = torch.empty((we.T * we.k, we.d), dtype=torch.bfloat16, device=dev)
-        ident = torch.arange(we.T * we.k, dtype=torch.int32, device=dev)
 
         # the expert weights are packed once, as at weight-load time
         eWp = mr.mr_expert_pack_weights(eW, stream=stream)
@@ -602,21 +605,26 @@ def run_ours(args, w: wl.Workload, rank: int, world: int):
         def fused_plain_layout():
             mr.mr_expert_gemm_gather(ex, we.k, eperm, eoff, eW, out=eout, stream=stream)
 
+        def gemm_on_sorted_rows():
+            mr.mr_expert_gemm_gather_packed(exs, we.k, None, eoff, eWp, we.N_r, n_out, out=eout,
+                                            stream=stream)
+
         def unfused():
             mr.mr_gather_rows(ex, we.k, perm=eperm, inv_perm=einv, xs=exs, stream=stream)
-            mr.mr_expert_gemm_gather_packed(exs, 1, ident, eoff, eWp, we.N_r, n_out, out=eout,
-                                            stream=stream)
+            gemm_on_sorted_rows()
 
         fms = time_alone(fused, n_alone)
         pms = time_alone(fused_plain_layout, max(3, n_alone // 4))
         ums = time_alone(unfused, n_alone)
+        gms = time_alone(gemm_on_sorted_rows, n_alone)
         ef = 2.0 * we.T * we.k * we.d * n_out
         wbytes = 2 * we.N_r * n_out * we.d
         expert = {"workload": we.name, "n_out": n_out, "ms": fms,
                   "tflops": ef / (fms / 1e3) / 1e12,
                   "weights": "packed tiles (mr_expert_pack_weights, once, outside the timing)",
                   "ms_plain_weight_layout": pms,
-                  "ms_unfused_gather_then_gemm": ums, "rows": we.T * we.k,
+                  "ms_unfused_gather_then_gemm": ums,
+                  "ms_grouped_gemm_on_sorted_rows_alone": gms, "rows": we.T * we.k,
                   "expert_weight_bytes": wbytes,
                   "hbm_bound_ms": None,
                   "saved_bytes": 2 * 2 * we.T * we.k * we.d,
@@ -877,6 +885,8 @@ def main(argv=None):
                     help="skip the prefill-router stages timed beside the step")
     ap.add_argument("--expert-weights", choices=("packed", "plain"), default="packed",
                     help="with --only expert: the expert weights' layout")
+    ap.add_argument("--expert-rows", choices=("gathered", "sorted"), default="gathered",
+                    help="with --only expert: rows gathered in the GEMM, or pre-sorted")
     ap.add_argument("--n-out", type=int, default=2048,
                     help="with --only expert: output columns of the expert layer")
     ap.add_argument("--only", choices=("router", "expert"), default=None,

@@ -386,7 +386,11 @@ int mr_ep_recv_order(const int32_t *recv_counts, int ep, int E_loc, int R,
  * accumulation in tensor memory, rounded to bf16 (nearest even) on output.
  *
  *   x        [T, d] bf16 token rows.
- *   perm     [T*k] int32, offsets [N_r + 1] int32: from mr_dispatch.
+ *   perm     [T*k] int32, offsets [N_r + 1] int32: from mr_dispatch.  perm
+ *            may be NULL: x is then [T*k, d], the rows already in
+ *            expert-sorted order (row j = sorted row j; e.g. from
+ *            mr_gather_rows), and the call is the plain grouped GEMM (one
+ *            tiled copy per 128-row block instead of the gathers).
  *   W_exp    [N_r, n_out, d] bf16 (nn.Linear layout per expert).
  *   out      [T*k, n_out] bf16 in expert-sorted order; rows from offsets[N_r]
  *            on (dropped ids) are not written.

@@ -44,14 +44,18 @@ CASES = [
 ]
 
 
-@pytest.mark.parametrize("bk", ["64", "32"])
+@pytest.mark.parametrize("bk", ["64", "64tma", "32"])
 @pytest.mark.parametrize("T,d,N_r,k,n_out,skew,n_check", CASES,
                          ids=[f"T{c[0]}_d{c[1]}_E{c[2]}_n{c[4]}" for c in CASES])
 def test_expert_gemm_gather_matches_oracle(T, d, N_r, k, n_out, skew, n_check, bk,
                                            monkeypatch):
-    """Both K-chunk widths: 64 bf16 (128-byte rows, the default) and 32."""
-    monkeypatch.setenv("MR_EG_BK", bk)
-    if bk == "32" and n_check is not None:
+    """Both K-chunk widths: 64 bf16 (128-byte rows, the default; rows copied
+    by the epilogue warps, or by TMA gathers when pinned) and 32 (TMA
+    gathers)."""
+    monkeypatch.setenv("MR_EG_BK", bk[:2])
+    if bk == "64tma":
+        monkeypatch.setenv("MR_EG_GATHER", "tma")
+    if bk != "64" and n_check is not None:
         pytest.skip("the full-size case runs with the default width")
     w = wl.Workload(f"expert_T{T}_d{d}", T=T, d=d, N_r=N_r, n_group=1, topk_group=1, k=k,
                     route_scale=1.0, mask_mode=0, seed=T + d + N_r)
@@ -131,3 +135,25 @@ def test_expert_gemm_packed_weights_bit_identical(T, d, N_r, k, n_out):
     packed = mr.mr_expert_gemm_gather_packed(x, k, perm, offsets, Wp, N_r, n_out)
     assert mr.mr_get_error() == mr.MR_OK
     assert torch.equal(plain.view(torch.int16), packed.view(torch.int16))
+
+
+def test_expert_gemm_on_sorted_rows_equals_fused_gather():
+    """Without perm the GEMM reads already-sorted rows (e.g. from
+    mr_gather_rows) with tiled copies: the same rows, the same arithmetic,
+    so the same bits as the fused gather."""
+    T, d, N_r, k, n_out = 300, 7168, 64, 8, 256
+    w = wl.Workload("expert_sorted_T300", T=T, d=d, N_r=N_r, n_group=1, topk_group=1, k=k,
+                    route_scale=1.0, mask_mode=0, seed=77)
+    rng = np.random.default_rng(w.seed)
+    x = _dev_bits(wl.to_bf16_bits(rng.standard_normal((T, d)).astype(np.float32)))
+    W = _dev_bits(wl.gen_expert_W(w, n_out))
+    counts, offsets, perm, inv = mr.mr_dispatch(torch.from_numpy(_ids(T, k, N_r, 7, True))
+                                                .cuda(), N_r)
+    fused = mr.mr_expert_gemm_gather(x, k, perm, offsets, W)
+    xs = mr.mr_gather_rows(x, k, perm=perm, inv_perm=inv)
+    plain = mr.mr_expert_gemm_gather(xs, k, None, offsets, W)
+    packed = mr.mr_expert_gemm_gather_packed(xs, k, None, offsets,
+                                             mr.mr_expert_pack_weights(W), N_r, n_out)
+    assert mr.mr_get_error() == mr.MR_OK
+    assert torch.equal(fused.view(torch.int16), plain.view(torch.int16))
+    assert torch.equal(fused.view(torch.int16), packed.view(torch.int16))

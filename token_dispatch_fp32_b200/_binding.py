@@ -333,7 +333,12 @@ def mr_expert_gemm_gather(x, k, perm, offsets, W_exp, out=None, stream=None):
     mr_dispatch), W_exp [N_r, n_out, d] bf16."""
     _need(x, "x", torch.bfloat16)
     T, d = x.shape
-    _need(perm, "perm", torch.int32, (T * k,))
+    if perm is None:  # x already holds the T*k expert-sorted rows
+        if T % k:
+            raise ValueError("without perm, x must have T*k rows")
+        T //= k
+    else:
+        _need(perm, "perm", torch.int32, (T * k,))
     _need(W_exp, "W_exp", torch.bfloat16)
     N_r, n_out, dw = W_exp.shape
     if dw != d:
@@ -363,7 +368,12 @@ def mr_expert_gemm_gather_packed(x, k, perm, offsets, W_packed, N_r, n_out, out=
     """mr_expert_gemm_gather with packed weights (mr_expert_pack_weights)."""
     _need(x, "x", torch.bfloat16)
     T, d = x.shape
-    _need(perm, "perm", torch.int32, (T * k,))
+    if perm is None:  # x already holds the T*k expert-sorted rows
+        if T % k:
+            raise ValueError("without perm, x must have T*k rows")
+        T //= k
+    else:
+        _need(perm, "perm", torch.int32, (T * k,))
     _need(offsets, "offsets", torch.int32, (N_r + 1,))
     _need(W_packed, "W_packed", torch.bfloat16)
     if W_packed.numel() * 2 < int(lib().mr_expert_packed_bytes(N_r, n_out, d)):

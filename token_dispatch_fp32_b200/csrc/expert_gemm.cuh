@@ -47,6 +47,7 @@ struct EgPlan {
 
 struct Params {
   int T, d, k, N_r, n_out;
+  const void* x;  // token rows (the copy warps read them directly)
   const int32_t* perm;
   const int32_t* offsets;
   const __nv_bfloat16* w_packed;  // packed weights (PACKED only)
@@ -82,10 +83,25 @@ __device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap* map
 // chunk c of row r at chunk c ^ (r % 8) of that row).  A stage's weight tile
 // is then one bulk copy of 32 contiguous KB instead of 256 row requests of
 // 128 bytes.
-template <int BKE, bool PACKED = false>
+// How a stage's A tile (128 sorted rows x BKE) reaches shared memory:
+//   kRowsSorted  the rows are already in expert-sorted order (x is [T*k, d],
+//                row j = sorted row j): one tiled copy of 128 consecutive
+//                rows -- the plain grouped GEMM without the fused gather;
+//   kGatherTma   TMA tile::gather4 copies, four token rows each (warp 0);
+//   kGatherLsu   the four epilogue warps, idle during the K loop, copy the
+//                token rows 16 bytes per thread (cp.async) straight into the
+//                128-byte-swizzled layout, three stages ahead; each warp
+//                waits for its copies, fences them to the async proxy and
+//                arrives on the stage's barrier (its arrival count is 5:
+//                warp 0's expect-tx arrival and the four copy warps).
+constexpr int kRowsSorted = 0, kGatherTma = 1, kGatherLsu = 2;
+
+template <int BKE, bool PACKED = false, int AMODE = kGatherTma>
 __global__ void __launch_bounds__(kThreads, 1)
     expert_gemm_gather_kernel(const __grid_constant__ CUtensorMap map_x,
                               const __grid_constant__ CUtensorMap map_w, const Params P) {
+  constexpr bool GATHER = AMODE != kRowsSorted;
+  static_assert(AMODE != kGatherLsu || BKE == 64, "the copy warps fill 128-byte rows");
   static_assert(!PACKED || BKE == 64, "the packed layout has 64-column tiles");
   using PL = EgPlan<BKE>;
   constexpr int kStages = PL::kStages;
@@ -146,7 +162,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n0 = blockIdx.y * kBN;
   const int KC = (P.d + BKE - 1) / BKE;
 
-  if (tid < BM) {
+  if (GATHER && tid < BM) {
     const int j = row0 + tid;
     // rows past the segment load some valid token row; their results are dropped
     tok_s[tid] = j < row_end ? P.perm[j] / P.k : P.perm[row0] / P.k;
@@ -155,7 +171,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_x)) : "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_w)) : "memory");
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(bar(B_FULL + s), 1);
+      mbar_init(bar(B_FULL + s), AMODE == kGatherLsu ? 5 : 1);
       mbar_init(bar(B_EMPTY + s), 1);
     }
     mbar_init(bar(B_ACC), 1);
@@ -176,8 +192,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ---- producer: 32 gather4 copies (one per lane) + the W tile ----------
-    const int r0 = tok_s[4 * lane], r1 = tok_s[4 * lane + 1], r2 = tok_s[4 * lane + 2],
-              r3 = tok_s[4 * lane + 3];
+    int r0 = 0, r1 = 0, r2 = 0, r3 = 0;
+    if (GATHER) {
+      r0 = tok_s[4 * lane];
+      r1 = tok_s[4 * lane + 1];
+      r2 = tok_s[4 * lane + 2];
+      r3 = tok_s[4 * lane + 3];
+    }
     int s = 0;
     uint32_t ph = 0;
     int issued = 0;
@@ -188,7 +209,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!go) break;
       const uint32_t base = smem0 + s * kStageBytes;
       if (lane == 0) {
-        mbar_arrive_expect_tx(bar(B_FULL + s), kStageBytes);
+        mbar_arrive_expect_tx(bar(B_FULL + s),
+                              AMODE == kGatherLsu ? PL::kBBytes : kStageBytes);
         if constexpr (PACKED)
           bulk_load(base + kABytes,
                     P.w_packed + ((long)(e * (int)gridDim.y + (int)blockIdx.y) * KC + kc) *
@@ -198,8 +220,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_2d(base + kABytes, &map_w, bar(B_FULL + s), kc * BKE, e * P.n_out + n0);
       }
       __syncwarp();
-      tma_gather4(base + (uint32_t)lane * 4u * (BKE * 2), &map_x, bar(B_FULL + s), kc * BKE, r0,
-                  r1, r2, r3);
+      if constexpr (AMODE == kGatherTma)
+        tma_gather4(base + (uint32_t)lane * 4u * (BKE * 2), &map_x, bar(B_FULL + s), kc * BKE,
+                    r0, r1, r2, r3);
+      else if (AMODE == kRowsSorted && lane == 0)  // 128 consecutive sorted rows
+        tma_load_2d(base, &map_x, bar(B_FULL + s), kc * BKE, row0);
       ++issued;
     }
     // every copy this CTA issued lands before the CTA may exit
@@ -231,6 +256,56 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   } else {
+    if constexpr (AMODE == kGatherLsu) {
+      // ---- A tiles: 128 token rows x 64 bf16 per stage, 16 bytes a copy ----
+      // copy i of a stage (i = ct + 128 * u): row i / 8, 16-byte chunk i % 8,
+      // stored at chunk (i % 8) ^ (row % 8) of the row (128-byte swizzle)
+      const int ct = tid - 64;  // 0..127
+      const __nv_bfloat16* xb = reinterpret_cast<const __nv_bfloat16*>(P.x);
+      constexpr int kLag = kStages - 1;  // stages in flight per thread
+      // hand over the stage issued kLag iterations ago: its copies have landed
+      // once at most kLag - 1 newer groups are pending
+      auto hand_over = [&](int st) {
+        asm volatile("cp.async.wait_group %0;" ::"n"(kLag - 1) : "memory");
+        fence_proxy_async();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(B_FULL + st));
+      };
+      int s = 0;
+      uint32_t ph = 0;
+      bool go = true;
+      for (int kc = 0; kc < KC; ++kc, (++s == kStages ? (s = 0, ph ^= 1u) : 0u)) {
+        // first the hand-over, so the MMA never waits on this warp's wait for
+        // a free stage below
+        if (kc >= kLag) hand_over((kc - kLag) % kStages);
+        if (kc >= kStages) {
+          bool g = true;
+          if (lane == 0) g = mbar_wait(bar(B_EMPTY + s), ph ^ 1u, abort);
+          go = __shfl_sync(0xffffffffu, g, 0);
+          if (!go) break;
+        }
+        const uint32_t base = smem0 + s * kStageBytes;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int i = ct + 128 * u, rr = i >> 3, c = i & 7;
+          const int col = kc * 64 + c * 8;
+          const uint32_t dst = base + (uint32_t)rr * 128u + ((uint32_t)(c ^ (rr & 7)) << 4);
+          const __nv_bfloat16* src = xb + (long)tok_s[rr] * P.d + (col < P.d ? col : 0);
+          const uint32_t nbytes = col < P.d ? 16u : 0u;  // K tail: zero fill
+          asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+                       "r"(nbytes)
+                       : "memory");
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+      }
+      // the last stages (and, after a give-up, every issued copy) land
+      asm volatile("cp.async.wait_group 0;" ::: "memory");
+      fence_proxy_async();
+      __syncwarp();
+      if (go && lane == 0)
+        for (int kc = KC - kLag < 0 ? 0 : KC - kLag; kc < KC; ++kc)
+          mbar_arrive(bar(B_FULL + kc % kStages));
+    }
     // ---- epilogue: warp w reads TMEM lanes 32*(w % 4).., one row per lane --
     const int q = warp & 3;
     const int r = q * 32 + lane;

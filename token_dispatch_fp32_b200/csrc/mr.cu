@@ -963,7 +963,8 @@ int launch_expert_gemm(const void* x, const int32_t* perm, const int32_t* offset
   if ((long long)T * k >= (1LL << 31) || (long long)N_r * n_out >= (1LL << 31))
     return MR_ERR_INVALID_ARG;
   if (T == 0) return MR_OK;
-  if (!x || !perm || !offsets || !W || !out) return MR_ERR_INVALID_ARG;
+  if (!x || !offsets || !W || !out) return MR_ERR_INVALID_ARG;
+  const bool gather = perm != nullptr;  // NULL: x already holds the sorted rows
   int sms = 0, cc = 0;
   if (!device_info(&sms, &cc)) return MR_ERR_CUDA;
   if (cc != 10 || d % 8 != 0 || n_out % 16 != 0 || N_r > mr::kDispMaxExperts ||
@@ -980,10 +981,11 @@ int launch_expert_gemm(const void* x, const int32_t* perm, const int32_t* offset
   const int KC64 = (d + 63) / 64;
   CUtensorMap mx, mw;
   {
-    // token rows, one-row boxes: each tile::gather4 copy fetches four of them
-    const cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)T};
+    // token rows, one-row boxes: each tile::gather4 copy fetches four of them;
+    // without perm, the [T*k, d] sorted rows in 128-row boxes
+    const cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)(gather ? T : (long)T * k)};
     const cuuint64_t strides[1] = {(cuuint64_t)d * 2};
-    const cuuint32_t box[2] = {(cuuint32_t)bke, 1};
+    const cuuint32_t box[2] = {(cuuint32_t)bke, gather ? 1u : (cuuint32_t)mr::tc::BM};
     const cuuint32_t estr[2] = {1, 1};
     if (enc(&mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -1012,11 +1014,23 @@ int launch_expert_gemm(const void* x, const int32_t* perm, const int32_t* offset
   P.n_out = n_out;
   P.perm = perm;
   P.offsets = offsets;
+  P.x = x;
   P.w_packed = packed ? static_cast<const __nv_bfloat16*>(W) : nullptr;
   P.out = static_cast<__nv_bfloat16*>(out);
-  auto kern = packed ? mr::eg::expert_gemm_gather_kernel<64, true>
-                     : (bke == 32 ? mr::eg::expert_gemm_gather_kernel<32, false>
-                                  : mr::eg::expert_gemm_gather_kernel<64, false>);
+  // gathered rows: copied by the four epilogue warps (cp.async, 64-wide K
+  // chunks) unless MR_EG_GATHER=tma pins the TMA tile::gather4 copies
+  const char* g_env = getenv("MR_EG_GATHER");
+  const bool tma_gather = bke == 32 || (g_env && g_env[0] == 't');
+  using namespace mr::eg;
+  auto kern = !gather ? (packed ? expert_gemm_gather_kernel<64, true, kRowsSorted>
+                                : (bke == 32 ? expert_gemm_gather_kernel<32, false, kRowsSorted>
+                                             : expert_gemm_gather_kernel<64, false, kRowsSorted>))
+            : tma_gather
+                ? (packed ? expert_gemm_gather_kernel<64, true, kGatherTma>
+                          : (bke == 32 ? expert_gemm_gather_kernel<32, false, kGatherTma>
+                                       : expert_gemm_gather_kernel<64, false, kGatherTma>))
+                : (packed ? expert_gemm_gather_kernel<64, true, kGatherLsu>
+                          : expert_gemm_gather_kernel<64, false, kGatherLsu>);
   const size_t smem = bke == 32 ? mr::eg::EgPlan<32>::kSmemBytes : mr::eg::EgPlan<64>::kSmemBytes;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
       cudaSuccess)
