@@ -473,15 +473,18 @@ int launch_tc(const void* x, const float* W, const float* bias, int T, int d, in
   P.logits_out = logits_out;
   const size_t smem = plan.total + 1024;
   const bool sm = (flags & MR_SCORE_SOFTMAX) != 0;
-  auto kern = nplanes == 1
-                  ? (pair ? (sm ? mr::tc::router_tc_kernel<true, true, 1>
-                                : mr::tc::router_tc_kernel<true, false, 1>)
-                          : (sm ? mr::tc::router_tc_kernel<false, true, 1>
-                                : mr::tc::router_tc_kernel<false, false, 1>))
-                  : (pair ? (sm ? mr::tc::router_tc_kernel<true, true, 3>
-                                : mr::tc::router_tc_kernel<true, false, 3>)
-                          : (sm ? mr::tc::router_tc_kernel<false, true, 3>
-                                : mr::tc::router_tc_kernel<false, false, 3>));
+  using mr::tc::router_tc_kernel;
+  const bool ksk = shp.ks > 1;  // the K-split instantiation (never with a pair)
+  auto kern =
+      nplanes == 1
+          ? (pair ? (sm ? router_tc_kernel<true, true, 1> : router_tc_kernel<true, false, 1>)
+                  : ksk ? (sm ? router_tc_kernel<false, true, 1, true>
+                              : router_tc_kernel<false, false, 1, true>)
+                        : (sm ? router_tc_kernel<false, true, 1> : router_tc_kernel<false, false, 1>))
+          : (pair ? (sm ? router_tc_kernel<true, true, 3> : router_tc_kernel<true, false, 3>)
+                  : ksk ? (sm ? router_tc_kernel<false, true, 3, true>
+                              : router_tc_kernel<false, false, 3, true>)
+                        : (sm ? router_tc_kernel<false, true, 3> : router_tc_kernel<false, false, 3>));
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
       cudaSuccess)
     return MR_ERR_CUDA;

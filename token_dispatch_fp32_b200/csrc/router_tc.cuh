@@ -523,7 +523,9 @@ __device__ __forceinline__ void select_groups(int G, int topk_group, int k, int 
 // cluster barriers are compiled out of the sigmoid kernel).
 // NPL: bf16 planes of W (3: bf16x3; 1: W stored in bf16; the tf32 paths
 // ignore it).  A compile-time count keeps the MMA issue loop fully unrolled.
-template <bool PAIR, bool SOFTMAX, int NPL = 3>
+// KS: the K-split instantiation (P.ksplit > 1); without it the K-split code
+// is compiled out of the one-CTA-per-tile kernel.
+template <bool PAIR, bool SOFTMAX, int NPL = 3, bool KS = false>
 __global__ void __launch_bounds__(kThreads, 1)
     router_tc_kernel(const __grid_constant__ CUtensorMap map_x,
                      const __grid_constant__ CUtensorMap map_w,
@@ -540,7 +542,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const Plan plan = make_plan(NL, bf16x3, pair, NP);
   const int STAGES = plan.stages;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int KSP = P.ksplit;
+  const int KSP = KS ? P.ksplit : 1;
   const uint32_t crank = (P.CS > 1 || pair || KSP > 1) ? cluster_rank() : 0u;
   const int tile = pair ? (int)blockIdx.x : (int)blockIdx.x / (P.CS * KSP);
   const int col0 = (pair || KSP > 1) ? 0 : (int)crank * NL;  // first expert of the accumulator
@@ -869,25 +871,39 @@ __global__ void __launch_bounds__(kThreads, 1)
             ld_peer_f32(reinterpret_cast<const float*>(const_cast<const int*>(abort)), (uint32_t)r));
       ok = ok && bad == 0;
       if (own_q && ok) {
+        // per 8 columns, every peer's two float4 loads are issued before the
+        // first add (one remote round trip per 8 columns, not one per load),
+        // then summed in rank order
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           const int c = h + 2 * i;
           if (c < n16) {
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const float* src = &xpart[row * NLp + c * 16 + 4 * j];
-              float4 sum = ld_peer_f32x4(src, 0u);
-              for (int r = 1; r < KSP; ++r) {
-                const float4 v = ld_peer_f32x4(src, (uint32_t)r);
-                sum.x += v.x;
-                sum.y += v.y;
-                sum.z += v.z;
-                sum.w += v.w;
+            for (int jj = 0; jj < 4; jj += 2) {
+              float4 v[4][2];  // [peer][float4]
+#pragma unroll
+              for (int r = 0; r < 4; ++r)
+                if (r < KSP)
+#pragma unroll
+                  for (int j = 0; j < 2; ++j)
+                    v[r][j] = ld_peer_f32x4(&xpart[row * NLp + c * 16 + 4 * (jj + j)],
+                                            (uint32_t)r);
+#pragma unroll
+              for (int j = 0; j < 2; ++j) {
+                float4 sum = v[0][j];
+#pragma unroll
+                for (int r = 1; r < 4; ++r)
+                  if (r < KSP) {
+                    sum.x += v[r][j].x;
+                    sum.y += v[r][j].y;
+                    sum.z += v[r][j].z;
+                    sum.w += v[r][j].w;
+                  }
+                acc[i][4 * (jj + j)] = sum.x;
+                acc[i][4 * (jj + j) + 1] = sum.y;
+                acc[i][4 * (jj + j) + 2] = sum.z;
+                acc[i][4 * (jj + j) + 3] = sum.w;
               }
-              acc[i][4 * j] = sum.x;
-              acc[i][4 * j + 1] = sum.y;
-              acc[i][4 * j + 2] = sum.z;
-              acc[i][4 * j + 3] = sum.w;
             }
           }
         }
