@@ -24,7 +24,8 @@
  *  - All tensor pointers are caller-owned DEVICE pointers on the current
  *    device, row-major and densely packed.  The library never allocates
  *    device memory, frees or synchronises (except mr_get_error, which must
- *    read the device); its only device memory is a few fixed arrays in its
+ *    read the device, and the mr_ipc_* calls, which map and unmap buffers of
+ *    other processes); its only device memory is a few fixed arrays in its
  *    own image, named below where they are used.
  *  - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy stream) and
  *    runs asynchronously.  Arguments are validated on the host before any
@@ -60,6 +61,7 @@ typedef struct CUstream_st *mr_stream_t;
 #define MR_ERR_CUDA (-3)        /* a CUDA launch or query failed              */
 #define MR_ERR_DEVICE (-4)      /* device flag: bad expert id seen            */
 #define MR_ERR_TIMEOUT (-5)     /* device flag: a bounded wait gave up        */
+#define MR_ERR_OVERFLOW (-6)    /* device flag: rows past a buffer's capacity */
 
 /* ---- element types of row tensors --------------------------------------- */
 #define MR_F32 0
@@ -371,6 +373,108 @@ int mr_ep_recv_order(const int32_t *recv_counts, int ep, int E_loc, int R,
                      int32_t *local_offsets, mr_stream_t stream);
 
 /*
+ * Expert parallelism over peer memory (Kimi K2 "Add shared output" page,
+ * moe_infer, ep_size > 1), without the two row all-to-alls and the
+ * receive-side sort: every source writes each of its rows straight into the
+ * owner's receive buffer at the row's final place, and the combine reads the
+ * expert outputs straight out of the owners' output buffers.  Rank r owns
+ * experts [r*E_loc, (r+1)*E_loc), E_loc = N_r / ep.  Owner o's receive
+ * buffer holds, in order: its local experts; within an expert, the sources in
+ * rank order; within a source, that source's rows in its own stable expert
+ * order (token order) -- exactly the rows and the order the page's
+ * all-to-all followed by the stable argsort of the received expert labels
+ * produces.  The place of every row follows from all ranks' counts alone.
+ *
+ * The buffers are device pointers of this process: this GPU's own memory,
+ * another GPU's memory with peer access enabled, or another process's buffer
+ * opened with mr_ipc_import.  The caller orders the ranks' steps: every
+ * rank's mr_ep_dispatch_p2p finished before any owner reads its receive
+ * buffer, every owner's outputs complete before any mr_ep_combine_p2p reads
+ * them, and every combine finished before an owner overwrites its output
+ * buffer (e.g. a collective on the stream between the steps).  The kernels
+ * never wait on another rank.
+ */
+
+/*
+ * mr_ep_dispatch_p2p -- rows of this rank to their owners' receive buffers.
+ *
+ *   x             [T, d] token rows of `dtype` (MR_BF16 or MR_F32).
+ *   idx           [T, k] int32 expert ids in [0, N_r).
+ *   inv_perm, offsets   this rank's mr_dispatch of idx (inv_perm [T*k],
+ *                 offsets [N_r + 1]).
+ *   counts_all    [ep, N_r] int32 (device): every rank's counts from
+ *                 mr_dispatch, rank-major (an all-gather of them).
+ *   rank, ep      this rank and the number of ranks (N_r % ep == 0).
+ *   recv_bufs     HOST array of ep device pointers: rank o's receive buffer,
+ *                 [capacity, d] of `dtype`, 16-byte aligned for the vector
+ *                 path.
+ *   dest          [T*k] int32 out: the row of slot t*k+j in its owner's
+ *                 buffer, -1 for a slot without one.
+ *   local_counts  [E_loc] int32 out: rows this rank receives per local
+ *                 expert; local_offsets [E_loc + 1] their exclusive prefix
+ *                 (the segments of its own receive buffer, for its experts).
+ * Two kernels: the destinations (every CTA rebuilds the per-expert bases
+ * from counts_all in shared memory), then one CTA per token reads its row
+ * once and stores it to its k destinations.
+ * Limits: 1 <= k <= 32, ep <= 64, N_r <= 1024.  Data faults do not trap: ids
+ * out of range and slots dropped by mr_dispatch get dest -1; counts below
+ * zero, or a row of counts_all for `rank` that disagrees with offsets, set
+ * every dest to -1 and the local counts to 0 (MR_ERR_DEVICE from
+ * mr_get_error); rows past an owner's capacity are not written, get dest -1
+ * and are not counted in local_counts (MR_ERR_OVERFLOW).  A capacity of
+ * ep * T_max * min(k, E_loc) rows never overflows.
+ */
+int mr_ep_dispatch_p2p(const void *x, int dtype, int T, int d, int k,
+                       const int32_t *idx, const int32_t *inv_perm,
+                       const int32_t *offsets, const int32_t *counts_all,
+                       int ep, int rank, int N_r, void *const *recv_bufs,
+                       int capacity, int32_t *dest, int32_t *local_counts,
+                       int32_t *local_offsets, mr_stream_t stream);
+
+/*
+ * mr_ep_combine_p2p -- the weighted combine and shared add of mr_combine,
+ * reading slot (t, j)'s expert output from row dest[t*k+j] of the output
+ * buffer of idx[t, j]'s owner.
+ *
+ *   out_bufs  HOST array of ep device pointers: rank o's expert outputs,
+ *             [capacity, d] of `dtype`, row i the output of its receive row i.
+ *   idx, dest [T*k] from this rank's mr_ep_dispatch_p2p.
+ *   w, shared, y, and the arithmetic: as mr_combine (slots without a row
+ *             contribute nothing).
+ * One kernel; the peers' rows are loaded through L2, not the read-only path.
+ * Limits: 1 <= k <= 32, ep <= 64.
+ */
+int mr_ep_combine_p2p(const void *const *out_bufs, int dtype, int d,
+                      const float *w, const int32_t *idx, const int32_t *dest,
+                      int ep, int N_r, int capacity, const void *shared,
+                      void *y, int T, int k, mr_stream_t stream);
+
+/*
+ * Buffers shared between processes (one process per GPU): an owner exports
+ * its receive and output buffers, every rank imports the others'.
+ *   mr_ipc_export  fills *out for `bytes` of device memory at dev_ptr, which
+ *                  must lie inside one allocation of the runtime allocator
+ *                  (cudaMalloc, as under PyTorch's caching allocator):
+ *                  MR_ERR_INVALID_ARG otherwise, MR_ERR_UNSUPPORTED for memory
+ *                  the IPC handles cannot name (the virtual memory API).
+ *   mr_ipc_import  opens a handle exported by ANOTHER process, on the current
+ *                  device, with peer access enabled on demand; *ptr is the
+ *                  buffer, *base the mapping to pass to mr_ipc_close.
+ *   mr_ipc_close   unmaps *base.
+ * The handle is plain bytes: send it through any channel (e.g. an
+ * all-gather of the processes' handles).
+ */
+typedef struct mr_ipc_handle {
+  unsigned char handle[64]; /* CUDA IPC handle of the allocation */
+  uint64_t offset;          /* buffer start within the allocation */
+  uint64_t bytes;           /* buffer size */
+} mr_ipc_handle_t;
+
+int mr_ipc_export(const void *dev_ptr, size_t bytes, mr_ipc_handle_t *out);
+int mr_ipc_import(const mr_ipc_handle_t *h, void **base, void **ptr);
+int mr_ipc_close(void *base);
+
+/*
  * mr_expert_gemm_gather -- one expert layer over the expert-sorted rows, with
  * the row gather fused into the GEMM (Kimi K2 "Add shared output" page,
  * moe_infer: sorted_tokens = x[idxs // k], then
@@ -486,8 +590,10 @@ int mr_selftest_bounded_wait(int which, mr_stream_t stream);
 /*
  * mr_get_error -- synchronise `stream`, then read and clear the current
  * device's sticky error flag.  Returns MR_OK, MR_ERR_DEVICE (a bad expert id
- * was seen), MR_ERR_TIMEOUT (a bounded wait inside a kernel gave up) or
- * MR_ERR_CUDA (the synchronisation itself failed).
+ * or inconsistent counts were seen), MR_ERR_TIMEOUT (a bounded wait inside a
+ * kernel gave up), MR_ERR_OVERFLOW (rows past a receive buffer's capacity
+ * were dropped) or MR_ERR_CUDA (the synchronisation itself failed).  When
+ * several were raised, the first of TIMEOUT, DEVICE, OVERFLOW is returned.
  */
 int mr_get_error(mr_stream_t stream);
 

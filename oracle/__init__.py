@@ -185,6 +185,45 @@ def all_to_all(send_blocks):
     return [np.concatenate([send_blocks[s][r] for s in range(ep)], axis=0) for r in range(ep)]
 
 
+def ep_dest(idx_all, N_r):
+    """Where each routed row of each rank lands in its owner's receive buffer
+    once the page's exchange has run (Kimi K2 "Add shared output" page,
+    moe_infer, ep_size > 1): every rank sorts its slots by expert (stable),
+    sends owner r the block of r's experts, the owner concatenates what it
+    receives in source order and sorts it by local expert (the stable argsort
+    of the received labels).  Here the exchange carries slot labels (source,
+    slot) instead of rows, so the position of a label in the owner's final
+    order is the row the slot's data takes there.
+
+    idx_all: list of ep [T_s, k] expert-id arrays (ids in [0, N_r)).
+    Returns (dest, local): dest[s] [T_s*k] int32 (row in the owner's buffer),
+    local[r] [E_loc] int32 (rows per local expert of owner r).
+    """
+    ep = len(idx_all)
+    if N_r % ep:
+        raise ValueError(f"{N_r} experts do not split over {ep} ranks")
+    per = [dispatch(np.asarray(i, np.int32), N_r) for i in idx_all]
+    counts_all = np.stack([c for c, _, _, _ in per])
+    send_blocks = []
+    for s, (_, offsets, perm, _) in enumerate(per):
+        labels = np.stack([np.full(int(offsets[-1]), s, np.int64),
+                           perm[:int(offsets[-1])].astype(np.int64)], axis=1)
+        send, _, _ = ep_splits(counts_all, s)
+        bounds = np.concatenate([[0], np.cumsum(send)])
+        send_blocks.append([labels[bounds[r]:bounds[r + 1]] for r in range(ep)])
+    received = all_to_all(send_blocks)
+    dest = [np.full(np.asarray(i).size, -1, np.int32) for i in idx_all]
+    local = []
+    for r in range(ep):
+        _, recv_counts, _ = ep_splits(counts_all, r)
+        order, local_r = ep_recv_order(recv_counts)
+        final = received[r][order]
+        for pos, (s, slot) in enumerate(final):
+            dest[s][slot] = pos
+        local.append(local_r)
+    return dest, local
+
+
 def expert_gemm(x_bits, k, perm, offsets, W_bits, rows=None, threads=0):
     """One expert layer over the expert-sorted rows (Kimi K2 "Add shared
     output" page, moe_infer: expert(sorted_tokens[start_idx:end_idx]) for

@@ -560,6 +560,49 @@ def test_all_to_all_emulation():
     assert got[0].tolist() == [1, 4, 5] and got[1].tolist() == [2, 3]
 
 
+def test_ep_dest_hand_case():
+    """Two ranks, four experts (rank 0 owns 0-1, rank 1 owns 2-3), two tokens
+    of two slots each.  Rank 0's slots carry experts 0, 2, 3, 0 and rank 1's
+    1, 2, 0, 3.  Owner 0 receives expert 0 from rank 0 (slots 0, 3) and rank 1
+    (slot 2), then expert 1 from rank 1 (slot 0); owner 1 receives expert 2
+    from rank 0 (slot 1) and rank 1 (slot 1), then expert 3 from rank 0
+    (slot 2) and rank 1 (slot 3)."""
+    dest, local = oracle.ep_dest([np.array([[0, 2], [3, 0]]), np.array([[1, 2], [0, 3]])], 4)
+    assert dest[0].tolist() == [0, 0, 2, 1]
+    assert dest[1].tolist() == [3, 1, 2, 3]
+    assert local[0].tolist() == [3, 1] and local[1].tolist() == [2, 2]
+
+
+@pytest.mark.parametrize("ep,N_r,k", [(1, 16, 4), (2, 16, 3), (4, 64, 8), (8, 256, 8),
+                                      (3, 12, 2)])
+def test_ep_dest_is_the_sorted_rank_of_expert_source_slot(ep, N_r, k):
+    """The destination against its plain definition: owner r's buffer lists
+    the slots routed to r's experts sorted by (expert, source rank, slot), so
+    a slot's row is its rank in that sort, computed here by numpy's lexsort
+    over all ranks' slots (ragged batch sizes, one rank with none).  With one
+    rank it is the inverse of the expert-sorted permutation."""
+    rng = np.random.default_rng(ep * 31 + N_r)
+    E_loc = N_r // ep
+    Ts = [int(rng.integers(0, 40)) for _ in range(ep)]
+    Ts[-1] = 0
+    idx_all = [np.stack([rng.choice(N_r, k, replace=False) for _ in range(T)]).astype(np.int32)
+               if T else np.zeros((0, k), np.int32) for T in Ts]
+    dest, local = oracle.ep_dest(idx_all, N_r)
+    g = np.concatenate([i.reshape(-1) for i in idx_all])
+    src = np.concatenate([np.full(i.size, s) for s, i in enumerate(idx_all)])
+    slot = np.concatenate([np.arange(i.size) for i in idx_all])
+    got = np.concatenate(dest)
+    for r in range(ep):
+        mine = np.nonzero(g // E_loc == r)[0]
+        order = mine[np.lexsort((slot[mine], src[mine], g[mine]))]
+        want = np.empty(mine.size, np.int64)
+        want[np.searchsorted(mine, order)] = np.arange(mine.size)
+        assert np.array_equal(got[mine], want)
+        assert np.array_equal(local[r], np.bincount(g[mine] - r * E_loc, minlength=E_loc))
+    if ep == 1:
+        assert np.array_equal(dest[0], oracle.dispatch(idx_all[0], N_r)[3])
+
+
 # --------------------------------------------------------------------------
 # One expert layer over the expert-sorted rows (the grouped GEMM the gather
 # feeds), against numpy's matmul on fancy-indexed rows, per expert segment.

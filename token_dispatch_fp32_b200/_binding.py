@@ -22,6 +22,7 @@ MR_ERR_UNSUPPORTED = -2
 MR_ERR_CUDA = -3
 MR_ERR_DEVICE = -4
 MR_ERR_TIMEOUT = -5
+MR_ERR_OVERFLOW = -6
 
 MR_F32 = 0
 MR_BF16 = 1
@@ -42,6 +43,12 @@ class MRError(RuntimeError):
     def __init__(self, fn: str, status: int):
         self.status = status
         super().__init__(f"{fn} failed: status {status} ({status_string(status)})")
+
+
+class _IpcHandle(C.Structure):
+    """mr_ipc_handle_t: the CUDA IPC handle of an allocation, the buffer's
+    offset in it and its size."""
+    _fields_ = [("handle", C.c_ubyte * 64), ("offset", C.c_uint64), ("bytes", C.c_uint64)]
 
 
 def lib():
@@ -79,6 +86,11 @@ def lib():
         L.mr_expert_packed_bytes.restype = sz
         L.mr_expert_pack_weights.argtypes = [p, i, i, i, p, sz, p]
         L.mr_combine.argtypes = [p, i, p, p, p, p, i, i, i, p]
+        L.mr_ep_dispatch_p2p.argtypes = [p, i, i, i, i, p, p, p, p, i, i, i, p, i, p, p, p, p]
+        L.mr_ep_combine_p2p.argtypes = [p, i, i, p, p, p, i, i, i, p, p, i, i, p]
+        L.mr_ipc_export.argtypes = [p, sz, C.POINTER(_IpcHandle)]
+        L.mr_ipc_import.argtypes = [C.POINTER(_IpcHandle), C.POINTER(p), C.POINTER(p)]
+        L.mr_ipc_close.argtypes = [p]
         L.mr_get_error.argtypes = [p]
         L.mr_selftest_bounded_wait.argtypes = [i, p]
         L.mr_launch_count.restype = C.c_uint64
@@ -417,6 +429,112 @@ def mr_combine(expert_out, w, inv_perm, shared=None, y=None, stream=None):
     _call("mr_combine", _device_of(expert_out, w, inv_perm, shared, y), stream,
           _ptr(expert_out), dt, _ptr(w), _ptr(inv_perm), _ptr(shared), _ptr(y), T, d, k)
     return y
+
+
+def _addresses(bufs, name, dev):
+    """HOST array of device addresses: each entry an int address or a CUDA
+    tensor on `dev`."""
+    out = []
+    for j, b in enumerate(bufs):
+        if isinstance(b, torch.Tensor):
+            if not b.is_cuda or b.device != dev:
+                raise ValueError(f"{name}[{j}] must be on {dev}")
+            out.append(b.data_ptr())
+        else:
+            out.append(int(b))
+    return (C.c_void_p * len(out))(*out)
+
+
+def mr_ep_dispatch_p2p(x, idx, inv_perm, offsets, counts_all, rank, recv_bufs, capacity,
+                       dest=None, local_counts=None, local_offsets=None, stream=None):
+    """This rank's rows to their owners' receive buffers (peer memory).
+    x [T,d] bf16/fp32, idx [T,k] int32, inv_perm/offsets from mr_dispatch,
+    counts_all [ep, N_r] int32 (every rank's counts), recv_bufs: ep device
+    addresses (int, e.g. from mr_ipc_import) or tensors, each a buffer of
+    capacity rows of d elements of x's dtype.  Returns (dest [T*k],
+    local_counts [E_loc], local_offsets [E_loc+1])."""
+    _need(x, "x")
+    T, d = x.shape
+    dt = _row_dtype(x)
+    _need(idx, "idx", torch.int32)
+    k = idx.shape[1]
+    _need(idx, "idx", torch.int32, (T, k))
+    _need(counts_all, "counts_all", torch.int32)
+    ep, N_r = counts_all.shape
+    _need(inv_perm, "inv_perm", torch.int32, (T * k,))
+    _need(offsets, "offsets", torch.int32, (N_r + 1,))
+    if len(recv_bufs) != ep:
+        raise ValueError(f"{len(recv_bufs)} receive buffers for {ep} ranks")
+    if N_r % ep:
+        raise ValueError(f"{N_r} experts do not split over {ep} ranks")
+    E_loc = N_r // ep
+    dev = _device_of(x, idx, inv_perm, offsets, counts_all)
+    dest = torch.empty(T * k, dtype=torch.int32, device=dev) if dest is None else \
+        _need(dest, "dest", torch.int32, (T * k,))
+    local_counts = torch.empty(E_loc, dtype=torch.int32, device=dev) if local_counts is None \
+        else _need(local_counts, "local_counts", torch.int32, (E_loc,))
+    local_offsets = torch.empty(E_loc + 1, dtype=torch.int32, device=dev) \
+        if local_offsets is None else _need(local_offsets, "local_offsets", torch.int32,
+                                            (E_loc + 1,))
+    _call("mr_ep_dispatch_p2p", _device_of(x, dest, local_counts, local_offsets), stream,
+          _ptr(x), dt, T, d, k, _ptr(idx), _ptr(inv_perm), _ptr(offsets), _ptr(counts_all), ep,
+          int(rank), N_r, _addresses(recv_bufs, "recv_bufs", dev), int(capacity), _ptr(dest),
+          _ptr(local_counts), _ptr(local_offsets))
+    return dest, local_counts, local_offsets
+
+
+def mr_ep_combine_p2p(out_bufs, w, idx, dest, N_r, capacity, d, dtype, shared=None, y=None,
+                      stream=None):
+    """y [T,d] = the weighted combine (+ shared [T,d]) of the expert outputs
+    in the owners' output buffers out_bufs (ep device addresses or tensors,
+    capacity rows of d elements of `dtype` each), slot t*k+j at row dest[t*k+j]
+    of idx[t,j]'s owner."""
+    _need(w, "w", torch.float32)
+    T, k = w.shape
+    _need(idx, "idx", torch.int32, (T, k))
+    _need(dest, "dest", torch.int32, (T * k,))
+    dev = _device_of(w, idx, dest)
+    dt = MR_BF16 if dtype == torch.bfloat16 else MR_F32 if dtype == torch.float32 else None
+    if dt is None:
+        raise TypeError("rows must be bfloat16 or float32")
+    if shared is not None:
+        _need(shared, "shared", dtype, (T, d))
+    y = torch.empty((T, d), dtype=dtype, device=dev) if y is None else \
+        _need(y, "y", dtype, (T, d))
+    ep = len(out_bufs)
+    _call("mr_ep_combine_p2p", _device_of(w, idx, dest, shared, y), stream,
+          _addresses(out_bufs, "out_bufs", dev), dt, int(d), _ptr(w), _ptr(idx), _ptr(dest), ep,
+          int(N_r), int(capacity), _ptr(shared), _ptr(y), T, k)
+    return y
+
+
+def mr_ipc_export(t) -> bytes:
+    """The IPC handle (bytes) of CUDA tensor t's memory, for another process."""
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError("t must be a CUDA tensor")
+    h = _IpcHandle()
+    with torch.cuda.device(t.device):
+        _check("mr_ipc_export", lib().mr_ipc_export(C.c_void_p(t.data_ptr()),
+                                                    t.numel() * t.element_size(), C.byref(h)))
+    return bytes(C.string_at(C.addressof(h), C.sizeof(h)))
+
+
+def mr_ipc_import(handle: bytes, device):
+    """Opens another process's handle on `device`: returns (base, address,
+    bytes); pass base to mr_ipc_close."""
+    if len(handle) != C.sizeof(_IpcHandle):
+        raise ValueError(f"an IPC handle has {C.sizeof(_IpcHandle)} bytes, got {len(handle)}")
+    h = _IpcHandle.from_buffer_copy(handle)
+    base, ptr = C.c_void_p(), C.c_void_p()
+    with torch.cuda.device(device):
+        _check("mr_ipc_import", lib().mr_ipc_import(C.byref(h), C.byref(base), C.byref(ptr)))
+    return base.value, ptr.value, int(h.bytes)
+
+
+def mr_ipc_close(base, device) -> None:
+    """Unmaps a buffer opened by mr_ipc_import."""
+    with torch.cuda.device(device):
+        _check("mr_ipc_close", lib().mr_ipc_close(C.c_void_p(base)))
 
 
 def mr_launch_count() -> int:

@@ -7,6 +7,8 @@
 // per token (grid-stride), 16-byte vectors when the row size allows.
 #pragma once
 
+#include <type_traits>
+
 #include "rows_common.cuh"
 
 namespace mr {
@@ -25,16 +27,19 @@ __device__ __forceinline__ float bf16_round(float v) {
   return __bfloat162float(__float2bfloat16_rn(v));
 }
 
-// bf16 rows, 8 elements (one uint4) per vector.
+// bf16 rows, 8 elements (one uint4) per vector.  `src` locates the expert
+// rows of each slot (SlotRowsLocal: one expert-sorted buffer through inv;
+// SlotRowsPeer: the owners' output buffers, peer memory included).
+template <typename Src>
 __global__ void __launch_bounds__(kRowThreads)
-    combine_bf16_vec_kernel(const uint4* __restrict__ E, const float* __restrict__ w,
-                            const int32_t* __restrict__ inv, const uint4* __restrict__ shared,
-                            uint4* __restrict__ y, long T, long nvec, int k) {
-  __shared__ long row[kRowMaxK];
+    combine_bf16_vec_kernel(Src src, const float* __restrict__ w,
+                            const uint4* __restrict__ shared, uint4* __restrict__ y, long T,
+                            long nvec, int k) {
+  __shared__ const uint4* row[kRowMaxK];
   __shared__ float wt[kRowMaxK];
   for (long t = blockIdx.x; t < T; t += gridDim.x) {
     if (threadIdx.x < k) {
-      row[threadIdx.x] = inv[t * k + threadIdx.x];
+      row[threadIdx.x] = src.row(t, threadIdx.x, k, nvec);
       wt[threadIdx.x] = w[t * k + threadIdx.x];
     }
     __syncthreads();
@@ -44,9 +49,9 @@ __global__ void __launch_bounds__(kRowThreads)
       for (int q = 0; q < 8; ++q) acc[q] = 0.0f;
 #pragma unroll 8
       for (int j = 0; j < k; ++j) {
-        const long r = row[j];
-        if (r < 0) continue;
-        const uint4 e = __ldg(E + r * nvec + v);
+        const uint4* r = row[j];
+        if (!r) continue;
+        const uint4 e = src.load(r + v);
         const float wj = wt[j];
         float lo, hi;
         bf16x2_unpack(e.x, lo, hi); acc[0] = fmaf(wj, lo, acc[0]); acc[1] = fmaf(wj, hi, acc[1]);
@@ -77,24 +82,25 @@ __global__ void __launch_bounds__(kRowThreads)
 }
 
 // fp32 rows, 4 elements (one float4) per vector.
+template <typename Src>
 __global__ void __launch_bounds__(kRowThreads)
-    combine_f32_vec_kernel(const float4* __restrict__ E, const float* __restrict__ w,
-                           const int32_t* __restrict__ inv, const float4* __restrict__ shared,
-                           float4* __restrict__ y, long T, long nvec, int k) {
-  __shared__ long row[kRowMaxK];
+    combine_f32_vec_kernel(Src src, const float* __restrict__ w,
+                           const float4* __restrict__ shared, float4* __restrict__ y, long T,
+                           long nvec, int k) {
+  __shared__ const float4* row[kRowMaxK];
   __shared__ float wt[kRowMaxK];
   for (long t = blockIdx.x; t < T; t += gridDim.x) {
     if (threadIdx.x < k) {
-      row[threadIdx.x] = inv[t * k + threadIdx.x];
+      row[threadIdx.x] = src.row(t, threadIdx.x, k, nvec);
       wt[threadIdx.x] = w[t * k + threadIdx.x];
     }
     __syncthreads();
     for (long v = threadIdx.x; v < nvec; v += kRowThreads) {
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
       for (int j = 0; j < k; ++j) {
-        const long r = row[j];
-        if (r < 0) continue;
-        const float4 e = __ldg(E + r * nvec + v);
+        const float4* r = row[j];
+        if (!r) continue;
+        const float4 e = src.load(r + v);
         const float wj = wt[j];
         acc.x = fmaf(wj, e.x, acc.x);
         acc.y = fmaf(wj, e.y, acc.y);
@@ -114,27 +120,30 @@ __global__ void __launch_bounds__(kRowThreads)
   }
 }
 
-// Any row size, element by element.
-template <bool BF16>
+// Any row size, element by element (Src over uint16_t for bf16 rows, float
+// for fp32).
+template <bool BF16, typename Src>
 __global__ void __launch_bounds__(kRowThreads)
-    combine_scalar_kernel(const void* __restrict__ Ev, const float* __restrict__ w,
-                          const int32_t* __restrict__ inv, const void* __restrict__ sharedv,
-                          void* __restrict__ yv, long T, long d, int k) {
-  __shared__ long row[kRowMaxK];
+    combine_scalar_kernel(Src src, const float* __restrict__ w,
+                          const void* __restrict__ sharedv, void* __restrict__ yv, long T,
+                          long d, int k) {
+  using E = typename std::conditional<BF16, uint16_t, float>::type;
+  __shared__ const E* row[kRowMaxK];
   __shared__ float wt[kRowMaxK];
   for (long t = blockIdx.x; t < T; t += gridDim.x) {
     if (threadIdx.x < k) {
-      row[threadIdx.x] = inv[t * k + threadIdx.x];
+      row[threadIdx.x] = src.row(t, threadIdx.x, k, d);
       wt[threadIdx.x] = w[t * k + threadIdx.x];
     }
     __syncthreads();
     for (long c = threadIdx.x; c < d; c += kRowThreads) {
       float acc = 0.0f;
       for (int j = 0; j < k; ++j) {
-        const long r = row[j];
-        if (r < 0) continue;
-        const float e = BF16 ? mr_bf16_to_f32(static_cast<const uint16_t*>(Ev)[r * d + c])
-                             : static_cast<const float*>(Ev)[r * d + c];
+        const E* r = row[j];
+        if (!r) continue;
+        const E raw = src.load(r + c);
+        float e;
+        if constexpr (BF16) e = mr_bf16_to_f32(raw); else e = raw;
         acc = fmaf(wt[j], e, acc);
       }
       if (BF16) {

@@ -118,4 +118,96 @@ __global__ void __launch_bounds__(kEpThreads)
   }
 }
 
+// ---- exchange over peer memory ---------------------------------------------
+//
+// Instead of two all-to-alls and a receive-side sort, every source writes
+// each of its rows straight into the owner's receive buffer at the row's final
+// place in the owner's local-expert-sorted order.  That place follows from
+// all ranks' tokens_per_expert (C[s][g], the all-gathered counts) alone:
+// owner o's buffer holds its experts in order, each expert's rows source by
+// source, each source's rows in the source's stable order, so slot (t, j) of
+// source s with expert g = o*E_loc + e, at position p of s's own sorted order,
+// goes to row
+//     sum_{e' < e} sum_{s'} C[s'][o*E_loc + e']     (the earlier local experts)
+//   + sum_{s' < s} C[s'][g]                          (earlier sources, same expert)
+//   + p - offsets[g]                                 (its place within s's segment)
+// One CTA of 1024 threads rebuilds the per-expert part (base[g], one thread per
+// expert) from C in shared memory, then maps its 4096 slots.
+
+// idx/inv/offsets: this rank's top-k ids and mr_dispatch's inverse
+// permutation and offsets; C [ep][N_r]; n = T*k.  Writes dest [n] (the row in
+// the owner's buffer, -1 for a slot without one) and, from CTA 0, this rank's
+// local_counts [E_loc] and local_offsets [E_loc + 1] as an owner, clamped to
+// the capacity.  Counts below zero, or a row of C for this rank that
+// disagrees with offsets, raise MR_FLAG_BAD_INDEX and leave every dest at -1
+// and the local counts at 0; a row past the capacity is dropped (dest -1)
+// and raises MR_FLAG_OVERFLOW.
+__global__ void __launch_bounds__(kEpThreads)
+    ep_dest_kernel(const int32_t* __restrict__ idx, const int32_t* __restrict__ inv,
+                   const int32_t* __restrict__ offsets, const int32_t* __restrict__ C, long n,
+                   int ep, int rank, int N_r, long capacity, int32_t* __restrict__ dest,
+                   int32_t* __restrict__ local_counts, int32_t* __restrict__ local_offsets) {
+  __shared__ int pre[kEpMaxSegments + 1];  // exclusive prefix of the column sums
+  __shared__ int base[kEpMaxSegments];
+  __shared__ int wsum[32];
+  __shared__ int bad_s, over_s;
+  const int tid = threadIdx.x;
+  const int E_loc = N_r / ep;
+  if (tid == 0) {
+    bad_s = 0;
+    over_s = 0;
+  }
+  __syncthreads();
+  int colsum = 0, before = 0;
+  if (tid < N_r) {
+    for (int s = 0; s < ep; ++s) {
+      const int c = C[(long)s * N_r + tid];
+      if (c < 0) bad_s = 1;
+      colsum += c;
+      if (s < rank) before += c;
+    }
+    if (C[(long)rank * N_r + tid] != offsets[tid + 1] - offsets[tid]) bad_s = 1;
+  }
+  int total = 0;
+  const int excl = ep_block_scan(tid < N_r ? colsum : 0, wsum, &total);
+  if (tid < N_r) pre[tid] = excl;
+  if (tid == 0) pre[N_r] = total;
+  __syncthreads();
+  const bool bad = bad_s != 0;
+  if (tid < N_r) base[tid] = pre[tid] - pre[(tid / E_loc) * E_loc] + before;
+  if (blockIdx.x == 0 && tid < E_loc) {
+    const int g0 = rank * E_loc;
+    const long lo = pre[g0 + tid] - pre[g0], hi = pre[g0 + tid + 1] - pre[g0];
+    const long clo = bad ? 0 : (lo < capacity ? lo : capacity);
+    const long chi = bad ? 0 : (hi < capacity ? hi : capacity);
+    local_counts[tid] = (int32_t)(chi - clo);
+    local_offsets[tid] = (int32_t)clo;
+    if (tid == E_loc - 1) local_offsets[E_loc] = (int32_t)chi;
+  }
+  __syncthreads();
+  const long i0 = (long)blockIdx.x * kEpRowsPerCta;
+  const long i1 = i0 + kEpRowsPerCta < n ? i0 + kEpRowsPerCta : n;
+  for (long i = i0 + tid; i < i1; i += kEpThreads) {
+    long r = -1;
+    const int g = idx[i];
+    const int p = inv[i];
+    if (!bad && g >= 0 && g < N_r && p >= 0) {
+      r = (long)base[g] + (p - offsets[g]);
+      if (r >= capacity) {
+        over_s = 1;
+        r = -1;
+      } else if (r < 0 || p >= offsets[g + 1]) {
+        bad_s = 1;  // inv and offsets disagree
+        r = -1;
+      }
+    }
+    dest[i] = (int32_t)r;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    if (bad_s) mr_raise(MR_FLAG_BAD_INDEX);
+    if (over_s) mr_raise(MR_FLAG_OVERFLOW);
+  }
+}
+
 }  // namespace mr

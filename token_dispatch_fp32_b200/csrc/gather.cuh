@@ -16,13 +16,15 @@ namespace mr {
 // DeepSeek-V3 batch against 354 us with 4 and plain stores (measured sweep).
 constexpr int kGatherUnroll = 8;
 
-template <typename V>
+// Each token row read once, stored to the k rows `dst` names for its slots
+// (SlotRowsLocal: the expert-sorted buffer through inv; SlotRowsPeer: the
+// receive buffers of the experts' owners, peer memory included).
+template <typename V, typename Dst>
 __global__ void __launch_bounds__(kRowThreads)
-    gather_inv_kernel(const V* __restrict__ x, long T, long nvec, int k,
-                      const int32_t* __restrict__ inv, V* __restrict__ xs) {
-  __shared__ long dst[kRowMaxK];
+    gather_inv_kernel(const V* __restrict__ x, long T, long nvec, int k, Dst dst) {
+  __shared__ V* out_row[kRowMaxK];
   for (long t = blockIdx.x; t < T; t += gridDim.x) {
-    if (threadIdx.x < k) dst[threadIdx.x] = inv[t * k + threadIdx.x];
+    if (threadIdx.x < k) out_row[threadIdx.x] = dst.row(t, threadIdx.x, k, nvec);
     __syncthreads();
     const V* src = x + t * nvec;
     for (long v0 = threadIdx.x; v0 < nvec; v0 += kGatherUnroll * kRowThreads) {
@@ -33,9 +35,8 @@ __global__ void __launch_bounds__(kRowThreads)
         if (v < nvec) val[u] = ld_stream(src + v);
       }
       for (int j = 0; j < k; ++j) {
-        const long r = dst[j];
-        if (r < 0) continue;
-        V* out = xs + r * nvec;
+        V* out = out_row[j];
+        if (!out) continue;
 #pragma unroll
         for (int u = 0; u < kGatherUnroll; ++u) {
           const long v = v0 + (long)u * kRowThreads;
@@ -45,6 +46,9 @@ __global__ void __launch_bounds__(kRowThreads)
     }
     __syncthreads();
   }
+  // stores into other GPUs' memory: ordered before whatever this GPU does
+  // next (the collective that tells the owners their rows are in)
+  if (Dst::kPeer) __threadfence_system();
 }
 
 template <typename V>

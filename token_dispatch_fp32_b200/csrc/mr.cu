@@ -6,7 +6,9 @@
 #include <cudaTypedefs.h>
 
 #include <atomic>
+#include <type_traits>
 #include <cstdlib>
+#include <cstring>
 #include <cmath>
 #include <mutex>
 
@@ -637,8 +639,9 @@ const char* mr_status_string(int status) {
     case MR_ERR_INVALID_ARG: return "invalid argument";
     case MR_ERR_UNSUPPORTED: return "unsupported shape, option or device";
     case MR_ERR_CUDA: return "CUDA launch or query failed";
-    case MR_ERR_DEVICE: return "device flag: expert id out of range";
+    case MR_ERR_DEVICE: return "device flag: expert id out of range or inconsistent counts";
     case MR_ERR_TIMEOUT: return "device flag: bounded wait timed out";
+    case MR_ERR_OVERFLOW: return "device flag: rows past a receive buffer's capacity dropped";
     default: return "unknown status";
   }
 }
@@ -1082,6 +1085,38 @@ int mr_expert_gemm_gather_packed(const void* x, const int32_t* perm, const int32
                             reinterpret_cast<cudaStream_t>(stream));
 }
 
+}  // extern "C"
+
+namespace {
+
+// The combine kernel for the row type: 16-byte vectors (bf16 or fp32) when
+// `vec`, elements otherwise.  make_src(V* tag) builds the slot-row policy
+// over the element or vector type V.
+template <typename MakeSrc>
+int launch_combine(bool vec, bool bf16, unsigned grid, cudaStream_t s, const float* w,
+                   const void* shared, void* y, long T, long d, int k, MakeSrc make_src) {
+  if (vec && bf16) {
+    auto src = make_src(static_cast<uint4*>(nullptr));
+    mr::combine_bf16_vec_kernel<<<grid, mr::kRowThreads, 0, s>>>(
+        src, w, static_cast<const uint4*>(shared), static_cast<uint4*>(y), T, d / 8, k);
+  } else if (vec) {
+    auto src = make_src(static_cast<float4*>(nullptr));
+    mr::combine_f32_vec_kernel<<<grid, mr::kRowThreads, 0, s>>>(
+        src, w, static_cast<const float4*>(shared), static_cast<float4*>(y), T, d / 4, k);
+  } else if (bf16) {
+    auto src = make_src(static_cast<uint16_t*>(nullptr));
+    mr::combine_scalar_kernel<true><<<grid, mr::kRowThreads, 0, s>>>(src, w, shared, y, T, d, k);
+  } else {
+    auto src = make_src(static_cast<float*>(nullptr));
+    mr::combine_scalar_kernel<false><<<grid, mr::kRowThreads, 0, s>>>(src, w, shared, y, T, d, k);
+  }
+  return launch_status();
+}
+
+}  // namespace
+
+extern "C" {
+
 // ---- gather / combine -------------------------------------------------------
 
 int mr_gather_rows(const void* x, int dtype, int T, int d, int k, const int32_t* perm,
@@ -1105,13 +1140,16 @@ int mr_gather_rows(const void* x, int dtype, int T, int d, int k, const int32_t*
   if (inv_perm) {
     if (vec)
       mr::gather_inv_kernel<uint4><<<grid_t, mr::kRowThreads, 0, s>>>(
-          static_cast<const uint4*>(x), T, row_bytes / 16, k, inv_perm, static_cast<uint4*>(xs));
+          static_cast<const uint4*>(x), T, row_bytes / 16, k,
+          mr::SlotRowsLocal<uint4>{static_cast<uint4*>(xs), inv_perm});
     else if (esz == 4)
       mr::gather_inv_kernel<uint32_t><<<grid_t, mr::kRowThreads, 0, s>>>(
-          static_cast<const uint32_t*>(x), T, d, k, inv_perm, static_cast<uint32_t*>(xs));
+          static_cast<const uint32_t*>(x), T, d, k,
+          mr::SlotRowsLocal<uint32_t>{static_cast<uint32_t*>(xs), inv_perm});
     else
       mr::gather_inv_kernel<uint16_t><<<grid_t, mr::kRowThreads, 0, s>>>(
-          static_cast<const uint16_t*>(x), T, d, k, inv_perm, static_cast<uint16_t*>(xs));
+          static_cast<const uint16_t*>(x), T, d, k,
+          mr::SlotRowsLocal<uint16_t>{static_cast<uint16_t*>(xs), inv_perm});
   } else {
     if (vec)
       mr::gather_perm_kernel<uint4><<<grid_r, mr::kRowThreads, 0, s>>>(
@@ -1143,21 +1181,150 @@ int mr_combine(const void* expert_out, int dtype, const float* w, const int32_t*
   // 64 CTAs per SM, grid-stride (369 us on the full DeepSeek-V3 batch; 372 us
   // with 32 per SM)
   const unsigned grid = (unsigned)std::min<long>(T, (long)sms * 64);
-  if (vec && dtype == MR_BF16)
-    mr::combine_bf16_vec_kernel<<<grid, mr::kRowThreads, 0, s>>>(
-        static_cast<const uint4*>(expert_out), w, inv_perm, static_cast<const uint4*>(shared),
-        static_cast<uint4*>(y), T, row_bytes / 16, k);
-  else if (vec)
-    mr::combine_f32_vec_kernel<<<grid, mr::kRowThreads, 0, s>>>(
-        static_cast<const float4*>(expert_out), w, inv_perm, static_cast<const float4*>(shared),
-        static_cast<float4*>(y), T, row_bytes / 16, k);
-  else if (dtype == MR_BF16)
-    mr::combine_scalar_kernel<true><<<grid, mr::kRowThreads, 0, s>>>(expert_out, w, inv_perm,
-                                                                     shared, y, T, d, k);
+  return launch_combine(vec, dtype == MR_BF16, grid, s, w, shared, y, T, d, k,
+                        [&](auto* tag) {
+                          using V = std::remove_const_t<std::remove_pointer_t<decltype(tag)>>;
+                          return mr::SlotRowsLocal<const V>{static_cast<const V*>(expert_out),
+                                                            inv_perm};
+                        });
+}
+
+// ---- expert parallelism over peer memory ------------------------------------
+
+int mr_ep_dispatch_p2p(const void* x, int dtype, int T, int d, int k, const int32_t* idx,
+                       const int32_t* inv_perm, const int32_t* offsets,
+                       const int32_t* counts_all, int ep, int rank, int N_r,
+                       void* const* recv_bufs, int capacity, int32_t* dest,
+                       int32_t* local_counts, int32_t* local_offsets, mr_stream_t stream) {
+  if (T < 0 || d <= 0 || k <= 0 || (dtype != MR_F32 && dtype != MR_BF16)) return MR_ERR_INVALID_ARG;
+  if ((long long)T * k >= (1LL << 31) || capacity < 0) return MR_ERR_INVALID_ARG;
+  if (ep <= 0 || rank < 0 || rank >= ep || N_r <= 0 || N_r % ep != 0) return MR_ERR_INVALID_ARG;
+  if (k > mr::kRowMaxK || ep > mr::kEpMaxRanks || N_r > mr::kEpMaxSegments)
+    return MR_ERR_UNSUPPORTED;
+  if (!counts_all || !recv_bufs || !local_counts || !local_offsets) return MR_ERR_INVALID_ARG;
+  if (T > 0 && (!x || !idx || !inv_perm || !offsets || !dest)) return MR_ERR_INVALID_ARG;
+  mr::EpPeers peers{};
+  for (int r = 0; r < ep; ++r) {
+    if (!recv_bufs[r]) return MR_ERR_INVALID_ARG;
+    peers.p[r] = recv_bufs[r];
+  }
+  int sms = 0, cc = 0;
+  if (!device_info(&sms, &cc)) return MR_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const long n = (long)T * k;
+  const unsigned grid_d =
+      (unsigned)std::max<long>(1, (n + mr::kEpRowsPerCta - 1) / mr::kEpRowsPerCta);
+  mr::ep_dest_kernel<<<grid_d, mr::kEpThreads, 0, s>>>(idx, inv_perm, offsets, counts_all, n, ep,
+                                                        rank, N_r, capacity, dest, local_counts,
+                                                        local_offsets);
+  if (launch_status() != MR_OK) return MR_ERR_CUDA;
+  if (T == 0) return MR_OK;
+  const long esz = dtype == MR_BF16 ? 2 : 4;
+  const long row_bytes = (long)d * esz;
+  bool vec = row_bytes % 16 == 0 && aligned16(x);
+  for (int r = 0; r < ep; ++r) vec = vec && aligned16(recv_bufs[r]);
+  const unsigned grid_t = (unsigned)std::min<long>(T, 1L << 30);
+  const int E_loc = N_r / ep;
+  if (vec)
+    mr::gather_inv_kernel<uint4><<<grid_t, mr::kRowThreads, 0, s>>>(
+        static_cast<const uint4*>(x), T, row_bytes / 16, k,
+        mr::SlotRowsPeer<uint4>{peers, idx, dest, E_loc, N_r, capacity});
+  else if (esz == 4)
+    mr::gather_inv_kernel<uint32_t><<<grid_t, mr::kRowThreads, 0, s>>>(
+        static_cast<const uint32_t*>(x), T, d, k,
+        mr::SlotRowsPeer<uint32_t>{peers, idx, dest, E_loc, N_r, capacity});
   else
-    mr::combine_scalar_kernel<false><<<grid, mr::kRowThreads, 0, s>>>(expert_out, w, inv_perm,
-                                                                      shared, y, T, d, k);
+    mr::gather_inv_kernel<uint16_t><<<grid_t, mr::kRowThreads, 0, s>>>(
+        static_cast<const uint16_t*>(x), T, d, k,
+        mr::SlotRowsPeer<uint16_t>{peers, idx, dest, E_loc, N_r, capacity});
   return launch_status();
+}
+
+int mr_ep_combine_p2p(const void* const* out_bufs, int dtype, int d, const float* w,
+                      const int32_t* idx, const int32_t* dest, int ep, int N_r, int capacity,
+                      const void* shared, void* y, int T, int k, mr_stream_t stream) {
+  if (T < 0 || d <= 0 || k <= 0 || (dtype != MR_F32 && dtype != MR_BF16)) return MR_ERR_INVALID_ARG;
+  if ((long long)T * k >= (1LL << 31) || capacity < 0) return MR_ERR_INVALID_ARG;
+  if (ep <= 0 || N_r <= 0 || N_r % ep != 0) return MR_ERR_INVALID_ARG;
+  if (k > mr::kRowMaxK || ep > mr::kEpMaxRanks) return MR_ERR_UNSUPPORTED;
+  if (!out_bufs) return MR_ERR_INVALID_ARG;
+  if (T == 0) return MR_OK;
+  if (!w || !idx || !dest || !y) return MR_ERR_INVALID_ARG;
+  mr::EpPeers peers{};
+  for (int r = 0; r < ep; ++r) {
+    if (!out_bufs[r]) return MR_ERR_INVALID_ARG;
+    peers.p[r] = const_cast<void*>(out_bufs[r]);
+  }
+  int sms = 0, cc = 0;
+  if (!device_info(&sms, &cc)) return MR_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const long esz = dtype == MR_BF16 ? 2 : 4;
+  bool vec = ((long)d * esz) % 16 == 0 && aligned16(y) && (!shared || aligned16(shared));
+  for (int r = 0; r < ep; ++r) vec = vec && aligned16(out_bufs[r]);
+  const unsigned grid = (unsigned)std::min<long>(T, (long)sms * 64);
+  const int E_loc = N_r / ep;
+  return launch_combine(vec, dtype == MR_BF16, grid, s, w, shared, y, T, d, k, [&](auto* tag) {
+    using V = std::remove_const_t<std::remove_pointer_t<decltype(tag)>>;
+    return mr::SlotRowsPeer<const V>{peers, idx, dest, E_loc, N_r, capacity};
+  });
+}
+
+// ---- peer buffers between processes -----------------------------------------
+
+static_assert(sizeof(cudaIpcMemHandle_t) == sizeof(((mr_ipc_handle_t*)nullptr)->handle),
+              "mr_ipc_handle_t.handle holds one CUDA IPC handle");
+
+int mr_ipc_export(const void* dev_ptr, size_t bytes, mr_ipc_handle_t* out) {
+  if (!dev_ptr || !out) return MR_ERR_INVALID_ARG;
+  static PFN_cuMemGetAddressRange_v3020 range = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuMemGetAddressRange", &fn, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      range = reinterpret_cast<PFN_cuMemGetAddressRange_v3020>(fn);
+  });
+  if (!range) return MR_ERR_CUDA;
+  CUdeviceptr base = 0;
+  size_t size = 0;
+  if (range(&base, &size, reinterpret_cast<CUdeviceptr>(dev_ptr)) != CUDA_SUCCESS)
+    return MR_ERR_INVALID_ARG;  // not device memory of this process
+  const uint64_t off = reinterpret_cast<CUdeviceptr>(dev_ptr) - base;
+  if (off + bytes > size) return MR_ERR_INVALID_ARG;
+  cudaIpcMemHandle_t h;
+  if (cudaIpcGetMemHandle(&h, reinterpret_cast<void*>(base)) != cudaSuccess) {
+    cudaGetLastError();
+    return MR_ERR_UNSUPPORTED;  // e.g. memory from the virtual memory API
+  }
+  memcpy(out->handle, &h, sizeof(h));
+  out->offset = off;
+  out->bytes = bytes;
+  return MR_OK;
+}
+
+int mr_ipc_import(const mr_ipc_handle_t* h, void** base, void** ptr) {
+  if (!h || !base || !ptr) return MR_ERR_INVALID_ARG;
+  cudaIpcMemHandle_t ch;
+  memcpy(&ch, h->handle, sizeof(ch));
+  void* b = nullptr;
+  if (cudaIpcOpenMemHandle(&b, ch, cudaIpcMemLazyEnablePeerAccess) != cudaSuccess) {
+    cudaGetLastError();
+    return MR_ERR_CUDA;
+  }
+  *base = b;
+  *ptr = static_cast<char*>(b) + h->offset;
+  return MR_OK;
+}
+
+int mr_ipc_close(void* base) {
+  if (!base) return MR_ERR_INVALID_ARG;
+  if (cudaIpcCloseMemHandle(base) != cudaSuccess) {
+    cudaGetLastError();
+    return MR_ERR_CUDA;
+  }
+  return MR_OK;
 }
 
 // ---- device error flag ----------------------------------------------------
@@ -1171,7 +1338,8 @@ int mr_get_error(mr_stream_t stream) {
   if (cudaMemcpyFromSymbol(&flag, g_mr_error_flag, sizeof(flag)) != cudaSuccess) return MR_ERR_CUDA;
   if (flag == 0) return MR_OK;
   if (cudaMemcpyToSymbol(g_mr_error_flag, &zero, sizeof(zero)) != cudaSuccess) return MR_ERR_CUDA;
-  return (flag & MR_FLAG_TIMEOUT) ? MR_ERR_TIMEOUT : MR_ERR_DEVICE;
+  if (flag & MR_FLAG_TIMEOUT) return MR_ERR_TIMEOUT;
+  return (flag & MR_FLAG_BAD_INDEX) ? MR_ERR_DEVICE : MR_ERR_OVERFLOW;
 }
 
 }  // extern "C"

@@ -11,6 +11,7 @@
 // The library is one translation unit, so the flag is defined here.
 #define MR_FLAG_BAD_INDEX 1u
 #define MR_FLAG_TIMEOUT 2u
+#define MR_FLAG_OVERFLOW 4u
 __device__ unsigned int g_mr_error_flag = 0;
 
 __device__ __forceinline__ void mr_raise(unsigned int f) { atomicOr(&g_mr_error_flag, f); }

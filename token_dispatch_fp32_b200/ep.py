@@ -26,10 +26,20 @@ variable-split all-to-all takes them as host integers (here one copy of
 2*N_r integers).  Every local step runs in libmr.so's
 kernels; this module only orders the steps, sums the split sizes on the host
 and moves buffers.
+
+The second half of the module does the same exchange over peer memory
+(ep_dispatch_p2p / ep_combine_p2p): every rank maps the others' receive and
+output buffers (PeerBuffers), an all-gather of tokens_per_expert replaces
+the count all-to-all, one kernel writes each row straight into its owner's
+receive buffer at its final local-expert-sorted place (steps 2, 4 and 5 in
+one pass, no host read-back), and one kernel combines straight out of the
+owners' output buffers (steps 6-8).  Collectives on the stream order the
+ranks' steps; no kernel waits on another rank.
 """
 from __future__ import annotations
 
 import dataclasses
+import threading
 
 import torch
 import torch.distributed as dist
@@ -121,3 +131,132 @@ def ep_combine(local_out, handle: EPHandle, w, shared=None, group=None, stream=N
     received = mr.mr_gather_rows(local_out, 1, inv_perm=handle.order, stream=stream)
     back = exchange_rows(received, handle.recv_splits, handle.send_splits, group)
     return mr.mr_combine(back, w, handle.inv_perm, shared, stream=stream)
+
+
+# ---- the exchange over peer memory ------------------------------------------
+
+_opened = {}  # (device index, allocation handle) -> [base, references]
+_opened_lock = threading.Lock()
+
+
+def _import(handle: bytes, device):
+    """Opens another process's buffer once per allocation (a second open of
+    the same allocation in one process is refused by CUDA): returns (key,
+    address)."""
+    key = (torch.device(device).index, handle[:64])
+    offset = int.from_bytes(handle[64:72], "little")  # mr_ipc_handle_t.offset
+    with _opened_lock:
+        ent = _opened.get(key)
+        if ent is None:
+            base, _, _ = mr.mr_ipc_import(handle, device)
+            ent = _opened[key] = [base, 0]
+        ent[1] += 1
+        return key, ent[0] + offset
+
+
+def _release(key, device) -> None:
+    with _opened_lock:
+        ent = _opened[key]
+        ent[1] -= 1
+        if ent[1] == 0:
+            del _opened[key]
+            mr.mr_ipc_close(ent[0], device)
+
+
+class PeerBuffers:
+    """One [rows, d] buffer per rank, all of them addressable from this
+    process: this rank's own (`local`, a tensor on its device) and every
+    other rank's, mapped through CUDA IPC (handles exchanged with an
+    all-gather over `group`).  `ptrs[r]` is rank r's buffer as seen here.
+    Ranks on different GPUs need peer access between them (NVLink/NVSwitch);
+    ranks may also share a GPU."""
+
+    def __init__(self, rows: int, d: int, dtype, group=None, device=None):
+        self.rows, self.d, self.dtype = int(rows), int(d), dtype
+        self.device = torch.device(device if device is not None else torch.cuda.current_device())
+        self.rank = dist.get_rank(group)
+        self.ep = dist.get_world_size(group)
+        self.local = torch.empty((self.rows, self.d), dtype=dtype, device=self.device)
+        mine = mr.mr_ipc_export(self.local)
+        handles = [None] * self.ep
+        dist.all_gather_object(handles, mine, group=group)
+        self._keys = []
+        self.ptrs = []
+        for r, h in enumerate(handles):
+            if r == self.rank:
+                self.ptrs.append(self.local.data_ptr())
+            else:
+                key, ptr = _import(h, self.device)
+                self._keys.append(key)
+                self.ptrs.append(ptr)
+
+    def close(self) -> None:
+        """Unmaps the other ranks' buffers (call on every rank once no kernel
+        uses them any more)."""
+        for key in self._keys:
+            _release(key, self.device)
+        self._keys = []
+        self.ptrs = []
+
+
+def stream_barrier(group=None) -> None:
+    """Orders the ranks' GPU work: with NCCL a one-element all-reduce on the
+    current stream (nothing after it on any rank's stream runs before every
+    rank's work before it is done); with other backends the stream is
+    synchronised and the ranks meet on the host."""
+    if dist.get_backend(group) == "nccl":
+        t = torch.zeros(1, dtype=torch.int32, device=torch.cuda.current_device())
+        dist.all_reduce(t, group=group)
+    else:
+        torch.cuda.current_stream().synchronize()
+        dist.barrier(group=group)
+
+
+def gather_counts(counts: torch.Tensor, group=None) -> torch.Tensor:
+    """Every rank's tokens_per_expert, rank-major [ep, N_r] on counts' device
+    (all-gather; on the device with NCCL, through the host otherwise)."""
+    ep = dist.get_world_size(group)
+    if dist.get_backend(group) == "nccl":
+        out = torch.empty((ep, counts.numel()), dtype=counts.dtype, device=counts.device)
+        dist.all_gather_into_tensor(out, counts.contiguous(), group=group)
+        return out
+    host = counts.cpu()
+    parts = [torch.empty_like(host) for _ in range(ep)]
+    dist.all_gather(parts, host, group=group)
+    return torch.stack(parts).to(counts.device)
+
+
+@dataclasses.dataclass
+class P2PHandle:
+    """What the combine needs from one dispatch over peer memory."""
+    idx: torch.Tensor
+    dest: torch.Tensor
+    N_r: int
+
+
+def ep_dispatch_p2p(x_rows, idx, N_r, recv: PeerBuffers, group=None):
+    """Dispatch of this rank's tokens straight into the owners' receive
+    buffers, on the current stream.  x_rows [T,d], idx [T,k] int32.  Returns (rows, local_counts,
+    local_offsets, handle): rows = this rank's receive buffer, whose first
+    local_offsets[-1] rows are what it received, sorted by local expert
+    (stable), local_counts [E_loc] / local_offsets [E_loc+1] on the device.
+    No host synchronisation: the expert layer reads the offsets on the
+    device (mr_expert_gemm_gather with perm=None)."""
+    counts, offsets, _, inv = mr.mr_dispatch(idx, N_r)
+    counts_all = gather_counts(counts, group)
+    dest, local_counts, local_offsets = mr.mr_ep_dispatch_p2p(
+        x_rows, idx, inv, offsets, counts_all, recv.rank, recv.ptrs, recv.rows)
+    stream_barrier(group)  # every source's rows are in
+    return recv.local, local_counts, local_offsets, P2PHandle(idx, dest, N_r)
+
+
+def ep_combine_p2p(out: PeerBuffers, handle: P2PHandle, w, shared=None, group=None):
+    """The weighted combine (+ shared [T,d]) of this rank's tokens, on the
+    current stream, reading
+    the expert outputs straight out of the owners' output buffers (row i of
+    owner r's `out` buffer is the output of its receive row i).  Returns y
+    [T,d].  The next ep_dispatch_p2p's count all-gather keeps the owners
+    from overwriting their outputs before every rank has combined."""
+    stream_barrier(group)  # every owner's outputs are complete
+    return mr.mr_ep_combine_p2p(out.ptrs, w, handle.idx, handle.dest, handle.N_r, out.rows,
+                                out.d, out.dtype, shared)
