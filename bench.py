@@ -40,14 +40,20 @@ import workloads as wl  # noqa: E402
 METRIC = "routed tokens/sec (router+dispatch+combine) at 1 B200; % of roofline"
 UNIT = "tokens/s"
 
+# B200 peer-to-peer copy bandwidth per direction over NVLink 5 / NVSwitch
+# (measured copy; 900 GB/s nominal): the bound of rows crossing to other GPUs.
+NVLINK_PEER_GBS = 770.0
+
 # DRAM traffic per launch measured with ncu (dram__bytes_read.sum +
 # dram__bytes_write.sum) for the dominant kernel, keyed by the SHA-256 of the
 # source file it was built from; reported only while the source is unchanged.
 NCU_TRAFFIC = {
-    # ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum on the full V3
-    # workload (T=16384), 64 CTAs per SM, streaming stores: 2.115 GB read +
-    # 223.45 MB written per launch.
-    "combine": {"src": "97f9ba70f1ba7f45", "bytes": 2.115008768e9 + 223.45088e6},
+    # ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum of the current
+    # source on the DeepSeek-V3 prefill batch (T=4096): 528.77 MB read + 47.72
+    # MB written per launch, scaled by the tokens (x4) to the full batch --
+    # reads scale exactly (2.115 GB read at T=16384 in a full-size capture of
+    # the kernel before its rows were located through a policy object).
+    "combine": {"src": "3556d6f06cf4dcd2", "bytes": 4 * (528.76992e6 + 47.716864e6)},
 }
 
 
@@ -636,6 +642,88 @@ def run_ours(args, w: wl.Workload, rank: int, world: int):
         del ex, ews, eW, eWp, eout, exs
         assert mr.mr_get_error(stream) == mr.MR_OK
 
+    # Expert parallelism over peer memory, 8 ranks emulated on this GPU: each
+    # rank routes a DeepSeek-V3 prefill batch of its own seed with the shared
+    # gate, and every owner's receive buffer lives in this GPU's memory (with
+    # 8 GPUs, the stores to the 7 other owners would cross NVLink instead).
+    # Timed alone: one source's mr_ep_dispatch_p2p (destinations + its rows
+    # stored into the 8 owners' buffers) beside mr_gather_rows of the same
+    # rows into one buffer, and one source's mr_ep_combine_p2p reading the 8
+    # buffers (identity experts) beside mr_combine of its own sorted rows.
+    ep_stage = None
+    if args.workload == wl.V3_FULL.name and not args.no_extra_stages:
+        n_ep, wp = 8, wl.V3_PREFILL
+        E_loc = wp.N_r // n_ep
+        gate = wl.gen_router_inputs(wp)
+        gW = torch.from_numpy(gate["W"]).to(dev)
+        gb = torch.from_numpy(gate["b"]).to(dev)
+        gws = torch.empty(max(4, mr.mr_router_workspace_size(wp.T, wp.d, wp.N_r)),
+                          dtype=torch.uint8, device=dev)
+        srcs = []
+        for r in range(n_ep):
+            xin = gate if r == 0 else wl.gen_router_inputs(wp.replace(seed=wp.seed + 7919 * r))
+            rx = torch.from_numpy(xin["x_bf16"]).view(torch.bfloat16).to(dev)
+            ridx, rwt = mr.mr_router_forward_ex(rx, gW, gb, wp.n_group, wp.topk_group, wp.k,
+                                                wp.route_scale, wp.mask_mode,
+                                                precision=mr.MR_PREC_BF16X3, workspace=gws,
+                                                stream=stream)
+            rc, ro, rperm, rinv = mr.mr_dispatch(ridx, wp.N_r, stream=stream)
+            srcs.append(dict(x=rx, idx=ridx, w=rwt, counts=rc, offsets=ro, perm=rperm, inv=rinv))
+        counts_all = torch.stack([s_["counts"] for s_ in srcs]).contiguous()
+        per_owner = counts_all.cpu().numpy().reshape(n_ep, n_ep, E_loc).sum(axis=(0, 2))
+        cap = int(per_owner.max())
+        bufs = [torch.empty((cap, wp.d), dtype=torch.bfloat16, device=dev) for _ in range(n_ep)]
+        for r, s_ in enumerate(srcs):  # every owner's buffer filled once
+            s_["dest"], s_["lc"], s_["lo"] = mr.mr_ep_dispatch_p2p(
+                s_["x"], s_["idx"], s_["inv"], s_["offsets"], counts_all, r, bufs, cap,
+                stream=stream)
+        s0 = srcs[0]
+        xs0 = torch.empty((wp.T * wp.k, wp.d), dtype=torch.bfloat16, device=dev)
+        sh0 = torch.randn((wp.T, wp.d), generator=torch.Generator(dev).manual_seed(wp.seed),
+                          device=dev).to(torch.bfloat16)
+        y0 = torch.empty((wp.T, wp.d), dtype=torch.bfloat16, device=dev)
+
+        def p2p_dispatch():
+            mr.mr_ep_dispatch_p2p(s0["x"], s0["idx"], s0["inv"], s0["offsets"], counts_all, 0,
+                                  bufs, cap, dest=s0["dest"], local_counts=s0["lc"],
+                                  local_offsets=s0["lo"], stream=stream)
+
+        def local_gather():
+            mr.mr_gather_rows(s0["x"], wp.k, perm=s0["perm"], inv_perm=s0["inv"], xs=xs0,
+                              stream=stream)
+
+        def p2p_combine():
+            mr.mr_ep_combine_p2p(bufs, s0["w"], s0["idx"], s0["dest"], wp.N_r, cap, wp.d,
+                                 torch.bfloat16, sh0, y=y0, stream=stream)
+
+        def local_combine():
+            mr.mr_combine(xs0, s0["w"], s0["inv"], sh0, y=y0, stream=stream)
+
+        pd_ms = time_alone(p2p_dispatch, n_alone)
+        lg_ms = time_alone(local_gather, n_alone)
+        pc_ms = time_alone(p2p_combine, n_alone)
+        lc_ms = time_alone(local_combine, n_alone)
+        assert mr.mr_get_error(stream) == mr.MR_OK
+        rows_b = wp.T * wp.k * wp.d * 2
+        d_bytes = wp.T * wp.d * 2 + rows_b + 3 * 4 * wp.T * wp.k  # x, rows, idx/inv/dest
+        c_bytes = rows_b + 2 * wp.T * wp.d * 2 + 3 * 4 * wp.T * wp.k  # rows, shared + y, w/idx/dest
+        remote = int(((s0["idx"] // E_loc) != 0).sum().item())
+        ep_stage = {
+            "workload": f"{n_ep} ranks x {wp.name}, ranks emulated on one GPU "
+                        "(every owner's buffer in this GPU's memory)",
+            "capacity_rows": cap, "rows_per_source": wp.T * wp.k,
+            "rows_to_other_owners": remote,
+            "dispatch_p2p_ms": pd_ms, "dispatch_p2p_gbs": d_bytes / (pd_ms / 1e3) / 1e9,
+            "gather_one_buffer_ms": lg_ms,
+            "combine_p2p_ms": pc_ms, "combine_p2p_gbs": c_bytes / (pc_ms / 1e3) / 1e9,
+            "combine_one_buffer_ms": lc_ms,
+            "nvlink_bound_ms_8_gpus": remote * wp.d * 2 / (NVLINK_PEER_GBS * 1e9) * 1e3,
+            "nvlink_note": f"rows to the other owners / {NVLINK_PEER_GBS} GB/s per direction "
+                           "(B200 peer copy, measured; 900 nominal): the dispatch's bound "
+                           "on 8 GPUs, unmeasured here",
+            "l2": "read pass over 512 MB before each call"}
+        del srcs, bufs, xs0, sh0, y0, gW, gb, gws, counts_all
+
     # The decode-size router (one position x batch 64): W read once per call.
     # Main figure: the plain entry point with the config's fp32 rows (split-K
     # over all SMs + reduce-and-route, no workspace).  Beside it: bf16 rows
@@ -820,6 +908,10 @@ def run_ours(args, w: wl.Workload, rank: int, world: int):
                                     expert["n_out"] / (peaks["bf16_tflops"] * 1e12) * 1e3)
         expert["frac_of_roofline"] = expert["roofline_ms"] / expert["ms"]
         stages["expert_gemm_gather_deepseek_v3_prefill_T4096"] = expert
+    if ep_stage is not None:
+        ep_stage["dispatch_p2p_frac_hbm"] = ep_stage["dispatch_p2p_gbs"] / peaks["hbm_gbs"]
+        ep_stage["combine_p2p_frac_hbm"] = ep_stage["combine_p2p_gbs"] / peaks["hbm_gbs"]
+        stages["ep_p2p_deepseek_v3_prefill_8_ranks"] = ep_stage
     if decode is not None:
         decode["frac_hbm"] = decode["gbs"] / peaks["hbm_gbs"]
         if decode.get("gbs_cuda_graph"):
