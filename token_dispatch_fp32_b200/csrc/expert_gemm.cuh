@@ -108,8 +108,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr uint32_t kABytes = PL::kABytes, kStageBytes = PL::kStageBytes,
                      kBarOff = PL::kBarOff;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // 1024-byte aligned start by pointer arithmetic on the shared array, so the
+  // compiler keeps the shared address space for every access through it (an
+  // integer round trip would turn them into generic loads and stores)
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kBarOff);
   int* tok_s = reinterpret_cast<int*>(smem + kBarOff + 256);      // [128] token of each row
   int* misc = reinterpret_cast<int*>(smem + kBarOff + 256 + 4 * BM);

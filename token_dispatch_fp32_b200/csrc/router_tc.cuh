@@ -531,8 +531,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                      const __grid_constant__ CUtensorMap map_w,
                      const __grid_constant__ CUtensorMap map_wlo, const Params P) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // 1024-byte aligned start by pointer arithmetic on the shared array, so the
+  // compiler keeps the shared address space for every access through it (an
+  // integer round trip would turn them into generic loads and stores)
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const int NL = P.NL;
   const bool bf16x3 = P.bf16x3 != 0;
   // The 2-SM instructions exist only in the PAIR instantiation: a kernel that
