@@ -1029,41 +1029,69 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok && c_beg < c_end) {
           float a1 = -INFINITY, a2 = -INFINITY;
           int g = (col0 + c_beg * 16) / S, next_b = (g + 1) * S;
-          auto body1 = [&](int c, float(&x)[16]) {
+          // S a multiple of 16: every 16-column chunk lies inside one group
+          const bool chunk_groups = (S % 16) == 0;
+          // one chunk per iteration (one copy of the body in the code: the
+          // routing runs once per CTA, so its instructions are fetched cold)
+#pragma unroll 1
+          for (int c = c_beg; c < c_end; ++c) {
+            __syncwarp();
+            tmem_ld16(tmem_base + lane_off + (uint32_t)(c * 16), v);
             load_bias(c);
             if constexpr (softmax) {
 #pragma unroll
-              for (int i = 0; i < 16; ++i) x[i] = __expf(x[i] - smx) * sinv;
+              for (int i = 0; i < 16; ++i) v[i] = __expf(v[i] - smx) * sinv;
             } else {
 #pragma unroll
-              for (int i = 0; i < 16; ++i) x[i] = mr_sigmoid(x[i]);
+              for (int i = 0; i < 16; ++i) v[i] = mr_sigmoid(v[i]);
             }
-            tmem_st16(tmem_base + lane_off + (uint32_t)(c * 16), x);
-            if (G == 1) return;
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const int e = col0 + c * 16 + i;
-              if (e == next_b) {
+            tmem_st16(tmem_base + lane_off + (uint32_t)(c * 16), v);
+            if (G == 1) continue;
+            if (chunk_groups) {
+              const int gc = (col0 + c * 16) / S;
+              if (gc != g) {
                 exA1[(h * G + g) * BM + row] = a1;
                 exA2[(h * G + g) * BM + row] = a2;
-                ++g;
-                next_b += S;
+                g = gc;
                 a1 = -INFINITY;
                 a2 = -INFINITY;
               }
-              const float cval = x[i] + bv[i];
-              a2 = fmaxf(a2, fminf(a1, cval));  // top-2 of the values seen
-              a1 = fmaxf(a1, cval);
+              // the chunk's top-2 of c = s + b as a tree of pair merges
+              float p1[8], p2[8];
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                const float x0 = v[2 * j] + bv[2 * j], x1 = v[2 * j + 1] + bv[2 * j + 1];
+                p1[j] = fmaxf(x0, x1);
+                p2[j] = fminf(x0, x1);
+              }
+#pragma unroll
+              for (int w = 4; w >= 1; w >>= 1)
+#pragma unroll
+                for (int j = 0; j < w; ++j) {
+                  const float hi = fmaxf(p1[j], p1[j + w]);
+                  p2[j] = fmaxf(fminf(p1[j], p1[j + w]), fmaxf(p2[j], p2[j + w]));
+                  p1[j] = hi;
+                }
+              const float hi = fmaxf(a1, p1[0]);
+              a2 = fmaxf(fminf(a1, p1[0]), fmaxf(a2, p2[0]));
+              a1 = hi;
+            } else {
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                const int e = col0 + c * 16 + i;
+                if (e == next_b) {
+                  exA1[(h * G + g) * BM + row] = a1;
+                  exA2[(h * G + g) * BM + row] = a2;
+                  ++g;
+                  next_b += S;
+                  a1 = -INFINITY;
+                  a2 = -INFINITY;
+                }
+                const float cval = v[i] + bv[i];
+                a2 = fmaxf(a2, fminf(a1, cval));  // top-2 of the values seen
+                a1 = fmaxf(a1, cval);
+              }
             }
-          };
-          // two chunks per TMEM round trip (the second load of an odd tail
-          // re-reads the first chunk and is ignored)
-          for (int c = c_beg; c < c_end; c += 2) {
-            const int c2 = c + 1 < c_end ? c + 1 : c;
-            tmem_ld16x2(tmem_base + lane_off + (uint32_t)(c * 16),
-                        tmem_base + lane_off + (uint32_t)(c2 * 16), v, v2);
-            body1(c, v);
-            if (c2 != c) body1(c2, v2);
           }
           asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
           if (G > 1) {
@@ -1110,50 +1138,57 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           cnt = 0;
         };
-        int g = (col0 + c_beg * 16) / S, next_b = (g + 1) * S;
-        auto body2 = [&](int c, float(&x)[16]) {
-          load_bias(c);
-          const float thr = top.v[kTopMax - 1];
-          uint32_t m = 0;
+        // bit i: expert col0 + 16c + i lies in a kept group
+        auto keep_mask = [&](int c) -> uint32_t {
+          if (G == 1) return 0xffffu;
+          const int e0 = col0 + c * 16;
+          if ((S % 16) == 0) return ((kept >> (e0 / S)) & 1u) ? 0xffffu : 0u;
+          uint32_t km = 0;
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int e = col0 + c * 16 + i;
-            if (e == next_b) {
-              ++g;
-              next_b += S;
-            }
-            const bool keep = G == 1 || ((kept >> g) & 1u);
-            // pass 1 (groups or softmax) left s in TMEM; otherwise x holds logits
-            const float sv = (G > 1 || softmax) ? x[i] : mr_sigmoid(x[i]);
-            const float cval = keep ? sv + bv[i] : (zero_fill ? 0.0f : -INFINITY);
-            x[i] = sv;
-            bv[i] = cval;
-            m |= (cval >= tau && cval > thr ? 1u : 0u) << i;
-          }
-          if (cnt + __popc(m) > kCandCap) flush();
-          // branch-free append in index order; non-candidates write the
-          // spare slot kCandCap
-          int p = cnt;
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const bool bit = (m >> i) & 1u;
-            const int slot = (bit ? p : kCandCap) * 32 * kWorkers + wt;
-            bufV[slot] = bv[i];
-            bufS[slot] = x[i];
-            bufI[slot] = col0 + c * 16 + i;
-            p += bit ? 1 : 0;
-          }
-          cnt = p;
+          for (int i = 0; i < 16; ++i) km |= ((kept >> ((e0 + i) / S)) & 1u) << i;
+          return km;
         };
-        for (int c = c_beg; c < c_end; c += 2) {
-          __syncwarp();  // the buffer flush diverges; tcgen05.ld is .aligned
-          const int c2 = c + 1 < c_end ? c + 1 : c;
-          tmem_ld16x2(tmem_base + lane_off + (uint32_t)(c * 16),
-                      tmem_base + lane_off + (uint32_t)(c2 * 16), v, v2);
-          body2(c, v);
-          if (c2 != c) body2(c2, v2);
+        // one chunk per iteration, and one more that flushes what is left
+        // (one copy of the body and of the flush in the code)
+#pragma unroll 1
+        for (int c = c_beg; c <= c_end; ++c) {
+          uint32_t m = 0;
+          if (c < c_end) {
+            __syncwarp();  // the buffer flush diverges; tcgen05.ld is .aligned
+            tmem_ld16(tmem_base + lane_off + (uint32_t)(c * 16), v);
+            load_bias(c);
+            const uint32_t km = keep_mask(c);
+            const float thr = top.v[kTopMax - 1];
+            uint32_t mlo = 0, mhi = 0;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              // pass 1 (groups or softmax) left s in TMEM; otherwise v holds logits
+              const float sv = (G > 1 || softmax) ? v[i] : mr_sigmoid(v[i]);
+              const float cval = ((km >> i) & 1u) ? sv + bv[i] : (zero_fill ? 0.0f : -INFINITY);
+              v[i] = sv;
+              bv[i] = cval;
+              const uint32_t bit = (cval >= tau && cval > thr ? 1u : 0u) << i;
+              if (i < 8) mlo |= bit; else mhi |= bit;
+            }
+            m = mlo | mhi;
+          }
+          if (c == c_end || cnt + __popc(m) > kCandCap) flush();
+          if (c < c_end) {
+            // branch-free append in index order; non-candidates write the
+            // spare slot kCandCap
+            int p = cnt;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const bool bit = (m >> i) & 1u;
+              const int slot = (bit ? p : kCandCap) * 32 * kWorkers + wt;
+              bufV[slot] = bv[i];
+              bufS[slot] = v[i];
+              bufI[slot] = col0 + c * 16 + i;
+              p += bit ? 1 : 0;
+            }
+            cnt = p;
+          }
         }
-        flush();
       }
 #pragma unroll
       for (int j = 0; j < kTopMax; ++j) {
