@@ -445,17 +445,26 @@ struct Top8 {
       for (int j = 0; j < kTopMax; ++j)
         if ((j & d) == 0) order(j, j + d);
   }
+  // Insert a candidate that beats the 8th entry.  Candidates arrive in index
+  // order, so an equal value already listed keeps its place ahead of it
+  // (lower index first): its slot is the count of listed values >= cv, and
+  // every slot below it shifts down by one -- all slots at once, no chain of
+  // compare-and-swap steps.
   __device__ __forceinline__ void push(float cv, int ci, float cs) {
-    v[kTopMax - 1] = cv;
-    i[kTopMax - 1] = ci;
-    s[kTopMax - 1] = cs;
+    int pos = 0;
+#pragma unroll
+    for (int j = 0; j < kTopMax; ++j) pos += v[j] >= cv ? 1 : 0;
 #pragma unroll
     for (int j = kTopMax - 1; j > 0; --j) {
-      if (v[j] > v[j - 1]) {
-        const float tv = v[j]; v[j] = v[j - 1]; v[j - 1] = tv;
-        const float ts = s[j]; s[j] = s[j - 1]; s[j - 1] = ts;
-        const int ti = i[j]; i[j] = i[j - 1]; i[j - 1] = ti;
-      }
+      const bool sh = j > pos, put = j == pos;
+      v[j] = sh ? v[j - 1] : (put ? cv : v[j]);
+      s[j] = sh ? s[j - 1] : (put ? cs : s[j]);
+      i[j] = sh ? i[j - 1] : (put ? ci : i[j]);
+    }
+    if (pos == 0) {
+      v[0] = cv;
+      s[0] = cs;
+      i[0] = ci;
     }
   }
 };
@@ -1020,7 +1029,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       // pass 1: s = sigmoid(L) (or softmax) back into TMEM; per-group top-2
       // of c = s + b
       uint32_t kept = 0xffffffffu;
-      if (G > 1 || softmax) {
+      // with one group, each chunk's top-2 goes to the candidate buffer
+      // (slots 2j, 2j + 1 of chunk c_beg + j) for the bound tau below
+      float* chunk_pairs = reinterpret_cast<float*>(smem + exchange_bytes(G));
+      {
         if (G > 1)
           for (int g = 0; g < G; ++g) {
             exA1[(h * G + g) * BM + row] = -INFINITY;
@@ -1046,10 +1058,9 @@ __global__ void __launch_bounds__(kThreads, 1)
               for (int i = 0; i < 16; ++i) v[i] = mr_sigmoid(v[i]);
             }
             tmem_st16(tmem_base + lane_off + (uint32_t)(c * 16), v);
-            if (G == 1) continue;
-            if (chunk_groups) {
+            if (G == 1 || chunk_groups) {
               const int gc = (col0 + c * 16) / S;
-              if (gc != g) {
+              if (G > 1 && gc != g) {
                 exA1[(h * G + g) * BM + row] = a1;
                 exA2[(h * G + g) * BM + row] = a2;
                 g = gc;
@@ -1072,6 +1083,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                   p2[j] = fmaxf(fminf(p1[j], p1[j + w]), fmaxf(p2[j], p2[j + w]));
                   p1[j] = hi;
                 }
+              if (G == 1) {
+                chunk_pairs[(2 * (c - c_beg)) * 32 * kWorkers + wt] = p1[0];
+                chunk_pairs[(2 * (c - c_beg) + 1) * 32 * kWorkers + wt] = p2[0];
+                continue;
+              }
               const float hi = fmaxf(a1, p1[0]);
               a2 = fmaxf(fminf(a1, p1[0]), fmaxf(a2, p2[0]));
               a1 = hi;
@@ -1107,6 +1123,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       // values are 2*topk_group distinct candidates, so when that is >= k
       // the k-th best of all candidates is >= the smallest of them.
       float tau = -INFINITY;
+      if (G == 1 && ok && c_beg < c_end) {
+        // One group: the ceil(k/2) chunks of this half with the largest
+        // maxima hold at least k distinct scores >= the smallest of their
+        // second-best values, so the half's -- and the token's -- k-th best
+        // is >= that value.
+        const int nc = c_end - c_beg, need = (P.k + 1) / 2;
+        if (nc >= need) {
+          float u1[8], u2[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            u1[j] = j < nc ? chunk_pairs[(2 * j) * 32 * kWorkers + wt] : -INFINITY;
+            u2[j] = j < nc ? chunk_pairs[(2 * j + 1) * 32 * kWorkers + wt] : -INFINITY;
+          }
+          float t = INFINITY;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            int rank = 0;
+#pragma unroll
+            for (int l = 0; l < 8; ++l) rank += (u1[l] > u1[j] || (u1[l] == u1[j] && l < j)) ? 1 : 0;
+            if (j < nc && rank < need) t = fminf(t, u2[j]);
+          }
+          tau = t;
+        }
+      }
       if (G > 1) {
         const bool gmax = (P.flags & MR_GROUP_MAX) != 0;
         if (G <= 8)
@@ -1162,8 +1202,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t mlo = 0, mhi = 0;
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-              // pass 1 (groups or softmax) left s in TMEM; otherwise v holds logits
-              const float sv = (G > 1 || softmax) ? v[i] : mr_sigmoid(v[i]);
+              const float sv = v[i];  // pass 1 left the scores in TMEM
               const float cval = ((km >> i) & 1u) ? sv + bv[i] : (zero_fill ? 0.0f : -INFINITY);
               v[i] = sv;
               bv[i] = cval;
