@@ -310,14 +310,20 @@ def test_router_splitk_routing_shapes(w):
 
 def test_router_workspace_for_large_batches_holds_w_planes():
     # three bf16 planes of W (which also covers W's fp32 tf32-residuals)
-    assert mr.mr_router_workspace_size(4096, 7168, 256) == 3 * 2 * 7168 * 256
+    # and, for a K-split batch, room after them for the partial sums the
+    # routing kernel adds (4096 tokens: 4 slices)
+    planes = 3 * 2 * 7168 * 256
+    assert mr.mr_router_workspace_size(16384, 7168, 256) == planes
+    assert mr.mr_router_workspace_size(4096, 7168, 256) >= planes + 4 * 4096 * 256 * 4
 
 
 @pytest.mark.parametrize("w", [SMALL[1], SMALL[2].replace(name="k2_like_T300", T=300),
                                wl.V3_PREFILL], ids=lambda w: w.name)
 def test_router_with_precomputed_residuals_is_identical(w):
     """Above 256 tokens a workspace makes the fused path read W's tf32
-    residuals precomputed (one extra launch); results are bit-identical."""
+    residuals precomputed (one extra launch; a K-split batch also hands its
+    partial sums to the routing kernel, one more); results are bit-identical
+    (the slices are added in the same order either way)."""
     assert w.T > 256  # (smaller batches take the split-K path instead)
     d = router_inputs(w)
     args = (to_dev(d["x_f32"]), to_dev(d["W"]), to_dev(d["b"]), w.n_group, w.topk_group, w.k,
@@ -326,7 +332,7 @@ def test_router_with_precomputed_residuals_is_identical(w):
                      device="cuda")
     l0 = mr.mr_launch_count()
     a = mr.mr_router_forward_ex(*args, workspace=ws)
-    assert mr.mr_launch_count() - l0 == 2
+    assert mr.mr_launch_count() - l0 in (2, 3)
     b = mr.mr_router_forward_ex(*args)
     assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
     assert mr.mr_get_error() == mr.MR_OK
@@ -721,3 +727,94 @@ def test_router_ksplit_is_deterministic_and_matches_one_cta():
         assert np.array_equal(u, v)
     ref = oracle_router(w, np.arange(w.T))
     compare_router(a[0], a[1], ref, a[2])
+
+
+# ---- K-split batches: the routing kernel and the GEMM's epilogue ----
+# With a workspace of mr_router_workspace_size bytes, the CTAs of a K-split
+# tile write their partial sums to the workspace and a routing kernel of P
+# lanes per token adds them and routes; MR_ROUTE_KERNEL=0 keeps the exchange
+# through distributed shared memory and the routing in the GEMM's epilogue,
+# MR_ROUTE_LANES pins P, MR_TC_CLUSTER=K2 / K4 forces the K split.
+
+def _launches(fn):
+    n0 = mr.mr_launch_count()
+    out = fn()
+    torch.cuda.synchronize()
+    return out, mr.mr_launch_count() - n0
+
+
+@pytest.mark.parametrize("route", ["kernel", "epilogue"])
+def test_router_routing_kernel_launches(route, monkeypatch):
+    """bf16x3 fused, K split: W split + GEMM + routing kernel (3 launches);
+    the epilogue routing: 2."""
+    monkeypatch.setenv("MR_TC_CLUSTER", "K2")
+    if route == "epilogue":
+        monkeypatch.setenv("MR_ROUTE_KERNEL", "0")
+    w = SMALL[1]
+    (idx, wt, lg), n = _launches(lambda: _run_bf16x3(w))
+    assert n == (3 if route == "kernel" else 2)
+    compare_router(idx, wt, oracle_router(w, np.arange(w.T)), lg)
+
+
+# shapes of the small cases with more than 256 tokens (smaller batches take
+# split-K): groups of 8, 16 and 32 experts, 2 or 4 lanes per group, no groups,
+# 64 to 512 experts, the zero fill, and N = 320 in groups of 32 split over
+# two CTAs (160 experts each), which no lane layout fits (epilogue routing)
+ROUTE_W = [SMALL[1], SMALL[3].replace(name="zero_mask_N128_T333", T=333, io_dtype="bf16"),
+           SMALL[4].replace(name="no_bias_N64_G8_T301", T=301, io_dtype="bf16"),
+           SMALL[7].replace(name="N512_G16_T290", T=290, io_dtype="bf16"),
+           BF16X3[3].replace(name="N320_G10_T280", T=280), BF16X3[5],
+           wl.K2_PREFILL.replace(name="k2_T300", T=300),
+           wl.V3_PREFILL.replace(name="v3_T777", T=777)]
+
+
+@pytest.mark.parametrize("lanes", ["8", "16", "32"])
+@pytest.mark.parametrize("w", ROUTE_W, ids=lambda w: w.name)
+def test_router_routing_kernel_every_lane_layout(w, lanes, monkeypatch):
+    """Every lane layout the shape allows (8, 16 or 32 lanes per token) gives
+    the oracle's routing; a layout that does not fit, or a shape without a K
+    split (more than 256 experts: two CTAs split the experts), is routed by
+    the epilogue (2 launches) with the same result."""
+    monkeypatch.setenv("MR_TC_CLUSTER", "K2")
+    monkeypatch.setenv("MR_ROUTE_LANES", lanes)
+    (idx, wt, lg), n = _launches(lambda: _run_bf16x3(w))
+    assert n in (2, 3)
+    compare_router(idx, wt, oracle_router(w, np.arange(w.T)), lg)
+
+
+@pytest.mark.parametrize("var", sorted(VARIANTS))
+@pytest.mark.parametrize("route", ["kernel", "epilogue"])
+@pytest.mark.parametrize("w", VAR_W, ids=[w.name for w in VAR_W])
+def test_router_scoring_variants_both_routings(w, route, var, monkeypatch):
+    monkeypatch.setenv("MR_TC_CLUSTER", "K2")
+    if route == "epilogue":
+        monkeypatch.setenv("MR_ROUTE_KERNEL", "0")
+    flags, okw = VARIANTS[var]
+    no_bias = var == "v32_softmax_nobias"
+    idx, wt, lg = _variant_run(w, flags, "bf16", mr.MR_PREC_BF16X3, no_bias)
+    tie_frac = 0.05 if okw.get("score") == "softmax" else 0.01
+    compare_router(idx, wt, _variant_ref(w, np.arange(w.T), okw, no_bias), lg,
+                   allow_tie_frac=tie_frac)
+
+
+@pytest.mark.parametrize("ks", ["1", "K2", "K4"])
+@pytest.mark.parametrize("route", ["kernel", "epilogue"])
+def test_router_ksplit_both_routings(ks, route, monkeypatch):
+    """K-split partial sums meet either in the routing kernel (slices added in
+    order from the workspace) or through distributed shared memory."""
+    monkeypatch.setenv("MR_TC_CLUSTER", ks)
+    if route == "epilogue":
+        monkeypatch.setenv("MR_ROUTE_KERNEL", "0")
+    for w in (SMALL[1], BF16X3[5]):
+        idx, wt, lg = _run_bf16x3(w)
+        compare_router(idx, wt, oracle_router(w, np.arange(w.T)), lg)
+        a = _run_bf16x3(w)
+        assert np.array_equal(a[0], idx) and np.array_equal(a[1], wt)
+
+
+@pytest.mark.parametrize("w", [wl.V3_PREFILL, wl.K2_PREFILL, wl.V3_FULL], ids=lambda w: w.name)
+def test_router_epilogue_routing_full_size_every_token(w, monkeypatch):
+    """The GEMM's own epilogue (no routing kernel) at full size, every token."""
+    monkeypatch.setenv("MR_ROUTE_KERNEL", "0")
+    idx, wt, logits = _run_bf16x3(w)
+    compare_router(idx, wt, oracle_router(w, np.arange(w.T)), logits)

@@ -19,6 +19,7 @@
 #include "router_ffma.cuh"
 #include "router_splitk.cuh"
 #include "router_tc.cuh"
+#include "route.cuh"
 #include "combine.cuh"
 #include "gather.cuh"
 
@@ -351,6 +352,41 @@ int launch_splitk(const void* x, bool x_bf16, const float* W, const float* bias,
   return MR_ERR_UNSUPPORTED;
 }
 
+// Routing kernel after the tensor-core router (part = its logits or K-split
+// partial sums, P lanes per token): a programmatic dependent of the router.
+template <int EL>
+int launch_route_el(const mr::rt::Params& rp, cudaStream_t st) {
+  cudaLaunchConfig_t cfg = {};
+  const int tpb = mr::rt::kThreads / rp.P;
+  cfg.gridDim = dim3((unsigned)((rp.T + tpb - 1) / tpb));
+  cfg.blockDim = dim3(mr::rt::kThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, mr::rt::route_kernel<EL>, rp);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  if (e != cudaSuccess) {
+    (void)cudaGetLastError();
+    return MR_ERR_CUDA;
+  }
+  return MR_OK;
+}
+
+int launch_route(const mr::rt::Params& rp, cudaStream_t st) {
+  switch (rp.N / rp.P) {
+    case 8: return launch_route_el<8>(rp, st);
+    case 12: return launch_route_el<12>(rp, st);
+    case 16: return launch_route_el<16>(rp, st);
+    case 24: return launch_route_el<24>(rp, st);
+    case 32: return launch_route_el<32>(rp, st);
+    default: return MR_ERR_UNSUPPORTED;
+  }
+}
+
 // How CTAs share a 128-token tile of the fused router:
 //  - ks = 2 or 4 (N_r <= 256): a cluster of ks CTAs splits the K loop of the
 //    tile (partial sums meet through distributed shared memory), taken while
@@ -396,6 +432,19 @@ TcShape tc_shape(int T, int N_r, int sms, bool bf16x3, int num_kc) {
 size_t wlo_bytes(int d, int N_r) { return (size_t)N_r * (size_t)d * sizeof(float); }
 // W's three bf16 planes [3, N_r, d] for bf16 activations.
 size_t planes_bytes(int d, int N_r) { return 3 * (size_t)N_r * (size_t)d * 2; }
+// The fused router's logits for the routing kernel, [ks][T][N_r] fp32, placed
+// after the planes (or W's residuals, which are smaller) in the workspace.
+size_t route_part_bytes(int T, int N_r, int ks) { return (size_t)ks * T * N_r * sizeof(float); }
+size_t route_part_offset(int d, int N_r) { return (planes_bytes(d, N_r) + 255) / 256 * 256; }
+float* route_part(void* ws, size_t ws_bytes, int d, int N_r) {
+  const size_t off = route_part_offset(d, N_r);
+  return ws && aligned16(ws) && ws_bytes > off
+             ? reinterpret_cast<float*>(static_cast<char*>(ws) + off)
+             : nullptr;
+}
+size_t route_part_cap(void* ws, size_t ws_bytes, int d, int N_r) {
+  return route_part(ws, ws_bytes, d, N_r) ? ws_bytes - route_part_offset(d, N_r) : 0;
+}
 
 // x fp32 with tf32 arithmetic (use3x: 3xTF32), or x bf16 with W as three
 // bf16 planes (bf16x3, planes written into `ws` here), or x bf16 with W
@@ -403,7 +452,8 @@ size_t planes_bytes(int d, int N_r) { return 3 * (size_t)N_r * (size_t)d * 2; }
 int launch_tc(const void* x, const float* W, const float* bias, int T, int d, int N_r,
               int n_group, int topk_group, int k, float route_scale, int mask_mode, int flags,
               bool use3x, bool bf16x3, int32_t* idx_out, float* w_out, float* logits_out,
-              float* wlo, void* ws, int sms, cudaStream_t st, const void* wbf16 = nullptr) {
+              float* wlo, void* ws, int sms, cudaStream_t st, const void* wbf16 = nullptr,
+              float* part = nullptr, size_t part_cap = 0) {
   const int nplanes = wbf16 ? 1 : 3;
   const int num_kc = (d + mr::tc::BK - 1) / mr::tc::BK;
   TcShape shp = tc_shape(T, N_r, sms, bf16x3, num_kc);
@@ -473,6 +523,23 @@ int launch_tc(const void* x, const float* W, const float* bias, int T, int d, in
   P.idx_out = idx_out;
   P.w_out = w_out;
   P.logits_out = logits_out;
+  // K-split batches: when the workspace holds the ks partial sums and the
+  // shape fits the routing kernel's layout, the CTAs write their partials and
+  // the routing kernel adds them and routes (instead of the exchange through
+  // distributed shared memory and an epilogue in which every CTA of a cluster
+  // routes all 128 tokens to write a quarter).  One CTA per tile keeps the
+  // routing in its epilogue, which measured faster than the routing kernel
+  // there.  MR_ROUTE_KERNEL=0 keeps the epilogue for K-split batches too,
+  // MR_ROUTE_LANES=8, 16 or 32 pins the lanes per token (both used by the
+  // tests).
+  int lanes = 0;
+  if (part && shp.ks > 1 && part_cap >= route_part_bytes(T, N_r, shp.ks)) {
+    const char* pin = getenv("MR_ROUTE_LANES");
+    lanes = mr::rt::lanes_per_token(T, N_r, n_group, k, sms, pin ? atoi(pin) : 0);
+    if (const char* env = getenv("MR_ROUTE_KERNEL"))
+      if (env[0] == '0') lanes = 0;
+  }
+  P.part = lanes ? part : nullptr;
   const size_t smem = plan.total + 1024;
   const bool sm = (flags & MR_SCORE_SOFTMAX) != 0;
   using mr::tc::router_tc_kernel;
@@ -515,7 +582,25 @@ int launch_tc(const void* x, const float* W, const float* bias, int T, int d, in
     g_launches.fetch_add(1, std::memory_order_relaxed);
     return MR_ERR_CUDA;
   }
-  return launch_status();
+  if (launch_status() != MR_OK) return MR_ERR_CUDA;
+  if (!lanes) return MR_OK;
+  mr::rt::Params rp;
+  rp.part = part;
+  rp.KS = shp.ks;
+  rp.T = T;
+  rp.N = N_r;
+  rp.P = lanes;
+  rp.n_group = n_group;
+  rp.topk_group = topk_group;
+  rp.k = k;
+  rp.mask_mode = mask_mode;
+  rp.flags = flags;
+  rp.route_scale = route_scale;
+  rp.bias = bias;
+  rp.idx_out = idx_out;
+  rp.w_out = w_out;
+  rp.logits_out = logits_out;
+  return launch_route(rp, st);
 }
 
 // ---- the plain router's split-K partials --------------------------------------
@@ -649,6 +734,13 @@ const char* mr_status_string(int status) {
 size_t mr_router_workspace_size(int T, int d, int N_r) {
   if (T <= 0 || d <= 0 || N_r <= 0 || N_r > 512) return 0;
   size_t need = planes_bytes(d, N_r);  // >= W residuals (fp32 x, fused path)
+  {
+    // then, for a K-split batch, the partial sums for the routing kernel
+    int sms = 0, cc = 0;
+    if (!device_info(&sms, &cc)) return 0;
+    const TcShape shp = tc_shape(T, N_r, sms, true, (d + mr::tc::BK - 1) / mr::tc::BK);
+    if (shp.ks > 1) need = route_part_offset(d, N_r) + route_part_bytes(T, N_r, shp.ks);
+  }
   if (splitk_applies(T, N_r)) {
     int sms = 0, cc = 0;
     if (!device_info(&sms, &cc)) return 0;
@@ -694,7 +786,9 @@ int mr_router_forward_ex2(const void* x, int x_dtype, const float* W, const floa
         workspace_bytes < planes_bytes(d, N_r))
       return MR_ERR_UNSUPPORTED;
     return launch_tc(x, W, bias, T, d, N_r, n_group, topk_group, k, route_scale, mask_mode, flags,
-                     true, true, idx_out, w_out, logits_out, nullptr, workspace, sms, s);
+                     true, true, idx_out, w_out, logits_out, nullptr, workspace, sms, s, nullptr,
+                     route_part(workspace, workspace_bytes, d, N_r),
+                     route_part_cap(workspace, workspace_bytes, d, N_r));
   }
   if (cc != 10 || !tc_shape_ok(x, x_dtype, W, d, N_r)) return MR_ERR_UNSUPPORTED;
   float* wlo = (workspace && aligned16(workspace) && workspace_bytes >= wlo_bytes(d, N_r))
@@ -702,7 +796,8 @@ int mr_router_forward_ex2(const void* x, int x_dtype, const float* W, const floa
                    : nullptr;
   return launch_tc(x, W, bias, T, d, N_r, n_group, topk_group, k, route_scale, mask_mode, flags,
                    precision == MR_PREC_3XTF32, false, idx_out, w_out, logits_out, wlo, nullptr,
-                   sms, s);
+                   sms, s, nullptr, route_part(workspace, workspace_bytes, d, N_r),
+                   route_part_cap(workspace, workspace_bytes, d, N_r));
 }
 
 int mr_router_forward_ex(const void* x, int x_dtype, const float* W, const float* bias, int T,

@@ -85,6 +85,11 @@ struct Params {
   // and only that CTA writes the quarter's tokens.
   int ksplit;
   int flags;  // MR_SCORE_SOFTMAX | MR_GROUP_MAX | MR_NORM_NO_EPS
+  // part (K-split instantiation only): each CTA's fp32 partial sums over its
+  // K chunks go to part[rank][token][expert] and the routing kernel that
+  // follows adds the slices in rank order and routes the tokens; no exchange
+  // and no epilogue run here
+  float* part;
   float route_scale;
   const float* bias;
   int32_t* idx_out;
@@ -618,6 +623,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   // preceding kernel (W's planes or residuals); no global input is read
   // before that grid has completed.
   asm volatile("griddepcontrol.wait;" ::: "memory");
+  // with part, the routing kernel is this grid's programmatic dependent: it
+  // may be scheduled now and waits for this grid's completion itself
+  if (KS && P.part) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   for (int e = threadIdx.x; e < NL; e += kThreads)
     bias_s[e] = P.bias ? P.bias[col0 + e] : 0.0f;
   tc_fence_before();
@@ -849,6 +857,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     while (ok && promoted < J) promote(promoted);
     ok = __all_sync(0xffffffffu, ok);
+
+    if (KS && P.part) {
+      // the fp32 sums of this CTA's rows over its K chunks to
+      // part[rank][token][expert]
+      const long tok = (long)m0 + q * 32 + lane;
+      if (ok && tok < P.T) {
+        float* dst = P.part + ((long)crank * P.T + tok) * P.N;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int c = h + 2 * i;
+          if (c < n16) {
+            float4* d4 = reinterpret_cast<float4*>(dst + c * 16);
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj)
+              d4[jj] = make_float4(acc[i][4 * jj], acc[i][4 * jj + 1], acc[i][4 * jj + 2],
+                                   acc[i][4 * jj + 3]);
+          }
+        }
+      }
+    } else {
 
     // K-split: the ksplit CTAs of the cluster hold partial sums over their K
     // chunks.  Each writes its partials to its (now idle) ring, [BM][NL + 4]
@@ -1278,6 +1306,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (cs > 1) cluster_sync_all();  // #3: the peer's lists have been read
     }
+    }  // !P.part
   }
 
   // Threads that take no part in the routing epilogue still join its cluster
@@ -1288,7 +1317,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < n_sync; ++i) cluster_sync_all();
   }
   // ... and the two barriers of the K-split exchange
-  if (KSP > 1 && warp < 2) {
+  if (KSP > 1 && !(KS && P.part) && warp < 2) {
     cluster_sync_all();
     cluster_sync_all();
   }
