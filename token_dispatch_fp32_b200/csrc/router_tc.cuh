@@ -227,6 +227,20 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster) {
 __device__ __forceinline__ void fence_proxy_async() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
+// Bulk copy of `bytes` (a multiple of 16, both addresses 16-byte aligned)
+// from this CTA's shared memory to global memory, in the thread's bulk group.
+__device__ __forceinline__ void bulk_store(void* gdst, uint32_t ssrc, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst), "r"(ssrc),
+               "r"(bytes)
+               : "memory");
+}
+// Commit the thread's bulk stores and wait until they have completed (their
+// writes performed, not only their shared-memory reads), so the grid's end
+// orders them before a dependent grid's reads.
+__device__ __forceinline__ void bulk_store_commit_and_wait() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
 __device__ __forceinline__ void tc_fence_before() {
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
 }
@@ -860,21 +874,30 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (KS && P.part) {
       // the fp32 sums of this CTA's rows over its K chunks to
-      // part[rank][token][expert]
-      const long tok = (long)m0 + q * 32 + lane;
-      if (ok && tok < P.T) {
-        float* dst = P.part + ((long)crank * P.T + tok) * P.N;
+      // part[rank][token][expert]: staged row by row in the idle ring
+      // ([BM][NL + 4], the pad keeps a warp's rows on distinct banks), then
+      // one bulk copy per row (a thread's own row stores would scatter every
+      // warp store over 32 rows)
+      const int row = q * 32 + lane;
+      const int NLp = NL + 4;
+      float* xrow = reinterpret_cast<float*>(smem) + row * NLp;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int c = h + 2 * i;
-          if (c < n16) {
-            float4* d4 = reinterpret_cast<float4*>(dst + c * 16);
+      for (int i = 0; i < 8; ++i) {
+        const int c = h + 2 * i;
+        if (c < n16) {
+          float4* d4 = reinterpret_cast<float4*>(xrow + c * 16);
 #pragma unroll
-            for (int jj = 0; jj < 4; ++jj)
-              d4[jj] = make_float4(acc[i][4 * jj], acc[i][4 * jj + 1], acc[i][4 * jj + 2],
-                                   acc[i][4 * jj + 3]);
-          }
+          for (int jj = 0; jj < 4; ++jj)
+            d4[jj] = make_float4(acc[i][4 * jj], acc[i][4 * jj + 1], acc[i][4 * jj + 2],
+                                 acc[i][4 * jj + 3]);
         }
+      }
+      fence_proxy_async();  // the generic writes, visible to the bulk copies
+      workers_sync();
+      if (ok && wt < BM && (long)m0 + wt < P.T) {
+        bulk_store(P.part + ((long)crank * P.T + m0 + wt) * P.N,
+                   smem_u32(reinterpret_cast<float*>(smem) + wt * NLp), (uint32_t)NL * 4);
+        bulk_store_commit_and_wait();
       }
     } else {
 
