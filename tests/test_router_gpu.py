@@ -729,11 +729,12 @@ def test_router_ksplit_is_deterministic_and_matches_one_cta():
     compare_router(a[0], a[1], ref, a[2])
 
 
-# ---- K-split batches: the routing kernel and the GEMM's epilogue ----
+# ---- routing after the GEMM: the routing kernel and the GEMM's epilogue ----
 # With a workspace of mr_router_workspace_size bytes, the CTAs of a K-split
-# tile write their partial sums to the workspace and a routing kernel of P
-# lanes per token adds them and routes; MR_ROUTE_KERNEL=0 keeps the exchange
-# through distributed shared memory and the routing in the GEMM's epilogue,
+# tile (or of an expert split) write their partial sums (their logits) to the
+# workspace and a routing kernel of P lanes per token adds them and routes;
+# MR_ROUTE_KERNEL=0 keeps the exchanges through distributed shared memory and
+# the routing in the GEMM's epilogue (=1 routes every shape after the GEMM),
 # MR_ROUTE_LANES pins P, MR_TC_CLUSTER=K2 / K4 forces the K split.
 
 def _launches(fn):
@@ -772,9 +773,9 @@ ROUTE_W = [SMALL[1], SMALL[3].replace(name="zero_mask_N128_T333", T=333, io_dtyp
 @pytest.mark.parametrize("w", ROUTE_W, ids=lambda w: w.name)
 def test_router_routing_kernel_every_lane_layout(w, lanes, monkeypatch):
     """Every lane layout the shape allows (8, 16 or 32 lanes per token) gives
-    the oracle's routing; a layout that does not fit, or a shape without a K
-    split (more than 256 experts: two CTAs split the experts), is routed by
-    the epilogue (2 launches) with the same result."""
+    the oracle's routing, after a K split or (more than 256 experts) two CTAs
+    splitting the experts; a layout that does not fit is routed by the
+    epilogue (2 launches) with the same result."""
     monkeypatch.setenv("MR_TC_CLUSTER", "K2")
     monkeypatch.setenv("MR_ROUTE_LANES", lanes)
     (idx, wt, lg), n = _launches(lambda: _run_bf16x3(w))
@@ -812,9 +813,11 @@ def test_router_ksplit_both_routings(ks, route, monkeypatch):
         assert np.array_equal(a[0], idx) and np.array_equal(a[1], wt)
 
 
+@pytest.mark.parametrize("route", ["0", "1"], ids=["epilogue", "routing_kernel"])
 @pytest.mark.parametrize("w", [wl.V3_PREFILL, wl.K2_PREFILL, wl.V3_FULL], ids=lambda w: w.name)
-def test_router_epilogue_routing_full_size_every_token(w, monkeypatch):
-    """The GEMM's own epilogue (no routing kernel) at full size, every token."""
-    monkeypatch.setenv("MR_ROUTE_KERNEL", "0")
+def test_router_both_routings_full_size_every_token(w, route, monkeypatch):
+    """Each routing for every full-size batch (whichever the default takes),
+    every token."""
+    monkeypatch.setenv("MR_ROUTE_KERNEL", route)
     idx, wt, logits = _run_bf16x3(w)
     compare_router(idx, wt, oracle_router(w, np.arange(w.T)), logits)

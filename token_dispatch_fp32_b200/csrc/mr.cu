@@ -436,6 +436,20 @@ size_t planes_bytes(int d, int N_r) { return 3 * (size_t)N_r * (size_t)d * 2; }
 // after the planes (or W's residuals, which are smaller) in the workspace.
 size_t route_part_bytes(int T, int N_r, int ks) { return (size_t)ks * T * N_r * sizeof(float); }
 size_t route_part_offset(int d, int N_r) { return (planes_bytes(d, N_r) + 255) / 256 * 256; }
+// Whether the routing kernel routes after the GEMM (when the workspace and
+// the shape allow): for K-split batches and for two CTAs splitting the
+// experts, where it measured faster than the epilogue (DeepSeek-V3 prefill
+// 85 -> 64 us, Kimi K2 prefill 150.5 -> 138 us); one CTA per tile keeps its
+// epilogue (the full batch: 161 us against 165-169 us with the routing
+// kernel).  MR_ROUTE_KERNEL=0 never, =1 for every shape (the tests and
+// measurements pin both).
+bool route_after_gemm(const TcShape& shp) {
+  if (const char* env = getenv("MR_ROUTE_KERNEL")) {
+    if (env[0] == '0') return false;
+    if (env[0] == '1') return true;
+  }
+  return shp.ks > 1 || shp.CS > 1;
+}
 float* route_part(void* ws, size_t ws_bytes, int d, int N_r) {
   const size_t off = route_part_offset(d, N_r);
   return ws && aligned16(ws) && ws_bytes > off
@@ -523,27 +537,27 @@ int launch_tc(const void* x, const float* W, const float* bias, int T, int d, in
   P.idx_out = idx_out;
   P.w_out = w_out;
   P.logits_out = logits_out;
-  // K-split batches: when the workspace holds the ks partial sums and the
-  // shape fits the routing kernel's layout, the CTAs write their partials and
-  // the routing kernel adds them and routes (instead of the exchange through
-  // distributed shared memory and an epilogue in which every CTA of a cluster
-  // routes all 128 tokens to write a quarter).  One CTA per tile keeps the
-  // routing in its epilogue, which measured faster than the routing kernel
-  // there.  MR_ROUTE_KERNEL=0 keeps the epilogue for K-split batches too,
-  // MR_ROUTE_LANES=8, 16 or 32 pins the lanes per token (both used by the
-  // tests).
+  // After the GEMM (route_after_gemm): when the workspace holds the logits
+  // (the ks partial sums of a K split) and the shape fits the routing
+  // kernel's layout, the CTAs write them and the routing kernel adds the
+  // slices and routes (instead of the exchanges through distributed shared
+  // memory and the epilogue); MR_ROUTE_LANES=8, 16 or 32 pins the lanes per
+  // token (the tests use it).
   int lanes = 0;
-  if (part && shp.ks > 1 && part_cap >= route_part_bytes(T, N_r, shp.ks)) {
+  // (the rows are staged in the ring: [128][NL + 4] fp32 must fit in it)
+  if (part && !pair && part_cap >= route_part_bytes(T, N_r, shp.ks) &&
+      (size_t)mr::tc::BM * (NL + 4) * 4 <= (size_t)plan.stages * plan.stage_bytes &&
+      route_after_gemm(shp)) {
     const char* pin = getenv("MR_ROUTE_LANES");
     lanes = mr::rt::lanes_per_token(T, N_r, n_group, k, sms, pin ? atoi(pin) : 0);
-    if (const char* env = getenv("MR_ROUTE_KERNEL"))
-      if (env[0] == '0') lanes = 0;
   }
   P.part = lanes ? part : nullptr;
   const size_t smem = plan.total + 1024;
   const bool sm = (flags & MR_SCORE_SOFTMAX) != 0;
   using mr::tc::router_tc_kernel;
-  const bool ksk = shp.ks > 1;  // the K-split instantiation (never with a pair)
+  // the K-split instantiation (never with a pair) also writes the logits for
+  // the routing kernel
+  const bool ksk = shp.ks > 1 || lanes > 0;
   auto kern =
       nplanes == 1
           ? (pair ? (sm ? router_tc_kernel<true, true, 1> : router_tc_kernel<true, false, 1>)
@@ -739,7 +753,8 @@ size_t mr_router_workspace_size(int T, int d, int N_r) {
     int sms = 0, cc = 0;
     if (!device_info(&sms, &cc)) return 0;
     const TcShape shp = tc_shape(T, N_r, sms, true, (d + mr::tc::BK - 1) / mr::tc::BK);
-    if (shp.ks > 1) need = route_part_offset(d, N_r) + route_part_bytes(T, N_r, shp.ks);
+    if (route_after_gemm(shp))
+      need = route_part_offset(d, N_r) + route_part_bytes(T, N_r, shp.ks);
   }
   if (splitk_applies(T, N_r)) {
     int sms = 0, cc = 0;

@@ -229,14 +229,15 @@ __global__ void __launch_bounds__(kThreads)
 }
 
 // Lanes per token for a batch of T tokens and N experts in groups of N/G:
-// 0 when the layout does not fit (the GEMM's epilogue routes instead).
-// Prefers fewer lanes per token as long as the batch has enough of them to
-// fill the SMs (about 24 warps per SM); pin > 0 asks for that many lanes (0
-// when they do not fit).
+// the most lanes whose layout fits (32, else 16, else 8 -- measured fastest
+// on the DeepSeek-V3 and Kimi K2 prefill batches), 0 when none does (the
+// GEMM's epilogue routes instead); pin > 0 asks for that many lanes (0 when
+// they do not fit).
 inline int lanes_per_token(long T, int N, int G, int k, int sms, int pin = 0) {
+  (void)T;
+  (void)sms;
   if (N > kMaxN || k > kTop) return 0;
-  const int cand[3] = {8, 16, 32};
-  int best = 0;
+  const int cand[3] = {32, 16, 8};
   for (int ci = 0; ci < 3; ++ci) {
     const int P = cand[ci];
     if (pin > 0 && P != pin) continue;
@@ -249,10 +250,9 @@ inline int lanes_per_token(long T, int N, int G, int k, int sms, int pin = 0) {
       const int LG = S / EL;
       if (LG & (LG - 1)) continue;  // a power of two: groups align with shuffle trees
     }
-    best = P;
-    if (T * P >= (long)sms * 32 * 24) break;
+    return P;
   }
-  return best;
+  return 0;
 }
 
 }  // namespace rt

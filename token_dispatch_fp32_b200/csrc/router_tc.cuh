@@ -85,10 +85,11 @@ struct Params {
   // and only that CTA writes the quarter's tokens.
   int ksplit;
   int flags;  // MR_SCORE_SOFTMAX | MR_GROUP_MAX | MR_NORM_NO_EPS
-  // part (K-split instantiation only): each CTA's fp32 partial sums over its
-  // K chunks go to part[rank][token][expert] and the routing kernel that
-  // follows adds the slices in rank order and routes the tokens; no exchange
-  // and no epilogue run here
+  // part (the KS instantiation only): each CTA's fp32 sums over its K chunks
+  // and expert columns go to part[slice][token][col0 + column], slice = its
+  // K-split rank (0 without a K split), and the routing kernel that follows
+  // adds the slices in order and routes the tokens; no exchange and no
+  // epilogue run here
   float* part;
   float route_scale;
   const float* bias;
@@ -895,7 +896,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_proxy_async();  // the generic writes, visible to the bulk copies
       workers_sync();
       if (ok && wt < BM && (long)m0 + wt < P.T) {
-        bulk_store(P.part + ((long)crank * P.T + m0 + wt) * P.N,
+        const long slice = KSP > 1 ? (long)crank : 0;
+        bulk_store(P.part + (slice * P.T + m0 + wt) * P.N + col0,
                    smem_u32(reinterpret_cast<float*>(smem) + wt * NLp), (uint32_t)NL * 4);
         bulk_store_commit_and_wait();
       }
@@ -1335,7 +1337,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // Threads that take no part in the routing epilogue still join its cluster
   // barriers (three; five with softmax scores), so a cluster always completes
   // them.
-  if (P.CS > 1 && warp < 2) {
+  if (P.CS > 1 && !(KS && P.part) && warp < 2) {
     const int n_sync = SOFTMAX ? 5 : 3;
     for (int i = 0; i < n_sync; ++i) cluster_sync_all();
   }
