@@ -327,8 +327,8 @@ int mr_dispatch(const int32_t *idx, int T, int k, int N_r, int32_t *counts,
  * the process exits.  The first call on a device looks up the array's device
  * address with that device current (cudaGetSymbolAddress) and keeps it; a
  * lookup that fails returns MR_ERR_CUDA and is tried again by the next call.
- * Make that first call before capturing a stream into a CUDA graph.  The entry point itself
- * calls no cudaMalloc, cudaFree or other allocating routine.  All calls on a
+ * The entry point itself calls no cudaMalloc, cudaFree or other allocating
+ * routine.  All calls on a
  * device share the one array, and it keeps whatever the last call left in
  * it: nothing in it needs to start at zero (each call rewrites every entry it
  * later reads), but calls that may overlap on the GPU -- on different streams
