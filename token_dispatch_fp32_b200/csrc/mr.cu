@@ -472,17 +472,16 @@ int launch_tc(const void* x, const float* W, const float* bias, int T, int d, in
   const int num_kc = (d + mr::tc::BK - 1) / mr::tc::BK;
   TcShape shp = tc_shape(T, N_r, sms, bf16x3, num_kc);
   auto fits = [&](const TcShape& t) {
-    const mr::tc::Plan p = mr::tc::make_plan(N_r / t.CS, bf16x3, t.pair, nplanes);
-    const uint32_t ring = p.stages * p.stage_bytes;
+    const mr::tc::Plan p = mr::tc::make_plan(N_r / t.CS, bf16x3, t.pair, nplanes, n_group);
     const uint32_t xk = t.ks > 1 ? (uint32_t)mr::tc::BM * (N_r + 4) * 4 : 0;  // K-split partials
-    return p.stages >= 2 && mr::tc::epilogue_smem_bytes(n_group) <= ring && xk <= ring;
+    return p.stages >= 2 && xk <= p.bar_off;
   };
   if (!fits(shp) && (shp.pair || shp.ks > 1)) shp = {1, false, 1};  // a pair's ring is half
   if (!fits(shp)) return MR_ERR_UNSUPPORTED;
   const int CS = shp.CS;
   const bool pair = shp.pair;
   const int NL = N_r / CS;
-  const mr::tc::Plan plan = mr::tc::make_plan(NL, bf16x3, pair, nplanes);
+  const mr::tc::Plan plan = mr::tc::make_plan(NL, bf16x3, pair, nplanes, n_group);
   CUtensorMap mx, mw, mwlo;
   const bool use_wlo = !bf16x3 && use3x && wlo != nullptr;
   if (bf16x3) {
@@ -546,7 +545,7 @@ int launch_tc(const void* x, const float* W, const float* bias, int T, int d, in
   int lanes = 0;
   // (the rows are staged in the ring: [128][NL + 4] fp32 must fit in it)
   if (part && !pair && part_cap >= route_part_bytes(T, N_r, shp.ks) &&
-      (size_t)mr::tc::BM * (NL + 4) * 4 <= (size_t)plan.stages * plan.stage_bytes &&
+      (size_t)mr::tc::BM * (NL + 4) * 4 <= (size_t)plan.bar_off &&
       route_after_gemm(shp)) {
     const char* pin = getenv("MR_ROUTE_LANES");
     lanes = mr::rt::lanes_per_token(T, N_r, n_group, k, sms, pin ? atoi(pin) : 0);

@@ -107,40 +107,51 @@ struct Plan {
 
 __host__ __device__ inline uint32_t align_up(uint32_t v, uint32_t a) { return (v + a - 1) / a * a; }
 
+// Bytes of epilogue exchange space (aliases the stage ring after the K loop):
+// per column half, group top-2 pairs and top-8 lists of 128 tokens, row
+// maxima and sums of exponentials.
+__host__ __device__ inline uint32_t exchange_bytes(int G) {
+  return 4u * 2u * (2u * G * BM + 3u * kTopMax * BM + 2u * BM);
+}
+// Then, with one group, each worker thread's chunk top-2 pairs (16 slots);
+// then the scores pass 1 leaves for pass 2, row by row ([BM][NL + 4] fp32).
+constexpr uint32_t kChunkPairBytes = 4u * 16u * 32u * kWorkers;
+__host__ __device__ inline uint32_t score_rows_offset(int G) {
+  return exchange_bytes(G) + (G == 1 ? kChunkPairBytes : 0u);
+}
+__host__ __device__ inline uint32_t epilogue_smem_bytes(int G, int NL) {
+  return score_rows_offset(G) + 4u * BM * (uint32_t)(NL + 4);
+}
+
 // Stage layout.  tf32: [x | W] fp32 tiles (hi) followed by their residuals
 // (lo), 128-byte rows.  bf16: [x | W1 | W2 | W3] bf16 tiles (nplanes = 3) or
-// [x | W] (nplanes = 1, W stored in bf16), 64-byte rows.
+// [x | W] (nplanes = 1, W stored in bf16), 64-byte rows.  The ring and, after
+// the K loop, the epilogue's space (G groups) share the front of shared
+// memory; the barriers, flags and bias slice follow the larger of the two.
 __host__ __device__ inline Plan make_plan(int NL, bool bf16x3 = false, bool pair = false,
-                                          int nplanes = 3) {
+                                          int nplanes = 3, int G = 1) {
   Plan p;
   const int esz = bf16x3 ? 2 : 4;
   p.a_bytes = BM * BK * esz;
   p.b_bytes = (pair ? NL / 2 : NL) * BK * esz;
   p.hi_bytes = p.a_bytes + (bf16x3 ? nplanes : 1) * p.b_bytes;
   p.stage_bytes = align_up((bf16x3 ? 1 : 2) * p.hi_bytes, 1024);
-  // after the ring: 256 B of mbarriers, 256 B of flags, the CTA's bias slice;
-  // the launch adds 1 KB so the ring can start on a 1024-byte boundary
+  // after the front: 256 B of mbarriers, 256 B of flags, the CTA's bias
+  // slice; the launch adds 1 KB so the ring can start on a 1024-byte boundary
   const uint32_t extras = 1024 + 256 + 256 + 4 * kMaxNL;
+  const uint32_t epi = align_up(epilogue_smem_bytes(G, NL), 16);
   int s = (int)((kSmemBudget - extras) / p.stage_bytes);
   p.stages = s > kMaxStages ? kMaxStages : s;
-  p.bar_off = p.stages * p.stage_bytes;
+  auto front = [&](int st) {
+    const uint32_t ring = (uint32_t)st * p.stage_bytes;
+    return ring > epi ? ring : epi;
+  };
+  while (p.stages > 0 && front(p.stages) + extras > kSmemBudget) --p.stages;
+  p.bar_off = front(p.stages);
   p.misc_off = p.bar_off + 256;
   p.bias_off = p.misc_off + 256;
   p.total = p.bias_off + 4 * kMaxNL;
   return p;
-}
-
-// Bytes of epilogue exchange space (aliases the stage ring after the K loop):
-// per column half, group top-2 pairs and top-8 lists of 128 tokens; followed
-// by the pass-2 candidate scratch (16 scores and 16 s per worker thread).
-__host__ __device__ inline uint32_t exchange_bytes(int G) {
-  return 4u * 2u * (2u * G * BM + 3u * kTopMax * BM + 2u * BM);
-}
-// Per-thread candidate buffer of the top-k scan (value, score, index):
-// kCandCap slots plus one slot that absorbs the stores of non-candidates.
-constexpr int kCandCap = 16;
-__host__ __device__ inline uint32_t epilogue_smem_bytes(int G) {
-  return exchange_bytes(G) + 4u * 3u * (kCandCap + 1) * 32u * kWorkers;
 }
 
 // ---- PTX wrappers ----------------------------------------------------------
@@ -570,7 +581,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // contains them must be launched in clusters of two.
   constexpr bool pair = PAIR;
   constexpr int NP = NPL;
-  const Plan plan = make_plan(NL, bf16x3, pair, NP);
+  const Plan plan = make_plan(NL, bf16x3, pair, NP, P.n_group);
   const int STAGES = plan.stages;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int KSP = KS ? P.ksplit : 1;
@@ -1079,12 +1090,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         sinv = 1.0f / zsum;
       }
 
-      // pass 1: s = sigmoid(L) (or softmax) back into TMEM; per-group top-2
-      // of c = s + b
+      // pass 1: s = sigmoid(L) (or softmax) into this row of shared memory;
+      // per-group top-2 of c = s + b
       uint32_t kept = 0xffffffffu;
-      // with one group, each chunk's top-2 goes to the candidate buffer
-      // (slots 2j, 2j + 1 of chunk c_beg + j) for the bound tau below
+      // with one group, each chunk's top-2 goes to slots 2j, 2j + 1 (chunk
+      // c_beg + j) of this thread's pairs, for the bound tau below
       float* chunk_pairs = reinterpret_cast<float*>(smem + exchange_bytes(G));
+      // the scores, [BM][NL + 4] (the pad keeps a warp's rows on distinct banks)
+      float* srow = reinterpret_cast<float*>(smem + score_rows_offset(G)) + row * (NL + 4);
       {
         if (G > 1)
           for (int g = 0; g < G; ++g) {
@@ -1110,7 +1123,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
               for (int i = 0; i < 16; ++i) v[i] = mr_sigmoid(v[i]);
             }
-            tmem_st16(tmem_base + lane_off + (uint32_t)(c * 16), v);
+            {
+              float4* d4 = reinterpret_cast<float4*>(srow + c * 16);
+#pragma unroll
+              for (int q4 = 0; q4 < 4; ++q4)
+                d4[q4] = make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
+            }
             if (G == 1 || chunk_groups) {
               const int gc = (col0 + c * 16) / S;
               if (G > 1 && gc != g) {
@@ -1162,7 +1180,6 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
             }
           }
-          asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
           if (G > 1) {
             exA1[(h * G + g) * BM + row] = a1;
             exA2[(h * G + g) * BM + row] = a2;
@@ -1209,28 +1226,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                                     tau);
       }
 
-      // pass 2: top-8 of this half's masked scores.  A score enters only if
-      // it is >= tau and beats the list's current 8th; such candidates are
-      // appended (in index order) to this thread's buffer in shared memory
-      // and inserted into the sorted list when the buffer fills and at the
-      // end, so the serial insertion runs ~k times per token, not once per
-      // score that beats a running threshold.
+      // pass 2: top-8 of this half's masked scores.  Each chunk's candidates
+      // (scores >= tau) are marked in a 16-bit mask from the scores pass 1
+      // left in shared memory; only the marked ones are read back and
+      // inserted, in index order, when they beat the list's current 8th.
       Top8 top;
       top.init();
       if (ok && c_beg < c_end) {
-        const bool zero_fill = (G > 1) && (P.mask_mode == MR_MASK_ZERO);
-        float* bufV = reinterpret_cast<float*>(smem + exchange_bytes(G));  // [kCandCap][256]
-        float* bufS = bufV + (kCandCap + 1) * 32 * kWorkers;
-        int* bufI = reinterpret_cast<int*>(bufS + (kCandCap + 1) * 32 * kWorkers);
-        int cnt = 0;
-        auto flush = [&]() {
-          for (int j = 0; j < cnt; ++j) {
-            const float cv = bufV[j * 32 * kWorkers + wt];
-            if (cv > top.v[kTopMax - 1])
-              top.push(cv, bufI[j * 32 * kWorkers + wt], bufS[j * 32 * kWorkers + wt]);
-          }
-          cnt = 0;
-        };
+        const float fill = (G > 1 && P.mask_mode == MR_MASK_ZERO) ? 0.0f : -INFINITY;
         // bit i: expert col0 + 16c + i lies in a kept group
         auto keep_mask = [&](int c) -> uint32_t {
           if (G == 1) return 0xffffu;
@@ -1241,44 +1244,29 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int i = 0; i < 16; ++i) km |= ((kept >> ((e0 + i) / S)) & 1u) << i;
           return km;
         };
-        // one chunk per iteration, and one more that flushes what is left
-        // (one copy of the body and of the flush in the code)
 #pragma unroll 1
-        for (int c = c_beg; c <= c_end; ++c) {
-          uint32_t m = 0;
-          if (c < c_end) {
-            __syncwarp();  // the buffer flush diverges; tcgen05.ld is .aligned
-            tmem_ld16(tmem_base + lane_off + (uint32_t)(c * 16), v);
-            load_bias(c);
-            const uint32_t km = keep_mask(c);
-            const float thr = top.v[kTopMax - 1];
-            uint32_t mlo = 0, mhi = 0;
+        for (int c = c_beg; c < c_end; ++c) {
+          load_bias(c);
+          const uint32_t km = keep_mask(c);
+          const float4* s4 = reinterpret_cast<const float4*>(srow + c * 16);
+          uint32_t mlo = 0, mhi = 0;
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const float sv = v[i];  // pass 1 left the scores in TMEM
-              const float cval = ((km >> i) & 1u) ? sv + bv[i] : (zero_fill ? 0.0f : -INFINITY);
-              v[i] = sv;
-              bv[i] = cval;
-              const uint32_t bit = (cval >= tau && cval > thr ? 1u : 0u) << i;
+          for (int q4 = 0; q4 < 4; ++q4) {
+            const float4 sv = s4[q4];
+            const float e4[4] = {sv.x, sv.y, sv.z, sv.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const int i = 4 * q4 + u;
+              const float cval = ((km >> i) & 1u) ? e4[u] + bv[i] : fill;
+              const uint32_t bit = (cval >= tau ? 1u : 0u) << i;
               if (i < 8) mlo |= bit; else mhi |= bit;
             }
-            m = mlo | mhi;
           }
-          if (c == c_end || cnt + __popc(m) > kCandCap) flush();
-          if (c < c_end) {
-            // branch-free append in index order; non-candidates write the
-            // spare slot kCandCap
-            int p = cnt;
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const bool bit = (m >> i) & 1u;
-              const int slot = (bit ? p : kCandCap) * 32 * kWorkers + wt;
-              bufV[slot] = bv[i];
-              bufS[slot] = v[i];
-              bufI[slot] = col0 + c * 16 + i;
-              p += bit ? 1 : 0;
-            }
-            cnt = p;
+          for (uint32_t m = mlo | mhi; m != 0u; m &= m - 1u) {
+            const int i = __ffs(m) - 1;
+            const float sv = srow[c * 16 + i];
+            const float cval = ((km >> i) & 1u) ? sv + bias_s[c * 16 + i] : fill;
+            if (cval > top.v[kTopMax - 1]) top.push(cval, col0 + c * 16 + i, sv);
           }
         }
       }
