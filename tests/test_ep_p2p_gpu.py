@@ -283,3 +283,41 @@ def _ipc_rank(rank, world, port):
 def test_two_processes_share_buffers_through_ipc():
     import torch.multiprocessing as tmp
     tmp.spawn(_ipc_rank, args=(2, _free_port()), nprocs=2, join=True)
+
+
+def test_package_p2p_over_one_rank_nccl_equals_single_rank():
+    """ep.ep_dispatch_p2p / ep.ep_combine_p2p through a real NCCL process
+    group of one rank: the count all-gather on the device, the stream-ordered
+    barriers (one-element all-reduces) and PeerBuffers with this rank's own
+    buffer only; a whole expert layer equals the single-rank path."""
+    import torch.distributed as dist
+
+    from token_dispatch_fp32_b200 import ep
+    N_r, k, d, n_out, T = 64, 6, 512, 128, 700
+    g = torch.Generator("cuda").manual_seed(11)
+    x = torch.randn((T, d), generator=g, device="cuda").to(torch.bfloat16)
+    idx = _idx(T, N_r, k, 12, hot=4)
+    w = torch.rand((T, k), generator=g, device="cuda")
+    shared = torch.randn((T, n_out), generator=g, device="cuda").to(torch.bfloat16)
+    W = (torch.randn((N_r, n_out, d), generator=g, device="cuda") / 16).to(torch.bfloat16)
+    counts, offsets, perm, inv = mr.mr_dispatch(idx, N_r)
+    y_ref = mr.mr_combine(mr.mr_expert_gemm_gather(x, k, perm, offsets, W), w, inv, shared)
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{_free_port()}", rank=0,
+                            world_size=1, timeout=datetime.timedelta(seconds=60),
+                            device_id=torch.device("cuda", torch.cuda.current_device()))
+    try:
+        recv = ep.PeerBuffers(T * k, d, torch.bfloat16)
+        out = ep.PeerBuffers(T * k, n_out, torch.bfloat16)
+        assert recv.ptrs == [recv.local.data_ptr()]
+        rows, lc, lo, h = ep.ep_dispatch_p2p(x, idx, N_r, recv)
+        mr.mr_expert_gemm_gather(rows, 1, None, lo, W, out=out.local)
+        y = ep.ep_combine_p2p(out, h, w, shared)
+        torch.cuda.synchronize()
+        recv.close()
+        out.close()
+    finally:
+        dist.destroy_process_group()
+    assert mr.mr_get_error() == mr.MR_OK
+    assert int(lo[-1].item()) == T * k
+    assert torch.equal(lc, counts)
+    assert torch.equal(y.view(torch.int16), y_ref.view(torch.int16))
