@@ -217,7 +217,9 @@ __device__ __forceinline__ bool disp_grid_barrier(int* counter, int target) {
         ok = 0;
         break;
       }
-      __nanosleep(64);
+      // the barrier usually opens within a few microseconds: poll without
+      // sleeping first, then back off
+      if (it >= 2048u) __nanosleep(64);
     }
     ok_s = ok;
   }
@@ -232,6 +234,7 @@ __global__ void __launch_bounds__(kDispThreads)
   extern __shared__ int sm[];  // max(kDispThreads, kDispWarps * N_r) ints, reused by the phases
   __shared__ int start_s[kDispMaxExperts];
   __shared__ int warp_tot[kDispWarps];
+  __shared__ int ids_s[kDispChunk];  // this chunk's ids from phase 1 (-1: none)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
   const int nchunks = gridDim.x, c = blockIdx.x;
   const long base = (long)c * kDispChunk + (long)warp * kDispSub;
@@ -242,6 +245,7 @@ __global__ void __launch_bounds__(kDispThreads)
   __syncthreads();
   for (int r = 0; r < kDispSub; r += 32) {
     const int e = disp_load(idx, base + r + lane, n, N_r, &bad);
+    ids_s[warp * kDispSub + r + lane] = e;
     const unsigned peers = __match_any_sync(0xffffffffu, e);
     if (e >= 0 && lane == __ffs(peers) - 1) atomicAdd(&sm[e], __popc(peers));
   }
@@ -341,7 +345,7 @@ __global__ void __launch_bounds__(kDispThreads)
   __syncthreads();
   int* mine = wbase + warp * N_r;
   for (int r = 0; r < kDispSub; r += 32) {
-    const int e = disp_load(idx, base + r + lane, n, N_r, &bad);
+    const int e = ids_s[warp * kDispSub + r + lane];
     const unsigned peers = __match_any_sync(0xffffffffu, e);
     if (e >= 0 && lane == __ffs(peers) - 1) mine[e] += __popc(peers);
     __syncwarp();
@@ -360,7 +364,7 @@ __global__ void __launch_bounds__(kDispThreads)
   const unsigned lt = (1u << lane) - 1u;
   for (int r = 0; r < kDispSub; r += 32) {
     const long i = base + r + lane;
-    const int e = disp_load(idx, i, n, N_r, &bad);
+    const int e = ids_s[warp * kDispSub + r + lane];
     const unsigned peers = __match_any_sync(0xffffffffu, e);
     if (e >= 0) {
       const int pos = mine[e] + __popc(peers & lt);
