@@ -537,7 +537,8 @@ int mr_expert_gemm_gather_packed(const void *x, const int32_t *perm,
  *   x         [T, d] rows of `dtype` (MR_BF16 or MR_F32).
  *   perm      [T*k] from mr_dispatch (used when inv_perm is NULL).
  *   inv_perm  [T*k] from mr_dispatch or NULL.  When given, each token row is
- *             read once and written to its k sorted positions.
+ *             read once and written to its k sorted positions; a slot whose
+ *             entry is -1 (an assignment mr_dispatch dropped) writes no row.
  *   xs        [T*k, d] output rows in expert-sorted order.
  * Limits: 1 <= k <= 32.
  */
@@ -553,7 +554,8 @@ int mr_gather_rows(const void *x, int dtype, int T, int d, int k,
  *   expert_out [T*k, d] expert outputs in expert-sorted order (row i belongs
  *              to slot perm[i]), `dtype` MR_BF16 or MR_F32.
  *   w          [T, k] fp32 router weights.
- *   inv_perm   [T*k] from mr_dispatch.
+ *   inv_perm   [T*k] from mr_dispatch; a slot whose entry is -1 (an
+ *              assignment mr_dispatch dropped) adds nothing.
  *   shared     [T, d] shared-expert output of `dtype`, or NULL.
  *   y          [T, d] output of `dtype`.
  * Per element: acc = sum_j w[t,j] * expert_out[inv_perm[t*k+j]] in fp32;

@@ -4,7 +4,8 @@
 // expert rows through the inverse permutation -- the scatter-back is fused
 // into the read -- accumulates in fp32 (FMA, slot order), rounds to the row
 // dtype, adds the shared row and rounds again (bf16, nearest-even).  One CTA
-// per token (grid-stride), 16-byte vectors when the row size allows.
+// per token (grid-stride); bf16 rows move in 32-byte vectors when they are
+// local and 32-byte multiples, 16-byte vectors when the row size allows.
 #pragma once
 
 #include <type_traits>
@@ -27,15 +28,21 @@ __device__ __forceinline__ float bf16_round(float v) {
   return __bfloat162float(__float2bfloat16_rn(v));
 }
 
-// bf16 rows, 8 elements (one uint4) per vector.  `src` locates the expert
-// rows of each slot (SlotRowsLocal: one expert-sorted buffer through inv;
-// SlotRowsPeer: the owners' output buffers, peer memory included).
-template <typename Src>
+// bf16 rows, two elements per 32-bit word of a vector V (uint4: 8 elements;
+// Vec32: 16).  `src` locates the expert rows of each slot (SlotRowsLocal: one
+// expert-sorted buffer through inv; SlotRowsPeer: the owners' output buffers,
+// peer memory included).  The loads of up to kCombineGroup rows and of the
+// shared row are issued before the group's FMAs, so a thread keeps that many
+// vectors in flight; the FMAs still run in slot order.
+constexpr int kCombineGroup = 8;
+
+template <typename V, typename Src>
 __global__ void __launch_bounds__(kRowThreads)
     combine_bf16_vec_kernel(Src src, const float* __restrict__ w,
-                            const uint4* __restrict__ shared, uint4* __restrict__ y, long T,
-                            long nvec, int k) {
-  __shared__ const uint4* row[kRowMaxK];
+                            const V* __restrict__ shared, V* __restrict__ y, long T, long nvec,
+                            int k) {
+  constexpr int W = (int)(sizeof(V) / 4);  // bf16 pairs per vector
+  __shared__ const V* row[kRowMaxK];
   __shared__ float wt[kRowMaxK];
   for (long t = blockIdx.x; t < T; t += gridDim.x) {
     if (threadIdx.x < k) {
@@ -44,36 +51,42 @@ __global__ void __launch_bounds__(kRowThreads)
     }
     __syncthreads();
     for (long v = threadIdx.x; v < nvec; v += kRowThreads) {
-      float acc[8];
+      float acc[2 * W];
 #pragma unroll
-      for (int q = 0; q < 8; ++q) acc[q] = 0.0f;
-#pragma unroll 8
-      for (int j = 0; j < k; ++j) {
-        const uint4* r = row[j];
-        if (!r) continue;
-        const uint4 e = src.load(r + v);
-        const float wj = wt[j];
-        float lo, hi;
-        bf16x2_unpack(e.x, lo, hi); acc[0] = fmaf(wj, lo, acc[0]); acc[1] = fmaf(wj, hi, acc[1]);
-        bf16x2_unpack(e.y, lo, hi); acc[2] = fmaf(wj, lo, acc[2]); acc[3] = fmaf(wj, hi, acc[3]);
-        bf16x2_unpack(e.z, lo, hi); acc[4] = fmaf(wj, lo, acc[4]); acc[5] = fmaf(wj, hi, acc[5]);
-        bf16x2_unpack(e.w, lo, hi); acc[6] = fmaf(wj, lo, acc[6]); acc[7] = fmaf(wj, hi, acc[7]);
-      }
-      uint4 o;
-      if (shared) {
-        const uint4 sv = __ldg(shared + t * nvec + v);
-        const uint32_t s4[4] = {sv.x, sv.y, sv.z, sv.w};
-        uint32_t r4[4];
+      for (int q = 0; q < 2 * W; ++q) acc[q] = 0.0f;
+      V sv{};
+      if (shared) sv = ld_stream(shared + t * nvec + v);
+      for (int j0 = 0; j0 < k; j0 += kCombineGroup) {
+        V e[kCombineGroup];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          float slo, shi;
-          bf16x2_unpack(s4[q], slo, shi);
-          r4[q] = bf16x2_pack_rn(bf16_round(acc[2 * q]) + slo, bf16_round(acc[2 * q + 1]) + shi);
+        for (int u = 0; u < kCombineGroup; ++u) {
+          const V* r = j0 + u < k ? row[j0 + u] : nullptr;
+          e[u] = r ? src.load(r + v) : V{};
         }
-        o = make_uint4(r4[0], r4[1], r4[2], r4[3]);
-      } else {
-        o = make_uint4(bf16x2_pack_rn(acc[0], acc[1]), bf16x2_pack_rn(acc[2], acc[3]),
-                       bf16x2_pack_rn(acc[4], acc[5]), bf16x2_pack_rn(acc[6], acc[7]));
+#pragma unroll
+        for (int u = 0; u < kCombineGroup; ++u) {
+          if (j0 + u >= k || !row[j0 + u]) continue;
+          const float wj = wt[j0 + u];
+#pragma unroll
+          for (int q = 0; q < W; ++q) {
+            float lo, hi;
+            bf16x2_unpack(word(e[u], q), lo, hi);
+            acc[2 * q] = fmaf(wj, lo, acc[2 * q]);
+            acc[2 * q + 1] = fmaf(wj, hi, acc[2 * q + 1]);
+          }
+        }
+      }
+      V o;
+#pragma unroll
+      for (int q = 0; q < W; ++q) {
+        if (shared) {
+          float slo, shi;
+          bf16x2_unpack(word(sv, q), slo, shi);
+          set_word(o, q,
+                   bf16x2_pack_rn(bf16_round(acc[2 * q]) + slo, bf16_round(acc[2 * q + 1]) + shi));
+        } else {
+          set_word(o, q, bf16x2_pack_rn(acc[2 * q], acc[2 * q + 1]));
+        }
       }
       st_stream(y + t * nvec + v, o);
     }

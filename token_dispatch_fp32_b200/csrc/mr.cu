@@ -55,6 +55,7 @@ int launch_status() {
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned32(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
 
 // ---- TMA descriptors -------------------------------------------------------
 
@@ -1198,12 +1199,23 @@ int mr_expert_gemm_gather_packed(const void* x, const int32_t* perm, const int32
 
 namespace {
 
-// The combine kernel for the row type: 16-byte vectors (bf16 or fp32) when
-// `vec`, elements otherwise.  make_src(V* tag) builds the slot-row policy
-// over the element or vector type V.
-template <typename MakeSrc>
-int launch_combine(bool vec, bool bf16, unsigned grid, cudaStream_t s, const float* w,
-                   const void* shared, void* y, long T, long d, int k, MakeSrc make_src) {
+// The combine kernel for the row type: 32-byte vectors for bf16 rows when
+// kVec32 and `vec32`, 16-byte vectors (bf16 or fp32) when `vec`, elements
+// otherwise.  make_src(V* tag) builds the slot-row policy over the element or
+// vector type V.
+template <bool kVec32, typename MakeSrc>
+int launch_combine(bool vec, bool vec32, bool bf16, unsigned grid, cudaStream_t s,
+                   const float* w, const void* shared, void* y, long T, long d, int k,
+                   MakeSrc make_src) {
+  if constexpr (kVec32) {
+    if (vec32 && bf16) {
+      auto src = make_src(static_cast<mr::Vec32*>(nullptr));
+      mr::combine_bf16_vec_kernel<<<grid, mr::kRowThreads, 0, s>>>(
+          src, w, static_cast<const mr::Vec32*>(shared), static_cast<mr::Vec32*>(y), T, d / 16,
+          k);
+      return launch_status();
+    }
+  }
   if (vec && bf16) {
     auto src = make_src(static_cast<uint4*>(nullptr));
     mr::combine_bf16_vec_kernel<<<grid, mr::kRowThreads, 0, s>>>(
@@ -1241,13 +1253,18 @@ int mr_gather_rows(const void* x, int dtype, int T, int d, int k, const int32_t*
   const long esz = dtype == MR_BF16 ? 2 : 4;
   const long row_bytes = (long)d * esz;
   const bool vec = row_bytes % 16 == 0 && aligned16(x) && aligned16(xs);
+  const bool vec32 = row_bytes % 32 == 0 && aligned32(x) && aligned32(xs);
   const long rows = (long)T * k;
   // one CTA per token: measured 353 us on the full DeepSeek-V3 batch against
   // 366 us for a grid-stride over 32 CTAs per SM
   const unsigned grid_t = (unsigned)std::min<long>(T, 1L << 30);
   const unsigned grid_r = (unsigned)std::min<long>(rows, (long)sms * 32);
   if (inv_perm) {
-    if (vec)
+    if (vec32)
+      mr::gather_inv_kernel<mr::Vec32><<<grid_t, mr::kRowThreads, 0, s>>>(
+          static_cast<const mr::Vec32*>(x), T, row_bytes / 32, k,
+          mr::SlotRowsLocal<mr::Vec32>{static_cast<mr::Vec32*>(xs), inv_perm});
+    else if (vec)
       mr::gather_inv_kernel<uint4><<<grid_t, mr::kRowThreads, 0, s>>>(
           static_cast<const uint4*>(x), T, row_bytes / 16, k,
           mr::SlotRowsLocal<uint4>{static_cast<uint4*>(xs), inv_perm});
@@ -1287,15 +1304,17 @@ int mr_combine(const void* expert_out, int dtype, const float* w, const int32_t*
   const long row_bytes = (long)d * esz;
   const bool vec = row_bytes % 16 == 0 && aligned16(expert_out) && aligned16(y) &&
                    (!shared || aligned16(shared));
+  const bool vec32 = row_bytes % 32 == 0 && aligned32(expert_out) && aligned32(y) &&
+                     (!shared || aligned32(shared));
   // 64 CTAs per SM, grid-stride (369 us on the full DeepSeek-V3 batch; 372 us
   // with 32 per SM)
   const unsigned grid = (unsigned)std::min<long>(T, (long)sms * 64);
-  return launch_combine(vec, dtype == MR_BF16, grid, s, w, shared, y, T, d, k,
-                        [&](auto* tag) {
-                          using V = std::remove_const_t<std::remove_pointer_t<decltype(tag)>>;
-                          return mr::SlotRowsLocal<const V>{static_cast<const V*>(expert_out),
-                                                            inv_perm};
-                        });
+  return launch_combine<true>(vec, vec32, dtype == MR_BF16, grid, s, w, shared, y, T, d, k,
+                              [&](auto* tag) {
+                                using V = std::remove_const_t<std::remove_pointer_t<decltype(tag)>>;
+                                return mr::SlotRowsLocal<const V>{
+                                    static_cast<const V*>(expert_out), inv_perm};
+                              });
 }
 
 // ---- expert parallelism over peer memory ------------------------------------
@@ -1372,10 +1391,12 @@ int mr_ep_combine_p2p(const void* const* out_bufs, int dtype, int d, const float
   for (int r = 0; r < ep; ++r) vec = vec && aligned16(out_bufs[r]);
   const unsigned grid = (unsigned)std::min<long>(T, (long)sms * 64);
   const int E_loc = N_r / ep;
-  return launch_combine(vec, dtype == MR_BF16, grid, s, w, shared, y, T, d, k, [&](auto* tag) {
-    using V = std::remove_const_t<std::remove_pointer_t<decltype(tag)>>;
-    return mr::SlotRowsPeer<const V>{peers, idx, dest, E_loc, N_r, capacity};
-  });
+  return launch_combine<false>(vec, false, dtype == MR_BF16, grid, s, w, shared, y, T, d, k,
+                               [&](auto* tag) {
+                                 using V = std::remove_const_t<std::remove_pointer_t<decltype(tag)>>;
+                                 return mr::SlotRowsPeer<const V>{peers, idx, dest, E_loc, N_r,
+                                                                  capacity};
+                               });
 }
 
 // ---- peer buffers between processes -----------------------------------------

@@ -8,8 +8,29 @@ namespace mr {
 
 
 constexpr int kRowThreads = 128;
-constexpr int kRowUnroll = 4;
 constexpr int kRowMaxK = 32;
+
+// 32-byte vector: sm_100 moves it with one load or store instruction
+// (ld/st .v8.b32), half the instructions of 16-byte vectors.  The local row
+// movers use it when the row size and every row base are multiples of 32
+// bytes: on the full DeepSeek-V3 batch the gather takes 334 us with it
+// against 346 us with 16-byte vectors, and the combine 362.5 us against
+// 368.6 us (same-box A/B).
+struct alignas(32) Vec32 {
+  uint32_t w[8];
+};
+
+__device__ __forceinline__ uint32_t word(const uint4& v, int q) {
+  return q == 0 ? v.x : q == 1 ? v.y : q == 2 ? v.z : v.w;
+}
+__device__ __forceinline__ uint32_t word(const Vec32& v, int q) { return v.w[q]; }
+__device__ __forceinline__ void set_word(uint4& v, int q, uint32_t x) {
+  if (q == 0) v.x = x;
+  else if (q == 1) v.y = x;
+  else if (q == 2) v.z = x;
+  else v.w = x;
+}
+__device__ __forceinline__ void set_word(Vec32& v, int q, uint32_t x) { v.w[q] = x; }
 
 template <typename V>
 __device__ __forceinline__ V ld_stream(const V* p) {
@@ -18,6 +39,15 @@ __device__ __forceinline__ V ld_stream(const V* p) {
 template <>
 __device__ __forceinline__ uint16_t ld_stream<uint16_t>(const uint16_t* p) {
   return *p;
+}
+template <>
+__device__ __forceinline__ Vec32 ld_stream<Vec32>(const Vec32* p) {
+  Vec32 r;
+  asm volatile("ld.global.nc.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(r.w[0]), "=r"(r.w[1]), "=r"(r.w[2]), "=r"(r.w[3]), "=r"(r.w[4]),
+                 "=r"(r.w[5]), "=r"(r.w[6]), "=r"(r.w[7])
+               : "l"(p));
+  return r;
 }
 
 // Store of an output row that is not read again by this kernel: streaming
@@ -29,6 +59,13 @@ __device__ __forceinline__ void st_stream(V* p, const V& v) {
 template <>
 __device__ __forceinline__ void st_stream<uint16_t>(uint16_t* p, const uint16_t& v) {
   *p = v;
+}
+template <>
+__device__ __forceinline__ void st_stream<Vec32>(Vec32* p, const Vec32& v) {
+  asm volatile("st.global.cs.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p),
+               "r"(v.w[0]), "r"(v.w[1]), "r"(v.w[2]), "r"(v.w[3]), "r"(v.w[4]), "r"(v.w[5]),
+               "r"(v.w[6]), "r"(v.w[7])
+               : "memory");
 }
 
 // Where the row of slot (t, j) lives, for the row movers: each policy returns
