@@ -49,11 +49,9 @@ NVLINK_PEER_GBS = 770.0
 # source file it was built from; reported only while the source is unchanged.
 NCU_TRAFFIC = {
     # ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum of the current
-    # source on the DeepSeek-V3 prefill batch (T=4096): 528.77 MB read + 47.72
-    # MB written per launch, scaled by the tokens (x4) to the full batch --
-    # reads scale exactly (2.115 GB read at T=16384 in a full-size capture of
-    # the kernel before its rows were located through a policy object).
-    "combine": {"src": "3556d6f06cf4dcd2", "bytes": 4 * (528.76992e6 + 47.716864e6)},
+    # source on the full DeepSeek-V3 batch (T=16384; one pass per launch):
+    # 2115.01 MB read + 224.75 MB written per launch.
+    "combine": {"src": "f0e65656306c92ab", "bytes": 2115008256 + 224749824},
 }
 
 
