@@ -369,10 +369,10 @@ def run_expert_only(args, w: wl.Workload):
     xb = torch.from_numpy(d["x_bf16"]).view(torch.bfloat16).to(dev)
     ws = torch.empty(max(4, mr.mr_router_workspace_size(w.T, w.d, w.N_r)), dtype=torch.uint8,
                      device=dev)
-    idx, _ = mr.mr_router_forward_ex(xb, torch.from_numpy(d["W"]).to(dev),
-                                     torch.from_numpy(d["b"]).to(dev), w.n_group, w.topk_group,
-                                     w.k, w.route_scale, w.mask_mode,
-                                     precision=mr.MR_PREC_BF16X3, workspace=ws, stream=stream)
+    idx, wt = mr.mr_router_forward_ex(xb, torch.from_numpy(d["W"]).to(dev),
+                                      torch.from_numpy(d["b"]).to(dev), w.n_group,
+                                      w.topk_group, w.k, w.route_scale, w.mask_mode,
+                                      precision=mr.MR_PREC_BF16X3, workspace=ws, stream=stream)
     _, offsets, perm, _ = mr.mr_dispatch(idx, w.N_r, stream=stream)
     eW = torch.from_numpy(wl.gen_expert_W(w, args.n_out)).view(torch.bfloat16).to(dev)
     out = torch.empty((w.T * w.k, args.n_out), dtype=torch.bfloat16, device=dev)
@@ -383,8 +383,21 @@ def run_expert_only(args, w: wl.Workload):
         rows = mr.mr_gather_rows(xb, w.k, perm=perm, stream=stream)
         rperm = None
 
+    if args.expert_epilogue == "combine":
+        if rperm is None:
+            raise SystemExit("--expert-epilogue combine needs --expert-rows gather")
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(w.seed + 1)
+        csh = torch.randn((w.T, args.n_out), generator=gen, device=dev).to(torch.bfloat16)
+        cacc = torch.empty((w.T, args.n_out), dtype=torch.float32, device=dev)
+        cy = torch.empty((w.T, args.n_out), dtype=torch.bfloat16, device=dev)
+
     def call():
-        if eWp is not None:
+        if args.expert_epilogue == "combine":
+            mr.mr_expert_gemm_gather_combine(
+                rows, w.k, rperm, offsets, eWp if eWp is not None else eW, wt, csh, N_r=w.N_r,
+                n_out=args.n_out, packed=eWp is not None, acc=cacc, y=cy, stream=stream)
+        elif eWp is not None:
             mr.mr_expert_gemm_gather_packed(rows, w.k, rperm, offsets, eWp, w.N_r, args.n_out,
                                             out=out, stream=stream)
         else:
@@ -404,6 +417,7 @@ def run_expert_only(args, w: wl.Workload):
     fl = 2.0 * w.T * w.k * w.d * args.n_out
     print(json.dumps({"only": "expert", "workload": w.name, "n_out": args.n_out, "ms": ms,
                       "weights": args.expert_weights, "rows": args.expert_rows,
+                      "epilogue": args.expert_epilogue,
                       "tflops": fl / (ms / 1e3) / 1e12, "steps": args.steps}), flush=True)
 
 
@@ -624,13 +638,39 @@ def run_ours(args, w: wl.Workload, rank: int, world: int):
             mr.mr_gather_rows(ex, we.k, perm=eperm, inv_perm=einv, xs=exs, stream=stream)
             gemm_on_sorted_rows()
 
+        # the combine fused into the same layer's epilogue (n_out-wide rows:
+        # weighted sum over the k slots, shared add) beside the layer's
+        # expert outputs written out and then mr_combine
+        egen = torch.Generator(device=dev)
+        egen.manual_seed(we.seed + 1)
+        esh = torch.randn((we.T, n_out), generator=egen, device=dev).to(torch.bfloat16)
+        eacc = torch.empty((we.T, n_out), dtype=torch.float32, device=dev)
+        ey = torch.empty((we.T, n_out), dtype=torch.bfloat16, device=dev)
+
+        def fused_combine():
+            mr.mr_expert_gemm_gather_combine(ex, we.k, eperm, eoff, eWp, ewt, esh, N_r=we.N_r,
+                                             n_out=n_out, packed=True, acc=eacc, y=ey,
+                                             stream=stream)
+
+        def layer_then_combine():
+            fused()
+            mr.mr_combine(eout, ewt, einv, esh, y=ey, stream=stream)
+
         fms = time_alone(fused, n_alone)
         pms = time_alone(fused_plain_layout, max(3, n_alone // 4))
         ums = time_alone(unfused, n_alone)
         gms = time_alone(gemm_on_sorted_rows, n_alone)
+        cms = time_alone(fused_combine, n_alone)
+        lcms = time_alone(layer_then_combine, n_alone)
         ef = 2.0 * we.T * we.k * we.d * n_out
         wbytes = 2 * we.N_r * n_out * we.d
         expert = {"workload": we.name, "n_out": n_out, "ms": fms,
+                  "ms_with_combine_fused": cms,
+                  "ms_layer_then_combine": lcms,
+                  "combine_fused_note": "mr_expert_gemm_gather_combine (memset of the fp32 "
+                                        "accumulator, GEMM with the weighted-sum epilogue, "
+                                        "finalize with the shared add) against the layer's "
+                                        "outputs written out and mr_combine",
                   "tflops": ef / (fms / 1e3) / 1e12,
                   "weights": "packed tiles (mr_expert_pack_weights, once, outside the timing)",
                   "ms_plain_weight_layout": pms,
@@ -640,7 +680,7 @@ def run_ours(args, w: wl.Workload, rank: int, world: int):
                   "hbm_bound_ms": None,
                   "saved_bytes": 2 * 2 * we.T * we.k * we.d,
                   "l2": "read pass over 512 MB before each call"}
-        del ex, ews, eW, eWp, eout, exs
+        del ex, ews, eW, eWp, eout, exs, esh, eacc, ey
         assert mr.mr_get_error(stream) == mr.MR_OK
 
     # Expert parallelism over peer memory, 8 ranks emulated on this GPU: each
@@ -1016,6 +1056,9 @@ def main(argv=None):
                     help="with --only expert: output columns of the expert layer")
     ap.add_argument("--only", choices=("router", "expert"), default=None,
                     help="time one stage alone (a profiling aid; no bench line)")
+    ap.add_argument("--expert-epilogue", choices=("out", "combine"), default="out",
+                    help="with --only expert: write the expert outputs, or fuse the weighted "
+                         "combine and shared add (mr_expert_gemm_gather_combine)")
     ap.add_argument("--router-weights", choices=("f32", "bf16"), default="f32",
                     help="with --only router: the gate weight's stored type")
     args = ap.parse_args(argv)

@@ -531,6 +531,41 @@ int mr_expert_gemm_gather_packed(const void *x, const int32_t *perm,
                                  void *out, mr_stream_t stream);
 
 /*
+ * mr_expert_gemm_gather_combine -- the expert layer of mr_expert_gemm_gather
+ * with the weighted combine fused into its epilogue (Kimi K2 "Add shared
+ * output" page, moe_infer: outs = expert(sorted rows), new_x[idxs] = outs,
+ * new_x.view(T, k, d) cast to the weights' dtype, multiplied by topk_weight
+ * and summed over k, cast back, then y + shared_experts(identity)): neither
+ * the gathered rows nor the expert outputs are written to memory.
+ *
+ *   x, perm, offsets, T, d, k, N_r, n_out   as mr_expert_gemm_gather (perm
+ *            required: it gives each sorted row's slot perm[j] = t*k + j').
+ *   W        the expert weights: [N_r, n_out, d] bf16 (nn.Linear layout)
+ *            when w_packed == 0, the layout of mr_expert_pack_weights when
+ *            w_packed == 1.
+ *   w        [T, k] fp32 router weights (row j is scaled by w[perm[j]]).
+ *   shared   [T, n_out] bf16 shared-expert output, or NULL.
+ *   acc      [T, n_out] fp32 scratch, caller-owned and 16-byte aligned; the
+ *            call zeroes it and leaves the fp32 routed sums in it.
+ *   y        [T, n_out] bf16 output, 16-byte aligned.
+ * Per element: out_j = bf16(x[perm[j]/k] . W[e(j)]^T) (as
+ * mr_expert_gemm_gather); acc[t] = sum over the token's routed slots of the
+ * fp32 products w_j * out_j, added with fp32 atomic reductions, so the order
+ * of the k terms is not fixed and acc can differ in its last bits from run to
+ * run; y = bf16(bf16(acc) + shared) (bf16(acc) without shared), both
+ * roundings to nearest even.  A token with no routed slot gets y = shared
+ * (or 0).  Three launches on `stream`: a memset of acc, the GEMM, the
+ * finalize.  Limits as mr_expert_gemm_gather; n_out % 16 == 0, shared 16-byte
+ * aligned (else MR_ERR_UNSUPPORTED).
+ */
+int mr_expert_gemm_gather_combine(const void *x, const int32_t *perm,
+                                  const int32_t *offsets, const void *W,
+                                  int w_packed, const float *w,
+                                  const void *shared, int T, int d, int k,
+                                  int N_r, int n_out, float *acc, void *y,
+                                  mr_stream_t stream);
+
+/*
  * mr_gather_rows -- sorted_tokens = x[idxs // k] (Kimi K2 "Add shared output"
  * page, moe_infer).  Copies rows bit for bit.
  *

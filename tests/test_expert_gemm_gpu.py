@@ -157,3 +157,156 @@ def test_expert_gemm_on_sorted_rows_equals_fused_gather():
     assert mr.mr_get_error() == mr.MR_OK
     assert torch.equal(fused.view(torch.int16), plain.view(torch.int16))
     assert torch.equal(fused.view(torch.int16), packed.view(torch.int16))
+
+
+# ---- the combine fused into the expert layer's epilogue ---------------------
+
+def _combine_case(T, d, N_r, k, n_out, seed, skew, integer, with_shared, drop=0.0):
+    """Inputs of one fused-combine case (bf16 bits, fp32 weights) and the
+    dispatch of its ids (oracle); `drop` > 0 puts that fraction of the slots
+    (and every slot of token 0) out of range, which dispatch drops."""
+    rng = np.random.default_rng(seed)
+    if integer:
+        # small integers: every product and every d-term sum is exact in fp32,
+        # so the tensor core's expert outputs are the rounded exact values
+        x = wl.to_bf16_bits(rng.integers(-2, 3, (T, d)).astype(np.float32))
+        W = wl.to_bf16_bits(rng.integers(-2, 3, (N_r, n_out, d)).astype(np.float32))
+    else:
+        x = wl.to_bf16_bits(rng.standard_normal((T, d)).astype(np.float32))
+        W = wl.gen_expert_W(wl.Workload(f"ecomb{seed}", T=T, d=d, N_r=N_r, n_group=1,
+                                        topk_group=1, k=k, route_scale=1.0, mask_mode=0,
+                                        seed=seed), n_out)
+    idx = _ids(T, k, N_r, seed, skew)
+    if drop > 0:
+        idx = np.where(rng.random((T, k)) < drop, N_r + 1, idx).astype(np.int32)
+        idx[0, :] = N_r + 3
+    w = rng.uniform(0.05, 1.0, (T, k)).astype(np.float32)
+    sh = (wl.to_bf16_bits(rng.standard_normal((T, n_out)).astype(np.float32))
+          if with_shared else None)
+    return x, W, idx, w, sh
+
+
+def _combine_reference(x, W, idx, w, sh, k, N_r, integer):
+    """The oracle's y and routed sums for the fused layer, and a per-element
+    bound on |y_gpu - y|: the expert outputs (tensor core, fp32 accumulation,
+    bf16 rounding) are within 2 ulp_bf16 + (d/16 + 2) 2^-23 sum|x W| of the
+    oracle's rounded exact ones (0 for integer inputs: exact accumulation);
+    the weighted sum adds fp32 products in some order ((k + 1) 2^-23 of
+    sum|w E|); the two bf16 roundings can each land one ulp away."""
+    T, d = x.shape
+    n_out = W.shape[1]
+    valid = (idx >= 0) & (idx < N_r)
+    # dropped slots go to an extra expert N_r: the stable sort keeps the valid
+    # slots first, in the order dispatch gives them
+    _, offsets, perm, inv = oracle.dispatch(np.where(valid, idx, N_r).astype(np.int32),
+                                            N_r + 1)
+    offsets = offsets[:N_r + 1]
+    n_valid = int(offsets[-1])
+    ref = oracle.expert_gemm(x, k, perm, offsets, W)  # [n_valid, n_out] exact
+    E_ref = oracle.round_bf16(ref)
+    if integer:
+        e_err = np.zeros_like(ref)
+    else:
+        xf = np.abs(wl.bf16_bits_to_f32(x).astype(np.float64))
+        Wf = np.abs(wl.bf16_bits_to_f32(W).astype(np.float64))
+        absdot = np.empty_like(ref)
+        for e in range(N_r):
+            lo, hi = offsets[e], offsets[e + 1]
+            if hi > lo:
+                absdot[lo:hi] = xf[perm[lo:hi] // k] @ Wf[e].T
+        e_err = 2 * bf16_ulp(ref) + (d / 16 + 2) * 2.0 ** -23 * absdot
+    w0 = np.where(valid, w, np.float32(0)).astype(np.float32)
+    inv0 = np.where(valid.reshape(-1), inv, 0).astype(np.int32)
+    E_full = np.zeros((T * k, n_out), np.float64)
+    E_full[:n_valid] = E_ref
+    err_full = np.zeros_like(E_full)
+    err_full[:n_valid] = e_err
+    E_bits = wl.to_bf16_bits(E_full.astype(np.float32))
+    ry, rr = oracle.combine(E_bits, w0, inv0, sh, k)
+    aw = np.abs(w0).astype(np.float64)[:, :, None]
+    s_err = (aw * err_full[inv0].reshape(T, k, n_out)).sum(1)
+    s_abs = (aw * np.abs(E_full[inv0]).reshape(T, k, n_out)).sum(1)
+    tol = bf16_ulp(rr) + bf16_ulp(ry) + 1.01 * (s_err + (k + 1) * 2.0 ** -23 * s_abs)
+    return ry, rr, tol
+
+
+COMBINE_CASES = [
+    # T, d, N_r, k, n_out, skew, integer, shared, packed, gather, drop
+    (300, 512, 32, 4, 256, False, True, True, False, "lsu", 0.0),
+    (257, 200, 32, 3, 144, True, True, True, True, "tma", 0.0),   # K tail, partial N tile
+    (257, 200, 32, 3, 144, True, False, False, False, "tma", 0.0),
+    (1000, 512, 64, 8, 256, True, False, True, True, "lsu", 0.0),  # skewed: many blocks
+    (256, 7168, 256, 8, 512, False, False, True, True, "lsu", 0.0),  # DeepSeek-V3 shapes
+    (600, 256, 16, 4, 256, False, False, True, False, "lsu", 0.1),  # dropped slots
+]
+
+
+@pytest.mark.parametrize("T,d,N_r,k,n_out,skew,integer,with_shared,packed,gather,drop",
+                         COMBINE_CASES,
+                         ids=[f"T{c[0]}_d{c[1]}_E{c[2]}_n{c[4]}_{'int' if c[6] else 'rand'}"
+                              f"{'_packed' if c[8] else ''}_{c[9]}{'_drop' if c[10] else ''}"
+                              for c in COMBINE_CASES])
+def test_expert_gemm_gather_combine_matches_oracle(T, d, N_r, k, n_out, skew, integer,
+                                                   with_shared, packed, gather, drop,
+                                                   monkeypatch):
+    """y of the fused layer against the oracle (expert layer rounded to bf16,
+    then the pages' weighted sum and shared add) within the derived bound of
+    _combine_reference; tokens without a routed slot get the shared row."""
+    if gather == "tma":
+        monkeypatch.setenv("MR_EG_GATHER", "tma")
+    seed = 11 * T + d + n_out
+    x, W, idx, w, sh = _combine_case(T, d, N_r, k, n_out, seed, skew, integer, with_shared,
+                                     drop)
+    counts, offsets, perm, inv = mr.mr_dispatch(torch.from_numpy(idx).cuda(), N_r)
+    assert mr.mr_get_error() == (mr.MR_ERR_DEVICE if drop > 0 else mr.MR_OK)
+    Wd = _dev_bits(W)
+    if packed:
+        Wd = mr.mr_expert_pack_weights(Wd)
+    acc = torch.full((T, n_out), float("nan"), dtype=torch.float32, device="cuda")
+    y = mr.mr_expert_gemm_gather_combine(_dev_bits(x), k, perm, offsets, Wd,
+                                         torch.from_numpy(w).cuda(),
+                                         None if sh is None else _dev_bits(sh), N_r=N_r,
+                                         n_out=n_out, packed=packed, acc=acc)
+    assert mr.mr_get_error() == mr.MR_OK
+    got = wl.bf16_bits_to_f32(y.view(torch.int16).cpu().numpy().view(np.uint16))
+    got = got.astype(np.float64)
+    ry, rr, tol = _combine_reference(x, W, idx, w, sh, k, N_r, integer)
+    err = np.abs(got - ry)
+    assert np.isfinite(got).all()
+    worst = np.unravel_index(np.argmax(err - tol), err.shape)
+    assert (err <= tol).all(), f"token {worst[0]} col {worst[1]}: {got[worst]} vs {ry[worst]}"
+    if drop > 0:  # token 0 has no routed slot: y = bf16(0 + shared) = shared
+        want = sh[0] if sh is not None else np.zeros(n_out, np.uint16)
+        assert np.array_equal(y[0].view(torch.int16).cpu().numpy().view(np.uint16), want)
+    stats = {"elems": int(err.size), "max_abs_err": float(err.max()),
+             "max_err_over_tol": float((err / tol).max()),
+             "y_differ_elems": int((err > 0).sum())}
+    record(f"expert_combine_T{T}_d{d}_E{N_r}_n{n_out}", "expert_gemm_gather_combine", stats)
+    print(stats)
+
+
+def test_expert_gemm_gather_combine_equals_layer_then_combine_within_bound():
+    """The fused layer against the two-step path on the same GPU (the expert
+    layer written out, then mr_combine): the same expert outputs, added in
+    another order and without the FMA.  The two fp32 sums are each within
+    (k + 1) 2^-24 sum|w E| of the exact one; each bf16 rounding can then land
+    one ulp apart."""
+    T, d, N_r, k, n_out = 512, 1024, 64, 8, 512
+    x, W, idx, w, sh = _combine_case(T, d, N_r, k, n_out, 5, True, False, True)
+    counts, offsets, perm, inv = mr.mr_dispatch(torch.from_numpy(idx).cuda(), N_r)
+    xd, Wd, wd, shd = _dev_bits(x), _dev_bits(W), torch.from_numpy(w).cuda(), _dev_bits(sh)
+    acc = torch.empty((T, n_out), dtype=torch.float32, device="cuda")
+    fused = mr.mr_expert_gemm_gather_combine(xd, k, perm, offsets, Wd, wd, shd, acc=acc)
+    E = mr.mr_expert_gemm_gather(xd, k, perm, offsets, Wd)
+    two = mr.mr_combine(E, wd, inv, shd)
+    assert mr.mr_get_error() == mr.MR_OK
+    a = fused.float().cpu().numpy().astype(np.float64)
+    b = two.float().cpu().numpy().astype(np.float64)
+    Ef = E.float().cpu().numpy().astype(np.float64)
+    s_abs = (np.abs(w).astype(np.float64)[:, :, None]
+             * np.abs(Ef[inv.cpu().numpy()]).reshape(T, k, n_out)).sum(1)
+    D = 2 * (k + 1) * 2.0 ** -24 * s_abs
+    r = np.abs(acc.cpu().numpy().astype(np.float64)) + D
+    tol = D + 2 * bf16_ulp(r) + 2 * bf16_ulp(np.abs(b) + D + 2 * bf16_ulp(r))
+    assert (np.abs(a - b) <= tol).all()
+    assert (a == b).mean() > 0.95  # most elements round identically

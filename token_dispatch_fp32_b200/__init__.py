@@ -9,7 +9,7 @@ from ._binding import (  # noqa: F401
     MR_GROUP_MAX, MR_NORM_NO_EPS, MR_PREC_BF16X3, MR_PREC_FFMA, MR_PREC_TF32, MR_SCORE_SOFTMAX,
     MRError, lib, mr_combine, mr_dispatch, mr_ep_combine_p2p, mr_ep_dispatch_p2p,
     mr_ep_recv_order, mr_expert_gemm_gather, mr_ipc_close, mr_ipc_export, mr_ipc_import,
-    mr_expert_gemm_gather_packed, mr_expert_pack_weights,
+    mr_expert_gemm_gather_combine, mr_expert_gemm_gather_packed, mr_expert_pack_weights,
     mr_dispatch_noalloc, mr_dispatch_noalloc_max_workspace,
     mr_dispatch_workspace_size, mr_gather_rows, mr_get_error, mr_launch_count, mr_router_forward,
     mr_router_forward_bf16w, mr_router_forward_ex, mr_router_forward_max_scratch, mr_router_workspace_size,

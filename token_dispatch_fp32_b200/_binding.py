@@ -82,6 +82,7 @@ def lib():
         L.mr_ep_recv_order.argtypes = [p, i, i, i, p, p, p, p, p]
         L.mr_expert_gemm_gather.argtypes = [p, p, p, p, i, i, i, i, i, p, p]
         L.mr_expert_gemm_gather_packed.argtypes = [p, p, p, p, i, i, i, i, i, p, p]
+        L.mr_expert_gemm_gather_combine.argtypes = [p, p, p, p, i, p, p, i, i, i, i, i, p, p, p]
         L.mr_expert_packed_bytes.argtypes = [i, i, i]
         L.mr_expert_packed_bytes.restype = sz
         L.mr_expert_pack_weights.argtypes = [p, i, i, i, p, sz, p]
@@ -395,6 +396,42 @@ def mr_expert_gemm_gather_packed(x, k, perm, offsets, W_packed, N_r, n_out, out=
     _call("mr_expert_gemm_gather_packed", _device_of(x, perm, offsets, W_packed, out), stream,
           _ptr(x), _ptr(perm), _ptr(offsets), _ptr(W_packed), T, d, k, N_r, n_out, _ptr(out))
     return out
+
+
+def mr_expert_gemm_gather_combine(x, k, perm, offsets, W, w, shared=None, N_r=None,
+                                  n_out=None, packed=False, acc=None, y=None, stream=None):
+    """The expert layer with the gather and the weighted combine fused in:
+    y [T, n_out] bf16 = bf16(bf16(sum_j w[t,j] * bf16(x[t] . W[e_j]^T)) +
+    shared[t]).  x [T,d] bf16; perm [T*k], offsets [N_r+1] int32 (from
+    mr_dispatch); W [N_r, n_out, d] bf16, or the packed layout
+    (mr_expert_pack_weights; packed=True, N_r and n_out given); w [T,k] fp32;
+    shared [T, n_out] bf16 or None.  acc: [T, n_out] fp32 scratch (allocated
+    when None; holds the fp32 routed sums afterwards).  Returns y."""
+    _need(x, "x", torch.bfloat16)
+    T, d = x.shape
+    _need(perm, "perm", torch.int32, (T * k,))
+    _need(W, "W", torch.bfloat16)
+    if packed:
+        if N_r is None or n_out is None:
+            raise ValueError("packed weights need N_r and n_out")
+        if W.numel() * 2 < int(lib().mr_expert_packed_bytes(N_r, n_out, d)):
+            raise ValueError("W is smaller than mr_expert_packed_bytes")
+    else:
+        N_r, n_out, dw = W.shape
+        if dw != d:
+            raise ValueError(f"W is [N_r, n_out, {dw}], x rows have {d} columns")
+    _need(offsets, "offsets", torch.int32, (N_r + 1,))
+    _need(w, "w", torch.float32, (T, k))
+    if shared is not None:
+        _need(shared, "shared", torch.bfloat16, (T, n_out))
+    acc = torch.empty((T, n_out), dtype=torch.float32, device=x.device) if acc is None \
+        else _need(acc, "acc", torch.float32, (T, n_out))
+    y = torch.empty((T, n_out), dtype=torch.bfloat16, device=x.device) if y is None \
+        else _need(y, "y", torch.bfloat16, (T, n_out))
+    _call("mr_expert_gemm_gather_combine", _device_of(x, perm, offsets, W, w, shared, acc, y),
+          stream, _ptr(x), _ptr(perm), _ptr(offsets), _ptr(W), 1 if packed else 0, _ptr(w),
+          _ptr(shared), T, d, k, N_r, n_out, _ptr(acc), _ptr(y))
+    return y
 
 
 def mr_gather_rows(x, k, perm=None, inv_perm=None, xs=None, stream=None):

@@ -21,6 +21,16 @@
 // Grid: x = 128-row blocks over all experts (an upper bound from the host;
 // each CTA finds its expert and block from the offsets, surplus CTAs exit),
 // y = 256-column blocks of n_out.  Every mbarrier wait is bounded.
+//
+// With the combine fused in (COMBINE; the same page: new_x[idxs] = outs,
+// weighted sum over k, cast back, plus the shared expert's output) the
+// expert outputs are never written either: the epilogue rounds each row to
+// bf16, multiplies it by its slot's router weight (fp32) and adds it into the
+// token's fp32 row of a [T, n_out] accumulator with vector reductions
+// (red.global.add.v4.f32, resolved in L2).  Rows of one expert segment belong
+// to distinct tokens, so the k additions into a token row come from k
+// different CTAs in no fixed order.  combine_acc_finalize_kernel then rounds
+// the accumulator to bf16, adds the shared row and rounds again.
 #pragma once
 
 #include "router_tc.cuh"
@@ -51,8 +61,18 @@ struct Params {
   const int32_t* perm;
   const int32_t* offsets;
   const __nv_bfloat16* w_packed;  // packed weights (PACKED only)
-  __nv_bfloat16* out;  // [offsets[N_r], n_out]
+  __nv_bfloat16* out;  // [offsets[N_r], n_out] (not COMBINE)
+  const float* wts;    // [T*k] router weights by slot (COMBINE)
+  float* acc;          // [T, n_out] fp32, zeroed before the launch (COMBINE)
 };
+
+// Adds four floats to 16 bytes of global memory (one vector reduction at the
+// L2; the address 16-byte aligned).
+__device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c),
+               "f"(d)
+               : "memory");
+}
 
 // One contiguous global -> shared copy completing on an mbarrier (16-byte
 // aligned addresses, a multiple of 16 bytes).
@@ -96,11 +116,15 @@ __device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap* map
 //                warp 0's expect-tx arrival and the four copy warps).
 constexpr int kRowsSorted = 0, kGatherTma = 1, kGatherLsu = 2;
 
-template <int BKE, bool PACKED = false, int AMODE = kGatherTma>
+// COMBINE: the epilogue does not write the expert outputs; it scales each
+// row (rounded to bf16, the expert's output dtype) by its slot's router weight
+// and adds it into the token's fp32 row of P.acc.
+template <int BKE, bool PACKED = false, int AMODE = kGatherTma, bool COMBINE = false>
 __global__ void __launch_bounds__(kThreads, 1)
     expert_gemm_gather_kernel(const __grid_constant__ CUtensorMap map_x,
                               const __grid_constant__ CUtensorMap map_w, const Params P) {
   constexpr bool GATHER = AMODE != kRowsSorted;
+  static_assert(!COMBINE || GATHER, "the combine needs each row's slot (perm)");
   static_assert(AMODE != kGatherLsu || BKE == 64, "the copy warps fill 128-byte rows");
   static_assert(!PACKED || BKE == 64, "the packed layout has 64-column tiles");
   using PL = EgPlan<BKE>;
@@ -316,8 +340,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int j = row0 + r;
     const bool store = ok && j < row_end;
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
-    __nv_bfloat16* dst = P.out + (long)j * P.n_out + n0;
-    for (int c = 0; c < kBN / 16; ++c) {
+    if constexpr (COMBINE) {
+      // slot perm[j] = t * k + slot: weight w[perm[j]], token row t of acc
+      const int slot = store ? P.perm[j] : 0;
+      const float wj = store ? P.wts[slot] : 0.0f;
+      float* arow = P.acc + (long)(slot / P.k) * P.n_out + n0;
+      for (int c = 0; c < kBN / 16; ++c) {
+        float v[16];
+        tmem_ld16(tmem_base + lane_off + (uint32_t)(c * 16), v);  // whole warp
+        if (store && n0 + c * 16 < P.n_out) {
+#pragma unroll
+          for (int i = 0; i < 16; i += 4)
+            red_add_v4(arow + c * 16 + i, wj * __bfloat162float(__float2bfloat16_rn(v[i])),
+                       wj * __bfloat162float(__float2bfloat16_rn(v[i + 1])),
+                       wj * __bfloat162float(__float2bfloat16_rn(v[i + 2])),
+                       wj * __bfloat162float(__float2bfloat16_rn(v[i + 3])));
+        }
+      }
+    }
+    __nv_bfloat16* dst = COMBINE ? nullptr : P.out + (long)j * P.n_out + n0;
+    for (int c = 0; c < (COMBINE ? 0 : kBN / 16); ++c) {
       float v[16];
       tmem_ld16(tmem_base + lane_off + (uint32_t)(c * 16), v);  // whole warp
       if (store && n0 + c * 16 < P.n_out) {
@@ -341,6 +383,38 @@ __global__ void __launch_bounds__(kThreads, 1)
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
                  "r"(kBN)
                  : "memory");
+  }
+}
+
+// y = bf16(bf16(acc) + shared) (or bf16(acc) without a shared row), eight
+// elements (two float4 of acc, one 16-byte vector of bf16) per thread and step.
+__global__ void __launch_bounds__(256)
+    combine_acc_finalize_kernel(const float4* __restrict__ acc, const uint4* __restrict__ shared,
+                                uint4* __restrict__ y, long n8) {
+  for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < n8;
+       i += (long)gridDim.x * blockDim.x) {
+    const float4 a0 = __ldcs(acc + 2 * i), a1 = __ldcs(acc + 2 * i + 1);
+    float v[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+    uint32_t o[4];
+    if (shared) {
+      const uint4 sv = __ldcs(shared + i);
+      const uint32_t s4[4] = {sv.x, sv.y, sv.z, sv.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float slo = __uint_as_float(s4[q] << 16), shi = __uint_as_float(s4[q] & 0xffff0000u);
+        const __nv_bfloat162 h = __floats2bfloat162_rn(
+            __bfloat162float(__float2bfloat16_rn(v[2 * q])) + slo,
+            __bfloat162float(__float2bfloat16_rn(v[2 * q + 1])) + shi);
+        o[q] = *reinterpret_cast<const uint32_t*>(&h);
+      }
+    } else {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * q], v[2 * q + 1]);
+        o[q] = *reinterpret_cast<const uint32_t*>(&h);
+      }
+    }
+    __stcs(y + i, make_uint4(o[0], o[1], o[2], o[3]));
   }
 }
 

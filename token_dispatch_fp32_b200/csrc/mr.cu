@@ -1072,19 +1072,24 @@ int mr_ep_recv_order(const int32_t* recv_counts, int ep, int E_loc, int R, int32
 namespace {
 
 // Shared by the plain and the packed-weight entry points.
+// wts/acc non-null: the combine epilogue (router weights by slot, the
+// zeroed fp32 [T, n_out] accumulator) instead of writing `out`.
 int launch_expert_gemm(const void* x, const int32_t* perm, const int32_t* offsets,
                        const void* W, bool packed, int T, int d, int k, int N_r, int n_out,
-                       void* out, cudaStream_t s) {
+                       void* out, cudaStream_t s, const float* wts = nullptr,
+                       float* acc = nullptr) {
   if (T < 0 || d <= 0 || k <= 0 || N_r <= 0 || n_out <= 0) return MR_ERR_INVALID_ARG;
   if ((long long)T * k >= (1LL << 31) || (long long)N_r * n_out >= (1LL << 31))
     return MR_ERR_INVALID_ARG;
   if (T == 0) return MR_OK;
-  if (!x || !offsets || !W || !out) return MR_ERR_INVALID_ARG;
+  const bool combine = acc != nullptr;
+  if (!x || !offsets || !W || (!combine && !out) || (combine && (!wts || !perm)))
+    return MR_ERR_INVALID_ARG;
   const bool gather = perm != nullptr;  // NULL: x already holds the sorted rows
   int sms = 0, cc = 0;
   if (!device_info(&sms, &cc)) return MR_ERR_CUDA;
   if (cc != 10 || d % 8 != 0 || n_out % 16 != 0 || N_r > mr::kDispMaxExperts ||
-      !aligned16(x) || !aligned16(W) || !aligned16(out))
+      !aligned16(x) || !aligned16(W) || (combine ? !aligned16(acc) : !aligned16(out)))
     return MR_ERR_UNSUPPORTED;
   auto enc = tensor_map_encoder();
   if (!enc) return MR_ERR_CUDA;
@@ -1133,12 +1138,21 @@ int launch_expert_gemm(const void* x, const int32_t* perm, const int32_t* offset
   P.x = x;
   P.w_packed = packed ? static_cast<const __nv_bfloat16*>(W) : nullptr;
   P.out = static_cast<__nv_bfloat16*>(out);
+  P.wts = wts;
+  P.acc = acc;
   // gathered rows: copied by the four epilogue warps (cp.async, 64-wide K
   // chunks) unless MR_EG_GATHER=tma pins the TMA tile::gather4 copies
   const char* g_env = getenv("MR_EG_GATHER");
   const bool tma_gather = bke == 32 || (g_env && g_env[0] == 't');
   using namespace mr::eg;
-  auto kern = !gather ? (packed ? expert_gemm_gather_kernel<64, true, kRowsSorted>
+  auto kern = combine ? (tma_gather
+                            ? (packed ? expert_gemm_gather_kernel<64, true, kGatherTma, true>
+                                      : (bke == 32
+                                             ? expert_gemm_gather_kernel<32, false, kGatherTma, true>
+                                             : expert_gemm_gather_kernel<64, false, kGatherTma, true>))
+                            : (packed ? expert_gemm_gather_kernel<64, true, kGatherLsu, true>
+                                      : expert_gemm_gather_kernel<64, false, kGatherLsu, true>))
+            : !gather ? (packed ? expert_gemm_gather_kernel<64, true, kRowsSorted>
                                 : (bke == 32 ? expert_gemm_gather_kernel<32, false, kRowsSorted>
                                              : expert_gemm_gather_kernel<64, false, kRowsSorted>))
             : tma_gather
@@ -1193,6 +1207,33 @@ int mr_expert_gemm_gather_packed(const void* x, const int32_t* perm, const int32
                                  void* out, mr_stream_t stream) {
   return launch_expert_gemm(x, perm, offsets, W_packed, true, T, d, k, N_r, n_out, out,
                             reinterpret_cast<cudaStream_t>(stream));
+}
+
+int mr_expert_gemm_gather_combine(const void* x, const int32_t* perm, const int32_t* offsets,
+                                  const void* W, int w_packed, const float* w,
+                                  const void* shared, int T, int d, int k, int N_r, int n_out,
+                                  float* acc, void* y, mr_stream_t stream) {
+  if (T < 0 || d <= 0 || k <= 0 || N_r <= 0 || n_out <= 0 || (w_packed != 0 && w_packed != 1))
+    return MR_ERR_INVALID_ARG;
+  if ((long long)T * n_out >= (1LL << 40)) return MR_ERR_INVALID_ARG;
+  if (T == 0) return MR_OK;
+  if (!x || !perm || !offsets || !W || !w || !acc || !y) return MR_ERR_INVALID_ARG;
+  if (n_out % 16 != 0 || !aligned16(acc) || !aligned16(y) || (shared && !aligned16(shared)))
+    return MR_ERR_UNSUPPORTED;
+  int sms = 0, cc = 0;
+  if (!device_info(&sms, &cc)) return MR_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const long n = (long)T * n_out;
+  if (cudaMemsetAsync(acc, 0, (size_t)n * sizeof(float), s) != cudaSuccess) return MR_ERR_CUDA;
+  const int rc = launch_expert_gemm(x, perm, offsets, W, w_packed != 0, T, d, k, N_r, n_out,
+                                    nullptr, s, w, acc);
+  if (rc != MR_OK) return rc;
+  const long n8 = n / 8;
+  const unsigned grid = (unsigned)std::min<long>((n8 + 255) / 256, (long)sms * 16);
+  mr::eg::combine_acc_finalize_kernel<<<grid, 256, 0, s>>>(
+      reinterpret_cast<const float4*>(acc), static_cast<const uint4*>(shared),
+      static_cast<uint4*>(y), n8);
+  return launch_status();
 }
 
 }  // extern "C"
