@@ -25,11 +25,11 @@
 // With the combine fused in (COMBINE; the same page: new_x[idxs] = outs,
 // weighted sum over k, cast back, plus the shared expert's output) the
 // expert outputs are never written either: the epilogue rounds each row to
-// bf16, multiplies it by its slot's router weight (fp32) and adds it into the
-// token's fp32 row of a [T, n_out] accumulator with vector reductions
-// (red.global.add.v4.f32, resolved in L2).  Rows of one expert segment belong
-// to distinct tokens, so the k additions into a token row come from k
-// different CTAs in no fixed order.  combine_acc_finalize_kernel then rounds
+// bf16, multiplies it by its slot's router weight (fp32), stages it in the
+// idle ring and adds it into the token's fp32 row of a [T, n_out] accumulator
+// with one bulk reduction per row (cp.reduce.async.bulk .add.f32, resolved in
+// L2).  Rows of one expert segment belong to distinct tokens, so the k
+// additions into a token row come from k different CTAs in no fixed order.  combine_acc_finalize_kernel then rounds
 // the accumulator to bf16, adds the shared row and rounds again.
 #pragma once
 
@@ -66,11 +66,14 @@ struct Params {
   float* acc;          // [T, n_out] fp32, zeroed before the launch (COMBINE)
 };
 
-// Adds four floats to 16 bytes of global memory (one vector reduction at the
-// L2; the address 16-byte aligned).
-__device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, float d) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c),
-               "f"(d)
+// Adds `bytes` of fp32 from shared memory into global memory element by
+// element (a bulk reduction by the copy engine, resolved in L2; both
+// addresses 16-byte aligned, bytes a multiple of 16); committed and waited
+// for with bulk_store_commit_and_wait.
+__device__ __forceinline__ void bulk_reduce_add_f32(float* gdst, uint32_t ssrc, uint32_t bytes) {
+  asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;" ::"l"(
+                   gdst),
+               "r"(ssrc), "r"(bytes)
                : "memory");
 }
 
@@ -341,21 +344,36 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool store = ok && j < row_end;
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
     if constexpr (COMBINE) {
-      // slot perm[j] = t * k + slot: weight w[perm[j]], token row t of acc
+      // slot perm[j] = t * k + slot: weight w[perm[j]], token row t of acc.
+      // The row, scaled, goes to the idle ring (every MMA that read it has
+      // completed: B_ACC), one [kBN] fp32 row per thread, rows kRedRow
+      // bytes apart so a quarter-warp's 16-byte stores fall on distinct
+      // banks; then one bulk reduction adds the whole row into acc (one
+      // coalesced kBN * 4-byte transfer, not 16-byte pieces of 32 rows).
+      constexpr uint32_t kRedRow = kBN * 4 + 16;
+      static_assert(BM * kRedRow <= kBarOff, "the scaled rows fit in the ring");
       const int slot = store ? P.perm[j] : 0;
       const float wj = store ? P.wts[slot] : 0.0f;
-      float* arow = P.acc + (long)(slot / P.k) * P.n_out + n0;
+      float* srow = reinterpret_cast<float*>(smem + (uint32_t)r * kRedRow);
+      const int ncols = P.n_out - n0 < kBN ? P.n_out - n0 : kBN;
       for (int c = 0; c < kBN / 16; ++c) {
         float v[16];
         tmem_ld16(tmem_base + lane_off + (uint32_t)(c * 16), v);  // whole warp
-        if (store && n0 + c * 16 < P.n_out) {
+        if (store && c * 16 < ncols) {
 #pragma unroll
           for (int i = 0; i < 16; i += 4)
-            red_add_v4(arow + c * 16 + i, wj * __bfloat162float(__float2bfloat16_rn(v[i])),
-                       wj * __bfloat162float(__float2bfloat16_rn(v[i + 1])),
-                       wj * __bfloat162float(__float2bfloat16_rn(v[i + 2])),
-                       wj * __bfloat162float(__float2bfloat16_rn(v[i + 3])));
+            *reinterpret_cast<float4*>(srow + c * 16 + i) =
+                make_float4(wj * __bfloat162float(__float2bfloat16_rn(v[i])),
+                            wj * __bfloat162float(__float2bfloat16_rn(v[i + 1])),
+                            wj * __bfloat162float(__float2bfloat16_rn(v[i + 2])),
+                            wj * __bfloat162float(__float2bfloat16_rn(v[i + 3])));
         }
+      }
+      if (store) {
+        fence_proxy_async();  // this thread's row, visible to the bulk copy
+        bulk_reduce_add_f32(P.acc + (long)(slot / P.k) * P.n_out + n0, smem_u32(srow),
+                            (uint32_t)ncols * 4u);
+        bulk_store_commit_and_wait();
       }
     }
     __nv_bfloat16* dst = COMBINE ? nullptr : P.out + (long)j * P.n_out + n0;
