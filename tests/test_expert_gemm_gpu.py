@@ -281,7 +281,8 @@ def test_expert_gemm_gather_combine_matches_oracle(T, d, N_r, k, n_out, skew, in
     stats = {"elems": int(err.size), "max_abs_err": float(err.max()),
              "max_err_over_tol": float((err / tol).max()),
              "y_differ_elems": int((err > 0).sum())}
-    record(f"expert_combine_T{T}_d{d}_E{N_r}_n{n_out}", "expert_gemm_gather_combine", stats)
+    record(f"expert_combine_T{T}_d{d}_E{N_r}_n{n_out}_{'int' if integer else 'rand'}"
+           f"{'_drop' if drop else ''}", "expert_gemm_gather_combine", stats)
     print(stats)
 
 
