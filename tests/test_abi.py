@@ -155,5 +155,35 @@ def test_rows_validation():
     assert L.mr_combine(None, 1, None, None, None, None, 0, 64, 8, None) == mr.MR_OK
 
 
+def test_expert_layer_validation():
+    """Argument checks of the expert-layer entry points that return before
+    any device call (so they hold on a machine without a GPU)."""
+    L = mr.lib()
+    p = C.c_void_p(64)
+    # mr_expert_gemm_gather(x, perm, offsets, W, T, d, k, N_r, n_out, out)
+    assert L.mr_expert_gemm_gather(p, p, p, p, -1, 64, 8, 16, 32, p, None) == \
+        mr.MR_ERR_INVALID_ARG
+    assert L.mr_expert_gemm_gather(None, p, p, p, 10, 64, 8, 16, 32, p, None) == \
+        mr.MR_ERR_INVALID_ARG
+    assert L.mr_expert_gemm_gather(p, p, p, p, 0, 64, 8, 16, 32, p, None) == mr.MR_OK
+    # mr_expert_gemm_gather_combine(x, perm, offsets, W, w_packed, w, shared,
+    #                               T, d, k, N_r, n_out, acc, y)
+    comb = L.mr_expert_gemm_gather_combine
+    assert comb(p, p, p, p, 0, p, None, -1, 64, 8, 16, 32, p, p, None) == mr.MR_ERR_INVALID_ARG
+    assert comb(p, p, p, p, 2, p, None, 10, 64, 8, 16, 32, p, p, None) == mr.MR_ERR_INVALID_ARG
+    assert comb(p, None, p, p, 0, p, None, 10, 64, 8, 16, 32, p, p, None) == \
+        mr.MR_ERR_INVALID_ARG  # perm is required: it gives each row's slot
+    assert comb(p, p, p, p, 0, None, None, 10, 64, 8, 16, 32, p, p, None) == \
+        mr.MR_ERR_INVALID_ARG  # no router weights
+    assert comb(p, p, p, p, 0, p, None, 10, 64, 8, 16, 32, None, p, None) == \
+        mr.MR_ERR_INVALID_ARG  # no accumulator
+    assert comb(p, p, p, p, 0, p, None, 10, 64, 8, 16, 24, p, p, None) == \
+        mr.MR_ERR_UNSUPPORTED  # n_out % 16 != 0
+    assert comb(p, p, p, p, 0, p, C.c_void_p(72), 10, 64, 8, 16, 32, p, p, None) == \
+        mr.MR_ERR_UNSUPPORTED  # shared not 16-byte aligned
+    assert comb(None, None, None, None, 0, None, None, 0, 64, 8, 16, 32, None, None, None) == \
+        mr.MR_OK
+
+
 def test_selftest_rejects_unknown_case():
     assert mr.lib().mr_selftest_bounded_wait(7, None) == mr.MR_ERR_INVALID_ARG
