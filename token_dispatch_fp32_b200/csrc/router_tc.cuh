@@ -596,7 +596,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // 3S+{2,3} acc free  3S+4 MMA drained
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + plan.misc_off);
   volatile int* abort = reinterpret_cast<volatile int*>(smem + plan.misc_off + 8);
-  // xnz[s][w]: worker warp w saw a nonzero x residual in stage s this round
+  // xnz[s][w]: worker warp w saw a nonzero x residual in stage s on this pass of the ring
   volatile uint32_t* xnz = reinterpret_cast<volatile uint32_t*>(smem + plan.misc_off + 32);
   float* bias_s = reinterpret_cast<float*>(smem + plan.bias_off);
 
