@@ -15,11 +15,12 @@
 //     shuffles; every lane gathers the G group scores (the top-2 sum, or the
 //     best score), keeps topk_group groups by counting the groups that beat
 //     each one (lower group first on ties);
-//   * top-k, grouped: the candidates >= tau (the smallest of the kept
-//     groups' top-2 values, a lower bound on the k-th best) are ranked by
-//     counting, each rank its slot;
-//   * else (one group, or a token with more candidates than lanes) k
-//     rounds: every lane offers the best of its experts not yet taken
+//   * top-k: the candidates >= tau (a lower bound on the k-th best: the
+//     smallest of the kept groups' top-2 values, or with one group the k-th
+//     largest of the lanes' maxima) are ranked by counting, each rank its
+//     slot;
+//   * else (a token with more candidates than lanes, or 2*topk_group < k)
+//     k rounds: every lane offers the best of its experts not yet taken
 //     (value desc, index asc); the token's best is found with two warp
 //     reductions when a token has the whole warp (the largest value as an
 //     order-preserving integer, then the smallest index among the lanes that
@@ -176,20 +177,35 @@ __global__ void __launch_bounds__(kThreads)
 
   // ---- candidates: the scores >= tau, a lower bound on the k-th best ----
   // With groups, the kept groups' top-2 values are 2*topk_group distinct
-  // experts, so when that is >= k the k-th best is >= the smallest of them.
-  // Every expert of the top-k is then a candidate and its rank among the
-  // candidates (value desc, index asc) is its slot, found by counting; the
-  // candidates go through shared memory, one slot per lane of the token.  A
-  // warp with a token of more candidates than lanes (ties at the 0.0 fill,
-  // say) takes the k rounds below instead -- the same result.  Measured on
-  // the DeepSeek-V3 prefill batch: router 60.4 -> 56.3 us (same-box A/B,
-  // outputs bit-identical).  Without groups the bound from the lanes' own
-  // top-2 pairs (the ceil(k/2) lanes with the largest maxima) left too many
-  // candidates on the Kimi K2 prefill batch (140.3 -> 144.4 us), so one
-  // group takes the k rounds.
-  if (G > 1 && 2 * p.topk_group >= k) {  // the same for every thread of the grid
-    float tau = keep ? a2 : INFINITY;        // a2: the group's second best
-    for (int off = 1; off < P; off <<= 1) tau = fminf(tau, __shfl_xor_sync(full, tau, off));
+  // experts, so when that is >= k the k-th best is >= the smallest of them;
+  // with one group, the k largest of the lanes' maxima are k distinct
+  // experts, so the k-th best is >= the k-th of them (a bitonic sort of the
+  // lanes' maxima).  Every expert of the top-k is then a candidate and its
+  // rank among the candidates (value desc, index asc) is its slot, found by
+  // counting; the candidates go through shared memory, one slot per lane of
+  // the token.  A warp with a token of more candidates than lanes (ties at
+  // the 0.0 fill, say) takes the k rounds below instead -- the same result.
+  // Measured (same-box A/Bs, outputs bit-identical): DeepSeek-V3 prefill
+  // router 60.4 -> 56.3 us, Kimi K2 prefill router 142.4 -> 138.2 us (a
+  // looser one-group bound, the smallest second-best of the ceil(k/2) lanes
+  // with the largest maxima, left too many candidates: 140.3 -> 144.4 us).
+  const bool grouped = G > 1 && 2 * p.topk_group >= k;  // the same for the whole grid
+  if (grouped || (G == 1 && k <= P)) {
+    float tau;
+    if (grouped) {
+      tau = keep ? a2 : INFINITY;  // a2: the group's second best
+      for (int off = 1; off < P; off <<= 1) tau = fminf(tau, __shfl_xor_sync(full, tau, off));
+    } else {
+      // one group: the k-th largest of the lanes' maxima (k distinct experts
+      // are >= it), by a bitonic sort of the token's P lanes, descending
+      float v = a1;
+      for (int size = 2; size <= P; size <<= 1)
+        for (int st = size >> 1; st > 0; st >>= 1) {
+          const float o = __shfl_xor_sync(full, v, st);
+          v = (((j & st) == 0) == ((j & size) == 0)) ? fmaxf(v, o) : fminf(v, o);
+        }
+      tau = __shfl_sync(full, v, seg0 + k - 1);
+    }
     int nl = 0;
 #pragma unroll
     for (int i = 0; i < EL; ++i) nl += (c[i] >= tau && c[i] > -INFINITY) ? 1 : 0;
