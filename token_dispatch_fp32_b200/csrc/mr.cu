@@ -279,6 +279,8 @@ int launch_reduce_nj(const float* part, int KS, int T, int N_r, const float* bia
   return MR_OK;
 }
 
+int launch_route(const mr::rt::Params& rp, cudaStream_t st);
+
 // W fp32 (3xTF32, or one tf32 product without use3x), or W stored in bf16
 // (wb16 non-null; x must be bf16: kind::f16 MMAs on the staged tiles).
 int launch_splitk(const void* x, bool x_bf16, const float* W, const float* bias, int T, int d,
@@ -339,6 +341,34 @@ int launch_splitk(const void* x, bool x_bf16, const float* W, const float* bias,
   }
   if (launch_status() != MR_OK) return MR_ERR_CUDA;
   const int KSr = sh.KS / sh.CL;
+  // Reduce and route: the routing kernel (one warp per token where the lane
+  // layout fits) unless MR_ROUTE_KERNEL=0 pins the one-CTA-per-token kernel
+  const char* rk_env = getenv("MR_ROUTE_KERNEL");
+  const int lanes = (rk_env && rk_env[0] == '0')
+                        ? 0
+                        : mr::rt::lanes_per_token(T, N_r, n_group, k, sms,
+                                                  getenv("MR_ROUTE_LANES")
+                                                      ? atoi(getenv("MR_ROUTE_LANES"))
+                                                      : 0);
+  if (lanes > 0) {
+    mr::rt::Params rp;
+    rp.part = P.part;
+    rp.KS = KSr;
+    rp.T = T;
+    rp.N = N_r;
+    rp.P = lanes;
+    rp.n_group = n_group;
+    rp.topk_group = topk_group;
+    rp.k = k;
+    rp.mask_mode = mask_mode;
+    rp.flags = flags;
+    rp.route_scale = route_scale;
+    rp.bias = bias;
+    rp.idx_out = idx_out;
+    rp.w_out = w_out;
+    rp.logits_out = logits_out;
+    return launch_route(rp, st);
+  }
   const int nj = (N_r + 31) / 32;
 #define MR_RED_CASE(NJV)                                                                      \
   if (nj <= NJV)                                                                              \

@@ -1,8 +1,9 @@
 // route.cuh -- routing of tokens whose logits are in memory (Kimi K2
 // "Normalize weights" page, MoEGate.forward after the linear map; DeepSeek-
 // V3.2-Exp "Normalize weights" page, Gate.forward), for the tensor-core
-// router when the caller's workspace holds its logits: part[s][t][e] fp32,
-// the K-split slices s < KS added in slice order.
+// router when the caller's workspace holds its logits and for the split-K
+// router of small batches: part[s][t][e] fp32, the slices s < KS added in
+// slice order.
 //
 // P lanes route one token (P = 8, 16 or 32 consecutive lanes of a warp), lane
 // j owning the contiguous experts [j*EL, (j+1)*EL), N = P*EL, so the work of
@@ -40,7 +41,7 @@ namespace rt {
 constexpr int kThreads = 256;
 constexpr int kMaxN = 512;
 constexpr int kTop = 8;
-constexpr int kMaxSlices = 4;  // K-split slices the routing kernel adds
+constexpr int kMaxSlices = 4;  // slices added with all their loads in flight at once
 
 struct Params {
   const float* part;  // [KS][T][N]
@@ -79,9 +80,37 @@ __global__ void __launch_bounds__(kThreads)
 
   // ---- logits: the slices added in order (all loads issued first) ----
   float L[EL];
-  {
-    const long stride = (long)p.T * N;
-    const float4* src = reinterpret_cast<const float4*>(p.part + (live ? t : 0) * N + e0);
+  const long stride = (long)p.T * N;
+  const float4* src = reinterpret_cast<const float4*>(p.part + (live ? t : 0) * N + e0);
+  if (p.KS > kMaxSlices) {
+    // more slices (the split-K GEMM of small batches): slice by slice, each
+    // slice's loads issued together, the sums still in slice order
+    constexpr int kSlUnroll = EL <= 8 ? 4 : (EL <= 16 ? 2 : 1);  // ~8 float4 loads in flight
+    float4 a[EL / 4];
+#pragma unroll
+    for (int m = 0; m < EL / 4; ++m) a[m] = live ? src[m] : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll kSlUnroll
+    for (int sl = 1; sl < p.KS; ++sl) {
+      float4 b[EL / 4];
+#pragma unroll
+      for (int m = 0; m < EL / 4; ++m)
+        b[m] = live ? src[sl * stride / 4 + m] : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int m = 0; m < EL / 4; ++m) {
+        a[m].x += b[m].x;
+        a[m].y += b[m].y;
+        a[m].z += b[m].z;
+        a[m].w += b[m].w;
+      }
+    }
+#pragma unroll
+    for (int m = 0; m < EL / 4; ++m) {
+      L[4 * m] = a[m].x;
+      L[4 * m + 1] = a[m].y;
+      L[4 * m + 2] = a[m].z;
+      L[4 * m + 3] = a[m].w;
+    }
+  } else {
 #pragma unroll
     for (int m = 0; m < EL / 4; ++m) {
       float4 v[kMaxSlices];
