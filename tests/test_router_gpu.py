@@ -227,13 +227,19 @@ SPLITK_CASES = [(w, "f32") for w in SPLITK] + [(w, "bf16") for w in SPLITK
                                                 if w.io_dtype == "bf16"]
 
 
+@pytest.mark.parametrize("routing", ["default", "cta"])
 @pytest.mark.parametrize("w,rows", SPLITK_CASES, ids=[f"{w.name}-{r}" for w, r in SPLITK_CASES])
-def test_router_splitk_small_batches(w, rows):
+def test_router_splitk_small_batches(w, rows, routing, monkeypatch):
     """Batches of up to 256 tokens with a workspace take the split-K path
     (K-sliced tensor-core GEMM over all SMs, cluster reduction, reduce-and-
     route), for fp32 rows and for bf16 rows (staged as bf16, widened in
     shared memory).  d = 7168 and 1000 reduce the K slices in clusters of 8;
-    d = 516 has too few K chunks for that and writes every slice."""
+    d = 516 has too few K chunks for that and writes every slice.  The
+    slices are reduced and routed by the routing kernel where its lane
+    layout fits (default) or, pinned by MR_ROUTE_KERNEL=0, by one CTA per
+    token (the kernel shapes without a lane layout take)."""
+    if routing == "cta":
+        monkeypatch.setenv("MR_ROUTE_KERNEL", "0")
     n = mr.mr_router_workspace_size(w.T, w.d, w.N_r)
     assert n > 0
     d = router_inputs(w)
@@ -288,10 +294,15 @@ ROUTE_SHAPES = [
 ]
 
 
+@pytest.mark.parametrize("routing", ["default", "cta"])
 @pytest.mark.parametrize("w", ROUTE_SHAPES, ids=[w.name for w in ROUTE_SHAPES])
-def test_router_splitk_routing_shapes(w):
+def test_router_splitk_routing_shapes(w, routing, monkeypatch):
     """Every token of each routing shape of the split-K path against the
-    oracle (expert sets exact outside near-ties, weights within tolerance)."""
+    oracle (expert sets exact outside near-ties, weights within tolerance),
+    reduced and routed by the routing kernel where its lane layout fits and
+    by one CTA per token (MR_ROUTE_KERNEL=0)."""
+    if routing == "cta":
+        monkeypatch.setenv("MR_ROUTE_KERNEL", "0")
     d = router_inputs(w)
     ws = torch.empty(mr.mr_router_workspace_size(w.T, w.d, w.N_r), dtype=torch.uint8,
                      device="cuda")
