@@ -26,9 +26,11 @@
 // the CL partials in rank order (deterministic) through distributed shared
 // memory and writes them to part[ks / CL][token][expert].  A second cluster
 // barrier keeps every CTA's shared memory alive until its peers have read it.
-// router_reduce_route_kernel (launched as a programmatic dependent of the
-// GEMM) sums the KS / CL slices in order and routes each token with the whole
-// CTA (route_token_cta), or with one warp for the shapes that does not cover.
+// The KS / CL slices are then summed in order and routed by a programmatic
+// dependent of the GEMM: the routing kernel of route.cuh (one warp per token)
+// where its lane layout fits, else router_reduce_route_kernel below, which
+// routes each token with the whole CTA (route_token_cta), or with one warp for
+// the shapes that does not cover.
 #pragma once
 
 #include "router_tc.cuh"
