@@ -1377,9 +1377,11 @@ int mr_combine(const void* expert_out, int dtype, const float* w, const int32_t*
                    (!shared || aligned16(shared));
   const bool vec32 = row_bytes % 32 == 0 && aligned32(expert_out) && aligned32(y) &&
                      (!shared || aligned32(shared));
-  // 64 CTAs per SM, grid-stride (369 us on the full DeepSeek-V3 batch; 372 us
-  // with 32 per SM)
-  const unsigned grid = (unsigned)std::min<long>(T, (long)sms * 64);
+  // grid-stride: 16 CTAs per SM with 32-byte vectors (360.5 us on the full
+  // DeepSeek-V3 batch against 362.5 us with 64 and 364.5 us with 4 or 32 per
+  // SM), 64 with 16-byte vectors (369 us; 372 us with 32 per SM)
+  const long per_sm = vec32 && dtype == MR_BF16 ? 16 : 64;
+  const unsigned grid = (unsigned)std::min<long>(T, (long)sms * per_sm);
   return launch_combine<true>(vec, vec32, dtype == MR_BF16, grid, s, w, shared, y, T, d, k,
                               [&](auto* tag) {
                                 using V = std::remove_const_t<std::remove_pointer_t<decltype(tag)>>;
